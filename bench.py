@@ -1,0 +1,318 @@
+"""Benchmark: GDN forward tokens/s on the minute-scale workload
+(B=1 per GPU, H=20, 121 frames x 880 tokens = 106,480 tokens, d_k = d_v = 112,
+bf16 q/k/v/o, fp32 alpha/beta/state), and the fraction of the binding
+roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--regime lit|slow]
+    python bench.py --impl reference ...     # the fp64 CPU oracle on a bounded sample
+
+Prints ONE JSON line on rank 0.  Multi-GPU (torchrun): every rank runs its
+own batch element (weak scaling, no data-path collective: the (b, h) chains
+are independent); the timed region is bracketed by a barrier and a device
+synchronise, and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "minute"
+# algorithmic work of the chunk = frame method (per frame-head, L tokens, d_k, d_v):
+#   intra-frame solve   L^2 (2 d_k + d_v)   (decayed beta K K^T lower half + forward substitution)
+#   output              L^2 (d_k + d_v) + 4 L d_k d_v   (masked Q K^T . U, Q Sig, W Sig)
+#   state               2 L d_k d_v          (carry to the next frame)
+# total F_alg = L^2 (3 d_k + 2 d_v) + 6 L d_k d_v
+
+
+def flops_intra(L, dk, dv):
+    return L * L * (2 * dk + dv)
+
+
+def flops_total(L, dk, dv):
+    return L * L * (3 * dk + 2 * dv) + 6 * L * dk * dv
+
+
+def bytes_alg(B, T, H, dk, dv, elem=2):
+    # read q, k, v; write o; alpha and beta fp32; state I/O (fp32 in + out)
+    return B * T * H * (2 * dk + 2 * dv) * elem + 8 * B * T * H + 2 * B * H * dk * dv * 4
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        for line in (self.out or "").splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(regime, frames, inp=None, nthreads=0):
+    """The fp64 oracle as it stands, timed on this host's cores over a bounded
+    sample: all 20 heads of the first `frames` frames of the workload (the
+    upcast of the stored inputs to fp64 is not timed)."""
+    import oracle
+    from gated_deltanet_linear_chunkwise_b200 import workloads as W
+    w = W.WORKLOADS[WORKLOAD]
+    if inp is None:
+        inp = W.make_inputs(w, regime, frames=frames)
+    n = frames * w.frame_len
+    x = {k: inp[k][:, :n].double().numpy() for k in ("q", "k", "v", "alpha", "beta")}
+    threads = nthreads or min(os.cpu_count() or 1, w.B * w.H)
+    t0 = time.perf_counter()
+    oracle.token_recurrence(x["q"], x["k"], x["v"], x["alpha"], x["beta"], None, nthreads=threads)
+    dt = time.perf_counter() - t0
+    tokens = w.B * frames * w.frame_len
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "B=1, 20 heads, first %d of 121 frames (%d tokens) of the minute workload, %.1f s"
+                      % (frames, tokens, dt)}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the oracle on host cores, each step a bounded sample."""
+    if rank != 0:
+        return
+    from gated_deltanet_linear_chunkwise_b200 import workloads as W
+    w = W.WORKLOADS[WORKLOAD]
+    inp = W.make_inputs(w, args.regime, frames=args.ref_frames)
+    cpu_baseline(args.regime, 1, inp)  # warm-up: one frame
+    vals = []
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(args.regime, args.ref_frames, inp))
+    value = statistics.median(v["value"] for v in vals)
+    cb = dict(vals[0])
+    cb["value"] = value
+    line = {
+        "impl": "reference", "metric": "GDN forward tokens/s at 106,480 tokens x 20 heads; % of binding roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.B * args.ref_frames * w.frame_len / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "minute: B=1 H=20 T=106480 (121 frames x 880) d_k=d_v=112; oracle sample of "
+                               "%d frames per step" % args.ref_frames, "gate_regime": args.regime},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--regime", default="slow", choices=["lit", "slow"])
+    ap.add_argument("--cpu-frames", type=int, default=60, help="frames in the oracle's timed sample")
+    ap.add_argument("--ref-frames", type=int, default=2, help="frames per --impl reference step")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import gated_deltanet_linear_chunkwise_b200 as g
+    from gated_deltanet_linear_chunkwise_b200 import workloads as W
+    from gated_deltanet_linear_chunkwise_b200.binding import NUM_STAGES, STAGES
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = W.WORKLOADS[WORKLOAD]
+    L, dk, dv, H = w.frame_len, w.d_k, w.d_v, w.H
+    # each rank draws its own batch element (weak scaling)
+    inp = W.make_inputs(w, args.regime, seed=W.SEEDS[WORKLOAD] + 7919 * rank)
+    d = {k: (None if t is None else t.to(dev).contiguous()) for k, t in inp.items()}
+    B, T = w.B, w.T
+    o = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
+    S_out = torch.empty(B, H, dv, dk, dtype=torch.float32, device=dev)
+    ws = torch.empty(g.workspace_bytes(B, H, T, L, dk, dv, "bf16"), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(stage_ms=None):
+        g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, None, S_out=S_out, o=o,
+                  workspace=ws, stream=stream, stage_ms=stage_ms)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # timed region: K steps, CUDA events on the launching stream
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+
+    # per-stage device times (events around each kernel on the same stream)
+    stage_sum = [0.0] * NUM_STAGES
+    reps = 5
+    for _ in range(reps):
+        arr = (ctypes.c_float * NUM_STAGES)()
+        step(stage_ms=arr)
+        for i in range(NUM_STAGES):
+            stage_sum[i] += arr[i] / reps
+    dominant = max(range(NUM_STAGES), key=lambda i: stage_sum[i])
+
+    # end to end through the public call with host buffers: pinned host inputs
+    # copied in, the pass, the output (and final state) copied back, every step
+    h = {k: (None if t is None else t.pin_memory()) for k, t in inp.items() if t is not None}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_host = torch.empty(S_out.shape, dtype=S_out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
+
+    def e2e_step():
+        for k, t in h.items():
+            d[k].copy_(t, non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+        S_host.copy_(S_out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    pk = peaks()
+    nfh = B * H * w.frames
+    if rank == 0:
+        f_dom = {0: flops_intra(L, dk, dv), 3: L * L * (dk + dv) + 4 * L * dk * dv,
+                 1: 4 * L * dk * dv, 2: 2 * dk * dk * dv}[dominant] * nfh
+        dom_ms = stage_sum[dominant]
+        achieved = f_dom / (dom_ms * 1e-3) / 1e12
+        f_all = flops_total(L, dk, dv) * nfh
+        tokens = B * T * world
+        line = {
+            "metric": "GDN forward tokens/s at 106,480 tokens x 20 heads; % of binding roofline",
+            "value": tokens / (ms_step * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "minute: B=1 per GPU, H=20, T=106480 (121 frames x 880 tokens), "
+                                   "d_k=d_v=112, bf16 q/k/v/o, fp32 gates and state, chunk = frame",
+                       "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
+                       "gate_regime": args.regime,
+                       "l2": "no flush: inputs 1.4 GB per step exceed the 126 MB L2"},
+            "roofline": {"bound": "tensor", "kernel": STAGES[dominant], "achieved": achieved,
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                         "traffic": None, "peak_source": pk["source"] + " bf16 burst",
+                         "stage_ms": dict(zip(STAGES, stage_sum))},
+            "path_roofline": {"flops": f_all, "bytes": bytes_alg(B, T, H, dk, dv),
+                              "achieved_tflops": f_all / (ms_step * 1e-3) / 1e12,
+                              "frac_tensor": f_all / (ms_step * 1e-3) / 1e12 / pk["bf16_tflops"],
+                              "frac_tensor_sustained": (f_all / (ms_step * 1e-3) / 1e12 / pk["bf16_tflops_sustained"]
+                                                        if pk["bf16_tflops_sustained"] else None)},
+            "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": NUM_STAGES * args.steps,
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(args.regime, args.cpu_frames, inp)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

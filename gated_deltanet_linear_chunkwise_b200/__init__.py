@@ -1,1 +1,12 @@
-"""B200-native chunkwise gated delta rule (placeholder; binding added with the C-ABI)."""
+"""B200-native (sm_100a) chunkwise gated delta rule.
+
+The computation lives in ``libgdn_b200.so`` (C ABI declared in
+``include/gdn.h``); this package re-exports a thin ctypes binding of it and
+the named synthetic workloads.  Importing the package does not load the
+library; the first call does, and fails loudly if it has not been built.
+"""
+from .binding import (GdnError, bidirectional, gdn_fwd, gdn_step, last_error, load_library,
+                      workspace_bytes)
+
+__all__ = ["GdnError", "bidirectional", "gdn_fwd", "gdn_step", "last_error", "load_library",
+           "workspace_bytes"]

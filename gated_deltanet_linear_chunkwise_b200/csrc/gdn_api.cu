@@ -1,0 +1,334 @@
+// gdn_api.cu -- the C ABI: argument validation, workspace, dispatch.
+//
+// Validation happens before anything is enqueued; on a validation error the
+// call returns its status with no launch and no output touched.  No C++
+// exception crosses the ABI (every entry point is noexcept and catches).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "gdn_internal.h"
+#include "gdn_tc.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+void set_err(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+
+bool misaligned(const void *ptr) { return ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u); }
+
+bool head_dim_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
+
+// Range [p, p+n) of two buffers overlap?
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || !na || !nb) return false;
+    const char *x = (const char *)a, *y = (const char *)b;
+    return x < y + nb && y < x + na;
+}
+
+int validate_sizes(const gdn_args &a) {
+    if (a.dtype != GDN_DTYPE_BF16 && a.dtype != GDN_DTYPE_F32) {
+        set_err("dtype %d is neither GDN_DTYPE_BF16 nor GDN_DTYPE_F32", a.dtype);
+        return GDN_ERR_INVALID_ARG;
+    }
+    if (a.B < 0 || a.H < 0 || a.T < 0) {
+        set_err("negative size: B=%d H=%d T=%lld", a.B, a.H, a.T);
+        return GDN_ERR_INVALID_ARG;
+    }
+    if (a.frame_len <= 0) {
+        set_err("frame_len must be positive (got %d)", a.frame_len);
+        return GDN_ERR_INVALID_ARG;
+    }
+    if (a.reverse != 0 && a.reverse != 1) { set_err("reverse must be 0 or 1"); return GDN_ERR_INVALID_ARG; }
+    if (a.accumulate_o != 0 && a.accumulate_o != 1) { set_err("accumulate_o must be 0 or 1"); return GDN_ERR_INVALID_ARG; }
+    if (a.check_finite != 0 && a.check_finite != 1) { set_err("check_finite must be 0 or 1"); return GDN_ERR_INVALID_ARG; }
+    if (a.reset_every < 0 || (a.reset_every > 0 && a.reset_every % a.frame_len != 0)) {
+        set_err("reset_every (%lld) must be 0 or a positive multiple of frame_len (%d)", a.reset_every, a.frame_len);
+        return GDN_ERR_INVALID_ARG;
+    }
+    if (a.T % a.frame_len != 0) {
+        set_err("T (%lld) is not a multiple of frame_len (%d)", a.T, a.frame_len);
+        return GDN_ERR_SHAPE;
+    }
+    if (!head_dim_ok(a.d_k) || !head_dim_ok(a.d_v)) {
+        set_err("head dims d_k=%d d_v=%d: each must be a multiple of 16 in [16, 128]", a.d_k, a.d_v);
+        return GDN_ERR_UNSUPPORTED;
+    }
+    if (a.frame_len > 4096) {
+        set_err("frame_len %d exceeds the supported maximum 4096", a.frame_len);
+        return GDN_ERR_UNSUPPORTED;
+    }
+    const long long dmax = a.d_k > a.d_v ? a.d_k : a.d_v;
+    // B*T*H*dmax < 2^62 and B*H*F < 2^31, checked without overflow
+    const long double elems = (long double)a.B * (long double)a.T * (long double)a.H * (long double)dmax;
+    if (elems >= 4.611686018427387904e18L) {
+        set_err("B*T*H*d = %.3Le elements overflows the 2^62 index range", elems);
+        return GDN_ERR_SHAPE;
+    }
+    const long long F = a.T / a.frame_len;
+    if ((long double)a.B * a.H * F >= 2147483648.0L) {
+        set_err("B*H*frames = %.3Le exceeds 2^31", (long double)a.B * a.H * F);
+        return GDN_ERR_SHAPE;
+    }
+    return GDN_OK;
+}
+
+int validate(const gdn_args &a, gdn::Problem &p) {
+    int st = validate_sizes(a);
+    if (st != GDN_OK) return st;
+    const long long F = a.T / a.frame_len;
+    const bool empty = (a.B == 0 || a.H == 0 || a.T == 0);
+    if (!empty && (!a.q || !a.k || !a.v || !a.alpha || !a.beta || !a.o)) {
+        set_err("q, k, v, alpha, beta and o are required (one is NULL)");
+        return GDN_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {a.q, a.k, a.v, a.alpha, a.beta, a.S_in, a.S_out, a.o};
+    const char *names[] = {"q", "k", "v", "alpha", "beta", "S_in", "S_out", "o"};
+    for (int i = 0; i < 8; ++i)
+        if (misaligned(ptrs[i])) {
+            set_err("%s = %p is not 16-byte aligned", names[i], ptrs[i]);
+            return GDN_ERR_ALIGNMENT;
+        }
+    if (a.workspace && (reinterpret_cast<uintptr_t>(a.workspace) & 255u)) {
+        set_err("workspace = %p is not 256-byte aligned", a.workspace);
+        return GDN_ERR_ALIGNMENT;
+    }
+    // outputs may not overlap inputs (S_in == S_out exactly is allowed)
+    const size_t es = a.dtype == GDN_DTYPE_BF16 ? 2 : 4;
+    const size_t nqk = (size_t)a.B * a.T * a.H * a.d_k * es, nv = (size_t)a.B * a.T * a.H * a.d_v * es;
+    const size_t ng = (size_t)a.B * a.T * a.H * 4, ns = (size_t)a.B * a.H * a.d_v * a.d_k * 4;
+    const void *ins[] = {a.q, a.k, a.v, a.alpha, a.beta, a.S_in};
+    const size_t insz[] = {nqk, nqk, nv, ng, ng, ns};
+    for (int i = 0; i < 6; ++i) {
+        if (overlap(a.o, nv, ins[i], insz[i])) {
+            set_err("o overlaps input %s", names[i]);
+            return GDN_ERR_INVALID_ARG;
+        }
+        if (a.S_out && !(i == 5 && a.S_out == a.S_in) && overlap(a.S_out, ns, ins[i], insz[i])) {
+            set_err("S_out overlaps input %s", names[i]);
+            return GDN_ERR_INVALID_ARG;
+        }
+    }
+    if (overlap(a.o, nv, a.S_out, ns)) { set_err("o overlaps S_out"); return GDN_ERR_INVALID_ARG; }
+
+    p.dtype = a.dtype;
+    p.q = a.q; p.k = a.k; p.v = a.v;
+    p.alpha = a.alpha; p.beta = a.beta;
+    p.S_in = a.S_in; p.S_out = a.S_out; p.o = a.o;
+    p.B = a.B; p.H = a.H; p.T = a.T; p.L = a.frame_len;
+    p.dk = a.d_k; p.dv = a.d_v; p.F = F;
+    p.reverse = a.reverse; p.accumulate = a.accumulate_o; p.reset_every = a.reset_every;
+    return GDN_OK;
+}
+
+// Which implementation serves this problem, and how much scratch it needs.
+bool use_tc(const gdn::Problem &p) { return gdn::tc_supports(p); }
+
+size_t workspace_for(const gdn::Problem &p) {
+    return use_tc(p) ? gdn::tc_workspace_bytes(p) : gdn::simt_workspace_bytes(p);
+}
+
+__global__ void nonfinite_scan_f32(const float *x, long long n, int *flag) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        if (!isfinite(x[i])) { atomicOr(flag, 1); return; }
+}
+__global__ void nonfinite_scan_bf16(const __nv_bfloat16 *x, long long n, int *flag) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        if (!isfinite(__bfloat162float(x[i]))) { atomicOr(flag, 1); return; }
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    set_err("%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+    return GDN_ERR_CUDA;
+}
+
+int run(const gdn_args &a) noexcept {
+    try {
+        g_err[0] = '\0';
+        if (a.struct_size != (int)sizeof(gdn_args)) {
+            set_err("gdn_args.struct_size = %d, this library expects %d", a.struct_size, (int)sizeof(gdn_args));
+            return GDN_ERR_INVALID_ARG;
+        }
+        gdn::Problem p;
+        int st = validate(a, p);
+        if (st != GDN_OK) return st;
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(a.stream);
+        const size_t sbytes = (size_t)a.B * a.H * a.d_v * a.d_k * sizeof(float);
+
+        if (a.B == 0 || a.H == 0) return GDN_OK;
+        if (a.T == 0) {  // nothing to scan: the final state is the initial state
+            if (a.S_out && a.S_out != a.S_in) {
+                cudaError_t e = a.S_in ? cudaMemcpyAsync(a.S_out, a.S_in, sbytes, cudaMemcpyDeviceToDevice, s)
+                                       : cudaMemsetAsync(a.S_out, 0, sbytes, s);
+                if (e) return cuda_fail(e, "state copy");
+            }
+            return GDN_OK;
+        }
+        const size_t need = workspace_for(p);
+        void *ws = a.workspace;
+        bool owned = false;
+        if (ws) {
+            if (a.workspace_bytes < need) {
+                set_err("workspace_bytes = %zu < %zu required", a.workspace_bytes, need);
+                return GDN_ERR_NO_MEMORY;
+            }
+        } else {
+            cudaError_t e = cudaMallocAsync(&ws, need, s);
+            if (e != cudaSuccess || !ws) {
+                cudaGetLastError();
+                set_err("cudaMallocAsync(%zu bytes) failed: %s", need, cudaGetErrorString(e));
+                return GDN_ERR_NO_MEMORY;
+            }
+            owned = true;
+        }
+        cudaEvent_t ev[GDN_NUM_STAGES + 1] = {};
+        cudaEvent_t *evp = nullptr;
+        if (a.stage_ms) {
+            for (int i = 0; i <= GDN_NUM_STAGES; ++i) {
+                cudaError_t ee = cudaEventCreate(&ev[i]);
+                if (ee) {
+                    for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+                    if (owned) cudaFreeAsync(ws, s);
+                    return cuda_fail(ee, "stage timing events");
+                }
+            }
+            evp = ev;
+        }
+        cudaError_t e = use_tc(p) ? gdn::launch_tc(p, ws, s, evp) : gdn::launch_simt(p, ws, s, evp);
+        if (owned) {
+            cudaError_t e2 = cudaFreeAsync(ws, s);
+            if (e == cudaSuccess) e = e2;
+        }
+        if (evp) {
+            if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+            for (int i = 0; i < GDN_NUM_STAGES; ++i) {
+                float ms = -1.f;
+                if (e == cudaSuccess && cudaEventElapsedTime(&ms, ev[i], ev[i + 1]) != cudaSuccess) ms = -1.f;
+                a.stage_ms[i] = ms;
+            }
+            for (int i = 0; i <= GDN_NUM_STAGES; ++i) cudaEventDestroy(ev[i]);
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+
+        if (a.check_finite) {
+            int *flag = nullptr;
+            int host = 0;
+            if ((e = cudaMallocAsync((void **)&flag, sizeof(int), s))) return cuda_fail(e, "finite-check flag");
+            cudaMemsetAsync(flag, 0, sizeof(int), s);
+            const long long no = (long long)a.B * a.T * a.H * a.d_v;
+            if (a.dtype == GDN_DTYPE_F32) nonfinite_scan_f32<<<1184, 256, 0, s>>>((const float *)a.o, no, flag);
+            else nonfinite_scan_bf16<<<1184, 256, 0, s>>>((const __nv_bfloat16 *)a.o, no, flag);
+            if (a.S_out) nonfinite_scan_f32<<<148, 256, 0, s>>>(a.S_out, (long long)(sbytes / 4), flag);
+            cudaMemcpyAsync(&host, flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+            cudaFreeAsync(flag, s);
+            if ((e = cudaStreamSynchronize(s))) return cuda_fail(e, "finite check");
+            if (host) {
+                set_err("o or S_out holds a NaN or Inf");
+                return GDN_ERR_NONFINITE;
+            }
+        }
+        return GDN_OK;
+    } catch (...) {
+        set_err("internal error (exception caught at the ABI boundary)");
+        return GDN_ERR_CUDA;
+    }
+}
+
+gdn_args make_args(int dtype, const void *q, const void *k, const void *v, const float *alpha,
+                   const float *beta, const float *S_in, float *S_out, void *o, int B, int H,
+                   long long T, int frame_len, int d_k, int d_v, gdn_stream_t stream) {
+    gdn_args a;
+    memset(&a, 0, sizeof(a));
+    a.struct_size = (int)sizeof(gdn_args);
+    a.dtype = dtype;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta;
+    a.S_in = S_in; a.S_out = S_out; a.o = o;
+    a.B = B; a.H = H; a.T = T; a.frame_len = frame_len; a.d_k = d_k; a.d_v = d_v;
+    a.stream = stream;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+            const float *S_in, float *S_out, void *o, int B, int H, long long T, int frame_len,
+            int d_k, int d_v, gdn_stream_t stream) {
+    return run(make_args(GDN_DTYPE_BF16, q, k, v, alpha, beta, S_in, S_out, o, B, H, T, frame_len, d_k, d_v, stream));
+}
+
+int gdn_fwd_f32(const float *q, const float *k, const float *v, const float *alpha, const float *beta,
+                const float *S_in, float *S_out, float *o, int B, int H, long long T, int frame_len,
+                int d_k, int d_v, gdn_stream_t stream) {
+    return run(make_args(GDN_DTYPE_F32, q, k, v, alpha, beta, S_in, S_out, o, B, H, T, frame_len, d_k, d_v, stream));
+}
+
+int gdn_step(const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+             const float *S_in, float *S_out, void *o, int B, int H, long long T, int frame_len,
+             int d_k, int d_v, gdn_stream_t stream) {
+    if (!S_in) {
+        set_err("gdn_step requires S_in (the carried state)");
+        return GDN_ERR_INVALID_ARG;
+    }
+    return gdn_fwd(q, k, v, alpha, beta, S_in, S_out, o, B, H, T, frame_len, d_k, d_v, stream);
+}
+
+int gdn_step_f32(const float *q, const float *k, const float *v, const float *alpha, const float *beta,
+                 const float *S_in, float *S_out, float *o, int B, int H, long long T, int frame_len,
+                 int d_k, int d_v, gdn_stream_t stream) {
+    if (!S_in) {
+        set_err("gdn_step_f32 requires S_in (the carried state)");
+        return GDN_ERR_INVALID_ARG;
+    }
+    return gdn_fwd_f32(q, k, v, alpha, beta, S_in, S_out, o, B, H, T, frame_len, d_k, d_v, stream);
+}
+
+int gdn_fwd_ex(const gdn_args *a) {
+    if (!a) {
+        set_err("gdn_fwd_ex: args is NULL");
+        return GDN_ERR_INVALID_ARG;
+    }
+    return run(*a);
+}
+
+size_t gdn_workspace_bytes(int B, int H, long long T, int frame_len, int d_k, int d_v, int dtype) {
+    gdn_args a = make_args(dtype, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                           B, H, T, frame_len, d_k, d_v, nullptr);
+    if (validate_sizes(a) != GDN_OK) return 0;
+    if (B == 0 || H == 0 || T == 0) return 0;
+    gdn::Problem p;
+    memset(&p, 0, sizeof(p));
+    p.dtype = dtype; p.B = B; p.H = H; p.T = T; p.L = frame_len; p.dk = d_k; p.dv = d_v;
+    p.F = T / frame_len;
+    return workspace_for(p);
+}
+
+const char *gdn_status_string(int s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_SHAPE: return "GDN_ERR_SHAPE";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_ALIGNMENT: return "GDN_ERR_ALIGNMENT";
+        case GDN_ERR_NO_MEMORY: return "GDN_ERR_NO_MEMORY";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_NONFINITE: return "GDN_ERR_NONFINITE";
+        case GDN_ERR_NOT_IMPLEMENTED: return "GDN_ERR_NOT_IMPLEMENTED";
+        default: return "GDN_ERR_UNKNOWN";
+    }
+}
+
+const char *gdn_last_error(void) { return g_err; }
+
+int gdn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,86 @@
+// gdn_internal.h -- shared host/device definitions of the CUDA library.
+//
+// Chunkwise evaluation of the token-wise gated delta rule with one chunk per
+// frame (SANA-WM summary, paper-graph-ui, "Memory-Efficient Long-Context
+// Modeling (Section 3.2)", paragraph "Frame-wise Gated DeltaNet (GDN)": one
+// latent frame per recurrence step, all of the frame's tokens in parallel).
+//
+// Per (b, h) chain and frame f, with L = frame_len tokens i, j in [0, L) and
+//   G_i   = sum_{m <= i} log alpha_m           (inclusive, within the frame)
+//   Sig   = S^T  (d_k x d_v), Sig_0 = the state entering the frame,
+// the substitution u_i = beta_i (v_i - alpha_i S_{i-1} k_i) turns the update
+// into S_i = alpha_i S_{i-1} + u_i k_i^T, hence
+//   (I + A) [Ub | W] = [diag(beta) V | diag(beta e^G) K],
+//   A_ij = beta_i e^{G_i - G_j} k_i.k_j  (j < i),           -- kernel 1
+//   U = Ub - W Sig_0,
+//   M = e^{G_L} I - Kt^T W,  N = Kt^T Ub,  Kt = diag(e^{G_L - G}) K   -- kernel 2
+//   Sig_next = M Sig_0 + N                                  -- kernel 3 (scan over frames)
+//   O = diag(e^G) Q Sig_0 + tril_incl(Q K^T o e^{G_i - G_j}) U  -- kernel 4
+// Every decay factor used is e^{G_i - G_j} with j <= i (<= 1), so no factor
+// overflows; log alpha is clamped at -200 so alpha = 0 (a full reset) stays
+// finite (e^{-200} is 0 in fp32).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+constexpr float kLogAlphaFloor = -200.0f;
+
+struct Problem {
+    int dtype;  // GDN_DTYPE_BF16 / GDN_DTYPE_F32
+    const void *q, *k, *v;
+    const float *alpha, *beta;
+    const float *S_in;
+    float *S_out;
+    void *o;
+    int B, H;
+    long long T;
+    int L;       // frame_len
+    int dk, dv;
+    long long F;  // frames per chain, T / L
+    int reverse;
+    int accumulate;
+    long long reset_every;  // tokens; 0 = never
+};
+
+// Physical token index of logical position i of logical frame f.  The
+// reversed-time scan visits frames and the tokens inside them backwards.
+__host__ __device__ __forceinline__ long long phys_token(const Problem &p, long long f, int i) {
+    return p.reverse ? ((p.F - 1 - f) * p.L + (p.L - 1 - i)) : (f * p.L + i);
+}
+
+// Row of token t of chain (b, h) in a [B, T, H, *] tensor.
+__host__ __device__ __forceinline__ long long tok_row(const Problem &p, int b, int h, long long t) {
+    return ((long long)b * p.T + t) * p.H + h;
+}
+
+// Does the state restart from zero before logical frame f (f > 0)?
+__host__ __device__ __forceinline__ bool frame_resets(const Problem &p, long long f) {
+    if (p.reset_every <= 0 || f == 0) return false;
+    if (!p.reverse) return (f * p.L) % p.reset_every == 0;
+    const long long pf = p.F - 1 - f;  // physical frame visited at logical f
+    return ((pf + 1) * p.L) % p.reset_every == 0;
+}
+
+// Workspace carved out of one allocation.
+struct Workspace {
+    void *base = nullptr;
+    size_t bytes = 0;
+};
+
+// Optional stage timing: when `ev` is non-null it holds GDN_NUM_STAGES + 1
+// events; ev[i] is recorded before stage i and ev[GDN_NUM_STAGES] after the last.
+inline cudaError_t mark(cudaEvent_t *ev, int i, cudaStream_t s) {
+    return ev ? cudaEventRecord(ev[i], s) : cudaSuccess;
+}
+
+size_t simt_workspace_bytes(const Problem &p);
+cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
+
+}  // namespace gdn

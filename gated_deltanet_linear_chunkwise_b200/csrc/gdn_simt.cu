@@ -1,0 +1,554 @@
+// gdn_simt.cu -- CUDA-core (fp32 FMA) kernels of the chunkwise gated delta rule.
+//
+// This is the full-precision path: it serves gdn_fwd_f32 / gdn_step_f32
+// (fp32 q/k/v/o, fp32 arithmetic, fp64 gate prefix sums) and any shape the
+// tensor-core path does not take.  The four kernels follow the chunk = frame
+// decomposition written out in gdn_internal.h:
+//   k1  intra-frame: A = strict_lower(diag(beta) K K^T o Gamma) and the
+//       blocked forward substitution (I + A)[Ub | W] = [beta V | beta e^G K]
+//   k2  per-frame affine map of the state: M = e^{G_L} I - Kt^T W, N = Kt^T Ub
+//   k3  scan over frames: Sig_f+1 = M_f Sig_f + N_f (state kept on chip)
+//   k4  U = Ub - W Sig_f and O = diag(e^G) Q Sig_f + tril_incl(Q K^T o Gamma) U
+// Row blocks are 32 tokens; every thread owns one output column and keeps
+// the block's 32 (or 16) rows of that column in registers.
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int RB = 32;        // token rows per block
+constexpr int NT = 256;       // threads per CTA
+constexpr int SCAN_COLS = 16; // state columns per scan CTA
+
+__host__ __device__ constexpr size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+
+template <typename T> __device__ __forceinline__ float ld_in(const T *p, long long i);
+template <> __device__ __forceinline__ float ld_in<float>(const float *p, long long i) { return p[i]; }
+template <> __device__ __forceinline__ float ld_in<__nv_bfloat16>(const __nv_bfloat16 *p, long long i) {
+    return __bfloat162float(p[i]);
+}
+template <typename T> __device__ __forceinline__ void st_out(T *p, long long i, float x);
+template <> __device__ __forceinline__ void st_out<float>(float *p, long long i, float x) { p[i] = x; }
+template <> __device__ __forceinline__ void st_out<__nv_bfloat16>(__nv_bfloat16 *p, long long i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+template <typename TG> __device__ __forceinline__ TG log_gate(float a) {
+    TG lg = a > 0.f ? (TG)log((TG)a) : (TG)kLogAlphaFloor;
+    return lg < (TG)kLogAlphaFloor ? (TG)kLogAlphaFloor : lg;
+}
+
+// Inclusive prefix of log(alpha) over logical frame f of chain (b,h) into
+// sG[0..L), and the frame's beta into sB[0..L).  Block-wide scan: each
+// thread takes a contiguous run, warps scan their totals with shuffles.
+template <typename TG>
+__device__ void frame_gates(const Problem &p, int b, int h, long long f, TG *sG, float *sB, TG *sScr) {
+    const int L = p.L, tid = threadIdx.x, nt = blockDim.x;
+    const int per = (L + nt - 1) / nt;
+    const int i0 = tid * per, i1 = min(i0 + per, L);
+    TG run = 0;
+    for (int i = i0; i < i1; ++i) {
+        const long long row = tok_row(p, b, h, phys_token(p, f, i));
+        run += log_gate<TG>(p.alpha[row]);
+        sG[i] = run;
+        sB[i] = p.beta[row];
+    }
+    const int lane = tid & 31, warp = tid >> 5, nw = (nt + 31) >> 5;
+    TG x = run;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        TG y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) sScr[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        TG w = lane < nw ? sScr[lane] : (TG)0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            TG y = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += y;
+        }
+        if (lane < nw) sScr[lane] = w;
+    }
+    __syncthreads();
+    const TG offset = (x - run) + (warp > 0 ? sScr[warp - 1] : (TG)0);
+    for (int i = i0; i < i1; ++i) sG[i] += offset;
+    __syncthreads();
+}
+
+// Shared-memory carve-up shared by the kernels that scan a frame's gates.
+template <typename TG> struct GateSmem {
+    static __host__ __device__ size_t bytes(int L) {
+        return align16(sizeof(TG) * (size_t)L) + align16(sizeof(TG) * 32) + align16(sizeof(float) * (size_t)L);
+    }
+};
+
+// ---------------------------------------------------------------- k1 intra-frame
+template <typename TIn, typename TG>
+__global__ void __launch_bounds__(NT) k1_intra_simt(Problem p, float *__restrict__ X) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int L = p.L, dk = p.dk, dv = p.dv, nc = dk + dv;
+    const long long fh = blockIdx.x;
+    const long long f = fh % p.F, chain = fh / p.F;
+    const int h = (int)(chain % p.H), b = (int)(chain / p.H);
+
+    unsigned char *ptr = smem;
+    TG *sG = (TG *)ptr;            ptr += align16(sizeof(TG) * L);
+    TG *sScr = (TG *)ptr;          ptr += align16(sizeof(TG) * 32);
+    float *sB = (float *)ptr;      ptr += align16(sizeof(float) * L);
+    float *sKiT = (float *)ptr;    ptr += sizeof(float) * dk * RB;   // [dk][32]
+    float *sKjT = (float *)ptr;    ptr += sizeof(float) * dk * RB;   // [dk][32]
+    float *sAT = (float *)ptr;     ptr += sizeof(float) * RB * RB;   // A^T [s][r]
+    float *sX = (float *)ptr;                                        // [32][nc]
+
+    frame_gates<TG>(p, b, h, f, sG, sB, sScr);
+    const TIn *k = (const TIn *)p.k, *v = (const TIn *)p.v;
+    float *Xf = X + fh * (long long)L * nc;
+    const int tid = threadIdx.x;
+    const int nblk = (L + RB - 1) / RB;
+
+    for (int ib = 0; ib < nblk; ++ib) {
+        const int r0 = ib * RB, nr = min(RB, L - r0);
+        for (int e = tid; e < RB * dk; e += NT) {
+            const int r = e / dk, c = e - r * dk;
+            float val = 0.f;
+            if (r < nr) val = ld_in(k, tok_row(p, b, h, phys_token(p, f, r0 + r)) * dk + c);
+            sKiT[c * RB + r] = val;
+        }
+        float acc[RB];
+#pragma unroll
+        for (int r = 0; r < RB; ++r) acc[r] = 0.f;
+        if (tid < nc) {
+#pragma unroll
+            for (int r = 0; r < RB; ++r) {
+                if (r < nr) {
+                    const long long row = tok_row(p, b, h, phys_token(p, f, r0 + r));
+                    const float be = sB[r0 + r];
+                    acc[r] = (tid < dv) ? be * ld_in(v, row * dv + tid)
+                                        : be * expf((float)sG[r0 + r]) * ld_in(k, row * dk + (tid - dv));
+                }
+            }
+        }
+        __syncthreads();
+        for (int jb = 0; jb <= ib; ++jb) {
+            const int s0 = jb * RB, ns = min(RB, L - s0);
+            const bool diag = (jb == ib);
+            if (!diag) {
+                for (int e = tid; e < RB * dk; e += NT) {
+                    const int s = e / dk, c = e - s * dk;
+                    sKjT[c * RB + s] = ld_in(k, tok_row(p, b, h, phys_token(p, f, s0 + s)) * dk + c);
+                }
+                for (int e = tid; e < RB * nc; e += NT) sX[e] = Xf[(long long)s0 * nc + e];
+            }
+            __syncthreads();
+            const float *KjT = diag ? sKiT : sKjT;
+            {
+                const int r = tid & 31, sg = tid >> 5;
+                float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+                for (int c = 0; c < dk; ++c) {
+                    const float a = sKiT[c * RB + r];
+                    const float4 kb = *reinterpret_cast<const float4 *>(&KjT[c * RB + sg * 4]);
+                    d0 += a * kb.x; d1 += a * kb.y; d2 += a * kb.z; d3 += a * kb.w;
+                }
+                const float dd[4] = {d0, d1, d2, d3};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int s = sg * 4 + u;
+                    float val = 0.f;
+                    if (r < nr && s < ns && (!diag || s < r))
+                        val = sB[r0 + r] * expf((float)(sG[r0 + r] - sG[s0 + s])) * dd[u];
+                    sAT[s * RB + r] = val;
+                }
+            }
+            __syncthreads();
+            if (tid < nc) {
+                if (!diag) {
+                    for (int s = 0; s < RB; ++s) {
+                        const float x = sX[s * nc + tid];
+#pragma unroll
+                        for (int r4 = 0; r4 < RB / 4; ++r4) {
+                            const float4 a = *reinterpret_cast<const float4 *>(&sAT[s * RB + r4 * 4]);
+                            acc[r4 * 4 + 0] -= a.x * x;
+                            acc[r4 * 4 + 1] -= a.y * x;
+                            acc[r4 * 4 + 2] -= a.z * x;
+                            acc[r4 * 4 + 3] -= a.w * x;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int r = 1; r < RB; ++r) {
+                        float x = acc[r];
+#pragma unroll
+                        for (int s = 0; s < r; ++s) x -= sAT[s * RB + r] * acc[s];
+                        acc[r] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        if (tid < nc) {
+#pragma unroll
+            for (int r = 0; r < RB; ++r)
+                if (r < nr) Xf[(long long)(r0 + r) * nc + tid] = acc[r];
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- k2 frame transition
+// grid (frame-heads, ceil(dk/32)); the block owns rows m0..m0+31 of [N | M].
+template <typename TIn, typename TG>
+__global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const float *__restrict__ X,
+                                                         float *__restrict__ Mb, float *__restrict__ Nb) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int L = p.L, dk = p.dk, dv = p.dv, nc = dk + dv;
+    const long long fh = blockIdx.x;
+    const long long f = fh % p.F, chain = fh / p.F;
+    const int h = (int)(chain % p.H), b = (int)(chain / p.H);
+    const int m0 = blockIdx.y * 32, nm = min(32, dk - m0);
+
+    unsigned char *ptr = smem;
+    TG *sG = (TG *)ptr;            ptr += align16(sizeof(TG) * L);
+    TG *sScr = (TG *)ptr;          ptr += align16(sizeof(TG) * 32);
+    float *sB = (float *)ptr;      ptr += align16(sizeof(float) * L);
+    float *sKt = (float *)ptr;     ptr += sizeof(float) * RB * 32;   // [s][m]
+    float *sX = (float *)ptr;                                        // [32][nc]
+
+    frame_gates<TG>(p, b, h, f, sG, sB, sScr);
+    const TIn *k = (const TIn *)p.k;
+    const float *Xf = X + fh * (long long)L * nc;
+    const int tid = threadIdx.x;
+    const TG GL = sG[L - 1];
+
+    float acc[32];
+#pragma unroll
+    for (int m = 0; m < 32; ++m) acc[m] = 0.f;
+    for (int s0 = 0; s0 < L; s0 += RB) {
+        const int ns = min(RB, L - s0);
+        for (int e = tid; e < RB * 32; e += NT) {
+            const int s = e >> 5, m = e & 31;
+            float val = 0.f;
+            if (s < ns && m < nm)
+                val = expf((float)(GL - sG[s0 + s])) *
+                      ld_in(k, tok_row(p, b, h, phys_token(p, f, s0 + s)) * dk + m0 + m);
+            sKt[e] = val;
+        }
+        for (int e = tid; e < RB * nc; e += NT) {
+            const int s = e / nc;
+            sX[e] = (s < ns) ? Xf[(long long)s0 * nc + e] : 0.f;
+        }
+        __syncthreads();
+        if (tid < nc) {
+            for (int s = 0; s < RB; ++s) {
+                const float x = sX[s * nc + tid];
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float4 kk = *reinterpret_cast<const float4 *>(&sKt[s * 32 + m4 * 4]);
+                    acc[m4 * 4 + 0] += kk.x * x;
+                    acc[m4 * 4 + 1] += kk.y * x;
+                    acc[m4 * 4 + 2] += kk.z * x;
+                    acc[m4 * 4 + 3] += kk.w * x;
+                }
+            }
+        }
+        __syncthreads();
+    }
+    if (tid < nc) {
+        const float eGL = expf((float)GL);
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+            if (m < nm) {
+                const int row = m0 + m;
+                if (tid < dv) {
+                    Nb[(fh * dk + row) * (long long)dv + tid] = acc[m];
+                } else {
+                    const int j = tid - dv;
+                    Mb[(fh * dk + row) * (long long)dk + j] = (row == j ? eGL : 0.f) - acc[m];
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- k3 scan over frames
+// grid (B*H, ceil(dv/16)); the block carries 16 columns of Sig = S^T through
+// all frames of its chain, writing the state entering each frame to Sig_in.
+__global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__restrict__ Mb,
+                                                   const float *__restrict__ Nb, float *__restrict__ SigIn) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int dk = p.dk, dv = p.dv;
+    const long long chain = blockIdx.x;
+    const int c0 = blockIdx.y * SCAN_COLS, ncol = min(SCAN_COLS, dv - c0);
+    float *sM = (float *)smem;                       // [dk][dk+1]
+    float *sS = sM + dk * (dk + 1);                  // [dk][16]
+    const int tid = threadIdx.x, c = tid & 15, g = tid >> 4;
+    const int ld = dk + 1;
+
+    for (int e = tid; e < dk * SCAN_COLS; e += NT) {
+        const int m = e >> 4, cc = e & 15;
+        float val = 0.f;
+        if (p.S_in && cc < ncol) val = p.S_in[(chain * dv + c0 + cc) * (long long)dk + m];
+        sS[e] = val;
+    }
+    constexpr int MAXR = 128 / 16;
+    for (long long f = 0; f < p.F; ++f) {
+        const long long fh = chain * p.F + f;
+        __syncthreads();
+        if (frame_resets(p, f))
+            for (int e = tid; e < dk * SCAN_COLS; e += NT) sS[e] = 0.f;
+        __syncthreads();
+        for (int e = tid; e < dk * SCAN_COLS; e += NT) {
+            const int m = e >> 4, cc = e & 15;
+            if (cc < ncol) SigIn[(fh * dk + m) * (long long)dv + c0 + cc] = sS[e];
+        }
+        const float *Mf = Mb + fh * (long long)dk * dk;
+        for (int e = tid; e < dk * dk; e += NT) {
+            const int m = e / dk, l = e - m * dk;
+            sM[m * ld + l] = Mf[e];
+        }
+        __syncthreads();
+        float nv[MAXR];
+#pragma unroll
+        for (int i = 0; i < MAXR; ++i) {
+            const int m = g + 16 * i;
+            float a = 0.f;
+            if (m < dk && c < ncol) {
+                a = Nb[(fh * dk + m) * (long long)dv + c0 + c];
+                for (int l = 0; l < dk; ++l) a += sM[m * ld + l] * sS[l * SCAN_COLS + c];
+            }
+            nv[i] = a;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < MAXR; ++i) {
+            const int m = g + 16 * i;
+            if (m < dk) sS[m * SCAN_COLS + c] = nv[i];
+        }
+    }
+    __syncthreads();
+    if (p.S_out) {
+        for (int e = tid; e < dk * SCAN_COLS; e += NT) {
+            const int m = e >> 4, cc = e & 15;
+            if (cc < ncol) p.S_out[(chain * dv + c0 + cc) * (long long)dk + m] = sS[e];
+        }
+    }
+}
+
+// ---------------------------------------------------------------- k4 output
+// grid (frame-heads); for each 32-row block I in order: U_I = Ub_I - W_I Sig
+// (kept in the U workspace for later blocks), then
+// O_I = diag(e^G) Q_I Sig + sum_{J <= I} mask(Q_I K_J^T o Gamma) U_J.
+template <typename TIn, typename TG>
+__global__ void __launch_bounds__(NT) k4_output_simt(Problem p, const float *__restrict__ X,
+                                                     const float *__restrict__ SigIn, float *__restrict__ U) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int L = p.L, dk = p.dk, dv = p.dv, nc = dk + dv;
+    const long long fh = blockIdx.x;
+    const long long f = fh % p.F, chain = fh / p.F;
+    const int h = (int)(chain % p.H), b = (int)(chain / p.H);
+
+    unsigned char *ptr = smem;
+    TG *sG = (TG *)ptr;            ptr += align16(sizeof(TG) * L);
+    TG *sScr = (TG *)ptr;          ptr += align16(sizeof(TG) * 32);
+    float *sB = (float *)ptr;      ptr += align16(sizeof(float) * L);
+    float *sSig = (float *)ptr;    ptr += sizeof(float) * dk * dv;   // [dk][dv]
+    float *sQT = (float *)ptr;     ptr += sizeof(float) * dk * RB;   // [dk][32]
+    float *sWT = (float *)ptr;     ptr += sizeof(float) * dk * RB;   // [dk][32]
+    float *sKT = (float *)ptr;     ptr += sizeof(float) * dk * RB;   // [dk][32]
+    float *sPT = (float *)ptr;     ptr += sizeof(float) * RB * RB;   // [s][r]
+    float *sU = (float *)ptr;                                        // [32][dv]
+
+    frame_gates<TG>(p, b, h, f, sG, sB, sScr);
+    const TIn *q = (const TIn *)p.q, *k = (const TIn *)p.k;
+    TIn *o = (TIn *)p.o;
+    const float *Xf = X + fh * (long long)L * nc;
+    float *Uf = U + fh * (long long)L * dv;
+    const float *Sf = SigIn + fh * (long long)dk * dv;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < dk * dv; e += NT) sSig[e] = Sf[e];
+
+    const int c = tid & 127, rh = tid >> 7;  // column, half of the row block
+    const bool active = c < dv;
+    const int nblk = (L + RB - 1) / RB;
+    for (int ib = 0; ib < nblk; ++ib) {
+        const int r0 = ib * RB, nr = min(RB, L - r0);
+        for (int e = tid; e < RB * dk; e += NT) {
+            const int r = e / dk, cc = e - r * dk;
+            float qv = 0.f, wv = 0.f;
+            if (r < nr) {
+                qv = ld_in(q, tok_row(p, b, h, phys_token(p, f, r0 + r)) * dk + cc);
+                wv = Xf[(long long)(r0 + r) * nc + dv + cc];
+            }
+            sQT[cc * RB + r] = qv;
+            sWT[cc * RB + r] = wv;
+        }
+        __syncthreads();
+        float acc[16];
+        if (active) {
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int rr = rh * 16 + r;
+                acc[r] = (rr < nr) ? Xf[(long long)(r0 + rr) * nc + c] : 0.f;
+            }
+            for (int l = 0; l < dk; ++l) {
+                const float sg = sSig[l * dv + c];
+#pragma unroll
+                for (int r4 = 0; r4 < 4; ++r4) {
+                    const float4 w = *reinterpret_cast<const float4 *>(&sWT[l * RB + rh * 16 + r4 * 4]);
+                    acc[r4 * 4 + 0] -= w.x * sg;
+                    acc[r4 * 4 + 1] -= w.y * sg;
+                    acc[r4 * 4 + 2] -= w.z * sg;
+                    acc[r4 * 4 + 3] -= w.w * sg;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int rr = rh * 16 + r;
+                if (rr < nr) Uf[(long long)(r0 + rr) * dv + c] = acc[r];
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+            for (int l = 0; l < dk; ++l) {
+                const float sg = sSig[l * dv + c];
+#pragma unroll
+                for (int r4 = 0; r4 < 4; ++r4) {
+                    const float4 qq = *reinterpret_cast<const float4 *>(&sQT[l * RB + rh * 16 + r4 * 4]);
+                    acc[r4 * 4 + 0] += qq.x * sg;
+                    acc[r4 * 4 + 1] += qq.y * sg;
+                    acc[r4 * 4 + 2] += qq.z * sg;
+                    acc[r4 * 4 + 3] += qq.w * sg;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int rr = rh * 16 + r;
+                acc[r] *= (rr < nr) ? expf((float)sG[r0 + rr]) : 0.f;
+            }
+        }
+        __syncthreads();  // this block's U rows are visible to the whole CTA
+        for (int jb = 0; jb <= ib; ++jb) {
+            const int s0 = jb * RB, ns = min(RB, L - s0);
+            const bool diag = (jb == ib);
+            for (int e = tid; e < RB * dk; e += NT) {
+                const int s = e / dk, cc = e - s * dk;
+                sKT[cc * RB + s] = (s < ns) ? ld_in(k, tok_row(p, b, h, phys_token(p, f, s0 + s)) * dk + cc) : 0.f;
+            }
+            for (int e = tid; e < RB * dv; e += NT) {
+                const int s = e / dv;
+                sU[e] = (s < ns) ? Uf[(long long)s0 * dv + e] : 0.f;
+            }
+            __syncthreads();
+            {
+                const int r = tid & 31, sg = tid >> 5;
+                float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+                for (int cc = 0; cc < dk; ++cc) {
+                    const float a = sQT[cc * RB + r];
+                    const float4 kb = *reinterpret_cast<const float4 *>(&sKT[cc * RB + sg * 4]);
+                    d0 += a * kb.x; d1 += a * kb.y; d2 += a * kb.z; d3 += a * kb.w;
+                }
+                const float dd[4] = {d0, d1, d2, d3};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int s = sg * 4 + u;
+                    float val = 0.f;
+                    if (r < nr && s < ns && (!diag || s <= r))
+                        val = expf((float)(sG[r0 + r] - sG[s0 + s])) * dd[u];
+                    sPT[s * RB + r] = val;
+                }
+            }
+            __syncthreads();
+            if (active) {
+                for (int s = 0; s < RB; ++s) {
+                    const float u = sU[s * dv + c];
+#pragma unroll
+                    for (int r4 = 0; r4 < 4; ++r4) {
+                        const float4 pp = *reinterpret_cast<const float4 *>(&sPT[s * RB + rh * 16 + r4 * 4]);
+                        acc[r4 * 4 + 0] += pp.x * u;
+                        acc[r4 * 4 + 1] += pp.y * u;
+                        acc[r4 * 4 + 2] += pp.z * u;
+                        acc[r4 * 4 + 3] += pp.w * u;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        if (active) {
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int rr = rh * 16 + r;
+                if (rr < nr) {
+                    const long long idx = tok_row(p, b, h, phys_token(p, f, r0 + rr)) * dv + c;
+                    float val = acc[r];
+                    if (p.accumulate) val += ld_in(o, idx);
+                    st_out(o, idx, val);
+                }
+            }
+        }
+    }
+}
+
+struct SimtLayout {
+    size_t X, U, M, N, Sig, total;
+};
+
+__host__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+SimtLayout simt_layout(const Problem &p) {
+    const size_t nfh = (size_t)p.B * p.H * p.F;
+    SimtLayout lay;
+    size_t off = 0;
+    lay.X = off;   off += align256(sizeof(float) * nfh * p.L * (p.dk + p.dv));
+    lay.U = off;   off += align256(sizeof(float) * nfh * p.L * p.dv);
+    lay.M = off;   off += align256(sizeof(float) * nfh * p.dk * p.dk);
+    lay.N = off;   off += align256(sizeof(float) * nfh * p.dk * p.dv);
+    lay.Sig = off; off += align256(sizeof(float) * nfh * p.dk * p.dv);
+    lay.total = off;
+    return lay;
+}
+
+template <typename TIn, typename TG>
+cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
+    const SimtLayout lay = simt_layout(p);
+    char *base = (char *)ws;
+    float *X = (float *)(base + lay.X), *U = (float *)(base + lay.U);
+    float *Mb = (float *)(base + lay.M), *Nb = (float *)(base + lay.N), *Sig = (float *)(base + lay.Sig);
+    const long long nfh = (long long)p.B * p.H * p.F;
+    const int dk = p.dk, dv = p.dv, nc = dk + dv;
+    const size_t gsm = GateSmem<TG>::bytes(p.L);
+
+    const size_t sm1 = gsm + sizeof(float) * (2 * dk * RB + RB * RB + RB * nc);
+    const size_t sm2 = gsm + sizeof(float) * (RB * 32 + RB * nc);
+    const size_t sm3 = sizeof(float) * (dk * (dk + 1) + dk * SCAN_COLS);
+    const size_t sm4 = gsm + sizeof(float) * (dk * dv + 3 * dk * RB + RB * RB + RB * dv);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k1_intra_simt<TIn, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1))) return e;
+    if ((e = cudaFuncSetAttribute(k2_transition_simt<TIn, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2))) return e;
+    if ((e = cudaFuncSetAttribute(k3_scan_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3))) return e;
+    if ((e = cudaFuncSetAttribute(k4_output_simt<TIn, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm4))) return e;
+
+    if ((e = mark(ev, 0, s))) return e;
+    k1_intra_simt<TIn, TG><<<(unsigned)nfh, NT, sm1, s>>>(p, X);
+    if ((e = cudaGetLastError())) return e;
+    if ((e = mark(ev, 1, s))) return e;
+    k2_transition_simt<TIn, TG><<<dim3((unsigned)nfh, (dk + 31) / 32), NT, sm2, s>>>(p, X, Mb, Nb);
+    if ((e = cudaGetLastError())) return e;
+    if ((e = mark(ev, 2, s))) return e;
+    k3_scan_simt<<<dim3((unsigned)(p.B * p.H), (dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm3, s>>>(p, Mb, Nb, Sig);
+    if ((e = cudaGetLastError())) return e;
+    if ((e = mark(ev, 3, s))) return e;
+    k4_output_simt<TIn, TG><<<(unsigned)nfh, NT, sm4, s>>>(p, X, Sig, U);
+    if ((e = cudaGetLastError())) return e;
+    return mark(ev, 4, s);
+}
+
+}  // namespace
+
+size_t simt_workspace_bytes(const Problem &p) { return simt_layout(p).total; }
+
+cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
+    if (p.dtype == GDN_DTYPE_F32) return launch_typed<float, double>(p, ws, s, ev);
+    return launch_typed<__nv_bfloat16, float>(p, ws, s, ev);
+}
+
+}  // namespace gdn

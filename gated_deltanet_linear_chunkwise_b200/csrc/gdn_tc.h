@@ -1,0 +1,13 @@
+// gdn_tc.h -- tensor-core (tcgen05 / TMEM / TMA) path for bf16 inputs.
+#pragma once
+#include "gdn_internal.h"
+
+namespace gdn {
+
+// Does the tensor-core path take this problem?  (Otherwise the CUDA-core
+// path in gdn_simt.cu runs it.)
+bool tc_supports(const Problem &p);
+size_t tc_workspace_bytes(const Problem &p);
+cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
+
+}  // namespace gdn

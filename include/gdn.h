@@ -1,0 +1,181 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) chunkwise gated delta rule.
+ *
+ * The operation (SANA-WM summary, paper-graph-ui, section 3.2
+ * "Memory-Efficient Long-Context Modeling", paragraph "Frame-wise Gated
+ * DeltaNet (GDN)", the token-wise update; SANA-WM teardown, thesatyajit,
+ * section "The linear part: a gated delta rule, one frame per step"), per
+ * batch b and head h, over tokens t = 0..T-1:
+ *
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t                      (the state AFTER token t's update)
+ *
+ * S is d_v x d_k and S_0 = S_in (or 0).  The library evaluates it in
+ * chunkwise form with one chunk per frame of frame_len tokens (one latent
+ * video frame per recurrence step, same paragraph); the result equals the
+ * token loop up to rounding.
+ *
+ * Layouts (all contiguous, row-major; the pages' D x S frame matrices are
+ * notation only):
+ *   q, k        [B, T, H, d_k]      token-major, as a fused QKV projection emits them
+ *   v, o        [B, T, H, d_v]
+ *   alpha, beta [B, T, H]  fp32     alpha in [0,1] (linear, not log), beta in [0,1]
+ *   S_in, S_out [B, H, d_v, d_k] fp32  (S as the page writes it: o = S q)
+ *   frame f covers tokens [f*frame_len, (f+1)*frame_len)
+ *
+ * Pointers: every tensor pointer is a DEVICE pointer owned by the caller
+ * (except gdn_fwd_host, whose tensors are host pointers).  The library keeps
+ * no pointer after the call returns.
+ *
+ * Supported: T % frame_len == 0; 1 <= frame_len <= 4096; d_k, d_v in
+ * {16, 32, ..., 128}; every base pointer 16-byte aligned; B*T*H*max(d_k,d_v)
+ * < 2^62 and B*H*(T/frame_len) < 2^31.
+ *
+ * Errors: arguments are validated before anything is enqueued; on a
+ * validation error nothing is launched and no output is touched.  A failed
+ * launch returns GDN_ERR_CUDA.  Execution is asynchronous on `stream`, so a
+ * device-side fault surfaces at the caller's next synchronisation.  No C++
+ * exception crosses this ABI.  gdn_last_error() gives a thread-local text
+ * for the most recent failure on the calling thread.
+ *
+ * S_in == NULL means a zero initial state; S_out == NULL means the final
+ * state is not stored (repeated denoising passes over one chunk read the
+ * same S_in); S_in == S_out is allowed (the state is updated in place).
+ * S_in and S_out may not partially overlap, and no output may overlap an
+ * input other than that S_in == S_out case.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-compatible with cudaStream_t / CUstream; NULL = the legacy default stream. */
+typedef struct CUstream_st *gdn_stream_t;
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,     /* null required pointer, negative size, bad flag */
+    GDN_ERR_SHAPE = 2,           /* T not a multiple of frame_len, size overflow */
+    GDN_ERR_UNSUPPORTED = 3,     /* head dim or frame length outside the supported set */
+    GDN_ERR_ALIGNMENT = 4,       /* a base pointer is not 16-byte aligned */
+    GDN_ERR_NO_MEMORY = 5,       /* workspace allocation failed or caller workspace too small */
+    GDN_ERR_CUDA = 6,            /* a CUDA runtime/driver call or a launch failed */
+    GDN_ERR_TIMEOUT = 7,         /* a bounded device-side wait gave up */
+    GDN_ERR_NONFINITE = 8,       /* finite-check requested and o / S_out holds NaN or Inf */
+    GDN_ERR_NOT_IMPLEMENTED = 9  /* a flag combination this build does not provide */
+} gdn_status;
+
+enum { GDN_DTYPE_BF16 = 0, GDN_DTYPE_F32 = 1 };
+
+/*
+ * gdn_fwd -- forward scan, bf16 q/k/v/o (fp32 alpha, beta and state).
+ * Tensor-core path: bf16 products with fp32 accumulation, fp32 gate math and
+ * fp32 state.  Returns a gdn_status.
+ */
+int gdn_fwd(const void *q, const void *k, const void *v,
+            const float *alpha, const float *beta,
+            const float *S_in, float *S_out, void *o,
+            int B, int H, long long T, int frame_len, int d_k, int d_v,
+            gdn_stream_t stream);
+
+/* gdn_fwd_f32 -- same operation with fp32 q/k/v/o; fp32 arithmetic
+ * throughout with fp64 gate prefix sums (for the tight-tolerance path). */
+int gdn_fwd_f32(const float *q, const float *k, const float *v,
+                const float *alpha, const float *beta,
+                const float *S_in, float *S_out, float *o,
+                int B, int H, long long T, int frame_len, int d_k, int d_v,
+                gdn_stream_t stream);
+
+/*
+ * gdn_step -- one call of a chunk-causal rollout: identical to gdn_fwd but
+ * S_in is required (the state carried from the previous call).  Chaining
+ * gdn_step calls S_out -> S_in over consecutive token ranges equals one
+ * gdn_fwd over their concatenation (SANA-WM summary, section 3.1 "Stage 4:
+ * Chunk-Causal Fine-Tuning", the global forward scan that carries past
+ * context across chunks).
+ */
+int gdn_step(const void *q, const void *k, const void *v,
+             const float *alpha, const float *beta,
+             const float *S_in, float *S_out, void *o,
+             int B, int H, long long T, int frame_len, int d_k, int d_v,
+             gdn_stream_t stream);
+
+int gdn_step_f32(const float *q, const float *k, const float *v,
+                 const float *alpha, const float *beta,
+                 const float *S_in, float *S_out, float *o,
+                 int B, int H, long long T, int frame_len, int d_k, int d_v,
+                 gdn_stream_t stream);
+
+/*
+ * Extended call.  Fields not listed for a flag are as in gdn_fwd.
+ *   struct_size     sizeof(gdn_args) as compiled by the caller (ABI guard).
+ *   dtype           GDN_DTYPE_BF16 or GDN_DTYPE_F32 (q/k/v/o element type).
+ *   workspace       optional device scratch of workspace_bytes bytes, at
+ *                   least gdn_workspace_bytes(...) and 256-byte aligned; NULL
+ *                   lets the call take stream-ordered memory (cudaMallocAsync)
+ *                   and return it before the call returns.
+ *   reverse         1: reversed-time scan (tokens visited T-1..0, each gate
+ *                   applied at its own token; SANA-WM summary, section 3.2,
+ *                   paragraph "Bidirectional and Chunk-Causal GDN Variants").
+ *   accumulate_o    1: o += result instead of o = result (sums the forward
+ *                   and reversed scans of the bidirectional variant).
+ *   reset_every     > 0: the state restarts from zero at each boundary of
+ *                   reset_every tokens, counted from token 0 (with reverse:
+ *                   the chunk-causal reversed scan); a multiple of
+ *                   frame_len.  0: no reset.
+ *   check_finite    1: after the pass, scan o (and S_out) and return
+ *                   GDN_ERR_NONFINITE if any NaN/Inf is found (synchronises
+ *                   the stream).
+ *   stage_ms        optional HOST array of GDN_NUM_STAGES floats: when set,
+ *                   CUDA events bracket each kernel stage on `stream` and the
+ *                   call synchronises the stream and writes each stage's
+ *                   device time in ms (tracing; off in production calls).
+ */
+typedef struct gdn_args {
+    int struct_size;
+    int dtype;
+    const void *q, *k, *v;
+    const float *alpha, *beta;
+    const float *S_in;
+    float *S_out;
+    void *o;
+    int B, H;
+    long long T;
+    int frame_len, d_k, d_v;
+    void *workspace;
+    size_t workspace_bytes;
+    int reverse;
+    int accumulate_o;
+    long long reset_every;
+    int check_finite;
+    gdn_stream_t stream;
+    float *stage_ms;
+} gdn_args;
+
+/* Kernel stages reported through gdn_args.stage_ms, in launch order:
+ * 0 intra-frame solve, 1 frame transition, 2 scan over frames, 3 output. */
+enum { GDN_NUM_STAGES = 4 };
+
+int gdn_fwd_ex(const gdn_args *a);
+
+/* Device scratch a call with these sizes needs (0 if the sizes are invalid). */
+size_t gdn_workspace_bytes(int B, int H, long long T, int frame_len, int d_k, int d_v, int dtype);
+
+/* Static text for a status code; never NULL. */
+const char *gdn_status_string(int status);
+
+/* Thread-local detail of the last failure on this thread ("" if none). */
+const char *gdn_last_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

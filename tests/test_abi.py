@@ -1,0 +1,103 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header
+declares, its argument struct matches the header, and argument validation
+returns the documented status before anything is enqueued.  The pointers
+below are never dereferenced: every call is rejected by validation first.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_deltanet_linear_chunkwise_b200 as g
+from gated_deltanet_linear_chunkwise_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+FAKE = 1 << 40  # aligned, never dereferenced (validation rejects first)
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_\w+)\s*\(", src)))
+
+
+def test_header_declarations_all_exported():
+    lib = g.load_library()
+    declared = _declared()
+    assert set(binding.EXPORTS) <= set(declared)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_exports_via_nm():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    syms = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    for name in _declared():
+        assert name in syms, name
+
+
+def test_struct_size_matches_header():
+    # the library rejects a struct whose size differs from its own
+    a = binding.GdnArgs()
+    a.struct_size = ctypes.sizeof(binding.GdnArgs) + 8
+    rc = g.load_library().gdn_fwd_ex(ctypes.byref(a))
+    assert rc == 1 and "struct_size" in g.last_error()
+    assert ctypes.sizeof(binding.GdnArgs) == 160  # LP64 layout of gdn_args
+
+
+def _call(fn="gdn_fwd", q=FAKE, k=FAKE + 1024, v=FAKE + 2048, alpha=FAKE + 4096, beta=FAKE + 8192,
+          S_in=None, S_out=None, o=FAKE + 16384, B=1, H=2, T=128, L=64, dk=64, dv=64):
+    lib = g.load_library()
+    return getattr(lib, fn)(q, k, v, alpha, beta, S_in, S_out, o, B, H, T, L, dk, dv, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=100, L=64), 2),                # T not a multiple of frame_len
+    (dict(L=0), 1),                        # frame_len must be positive
+    (dict(B=-1), 1),
+    (dict(dk=120), 3), (dict(dv=136), 3), (dict(dk=8), 3),
+    (dict(L=8192, T=8192), 3),             # frame_len above 4096
+    (dict(q=None), 1), (dict(o=None), 1), (dict(alpha=None), 1),
+    (dict(k=FAKE + 8), 4), (dict(S_in=FAKE + 3), 4),
+    (dict(B=1 << 20, H=1 << 10, T=1 << 30, L=1 << 10), 2),   # index overflow
+])
+def test_validation_errors(kw, status):
+    assert _call(**kw) == status
+    assert g.last_error() != ""
+
+
+def test_overlap_rejected():
+    # o aliasing q
+    assert _call(o=FAKE) == 1 and "overlaps" in g.last_error()
+
+
+def test_step_requires_state():
+    assert _call(fn="gdn_step") == 1
+    assert _call(fn="gdn_step_f32") == 1
+
+
+def test_status_strings():
+    lib = g.load_library()
+    for code, name in binding.STATUS.items():
+        assert lib.gdn_status_string(code).decode() == name
+    assert lib.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+
+
+def test_workspace_bytes():
+    assert g.workspace_bytes(1, 20, 106480, 880, 112, 112) > 0
+    assert g.workspace_bytes(1, 20, 100, 880, 112, 112) == 0      # invalid shape
+    assert g.workspace_bytes(0, 20, 880, 880, 112, 112) == 0      # empty
+    # grows with the batch
+    assert g.workspace_bytes(2, 4, 880, 880, 64, 64) > g.workspace_bytes(1, 4, 880, 880, 64, 64)
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 64, 1, 16)
+    with pytest.raises(g.GdnError):
+        g.gdn_fwd(x, x, x, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1), 64)
