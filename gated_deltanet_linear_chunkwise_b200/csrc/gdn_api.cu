@@ -257,6 +257,12 @@ gdn_args make_args(int dtype, const void *q, const void *k, const void *v, const
 
 }  // namespace
 
+namespace gdn {
+// Validation and error text shared with the other entry-point files.
+int validate_args(const gdn_args &a, Problem &p) { return validate(a, p); }
+void set_error_text(const char *msg) { set_err("%s", msg); }
+}  // namespace gdn
+
 extern "C" {
 
 int gdn_fwd(const void *q, const void *k, const void *v, const float *alpha, const float *beta,

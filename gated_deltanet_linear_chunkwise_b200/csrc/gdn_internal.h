@@ -80,6 +80,11 @@ inline cudaError_t mark(cudaEvent_t *ev, int i, cudaStream_t s) {
     return ev ? cudaEventRecord(ev[i], s) : cudaSuccess;
 }
 
+// Argument validation of the C ABI (gdn_api.cu): fills p or returns a gdn_status.
+int validate_args(const gdn_args &a, Problem &p);
+// Sets the thread-local text gdn_last_error() returns.
+void set_error_text(const char *msg);
+
 size_t simt_workspace_bytes(const Problem &p);
 cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
 

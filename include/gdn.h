@@ -111,6 +111,38 @@ int gdn_step_f32(const float *q, const float *k, const float *v,
                  gdn_stream_t stream);
 
 /*
+ * gdn_fwd_noalloc -- gdn_fwd for callers that cannot allocate device memory.
+ * (The SANA-WM pages have no counterpart: this is a deployment variant.)
+ *
+ * Some callers may not allocate on the path of a pass: a streaming decode
+ * loop whose latency budget cannot take an allocation (cudaMalloc can
+ * synchronise the device), a host whose own pool owns all device memory, or
+ * code running where allocating is not allowed.  This entry point computes
+ * exactly what gdn_fwd computes (bf16 q/k/v/o, fp32 gates and state; same
+ * arguments, layouts and errors) on the CUDA-core kernels, with its scratch
+ * in one fixed device array of GDN_NOALLOC_SCRATCH_BYTES that every GPU
+ * loading the library holds until the process exits.  It calls no
+ * allocator.  A problem whose scratch would exceed that size is rejected
+ * with GDN_ERR_UNSUPPORTED before anything is launched (at 880-token frames
+ * and d_k = d_v = 112 each frame-head needs about 1.33 MB, so up to 50
+ * frame-heads fit, e.g. one frame of B = 2, H = 20).
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it: make that first call before any
+ * stream capture.  All calls share the array and it keeps the last call's
+ * contents (no part needs to start at zero); calls whose executions overlap
+ * on the GPU (other streams, or unordered host threads) race on it, so
+ * issue them on one stream or order them with events.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+int gdn_fwd_noalloc(const void *q, const void *k, const void *v,
+                    const float *alpha, const float *beta,
+                    const float *S_in, float *S_out, void *o,
+                    int B, int H, long long T, int frame_len, int d_k, int d_v,
+                    gdn_stream_t stream);
+
+/*
  * Extended call.  Fields not listed for a flag are as in gdn_fwd.
  *   struct_size     sizeof(gdn_args) as compiled by the caller (ABI guard).
  *   dtype           GDN_DTYPE_BF16 or GDN_DTYPE_F32 (q/k/v/o element type).
