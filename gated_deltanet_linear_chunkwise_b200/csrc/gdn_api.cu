@@ -201,7 +201,14 @@ int run(const gdn_args &a) noexcept {
             }
             evp = ev;
         }
-        cudaError_t e = use_tc(p) ? gdn::launch_tc(p, ws, s, evp) : gdn::launch_simt(p, ws, s, evp);
+        const bool tc = use_tc(p);
+        cudaError_t e = tc ? gdn::launch_tc(p, ws, s, evp) : gdn::launch_simt(p, ws, s, evp);
+        // synchronous modes also report a device-side wait that gave up
+        int timed_out = 0;
+        if (e == cudaSuccess && tc && (a.stage_ms || a.check_finite)) {
+            e = cudaMemcpyAsync(&timed_out, gdn::tc_error_word(p, ws), sizeof(int), cudaMemcpyDeviceToHost, s);
+            if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        }
         if (owned) {
             cudaError_t e2 = cudaFreeAsync(ws, s);
             if (e == cudaSuccess) e = e2;
@@ -216,6 +223,10 @@ int run(const gdn_args &a) noexcept {
             for (int i = 0; i <= GDN_NUM_STAGES; ++i) cudaEventDestroy(ev[i]);
         }
         if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+        if (timed_out) {
+            set_err("a bounded device-side wait gave up (error word %d)", timed_out);
+            return GDN_ERR_TIMEOUT;
+        }
 
         if (a.check_finite) {
             int *flag = nullptr;

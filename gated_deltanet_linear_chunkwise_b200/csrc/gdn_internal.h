@@ -85,6 +85,13 @@ int validate_args(const gdn_args &a, Problem &p);
 // Sets the thread-local text gdn_last_error() returns.
 void set_error_text(const char *msg);
 
+// Scratch layout of the CUDA-core path (byte offsets into the workspace).
+struct SimtLayout {
+    size_t X, U, M, N, Sig, total;
+};
+__host__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+SimtLayout simt_layout(const Problem &p);
+
 size_t simt_workspace_bytes(const Problem &p);
 cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
 

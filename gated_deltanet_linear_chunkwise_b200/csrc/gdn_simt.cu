@@ -11,6 +11,7 @@
 //   k4  U = Ub - W Sig_f and O = diag(e^G) Q Sig_f + tril_incl(Q K^T o Gamma) U
 // Row blocks are 32 tokens; every thread owns one output column and keeps
 // the block's 32 (or 16) rows of that column in registers.
+#include "gates.cuh"
 #include "gdn_internal.h"
 
 namespace gdn {
@@ -31,50 +32,6 @@ template <typename T> __device__ __forceinline__ void st_out(T *p, long long i, 
 template <> __device__ __forceinline__ void st_out<float>(float *p, long long i, float x) { p[i] = x; }
 template <> __device__ __forceinline__ void st_out<__nv_bfloat16>(__nv_bfloat16 *p, long long i, float x) {
     p[i] = __float2bfloat16_rn(x);
-}
-
-template <typename TG> __device__ __forceinline__ TG log_gate(float a) {
-    TG lg = a > 0.f ? (TG)log((TG)a) : (TG)kLogAlphaFloor;
-    return lg < (TG)kLogAlphaFloor ? (TG)kLogAlphaFloor : lg;
-}
-
-// Inclusive prefix of log(alpha) over logical frame f of chain (b,h) into
-// sG[0..L), and the frame's beta into sB[0..L).  Block-wide scan: each
-// thread takes a contiguous run, warps scan their totals with shuffles.
-template <typename TG>
-__device__ void frame_gates(const Problem &p, int b, int h, long long f, TG *sG, float *sB, TG *sScr) {
-    const int L = p.L, tid = threadIdx.x, nt = blockDim.x;
-    const int per = (L + nt - 1) / nt;
-    const int i0 = tid * per, i1 = min(i0 + per, L);
-    TG run = 0;
-    for (int i = i0; i < i1; ++i) {
-        const long long row = tok_row(p, b, h, phys_token(p, f, i));
-        run += log_gate<TG>(p.alpha[row]);
-        sG[i] = run;
-        sB[i] = p.beta[row];
-    }
-    const int lane = tid & 31, warp = tid >> 5, nw = (nt + 31) >> 5;
-    TG x = run;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        TG y = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += y;
-    }
-    if (lane == 31) sScr[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        TG w = lane < nw ? sScr[lane] : (TG)0;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            TG y = __shfl_up_sync(0xffffffffu, w, off);
-            if (lane >= off) w += y;
-        }
-        if (lane < nw) sScr[lane] = w;
-    }
-    __syncthreads();
-    const TG offset = (x - run) + (warp > 0 ? sScr[warp - 1] : (TG)0);
-    for (int i = i0; i < i1; ++i) sG[i] += offset;
-    __syncthreads();
 }
 
 // Shared-memory carve-up shared by the kernels that scan a frame's gates.
@@ -488,25 +445,6 @@ __global__ void __launch_bounds__(NT) k4_output_simt(Problem p, const float *__r
     }
 }
 
-struct SimtLayout {
-    size_t X, U, M, N, Sig, total;
-};
-
-__host__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-SimtLayout simt_layout(const Problem &p) {
-    const size_t nfh = (size_t)p.B * p.H * p.F;
-    SimtLayout lay;
-    size_t off = 0;
-    lay.X = off;   off += align256(sizeof(float) * nfh * p.L * (p.dk + p.dv));
-    lay.U = off;   off += align256(sizeof(float) * nfh * p.L * p.dv);
-    lay.M = off;   off += align256(sizeof(float) * nfh * p.dk * p.dk);
-    lay.N = off;   off += align256(sizeof(float) * nfh * p.dk * p.dv);
-    lay.Sig = off; off += align256(sizeof(float) * nfh * p.dk * p.dv);
-    lay.total = off;
-    return lay;
-}
-
 template <typename TIn, typename TG>
 cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
     const SimtLayout lay = simt_layout(p);
@@ -543,6 +481,19 @@ cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t
 }
 
 }  // namespace
+
+SimtLayout simt_layout(const Problem &p) {
+    const size_t nfh = (size_t)p.B * p.H * p.F;
+    SimtLayout lay;
+    size_t off = 0;
+    lay.X = off;   off += align256(sizeof(float) * nfh * p.L * (p.dk + p.dv));
+    lay.U = off;   off += align256(sizeof(float) * nfh * p.L * p.dv);
+    lay.M = off;   off += align256(sizeof(float) * nfh * p.dk * p.dk);
+    lay.N = off;   off += align256(sizeof(float) * nfh * p.dk * p.dv);
+    lay.Sig = off; off += align256(sizeof(float) * nfh * p.dk * p.dv);
+    lay.total = off;
+    return lay;
+}
 
 size_t simt_workspace_bytes(const Problem &p) { return simt_layout(p).total; }
 

@@ -1,11 +1,162 @@
-// gdn_tc.cu -- tensor-core path (not yet enabled: every problem runs on the
-// CUDA-core kernels).
+// gdn_tc.cu -- the tensor-core path for bf16 inputs: workspace layout, TMA
+// tensor maps, the gate prologue and the stage sequence.
+//
+// Stage sequence (forward scans, bf16 q/k/v/o):
+//   gates    G = per-frame prefix of log alpha (fp32)
+//   intra, transition, scan  (CUDA-core kernels for now; fp32 workspace)
+//   convert  U and the entering states to bf16 operands
+//   output   tcgen05 kernel (tc_output.cu)
+#include <cstdlib>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "gates.cuh"
 #include "gdn_tc.h"
+#include "tc_common.cuh"
 
 namespace gdn {
+namespace {
 
-bool tc_supports(const Problem &) { return false; }
-size_t tc_workspace_bytes(const Problem &) { return 0; }
-cudaError_t launch_tc(const Problem &, void *, cudaStream_t, cudaEvent_t *) { return cudaErrorNotSupported; }
+struct TcLayout {
+    size_t simt, G, Ub, SigB, err, total;
+};
+
+TcLayout tc_layout(const Problem &p) {
+    const size_t nfh = (size_t)p.B * p.H * p.F;
+    TcLayout lay;
+    size_t off = 0;
+    lay.simt = off; off += align256(simt_workspace_bytes(p));
+    lay.G = off;    off += align256(sizeof(float) * nfh * p.L);
+    lay.Ub = off;   off += align256(2 * nfh * p.L * p.dv);
+    lay.SigB = off; off += align256(2 * nfh * p.dk * p.dv);
+    lay.err = off;  off += 256;
+    lay.total = off;
+    return lay;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first
+// (strides in bytes for dims 1..rank-1).
+bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+              const cuuint32_t *box) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// q/k [B,T,H,d] seen as 4-D (d, H, L, B*F): a frame-head's 128-token tile is
+// one box (64 columns, 1 head, 128 tokens, 1 frame); rows past the frame are
+// out of bounds and read as zeros.
+bool map_tokens(CUtensorMap *m, const void *x, const Problem &p, int d) {
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)p.H, (cuuint64_t)p.L, (cuuint64_t)(p.B * p.F)};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)p.H * d * 2, (cuuint64_t)p.L * p.H * d * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    return make_map(m, x, 4, dims, strides, box);
+}
+
+// Workspace [n_fh][rows][cols] bf16 seen as 3-D (cols, rows, n_fh).
+bool map_rows(CUtensorMap *m, const void *x, long long nfh, int rows, int cols, int box_rows) {
+    const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)nfh};
+    const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)rows * cols * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    return make_map(m, x, 3, dims, strides, box);
+}
+
+__global__ void __launch_bounds__(256) gate_prefix_kernel(Problem p, float *__restrict__ G) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const long long fh = blockIdx.x;
+    const long long f = fh % p.F, chain = fh / p.F;
+    const int h = (int)(chain % p.H), b = (int)(chain / p.H);
+    float *sG = (float *)smem;
+    float *sB = sG + p.L;
+    float *sScr = sB + p.L;
+    frame_gates<float>(p, b, h, f, sG, sB, sScr);
+    for (int i = threadIdx.x; i < p.L; i += blockDim.x) G[fh * p.L + i] = sG[i];
+}
+
+__global__ void f32_to_bf16_kernel(const float *__restrict__ in, __nv_bfloat16 *__restrict__ out, long long n) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        out[i] = __float2bfloat16_rn(in[i]);
+}
+
+bool tc_disabled_by_env() {
+    const char *e = getenv("GDN_DISABLE_TC");
+    return e && e[0] == '1';
+}
+
+}  // namespace
+
+bool tc_supports(const Problem &p) {
+    static const bool disabled = tc_disabled_by_env();
+    return !disabled && p.dtype == GDN_DTYPE_BF16 && !p.reverse && !p.accumulate;
+}
+
+size_t tc_workspace_bytes(const Problem &p) { return tc_layout(p).total; }
+
+cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
+    const TcLayout lay = tc_layout(p);
+    char *base = (char *)ws;
+    const long long nfh = (long long)p.B * p.H * p.F;
+    const int nblk = (p.L + tc::BM - 1) / tc::BM;
+    float *G = (float *)(base + lay.G);
+    __nv_bfloat16 *Ub = (__nv_bfloat16 *)(base + lay.Ub);
+    __nv_bfloat16 *SigB = (__nv_bfloat16 *)(base + lay.SigB);
+    int *err = (int *)(base + lay.err);
+    cudaError_t e;
+
+    CUtensorMap tm_q, tm_k, tm_u, tm_sig;
+    if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
+        !map_rows(&tm_u, Ub, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk))
+        return cudaErrorInvalidValue;
+
+    if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
+    // stages 0-2 (and a CUDA-core output, overwritten below) on the CUDA-core kernels
+    if ((e = launch_simt(p, base + lay.simt, s, ev))) return e;
+    const SimtLayout sl = simt_layout(p);
+    const float *U32 = (const float *)(base + lay.simt + sl.U);
+    const float *Sig32 = (const float *)(base + lay.simt + sl.Sig);
+
+    const size_t gsm = sizeof(float) * (2 * p.L + 32);
+    if (gsm > 48 * 1024 &&
+        (e = cudaFuncSetAttribute(gate_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm)))
+        return e;
+    gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G);
+    if ((e = cudaGetLastError())) return e;
+    f32_to_bf16_kernel<<<1184, 256, 0, s>>>(U32, Ub, nfh * p.L * p.dv);
+    if ((e = cudaGetLastError())) return e;
+    f32_to_bf16_kernel<<<1184, 256, 0, s>>>(Sig32, SigB, nfh * p.dk * p.dv);
+    if ((e = cudaGetLastError())) return e;
+    // poison o so that any row the tensor-core kernel fails to write shows up
+    if ((e = cudaMemsetAsync(p.o, 0xFF, (size_t)p.B * p.T * p.H * p.dv * 2, s))) return e;
+
+    tc::OutParams op;
+    op.G = G;
+    op.o = p.o;
+    op.L = p.L; op.dk = p.dk; op.dv = p.dv; op.H = p.H; op.nblk = nblk;
+    op.F = p.F; op.T = p.T;
+    op.accumulate = p.accumulate;
+    op.err = err;
+    if ((e = mark(ev, 3, s))) return e;  // the output stage is timed on the tensor-core kernel
+    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u, tm_sig, op, nfh, s))) return e;
+    return mark(ev, 4, s);
+}
+
+int *tc_error_word(const Problem &p, void *ws) { return (int *)((char *)ws + tc_layout(p).err); }
 
 }  // namespace gdn

@@ -9,5 +9,7 @@ namespace gdn {
 bool tc_supports(const Problem &p);
 size_t tc_workspace_bytes(const Problem &p);
 cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
+// Device word in the workspace where a bounded wait that gave up records it.
+int *tc_error_word(const Problem &p, void *ws);
 
 }  // namespace gdn

@@ -1,0 +1,53 @@
+// tc_common.cuh -- shared pieces of the tensor-core (tcgen05) kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "gdn_internal.h"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace tc {
+
+constexpr int BM = 128;          // token rows per tile (UMMA M)
+constexpr int SLAB = 64;         // bf16 columns per 128-byte swizzle slab
+constexpr int SLAB_BYTES = BM * 128;  // one 128-row slab
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Barrier among `nthreads` threads (a multiple of 32) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// K-major SW128 operand: tile of `rows` rows, 64-column slabs; K step ks (16 columns).
+__device__ __forceinline__ uint64_t desc_kmajor(const void *tile, int ks, int rows) {
+    const uint32_t a = sm100::smem_u32(tile) + (uint32_t)((ks >> 2) * rows * 128 + (ks & 3) * 32);
+    return sm100::smem_desc(a, 16, 1024, sm100::kSwizzle128B);
+}
+
+// MN-major SW128 operand: `krows` rows along K, 64-column slabs along MN
+// (slab stride krows*128 bytes); K step ks covers rows 16ks..16ks+15.
+__device__ __forceinline__ uint64_t desc_mnmajor(const void *tile, int ks, int krows) {
+    const uint32_t a = sm100::smem_u32(tile) + (uint32_t)(ks * 16 * 128);
+    return sm100::smem_desc(a, (uint32_t)krows * 128, 1024, sm100::kSwizzle128B);
+}
+
+struct OutParams {
+    const float *G;          // [n_fh][L] inclusive prefix of clamped log alpha per frame
+    void *o;                 // [B,T,H,dv] bf16
+    int L, dk, dv, H, nblk;
+    long long F, T;
+    int accumulate;
+    int *err;
+};
+
+cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
+                             const CUtensorMap &tm_sig, const OutParams &prm, long long n_fh, cudaStream_t s);
+
+}  // namespace tc
+}  // namespace gdn
