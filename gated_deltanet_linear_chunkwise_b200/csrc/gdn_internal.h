@@ -93,6 +93,15 @@ __host__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 SimtLayout simt_layout(const Problem &p);
 
 size_t simt_workspace_bytes(const Problem &p);
+
+// Single CUDA-core stages over bf16 [Ub | W] rows, used as interim stages of
+// the tensor-core path (bf16 inputs).
+cudaError_t simt_intra_bf16x(const Problem &p, __nv_bfloat16 *X, cudaStream_t s);
+cudaError_t simt_transition_bf16x(const Problem &p, const __nv_bfloat16 *X, float *Mb, float *Nb, cudaStream_t s);
+cudaError_t simt_scan(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
+                      cudaStream_t s);
+cudaError_t simt_u_bf16x(const Problem &p, const __nv_bfloat16 *X, const float *Sig, __nv_bfloat16 *U,
+                         cudaStream_t s);
 cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
 
 }  // namespace gdn

@@ -42,8 +42,8 @@ template <typename TG> struct GateSmem {
 };
 
 // ---------------------------------------------------------------- k1 intra-frame
-template <typename TIn, typename TG>
-__global__ void __launch_bounds__(NT) k1_intra_simt(Problem p, float *__restrict__ X) {
+template <typename TIn, typename TG, typename TX>
+__global__ void __launch_bounds__(NT) k1_intra_simt(Problem p, TX *__restrict__ X) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int L = p.L, dk = p.dk, dv = p.dv, nc = dk + dv;
     const long long fh = blockIdx.x;
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(NT) k1_intra_simt(Problem p, float *__restrict
 
     frame_gates<TG>(p, b, h, f, sG, sB, sScr);
     const TIn *k = (const TIn *)p.k, *v = (const TIn *)p.v;
-    float *Xf = X + fh * (long long)L * nc;
+    TX *Xf = X + fh * (long long)L * nc;
     const int tid = threadIdx.x;
     const int nblk = (L + RB - 1) / RB;
 
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(NT) k1_intra_simt(Problem p, float *__restrict
                     const int s = e / dk, c = e - s * dk;
                     sKjT[c * RB + s] = ld_in(k, tok_row(p, b, h, phys_token(p, f, s0 + s)) * dk + c);
                 }
-                for (int e = tid; e < RB * nc; e += NT) sX[e] = Xf[(long long)s0 * nc + e];
+                for (int e = tid; e < RB * nc; e += NT) sX[e] = ld_in(Xf, (long long)s0 * nc + e);
             }
             __syncthreads();
             const float *KjT = diag ? sKiT : sKjT;
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(NT) k1_intra_simt(Problem p, float *__restrict
         if (tid < nc) {
 #pragma unroll
             for (int r = 0; r < RB; ++r)
-                if (r < nr) Xf[(long long)(r0 + r) * nc + tid] = acc[r];
+                if (r < nr) st_out(Xf, (long long)(r0 + r) * nc + tid, acc[r]);
         }
         __syncthreads();
     }
@@ -155,8 +155,8 @@ __global__ void __launch_bounds__(NT) k1_intra_simt(Problem p, float *__restrict
 
 // ---------------------------------------------------------------- k2 frame transition
 // grid (frame-heads, ceil(dk/32)); the block owns rows m0..m0+31 of [N | M].
-template <typename TIn, typename TG>
-__global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const float *__restrict__ X,
+template <typename TIn, typename TG, typename TX>
+__global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const TX *__restrict__ X,
                                                          float *__restrict__ Mb, float *__restrict__ Nb) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int L = p.L, dk = p.dk, dv = p.dv, nc = dk + dv;
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const float 
 
     frame_gates<TG>(p, b, h, f, sG, sB, sScr);
     const TIn *k = (const TIn *)p.k;
-    const float *Xf = X + fh * (long long)L * nc;
+    const TX *Xf = X + fh * (long long)L * nc;
     const int tid = threadIdx.x;
     const TG GL = sG[L - 1];
 
@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const float 
         }
         for (int e = tid; e < RB * nc; e += NT) {
             const int s = e / nc;
-            sX[e] = (s < ns) ? Xf[(long long)s0 * nc + e] : 0.f;
+            sX[e] = (s < ns) ? ld_in(Xf, (long long)s0 * nc + e) : 0.f;
         }
         __syncthreads();
         if (tid < nc) {
@@ -232,7 +232,8 @@ __global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const float 
 // grid (B*H, ceil(dv/16)); the block carries 16 columns of Sig = S^T through
 // all frames of its chain, writing the state entering each frame to Sig_in.
 __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__restrict__ Mb,
-                                                   const float *__restrict__ Nb, float *__restrict__ SigIn) {
+                                                   const float *__restrict__ Nb, float *__restrict__ SigIn,
+                                                   __nv_bfloat16 *__restrict__ SigB) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int dk = p.dk, dv = p.dv;
     const long long chain = blockIdx.x;
@@ -257,7 +258,11 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
         __syncthreads();
         for (int e = tid; e < dk * SCAN_COLS; e += NT) {
             const int m = e >> 4, cc = e & 15;
-            if (cc < ncol) SigIn[(fh * dk + m) * (long long)dv + c0 + cc] = sS[e];
+            if (cc < ncol) {
+                const long long idx = (fh * dk + m) * (long long)dv + c0 + cc;
+                if (SigIn) SigIn[idx] = sS[e];
+                if (SigB) SigB[idx] = __float2bfloat16_rn(sS[e]);
+            }
         }
         const float *Mf = Mb + fh * (long long)dk * dk;
         for (int e = tid; e < dk * dk; e += NT) {
@@ -445,6 +450,62 @@ __global__ void __launch_bounds__(NT) k4_output_simt(Problem p, const float *__r
     }
 }
 
+
+// ---------------------------------------------------------------- U = Ub - W Sig
+// grid (frame-heads, ceil(L/128)); 128 rows per block in four 32-row passes.
+// Reads [Ub | W] (TX) and the entering state Sig (fp32), writes U in bf16.
+template <typename TX>
+__global__ void __launch_bounds__(NT) ku_simt(Problem p, const TX *__restrict__ X, const float *__restrict__ SigIn,
+                                              __nv_bfloat16 *__restrict__ U) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int L = p.L, dk = p.dk, dv = p.dv, nc = dk + dv;
+    const long long fh = blockIdx.x;
+    float *sSig = (float *)smem;          // [dk][dv]
+    float *sWT = sSig + dk * dv;          // [dk][32]
+    const TX *Xf = X + fh * (long long)L * nc;
+    const float *Sf = SigIn + fh * (long long)dk * dv;
+    __nv_bfloat16 *Uf = U + fh * (long long)L * dv;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < dk * dv; e += NT) sSig[e] = Sf[e];
+    const int c = tid & 127, rh = tid >> 7;
+    const bool active = c < dv;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int r0 = blockIdx.y * 128 + pass * RB;
+        if (r0 >= L) break;
+        const int nr = min(RB, L - r0);
+        __syncthreads();
+        for (int e = tid; e < RB * dk; e += NT) {
+            const int r = e / dk, cc = e - r * dk;
+            sWT[cc * RB + r] = (r < nr) ? ld_in(Xf, (long long)(r0 + r) * nc + dv + cc) : 0.f;
+        }
+        __syncthreads();
+        if (active) {
+            float acc[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int rr = rh * 16 + r;
+                acc[r] = (rr < nr) ? ld_in(Xf, (long long)(r0 + rr) * nc + c) : 0.f;
+            }
+            for (int l = 0; l < dk; ++l) {
+                const float sg = sSig[l * dv + c];
+#pragma unroll
+                for (int r4 = 0; r4 < 4; ++r4) {
+                    const float4 w = *reinterpret_cast<const float4 *>(&sWT[l * RB + rh * 16 + r4 * 4]);
+                    acc[r4 * 4 + 0] -= w.x * sg;
+                    acc[r4 * 4 + 1] -= w.y * sg;
+                    acc[r4 * 4 + 2] -= w.z * sg;
+                    acc[r4 * 4 + 3] -= w.w * sg;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int rr = rh * 16 + r;
+                if (rr < nr) Uf[(long long)(r0 + rr) * dv + c] = __float2bfloat16_rn(acc[r]);
+            }
+        }
+    }
+}
+
 template <typename TIn, typename TG>
 cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
     const SimtLayout lay = simt_layout(p);
@@ -460,19 +521,20 @@ cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t
     const size_t sm3 = sizeof(float) * (dk * (dk + 1) + dk * SCAN_COLS);
     const size_t sm4 = gsm + sizeof(float) * (dk * dv + 3 * dk * RB + RB * RB + RB * dv);
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(k1_intra_simt<TIn, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1))) return e;
-    if ((e = cudaFuncSetAttribute(k2_transition_simt<TIn, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2))) return e;
+    if ((e = cudaFuncSetAttribute(k1_intra_simt<TIn, TG, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1))) return e;
+    if ((e = cudaFuncSetAttribute(k2_transition_simt<TIn, TG, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2))) return e;
     if ((e = cudaFuncSetAttribute(k3_scan_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3))) return e;
     if ((e = cudaFuncSetAttribute(k4_output_simt<TIn, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm4))) return e;
 
     if ((e = mark(ev, 0, s))) return e;
-    k1_intra_simt<TIn, TG><<<(unsigned)nfh, NT, sm1, s>>>(p, X);
+    k1_intra_simt<TIn, TG, float><<<(unsigned)nfh, NT, sm1, s>>>(p, X);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 1, s))) return e;
-    k2_transition_simt<TIn, TG><<<dim3((unsigned)nfh, (dk + 31) / 32), NT, sm2, s>>>(p, X, Mb, Nb);
+    k2_transition_simt<TIn, TG, float><<<dim3((unsigned)nfh, (dk + 31) / 32), NT, sm2, s>>>(p, X, Mb, Nb);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 2, s))) return e;
-    k3_scan_simt<<<dim3((unsigned)(p.B * p.H), (dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm3, s>>>(p, Mb, Nb, Sig);
+    k3_scan_simt<<<dim3((unsigned)(p.B * p.H), (dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm3, s>>>(p, Mb, Nb, Sig,
+                                                                                             nullptr);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 3, s))) return e;
     k4_output_simt<TIn, TG><<<(unsigned)nfh, NT, sm4, s>>>(p, X, Sig, U);
@@ -500,6 +562,46 @@ size_t simt_workspace_bytes(const Problem &p) { return simt_layout(p).total; }
 cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
     if (p.dtype == GDN_DTYPE_F32) return launch_typed<float, double>(p, ws, s, ev);
     return launch_typed<__nv_bfloat16, float>(p, ws, s, ev);
+}
+
+cudaError_t simt_intra_bf16x(const Problem &p, __nv_bfloat16 *X, cudaStream_t s) {
+    const int dk = p.dk, nc = p.dk + p.dv;
+    const size_t sm = GateSmem<float>::bytes(p.L) + sizeof(float) * (2 * dk * RB + RB * RB + RB * nc);
+    auto k = k1_intra_simt<__nv_bfloat16, float, __nv_bfloat16>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e) return e;
+    k<<<(unsigned)((long long)p.B * p.H * p.F), NT, sm, s>>>(p, X);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_transition_bf16x(const Problem &p, const __nv_bfloat16 *X, float *Mb, float *Nb, cudaStream_t s) {
+    const int nc = p.dk + p.dv;
+    const size_t sm = GateSmem<float>::bytes(p.L) + sizeof(float) * (RB * 32 + RB * nc);
+    auto k = k2_transition_simt<__nv_bfloat16, float, __nv_bfloat16>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e) return e;
+    k<<<dim3((unsigned)((long long)p.B * p.H * p.F), (p.dk + 31) / 32), NT, sm, s>>>(p, X, Mb, Nb);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_scan(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
+                      cudaStream_t s) {
+    const size_t sm = sizeof(float) * (p.dk * (p.dk + 1) + p.dk * SCAN_COLS);
+    cudaError_t e = cudaFuncSetAttribute(k3_scan_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e) return e;
+    k3_scan_simt<<<dim3((unsigned)(p.B * p.H), (p.dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm, s>>>(p, Mb, Nb, Sig,
+                                                                                                 SigB);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_u_bf16x(const Problem &p, const __nv_bfloat16 *X, const float *Sig, __nv_bfloat16 *U,
+                         cudaStream_t s) {
+    const size_t sm = sizeof(float) * (p.dk * p.dv + p.dk * RB);
+    auto k = ku_simt<__nv_bfloat16>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e) return e;
+    k<<<dim3((unsigned)((long long)p.B * p.H * p.F), (p.L + 127) / 128), NT, sm, s>>>(p, X, Sig, U);
+    return cudaGetLastError();
 }
 
 }  // namespace gdn

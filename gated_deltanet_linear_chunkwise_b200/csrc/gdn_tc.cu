@@ -2,10 +2,11 @@
 // tensor maps, the gate prologue and the stage sequence.
 //
 // Stage sequence (forward scans, bf16 q/k/v/o):
-//   gates    G = per-frame prefix of log alpha (fp32)
-//   intra, transition, scan  (CUDA-core kernels for now; fp32 workspace)
-//   convert  U and the entering states to bf16 operands
-//   output   tcgen05 kernel (tc_output.cu)
+//   gates       G = per-frame prefix of log alpha (fp32)
+//   intra       [Ub | W] per frame-head, bf16            (CUDA cores for now)
+//   transition  M, N per frame-head, fp32                 (CUDA cores for now)
+//   scan        entering state per frame, fp32 + bf16     (CUDA cores)
+//   output      U = Ub - W Sig (bf16), then the tcgen05 output kernel
 #include <cstdlib>
 #include <mutex>
 
@@ -19,17 +20,21 @@ namespace gdn {
 namespace {
 
 struct TcLayout {
-    size_t simt, G, Ub, SigB, err, total;
+    size_t G, X, M, N, Sig, SigB, U, err, total;
 };
 
 TcLayout tc_layout(const Problem &p) {
     const size_t nfh = (size_t)p.B * p.H * p.F;
+    const size_t nc = (size_t)p.dk + p.dv;
     TcLayout lay;
     size_t off = 0;
-    lay.simt = off; off += align256(simt_workspace_bytes(p));
     lay.G = off;    off += align256(sizeof(float) * nfh * p.L);
-    lay.Ub = off;   off += align256(2 * nfh * p.L * p.dv);
+    lay.X = off;    off += align256(2 * nfh * p.L * nc);
+    lay.M = off;    off += align256(sizeof(float) * nfh * p.dk * p.dk);
+    lay.N = off;    off += align256(sizeof(float) * nfh * p.dk * p.dv);
+    lay.Sig = off;  off += align256(sizeof(float) * nfh * p.dk * p.dv);
     lay.SigB = off; off += align256(2 * nfh * p.dk * p.dv);
+    lay.U = off;    off += align256(2 * nfh * p.L * p.dv);
     lay.err = off;  off += 256;
     lay.total = off;
     return lay;
@@ -90,11 +95,6 @@ __global__ void __launch_bounds__(256) gate_prefix_kernel(Problem p, float *__re
     for (int i = threadIdx.x; i < p.L; i += blockDim.x) G[fh * p.L + i] = sG[i];
 }
 
-__global__ void f32_to_bf16_kernel(const float *__restrict__ in, __nv_bfloat16 *__restrict__ out, long long n) {
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
-        out[i] = __float2bfloat16_rn(in[i]);
-}
-
 bool tc_disabled_by_env() {
     const char *e = getenv("GDN_DISABLE_TC");
     return e && e[0] == '1';
@@ -115,35 +115,33 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     const long long nfh = (long long)p.B * p.H * p.F;
     const int nblk = (p.L + tc::BM - 1) / tc::BM;
     float *G = (float *)(base + lay.G);
-    __nv_bfloat16 *Ub = (__nv_bfloat16 *)(base + lay.Ub);
+    __nv_bfloat16 *X = (__nv_bfloat16 *)(base + lay.X);
+    float *Mb = (float *)(base + lay.M), *Nb = (float *)(base + lay.N), *Sig = (float *)(base + lay.Sig);
     __nv_bfloat16 *SigB = (__nv_bfloat16 *)(base + lay.SigB);
+    __nv_bfloat16 *U = (__nv_bfloat16 *)(base + lay.U);
     int *err = (int *)(base + lay.err);
     cudaError_t e;
 
     CUtensorMap tm_q, tm_k, tm_u, tm_sig;
     if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
-        !map_rows(&tm_u, Ub, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk))
+        !map_rows(&tm_u, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk))
         return cudaErrorInvalidValue;
 
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
-    // stages 0-2 (and a CUDA-core output, overwritten below) on the CUDA-core kernels
-    if ((e = launch_simt(p, base + lay.simt, s, ev))) return e;
-    const SimtLayout sl = simt_layout(p);
-    const float *U32 = (const float *)(base + lay.simt + sl.U);
-    const float *Sig32 = (const float *)(base + lay.simt + sl.Sig);
-
     const size_t gsm = sizeof(float) * (2 * p.L + 32);
     if (gsm > 48 * 1024 &&
         (e = cudaFuncSetAttribute(gate_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm)))
         return e;
+    if ((e = mark(ev, 0, s))) return e;
     gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G);
     if ((e = cudaGetLastError())) return e;
-    f32_to_bf16_kernel<<<1184, 256, 0, s>>>(U32, Ub, nfh * p.L * p.dv);
-    if ((e = cudaGetLastError())) return e;
-    f32_to_bf16_kernel<<<1184, 256, 0, s>>>(Sig32, SigB, nfh * p.dk * p.dv);
-    if ((e = cudaGetLastError())) return e;
-    // poison o so that any row the tensor-core kernel fails to write shows up
-    if ((e = cudaMemsetAsync(p.o, 0xFF, (size_t)p.B * p.T * p.H * p.dv * 2, s))) return e;
+    if ((e = simt_intra_bf16x(p, X, s))) return e;
+    if ((e = mark(ev, 1, s))) return e;
+    if ((e = simt_transition_bf16x(p, X, Mb, Nb, s))) return e;
+    if ((e = mark(ev, 2, s))) return e;
+    if ((e = simt_scan(p, Mb, Nb, Sig, SigB, s))) return e;
+    if ((e = mark(ev, 3, s))) return e;
+    if ((e = simt_u_bf16x(p, X, Sig, U, s))) return e;
 
     tc::OutParams op;
     op.G = G;
@@ -152,7 +150,6 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     op.F = p.F; op.T = p.T;
     op.accumulate = p.accumulate;
     op.err = err;
-    if ((e = mark(ev, 3, s))) return e;  // the output stage is timed on the tensor-core kernel
     if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u, tm_sig, op, nfh, s))) return e;
     return mark(ev, 4, s);
 }
