@@ -3,7 +3,8 @@
 //
 // Stage sequence (forward scans, bf16 q/k/v/o):
 //   gates       G = per-frame prefix of log alpha (fp32)
-//   intra       [Ub | W] per frame-head, bf16            (CUDA cores for now)
+//   inverse     T_ii = (I + A_ii)^{-1} per 128-row diagonal block (mma.sync)
+//   intra       [Ub | W] per frame-head, bf16, blocked forward substitution (tcgen05)
 //   transition  M, N per frame-head, fp32                 (CUDA cores for now)
 //   scan        entering state per frame, fp32 + bf16     (CUDA cores)
 //   output      U = Ub - W Sig (bf16), then the tcgen05 output kernel
@@ -20,7 +21,7 @@ namespace gdn {
 namespace {
 
 struct TcLayout {
-    size_t G, X, M, N, Sig, SigB, U, err, total;
+    size_t G, Tinv, X, M, N, Sig, SigB, U, err, total;
 };
 
 TcLayout tc_layout(const Problem &p) {
@@ -29,6 +30,7 @@ TcLayout tc_layout(const Problem &p) {
     TcLayout lay;
     size_t off = 0;
     lay.G = off;    off += align256(sizeof(float) * nfh * p.L);
+    lay.Tinv = off; off += align256(2 * nfh * (size_t)((p.L + 127) / 128) * 128 * 128);
     lay.X = off;    off += align256(2 * nfh * p.L * nc);
     lay.M = off;    off += align256(sizeof(float) * nfh * p.dk * p.dk);
     lay.N = off;    off += align256(sizeof(float) * nfh * p.dk * p.dv);
@@ -68,10 +70,10 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims
 // q/k [B,T,H,d] seen as 4-D (d, H, L, B*F): a frame-head's 128-token tile is
 // one box (64 columns, 1 head, 128 tokens, 1 frame); rows past the frame are
 // out of bounds and read as zeros.
-bool map_tokens(CUtensorMap *m, const void *x, const Problem &p, int d) {
+bool map_tokens(CUtensorMap *m, const void *x, const Problem &p, int d, int box_rows = 128) {
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)p.H, (cuuint64_t)p.L, (cuuint64_t)(p.B * p.F)};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)p.H * d * 2, (cuuint64_t)p.L * p.H * d * 2};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     return make_map(m, x, 4, dims, strides, box);
 }
 
@@ -122,9 +124,13 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     int *err = (int *)(base + lay.err);
     cudaError_t e;
 
-    CUtensorMap tm_q, tm_k, tm_u, tm_sig;
+    __nv_bfloat16 *Tinv = (__nv_bfloat16 *)(base + lay.Tinv);
+    const int nc = p.dk + p.dv;
+    CUtensorMap tm_q, tm_k, tm_u, tm_sig, tm_k64, tm_x, tm_t;
     if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
-        !map_rows(&tm_u, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk))
+        !map_rows(&tm_u, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
+        !map_tokens(&tm_k64, p.k, p, p.dk, 64) || !map_rows(&tm_x, X, nfh, p.L, nc, 64) ||
+        !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128))
         return cudaErrorInvalidValue;
 
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
@@ -135,7 +141,14 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     if ((e = mark(ev, 0, s))) return e;
     gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G);
     if ((e = cudaGetLastError())) return e;
-    if ((e = simt_intra_bf16x(p, X, s))) return e;
+    if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
+                                     nfh, s)))
+        return e;
+    tc::IntraParams ip;
+    ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.X = X;
+    ip.L = p.L; ip.dk = p.dk; ip.dv = p.dv; ip.H = p.H; ip.nblk = nblk;
+    ip.F = p.F; ip.T = p.T; ip.err = err;
+    if ((e = tc::launch_intra_tc(tm_k64, tm_x, tm_t, ip, nfh, s))) return e;
     if ((e = mark(ev, 1, s))) return e;
     if ((e = simt_transition_bf16x(p, X, Mb, Nb, s))) return e;
     if ((e = mark(ev, 2, s))) return e;

@@ -46,6 +46,23 @@ struct OutParams {
     int *err;
 };
 
+struct IntraParams {
+    const float *G;            // [n_fh][L]
+    const float *beta;         // [B,T,H]
+    const __nv_bfloat16 *v;    // [B,T,H,dv]
+    __nv_bfloat16 *X;          // [n_fh][L][dk + dv]: Ub (first dv columns) then W
+    int L, dk, dv, H, nblk;
+    long long F, T;
+    int *err;
+};
+
+cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_t,
+                            const IntraParams &prm, long long n_fh, cudaStream_t s);
+
+cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
+                                int L, int dk, int H, int nblk, long long F, long long T, long long n_fh,
+                                cudaStream_t s);
+
 cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
                              const CUtensorMap &tm_sig, const OutParams &prm, long long n_fh, cudaStream_t s);
 

@@ -1,0 +1,354 @@
+// tc_intra.cu -- intra-frame blocked forward substitution on the tensor cores.
+//
+// Solves, per frame-head, the unit lower triangular system of the chunkwise
+// gated delta rule (one chunk per frame; SANA-WM summary,
+// "Memory-Efficient Long-Context Modeling (Section 3.2)", frame-wise GDN):
+//   (I + A) X = R,   X = [Ub | W],   R = [beta V | beta e^G K],
+//   A_rs = beta_r e^{G_r - G_s} k_r.k_s  (s < r)
+// over 128-row blocks i, in order:
+//   acc_i = sum_{64-token tiles j before block i} P_ij X_j,  P_ij = -A_ij
+//   Y_i   = R_i + acc_i
+//   X_i   = T_ii Y_i,   T_ii = (I + A_ii)^{-1}  (from tc_diag_inverse.cu)
+// X_i goes to the [n_fh][L][d_v + d_k] bf16 workspace, from where later
+// blocks load it again (L2-resident) by TMA.
+//
+// Warp roles (192 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
+// warps 2-5 epilogue (one block row per thread).
+//   TMEM: S tiles 2 x 64 cols, acc / X_i d_v + d_k cols.
+//   SMEM: K_i, K_j x2, X_j x2 (Y_i aliases them), P x2, T_ii.
+// Decay factors use a per-tile anchor a = G at the tile's last token:
+// e^{G_r - G_s} = e^{G_r - a} e^{a - G_s}, both <= 1.
+#include "tc_common.cuh"
+
+namespace gdn {
+namespace tc {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int JT = 64;                       // tokens per off-diagonal tile
+constexpr int KJ_SLAB = JT * 128;            // 64-row slab
+constexpr int XJ_BYTES = 4 * KJ_SLAB;        // X_j tile: 4 slabs of 64 columns
+
+struct Smem {
+    static constexpr uint32_t KI = 0;                          // 2 slabs x 128 rows
+    static constexpr uint32_t KJ = KI + 2 * SLAB_BYTES;        // 2 stages x 2 slabs x 64 rows
+    static constexpr uint32_t XJ = KJ + 4 * KJ_SLAB;           // 2 stages x 32 KB; Y_i (64 KB) aliases
+    static constexpr uint32_t P = XJ + 2 * XJ_BYTES;           // 2 stages x 1 slab x 128 rows
+    static constexpr uint32_t T = P + 2 * SLAB_BYTES;          // 2 slabs x 128 rows
+    static constexpr uint32_t F = T + 2 * SLAB_BYTES;          // floats: G[L], cf[L]
+};
+
+enum Bar { KIFULL, KIEMPTY, TFULL, TEMPTY, KXFULL0, KXFULL1, KXEMPTY0, KXEMPTY1, SFULL0, SFULL1, SEMPTY0,
+           SEMPTY1, PFULL0, PFULL1, PEMPTY0, PEMPTY1, ACCFULL, YFULL, XFULL, XDONE, NBAR };
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_x,
+           const __grid_constant__ CUtensorMap tm_t, const IntraParams prm) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
+    const long long fh = blockIdx.x;
+    const long long F = prm.F;
+    const long long f = fh % F, chain = fh / F;
+    const int h = (int)(chain % prm.H), b = (int)(chain / prm.H);
+    const int bf = (int)(b * F + f);
+
+    unsigned char *sKi = smem + Smem::KI;
+    unsigned char *sKj = smem + Smem::KJ;
+    unsigned char *sXj = smem + Smem::XJ;
+    unsigned char *sY = sXj;
+    unsigned char *sP = smem + Smem::P;
+    unsigned char *sT = smem + Smem::T;
+    float *sG = (float *)(smem + Smem::F);
+    float *sCf = sG + L;
+    uint64_t *bars = (uint64_t *)(((uintptr_t)(sCf + L) + 7) & ~(uintptr_t)7);
+    uint32_t *tmem_slot = (uint32_t *)(bars + NBAR);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int *err = prm.err;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NBAR; ++i) {
+            uint32_t cnt = 1;
+            if (i == KIEMPTY || i == SEMPTY0 || i == SEMPTY1 || i == PFULL0 || i == PFULL1 || i == YFULL ||
+                i == XDONE)
+                cnt = 128;
+            sm100::mbar_init(&bars[i], cnt);
+        }
+        sm100::fence_barrier_init();
+    }
+    if (warp == 1) {
+        sm100::tmem_alloc(tmem_slot, 512);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t t_s0 = tbase, t_acc = tbase + 256;
+    const int nks_d = dk / 16;
+    const int nslab_k = (dk + SLAB - 1) / SLAB;
+    const int nslab_x = (nc + SLAB - 1) / SLAB;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            sm100::tma_prefetch_desc(&tm_k);
+            sm100::tma_prefetch_desc(&tm_x);
+            sm100::tma_prefetch_desc(&tm_t);
+            bool ok = true;
+            int n = 0;
+            for (int i = 0; i < nblk && ok; ++i) {
+                if (i >= 1) ok = sm100::mbar_wait(&bars[KIEMPTY], (i - 1) & 1, err) &&
+                                 sm100::mbar_wait(&bars[TEMPTY], (i - 1) & 1, err);
+                if (!ok) break;
+                sm100::mbar_arrive_expect_tx(&bars[KIFULL], (uint32_t)(nslab_k * SLAB_BYTES));
+                for (int sl = 0; sl < nslab_k; ++sl)
+                    for (int half = 0; half < 2; ++half)
+                        sm100::tma_load_4d(sKi + sl * SLAB_BYTES + half * KJ_SLAB, &tm_k, &bars[KIFULL], sl * SLAB,
+                                           h, i * BM + half * JT, bf);
+                sm100::mbar_arrive_expect_tx(&bars[TFULL], (uint32_t)(2 * SLAB_BYTES));
+                for (int sl = 0; sl < 2; ++sl)
+                    sm100::tma_load_3d(sT + sl * SLAB_BYTES, &tm_t, &bars[TFULL], sl * SLAB, 0,
+                                       (int)(fh * nblk + i));
+                for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
+                    const int st = n & 1;
+                    if (n >= 2) ok = sm100::mbar_wait(&bars[KXEMPTY0 + st], ((n - 2) >> 1) & 1, err);
+                    if (ok && jt == 2 * (i - 1)) ok = sm100::mbar_wait(&bars[XDONE], (i - 1) & 1, err);
+                    if (!ok) break;
+                    sm100::mbar_arrive_expect_tx(&bars[KXFULL0 + st],
+                                                 (uint32_t)(nslab_k * KJ_SLAB + nslab_x * KJ_SLAB));
+                    for (int sl = 0; sl < nslab_k; ++sl)
+                        sm100::tma_load_4d(sKj + (st * 2 + sl) * KJ_SLAB, &tm_k, &bars[KXFULL0 + st], sl * SLAB, h,
+                                           jt * JT, bf);
+                    for (int sl = 0; sl < nslab_x; ++sl)
+                        sm100::tma_load_3d(sXj + st * XJ_BYTES + sl * KJ_SLAB, &tm_x, &bars[KXFULL0 + st],
+                                           sl * SLAB, jt * JT, (int)fh);
+                }
+            }
+            // leave with no copy in flight
+            if (ok) ok = sm100::mbar_wait(&bars[TEMPTY], (nblk - 1) & 1, err);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = sm100::idesc_bf16(BM, JT, 0, 0);
+            const uint32_t id_x = sm100::idesc_bf16(BM, nc, 0, 1);
+            bool ok = true;
+            int n = 0;
+            auto issue_px = [&](int m, bool first_of_block, int i) -> bool {
+                const int pb = m & 1;
+                if (!sm100::mbar_wait(&bars[PFULL0 + pb], (m >> 1) & 1, err)) return false;
+                if (first_of_block && i >= 1 && !sm100::mbar_wait(&bars[XDONE], (i - 1) & 1, err)) return false;
+                sm100::tc_fence_after();
+                const unsigned char *xt = sXj + (m & 1) * XJ_BYTES;
+                const unsigned char *pt = sP + pb * SLAB_BYTES;
+                for (int ks = 0; ks < JT / 16; ++ks)
+                    sm100::mma_bf16_ss(t_acc, desc_kmajor(pt, ks, BM), desc_mnmajor(xt, ks, JT), id_x,
+                                       (first_of_block && ks == 0) ? 0u : 1u);
+                sm100::mma_commit(&bars[PEMPTY0 + pb]);
+                sm100::mma_commit(&bars[KXEMPTY0 + (m & 1)]);
+                return true;
+            };
+            for (int i = 0; i < nblk && ok; ++i) {
+                ok = sm100::mbar_wait(&bars[KIFULL], i & 1, err);
+                const int first = n;
+                for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
+                    const int st = n & 1;
+                    ok = sm100::mbar_wait(&bars[KXFULL0 + st], (n >> 1) & 1, err);
+                    if (ok && n >= 2) ok = sm100::mbar_wait(&bars[SEMPTY0 + st], ((n - 2) >> 1) & 1, err);
+                    if (!ok) break;
+                    sm100::tc_fence_after();
+                    const unsigned char *kt = sKj + st * 2 * KJ_SLAB;
+                    for (int ks = 0; ks < nks_d; ++ks)
+                        sm100::mma_bf16_ss(t_s0 + st * JT, desc_kmajor(sKi, ks, BM), desc_kmajor(kt, ks, JT), id_s,
+                                           ks > 0);
+                    sm100::mma_commit(&bars[SFULL0 + st]);
+                    if (jt >= 1) ok = issue_px(n - 1, n - 1 == first, i);
+                }
+                if (ok && i >= 1) ok = issue_px(n - 1, n - 1 == first, i);
+                if (!ok) break;
+                sm100::mma_commit(&bars[ACCFULL]);
+                ok = sm100::mbar_wait(&bars[YFULL], i & 1, err) && sm100::mbar_wait(&bars[TFULL], i & 1, err);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                for (int ks = 0; ks < BM / 16; ++ks)
+                    sm100::mma_bf16_ss(t_acc, desc_kmajor(sT, ks, BM), desc_mnmajor(sY, ks, BM), id_x, ks > 0);
+                sm100::mma_commit(&bars[XFULL]);
+                sm100::mma_commit(&bars[TEMPTY]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - 64;
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const float *Gf = prm.G + fh * (long long)L;
+        for (int s = et; s < L; s += 128) {
+            const int tile_end = min((s / JT) * JT + JT - 1, L - 1);
+            const float g = Gf[s];
+            sG[s] = g;
+            sCf[s] = __expf(Gf[tile_end] - g);  // <= 1: the tile's end is its most decayed token
+        }
+        named_sync(1, 128);  // the only epilogue-wide barrier: before any bounded wait
+
+        bool ok = true;
+        int n = 0;
+        for (int i = 0; i < nblk && ok; ++i) {
+            const int row = i * BM + r;
+            const bool valid = row < L;
+            const float Gr = valid ? sG[row] : 0.f;
+            const long long t = f * L + row;
+            const long long tok = ((long long)b * prm.T + t) * prm.H + h;
+            const float be = valid ? prm.beta[tok] : 0.f;
+            // this row's values (bf16), read before the waits to hide their latency
+            uint4 vrow[16];
+#pragma unroll
+            for (int c8 = 0; c8 < 16; ++c8)
+                vrow[c8] = (valid && c8 < dv / 8) ? *reinterpret_cast<const uint4 *>(prm.v + tok * dv + c8 * 8)
+                                                  : make_uint4(0, 0, 0, 0);
+
+            for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
+                const int sb = n & 1;
+                ok = sm100::mbar_wait(&bars[SFULL0 + sb], (n >> 1) & 1, err);
+                if (ok && n >= 2) ok = sm100::mbar_wait(&bars[PEMPTY0 + sb], ((n - 2) >> 1) & 1, err);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                const float a = sG[jt * JT + JT - 1];
+                const float rf = valid ? -be * __expf(Gr - a) : 0.f;
+                const float *cf = sCf + jt * JT;
+                unsigned char *pt = sP + sb * SLAB_BYTES;
+#pragma unroll 1
+                for (int c = 0; c < 2; ++c) {
+                    float v[32];
+                    sm100::tmem_ld32(t_s0 + sb * JT + lane_off + c * 32, v);
+                    sm100::tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c8 = c * 4 + u;  // 8-column chunk within the 64-column tile
+                        uint4 val = make_uint4(pack_bf16(rf * cf[c8 * 8 + 0] * v[u * 8 + 0], rf * cf[c8 * 8 + 1] * v[u * 8 + 1]),
+                                               pack_bf16(rf * cf[c8 * 8 + 2] * v[u * 8 + 2], rf * cf[c8 * 8 + 3] * v[u * 8 + 3]),
+                                               pack_bf16(rf * cf[c8 * 8 + 4] * v[u * 8 + 4], rf * cf[c8 * 8 + 5] * v[u * 8 + 5]),
+                                               pack_bf16(rf * cf[c8 * 8 + 6] * v[u * 8 + 6], rf * cf[c8 * 8 + 7] * v[u * 8 + 7]));
+                        *reinterpret_cast<uint4 *>(pt + r * 128 + ((c8 ^ (r & 7)) << 4)) = val;
+                    }
+                }
+                sm100::tc_fence_before();
+                sm100::mbar_arrive(&bars[SEMPTY0 + sb]);
+                sm100::fence_proxy_async_smem();
+                sm100::mbar_arrive(&bars[PFULL0 + sb]);
+            }
+            if (!ok) break;
+            // ---- Y_i = R_i + acc_i  -> sY (MN-major: row = K index of the T_ii Y_i product)
+            ok = sm100::mbar_wait(&bars[ACCFULL], i & 1, err);
+            if (!ok) break;
+            sm100::tc_fence_after();
+            const float rk = be * __expf(Gr);  // beta_r e^{G_r}
+#pragma unroll
+            for (int c0 = 0; c0 < 256; c0 += 32) {
+                if (c0 >= nc) break;
+                float acc[32];
+                if (i > 0) {
+                    sm100::tmem_ld32(t_acc + lane_off + c0, acc);
+                    sm100::tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u * 8;
+                    if (c >= nc) break;
+                    float y[8];
+                    if (c < dv) {
+                        const __nv_bfloat162 *vb = reinterpret_cast<const __nv_bfloat162 *>(&vrow[c >> 3]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 fv = __bfloat1622float2(vb[e]);
+                            y[2 * e] = be * fv.x;
+                            y[2 * e + 1] = be * fv.y;
+                        }
+                    } else {
+                        const int kc = c - dv;
+                        const uint4 kv = *reinterpret_cast<const uint4 *>(
+                            sKi + (kc >> 6) * SLAB_BYTES + r * 128 + ((((kc & 63) >> 3) ^ (r & 7)) << 4));
+                        const __nv_bfloat162 *kb = reinterpret_cast<const __nv_bfloat162 *>(&kv);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 fk = __bfloat1622float2(kb[e]);
+                            y[2 * e] = rk * fk.x;
+                            y[2 * e + 1] = rk * fk.y;
+                        }
+                    }
+                    uint4 val;
+                    if (valid) {
+                        val = make_uint4(pack_bf16(y[0] + acc[u * 8 + 0], y[1] + acc[u * 8 + 1]),
+                                         pack_bf16(y[2] + acc[u * 8 + 2], y[3] + acc[u * 8 + 3]),
+                                         pack_bf16(y[4] + acc[u * 8 + 4], y[5] + acc[u * 8 + 5]),
+                                         pack_bf16(y[6] + acc[u * 8 + 6], y[7] + acc[u * 8 + 7]));
+                    } else {
+                        val = make_uint4(0, 0, 0, 0);
+                    }
+                    *reinterpret_cast<uint4 *>(sY + (c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4)) =
+                        val;
+                }
+            }
+            sm100::tc_fence_before();
+            sm100::fence_proxy_async_smem();
+            sm100::mbar_arrive(&bars[YFULL]);
+            sm100::mbar_arrive(&bars[KIEMPTY]);
+            // ---- X_i = T_ii Y_i  -> global
+            ok = sm100::mbar_wait(&bars[XFULL], i & 1, err);
+            if (!ok) break;
+            sm100::tc_fence_after();
+            __nv_bfloat16 *xrow = prm.X + (fh * (long long)L + row) * nc;
+            for (int c0 = 0; c0 < nc; c0 += 32) {
+                float x[32];
+                sm100::tmem_ld32(t_acc + lane_off + c0, x);
+                sm100::tmem_ld_wait();
+                if (valid) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = c0 + u * 8;
+                        if (c >= nc) break;
+                        uint4 val = make_uint4(pack_bf16(x[u * 8 + 0], x[u * 8 + 1]), pack_bf16(x[u * 8 + 2], x[u * 8 + 3]),
+                                               pack_bf16(x[u * 8 + 4], x[u * 8 + 5]), pack_bf16(x[u * 8 + 6], x[u * 8 + 7]));
+                        *reinterpret_cast<uint4 *>(xrow + c) = val;
+                    }
+                }
+            }
+            fence_proxy_async_global();
+            sm100::tc_fence_before();
+            sm100::mbar_arrive(&bars[XDONE]);
+        }
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tbase, 512);
+    }
+}
+
+}  // namespace
+
+size_t intra_tc_smem_bytes(int L) {
+    return 1024 + Smem::F + sizeof(float) * 2 * L + 8 + sizeof(uint64_t) * NBAR + 16;
+}
+
+cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_t,
+                            const IntraParams &prm, long long n_fh, cudaStream_t s) {
+    const size_t smem = intra_tc_smem_bytes(prm.L);
+    cudaError_t e = cudaFuncSetAttribute(k_intra_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_t, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace gdn
