@@ -13,6 +13,7 @@
 // the block's 32 (or 16) rows of that column in registers.
 #include "gates.cuh"
 #include "gdn_internal.h"
+#include "sm100.cuh"
 
 namespace gdn {
 namespace {
@@ -230,7 +231,17 @@ __global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const TX *__
 
 // ---------------------------------------------------------------- k3 scan over frames
 // grid (B*H, ceil(dv/16)); the block carries 16 columns of Sig = S^T through
-// all frames of its chain, writing the state entering each frame to Sig_in.
+// all frames of its chain (Sig_next = M Sig + N), writing the state entering
+// each frame to SigIn (fp32) and/or SigB (bf16).  The next frame's M is
+// brought in by a bulk async copy into the other half of a double buffer
+// while the current step computes; every wait is bounded.
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(bytes), "r"((uint32_t)__cvta_generic_to_shared(bar))
+                 : "memory");
+}
+
 __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__restrict__ Mb,
                                                    const float *__restrict__ Nb, float *__restrict__ SigIn,
                                                    __nv_bfloat16 *__restrict__ SigB) {
@@ -238,62 +249,88 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
     const int dk = p.dk, dv = p.dv;
     const long long chain = blockIdx.x;
     const int c0 = blockIdx.y * SCAN_COLS, ncol = min(SCAN_COLS, dv - c0);
-    float *sM = (float *)smem;                       // [dk][dk+1]
-    float *sS = sM + dk * (dk + 1);                  // [dk][16]
+    float *sM = (float *)smem;                       // 2 x [dk][dk]
+    float *sS = sM + 2 * dk * dk;                    // [dk][16]
+    uint64_t *bar = (uint64_t *)(sS + dk * SCAN_COLS);
+    __shared__ int s_err;
     const int tid = threadIdx.x, c = tid & 15, g = tid >> 4;
-    const int ld = dk + 1;
+    const uint32_t mbytes = (uint32_t)(dk * dk * sizeof(float));
+    constexpr int MAXR = 128 / 16;
 
+    if (tid == 0) {
+        s_err = 0;
+        gdn::sm100::mbar_init(&bar[0], 1);
+        gdn::sm100::mbar_init(&bar[1], 1);
+        gdn::sm100::fence_barrier_init();
+    }
     for (int e = tid; e < dk * SCAN_COLS; e += NT) {
         const int m = e >> 4, cc = e & 15;
         float val = 0.f;
         if (p.S_in && cc < ncol) val = p.S_in[(chain * dv + c0 + cc) * (long long)dk + m];
         sS[e] = val;
     }
-    constexpr int MAXR = 128 / 16;
-    for (long long f = 0; f < p.F; ++f) {
-        const long long fh = chain * p.F + f;
-        __syncthreads();
-        if (frame_resets(p, f))
-            for (int e = tid; e < dk * SCAN_COLS; e += NT) sS[e] = 0.f;
-        __syncthreads();
-        for (int e = tid; e < dk * SCAN_COLS; e += NT) {
-            const int m = e >> 4, cc = e & 15;
-            if (cc < ncol) {
-                const long long idx = (fh * dk + m) * (long long)dv + c0 + cc;
-                if (SigIn) SigIn[idx] = sS[e];
-                if (SigB) SigB[idx] = __float2bfloat16_rn(sS[e]);
-            }
-        }
-        const float *Mf = Mb + fh * (long long)dk * dk;
-        for (int e = tid; e < dk * dk; e += NT) {
-            const int m = e / dk, l = e - m * dk;
-            sM[m * ld + l] = Mf[e];
-        }
-        __syncthreads();
-        float nv[MAXR];
-#pragma unroll
-        for (int i = 0; i < MAXR; ++i) {
-            const int m = g + 16 * i;
-            float a = 0.f;
-            if (m < dk && c < ncol) {
-                a = Nb[(fh * dk + m) * (long long)dv + c0 + c];
-                for (int l = 0; l < dk; ++l) a += sM[m * ld + l] * sS[l * SCAN_COLS + c];
-            }
-            nv[i] = a;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < MAXR; ++i) {
-            const int m = g + 16 * i;
-            if (m < dk) sS[m * SCAN_COLS + c] = nv[i];
-        }
-    }
     __syncthreads();
-    if (p.S_out) {
+    if (tid == 0 && p.F > 0) {
+        gdn::sm100::mbar_arrive_expect_tx(&bar[0], mbytes);
+        bulk_copy_g2s(sM, Mb + chain * p.F * (long long)dk * dk, mbytes, &bar[0]);
+    }
+    bool ok = true;
+    for (long long f = 0; f < p.F && ok; ++f) {
+        const long long fh = chain * p.F + f;
+        const int buf = (int)(f & 1);
+        if (tid == 0 && f + 1 < p.F) {  // prefetch the next frame's M into the other buffer
+            gdn::sm100::mbar_arrive_expect_tx(&bar[buf ^ 1], mbytes);
+            bulk_copy_g2s(sM + (buf ^ 1) * dk * dk, Mb + (fh + 1) * (long long)dk * dk, mbytes, &bar[buf ^ 1]);
+        }
+        if (frame_resets(p, f)) {
+            for (int e = tid; e < dk * SCAN_COLS; e += NT) sS[e] = 0.f;
+            __syncthreads();
+        }
+        float acc[MAXR];
+#pragma unroll
+        for (int i = 0; i < MAXR; ++i) {
+            const int m = g + 16 * i;
+            acc[i] = 0.f;
+            if (m < dk && c < ncol) {
+                const long long idx = (fh * dk + m) * (long long)dv + c0 + c;
+                const float cur = sS[m * SCAN_COLS + c];
+                if (SigIn) SigIn[idx] = cur;
+                if (SigB) SigB[idx] = __float2bfloat16_rn(cur);
+                acc[i] = Nb[idx];
+            }
+        }
+        ok = gdn::sm100::mbar_wait(&bar[buf], (uint32_t)((f >> 1) & 1), &s_err);
+        if (!ok) break;
+        const float *Mf = sM + buf * dk * dk;
+        for (int l = 0; l < dk; l += 4) {
+            const float s0 = sS[(l + 0) * SCAN_COLS + c], s1 = sS[(l + 1) * SCAN_COLS + c];
+            const float s2 = sS[(l + 2) * SCAN_COLS + c], s3 = sS[(l + 3) * SCAN_COLS + c];
+#pragma unroll
+            for (int i = 0; i < MAXR; ++i) {
+                const int m = g + 16 * i;
+                if (m < dk) {
+                    const float4 mm = *reinterpret_cast<const float4 *>(&Mf[m * dk + l]);
+                    acc[i] += mm.x * s0 + mm.y * s1 + mm.z * s2 + mm.w * s3;
+                }
+            }
+        }
+        __syncthreads();  // every read of sS and of this M buffer is done
+#pragma unroll
+        for (int i = 0; i < MAXR; ++i) {
+            const int m = g + 16 * i;
+            if (m < dk) sS[m * SCAN_COLS + c] = (c < ncol) ? acc[i] : 0.f;
+        }
+        __syncthreads();
+    }
+    if (ok && p.S_out) {
         for (int e = tid; e < dk * SCAN_COLS; e += NT) {
             const int m = e >> 4, cc = e & 15;
             if (cc < ncol) p.S_out[(chain * dv + c0 + cc) * (long long)dk + m] = sS[e];
         }
+    }
+    // leave with no copy in flight
+    if (tid == 0 && !ok) {
+        for (int b2 = 0; b2 < 2; ++b2) gdn::sm100::mbar_wait(&bar[b2], 0, &s_err);
     }
 }
 
@@ -518,7 +555,7 @@ cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t
 
     const size_t sm1 = gsm + sizeof(float) * (2 * dk * RB + RB * RB + RB * nc);
     const size_t sm2 = gsm + sizeof(float) * (RB * 32 + RB * nc);
-    const size_t sm3 = sizeof(float) * (dk * (dk + 1) + dk * SCAN_COLS);
+    const size_t sm3 = sizeof(float) * (2 * dk * dk + dk * SCAN_COLS) + 2 * sizeof(uint64_t);
     const size_t sm4 = gsm + sizeof(float) * (dk * dv + 3 * dk * RB + RB * RB + RB * dv);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k1_intra_simt<TIn, TG, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1))) return e;
@@ -586,7 +623,7 @@ cudaError_t simt_transition_bf16x(const Problem &p, const __nv_bfloat16 *X, floa
 
 cudaError_t simt_scan(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
                       cudaStream_t s) {
-    const size_t sm = sizeof(float) * (p.dk * (p.dk + 1) + p.dk * SCAN_COLS);
+    const size_t sm = sizeof(float) * (2 * p.dk * p.dk + p.dk * SCAN_COLS) + 2 * sizeof(uint64_t);
     cudaError_t e = cudaFuncSetAttribute(k3_scan_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e) return e;
     k3_scan_simt<<<dim3((unsigned)(p.B * p.H), (p.dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm, s>>>(p, Mb, Nb, Sig,

@@ -5,9 +5,9 @@
 //   gates       G = per-frame prefix of log alpha (fp32)
 //   inverse     T_ii = (I + A_ii)^{-1} per 128-row diagonal block (mma.sync)
 //   intra       [Ub | W] per frame-head, bf16, blocked forward substitution (tcgen05)
-//   transition  M, N per frame-head, fp32                 (CUDA cores for now)
+//   transition  M, N per frame-head, fp32                 (tcgen05)
 //   scan        entering state per frame, fp32 + bf16     (CUDA cores)
-//   output      U = Ub - W Sig (bf16), then the tcgen05 output kernel
+//   output      U = Ub - W Sig (bf16, tcgen05), then the tcgen05 output kernel
 #include <cstdlib>
 #include <mutex>
 
@@ -126,11 +126,11 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
 
     __nv_bfloat16 *Tinv = (__nv_bfloat16 *)(base + lay.Tinv);
     const int nc = p.dk + p.dv;
-    CUtensorMap tm_q, tm_k, tm_u, tm_sig, tm_k64, tm_x, tm_t;
+    CUtensorMap tm_q, tm_k, tm_u, tm_sig, tm_k64, tm_x, tm_t, tm_x128;
     if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
         !map_rows(&tm_u, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
         !map_tokens(&tm_k64, p.k, p, p.dk, 64) || !map_rows(&tm_x, X, nfh, p.L, nc, 64) ||
-        !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128))
+        !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128) || !map_rows(&tm_x128, X, nfh, p.L, nc, 128))
         return cudaErrorInvalidValue;
 
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
@@ -150,11 +150,17 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     ip.F = p.F; ip.T = p.T; ip.err = err;
     if ((e = tc::launch_intra_tc(tm_k64, tm_x, tm_t, ip, nfh, s))) return e;
     if ((e = mark(ev, 1, s))) return e;
-    if ((e = simt_transition_bf16x(p, X, Mb, Nb, s))) return e;
+    tc::TransParams tp;
+    tp.G = G; tp.M = Mb; tp.N = Nb;
+    tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
+    if ((e = tc::launch_transition_tc(tm_k, tm_x128, tp, nfh, s))) return e;
     if ((e = mark(ev, 2, s))) return e;
     if ((e = simt_scan(p, Mb, Nb, Sig, SigB, s))) return e;
     if ((e = mark(ev, 3, s))) return e;
-    if ((e = simt_u_bf16x(p, X, Sig, U, s))) return e;
+    tc::UParams up;
+    up.X = X; up.U = U;
+    up.L = p.L; up.dk = p.dk; up.dv = p.dv; up.nblk = nblk; up.err = err;
+    if ((e = tc::launch_u_tc(tm_x128, tm_sig, up, nfh, s))) return e;
 
     tc::OutParams op;
     op.G = G;

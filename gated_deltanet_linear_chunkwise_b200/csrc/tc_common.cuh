@@ -56,6 +56,27 @@ struct IntraParams {
     int *err;
 };
 
+struct TransParams {
+    const float *G;            // [n_fh][L]
+    float *M;                  // [n_fh][dk][dk]
+    float *N;                  // [n_fh][dk][dv]
+    int L, dk, dv, H, nblk;
+    long long F;
+    int *err;
+};
+
+struct UParams {
+    const __nv_bfloat16 *X;    // [n_fh][L][dv + dk]
+    __nv_bfloat16 *U;          // [n_fh][L][dv]
+    int L, dk, dv, nblk;
+    int *err;
+};
+
+cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const TransParams &prm,
+                                 long long n_fh, cudaStream_t s);
+cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_sig, const UParams &prm, long long n_fh,
+                        cudaStream_t s);
+
 cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_t,
                             const IntraParams &prm, long long n_fh, cudaStream_t s);
 
