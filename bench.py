@@ -166,6 +166,8 @@ def main():
     ap.add_argument("--ref-frames", type=int, default=2, help="frames per --impl reference step")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, help="named workload (the metric is quoted on 'minute'; "
+                                                          "others are for profiling small cases)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -190,10 +192,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    w = W.WORKLOADS[WORKLOAD]
+    w = W.WORKLOADS[args.workload]
     L, dk, dv, H = w.frame_len, w.d_k, w.d_v, w.H
     # each rank draws its own batch element (weak scaling)
-    inp = W.make_inputs(w, args.regime, seed=W.SEEDS[WORKLOAD] + 7919 * rank)
+    inp = W.make_inputs(w, args.regime, seed=W.SEEDS[args.workload] + 7919 * rank, call=0)
     d = {k: (None if t is None else t.to(dev).contiguous()) for k, t in inp.items()}
     B, T = w.B, w.T
     o = torch.empty(B, T, H, dv, dtype=torch.bfloat16, device=dev)
@@ -287,8 +289,11 @@ def main():
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "minute: B=1 per GPU, H=20, T=106480 (121 frames x 880 tokens), "
-                                   "d_k=d_v=112, bf16 q/k/v/o, fp32 gates and state, chunk = frame",
+            "config": {"workload": ("minute: B=1 per GPU, H=20, T=106480 (121 frames x 880 tokens), "
+                                    "d_k=d_v=112, bf16 q/k/v/o, fp32 gates and state, chunk = frame")
+                                   if args.workload == WORKLOAD else
+                                   "%s: B=%d H=%d T=%d (%d x %d) d_k=%d d_v=%d (profiling case)"
+                                   % (w.name, B, H, T, w.frames, L, dk, dv),
                        "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
                        "gate_regime": args.regime,
                        "l2": "no flush: inputs 1.4 GB per step exceed the 126 MB L2"},
@@ -306,7 +311,7 @@ def main():
             "gpu_launches": NUM_STAGES * args.steps,
             "clocks": clk.summary(),
         }
-        if not args.no_cpu_baseline and world == 1:
+        if not args.no_cpu_baseline and world == 1 and args.workload == WORKLOAD:
             line["cpu_baseline"] = cpu_baseline(args.regime, args.cpu_frames, inp)
         print(json.dumps(line), flush=True)
     if world > 1:

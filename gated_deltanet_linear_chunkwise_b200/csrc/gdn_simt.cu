@@ -233,15 +233,21 @@ __global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const TX *__
 // grid (B*H, ceil(dv/16)); the block carries 16 columns of Sig = S^T through
 // all frames of its chain (Sig_next = M Sig + N), writing the state entering
 // each frame to SigIn (fp32) and/or SigB (bf16).  The next frame's M is
-// brought in by a bulk async copy into the other half of a double buffer
-// while the current step computes; every wait is bounded.
-__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     (uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src), "r"(bytes), "r"((uint32_t)__cvta_generic_to_shared(bar))
+// brought in by cp.async into the other half of a double buffer while the
+// current step computes.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// Thread layout: 256 threads = 2 halves of the contraction index l x 8
+// column pairs x 16 row groups; each thread accumulates rows m = g + 16i of
+// two columns over its half of l (14 independent sums at d_k = 112), and
+// the halves are added through shared memory.  N for the next frame is
+// loaded one step ahead.
 __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__restrict__ Mb,
                                                    const float *__restrict__ Nb, float *__restrict__ SigIn,
                                                    __nv_bfloat16 *__restrict__ SigB) {
@@ -251,18 +257,13 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
     const int c0 = blockIdx.y * SCAN_COLS, ncol = min(SCAN_COLS, dv - c0);
     float *sM = (float *)smem;                       // 2 x [dk][dk]
     float *sS = sM + 2 * dk * dk;                    // [dk][16]
-    uint64_t *bar = (uint64_t *)(sS + dk * SCAN_COLS);
-    __shared__ int s_err;
-    const int tid = threadIdx.x, c = tid & 15, g = tid >> 4;
-    const uint32_t mbytes = (uint32_t)(dk * dk * sizeof(float));
+    float *sRed = sS + dk * SCAN_COLS;               // [8][128][2] partial sums of the upper l half
+    const int tid = threadIdx.x;
+    const int kh = tid >> 7, t7 = tid & 127, cp = t7 & 7, g = t7 >> 3;
+    const int ca = 2 * cp, cb = 2 * cp + 1;          // this thread's two columns
+    const int l0 = kh * (dk / 2), l1 = l0 + dk / 2;
     constexpr int MAXR = 128 / 16;
 
-    if (tid == 0) {
-        s_err = 0;
-        gdn::sm100::mbar_init(&bar[0], 1);
-        gdn::sm100::mbar_init(&bar[1], 1);
-        gdn::sm100::fence_barrier_init();
-    }
     for (int e = tid; e < dk * SCAN_COLS; e += NT) {
         const int m = e >> 4, cc = e & 15;
         float val = 0.f;
@@ -270,68 +271,110 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
         sS[e] = val;
     }
     __syncthreads();
-    if (tid == 0 && p.F > 0) {
-        gdn::sm100::mbar_arrive_expect_tx(&bar[0], mbytes);
-        bulk_copy_g2s(sM, Mb + chain * p.F * (long long)dk * dk, mbytes, &bar[0]);
+    const int nvec = dk * dk / 4;  // 16-byte pieces of one M
+    if (p.F > 0) {
+        const float4 *src = reinterpret_cast<const float4 *>(Mb + chain * p.F * (long long)dk * dk);
+        for (int e = tid; e < nvec; e += NT) cp_async16(sM + 4 * e, src + e);
     }
-    bool ok = true;
-    for (long long f = 0; f < p.F && ok; ++f) {
+    cp_async_commit();
+    // N of the first frame (the lower l half adds N; the upper half does not)
+    float2 nxt[MAXR];
+#pragma unroll
+    for (int i = 0; i < MAXR; ++i) {
+        const int m = g + 16 * i;
+        nxt[i] = make_float2(0.f, 0.f);
+        if (kh == 0 && m < dk && p.F > 0) {
+            const long long idx = (chain * p.F * dk + m) * (long long)dv + c0;
+            nxt[i].x = ca < ncol ? Nb[idx + ca] : 0.f;
+            nxt[i].y = cb < ncol ? Nb[idx + cb] : 0.f;
+        }
+    }
+    for (long long f = 0; f < p.F; ++f) {
         const long long fh = chain * p.F + f;
         const int buf = (int)(f & 1);
-        if (tid == 0 && f + 1 < p.F) {  // prefetch the next frame's M into the other buffer
-            gdn::sm100::mbar_arrive_expect_tx(&bar[buf ^ 1], mbytes);
-            bulk_copy_g2s(sM + (buf ^ 1) * dk * dk, Mb + (fh + 1) * (long long)dk * dk, mbytes, &bar[buf ^ 1]);
+        if (f + 1 < p.F) {  // prefetch the next frame's M into the other buffer
+            const float4 *src = reinterpret_cast<const float4 *>(Mb + (fh + 1) * (long long)dk * dk);
+            float *dst = sM + (buf ^ 1) * dk * dk;
+            for (int e = tid; e < nvec; e += NT) cp_async16(dst + 4 * e, src + e);
         }
+        cp_async_commit();
         if (frame_resets(p, f)) {
             for (int e = tid; e < dk * SCAN_COLS; e += NT) sS[e] = 0.f;
             __syncthreads();
         }
-        float acc[MAXR];
+        float2 acc[MAXR];
 #pragma unroll
         for (int i = 0; i < MAXR; ++i) {
             const int m = g + 16 * i;
-            acc[i] = 0.f;
-            if (m < dk && c < ncol) {
-                const long long idx = (fh * dk + m) * (long long)dv + c0 + c;
-                const float cur = sS[m * SCAN_COLS + c];
-                if (SigIn) SigIn[idx] = cur;
-                if (SigB) SigB[idx] = __float2bfloat16_rn(cur);
-                acc[i] = Nb[idx];
+            acc[i] = nxt[i];
+            nxt[i] = make_float2(0.f, 0.f);
+            if (kh == 0 && m < dk) {
+                const long long idx = (fh * dk + m) * (long long)dv + c0;
+                const float sa = sS[m * SCAN_COLS + ca], sb = sS[m * SCAN_COLS + cb];
+                if (ca < ncol) {
+                    if (SigIn) SigIn[idx + ca] = sa;
+                    if (SigB) SigB[idx + ca] = __float2bfloat16_rn(sa);
+                }
+                if (cb < ncol) {
+                    if (SigIn) SigIn[idx + cb] = sb;
+                    if (SigB) SigB[idx + cb] = __float2bfloat16_rn(sb);
+                }
+                if (f + 1 < p.F) {
+                    const long long nidx = ((fh + 1) * dk + m) * (long long)dv + c0;
+                    nxt[i].x = ca < ncol ? Nb[nidx + ca] : 0.f;
+                    nxt[i].y = cb < ncol ? Nb[nidx + cb] : 0.f;
+                }
             }
         }
-        ok = gdn::sm100::mbar_wait(&bar[buf], (uint32_t)((f >> 1) & 1), &s_err);
-        if (!ok) break;
+        cp_async_wait_one();  // this frame's M (committed one step earlier) has landed
+        __syncthreads();
         const float *Mf = sM + buf * dk * dk;
-        for (int l = 0; l < dk; l += 4) {
-            const float s0 = sS[(l + 0) * SCAN_COLS + c], s1 = sS[(l + 1) * SCAN_COLS + c];
-            const float s2 = sS[(l + 2) * SCAN_COLS + c], s3 = sS[(l + 3) * SCAN_COLS + c];
+        for (int l = l0; l < l1; l += 4) {
+            const float2 s0 = *reinterpret_cast<const float2 *>(&sS[(l + 0) * SCAN_COLS + ca]);
+            const float2 s1 = *reinterpret_cast<const float2 *>(&sS[(l + 1) * SCAN_COLS + ca]);
+            const float2 s2 = *reinterpret_cast<const float2 *>(&sS[(l + 2) * SCAN_COLS + ca]);
+            const float2 s3 = *reinterpret_cast<const float2 *>(&sS[(l + 3) * SCAN_COLS + ca]);
 #pragma unroll
             for (int i = 0; i < MAXR; ++i) {
                 const int m = g + 16 * i;
                 if (m < dk) {
                     const float4 mm = *reinterpret_cast<const float4 *>(&Mf[m * dk + l]);
-                    acc[i] += mm.x * s0 + mm.y * s1 + mm.z * s2 + mm.w * s3;
+                    acc[i].x += mm.x * s0.x;
+                    acc[i].y += mm.x * s0.y;
+                    acc[i].x += mm.y * s1.x;
+                    acc[i].y += mm.y * s1.y;
+                    acc[i].x += mm.z * s2.x;
+                    acc[i].y += mm.z * s2.y;
+                    acc[i].x += mm.w * s3.x;
+                    acc[i].y += mm.w * s3.y;
                 }
             }
         }
-        __syncthreads();  // every read of sS and of this M buffer is done
+        if (kh == 1) {
 #pragma unroll
-        for (int i = 0; i < MAXR; ++i) {
-            const int m = g + 16 * i;
-            if (m < dk) sS[m * SCAN_COLS + c] = (c < ncol) ? acc[i] : 0.f;
+            for (int i = 0; i < MAXR; ++i) reinterpret_cast<float2 *>(sRed)[i * 128 + t7] = acc[i];
+        }
+        __syncthreads();  // every read of sS and of this M buffer is done; partial sums are in sRed
+        if (kh == 0) {
+#pragma unroll
+            for (int i = 0; i < MAXR; ++i) {
+                const int m = g + 16 * i;
+                if (m < dk) {
+                    const float2 o = reinterpret_cast<const float2 *>(sRed)[i * 128 + t7];
+                    sS[m * SCAN_COLS + ca] = (ca < ncol) ? acc[i].x + o.x : 0.f;
+                    sS[m * SCAN_COLS + cb] = (cb < ncol) ? acc[i].y + o.y : 0.f;
+                }
+            }
         }
         __syncthreads();
     }
-    if (ok && p.S_out) {
+    if (p.S_out) {
         for (int e = tid; e < dk * SCAN_COLS; e += NT) {
             const int m = e >> 4, cc = e & 15;
             if (cc < ncol) p.S_out[(chain * dv + c0 + cc) * (long long)dk + m] = sS[e];
         }
     }
-    // leave with no copy in flight
-    if (tid == 0 && !ok) {
-        for (int b2 = 0; b2 < 2; ++b2) gdn::sm100::mbar_wait(&bar[b2], 0, &s_err);
-    }
+    cp_async_wait_all();  // leave with no copy in flight
 }
 
 // ---------------------------------------------------------------- k4 output
@@ -555,7 +598,7 @@ cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t
 
     const size_t sm1 = gsm + sizeof(float) * (2 * dk * RB + RB * RB + RB * nc);
     const size_t sm2 = gsm + sizeof(float) * (RB * 32 + RB * nc);
-    const size_t sm3 = sizeof(float) * (2 * dk * dk + dk * SCAN_COLS) + 2 * sizeof(uint64_t);
+    const size_t sm3 = sizeof(float) * (2 * dk * dk + dk * SCAN_COLS + 8 * 128 * 2);
     const size_t sm4 = gsm + sizeof(float) * (dk * dv + 3 * dk * RB + RB * RB + RB * dv);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k1_intra_simt<TIn, TG, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1))) return e;
@@ -623,7 +666,7 @@ cudaError_t simt_transition_bf16x(const Problem &p, const __nv_bfloat16 *X, floa
 
 cudaError_t simt_scan(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
                       cudaStream_t s) {
-    const size_t sm = sizeof(float) * (2 * p.dk * p.dk + p.dk * SCAN_COLS) + 2 * sizeof(uint64_t);
+    const size_t sm = sizeof(float) * (2 * p.dk * p.dk + p.dk * SCAN_COLS + 8 * 128 * 2);
     cudaError_t e = cudaFuncSetAttribute(k3_scan_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e) return e;
     k3_scan_simt<<<dim3((unsigned)(p.B * p.H), (p.dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm, s>>>(p, Mb, Nb, Sig,

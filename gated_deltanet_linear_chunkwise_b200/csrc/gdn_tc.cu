@@ -20,8 +20,12 @@
 namespace gdn {
 namespace {
 
+// Row stride of the column-factor rows: a multiple of 4 floats so that
+// every row starts on a 16-byte boundary (they are read as float4).
+inline int cf_stride(int L) { return (L + 3) & ~3; }
+
 struct TcLayout {
-    size_t G, Tinv, X, M, N, Sig, SigB, U, err, total;
+    size_t G, CF, Tinv, X, M, N, Sig, SigB, U, err, total;
 };
 
 TcLayout tc_layout(const Problem &p) {
@@ -29,7 +33,8 @@ TcLayout tc_layout(const Problem &p) {
     const size_t nc = (size_t)p.dk + p.dv;
     TcLayout lay;
     size_t off = 0;
-    lay.G = off;    off += align256(sizeof(float) * nfh * p.L);
+    lay.G = off;    off += align256(sizeof(float) * nfh * (size_t)cf_stride(p.L));
+    lay.CF = off;   off += align256(sizeof(float) * nfh * (size_t)cf_stride(p.L));
     lay.Tinv = off; off += align256(2 * nfh * (size_t)((p.L + 127) / 128) * 128 * 128);
     lay.X = off;    off += align256(2 * nfh * p.L * nc);
     lay.M = off;    off += align256(sizeof(float) * nfh * p.dk * p.dk);
@@ -77,6 +82,20 @@ bool map_tokens(CUtensorMap *m, const void *x, const Problem &p, int d, int box_
     return make_map(m, x, 4, dims, strides, box);
 }
 
+// fp32 rows [n_fh][stride] seen as 2-D (len, n_fh), boxes of 128 elements, no swizzle;
+// elements past `len` read as zeros.
+bool map_f32_rows(CUtensorMap *m, const float *x, long long nfh, int len, int stride) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)len, (cuuint64_t)nfh};
+    const cuuint64_t strides[1] = {(cuuint64_t)stride * 4};
+    const cuuint32_t box[2] = {128, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(x), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Workspace [n_fh][rows][cols] bf16 seen as 3-D (cols, rows, n_fh).
 bool map_rows(CUtensorMap *m, const void *x, long long nfh, int rows, int cols, int box_rows) {
     const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)nfh};
@@ -85,7 +104,10 @@ bool map_rows(CUtensorMap *m, const void *x, long long nfh, int rows, int cols, 
     return make_map(m, x, 3, dims, strides, box);
 }
 
-__global__ void __launch_bounds__(256) gate_prefix_kernel(Problem p, float *__restrict__ G) {
+// G = per-frame inclusive prefix of log alpha; CF = e^{a(s) - G_s} with a(s)
+// = G at the last token of s's 64-token tile (<= 1): the column half of the
+// split decay factor e^{G_r - G_s} = e^{G_r - a} e^{a - G_s}.
+__global__ void __launch_bounds__(256) gate_prefix_kernel(Problem p, float *__restrict__ G, float *__restrict__ CF) {
     extern __shared__ __align__(16) unsigned char smem[];
     const long long fh = blockIdx.x;
     const long long f = fh % p.F, chain = fh / p.F;
@@ -94,7 +116,12 @@ __global__ void __launch_bounds__(256) gate_prefix_kernel(Problem p, float *__re
     float *sB = sG + p.L;
     float *sScr = sB + p.L;
     frame_gates<float>(p, b, h, f, sG, sB, sScr);
-    for (int i = threadIdx.x; i < p.L; i += blockDim.x) G[fh * p.L + i] = sG[i];
+    const int cfs = (p.L + 3) & ~3;  // cf_stride(L): G and CF rows start on 16-byte boundaries
+    for (int i = threadIdx.x; i < p.L; i += blockDim.x) {
+        const int end = min((i / 64) * 64 + 63, p.L - 1);
+        G[fh * cfs + i] = sG[i];
+        CF[fh * cfs + i] = __expf(sG[end] - sG[i]);
+    }
 }
 
 bool tc_disabled_by_env() {
@@ -117,6 +144,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     const long long nfh = (long long)p.B * p.H * p.F;
     const int nblk = (p.L + tc::BM - 1) / tc::BM;
     float *G = (float *)(base + lay.G);
+    float *CF = (float *)(base + lay.CF);
     __nv_bfloat16 *X = (__nv_bfloat16 *)(base + lay.X);
     float *Mb = (float *)(base + lay.M), *Nb = (float *)(base + lay.N), *Sig = (float *)(base + lay.Sig);
     __nv_bfloat16 *SigB = (__nv_bfloat16 *)(base + lay.SigB);
@@ -126,11 +154,12 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
 
     __nv_bfloat16 *Tinv = (__nv_bfloat16 *)(base + lay.Tinv);
     const int nc = p.dk + p.dv;
-    CUtensorMap tm_q, tm_k, tm_u, tm_sig, tm_k64, tm_x, tm_t, tm_x128;
+    CUtensorMap tm_q, tm_k, tm_u, tm_sig, tm_k64, tm_x, tm_t, tm_x128, tm_g, tm_cf;
     if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
         !map_rows(&tm_u, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
         !map_tokens(&tm_k64, p.k, p, p.dk, 64) || !map_rows(&tm_x, X, nfh, p.L, nc, 64) ||
-        !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128) || !map_rows(&tm_x128, X, nfh, p.L, nc, 128))
+        !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128) || !map_rows(&tm_x128, X, nfh, p.L, nc, 128) ||
+        !map_f32_rows(&tm_g, G, nfh, p.L, cf_stride(p.L)) || !map_f32_rows(&tm_cf, CF, nfh, p.L, cf_stride(p.L)))
         return cudaErrorInvalidValue;
 
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
@@ -139,7 +168,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
         (e = cudaFuncSetAttribute(gate_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm)))
         return e;
     if ((e = mark(ev, 0, s))) return e;
-    gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G);
+    gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF);
     if ((e = cudaGetLastError())) return e;
     if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
                                      nfh, s)))
@@ -164,12 +193,15 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
 
     tc::OutParams op;
     op.G = G;
+    op.CF = CF;
     op.o = p.o;
     op.L = p.L; op.dk = p.dk; op.dv = p.dv; op.H = p.H; op.nblk = nblk;
-    op.F = p.F; op.T = p.T;
+    op.F = p.F; op.T = p.T; op.n_fh = nfh;
     op.accumulate = p.accumulate;
     op.err = err;
-    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u, tm_sig, op, nfh, s))) return e;
+    int dev = 0, num_sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u, tm_sig, tm_g, tm_cf, op, num_sms, s))) return e;
     return mark(ev, 4, s);
 }
 

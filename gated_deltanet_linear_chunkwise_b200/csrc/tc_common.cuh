@@ -38,16 +38,18 @@ __device__ __forceinline__ uint64_t desc_mnmajor(const void *tile, int ks, int k
 }
 
 struct OutParams {
-    const float *G;          // [n_fh][L] inclusive prefix of clamped log alpha per frame
+    const float *G;          // [n_fh][(L+3)&~3] inclusive prefix of clamped log alpha per frame
+    const float *CF;         // [n_fh][(L+3)&~3] column decay factors e^{a(s) - G_s}, a = G at the end of s's
+                             // 64-token tile (G and cf rows are padded to a multiple of 4 floats)
     void *o;                 // [B,T,H,dv] bf16
     int L, dk, dv, H, nblk;
-    long long F, T;
+    long long F, T, n_fh;
     int accumulate;
     int *err;
 };
 
 struct IntraParams {
-    const float *G;            // [n_fh][L]
+    const float *G;            // [n_fh][(L+3)&~3]
     const float *beta;         // [B,T,H]
     const __nv_bfloat16 *v;    // [B,T,H,dv]
     __nv_bfloat16 *X;          // [n_fh][L][dk + dv]: Ub (first dv columns) then W
@@ -57,7 +59,7 @@ struct IntraParams {
 };
 
 struct TransParams {
-    const float *G;            // [n_fh][L]
+    const float *G;            // [n_fh][(L+3)&~3]
     float *M;                  // [n_fh][dk][dk]
     float *N;                  // [n_fh][dk][dv]
     int L, dk, dv, H, nblk;
@@ -85,7 +87,8 @@ cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const
                                 cudaStream_t s);
 
 cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
-                             const CUtensorMap &tm_sig, const OutParams &prm, long long n_fh, cudaStream_t s);
+                             const CUtensorMap &tm_sig, const CUtensorMap &tm_g, const CUtensorMap &tm_cf,
+                             const OutParams &prm, int num_sms, cudaStream_t s);
 
 }  // namespace tc
 }  // namespace gdn

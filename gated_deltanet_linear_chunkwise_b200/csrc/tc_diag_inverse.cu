@@ -25,6 +25,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int LDK = 128 + 8;   // bf16 row stride of the K tile (conflict-free ldmatrix)
 constexpr int LDT = 128 + 8;   // bf16 row stride of the A / T / scratch tiles
+static_assert(LDK == LDT, "the scratch tile reuses the K tile");
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -101,13 +102,13 @@ struct InvParams {
     long long F, T;
 };
 
-__global__ void __launch_bounds__(kThreads) k_diag_inverse(const InvParams prm) {
+__global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams prm) {
     extern __shared__ __align__(16) unsigned char smem[];
     __nv_bfloat16 *sK = (__nv_bfloat16 *)smem;          // [128][LDK]
     __nv_bfloat16 *sA = sK + 128 * LDK;                 // [128][LDT]  A (strictly lower)
     __nv_bfloat16 *sT = sA + 128 * LDT;                 // [128][LDT]  T
-    __nv_bfloat16 *sX = sT + 128 * LDT;                 // [128][LDT]  scratch products
-    float *sAd = (float *)(sX + 128 * LDT);             // [8][16][16] fp32 diagonal leaves of A
+    __nv_bfloat16 *sX = sK;                             // scratch products reuse the K tile (LDK == LDT)
+    float *sAd = (float *)(sT + 128 * LDT);             // [8][16][16] fp32 diagonal leaves of A
     float *sG = sAd + 8 * 256;                          // [128]
     float *sB = sG + 128;                               // [128]
 
@@ -140,7 +141,7 @@ __global__ void __launch_bounds__(kThreads) k_diag_inverse(const InvParams prm) 
     }
     if (tid < 128) {
         const int r = r_base + tid;
-        const float *Gf = prm.G + fh * (long long)L;
+        const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
         sG[tid] = Gf[r < L ? r : L - 1];
         sB[tid] = (r < L) ? prm.beta[((long long)b * prm.T + f * L + r) * prm.H + h] : 0.f;
     }
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(kThreads) k_diag_inverse(const InvParams prm) 
 }  // namespace
 
 size_t diag_inverse_smem_bytes() {
-    return sizeof(__nv_bfloat16) * (128 * LDK + 3 * 128 * LDT) + sizeof(float) * (8 * 256 + 256);
+    return sizeof(__nv_bfloat16) * (128 * LDK + 2 * 128 * LDT) + sizeof(float) * (8 * 256 + 256);
 }
 
 cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, __nv_bfloat16 *Tinv,

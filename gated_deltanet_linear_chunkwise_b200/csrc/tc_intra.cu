@@ -188,7 +188,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        const float *Gf = prm.G + fh * (long long)L;
+        const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
         for (int s = et; s < L; s += 128) {
             const int tile_end = min((s / JT) * JT + JT - 1, L - 1);
             const float g = Gf[s];

@@ -100,7 +100,7 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     } else {
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;  // token row of each block; at the end, key dimension m
-        const float *Gf = prm.G + fh * (long long)L;
+        const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
         const float GL = Gf[L - 1];
         bool ok = true;
         for (int i = 0; i < nblk && ok; ++i) {
