@@ -245,136 +245,150 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 // Thread layout: 256 threads = 2 halves of the contraction index l x 8
 // column pairs x 16 row groups; each thread accumulates rows m = g + 16i of
-// two columns over its half of l (14 independent sums at d_k = 112), and
-// the halves are added through shared memory.  N for the next frame is
-// loaded one step ahead.
+// two columns over its half of l (2 DK/16 independent sums), and the halves
+// are added through shared memory.  N for the next frame is loaded one step
+// ahead.  DK is a template parameter so every loop has a fixed trip count.
+template <int DK>
 __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__restrict__ Mb,
                                                    const float *__restrict__ Nb, float *__restrict__ SigIn,
                                                    __nv_bfloat16 *__restrict__ SigB) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int dk = p.dk, dv = p.dv;
+    constexpr int R = DK / 16;                       // rows per thread
+    constexpr int HALF = DK / 2;                     // contraction length per thread half
+    const int dv = p.dv;
     const long long chain = blockIdx.x;
     const int c0 = blockIdx.y * SCAN_COLS, ncol = min(SCAN_COLS, dv - c0);
-    float *sM = (float *)smem;                       // 2 x [dk][dk]
-    float *sS = sM + 2 * dk * dk;                    // [dk][16]
-    float *sRed = sS + dk * SCAN_COLS;               // [8][128][2] partial sums of the upper l half
+    float *sM = (float *)smem;                       // 2 x [DK][DK]
+    float *sS = sM + 2 * DK * DK;                    // [DK][16]
+    float2 *sRed = reinterpret_cast<float2 *>(sS + DK * SCAN_COLS);  // [R][128] partial sums of the upper half
     const int tid = threadIdx.x;
     const int kh = tid >> 7, t7 = tid & 127, cp = t7 & 7, g = t7 >> 3;
     const int ca = 2 * cp, cb = 2 * cp + 1;          // this thread's two columns
-    const int l0 = kh * (dk / 2), l1 = l0 + dk / 2;
-    constexpr int MAXR = 128 / 16;
+    const int l0 = kh * HALF;
 
-    for (int e = tid; e < dk * SCAN_COLS; e += NT) {
+    for (int e = tid; e < DK * SCAN_COLS; e += NT) {
         const int m = e >> 4, cc = e & 15;
         float val = 0.f;
-        if (p.S_in && cc < ncol) val = p.S_in[(chain * dv + c0 + cc) * (long long)dk + m];
+        if (p.S_in && cc < ncol) val = p.S_in[(chain * dv + c0 + cc) * (long long)DK + m];
         sS[e] = val;
     }
-    __syncthreads();
-    const int nvec = dk * dk / 4;  // 16-byte pieces of one M
+    constexpr int NVEC = DK * DK / 4;  // 16-byte pieces of one M
     if (p.F > 0) {
-        const float4 *src = reinterpret_cast<const float4 *>(Mb + chain * p.F * (long long)dk * dk);
-        for (int e = tid; e < nvec; e += NT) cp_async16(sM + 4 * e, src + e);
+        const float4 *src = reinterpret_cast<const float4 *>(Mb + chain * p.F * (long long)DK * DK);
+        for (int e = tid; e < NVEC; e += NT) cp_async16(sM + 4 * e, src + e);
     }
     cp_async_commit();
     // N of the first frame (the lower l half adds N; the upper half does not)
-    float2 nxt[MAXR];
+    float2 nxt[R];
 #pragma unroll
-    for (int i = 0; i < MAXR; ++i) {
+    for (int i = 0; i < R; ++i) {
         const int m = g + 16 * i;
         nxt[i] = make_float2(0.f, 0.f);
-        if (kh == 0 && m < dk && p.F > 0) {
-            const long long idx = (chain * p.F * dk + m) * (long long)dv + c0;
+        if (kh == 0 && p.F > 0) {
+            const long long idx = (chain * p.F * DK + m) * (long long)dv + c0;
             nxt[i].x = ca < ncol ? Nb[idx + ca] : 0.f;
             nxt[i].y = cb < ncol ? Nb[idx + cb] : 0.f;
         }
     }
+    __syncthreads();
     for (long long f = 0; f < p.F; ++f) {
         const long long fh = chain * p.F + f;
         const int buf = (int)(f & 1);
         if (f + 1 < p.F) {  // prefetch the next frame's M into the other buffer
-            const float4 *src = reinterpret_cast<const float4 *>(Mb + (fh + 1) * (long long)dk * dk);
-            float *dst = sM + (buf ^ 1) * dk * dk;
-            for (int e = tid; e < nvec; e += NT) cp_async16(dst + 4 * e, src + e);
+            const float4 *src = reinterpret_cast<const float4 *>(Mb + (fh + 1) * (long long)DK * DK);
+            float *dst = sM + (buf ^ 1) * DK * DK;
+            for (int e = tid; e < NVEC; e += NT) cp_async16(dst + 4 * e, src + e);
         }
         cp_async_commit();
         if (frame_resets(p, f)) {
-            for (int e = tid; e < dk * SCAN_COLS; e += NT) sS[e] = 0.f;
+            for (int e = tid; e < DK * SCAN_COLS; e += NT) sS[e] = 0.f;
             __syncthreads();
         }
-        float2 acc[MAXR];
+        float2 acc[R];
 #pragma unroll
-        for (int i = 0; i < MAXR; ++i) {
+        for (int i = 0; i < R; ++i) {
             const int m = g + 16 * i;
             acc[i] = nxt[i];
             nxt[i] = make_float2(0.f, 0.f);
-            if (kh == 0 && m < dk) {
-                const long long idx = (fh * dk + m) * (long long)dv + c0;
-                const float sa = sS[m * SCAN_COLS + ca], sb = sS[m * SCAN_COLS + cb];
-                if (ca < ncol) {
-                    if (SigIn) SigIn[idx + ca] = sa;
-                    if (SigB) SigB[idx + ca] = __float2bfloat16_rn(sa);
-                }
-                if (cb < ncol) {
-                    if (SigIn) SigIn[idx + cb] = sb;
-                    if (SigB) SigB[idx + cb] = __float2bfloat16_rn(sb);
-                }
-                if (f + 1 < p.F) {
-                    const long long nidx = ((fh + 1) * dk + m) * (long long)dv + c0;
-                    nxt[i].x = ca < ncol ? Nb[nidx + ca] : 0.f;
-                    nxt[i].y = cb < ncol ? Nb[nidx + cb] : 0.f;
-                }
+            if (kh == 0) {
+                const long long idx = (fh * DK + m) * (long long)dv + c0;
+                const float2 cur = *reinterpret_cast<const float2 *>(&sS[m * SCAN_COLS + ca]);
+                if (SigIn) *reinterpret_cast<float2 *>(SigIn + idx + ca) = cur;
+                if (SigB) *reinterpret_cast<__nv_bfloat162 *>(SigB + idx + ca) = __floats2bfloat162_rn(cur.x, cur.y);
+                if (f + 1 < p.F) nxt[i] = *reinterpret_cast<const float2 *>(Nb + ((fh + 1) * DK + m) * (long long)dv + c0 + ca);
             }
         }
         cp_async_wait_one();  // this frame's M (committed one step earlier) has landed
         __syncthreads();
-        const float *Mf = sM + buf * dk * dk;
-        for (int l = l0; l < l1; l += 4) {
-            const float2 s0 = *reinterpret_cast<const float2 *>(&sS[(l + 0) * SCAN_COLS + ca]);
-            const float2 s1 = *reinterpret_cast<const float2 *>(&sS[(l + 1) * SCAN_COLS + ca]);
-            const float2 s2 = *reinterpret_cast<const float2 *>(&sS[(l + 2) * SCAN_COLS + ca]);
-            const float2 s3 = *reinterpret_cast<const float2 *>(&sS[(l + 3) * SCAN_COLS + ca]);
+        const float *Mf = sM + buf * DK * DK + l0;
+        const float *Sf = sS + l0 * SCAN_COLS + ca;
+#pragma unroll 2
+        for (int l = 0; l < HALF; l += 4) {
+            const float2 s0 = *reinterpret_cast<const float2 *>(&Sf[(l + 0) * SCAN_COLS]);
+            const float2 s1 = *reinterpret_cast<const float2 *>(&Sf[(l + 1) * SCAN_COLS]);
+            const float2 s2 = *reinterpret_cast<const float2 *>(&Sf[(l + 2) * SCAN_COLS]);
+            const float2 s3 = *reinterpret_cast<const float2 *>(&Sf[(l + 3) * SCAN_COLS]);
 #pragma unroll
-            for (int i = 0; i < MAXR; ++i) {
-                const int m = g + 16 * i;
-                if (m < dk) {
-                    const float4 mm = *reinterpret_cast<const float4 *>(&Mf[m * dk + l]);
-                    acc[i].x += mm.x * s0.x;
-                    acc[i].y += mm.x * s0.y;
-                    acc[i].x += mm.y * s1.x;
-                    acc[i].y += mm.y * s1.y;
-                    acc[i].x += mm.z * s2.x;
-                    acc[i].y += mm.z * s2.y;
-                    acc[i].x += mm.w * s3.x;
-                    acc[i].y += mm.w * s3.y;
-                }
+            for (int i = 0; i < R; ++i) {
+                const float4 mm = *reinterpret_cast<const float4 *>(&Mf[(g + 16 * i) * DK + l]);
+                acc[i].x = fmaf(mm.x, s0.x, acc[i].x);
+                acc[i].y = fmaf(mm.x, s0.y, acc[i].y);
+                acc[i].x = fmaf(mm.y, s1.x, acc[i].x);
+                acc[i].y = fmaf(mm.y, s1.y, acc[i].y);
+                acc[i].x = fmaf(mm.z, s2.x, acc[i].x);
+                acc[i].y = fmaf(mm.z, s2.y, acc[i].y);
+                acc[i].x = fmaf(mm.w, s3.x, acc[i].x);
+                acc[i].y = fmaf(mm.w, s3.y, acc[i].y);
             }
         }
         if (kh == 1) {
 #pragma unroll
-            for (int i = 0; i < MAXR; ++i) reinterpret_cast<float2 *>(sRed)[i * 128 + t7] = acc[i];
+            for (int i = 0; i < R; ++i) sRed[i * 128 + t7] = acc[i];
         }
         __syncthreads();  // every read of sS and of this M buffer is done; partial sums are in sRed
         if (kh == 0) {
 #pragma unroll
-            for (int i = 0; i < MAXR; ++i) {
+            for (int i = 0; i < R; ++i) {
                 const int m = g + 16 * i;
-                if (m < dk) {
-                    const float2 o = reinterpret_cast<const float2 *>(sRed)[i * 128 + t7];
-                    sS[m * SCAN_COLS + ca] = (ca < ncol) ? acc[i].x + o.x : 0.f;
-                    sS[m * SCAN_COLS + cb] = (cb < ncol) ? acc[i].y + o.y : 0.f;
-                }
+                const float2 o = sRed[i * 128 + t7];
+                *reinterpret_cast<float2 *>(&sS[m * SCAN_COLS + ca]) = make_float2(acc[i].x + o.x, acc[i].y + o.y);
             }
         }
         __syncthreads();
     }
     if (p.S_out) {
-        for (int e = tid; e < dk * SCAN_COLS; e += NT) {
+        for (int e = tid; e < DK * SCAN_COLS; e += NT) {
             const int m = e >> 4, cc = e & 15;
-            if (cc < ncol) p.S_out[(chain * dv + c0 + cc) * (long long)dk + m] = sS[e];
+            if (cc < ncol) p.S_out[(chain * dv + c0 + cc) * (long long)DK + m] = sS[e];
         }
     }
     cp_async_wait_all();  // leave with no copy in flight
+}
+
+template <int DK>
+cudaError_t launch_scan_dk(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
+                           cudaStream_t s) {
+    const size_t sm = sizeof(float) * (2 * DK * DK + DK * SCAN_COLS) + sizeof(float2) * (DK / 16) * 128;
+    cudaError_t e = cudaFuncSetAttribute(k3_scan_simt<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e) return e;
+    k3_scan_simt<DK><<<dim3((unsigned)(p.B * p.H), (p.dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm, s>>>(p, Mb, Nb, Sig,
+                                                                                                      SigB);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
+                        cudaStream_t s) {
+    switch (p.dk) {
+        case 16: return launch_scan_dk<16>(p, Mb, Nb, Sig, SigB, s);
+        case 32: return launch_scan_dk<32>(p, Mb, Nb, Sig, SigB, s);
+        case 48: return launch_scan_dk<48>(p, Mb, Nb, Sig, SigB, s);
+        case 64: return launch_scan_dk<64>(p, Mb, Nb, Sig, SigB, s);
+        case 80: return launch_scan_dk<80>(p, Mb, Nb, Sig, SigB, s);
+        case 96: return launch_scan_dk<96>(p, Mb, Nb, Sig, SigB, s);
+        case 112: return launch_scan_dk<112>(p, Mb, Nb, Sig, SigB, s);
+        case 128: return launch_scan_dk<128>(p, Mb, Nb, Sig, SigB, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 // ---------------------------------------------------------------- k4 output
@@ -598,12 +612,10 @@ cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t
 
     const size_t sm1 = gsm + sizeof(float) * (2 * dk * RB + RB * RB + RB * nc);
     const size_t sm2 = gsm + sizeof(float) * (RB * 32 + RB * nc);
-    const size_t sm3 = sizeof(float) * (2 * dk * dk + dk * SCAN_COLS + 8 * 128 * 2);
     const size_t sm4 = gsm + sizeof(float) * (dk * dv + 3 * dk * RB + RB * RB + RB * dv);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k1_intra_simt<TIn, TG, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1))) return e;
     if ((e = cudaFuncSetAttribute(k2_transition_simt<TIn, TG, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2))) return e;
-    if ((e = cudaFuncSetAttribute(k3_scan_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3))) return e;
     if ((e = cudaFuncSetAttribute(k4_output_simt<TIn, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm4))) return e;
 
     if ((e = mark(ev, 0, s))) return e;
@@ -613,8 +625,7 @@ cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t
     k2_transition_simt<TIn, TG, float><<<dim3((unsigned)nfh, (dk + 31) / 32), NT, sm2, s>>>(p, X, Mb, Nb);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 2, s))) return e;
-    k3_scan_simt<<<dim3((unsigned)(p.B * p.H), (dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm3, s>>>(p, Mb, Nb, Sig,
-                                                                                             nullptr);
+    if ((e = launch_scan(p, Mb, Nb, Sig, nullptr, s))) return e;
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 3, s))) return e;
     k4_output_simt<TIn, TG><<<(unsigned)nfh, NT, sm4, s>>>(p, X, Sig, U);
@@ -666,12 +677,7 @@ cudaError_t simt_transition_bf16x(const Problem &p, const __nv_bfloat16 *X, floa
 
 cudaError_t simt_scan(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
                       cudaStream_t s) {
-    const size_t sm = sizeof(float) * (2 * p.dk * p.dk + p.dk * SCAN_COLS + 8 * 128 * 2);
-    cudaError_t e = cudaFuncSetAttribute(k3_scan_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e) return e;
-    k3_scan_simt<<<dim3((unsigned)(p.B * p.H), (p.dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm, s>>>(p, Mb, Nb, Sig,
-                                                                                                 SigB);
-    return cudaGetLastError();
+    return launch_scan(p, Mb, Nb, Sig, SigB, s);
 }
 
 cudaError_t simt_u_bf16x(const Problem &p, const __nv_bfloat16 *X, const float *Sig, __nv_bfloat16 *U,
