@@ -12,8 +12,9 @@
 // X_i goes to the [n_fh][L][d_v + d_k] bf16 workspace, from where later
 // blocks load it again (L2-resident) by TMA.
 //
-// Warp roles (192 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
-// warps 2-5 epilogue (one block row per thread).
+// Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
+// warps 2-9 epilogue (two warpgroups; one block row and one column half
+// per thread).
 //   TMEM: S tiles 2 x 64 cols, acc / X_i d_v + d_k cols.
 //   SMEM: K_i, K_j x2, X_j x2 (Y_i aliases them), P x2, T_ii.
 // Decay factors use a per-tile anchor a = G at the tile's last token:
@@ -24,7 +25,8 @@ namespace gdn {
 namespace tc {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kEpi = 256;                    // epilogue threads
 constexpr int JT = 64;                       // tokens per off-diagonal tile
 constexpr int KJ_SLAB = JT * 128;            // 64-row slab
 constexpr int XJ_BYTES = 4 * KJ_SLAB;        // X_j tile: 4 slabs of 64 columns
@@ -76,7 +78,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             uint32_t cnt = 1;
             if (i == KIEMPTY || i == SEMPTY0 || i == SEMPTY1 || i == PFULL0 || i == PFULL1 || i == YFULL ||
                 i == XDONE)
-                cnt = 128;
+                cnt = kEpi;
             sm100::mbar_init(&bars[i], cnt);
         }
         sm100::fence_barrier_init();
@@ -184,18 +186,23 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Two warpgroups: each thread owns one block row (TMEM lane quadrant =
+        // warp % 4) and one half of the columns -- 32 of the 64 columns of an
+        // off-diagonal tile, and in the diagonal step the Ub columns (half 0,
+        // which needs v) or the W columns (half 1, which needs k).
         const int et = threadIdx.x - 64;
         const int q4 = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
-        for (int s = et; s < L; s += 128) {
+        for (int s = et; s < L; s += kEpi) {
             const int tile_end = min((s / JT) * JT + JT - 1, L - 1);
             const float g = Gf[s];
             sG[s] = g;
             sCf[s] = __expf(Gf[tile_end] - g);  // <= 1: the tile's end is its most decayed token
         }
-        named_sync(1, 128);  // the only epilogue-wide barrier: before any bounded wait
+        named_sync(1, kEpi);  // the only epilogue-wide barrier: before any bounded wait
 
         bool ok = true;
         int n = 0;
@@ -206,12 +213,13 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             const long long t = f * L + row;
             const long long tok = ((long long)b * prm.T + t) * prm.H + h;
             const float be = valid ? prm.beta[tok] : 0.f;
-            // this row's values (bf16), read before the waits to hide their latency
+            // half 0 reads this row's values (bf16) before the waits to hide their latency
             uint4 vrow[16];
 #pragma unroll
             for (int c8 = 0; c8 < 16; ++c8)
-                vrow[c8] = (valid && c8 < dv / 8) ? *reinterpret_cast<const uint4 *>(prm.v + tok * dv + c8 * 8)
-                                                  : make_uint4(0, 0, 0, 0);
+                vrow[c8] = (half == 0 && valid && c8 < dv / 8)
+                               ? *reinterpret_cast<const uint4 *>(prm.v + tok * dv + c8 * 8)
+                               : make_uint4(0, 0, 0, 0);
 
             for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
                 const int sb = n & 1;
@@ -221,22 +229,19 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 sm100::tc_fence_after();
                 const float a = sG[jt * JT + JT - 1];
                 const float rf = valid ? -be * __expf(Gr - a) : 0.f;
-                const float *cf = sCf + jt * JT;
+                const float *cf = sCf + jt * JT + 32 * half;
                 unsigned char *pt = sP + sb * SLAB_BYTES;
-#pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
-                    float v[32];
-                    sm100::tmem_ld32(t_s0 + sb * JT + lane_off + c * 32, v);
-                    sm100::tmem_ld_wait();
+                float v[32];
+                sm100::tmem_ld32(t_s0 + sb * JT + lane_off + 32 * half, v);
+                sm100::tmem_ld_wait();
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c8 = c * 4 + u;  // 8-column chunk within the 64-column tile
-                        uint4 val = make_uint4(pack_bf16(rf * cf[c8 * 8 + 0] * v[u * 8 + 0], rf * cf[c8 * 8 + 1] * v[u * 8 + 1]),
-                                               pack_bf16(rf * cf[c8 * 8 + 2] * v[u * 8 + 2], rf * cf[c8 * 8 + 3] * v[u * 8 + 3]),
-                                               pack_bf16(rf * cf[c8 * 8 + 4] * v[u * 8 + 4], rf * cf[c8 * 8 + 5] * v[u * 8 + 5]),
-                                               pack_bf16(rf * cf[c8 * 8 + 6] * v[u * 8 + 6], rf * cf[c8 * 8 + 7] * v[u * 8 + 7]));
-                        *reinterpret_cast<uint4 *>(pt + r * 128 + ((c8 ^ (r & 7)) << 4)) = val;
-                    }
+                for (int u = 0; u < 4; ++u) {
+                    const int c8 = 4 * half + u;  // 8-column chunk within the 64-column tile
+                    uint4 val = make_uint4(pack_bf16(rf * cf[u * 8 + 0] * v[u * 8 + 0], rf * cf[u * 8 + 1] * v[u * 8 + 1]),
+                                           pack_bf16(rf * cf[u * 8 + 2] * v[u * 8 + 2], rf * cf[u * 8 + 3] * v[u * 8 + 3]),
+                                           pack_bf16(rf * cf[u * 8 + 4] * v[u * 8 + 4], rf * cf[u * 8 + 5] * v[u * 8 + 5]),
+                                           pack_bf16(rf * cf[u * 8 + 6] * v[u * 8 + 6], rf * cf[u * 8 + 7] * v[u * 8 + 7]));
+                    *reinterpret_cast<uint4 *>(pt + r * 128 + ((c8 ^ (r & 7)) << 4)) = val;
                 }
                 sm100::tc_fence_before();
                 sm100::mbar_arrive(&bars[SEMPTY0 + sb]);
@@ -248,78 +253,90 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             ok = sm100::mbar_wait(&bars[ACCFULL], i & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
-            const float rk = be * __expf(Gr);  // beta_r e^{G_r}
+            auto store_y = [&](int c, const float (&y)[8]) {
+                const uint4 val = valid ? make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]),
+                                                     pack_bf16(y[4], y[5]), pack_bf16(y[6], y[7]))
+                                        : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(sY + (c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4)) = val;
+            };
+            if (half == 0) {  // Ub columns: beta_r v_r + acc
 #pragma unroll
-            for (int c0 = 0; c0 < 256; c0 += 32) {
-                if (c0 >= nc) break;
-                float acc[32];
-                if (i > 0) {
-                    sm100::tmem_ld32(t_acc + lane_off + c0, acc);
-                    sm100::tmem_ld_wait();
-                } else {
+                for (int j = 0; j < 8; ++j) {
+                    const int c16 = 16 * j;
+                    if (c16 >= dv) break;
+                    float acc[16];
+                    if (i > 0) {
+                        sm100::tmem_ld16(t_acc + lane_off + c16, acc);
+                        sm100::tmem_ld_wait();
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-                }
+                        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+                    }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + u * 8;
-                    if (c >= nc) break;
-                    float y[8];
-                    if (c < dv) {
-                        const __nv_bfloat162 *vb = reinterpret_cast<const __nv_bfloat162 *>(&vrow[c >> 3]);
+                    for (int u = 0; u < 2; ++u) {
+                        const __nv_bfloat162 *vb = reinterpret_cast<const __nv_bfloat162 *>(&vrow[2 * j + u]);
+                        float y[8];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 fv = __bfloat1622float2(vb[e]);
-                            y[2 * e] = be * fv.x;
-                            y[2 * e + 1] = be * fv.y;
+                            y[2 * e] = be * fv.x + acc[u * 8 + 2 * e];
+                            y[2 * e + 1] = be * fv.y + acc[u * 8 + 2 * e + 1];
                         }
+                        store_y(c16 + 8 * u, y);
+                    }
+                }
+            } else {  // W columns: beta_r e^{G_r} k_r + acc
+                const float rk = be * __expf(Gr);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int kc16 = 16 * j;
+                    if (kc16 >= dk) break;
+                    float acc[16];
+                    if (i > 0) {
+                        sm100::tmem_ld16(t_acc + lane_off + dv + kc16, acc);
+                        sm100::tmem_ld_wait();
                     } else {
-                        const int kc = c - dv;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int kc = kc16 + 8 * u;
                         const uint4 kv = *reinterpret_cast<const uint4 *>(
                             sKi + (kc >> 6) * SLAB_BYTES + r * 128 + ((((kc & 63) >> 3) ^ (r & 7)) << 4));
                         const __nv_bfloat162 *kb = reinterpret_cast<const __nv_bfloat162 *>(&kv);
+                        float y[8];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 fk = __bfloat1622float2(kb[e]);
-                            y[2 * e] = rk * fk.x;
-                            y[2 * e + 1] = rk * fk.y;
+                            y[2 * e] = rk * fk.x + acc[u * 8 + 2 * e];
+                            y[2 * e + 1] = rk * fk.y + acc[u * 8 + 2 * e + 1];
                         }
+                        store_y(dv + kc, y);
                     }
-                    uint4 val;
-                    if (valid) {
-                        val = make_uint4(pack_bf16(y[0] + acc[u * 8 + 0], y[1] + acc[u * 8 + 1]),
-                                         pack_bf16(y[2] + acc[u * 8 + 2], y[3] + acc[u * 8 + 3]),
-                                         pack_bf16(y[4] + acc[u * 8 + 4], y[5] + acc[u * 8 + 5]),
-                                         pack_bf16(y[6] + acc[u * 8 + 6], y[7] + acc[u * 8 + 7]));
-                    } else {
-                        val = make_uint4(0, 0, 0, 0);
-                    }
-                    *reinterpret_cast<uint4 *>(sY + (c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4)) =
-                        val;
                 }
             }
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();
             sm100::mbar_arrive(&bars[YFULL]);
             sm100::mbar_arrive(&bars[KIEMPTY]);
-            // ---- X_i = T_ii Y_i  -> global
+            // ---- X_i = T_ii Y_i  -> global (half 0 the Ub columns, half 1 the W columns)
             ok = sm100::mbar_wait(&bars[XFULL], i & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
             __nv_bfloat16 *xrow = prm.X + (fh * (long long)L + row) * nc;
-            for (int c0 = 0; c0 < nc; c0 += 32) {
-                float x[32];
-                sm100::tmem_ld32(t_acc + lane_off + c0, x);
+            const int c_lo = half ? dv : 0, c_hi = half ? nc : dv;
+            for (int c16 = c_lo; c16 < c_hi; c16 += 16) {
+                float x[16];
+                sm100::tmem_ld16(t_acc + lane_off + c16, x);
                 sm100::tmem_ld_wait();
                 if (valid) {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c = c0 + u * 8;
-                        if (c >= nc) break;
-                        uint4 val = make_uint4(pack_bf16(x[u * 8 + 0], x[u * 8 + 1]), pack_bf16(x[u * 8 + 2], x[u * 8 + 3]),
-                                               pack_bf16(x[u * 8 + 4], x[u * 8 + 5]), pack_bf16(x[u * 8 + 6], x[u * 8 + 7]));
-                        *reinterpret_cast<uint4 *>(xrow + c) = val;
-                    }
+                    reinterpret_cast<uint4 *>(xrow + c16)[0] =
+                        make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                                   pack_bf16(x[6], x[7]));
+                    reinterpret_cast<uint4 *>(xrow + c16)[1] =
+                        make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]), pack_bf16(x[12], x[13]),
+                                   pack_bf16(x[14], x[15]));
                 }
             }
             fence_proxy_async_global();

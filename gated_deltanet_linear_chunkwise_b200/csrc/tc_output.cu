@@ -9,12 +9,14 @@
 // Persistent kernel: one CTA per SM walks (frame-head, block) items in
 // frame-head order (neighbouring CTAs share a frame's K and U tiles in L2),
 // with TMEM and barriers set up once.
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues tcgen05.mma from one thread, warps 2-5 are the epilogue (one tile
-// row per thread, TMEM lane quadrant = warp % 4).
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues tcgen05.mma from one thread, warps 2-9 are the epilogue: two
+// warpgroups, each thread owning one tile row (TMEM lane quadrant =
+// warp % 4) and one half of the tile's columns.
 //   TMEM: two S/P buffers (128 columns each) and two O buffers (128 each).
-//         The epilogue turns S (fp32) into P (bf16) in place and the
-//         O += P U product reads P straight from tensor memory.
+//         The epilogue turns S (fp32) into P (bf16) in place -- each
+//         column half into the first 32 TMEM columns of its own range --
+//         and the O += P U product reads P straight from tensor memory.
 //   SMEM: Q_I double buffer; a 2-stage ring of (K_J, U_J, G_J, cf_J) tiles.
 // The state term is a pseudo-tile in front of the J tiles: the epilogue
 // writes Q~ = diag(e^G) Q_I into an S/P buffer and the ring delivers Sig
@@ -28,7 +30,8 @@ namespace gdn {
 namespace tc {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kEpi = 256;  // epilogue threads
 constexpr int GC_BYTES = 2 * BM * 4;  // G and cf of one 128-column tile
 
 struct Smem {
@@ -65,7 +68,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) {
             uint32_t cnt = 1;
-            if (i == PFULL0 || i == PFULL1 || i == OEMPTY0 || i == OEMPTY1) cnt = 128;
+            if (i == PFULL0 || i == PFULL1 || i == OEMPTY0 || i == OEMPTY1) cnt = kEpi;
             sm100::mbar_init(&bars[i], cnt);
         }
         sm100::fence_barrier_init();
@@ -174,8 +177,10 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     if (!sm100::mbar_wait(&bars[PFULL0 + psb], (psc >> 1) & 1, err)) return false;
                     sm100::tc_fence_after();
                     const unsigned char *u = sU + pst * 2 * SLAB_BYTES;
+                    // P columns k = 0..63 sit in TMEM columns 0..31, k = 64..127 in columns 64..95
                     for (int ks = 0; ks < BM / 16; ++ks)
-                        sm100::mma_bf16_ts(t_o, t_s0 + psb * 128 + ks * 8, desc_mnmajor(u, ks, BM), id_o, 1u);
+                        sm100::mma_bf16_ts(t_o, t_s0 + psb * 128 + ks * 8 + (ks >> 2) * 32, desc_mnmajor(u, ks, BM),
+                                           id_o, 1u);
                     sm100::mma_commit(&bars[SFREE0 + psb]);
                     sm100::mma_commit(&bars[REMPTY0 + pst]);
                     return true;
@@ -210,6 +215,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // so one item's O drains while the tensor cores work on the next.
         const int q4 = warp & 3;                  // TMEM lane quadrant
         const int r = q4 * 32 + lane;             // tile row owned by this thread
+        const int half = (warp - 2) >> 2;         // which half of the tile's columns
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         int sc = 0, n = 0;
         struct Item {
@@ -259,7 +265,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (!sm100::mbar_wait(&bars[QFULL0 + qb], (t >> 1) & 1, err)) return false;
             sm100::tc_fence_after();
             const float eg = it.valid ? __expf(it.Gr) : 0.f;
-            for (int c16 = 0; c16 * 32 < dk; ++c16) {  // 32 bf16 -> 16 TMEM columns per group
+            for (int c16 = half; c16 * 32 < dk; c16 += 2) {  // 32 bf16 -> 16 TMEM columns per group
                 uint32_t pk[16];
                 q_group(qb, c16, eg, pk);
                 sm100::tmem_st16(t_s0 + sb * 128 + lane_off + c16 * 16, pk);
@@ -279,16 +285,15 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 if (!sm100::mbar_wait(&bars[RFULL0 + st], (n >> 1) & 1, err)) return false;  // this tile's G, cf
                 sm100::tc_fence_after();
                 const float *gJ = sGC + st * 2 * BM, *cfJ = gJ + BM;
-                const float rf0 = it.valid ? __expf(it.Gr - gJ[63]) : 0.f;
-                const float rf1 = it.valid ? __expf(it.Gr - gJ[127]) : 0.f;
+                // this half's 64 columns share one 64-token anchor
+                const float rf = it.valid ? __expf(it.Gr - gJ[64 * half + 63]) : 0.f;
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 2 * half; c < 2 * half + 2; ++c) {
                     float v[32];
                     sm100::tmem_ld32(t_s0 + sb * 128 + lane_off + c * 32, v);
                     sm100::tmem_ld_wait();
                     uint32_t pk[16];
                     if (!diag) {
-                        const float rf = c < 2 ? rf0 : rf1;
 #pragma unroll
                         for (int e = 0; e < 32; e += 2)
                             pk[e >> 1] = pack_bf16(v[e] * rf * cfJ[c * 32 + e], v[e + 1] * rf * cfJ[c * 32 + e + 1]);
@@ -301,8 +306,9 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                             pk[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
                         }
                     }
-                    // P columns [16c, 16c+16) overwrite S columns that have already been read
-                    sm100::tmem_st16(t_s0 + sb * 128 + lane_off + c * 16, pk);
+                    // P (bf16 pairs) of this half's 64 columns goes to TMEM columns
+                    // [64 half, 64 half + 32): S columns this half has already read
+                    sm100::tmem_st16(t_s0 + sb * 128 + lane_off + 64 * half + (c - 2 * half) * 16, pk);
                 }
                 sm100::tmem_st_wait();
                 sm100::tc_fence_before();
@@ -316,7 +322,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             sm100::tc_fence_after();
             const long long tt = it.f * L + it.row;
             __nv_bfloat16 *o = (__nv_bfloat16 *)prm.o + ((((long long)it.b * prm.T + tt) * prm.H + it.h) * dv);
-            for (int c = 0; c < dv; c += 16) {
+            for (int c = 16 * half; c < dv; c += 32) {
                 float acc[16];
                 sm100::tmem_ld16(t_o0 + ob * 128 + lane_off + c, acc);
                 sm100::tmem_ld_wait();
