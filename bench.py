@@ -33,8 +33,36 @@ WORKLOAD = "minute"
 # total F_alg = L^2 (3 d_k + 2 d_v) + 6 L d_k d_v
 
 
-def flops_intra(L, dk, dv):
-    return L * L * (2 * dk + dv)
+def kernel_work(L, dk, dv, BM=128):
+    """Algorithmic work of each kernel per frame-head: (FLOPs, bytes).
+    Matrix products count 2 FLOPs per multiply-add over the entries the
+    method needs (lower triangles only); bytes count each operand once.
+      gates        G and cf of every token: read alpha, write G, cf (fp32)
+      diag_inverse Gram of each 128-row diagonal block (lower half) and its
+                   unit triangular inverse (n^3 / 3)
+      intra        off-diagonal S = K_i K_j^T and P X_j over the 128-column
+                   blocks before each row's block, plus the lower-triangular
+                   T_ii Y_i
+      transition   Kt^T [Ub | W]
+      scan         Sig M + N per frame (fp32 M, N in; fp32 + bf16 Sig out)
+      u            W Sig
+      output       masked Q K^T (lower triangle incl. diagonal), its product
+                   with U, and Q Sig
+    """
+    nc = dk + dv
+    off = sum(BM * (r // BM) for r in range(L))
+    tri = sum((r % BM) + 1 for r in range(L))
+    nblk = (L + BM - 1) // BM
+    blk = [min(BM, L - i * BM) for i in range(nblk)]
+    return {
+        "gates": (0, 12 * L),
+        "diag_inverse": (sum(n * n * dk + n ** 3 // 3 for n in blk), 2 * L * dk + 2 * L * BM),
+        "intra": (2 * off * (dk + nc) + 2 * tri * nc, 2 * L * (dk + dv) + 2 * L * nc),
+        "transition": (2 * L * dk * nc, 2 * L * dk + 2 * L * nc + 4 * dk * nc),
+        "scan": (2 * dk * dk * dv, 4 * dk * dk + 4 * dk * dv + 6 * dk * dv),
+        "u": (2 * L * dk * dv, 2 * L * dk + 2 * dk * dv + 4 * L * dv),
+        "output": (tri * 2 * (dk + dv) + 2 * L * dk * dv, 2 * L * (dk + dk + dv + dv) + 2 * dk * dv),
+    }
 
 
 def flops_total(L, dk, dv):
@@ -242,20 +270,18 @@ def main():
             stage_sum[i] += arr[i] / reps
     dominant = max(range(NUM_STAGES), key=lambda i: stage_sum[i])
 
-    # end to end through the public call with host buffers: pinned host inputs
-    # copied in, the pass, the output (and final state) copied back, every step
-    h = {k: (None if t is None else t.pin_memory()) for k, t in inp.items() if t is not None}
+    # end to end through the host-buffer entry point gdn_fwd_host: every step
+    # copies the pinned host inputs in, runs the pass, copies o and the final
+    # state back and synchronises
+    h = {k: t.contiguous().pin_memory() for k, t in inp.items() if t is not None}
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     S_host = torch.empty(S_out.shape, dtype=S_out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in h.values())
     d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
 
     def e2e_step():
-        for k, t in h.items():
-            d[k].copy_(t, non_blocking=True)
-        step()
-        o_host.copy_(o, non_blocking=True)
-        S_host.copy_(S_out, non_blocking=True)
+        g.gdn_fwd_host(h["q"], h["k"], h["v"], h["alpha"], h["beta"], L, h.get("S_in"), S_out=S_host,
+                       o=o_host, stream=stream, device=dev)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -276,10 +302,15 @@ def main():
     pk = peaks()
     nfh = B * H * w.frames
     if rank == 0:
-        f_dom = {0: flops_intra(L, dk, dv), 3: L * L * (dk + dv) + 4 * L * dk * dv,
-                 1: 4 * L * dk * dv, 2: 2 * dk * dk * dv}[dominant] * nfh
+        work = kernel_work(L, dk, dv)
+        f_dom, b_dom = (x * nfh for x in work[STAGES[dominant]])
         dom_ms = stage_sum[dominant]
-        achieved = f_dom / (dom_ms * 1e-3) / 1e12
+        # a kernel whose FLOP:byte ratio is below the ridge point is bandwidth bound
+        tensor_bound = f_dom / max(b_dom, 1) > pk["bf16_tflops"] / pk["hbm_gbs"] * 1e3
+        if tensor_bound:
+            achieved, peak, unit = f_dom / (dom_ms * 1e-3) / 1e12, pk["bf16_tflops"], "TFLOP/s"
+        else:
+            achieved, peak, unit = b_dom / (dom_ms * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s"
         f_all = flops_total(L, dk, dv) * nfh
         tokens = B * T * world
         line = {
@@ -297,9 +328,11 @@ def main():
                        "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
                        "gate_regime": args.regime,
                        "l2": "no flush: inputs 1.4 GB per step exceed the 126 MB L2"},
-            "roofline": {"bound": "tensor", "kernel": STAGES[dominant], "achieved": achieved,
-                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                         "traffic": None, "peak_source": pk["source"] + " bf16 burst",
+            "roofline": {"bound": "tensor" if tensor_bound else "hbm", "kernel": STAGES[dominant],
+                         "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                         "traffic": None,
+                         "peak_source": pk["source"] + (" bf16 burst" if tensor_bound else " copy bandwidth"),
+                         "per_launch": {"flops": f_dom, "bytes": b_dom, "ms": dom_ms},
                          "stage_ms": dict(zip(STAGES, stage_sum))},
             "path_roofline": {"flops": f_all, "bytes": bytes_alg(B, T, H, dk, dv),
                               "achieved_tflops": f_all / (ms_step * 1e-3) / 1e12,
@@ -308,6 +341,7 @@ def main():
                                                         if pk["bf16_tflops_sustained"] else None)},
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
+            # one kernel per stage: gates, diagonal inverses, intra, transition, scan, U, output
             "gpu_launches": NUM_STAGES * args.steps,
             "clocks": clk.summary(),
         }

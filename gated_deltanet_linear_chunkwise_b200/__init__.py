@@ -5,8 +5,8 @@ The computation lives in ``libgdn_b200.so`` (C ABI declared in
 the named synthetic workloads.  Importing the package does not load the
 library; the first call does, and fails loudly if it has not been built.
 """
-from .binding import (GdnError, bidirectional, gdn_fwd, gdn_step, last_error, load_library,
-                      workspace_bytes)
+from .binding import (GdnError, bidirectional, gdn_fwd, gdn_fwd_host, gdn_step, last_error,
+                      load_library, workspace_bytes)
 
-__all__ = ["GdnError", "bidirectional", "gdn_fwd", "gdn_step", "last_error", "load_library",
-           "workspace_bytes"]
+__all__ = ["GdnError", "bidirectional", "gdn_fwd", "gdn_fwd_host", "gdn_step", "last_error",
+           "load_library", "workspace_bytes"]

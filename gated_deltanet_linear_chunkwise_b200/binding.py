@@ -22,7 +22,7 @@ STATUS = {
 }
 
 # every symbol include/gdn.h declares
-EXPORTS = ("gdn_fwd", "gdn_fwd_f32", "gdn_step", "gdn_step_f32", "gdn_fwd_ex",
+EXPORTS = ("gdn_fwd", "gdn_fwd_f32", "gdn_step", "gdn_step_f32", "gdn_fwd_ex", "gdn_fwd_host",
            "gdn_workspace_bytes", "gdn_status_string", "gdn_last_error", "gdn_version")
 
 
@@ -48,8 +48,8 @@ class GdnArgs(ctypes.Structure):
         ("stream", ctypes.c_void_p), ("stage_ms", ctypes.c_void_p),
     ]
 
-NUM_STAGES = 4
-STAGES = ("intra", "transition", "scan", "output")
+NUM_STAGES = 7
+STAGES = ("gates", "diag_inverse", "intra", "transition", "scan", "u", "output")
 
 
 _lib = None
@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH):
         fn = getattr(lib, name)
         fn.argtypes = fwd_sig
         fn.restype = I
+    lib.gdn_fwd_host.argtypes = [I] + fwd_sig
+    lib.gdn_fwd_host.restype = I
     lib.gdn_fwd_ex.argtypes = [ctypes.POINTER(GdnArgs)]
     lib.gdn_fwd_ex.restype = I
     lib.gdn_workspace_bytes.argtypes = [I, I, LL, I, I, I, I]
@@ -158,6 +160,36 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     if stage_ms is not None:  # a ctypes float array of NUM_STAGES; the call synchronises
         a.stage_ms = ctypes.cast(stage_ms, ctypes.c_void_p)
     check(load_library().gdn_fwd_ex(ctypes.byref(a)))
+    return o, S_out
+
+
+def gdn_fwd_host(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
+                 return_state=False, stream=None, device=None):
+    """The whole pass from HOST (CPU) tensors through ``gdn_fwd_host``: the
+    library copies the inputs to the GPU, runs the pass, copies o (and the
+    state) back and synchronises.  Pinned tensors copy fastest.  Same shapes
+    and dtypes as ``gdn_fwd``; returns (o, S_out or None) on the host."""
+    import torch
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta), ("S_in", S_in),
+                    ("S_out", S_out), ("o", o)):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise GdnError(1, "%s must be a contiguous host tensor" % name)
+    if q.dtype != k.dtype or q.dtype != v.dtype or q.dtype not in (torch.bfloat16, torch.float32):
+        raise GdnError(1, "q/k/v must share one dtype, bf16 or fp32")
+    if alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise GdnError(1, "alpha and beta must be fp32")
+    if o is None:
+        o = torch.empty((B, T, H, d_v), dtype=q.dtype)
+    if S_out is None and return_state:
+        S_out = torch.empty((B, H, d_v, d_k), dtype=torch.float32)
+    dt = GDN_DTYPE_BF16 if q.dtype == torch.bfloat16 else GDN_DTYPE_F32
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    check(load_library().gdn_fwd_host(dt, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S_in),
+                                      _ptr(S_out), _ptr(o), B, H, T, int(frame_len), d_k, d_v,
+                                      _stream_handle(stream, device)))
     return o, S_out
 
 

@@ -316,6 +316,67 @@ int gdn_fwd_ex(const gdn_args *a) {
     return run(*a);
 }
 
+int gdn_fwd_host(int dtype, const void *q, const void *k, const void *v, const float *alpha, const float *beta,
+                 const float *S_in, float *S_out, void *o, int B, int H, long long T, int frame_len, int d_k,
+                 int d_v, gdn_stream_t stream) {
+    try {
+        g_err[0] = '\0';
+        gdn_args a = make_args(dtype, q, k, v, alpha, beta, S_in, S_out, o, B, H, T, frame_len, d_k, d_v, stream);
+        int st = validate_sizes(a);
+        if (st != GDN_OK) return st;
+        if (B == 0 || H == 0) return GDN_OK;
+        if (T > 0 && (!q || !k || !v || !alpha || !beta || !o)) {
+            set_err("q, k, v, alpha, beta and o are required (one is NULL)");
+            return GDN_ERR_INVALID_ARG;
+        }
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        const size_t es = dtype == GDN_DTYPE_BF16 ? 2 : 4;
+        const size_t ntok = (size_t)B * T * H;
+        const size_t nq = ntok * d_k * es, nv = ntok * d_v * es, ng = ntok * 4;
+        const size_t ns = (size_t)B * H * d_v * d_k * 4;
+        // one device block: q | k | v | alpha | beta | S_in | S_out | o | workspace
+        const size_t sz[8] = {nq, nq, nv, ng, ng, S_in ? ns : 0, S_out ? ns : 0, nv};
+        size_t off[9];
+        off[0] = 0;
+        for (int i = 0; i < 8; ++i) off[i + 1] = off[i] + ((sz[i] + 255) & ~(size_t)255);
+        const size_t wsb = gdn_workspace_bytes(B, H, T, frame_len, d_k, d_v, dtype);
+        char *dev = nullptr;
+        cudaError_t e = cudaMallocAsync((void **)&dev, off[8] + wsb, s);
+        if (e != cudaSuccess || !dev) {
+            cudaGetLastError();
+            set_err("cudaMallocAsync(%zu bytes) failed: %s", off[8] + wsb, cudaGetErrorString(e));
+            return GDN_ERR_NO_MEMORY;
+        }
+        const void *hin[6] = {q, k, v, alpha, beta, S_in};
+        for (int i = 0; i < 6 && e == cudaSuccess; ++i)
+            if (sz[i]) e = cudaMemcpyAsync(dev + off[i], hin[i], sz[i], cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) {
+            cudaFreeAsync(dev, s);
+            return cuda_fail(e, "host-to-device copy");
+        }
+        gdn_args d = make_args(dtype, dev + off[0], dev + off[1], dev + off[2], (const float *)(dev + off[3]),
+                               (const float *)(dev + off[4]), S_in ? (const float *)(dev + off[5]) : nullptr,
+                               S_out ? (float *)(dev + off[6]) : nullptr, dev + off[7], B, H, T, frame_len, d_k,
+                               d_v, stream);
+        d.workspace = wsb ? dev + off[8] : nullptr;
+        d.workspace_bytes = wsb;
+        st = run(d);
+        if (st == GDN_OK) {
+            e = cudaMemcpyAsync(o, dev + off[7], sz[7], cudaMemcpyDeviceToHost, s);
+            if (e == cudaSuccess && S_out) e = cudaMemcpyAsync(S_out, dev + off[6], ns, cudaMemcpyDeviceToHost, s);
+        }
+        cudaError_t e2 = cudaFreeAsync(dev, s);
+        cudaError_t e3 = cudaStreamSynchronize(s);
+        if (st != GDN_OK) return st;
+        if (e == cudaSuccess) e = e2 ? e2 : e3;
+        if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+        return GDN_OK;
+    } catch (...) {
+        set_err("internal error (exception caught at the ABI boundary)");
+        return GDN_ERR_CUDA;
+    }
+}
+
 size_t gdn_workspace_bytes(int B, int H, long long T, int frame_len, int d_k, int d_v, int dtype) {
     gdn_args a = make_args(dtype, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                            B, H, T, frame_len, d_k, d_v, nullptr);

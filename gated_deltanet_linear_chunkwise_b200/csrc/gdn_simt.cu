@@ -618,19 +618,21 @@ cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t
     if ((e = cudaFuncSetAttribute(k2_transition_simt<TIn, TG, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2))) return e;
     if ((e = cudaFuncSetAttribute(k4_output_simt<TIn, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm4))) return e;
 
-    if ((e = mark(ev, 0, s))) return e;
+    // stages 0, 1 (gates, diagonal inverses) are folded into the intra kernel, 5 (U) into the output
+    for (int i = 0; i <= 2; ++i)
+        if ((e = mark(ev, i, s))) return e;
     k1_intra_simt<TIn, TG, float><<<(unsigned)nfh, NT, sm1, s>>>(p, X);
     if ((e = cudaGetLastError())) return e;
-    if ((e = mark(ev, 1, s))) return e;
+    if ((e = mark(ev, 3, s))) return e;
     k2_transition_simt<TIn, TG, float><<<dim3((unsigned)nfh, (dk + 31) / 32), NT, sm2, s>>>(p, X, Mb, Nb);
     if ((e = cudaGetLastError())) return e;
-    if ((e = mark(ev, 2, s))) return e;
+    if ((e = mark(ev, 4, s))) return e;
     if ((e = launch_scan(p, Mb, Nb, Sig, nullptr, s))) return e;
     if ((e = cudaGetLastError())) return e;
-    if ((e = mark(ev, 3, s))) return e;
+    if ((e = mark(ev, 5, s)) || (e = mark(ev, 6, s))) return e;
     k4_output_simt<TIn, TG><<<(unsigned)nfh, NT, sm4, s>>>(p, X, Sig, U);
     if ((e = cudaGetLastError())) return e;
-    return mark(ev, 4, s);
+    return mark(ev, 7, s);
 }
 
 }  // namespace

@@ -82,14 +82,14 @@ bool map_tokens(CUtensorMap *m, const void *x, const Problem &p, int d, int box_
     return make_map(m, x, 4, dims, strides, box);
 }
 
-// fp32 rows [n_fh][stride] seen as 2-D (len, n_fh), boxes of 128 elements, no swizzle;
+// fp32 rows [n_fh][stride] seen as 2-D (len, n_fh), boxes of `box` elements, no swizzle;
 // elements past `len` read as zeros.
-bool map_f32_rows(CUtensorMap *m, const float *x, long long nfh, int len, int stride) {
+bool map_f32_rows(CUtensorMap *m, const float *x, long long nfh, int len, int stride, int box_len) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)len, (cuuint64_t)nfh};
     const cuuint64_t strides[1] = {(cuuint64_t)stride * 4};
-    const cuuint32_t box[2] = {128, 1};
+    const cuuint32_t box[2] = {(cuuint32_t)box_len, 1};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(x), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -154,12 +154,13 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
 
     __nv_bfloat16 *Tinv = (__nv_bfloat16 *)(base + lay.Tinv);
     const int nc = p.dk + p.dv;
-    CUtensorMap tm_q, tm_k, tm_u, tm_sig, tm_k64, tm_x, tm_t, tm_x128, tm_g, tm_cf;
+    CUtensorMap tm_q, tm_k, tm_u64, tm_sig, tm_k64, tm_x, tm_t, tm_x128, tm_g, tm_cf;
     if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
-        !map_rows(&tm_u, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
+        !map_rows(&tm_u64, U, nfh, p.L, p.dv, 64) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
         !map_tokens(&tm_k64, p.k, p, p.dk, 64) || !map_rows(&tm_x, X, nfh, p.L, nc, 64) ||
         !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128) || !map_rows(&tm_x128, X, nfh, p.L, nc, 128) ||
-        !map_f32_rows(&tm_g, G, nfh, p.L, cf_stride(p.L)) || !map_f32_rows(&tm_cf, CF, nfh, p.L, cf_stride(p.L)))
+        !map_f32_rows(&tm_g, G, nfh, p.L, cf_stride(p.L), 64) ||
+        !map_f32_rows(&tm_cf, CF, nfh, p.L, cf_stride(p.L), 64))
         return cudaErrorInvalidValue;
 
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
@@ -170,26 +171,29 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     if ((e = mark(ev, 0, s))) return e;
     gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF);
     if ((e = cudaGetLastError())) return e;
+    if ((e = mark(ev, 1, s))) return e;
     if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
                                      nfh, s)))
         return e;
+    if ((e = mark(ev, 2, s))) return e;
     tc::IntraParams ip;
     ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.X = X;
     ip.L = p.L; ip.dk = p.dk; ip.dv = p.dv; ip.H = p.H; ip.nblk = nblk;
     ip.F = p.F; ip.T = p.T; ip.err = err;
-    if ((e = tc::launch_intra_tc(tm_k64, tm_x, tm_t, ip, nfh, s))) return e;
-    if ((e = mark(ev, 1, s))) return e;
+    if ((e = tc::launch_intra_tc(tm_k64, tm_x, tm_t, tm_g, tm_cf, ip, nfh, s))) return e;
+    if ((e = mark(ev, 3, s))) return e;
     tc::TransParams tp;
     tp.G = G; tp.M = Mb; tp.N = Nb;
     tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
     if ((e = tc::launch_transition_tc(tm_k, tm_x128, tp, nfh, s))) return e;
-    if ((e = mark(ev, 2, s))) return e;
+    if ((e = mark(ev, 4, s))) return e;
     if ((e = simt_scan(p, Mb, Nb, Sig, SigB, s))) return e;
-    if ((e = mark(ev, 3, s))) return e;
+    if ((e = mark(ev, 5, s))) return e;
     tc::UParams up;
     up.X = X; up.U = U;
     up.L = p.L; up.dk = p.dk; up.dv = p.dv; up.nblk = nblk; up.err = err;
     if ((e = tc::launch_u_tc(tm_x128, tm_sig, up, nfh, s))) return e;
+    if ((e = mark(ev, 6, s))) return e;
 
     tc::OutParams op;
     op.G = G;
@@ -201,8 +205,8 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     op.err = err;
     int dev = 0, num_sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u, tm_sig, tm_g, tm_cf, op, num_sms, s))) return e;
-    return mark(ev, 4, s);
+    if ((e = tc::launch_output_tc(tm_q, tm_k64, tm_u64, tm_sig, tm_g, tm_cf, op, num_sms, s))) return e;
+    return mark(ev, 7, s);
 }
 
 int *tc_error_word(const Problem &p, void *ws) { return (int *)((char *)ws + tc_layout(p).err); }

@@ -15,8 +15,11 @@
 // Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
 // warps 2-9 epilogue (two warpgroups; one block row and one column half
 // per thread).
-//   TMEM: S tiles 2 x 64 cols, acc / X_i d_v + d_k cols.
-//   SMEM: K_i, K_j x2, X_j x2 (Y_i aliases them), P x2, T_ii.
+//   TMEM: four S/P buffers (64 columns each; the epilogue turns S into the
+//         bf16 P in place and acc += P X_j reads P from tensor memory) and
+//         acc / X_i (d_v + d_k columns).
+//   SMEM: K_i, T_ii, and a 3-deep ring of (K_j, X_j, G_j, cf_j) tiles; Y_i
+//         aliases the first two ring slots during the diagonal step.
 // Decay factors use a per-tile anchor a = G at the tile's last token:
 // e^{G_r - G_s} = e^{G_r - a} e^{a - G_s}, both <= 1.
 #include "tc_common.cuh"
@@ -28,20 +31,26 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kEpi = 256;                    // epilogue threads
 constexpr int JT = 64;                       // tokens per off-diagonal tile
+constexpr int NSLOT = 3;                     // ring depth
+constexpr int NSB = 4;                       // S/P buffers in TMEM
 constexpr int KJ_SLAB = JT * 128;            // 64-row slab
-constexpr int XJ_BYTES = 4 * KJ_SLAB;        // X_j tile: 4 slabs of 64 columns
+constexpr int SLOT_BYTES = 6 * KJ_SLAB;      // K_j (2 slabs) + X_j (4 slabs)
+constexpr int GC_BYTES = 2 * JT * 4;         // G and cf of one tile
 
 struct Smem {
     static constexpr uint32_t KI = 0;                          // 2 slabs x 128 rows
-    static constexpr uint32_t KJ = KI + 2 * SLAB_BYTES;        // 2 stages x 2 slabs x 64 rows
-    static constexpr uint32_t XJ = KJ + 4 * KJ_SLAB;           // 2 stages x 32 KB; Y_i (64 KB) aliases
-    static constexpr uint32_t P = XJ + 2 * XJ_BYTES;           // 2 stages x 1 slab x 128 rows
-    static constexpr uint32_t T = P + 2 * SLAB_BYTES;          // 2 slabs x 128 rows
-    static constexpr uint32_t F = T + 2 * SLAB_BYTES;          // floats: G[L], cf[L]
+    static constexpr uint32_t T = KI + 2 * SLAB_BYTES;         // 2 slabs x 128 rows
+    static constexpr uint32_t RING = T + 2 * SLAB_BYTES;       // NSLOT x 48 KB; Y_i (64 KB) aliases the start
+    static constexpr uint32_t GC = RING + NSLOT * SLOT_BYTES;  // NSLOT x (G[64], cf[64])
+    static constexpr uint32_t END = GC + NSLOT * GC_BYTES;
 };
+static_assert(2 * SLOT_BYTES >= 4 * SLAB_BYTES, "Y_i must fit in the first two ring slots");
 
-enum Bar { KIFULL, KIEMPTY, TFULL, TEMPTY, KXFULL0, KXFULL1, KXEMPTY0, KXEMPTY1, SFULL0, SFULL1, SEMPTY0,
-           SEMPTY1, PFULL0, PFULL1, PEMPTY0, PEMPTY1, ACCFULL, YFULL, XFULL, XDONE, NBAR };
+enum Bar {
+    KIFULL = 0, KIEMPTY, TFULL, TEMPTY, ACCFULL, YFULL, XFULL, XDONE,
+    KXFULL, KXEMPTY = KXFULL + NSLOT, SFULL = KXEMPTY + NSLOT, SFREE = SFULL + NSB, PFULL = SFREE + NSB,
+    NBAR = PFULL + NSB
+};
 
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -49,7 +58,8 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_x,
-           const __grid_constant__ CUtensorMap tm_t, const IntraParams prm) {
+           const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_g,
+           const __grid_constant__ CUtensorMap tm_cf, const IntraParams prm) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
@@ -60,14 +70,11 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     const int bf = (int)(b * F + f);
 
     unsigned char *sKi = smem + Smem::KI;
-    unsigned char *sKj = smem + Smem::KJ;
-    unsigned char *sXj = smem + Smem::XJ;
-    unsigned char *sY = sXj;
-    unsigned char *sP = smem + Smem::P;
     unsigned char *sT = smem + Smem::T;
-    float *sG = (float *)(smem + Smem::F);
-    float *sCf = sG + L;
-    uint64_t *bars = (uint64_t *)(((uintptr_t)(sCf + L) + 7) & ~(uintptr_t)7);
+    unsigned char *sRing = smem + Smem::RING;
+    unsigned char *sY = sRing;
+    float *sGC = (float *)(smem + Smem::GC);
+    uint64_t *bars = (uint64_t *)(smem + Smem::END);
     uint32_t *tmem_slot = (uint32_t *)(bars + NBAR);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -75,11 +82,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) {
-            uint32_t cnt = 1;
-            if (i == KIEMPTY || i == SEMPTY0 || i == SEMPTY1 || i == PFULL0 || i == PFULL1 || i == YFULL ||
-                i == XDONE)
-                cnt = kEpi;
-            sm100::mbar_init(&bars[i], cnt);
+            const bool epi = i == KIEMPTY || i == YFULL || i == XDONE || (i >= PFULL && i < PFULL + NSB);
+            sm100::mbar_init(&bars[i], epi ? kEpi : 1);
         }
         sm100::fence_barrier_init();
     }
@@ -102,34 +106,39 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::tma_prefetch_desc(&tm_k);
             sm100::tma_prefetch_desc(&tm_x);
             sm100::tma_prefetch_desc(&tm_t);
+            sm100::tma_prefetch_desc(&tm_g);
+            sm100::tma_prefetch_desc(&tm_cf);
             bool ok = true;
             int n = 0;
             for (int i = 0; i < nblk && ok; ++i) {
+                // K_i after the previous block's R_i read; T_ii and the ring after its T Y product
                 if (i >= 1) ok = sm100::mbar_wait(&bars[KIEMPTY], (i - 1) & 1, err) &&
                                  sm100::mbar_wait(&bars[TEMPTY], (i - 1) & 1, err);
                 if (!ok) break;
                 sm100::mbar_arrive_expect_tx(&bars[KIFULL], (uint32_t)(nslab_k * SLAB_BYTES));
                 for (int sl = 0; sl < nslab_k; ++sl)
-                    for (int half = 0; half < 2; ++half)
-                        sm100::tma_load_4d(sKi + sl * SLAB_BYTES + half * KJ_SLAB, &tm_k, &bars[KIFULL], sl * SLAB,
-                                           h, i * BM + half * JT, bf);
+                    for (int hf = 0; hf < 2; ++hf)
+                        sm100::tma_load_4d(sKi + sl * SLAB_BYTES + hf * KJ_SLAB, &tm_k, &bars[KIFULL], sl * SLAB, h,
+                                           i * BM + hf * JT, bf);
                 sm100::mbar_arrive_expect_tx(&bars[TFULL], (uint32_t)(2 * SLAB_BYTES));
                 for (int sl = 0; sl < 2; ++sl)
-                    sm100::tma_load_3d(sT + sl * SLAB_BYTES, &tm_t, &bars[TFULL], sl * SLAB, 0,
-                                       (int)(fh * nblk + i));
+                    sm100::tma_load_3d(sT + sl * SLAB_BYTES, &tm_t, &bars[TFULL], sl * SLAB, 0, (int)(fh * nblk + i));
                 for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
-                    const int st = n & 1;
-                    if (n >= 2) ok = sm100::mbar_wait(&bars[KXEMPTY0 + st], ((n - 2) >> 1) & 1, err);
+                    const int st = n % NSLOT;
+                    if (n >= NSLOT) ok = sm100::mbar_wait(&bars[KXEMPTY + st], ((n / NSLOT) - 1) & 1, err);
                     if (ok && jt == 2 * (i - 1)) ok = sm100::mbar_wait(&bars[XDONE], (i - 1) & 1, err);
                     if (!ok) break;
-                    sm100::mbar_arrive_expect_tx(&bars[KXFULL0 + st],
-                                                 (uint32_t)(nslab_k * KJ_SLAB + nslab_x * KJ_SLAB));
+                    unsigned char *slot = sRing + st * SLOT_BYTES;
+                    sm100::mbar_arrive_expect_tx(&bars[KXFULL + st],
+                                                 (uint32_t)((nslab_k + nslab_x) * KJ_SLAB + GC_BYTES));
                     for (int sl = 0; sl < nslab_k; ++sl)
-                        sm100::tma_load_4d(sKj + (st * 2 + sl) * KJ_SLAB, &tm_k, &bars[KXFULL0 + st], sl * SLAB, h,
-                                           jt * JT, bf);
+                        sm100::tma_load_4d(slot + sl * KJ_SLAB, &tm_k, &bars[KXFULL + st], sl * SLAB, h, jt * JT, bf);
                     for (int sl = 0; sl < nslab_x; ++sl)
-                        sm100::tma_load_3d(sXj + st * XJ_BYTES + sl * KJ_SLAB, &tm_x, &bars[KXFULL0 + st],
-                                           sl * SLAB, jt * JT, (int)fh);
+                        sm100::tma_load_3d(slot + (2 + sl) * KJ_SLAB, &tm_x, &bars[KXFULL + st], sl * SLAB, jt * JT,
+                                           (int)fh);
+                    float *gc = sGC + st * 2 * JT;
+                    sm100::tma_load_2d(gc, &tm_g, &bars[KXFULL + st], jt * JT, (int)fh);
+                    sm100::tma_load_2d(gc + JT, &tm_cf, &bars[KXFULL + st], jt * JT, (int)fh);
                 }
             }
             // leave with no copy in flight
@@ -143,33 +152,33 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             bool ok = true;
             int n = 0;
             auto issue_px = [&](int m, bool first_of_block, int i) -> bool {
-                const int pb = m & 1;
-                if (!sm100::mbar_wait(&bars[PFULL0 + pb], (m >> 1) & 1, err)) return false;
+                const int pb = m % NSB, st = m % NSLOT;
+                if (!sm100::mbar_wait(&bars[PFULL + pb], (m / NSB) & 1, err)) return false;
                 if (first_of_block && i >= 1 && !sm100::mbar_wait(&bars[XDONE], (i - 1) & 1, err)) return false;
                 sm100::tc_fence_after();
-                const unsigned char *xt = sXj + (m & 1) * XJ_BYTES;
-                const unsigned char *pt = sP + pb * SLAB_BYTES;
+                const unsigned char *xt = sRing + st * SLOT_BYTES + 2 * KJ_SLAB;
+                // P columns k = 0..31 sit in TMEM columns 0..15, k = 32..63 in columns 32..47
                 for (int ks = 0; ks < JT / 16; ++ks)
-                    sm100::mma_bf16_ss(t_acc, desc_kmajor(pt, ks, BM), desc_mnmajor(xt, ks, JT), id_x,
-                                       (first_of_block && ks == 0) ? 0u : 1u);
-                sm100::mma_commit(&bars[PEMPTY0 + pb]);
-                sm100::mma_commit(&bars[KXEMPTY0 + (m & 1)]);
+                    sm100::mma_bf16_ts(t_acc, t_s0 + pb * JT + ks * 8 + (ks >> 1) * 16, desc_mnmajor(xt, ks, JT),
+                                       id_x, (first_of_block && ks == 0) ? 0u : 1u);
+                sm100::mma_commit(&bars[SFREE + pb]);
+                sm100::mma_commit(&bars[KXEMPTY + st]);
                 return true;
             };
             for (int i = 0; i < nblk && ok; ++i) {
                 ok = sm100::mbar_wait(&bars[KIFULL], i & 1, err);
                 const int first = n;
                 for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
-                    const int st = n & 1;
-                    ok = sm100::mbar_wait(&bars[KXFULL0 + st], (n >> 1) & 1, err);
-                    if (ok && n >= 2) ok = sm100::mbar_wait(&bars[SEMPTY0 + st], ((n - 2) >> 1) & 1, err);
+                    const int st = n % NSLOT, sb = n % NSB;
+                    ok = sm100::mbar_wait(&bars[KXFULL + st], (n / NSLOT) & 1, err);
+                    if (ok && n >= NSB) ok = sm100::mbar_wait(&bars[SFREE + sb], ((n / NSB) - 1) & 1, err);
                     if (!ok) break;
                     sm100::tc_fence_after();
-                    const unsigned char *kt = sKj + st * 2 * KJ_SLAB;
+                    const unsigned char *kt = sRing + st * SLOT_BYTES;
                     for (int ks = 0; ks < nks_d; ++ks)
-                        sm100::mma_bf16_ss(t_s0 + st * JT, desc_kmajor(sKi, ks, BM), desc_kmajor(kt, ks, JT), id_s,
+                        sm100::mma_bf16_ss(t_s0 + sb * JT, desc_kmajor(sKi, ks, BM), desc_kmajor(kt, ks, JT), id_s,
                                            ks > 0);
-                    sm100::mma_commit(&bars[SFULL0 + st]);
+                    sm100::mma_commit(&bars[SFULL + sb]);
                     if (jt >= 1) ok = issue_px(n - 1, n - 1 == first, i);
                 }
                 if (ok && i >= 1) ok = issue_px(n - 1, n - 1 == first, i);
@@ -190,26 +199,18 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         // warp % 4) and one half of the columns -- 32 of the 64 columns of an
         // off-diagonal tile, and in the diagonal step the Ub columns (half 0,
         // which needs v) or the W columns (half 1, which needs k).
-        const int et = threadIdx.x - 64;
         const int q4 = warp & 3;
         const int half = (warp - 2) >> 2;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
-        for (int s = et; s < L; s += kEpi) {
-            const int tile_end = min((s / JT) * JT + JT - 1, L - 1);
-            const float g = Gf[s];
-            sG[s] = g;
-            sCf[s] = __expf(Gf[tile_end] - g);  // <= 1: the tile's end is its most decayed token
-        }
-        named_sync(1, kEpi);  // the only epilogue-wide barrier: before any bounded wait
 
         bool ok = true;
         int n = 0;
         for (int i = 0; i < nblk && ok; ++i) {
             const int row = i * BM + r;
             const bool valid = row < L;
-            const float Gr = valid ? sG[row] : 0.f;
+            const float Gr = valid ? Gf[row] : 0.f;
             const long long t = f * L + row;
             const long long tok = ((long long)b * prm.T + t) * prm.H + h;
             const float be = valid ? prm.beta[tok] : 0.f;
@@ -222,31 +223,26 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                                : make_uint4(0, 0, 0, 0);
 
             for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
-                const int sb = n & 1;
-                ok = sm100::mbar_wait(&bars[SFULL0 + sb], (n >> 1) & 1, err);
-                if (ok && n >= 2) ok = sm100::mbar_wait(&bars[PEMPTY0 + sb], ((n - 2) >> 1) & 1, err);
+                const int sb = n % NSB, st = n % NSLOT;
+                ok = sm100::mbar_wait(&bars[SFULL + sb], (n / NSB) & 1, err) &&
+                     sm100::mbar_wait(&bars[KXFULL + st], (n / NSLOT) & 1, err);  // G_j, cf_j
                 if (!ok) break;
                 sm100::tc_fence_after();
-                const float a = sG[jt * JT + JT - 1];
-                const float rf = valid ? -be * __expf(Gr - a) : 0.f;
-                const float *cf = sCf + jt * JT + 32 * half;
-                unsigned char *pt = sP + sb * SLAB_BYTES;
+                // the tile is full (it lies before block i): its anchor is G at token 63
+                const float *gj = sGC + st * 2 * JT;
+                const float rf = valid ? -be * __expf(Gr - gj[JT - 1]) : 0.f;
+                const float *cf = gj + JT + 32 * half;
                 float v[32];
                 sm100::tmem_ld32(t_s0 + sb * JT + lane_off + 32 * half, v);
                 sm100::tmem_ld_wait();
+                uint32_t pk[16];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c8 = 4 * half + u;  // 8-column chunk within the 64-column tile
-                    uint4 val = make_uint4(pack_bf16(rf * cf[u * 8 + 0] * v[u * 8 + 0], rf * cf[u * 8 + 1] * v[u * 8 + 1]),
-                                           pack_bf16(rf * cf[u * 8 + 2] * v[u * 8 + 2], rf * cf[u * 8 + 3] * v[u * 8 + 3]),
-                                           pack_bf16(rf * cf[u * 8 + 4] * v[u * 8 + 4], rf * cf[u * 8 + 5] * v[u * 8 + 5]),
-                                           pack_bf16(rf * cf[u * 8 + 6] * v[u * 8 + 6], rf * cf[u * 8 + 7] * v[u * 8 + 7]));
-                    *reinterpret_cast<uint4 *>(pt + r * 128 + ((c8 ^ (r & 7)) << 4)) = val;
-                }
+                for (int e = 0; e < 32; e += 2) pk[e >> 1] = pack_bf16(rf * cf[e] * v[e], rf * cf[e + 1] * v[e + 1]);
+                // this half's P goes to TMEM columns [32 half, 32 half + 16): S columns it has read
+                sm100::tmem_st16(t_s0 + sb * JT + lane_off + 32 * half, pk);
+                sm100::tmem_st_wait();
                 sm100::tc_fence_before();
-                sm100::mbar_arrive(&bars[SEMPTY0 + sb]);
-                sm100::fence_proxy_async_smem();
-                sm100::mbar_arrive(&bars[PFULL0 + sb]);
+                sm100::mbar_arrive(&bars[PFULL + sb]);
             }
             if (!ok) break;
             // ---- Y_i = R_i + acc_i  -> sY (MN-major: row = K index of the T_ii Y_i product)
@@ -354,16 +350,13 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
 }  // namespace
 
-size_t intra_tc_smem_bytes(int L) {
-    return 1024 + Smem::F + sizeof(float) * 2 * L + 8 + sizeof(uint64_t) * NBAR + 16;
-}
-
 cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_t,
-                            const IntraParams &prm, long long n_fh, cudaStream_t s) {
-    const size_t smem = intra_tc_smem_bytes(prm.L);
+                            const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const IntraParams &prm, long long n_fh,
+                            cudaStream_t s) {
+    const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
     cudaError_t e = cudaFuncSetAttribute(k_intra_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_t, prm);
+    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_t, tm_g, tm_cf, prm);
     return cudaGetLastError();
 }
 

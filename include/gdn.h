@@ -111,6 +111,24 @@ int gdn_step_f32(const float *q, const float *k, const float *v,
                  gdn_stream_t stream);
 
 /*
+ * gdn_fwd_host -- the whole pass from HOST buffers: the same operation,
+ * arguments and layouts as gdn_fwd (dtype = GDN_DTYPE_BF16) or gdn_fwd_f32
+ * (GDN_DTYPE_F32), except that q, k, v, alpha, beta, S_in, S_out and o are
+ * host pointers (pinned memory gives the fastest copies; pageable works).
+ * The call allocates device buffers with cudaMallocAsync on `stream`, copies
+ * the inputs in, runs the pass, copies o (and S_out) out, frees the buffers
+ * and synchronises `stream` before it returns, so the host outputs are
+ * ready.  Host pointers need no alignment.  Errors as gdn_fwd, plus
+ * GDN_ERR_NO_MEMORY when the device buffers cannot be allocated; on any
+ * error after the copies began, o and S_out may be partly written.
+ */
+int gdn_fwd_host(int dtype, const void *q, const void *k, const void *v,
+                 const float *alpha, const float *beta,
+                 const float *S_in, float *S_out, void *o,
+                 int B, int H, long long T, int frame_len, int d_k, int d_v,
+                 gdn_stream_t stream);
+
+/*
  * gdn_fwd_noalloc -- gdn_fwd for callers that cannot allocate device memory.
  * (The SANA-WM pages have no counterpart: this is a deployment variant.)
  *
@@ -189,8 +207,12 @@ typedef struct gdn_args {
 } gdn_args;
 
 /* Kernel stages reported through gdn_args.stage_ms, in launch order:
- * 0 intra-frame solve, 1 frame transition, 2 scan over frames, 3 output. */
-enum { GDN_NUM_STAGES = 4 };
+ * 0 per-frame gate prefix sums, 1 inverses of the 128 x 128 diagonal blocks
+ * of the intra-frame system, 2 intra-frame solve, 3 frame transition,
+ * 4 scan over frames, 5 pseudo-values U, 6 output.  A path that folds a
+ * stage into the next one (the fp32 and reversed paths fold 0, 1 into 2 and
+ * 5 into 6) reports 0 for it. */
+enum { GDN_NUM_STAGES = 7 };
 
 int gdn_fwd_ex(const gdn_args *a);
 

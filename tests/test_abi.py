@@ -50,6 +50,12 @@ def test_struct_size_matches_header():
     assert ctypes.sizeof(binding.GdnArgs) == 160  # LP64 layout of gdn_args
 
 
+def test_stage_count_matches_header():
+    src = open(HEADER).read()
+    m = re.search(r"GDN_NUM_STAGES\s*=\s*(\d+)", src)
+    assert m and int(m.group(1)) == binding.NUM_STAGES == len(binding.STAGES)
+
+
 def _call(fn="gdn_fwd", q=FAKE, k=FAKE + 1024, v=FAKE + 2048, alpha=FAKE + 4096, beta=FAKE + 8192,
           S_in=None, S_out=None, o=FAKE + 16384, B=1, H=2, T=128, L=64, dk=64, dv=64):
     lib = g.load_library()
@@ -101,3 +107,26 @@ def test_python_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 64, 1, 16)
     with pytest.raises(g.GdnError):
         g.gdn_fwd(x, x, x, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1), 64)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=100, L=64), 2), (dict(L=0), 1), (dict(dk=120), 3), (dict(q=None), 1), (dict(o=None), 1),
+])
+def test_host_entry_validates_before_touching_the_gpu(kw, status):
+    # gdn_fwd_host takes host pointers: its size checks run before any CUDA call
+    args = dict(q=FAKE, k=FAKE + 1024, v=FAKE + 2048, alpha=FAKE + 4096, beta=FAKE + 8192, S_in=None,
+                S_out=None, o=FAKE + 16384, B=1, H=2, T=128, L=64, dk=64, dv=64)
+    args.update(kw)
+    lib = g.load_library()
+    rc = lib.gdn_fwd_host(binding.GDN_DTYPE_BF16, args["q"], args["k"], args["v"], args["alpha"], args["beta"],
+                          args["S_in"], args["S_out"], args["o"], args["B"], args["H"], args["T"], args["L"],
+                          args["dk"], args["dv"], None)
+    assert rc == status, g.last_error()
+    assert g.last_error()
+
+
+def test_host_binding_rejects_device_tensors_by_type():
+    import torch
+    x = torch.zeros(1, 64, 1, 16, dtype=torch.float16)
+    with pytest.raises(g.GdnError):
+        g.gdn_fwd_host(x, x, x, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1), 64)

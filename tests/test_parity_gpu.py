@@ -162,6 +162,18 @@ def test_step_chain_equals_single_call(dtype):
     assert rel(o_chain.double().cpu(), o_full.double().cpu()) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_host_entry_matches_device_call(dtype):
+    # gdn_fwd_host runs the same kernels on copies of the host buffers
+    inp = W.draw(1, 3, 2 * 200, 64, 96, frame_len=200, seed=5, regime="slow", dtype=dtype, state_std=0.1)
+    o_dev, S_dev = gpu_fwd(inp, 200, S_in=inp["S_in"])
+    h = {k: (None if v is None else v.contiguous().pin_memory()) for k, v in inp.items()}
+    o_h, S_h = g.gdn_fwd_host(h["q"], h["k"], h["v"], h["alpha"], h["beta"], 200, h["S_in"], return_state=True)
+    assert np.array_equal(o_h.double().numpy(), o_dev) and np.array_equal(S_h.double().numpy(), S_dev)
+    o_ref, S_ref = ora(inp, inp["S_in"])
+    assert rel(o_h.double().numpy(), o_ref) <= TOL[dtype]
+
+
 def test_deterministic():
     inp = W.draw(1, 4, 2 * 880, 112, 112, frame_len=880, seed=3, regime="slow", dtype="bf16")
     d = dev(inp)
