@@ -180,7 +180,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.X = X;
     ip.L = p.L; ip.dk = p.dk; ip.dv = p.dv; ip.H = p.H; ip.nblk = nblk;
     ip.F = p.F; ip.T = p.T; ip.err = err;
-    if ((e = tc::launch_intra_tc(tm_k64, tm_x, tm_t, tm_g, tm_cf, ip, nfh, s))) return e;
+    if ((e = tc::launch_intra_tc(tm_k64, tm_x, tm_t, tm_g, tm_cf, tm_x128, ip, nfh, s))) return e;
     if ((e = mark(ev, 3, s))) return e;
     tc::TransParams tp;
     tp.G = G; tp.M = Mb; tp.N = Nb;

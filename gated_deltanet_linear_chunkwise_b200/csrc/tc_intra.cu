@@ -9,8 +9,9 @@
 //   acc_i = sum_{64-token tiles j before block i} P_ij X_j,  P_ij = -A_ij
 //   Y_i   = R_i + acc_i
 //   X_i   = T_ii Y_i,   T_ii = (I + A_ii)^{-1}  (from tc_diag_inverse.cu)
-// X_i goes to the [n_fh][L][d_v + d_k] bf16 workspace, from where later
-// blocks load it again (L2-resident) by TMA.
+// X_i is staged in shared memory (over K_i and T_ii, both dead by then) and
+// stored by TMA to the [n_fh][L][d_v + d_k] bf16 workspace, from where later
+// blocks load it again (L2-resident).
 //
 // Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
 // warps 2-9 epilogue (two warpgroups; one block row and one column half
@@ -19,7 +20,8 @@
 //         bf16 P in place and acc += P X_j reads P from tensor memory) and
 //         acc / X_i (d_v + d_k columns).
 //   SMEM: K_i, T_ii, and a 3-deep ring of (K_j, X_j, G_j, cf_j) tiles; Y_i
-//         aliases the first two ring slots during the diagonal step.
+//         aliases the first two ring slots during the diagonal step, the
+//         bf16 X_i the K_i and T_ii buffers until its TMA store has read it.
 // Decay factors use a per-tile anchor a = G at the tile's last token:
 // e^{G_r - G_s} = e^{G_r - a} e^{a - G_s}, both <= 1.
 #include "tc_common.cuh"
@@ -47,19 +49,16 @@ struct Smem {
 static_assert(2 * SLOT_BYTES >= 4 * SLAB_BYTES, "Y_i must fit in the first two ring slots");
 
 enum Bar {
-    KIFULL = 0, KIEMPTY, TFULL, TEMPTY, ACCFULL, YFULL, XFULL, XDONE,
+    KIFULL = 0, TFULL, ACCFULL, YFULL, XFULL, ACCFREE, XSTAGED,
     KXFULL, KXEMPTY = KXFULL + NSLOT, SFULL = KXEMPTY + NSLOT, SFREE = SFULL + NSB, PFULL = SFREE + NSB,
     NBAR = PFULL + NSB
 };
 
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_x,
            const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_g,
-           const __grid_constant__ CUtensorMap tm_cf, const IntraParams prm) {
+           const __grid_constant__ CUtensorMap tm_cf, const __grid_constant__ CUtensorMap tm_xs,
+           const IntraParams prm) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
@@ -73,6 +72,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     unsigned char *sT = smem + Smem::T;
     unsigned char *sRing = smem + Smem::RING;
     unsigned char *sY = sRing;
+    unsigned char *sXs = smem + Smem::KI;  // X_i staging: K_i and T_ii, 4 slabs of 128 rows
+    static_assert(Smem::T == Smem::KI + 2 * SLAB_BYTES, "the staging slabs must be contiguous");
     float *sGC = (float *)(smem + Smem::GC);
     uint64_t *bars = (uint64_t *)(smem + Smem::END);
     uint32_t *tmem_slot = (uint32_t *)(bars + NBAR);
@@ -82,7 +83,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) {
-            const bool epi = i == KIEMPTY || i == YFULL || i == XDONE || (i >= PFULL && i < PFULL + NSB);
+            const bool epi = i == YFULL || i == ACCFREE || i == XSTAGED || (i >= PFULL && i < PFULL + NSB);
             sm100::mbar_init(&bars[i], epi ? kEpi : 1);
         }
         sm100::fence_barrier_init();
@@ -108,12 +109,45 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::tma_prefetch_desc(&tm_t);
             sm100::tma_prefetch_desc(&tm_g);
             sm100::tma_prefetch_desc(&tm_cf);
+            sm100::tma_prefetch_desc(&tm_xs);
             bool ok = true;
             int n = 0;
+            auto load_tile = [&](int jt, int i) -> bool {
+                const int st = n % NSLOT;
+                if (n >= NSLOT && !sm100::mbar_wait(&bars[KXEMPTY + st], ((n / NSLOT) - 1) & 1, err)) return false;
+                if (jt == 2 * (i - 1)) sm100::bulk_wait0();  // the rows of X_{i-1} are in global memory
+                unsigned char *slot = sRing + st * SLOT_BYTES;
+                sm100::mbar_arrive_expect_tx(&bars[KXFULL + st], (uint32_t)((nslab_k + nslab_x) * KJ_SLAB + GC_BYTES));
+                for (int sl = 0; sl < nslab_k; ++sl)
+                    sm100::tma_load_4d(slot + sl * KJ_SLAB, &tm_k, &bars[KXFULL + st], sl * SLAB, h, jt * JT, bf);
+                for (int sl = 0; sl < nslab_x; ++sl)
+                    sm100::tma_load_3d(slot + (2 + sl) * KJ_SLAB, &tm_x, &bars[KXFULL + st], sl * SLAB, jt * JT,
+                                       (int)fh);
+                float *gc = sGC + st * 2 * JT;
+                sm100::tma_load_2d(gc, &tm_g, &bars[KXFULL + st], jt * JT, (int)fh);
+                sm100::tma_load_2d(gc + JT, &tm_cf, &bars[KXFULL + st], jt * JT, (int)fh);
+                ++n;
+                return true;
+            };
+            // store the staged X_{i}: rows past the frame and columns past d_v + d_k are clipped
+            auto store_x = [&](int i) -> bool {
+                if (!sm100::mbar_wait(&bars[XSTAGED], i & 1, err)) return false;
+                for (int sl = 0; sl < nslab_x; ++sl)
+                    sm100::tma_store_3d(&tm_xs, sXs + sl * SLAB_BYTES, sl * SLAB, i * BM, (int)fh);
+                sm100::bulk_commit();
+                sm100::bulk_wait_read0();
+                return true;
+            };
             for (int i = 0; i < nblk && ok; ++i) {
-                // K_i after the previous block's R_i read; T_ii and the ring after its T Y product
-                if (i >= 1) ok = sm100::mbar_wait(&bars[KIEMPTY], (i - 1) & 1, err) &&
-                                 sm100::mbar_wait(&bars[TEMPTY], (i - 1) & 1, err);
+                int jt = 0;
+                if (i >= 1) {
+                    // Y_{i-1} is consumed once X_{i-1} = T Y is in TMEM: the ring may refill
+                    ok = sm100::mbar_wait(&bars[XFULL], (i - 1) & 1, err);
+                    const int pre = min(2 * i - 2, NSLOT);  // tiles that do not read X_{i-1}
+                    for (; jt < pre && ok; ++jt) ok = load_tile(jt, i);
+                    // K_i and T_ii overwrite the staging buffer once the store has read it
+                    if (ok) ok = store_x(i - 1);
+                }
                 if (!ok) break;
                 sm100::mbar_arrive_expect_tx(&bars[KIFULL], (uint32_t)(nslab_k * SLAB_BYTES));
                 for (int sl = 0; sl < nslab_k; ++sl)
@@ -123,26 +157,10 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 sm100::mbar_arrive_expect_tx(&bars[TFULL], (uint32_t)(2 * SLAB_BYTES));
                 for (int sl = 0; sl < 2; ++sl)
                     sm100::tma_load_3d(sT + sl * SLAB_BYTES, &tm_t, &bars[TFULL], sl * SLAB, 0, (int)(fh * nblk + i));
-                for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
-                    const int st = n % NSLOT;
-                    if (n >= NSLOT) ok = sm100::mbar_wait(&bars[KXEMPTY + st], ((n / NSLOT) - 1) & 1, err);
-                    if (ok && jt == 2 * (i - 1)) ok = sm100::mbar_wait(&bars[XDONE], (i - 1) & 1, err);
-                    if (!ok) break;
-                    unsigned char *slot = sRing + st * SLOT_BYTES;
-                    sm100::mbar_arrive_expect_tx(&bars[KXFULL + st],
-                                                 (uint32_t)((nslab_k + nslab_x) * KJ_SLAB + GC_BYTES));
-                    for (int sl = 0; sl < nslab_k; ++sl)
-                        sm100::tma_load_4d(slot + sl * KJ_SLAB, &tm_k, &bars[KXFULL + st], sl * SLAB, h, jt * JT, bf);
-                    for (int sl = 0; sl < nslab_x; ++sl)
-                        sm100::tma_load_3d(slot + (2 + sl) * KJ_SLAB, &tm_x, &bars[KXFULL + st], sl * SLAB, jt * JT,
-                                           (int)fh);
-                    float *gc = sGC + st * 2 * JT;
-                    sm100::tma_load_2d(gc, &tm_g, &bars[KXFULL + st], jt * JT, (int)fh);
-                    sm100::tma_load_2d(gc + JT, &tm_cf, &bars[KXFULL + st], jt * JT, (int)fh);
-                }
+                for (; jt < 2 * i && ok; ++jt) ok = load_tile(jt, i);
             }
-            // leave with no copy in flight
-            if (ok) ok = sm100::mbar_wait(&bars[TEMPTY], (nblk - 1) & 1, err);
+            if (ok) ok = store_x(nblk - 1);
+            sm100::bulk_wait0();  // leave with no store in flight
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -154,7 +172,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             auto issue_px = [&](int m, bool first_of_block, int i) -> bool {
                 const int pb = m % NSB, st = m % NSLOT;
                 if (!sm100::mbar_wait(&bars[PFULL + pb], (m / NSB) & 1, err)) return false;
-                if (first_of_block && i >= 1 && !sm100::mbar_wait(&bars[XDONE], (i - 1) & 1, err)) return false;
+                // the first product of a block overwrites acc: X_{i-1} must have been read out
+                if (first_of_block && i >= 1 && !sm100::mbar_wait(&bars[ACCFREE], (i - 1) & 1, err)) return false;
                 sm100::tc_fence_after();
                 const unsigned char *xt = sRing + st * SLOT_BYTES + 2 * KJ_SLAB;
                 // P columns k = 0..31 sit in TMEM columns 0..15, k = 32..63 in columns 32..47
@@ -190,7 +209,6 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 for (int ks = 0; ks < BM / 16; ++ks)
                     sm100::mma_bf16_ss(t_acc, desc_kmajor(sT, ks, BM), desc_mnmajor(sY, ks, BM), id_x, ks > 0);
                 sm100::mma_commit(&bars[XFULL]);
-                sm100::mma_commit(&bars[TEMPTY]);
             }
         }
     } else {
@@ -214,13 +232,12 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             const long long t = f * L + row;
             const long long tok = ((long long)b * prm.T + t) * prm.H + h;
             const float be = valid ? prm.beta[tok] : 0.f;
-            // half 0 reads this row's values (bf16) before the waits to hide their latency
-            uint4 vrow[16];
-#pragma unroll
-            for (int c8 = 0; c8 < 16; ++c8)
-                vrow[c8] = (half == 0 && valid && c8 < dv / 8)
-                               ? *reinterpret_cast<const uint4 *>(prm.v + tok * dv + c8 * 8)
-                               : make_uint4(0, 0, 0, 0);
+            // half 0 needs this row's values in the diagonal step: pull them into L2 now
+            const __nv_bfloat16 *vp = prm.v + tok * dv;
+            if (half == 0 && valid)
+                for (int by = 0; by < dv * 2; by += 128)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"((const char *)vp + by));
+            if (half == 0 && valid) asm volatile("prefetch.global.L2 [%0];" ::"l"((const char *)vp + dv * 2 - 1));
 
             for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
                 const int sb = n % NSB, st = n % NSLOT;
@@ -256,6 +273,11 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 *reinterpret_cast<uint4 *>(sY + (c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4)) = val;
             };
             if (half == 0) {  // Ub columns: beta_r v_r + acc
+                uint4 vrow[16];
+#pragma unroll
+                for (int c8 = 0; c8 < 16; ++c8)
+                    vrow[c8] = (valid && c8 < dv / 8) ? __ldg(reinterpret_cast<const uint4 *>(vp) + c8)
+                                                      : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int c16 = 16 * j;
@@ -315,29 +337,27 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();
             sm100::mbar_arrive(&bars[YFULL]);
-            sm100::mbar_arrive(&bars[KIEMPTY]);
-            // ---- X_i = T_ii Y_i  -> global (half 0 the Ub columns, half 1 the W columns)
+            // ---- X_i = T_ii Y_i  -> bf16 staging (same layout as Y; half 0 the Ub columns, half 1 the W columns)
             ok = sm100::mbar_wait(&bars[XFULL], i & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
-            __nv_bfloat16 *xrow = prm.X + (fh * (long long)L + row) * nc;
             const int c_lo = half ? dv : 0, c_hi = half ? nc : dv;
             for (int c16 = c_lo; c16 < c_hi; c16 += 16) {
                 float x[16];
                 sm100::tmem_ld16(t_acc + lane_off + c16, x);
                 sm100::tmem_ld_wait();
-                if (valid) {
-                    reinterpret_cast<uint4 *>(xrow + c16)[0] =
-                        make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                                   pack_bf16(x[6], x[7]));
-                    reinterpret_cast<uint4 *>(xrow + c16)[1] =
-                        make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]), pack_bf16(x[12], x[13]),
-                                   pack_bf16(x[14], x[15]));
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int c = c16 + 8 * u;
+                    *reinterpret_cast<uint4 *>(sXs + (c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4)) =
+                        make_uint4(pack_bf16(x[8 * u], x[8 * u + 1]), pack_bf16(x[8 * u + 2], x[8 * u + 3]),
+                                   pack_bf16(x[8 * u + 4], x[8 * u + 5]), pack_bf16(x[8 * u + 6], x[8 * u + 7]));
                 }
             }
-            fence_proxy_async_global();
             sm100::tc_fence_before();
-            sm100::mbar_arrive(&bars[XDONE]);
+            sm100::mbar_arrive(&bars[ACCFREE]);
+            sm100::fence_proxy_async_smem();
+            sm100::mbar_arrive(&bars[XSTAGED]);
         }
     }
     sm100::tc_fence_before();
@@ -351,12 +371,12 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 }  // namespace
 
 cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_t,
-                            const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const IntraParams &prm, long long n_fh,
-                            cudaStream_t s) {
+                            const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const CUtensorMap &tm_xs,
+                            const IntraParams &prm, long long n_fh, cudaStream_t s) {
     const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
     cudaError_t e = cudaFuncSetAttribute(k_intra_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_t, tm_g, tm_cf, prm);
+    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_t, tm_g, tm_cf, tm_xs, prm);
     return cudaGetLastError();
 }
 
