@@ -57,6 +57,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs, records kErrTimeout in *err and returns false; every caller
 // then leaves its loop so the kernel can release TMEM and exit.
@@ -74,6 +87,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
         }
     }
 }
+
+// Watchdog for a loop that polls several barriers with mbar_test: reset()
+// after an iteration that made progress, tick() after one that did not.
+// tick() gives up like mbar_wait after kWaitLimitNs without progress.
+struct Spin {
+    uint32_t it = 0;
+    uint64_t t0 = 0;
+    __device__ __forceinline__ void reset() { it = 0; }
+    __device__ __forceinline__ bool tick(int *err) {
+        if (it == 0) t0 = globaltimer_ns();
+        if ((++it & 255u) == 0) {
+            if (*(volatile int *)err != kErrNone) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicCAS(err, kErrNone, kErrTimeout);
+                return false;
+            }
+        }
+        return true;
+    }
+};
 
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {

@@ -6,10 +6,13 @@
 // the causal mask includes the diagonal; SANA-WM summary, "Memory-Efficient
 // Long-Context Modeling (Section 3.2)", frame-wise GDN).
 //
-// Persistent kernel: one CTA per SM walks (frame-head, block) items in
-// frame-head order (neighbouring CTAs share a frame's K and U tiles in L2),
-// with TMEM and barriers set up once.  The columns s come in 64-token tiles
-// through a 4-deep ring so the TMA latency hides behind the tensor work.
+// Persistent kernel: one CTA per SM walks a contiguous range of (frame-head,
+// block) items (ranges balanced by tile count), so a frame's K and U tiles
+// come from HBM once and are re-read from L2 by the same CTA for the frame's
+// other blocks; TMEM and barriers are set up once.  The columns s come in
+// 64-token tiles through a 4-deep ring; the MMA thread issues each tile's
+// S = Q K^T as soon as its data and an S/P buffer are there and each O += P U
+// as soon as the epilogue has written P (polling both in one loop).
 // Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
 // issues tcgen05.mma from one thread, warps 2-9 are the epilogue: two
 // warpgroups, each thread owning one tile row (TMEM lane quadrant =
@@ -97,6 +100,19 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     auto item_blk = [&](long long w) { return nblk - 1 - (int)(w % nblk); };
     auto item_fh = [&](long long w) { return w / nblk; };
     auto item_ntiles = [&](int I) { return min(2 * I + 2, ntile_frame); };
+    // CTA c takes items [item_start(c), item_start(c + 1)): equal shares of the
+    // total weight, an item weighing its tiles plus two (state term, drain)
+    auto item_start = [&](long long c) -> long long {
+        long long wfh = 0;
+        for (int I = 0; I < nblk; ++I) wfh += item_ntiles(I) + 2;
+        const long long target = (c * wfh * nfh + gridDim.x - 1) / gridDim.x;
+        const long long fh = target / wfh;
+        long long rem = target - fh * wfh;
+        int k = 0;
+        while (k < nblk && rem > 0) rem -= item_ntiles(nblk - 1 - k++) + 2;
+        return min(fh * nblk + k, nitems);
+    };
+    const long long w_begin = item_start(blockIdx.x), w_end = item_start(blockIdx.x + 1);
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -109,7 +125,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             sm100::tma_prefetch_desc(&tm_cf);
             bool ok = true;
             int n = 0, t = 0;
-            for (long long w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++t) {
+            for (long long w = w_begin; w < w_end && ok; ++w, ++t) {
                 const int I = item_blk(w);
                 const long long fh = item_fh(w);
                 const long long f = fh % F, chain = fh / F;
@@ -156,7 +172,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const uint32_t id_o = sm100::idesc_bf16(BM, dv, 0, 1);
             bool ok = true;
             int n = 0, sc = 0, t = 0;
-            for (long long w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++t) {
+            for (long long w = w_begin; w < w_end && ok; ++w, ++t) {
                 const int I = item_blk(w);
                 const int nt = item_ntiles(I);
                 const int ob = t & 1, qb = t & 1;
@@ -179,39 +195,51 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 sm100::mma_commit(&bars[REMPTY + st]);
                 ++n;
                 ++sc;
-                // ---- column tiles: S = Q K^T, then O += P U one tile behind
-                int psb = 0, pst = 0, psc = 0;
-                auto issue_pu = [&]() -> bool {
-                    if (!sm100::mbar_wait(&bars[PFULL + psb], (psc / NSB) & 1, err)) return false;
-                    sm100::tc_fence_after();
-                    const unsigned char *u = sRing + pst * SLOT_BYTES + 2 * JSLAB;
-                    // P columns k = 0..31 sit in TMEM columns 0..15, k = 32..63 in columns 32..47
-                    for (int ks = 0; ks < JT / 16; ++ks)
-                        sm100::mma_bf16_ts(t_o, t_s0 + psb * JT + ks * 8 + (ks >> 1) * 16, desc_mnmajor(u, ks, JT),
-                                           id_o, 1u);
-                    sm100::mma_commit(&bars[SFREE + psb]);
-                    sm100::mma_commit(&bars[REMPTY + pst]);
-                    return true;
-                };
+                // ---- column tiles: S = Q K^T as soon as a tile and an S/P buffer are ready,
+                //      O += P U as soon as the epilogue has written P
                 if (ok) ok = sm100::mbar_wait(&bars[QFULL + qb], (t >> 1) & 1, err);
-                for (int j = 0; j < nt && ok; ++j, ++n, ++sc) {
-                    sb = sc % NSB;
-                    st = n % NSLOT;
-                    ok = sm100::mbar_wait(&bars[RFULL + st], (n / NSLOT) & 1, err);
-                    if (ok && sc >= NSB) ok = sm100::mbar_wait(&bars[SFREE + sb], ((sc / NSB) - 1) & 1, err);
-                    if (!ok) break;
-                    sm100::tc_fence_after();
-                    const unsigned char *kt = sRing + st * SLOT_BYTES;
-                    for (int ks = 0; ks < nks_d; ++ks)
-                        sm100::mma_bf16_ss(t_s0 + sb * JT, desc_kmajor(qt, ks, BM), desc_kmajor(kt, ks, JT), id_s,
-                                           ks > 0);
-                    sm100::mma_commit(&bars[SFULL + sb]);
-                    if (j >= 1) ok = issue_pu();
-                    psb = sb;
-                    pst = st;
-                    psc = sc;
+                const int n0 = n, s0 = sc;
+                int js = 0, jp = 0;
+                sm100::Spin spin;
+                while (ok && jp < nt) {
+                    bool prog = false;
+                    if (js < nt && js - jp < NSB) {  // the buffer's previous product has been issued
+                        const int cs = s0 + js, nn = n0 + js;
+                        sb = cs % NSB;
+                        st = nn % NSLOT;
+                        if (sm100::mbar_test(&bars[RFULL + st], (nn / NSLOT) & 1) &&
+                            (cs < NSB || sm100::mbar_test(&bars[SFREE + sb], ((cs / NSB) - 1) & 1))) {
+                            sm100::tc_fence_after();
+                            const unsigned char *kt = sRing + st * SLOT_BYTES;
+                            for (int ks = 0; ks < nks_d; ++ks)
+                                sm100::mma_bf16_ss(t_s0 + sb * JT, desc_kmajor(qt, ks, BM), desc_kmajor(kt, ks, JT),
+                                                   id_s, ks > 0);
+                            sm100::mma_commit(&bars[SFULL + sb]);
+                            ++js;
+                            prog = true;
+                        }
+                    }
+                    if (jp < js) {
+                        const int cs = s0 + jp, nn = n0 + jp;
+                        const int pb = cs % NSB, pst = nn % NSLOT;
+                        if (sm100::mbar_test(&bars[PFULL + pb], (cs / NSB) & 1)) {
+                            sm100::tc_fence_after();
+                            const unsigned char *u = sRing + pst * SLOT_BYTES + 2 * JSLAB;
+                            // P columns k = 0..31 sit in TMEM columns 0..15, k = 32..63 in columns 32..47
+                            for (int ks = 0; ks < JT / 16; ++ks)
+                                sm100::mma_bf16_ts(t_o, t_s0 + pb * JT + ks * 8 + (ks >> 1) * 16,
+                                                   desc_mnmajor(u, ks, JT), id_o, 1u);
+                            sm100::mma_commit(&bars[SFREE + pb]);
+                            sm100::mma_commit(&bars[REMPTY + pst]);
+                            ++jp;
+                            prog = true;
+                        }
+                    }
+                    if (prog) spin.reset();
+                    else if (!spin.tick(err)) ok = false;
                 }
-                if (ok) ok = issue_pu();
+                n = n0 + nt;
+                sc = s0 + nt;
                 if (!ok) break;
                 sm100::mma_commit(&bars[OFULL + ob]);
                 sm100::mma_commit(&bars[QEMPTY + qb]);
@@ -354,8 +382,8 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             sm100::mbar_arrive(&bars[OEMPTY + ob]);
             return true;
         };
-        long long w = blockIdx.x;
-        bool ok = w < nitems;
+        long long w = w_begin;
+        bool ok = w < w_end;
         Item cur;
         if (ok) {
             cur = item_of(w);
@@ -364,15 +392,15 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int t = 0; ok; ++t) {
             ok = tiles(cur);
             if (!ok) break;
-            const long long wn = w + gridDim.x;
+            const long long wn = w + 1;
             Item nxt;
-            if (wn < nitems) {
+            if (wn < w_end) {
                 nxt = item_of(wn);
                 ok = pseudo(nxt, t + 1);
                 if (!ok) break;
             }
             ok = drain(cur, t);
-            if (!ok || wn >= nitems) break;
+            if (!ok || wn >= w_end) break;
             w = wn;
             cur = nxt;
         }
