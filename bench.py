@@ -200,9 +200,8 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from gated_deltanet_linear_chunkwise_b200 import dist as gdist
+    rank, local, world = gdist.env_rank_world()
 
     if args.impl == "reference":
         return run_reference(args, rank, world)
@@ -216,9 +215,7 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        gdist.init("nccl", timeout_s=120, device=dev)
 
     w = W.WORKLOADS[args.workload]
     L, dk, dv, H = w.frame_len, w.d_k, w.d_v, w.H
@@ -240,8 +237,7 @@ def main():
     torch.cuda.synchronize(dev)
 
     # timed region: K steps, CUDA events on the launching stream
-    if world > 1:
-        dist.barrier()
+    gdist.barrier()
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
@@ -251,13 +247,8 @@ def main():
             step()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    gdist.barrier()
+    ms_total = gdist.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
     ms_step = ms_total / args.steps
 
     # per-stage device times (events around each kernel on the same stream)
@@ -285,19 +276,14 @@ def main():
 
     e2e_step()
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    gdist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.e2e_steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, device=dev)
 
     pk = peaks()
     nfh = B * H * w.frames
@@ -349,7 +335,7 @@ def main():
             line["cpu_baseline"] = cpu_baseline(args.regime, args.cpu_frames, inp)
         print(json.dumps(line), flush=True)
     if world > 1:
-        dist.barrier()
+        gdist.barrier()
         dist.destroy_process_group()
 
 

@@ -177,7 +177,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
         return e;
     if ((e = mark(ev, 2, s))) return e;
     tc::IntraParams ip;
-    ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.X = X;
+    ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.k = (const __nv_bfloat16 *)p.k; ip.X = X;
     ip.L = p.L; ip.dk = p.dk; ip.dv = p.dv; ip.H = p.H; ip.nblk = nblk;
     ip.F = p.F; ip.T = p.T; ip.err = err;
     if ((e = tc::launch_intra_tc(tm_k64, tm_x, tm_t, tm_g, tm_cf, tm_x128, ip, nfh, s))) return e;
@@ -185,7 +185,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     tc::TransParams tp;
     tp.G = G; tp.M = Mb; tp.N = Nb;
     tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
-    if ((e = tc::launch_transition_tc(tm_k, tm_x128, tp, nfh, s))) return e;
+    if ((e = tc::launch_transition_tc(tm_k64, tm_x, tp, nfh, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
     if ((e = simt_scan(p, Mb, Nb, Sig, SigB, s))) return e;
     if ((e = mark(ev, 5, s))) return e;

@@ -52,6 +52,7 @@ struct IntraParams {
     const float *G;            // [n_fh][(L+3)&~3]
     const float *beta;         // [B,T,H]
     const __nv_bfloat16 *v;    // [B,T,H,dv]
+    const __nv_bfloat16 *k;    // [B,T,H,dk]
     __nv_bfloat16 *X;          // [n_fh][L][dk + dv]: Ub (first dv columns) then W
     int L, dk, dv, H, nblk;
     long long F, T;
@@ -74,8 +75,10 @@ struct UParams {
     int *err;
 };
 
+// tm_k / tm_x deliver 64-token boxes.
 cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const TransParams &prm,
                                  long long n_fh, cudaStream_t s);
+// tm_x delivers 128-row boxes of X, tm_sig the bf16 state of a frame-head.
 cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_sig, const UParams &prm, long long n_fh,
                         cudaStream_t s);
 

@@ -14,6 +14,10 @@
 //      fp32 (one column per lane),
 //   3. three doubling levels 16 -> 32 -> 64 -> 128:
 //      T21 = -T22 (A21 T11)  on the tensor cores (mma.sync, fp32 accumulate).
+// The products are short dependent chains of mma.sync, whose latency is long
+// next to its issue rate, so every warp keeps several independent
+// accumulators in flight (all its Gram blocks at once; two output tiles and
+// two partial sums over K in the doubling steps).
 // T_ii is written row-major bf16 [n_fh][nblk][128][128] (unit diagonal,
 // zeros above it), the A operand layout of the solve's T_ii Y_i product.
 #include "tc_common.cuh"
@@ -66,18 +70,6 @@ __device__ __forceinline__ void load_b_trans(uint32_t (&b)[4], const __nv_bfloat
     ldsm_x4_t(b, t + k * ld + n);
 }
 
-// D(16x16) = sum over K of A(16xK) B(Kx16); A row-major at (ra, ca), B = M[k][n] row-major at (kb, nb).
-__device__ __forceinline__ void mm16_trans(float (&d0)[4], float (&d1)[4], const __nv_bfloat16 *A, int ra, int ca,
-                                           const __nv_bfloat16 *M, int kb, int nb, int K, int lane) {
-    for (int k = 0; k < K; k += 16) {
-        uint32_t a[4], b[4];
-        load_a(a, A, LDT, ra, ca + k, lane);
-        load_b_trans(b, M, LDT, kb + k, nb, lane);
-        mma16816(d0, a, b[0], b[1]);
-        mma16816(d1, a, b[2], b[3]);
-    }
-}
-
 // Store a 16x16 fp32 accumulator pair as bf16 at (r0, c0), times `scale`.
 __device__ __forceinline__ void store16(__nv_bfloat16 *t, int r0, int c0, const float (&d0)[4],
                                         const float (&d1)[4], float scale, int lane) {
@@ -120,16 +112,23 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r_base = blk * 128;
 
-    // ---- load K_i (rows past the frame are zero), gates, clear T
+    // ---- load K_i (rows past the frame zero-filled) and the gates with asynchronous
+    //      copies all in flight at once, clear T and A meanwhile
     for (int e = tid; e < 128 * (dk / 8); e += kThreads) {
         const int r = e / (dk / 8), c8 = e % (dk / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r_base + r < L) {
-            const long long t = f * L + r_base + r;
-            v = *reinterpret_cast<const uint4 *>(prm.k + (((long long)b * prm.T + t) * prm.H + h) * dk + c8 * 8);
-        }
-        *reinterpret_cast<uint4 *>(sK + r * LDK + c8 * 8) = v;
+        const bool in = r_base + r < L;
+        const long long t = f * L + (in ? r_base + r : 0);
+        sm100::cp_async16(sK + r * LDK + c8 * 8, prm.k + (((long long)b * prm.T + t) * prm.H + h) * dk + c8 * 8,
+                          in ? 16u : 0u);
     }
+    if (tid < 128) {
+        const int r = r_base + tid;
+        const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
+        sm100::cp_async4(sG + tid, Gf + (r < L ? r : L - 1));
+        if (r < L) sm100::cp_async4(sB + tid, prm.beta + ((long long)b * prm.T + f * L + r) * prm.H + h);
+        else sB[tid] = 0.f;
+    }
+    sm100::cp_async_commit();
     for (int e = tid; e < 128 * ((128 - dk) / 8); e += kThreads) {  // zero the padding columns up to 128
         const int r = e / ((128 - dk) / 8), c8 = e % ((128 - dk) / 8);
         *reinterpret_cast<uint4 *>(sK + r * LDK + dk + c8 * 8) = make_uint4(0, 0, 0, 0);
@@ -139,34 +138,22 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
         *reinterpret_cast<uint4 *>(sT + r * LDT + c8 * 8) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4 *>(sA + r * LDT + c8 * 8) = make_uint4(0, 0, 0, 0);
     }
-    if (tid < 128) {
-        const int r = r_base + tid;
-        const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
-        sG[tid] = Gf[r < L ? r : L - 1];
-        sB[tid] = (r < L) ? prm.beta[((long long)b * prm.T + f * L + r) * prm.H + h] : 0.f;
-    }
+    sm100::cp_async_wait_all();
     __syncthreads();
 
     // ---- A = beta_r e^{G_r - G_s} (K K^T)[r][s], s < r, on the 36 lower 16x16 blocks
     const int g = lane >> 2, q = lane & 3;
-    for (int blkid = warp; blkid < 36; blkid += 8) {
-        int ab = 0, rem = blkid;  // block row ab, block column cb <= ab
-        while (rem > ab) { rem -= ab + 1; ++ab; }
-        const int cb = rem;
-        float d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-        for (int kk = 0; kk < dk; kk += 16) {
-            uint32_t a[4], bb[4];
-            load_a(a, sK, LDK, ab * 16, kk, lane);
-            load_b_rows(bb, sK, LDK, cb * 16, kk, lane);
-            mma16816(d0, a, bb[0], bb[1]);
-            mma16816(d1, a, bb[2], bb[3]);
-        }
-        // element (r, s) of this thread's fragments
+    auto block_of = [](int id, int &ab, int &cb) {  // block row ab, block column cb <= ab
+        ab = 0;
+        while (id > ab) { id -= ab + 1; ++ab; }
+        cb = id;
+    };
+    auto finish = [&](int ab, int cb, const float (&d0)[4], const float (&d1)[4]) {
         const float *dd[2] = {d0, d1};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 4; ++e) {  // element (r, s) of this thread's fragments
                 const int r = ab * 16 + g + (e >> 1) * 8;
                 const int s = cb * 16 + nt * 8 + 2 * q + (e & 1);
                 const float val = (s < r) ? sB[r] * __expf(sG[r] - sG[s]) * dd[nt][e] : 0.f;
@@ -174,7 +161,32 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
                 if (ab == cb) sAd[ab * 256 + (r - ab * 16) * 16 + (s - cb * 16)] = val;
             }
         }
+    };
+    // warp w owns blocks w, w + 8, ..., all accumulated at once: ten independent
+    // accumulation chains hide the latency of the tensor-core instructions
+    constexpr int NB = 5;  // ceil(36 / 8)
+    int ab[NB], cb[NB];
+#pragma unroll
+    for (int u = 0; u < NB; ++u) block_of(min(warp + 8 * u, 35), ab[u], cb[u]);
+    float acc[NB][2][4] = {};
+#pragma unroll
+    for (int kk = 0; kk < 128; kk += 16) {
+        if (kk < dk) {
+#pragma unroll
+            for (int u = 0; u < NB; ++u) {
+                if (warp + 8 * u < 36) {
+                    uint32_t a[4], bb[4];
+                    load_a(a, sK, LDK, ab[u] * 16, kk, lane);
+                    load_b_rows(bb, sK, LDK, cb[u] * 16, kk, lane);
+                    mma16816(acc[u][0], a, bb[0], bb[1]);
+                    mma16816(acc[u][1], a, bb[2], bb[3]);
+                }
+            }
+        }
     }
+#pragma unroll
+    for (int u = 0; u < NB; ++u)
+        if (warp + 8 * u < 36) finish(ab[u], cb[u], acc[u][0], acc[u][1]);
     __syncthreads();
 
     // ---- leaves: warp w inverts diagonal block w; lane c < 16 owns column c
@@ -194,30 +206,60 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
     }
     __syncthreads();
 
-    // ---- doubling: T21 = -T22 (A21 T11) for block sizes 16, 32, 64
+    // ---- doubling: T21 = -T22 (A21 T11) for block sizes 16, 32, 64; each warp runs two
+    //      16x16 output tiles at a time
     for (int sz = 16; sz <= 64; sz <<= 1) {
-        const int nmerge = 128 / (2 * sz);
-        const int tiles = (sz / 16) * (sz / 16);   // 16x16 output tiles per merge
-        // X = A21 T11 into sX (rows of the lower half, cols of the upper half)
-        for (int w = warp; w < nmerge * tiles; w += 8) {
-            const int m = w / tiles, tt = w % tiles;
-            const int base = m * 2 * sz;
-            const int tr = (tt / (sz / 16)) * 16, tc = (tt % (sz / 16)) * 16;
-            float d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-            mm16_trans(d0, d1, sA, base + sz + tr, base, sT, base, base + tc, sz, lane);
-            store16(sX, base + sz + tr, base + tc, d0, d1, 1.f, lane);
+        const int per = (sz / 16) * (sz / 16);  // 16x16 output tiles per merge
+        const int total = (128 / (2 * sz)) * per;
+        for (int pass = 0; pass < 2; ++pass) {
+            // pass 0: X = A21 T11 -> sX;  pass 1: T21 = -T22 X -> sT
+            const __nv_bfloat16 *Am = pass ? sT : sA;
+            const __nv_bfloat16 *Bm = pass ? sX : sT;
+            __nv_bfloat16 *Dm = pass ? sT : sX;
+            for (int w0 = warp; w0 < total; w0 += 16) {
+                const int w1 = w0 + 8;
+                const bool two = w1 < total;
+                int ra[2], ca[2], kb[2], nb[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int w = (u && two) ? w1 : w0;
+                    const int m = w / per, tt = w % per;
+                    const int base = m * 2 * sz;
+                    const int tr = (tt / (sz / 16)) * 16, tc = (tt % (sz / 16)) * 16;
+                    ra[u] = base + sz + tr;                 // output / A rows (lower half)
+                    ca[u] = pass ? base + sz : base;        // A columns: T22 or A21
+                    kb[u] = pass ? base + sz : base;        // B rows: X (lower half) or T11
+                    nb[u] = base + tc;                      // output columns (upper half)
+                }
+                // two tiles, each as two partial sums over alternate 16-wide K slices
+                float d[2][2][2][4] = {};
+                for (int k = 0; k < sz; k += 32) {
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        if (k + 16 * h2 < sz) {
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                uint32_t af[4], bf[4];
+                                load_a(af, Am, LDT, ra[u], ca[u] + k + 16 * h2, lane);
+                                load_b_trans(bf, Bm, LDT, kb[u] + k + 16 * h2, nb[u], lane);
+                                mma16816(d[u][h2][0], af, bf[0], bf[1]);
+                                mma16816(d[u][h2][1], af, bf[2], bf[3]);
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        d[u][0][0][e] += d[u][1][0][e];
+                        d[u][0][1][e] += d[u][1][1][e];
+                    }
+                store16(Dm, ra[0], nb[0], d[0][0][0], d[0][0][1], pass ? -1.f : 1.f, lane);
+                if (two) store16(Dm, ra[1], nb[1], d[1][0][0], d[1][0][1], pass ? -1.f : 1.f, lane);
+            }
+            __syncthreads();
         }
-        __syncthreads();
-        // T21 = -T22 X
-        for (int w = warp; w < nmerge * tiles; w += 8) {
-            const int m = w / tiles, tt = w % tiles;
-            const int base = m * 2 * sz;
-            const int tr = (tt / (sz / 16)) * 16, tc = (tt % (sz / 16)) * 16;
-            float d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
-            mm16_trans(d0, d1, sT, base + sz + tr, base + sz, sX, base + sz, base + tc, sz, lane);
-            store16(sT, base + sz + tr, base + tc, d0, d1, -1.f, lane);
-        }
-        __syncthreads();
     }
 
     // ---- write T_ii row-major

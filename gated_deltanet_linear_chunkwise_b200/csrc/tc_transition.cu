@@ -6,12 +6,14 @@
 // (the per-frame transition of the chunk = frame decomposition; the pages
 // compose these maps with a prefix sum over frames: cliffmar.tech article,
 // "NVIDIA SANA-WM", the training section on context parallelism).
-// One CTA per frame-head accumulates Kt^T [Ub | W] over 128-token blocks:
-// A = Kt as an MN-major operand (the K tile's rows are tokens, i.e. the
-// contraction index), B = the [Ub | W] block (MN-major), D in TMEM with one
-// lane per key dimension.  The epilogue warps scale the K rows in shared
-// memory by e^{G_L - G_r} (a per-row factor, so the swizzle does not
-// matter) and finally write M and N in fp32.
+// One CTA per frame-head accumulates Kt^T [Ub | W] over 64-token chunks that
+// stream through a 2-deep ring, two CTAs per SM so that one CTA's loads
+// overlap the other's start-up and final stores (the kernel is bound by the
+// rate at which the chunks arrive from HBM): A = Kt as an MN-major operand (the K chunk's rows are
+// tokens, i.e. the contraction index), B = the [Ub | W] chunk (MN-major), D
+// in TMEM with one lane per key dimension.  The epilogue warps scale the K
+// rows in shared memory by e^{G_L - G_r} (a per-row factor, so the swizzle
+// does not matter) and finally write M and N in fp32.
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -19,28 +21,30 @@ namespace tc {
 namespace {
 
 constexpr int kThreads = 192;
+constexpr int CH = 64;                         // tokens per chunk
+constexpr int NST = 2;                         // ring depth (two CTAs per SM)
+constexpr int CSLAB = CH * 128;                // one 64-row slab
+constexpr int STAGE = 6 * CSLAB;               // K (2 slabs) + [Ub | W] (4 slabs)
 
 struct Smem {
-    static constexpr uint32_t K = 0;                       // 2 stages x 2 slabs x 128 rows
-    static constexpr uint32_t X = K + 4 * SLAB_BYTES;      // 2 stages x 4 slabs x 128 rows
-    static constexpr uint32_t END = X + 8 * SLAB_BYTES;
+    static constexpr uint32_t RING = 0;
+    static constexpr uint32_t END = RING + NST * STAGE;
 };
 
-enum Bar { FULL0, FULL1, SCALED0, SCALED1, EMPTY0, EMPTY1, DONE, NBAR };
+enum Bar { FULL = 0, SCALED = FULL + NST, EMPTY = SCALED + NST, DONE = EMPTY + NST, NBAR };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_x,
                 const TransParams prm) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
+    const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv;
     const long long fh = blockIdx.x;
     const long long F = prm.F;
     const long long f = fh % F, chain = fh / F;
     const int h = (int)(chain % prm.H), b = (int)(chain / prm.H);
     const int bf = (int)(b * F + f);
-    unsigned char *sK = smem + Smem::K;
-    unsigned char *sX = smem + Smem::X;
+    unsigned char *sRing = smem + Smem::RING;
     uint64_t *bars = (uint64_t *)(smem + Smem::END);
     uint32_t *tmem_slot = (uint32_t *)(bars + NBAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -48,7 +52,7 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_x = (nc + SLAB - 1) / SLAB;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NBAR; ++i) sm100::mbar_init(&bars[i], (i == SCALED0 || i == SCALED1) ? 128 : 1);
+        for (int i = 0; i < NBAR; ++i) sm100::mbar_init(&bars[i], (i >= SCALED && i < SCALED + NST) ? 128 : 1);
         sm100::fence_barrier_init();
     }
     if (warp == 1) {
@@ -60,22 +64,22 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     sm100::tc_fence_after();
     const uint32_t t_d = *tmem_slot;
 
+    const int nch = (L + CH - 1) / CH;
     if (warp == 0) {
         if (lane == 0) {
             sm100::tma_prefetch_desc(&tm_k);
             sm100::tma_prefetch_desc(&tm_x);
             bool ok = true;
-            for (int i = 0; i < nblk && ok; ++i) {
-                const int st = i & 1;
-                if (i >= 2) ok = sm100::mbar_wait(&bars[EMPTY0 + st], ((i - 2) >> 1) & 1, err);
+            for (int c = 0; c < nch && ok; ++c) {
+                const int st = c % NST;
+                if (c >= NST) ok = sm100::mbar_wait(&bars[EMPTY + st], ((c / NST) - 1) & 1, err);
                 if (!ok) break;
-                sm100::mbar_arrive_expect_tx(&bars[FULL0 + st], (uint32_t)((nslab_k + nslab_x) * SLAB_BYTES));
+                unsigned char *stage = sRing + st * STAGE;
+                sm100::mbar_arrive_expect_tx(&bars[FULL + st], (uint32_t)((nslab_k + nslab_x) * CSLAB));
                 for (int sl = 0; sl < nslab_k; ++sl)
-                    sm100::tma_load_4d(sK + (st * 2 + sl) * SLAB_BYTES, &tm_k, &bars[FULL0 + st], sl * SLAB, h,
-                                       i * BM, bf);
+                    sm100::tma_load_4d(stage + sl * CSLAB, &tm_k, &bars[FULL + st], sl * SLAB, h, c * CH, bf);
                 for (int sl = 0; sl < nslab_x; ++sl)
-                    sm100::tma_load_3d(sX + (st * 4 + sl) * SLAB_BYTES, &tm_x, &bars[FULL0 + st], sl * SLAB, i * BM,
-                                       (int)fh);
+                    sm100::tma_load_3d(stage + (2 + sl) * CSLAB, &tm_x, &bars[FULL + st], sl * SLAB, c * CH, (int)fh);
             }
             if (ok) sm100::mbar_wait(&bars[DONE], 0, err);  // no copy left in flight
         }
@@ -83,49 +87,50 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (lane == 0) {
             const uint32_t id = sm100::idesc_bf16(BM, nc, 1, 1);
             bool ok = true;
-            for (int i = 0; i < nblk && ok; ++i) {
-                const int st = i & 1;
-                ok = sm100::mbar_wait(&bars[SCALED0 + st], (i >> 1) & 1, err);
+            for (int c = 0; c < nch && ok; ++c) {
+                const int st = c % NST;
+                ok = sm100::mbar_wait(&bars[SCALED + st], (c / NST) & 1, err);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                const unsigned char *kt = sK + st * 2 * SLAB_BYTES;
-                const unsigned char *xt = sX + st * 4 * SLAB_BYTES;
-                for (int ks = 0; ks < BM / 16; ++ks)
-                    sm100::mma_bf16_ss(t_d, desc_mnmajor(kt, ks, BM), desc_mnmajor(xt, ks, BM), id,
-                                       (i > 0 || ks > 0) ? 1u : 0u);
-                sm100::mma_commit(&bars[EMPTY0 + st]);
+                const unsigned char *kt = sRing + st * STAGE;
+                const unsigned char *xt = kt + 2 * CSLAB;
+                for (int ks = 0; ks < CH / 16; ++ks)
+                    sm100::mma_bf16_ss(t_d, desc_mnmajor(kt, ks, CH), desc_mnmajor(xt, ks, CH), id,
+                                       (c > 0 || ks > 0) ? 1u : 0u);
+                sm100::mma_commit(&bars[EMPTY + st]);
             }
             if (ok) sm100::mma_commit(&bars[DONE]);
         }
     } else {
         const int q4 = warp & 3;
-        const int r = q4 * 32 + lane;  // token row of each block; at the end, key dimension m
+        const int r = q4 * 32 + lane;  // the epilogue's 128 threads; at the end, key dimension m
         const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
         const float GL = Gf[L - 1];
         bool ok = true;
-        for (int i = 0; i < nblk && ok; ++i) {
-            const int st = i & 1;
-            const int row = i * BM + r;
+        // thread r scales row r % 64 of the chunk's K, slab r / 64
+        const int row_in = r & (CH - 1), sl = r >> 6;
+        for (int c = 0; c < nch && ok; ++c) {
+            const int st = c % NST;
+            const int row = c * CH + row_in;
             const float sc = row < L ? __expf(GL - Gf[row]) : 0.f;
-            ok = sm100::mbar_wait(&bars[FULL0 + st], (i >> 1) & 1, err);
+            ok = sm100::mbar_wait(&bars[FULL + st], (c / NST) & 1, err);
             if (!ok) break;
-            unsigned char *kt = sK + st * 2 * SLAB_BYTES;
-            for (int sl = 0; sl < nslab_k; ++sl) {
-                uint4 *rowp = reinterpret_cast<uint4 *>(kt + sl * SLAB_BYTES + r * 128);
+            if (sl < nslab_k) {
+                uint4 *rowp = reinterpret_cast<uint4 *>(sRing + st * STAGE + sl * CSLAB + row_in * 128);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 v = rowp[c];
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint4 v = rowp[cc];
                     __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&v);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         float2 x = __bfloat1622float2(p2[e]);
                         p2[e] = __floats2bfloat162_rn(sc * x.x, sc * x.y);
                     }
-                    rowp[c] = v;
+                    rowp[cc] = v;
                 }
             }
             sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(&bars[SCALED0 + st]);
+            sm100::mbar_arrive(&bars[SCALED + st]);
         }
         if (ok) ok = sm100::mbar_wait(&bars[DONE], 0, err);
         if (ok) {

@@ -100,24 +100,32 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
             const bool valid = row < L;
             const __nv_bfloat16 *xrow = prm.X + (fh * (long long)L + (valid ? row : 0)) * nc;
             __nv_bfloat16 *urow = prm.U + (fh * (long long)L + (valid ? row : 0)) * dv;
+            // this row's Ub (bf16) in registers before the wait, so its latency hides behind the MMA
+            uint4 ub[16];
+#pragma unroll
+            for (int c8 = 0; c8 < 16; ++c8)
+                ub[c8] = (valid && c8 < dv / 8) ? __ldg(reinterpret_cast<const uint4 *>(xrow) + c8)
+                                                : make_uint4(0, 0, 0, 0);
             ok = sm100::mbar_wait(&bars[DFULL0 + st], (i >> 1) & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
-            for (int c0 = 0; c0 < dv; c0 += 16) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int c0 = 16 * j;
+                if (c0 >= dv) break;
                 float d[16];
                 sm100::tmem_ld16(t_d + st * 128 + lane_off + c0, d);
                 sm100::tmem_ld_wait();
                 if (valid) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(xrow + c0);
                     uint4 out[2];
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
-                        uint4 xv = src[w];
+                        uint4 xv = ub[2 * j + w];
                         __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&xv);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const float2 ub = __bfloat1622float2(p2[e]);
-                            p2[e] = __floats2bfloat162_rn(ub.x - d[w * 8 + 2 * e], ub.y - d[w * 8 + 2 * e + 1]);
+                            const float2 u = __bfloat1622float2(p2[e]);
+                            p2[e] = __floats2bfloat162_rn(u.x - d[w * 8 + 2 * e], u.y - d[w * 8 + 2 * e + 1]);
                         }
                         out[w] = xv;
                     }
