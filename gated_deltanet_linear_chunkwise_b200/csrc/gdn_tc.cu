@@ -25,7 +25,7 @@ namespace {
 inline int cf_stride(int L) { return (L + 3) & ~3; }
 
 struct TcLayout {
-    size_t G, CF, Tinv, X, M, N, Sig, SigB, U, err, total;
+    size_t G, CF, GCT, Tinv, X, M, N, Sig, SigB, U, err, total;
 };
 
 TcLayout tc_layout(const Problem &p) {
@@ -35,6 +35,7 @@ TcLayout tc_layout(const Problem &p) {
     size_t off = 0;
     lay.G = off;    off += align256(sizeof(float) * nfh * (size_t)cf_stride(p.L));
     lay.CF = off;   off += align256(sizeof(float) * nfh * (size_t)cf_stride(p.L));
+    lay.GCT = off;  off += align256(sizeof(float) * nfh * (size_t)((p.L + 127) / 128) * 256);
     lay.Tinv = off; off += align256(2 * nfh * (size_t)((p.L + 127) / 128) * 128 * 128);
     lay.X = off;    off += align256(2 * nfh * p.L * nc);
     lay.M = off;    off += align256(sizeof(float) * nfh * p.dk * p.dk);
@@ -107,7 +108,10 @@ bool map_rows(CUtensorMap *m, const void *x, long long nfh, int rows, int cols, 
 // G = per-frame inclusive prefix of log alpha; CF = e^{a(s) - G_s} with a(s)
 // = G at the last token of s's 64-token tile (<= 1): the column half of the
 // split decay factor e^{G_r - G_s} = e^{G_r - a} e^{a - G_s}.
-__global__ void __launch_bounds__(256) gate_prefix_kernel(Problem p, float *__restrict__ G, float *__restrict__ CF) {
+// GCT = the same G and CF regrouped per 128-token tile, [n_fh][tile][G[128], CF[128]]
+// (zeros past the frame), so one TMA box delivers both for a tile.
+__global__ void __launch_bounds__(256)
+gate_prefix_kernel(Problem p, float *__restrict__ G, float *__restrict__ CF, float *__restrict__ GCT) {
     extern __shared__ __align__(16) unsigned char smem[];
     const long long fh = blockIdx.x;
     const long long f = fh % p.F, chain = fh / p.F;
@@ -117,10 +121,19 @@ __global__ void __launch_bounds__(256) gate_prefix_kernel(Problem p, float *__re
     float *sScr = sB + p.L;
     frame_gates<float>(p, b, h, f, sG, sB, sScr);
     const int cfs = (p.L + 3) & ~3;  // cf_stride(L): G and CF rows start on 16-byte boundaries
-    for (int i = threadIdx.x; i < p.L; i += blockDim.x) {
-        const int end = min((i / 64) * 64 + 63, p.L - 1);
-        G[fh * cfs + i] = sG[i];
-        CF[fh * cfs + i] = __expf(sG[end] - sG[i]);
+    const int nt = (p.L + 127) / 128;
+    float *gct = GCT + fh * (long long)nt * 256;
+    for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) {
+        float g = 0.f, cf = 0.f;
+        if (i < p.L) {
+            const int end = min((i / 64) * 64 + 63, p.L - 1);
+            g = sG[i];
+            cf = __expf(sG[end] - sG[i]);
+            G[fh * cfs + i] = g;
+            CF[fh * cfs + i] = cf;
+        }
+        gct[(i / 128) * 256 + (i & 127)] = g;
+        gct[(i / 128) * 256 + 128 + (i & 127)] = cf;
     }
 }
 
@@ -145,6 +158,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     const int nblk = (p.L + tc::BM - 1) / tc::BM;
     float *G = (float *)(base + lay.G);
     float *CF = (float *)(base + lay.CF);
+    float *GCT = (float *)(base + lay.GCT);
     __nv_bfloat16 *X = (__nv_bfloat16 *)(base + lay.X);
     float *Mb = (float *)(base + lay.M), *Nb = (float *)(base + lay.N), *Sig = (float *)(base + lay.Sig);
     __nv_bfloat16 *SigB = (__nv_bfloat16 *)(base + lay.SigB);
@@ -154,13 +168,15 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
 
     __nv_bfloat16 *Tinv = (__nv_bfloat16 *)(base + lay.Tinv);
     const int nc = p.dk + p.dv;
-    CUtensorMap tm_q, tm_k, tm_u64, tm_sig, tm_k64, tm_x, tm_t, tm_x128, tm_g, tm_cf;
+    CUtensorMap tm_q, tm_k, tm_u128, tm_sig, tm_k64, tm_x, tm_t, tm_x128, tm_g128, tm_cf128, tm_gct;
+    const int nt128 = (p.L + 127) / 128;
     if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
-        !map_rows(&tm_u64, U, nfh, p.L, p.dv, 64) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
+        !map_rows(&tm_u128, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
         !map_tokens(&tm_k64, p.k, p, p.dk, 64) || !map_rows(&tm_x, X, nfh, p.L, nc, 64) ||
         !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128) || !map_rows(&tm_x128, X, nfh, p.L, nc, 128) ||
-        !map_f32_rows(&tm_g, G, nfh, p.L, cf_stride(p.L), 64) ||
-        !map_f32_rows(&tm_cf, CF, nfh, p.L, cf_stride(p.L), 64))
+        !map_f32_rows(&tm_gct, GCT, nfh * nt128, 256, 256, 256) ||
+        !map_f32_rows(&tm_g128, G, nfh, p.L, cf_stride(p.L), 128) ||
+        !map_f32_rows(&tm_cf128, CF, nfh, p.L, cf_stride(p.L), 128))
         return cudaErrorInvalidValue;
 
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
@@ -169,7 +185,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
         (e = cudaFuncSetAttribute(gate_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm)))
         return e;
     if ((e = mark(ev, 0, s))) return e;
-    gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF);
+    gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF, GCT);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 1, s))) return e;
     if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
@@ -180,7 +196,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.k = (const __nv_bfloat16 *)p.k; ip.X = X;
     ip.L = p.L; ip.dk = p.dk; ip.dv = p.dv; ip.H = p.H; ip.nblk = nblk;
     ip.F = p.F; ip.T = p.T; ip.err = err;
-    if ((e = tc::launch_intra_tc(tm_k64, tm_x, tm_t, tm_g, tm_cf, tm_x128, ip, nfh, s))) return e;
+    if ((e = tc::launch_intra_tc(tm_k, tm_x, tm_t, tm_gct, tm_x128, ip, nfh, s))) return e;
     if ((e = mark(ev, 3, s))) return e;
     tc::TransParams tp;
     tp.G = G; tp.M = Mb; tp.N = Nb;
@@ -205,7 +221,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     op.err = err;
     int dev = 0, num_sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if ((e = tc::launch_output_tc(tm_q, tm_k64, tm_u64, tm_sig, tm_g, tm_cf, op, num_sms, s))) return e;
+    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u128, tm_sig, tm_g128, tm_cf128, op, num_sms, s))) return e;
     return mark(ev, 7, s);
 }
 

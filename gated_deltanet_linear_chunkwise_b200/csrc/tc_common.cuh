@@ -82,18 +82,19 @@ cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_
 cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_sig, const UParams &prm, long long n_fh,
                         cudaStream_t s);
 
-// tm_k / tm_x / tm_g / tm_cf deliver 64-token boxes, tm_t one 128 x 128 block;
-// tm_xs stores 128-row boxes of X.
-cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_t,
-                            const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const CUtensorMap &tm_xs,
-                            const IntraParams &prm, long long n_fh, cudaStream_t s);
+// tm_k delivers 128-token boxes of k, tm_x64 64-row boxes of X, tm_t one
+// 128 x 128 block, tm_gct the G and cf of one 128-token tile; tm_xs stores
+// 128-row boxes of X.
+cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x64, const CUtensorMap &tm_t,
+                            const CUtensorMap &tm_gct, const CUtensorMap &tm_xs, const IntraParams &prm,
+                            long long n_fh, cudaStream_t s);
 
 cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
                                 int L, int dk, int H, int nblk, long long F, long long T, long long n_fh,
                                 cudaStream_t s);
 
-// tm_k64 / tm_u64 / tm_g / tm_cf deliver 64-token boxes; tm_q 128-token boxes.
-cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k64, const CUtensorMap &tm_u64,
+// tm_q / tm_k / tm_u / tm_g / tm_cf deliver 128-token boxes.
+cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
                              const CUtensorMap &tm_sig, const CUtensorMap &tm_g, const CUtensorMap &tm_cf,
                              const OutParams &prm, int num_sms, cudaStream_t s);
 

@@ -6,24 +6,29 @@
 //   (I + A) X = R,   X = [Ub | W],   R = [beta V | beta e^G K],
 //   A_rs = beta_r e^{G_r - G_s} k_r.k_s  (s < r)
 // over 128-row blocks i, in order:
-//   acc_i = sum_{64-token tiles j before block i} P_ij X_j,  P_ij = -A_ij
+//   acc_i = sum_{128-token tiles c before block i} P_ic X_c,  P_ic = -A_ic
 //   Y_i   = R_i + acc_i
 //   X_i   = T_ii Y_i,   T_ii = (I + A_ii)^{-1}  (from tc_diag_inverse.cu)
-// X_i is staged in shared memory (over K_i and T_ii, both dead by then) and
-// stored by TMA to the [n_fh][L][d_v + d_k] bf16 workspace, from where later
-// blocks load it again (L2-resident).
+// X_i is staged in shared memory and stored by TMA to the [n_fh][L][d_v + d_k]
+// bf16 workspace, from where later blocks load it again (L2-resident).
 //
-// Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer,
-// warps 2-9 epilogue (two warpgroups; one block row and one column half
-// per thread).
-//   TMEM: four S/P buffers (64 columns each; the epilogue turns S into the
-//         bf16 P in place and acc += P X_j reads P from tensor memory) and
-//         acc / X_i (d_v + d_k columns).
-//   SMEM: K_i, T_ii, and a 3-deep ring of (K_j, X_j, G_j, cf_j) tiles; Y_i
-//         aliases the first two ring slots during the diagonal step, the
-//         bf16 X_i the K_i and T_ii buffers until its TMA store has read it.
-// Decay factors use a per-tile anchor a = G at the tile's last token:
-// e^{G_r - G_s} = e^{G_r - a} e^{a - G_s}, both <= 1.
+// A tcgen05.mma costs the same for every N up to 128, so S = K_i K_c^T is
+// issued on 128-token tiles (N = 128).  Two rings feed the tensor cores:
+//   K ring (2 x 32 KB): the K tile of each S product with its G and cf
+//                       (one TMA box), and T_ii as the block's last item;
+//   X ring (3 x 32 KB): the 64-token halves of X_c for acc += P X.
+// Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer (one
+// thread), warps 2-9 epilogue: two warpgroups, each thread owning one block
+// row (TMEM lane quadrant = warp % 4) and one half of the columns -- 64 of
+// the 128 columns of an S tile, and in the diagonal step the Ub columns
+// (half 0, which needs v) or the W columns (half 1, which needs k).
+//   TMEM: two S/P buffers of 128 columns (the epilogue turns S into bf16 P in
+//         place; acc += P X reads P from tensor memory) and acc (256 columns).
+//   SMEM: K_i, the two rings; Y_i and then the staged X_i occupy the first
+//         two X-ring slots during the diagonal step.
+// Decay factors use the gate kernel's 64-token anchors: a = G at the end of
+// the 64-token group, e^{G_r - G_s} = e^{G_r - a} cf_s, cf_s = e^{a - G_s}.
+// Every wait is bounded (sm100::mbar_wait).
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -32,33 +37,39 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kEpi = 256;                    // epilogue threads
-constexpr int JT = 64;                       // tokens per off-diagonal tile
-constexpr int NSLOT = 3;                     // ring depth
-constexpr int NSB = 4;                       // S/P buffers in TMEM
-constexpr int KJ_SLAB = JT * 128;            // 64-row slab
-constexpr int SLOT_BYTES = 6 * KJ_SLAB;      // K_j (2 slabs) + X_j (4 slabs)
-constexpr int GC_BYTES = 2 * JT * 4;         // G and cf of one tile
+constexpr int CT = 128;                      // tokens per S tile
+constexpr int XT = 64;                       // tokens per X tile
+constexpr int NK = 2;                        // K ring depth
+constexpr int NX = 3;                        // X ring depth
+constexpr int NSB = 2;                       // S/P buffers
+constexpr int KSLOT = 2 * SLAB_BYTES;        // 128 rows x 2 slabs (a K tile or T_ii)
+constexpr int XSLAB = XT * 128;              // one 64-row slab
+constexpr int XSLOT = 4 * XSLAB;             // 64 rows x 4 slabs
+constexpr int GCT_FLOATS = 2 * CT;           // G[128], cf[128] of a tile
 
 struct Smem {
-    static constexpr uint32_t KI = 0;                          // 2 slabs x 128 rows
-    static constexpr uint32_t T = KI + 2 * SLAB_BYTES;         // 2 slabs x 128 rows
-    static constexpr uint32_t RING = T + 2 * SLAB_BYTES;       // NSLOT x 48 KB; Y_i (64 KB) aliases the start
-    static constexpr uint32_t GC = RING + NSLOT * SLOT_BYTES;  // NSLOT x (G[64], cf[64])
-    static constexpr uint32_t END = GC + NSLOT * GC_BYTES;
+    static constexpr uint32_t KI = 0;                       // 128 rows x 2 slabs
+    static constexpr uint32_t KR = KI + 2 * SLAB_BYTES;     // NK x 32 KB
+    static constexpr uint32_t XR = KR + NK * KSLOT;         // NX x 32 KB; Y_i / X_i use the first 64 KB
+    static constexpr uint32_t GC = XR + NX * XSLOT;         // NK x (G[128], cf[128])
+    static constexpr uint32_t END = GC + NK * GCT_FLOATS * 4;
 };
-static_assert(2 * SLOT_BYTES >= 4 * SLAB_BYTES, "Y_i must fit in the first two ring slots");
+static_assert(2 * XSLOT == 4 * SLAB_BYTES, "Y_i must fill the first two X slots exactly");
 
 enum Bar {
-    KIFULL = 0, TFULL, ACCFULL, YFULL, XFULL, ACCFREE, XSTAGED,
-    KXFULL, KXEMPTY = KXFULL + NSLOT, SFULL = KXEMPTY + NSLOT, SFREE = SFULL + NSB, PFULL = SFREE + NSB,
-    NBAR = PFULL + NSB
+    KIFULL = 0, KIEMPTY, ACCFULL, YFULL, XFULL, XSTAGED,
+    KRFULL, KREMPTY = KRFULL + NK, XRFULL = KREMPTY + NK, XREMPTY = XRFULL + NX,
+    SFULL = XREMPTY + NX, SFREE = SFULL + NSB, PFULL = SFREE + NSB, NBAR = PFULL + NSB
 };
 
+__device__ __forceinline__ uint32_t yx_offset(int c, int r) {  // bf16 column c, row r of Y_i / X_i
+    return (uint32_t)((c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_x,
-           const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_g,
-           const __grid_constant__ CUtensorMap tm_cf, const __grid_constant__ CUtensorMap tm_xs,
-           const IntraParams prm) {
+k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_x64,
+           const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_gct,
+           const __grid_constant__ CUtensorMap tm_xs, const IntraParams prm) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
@@ -69,11 +80,9 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     const int bf = (int)(b * F + f);
 
     unsigned char *sKi = smem + Smem::KI;
-    unsigned char *sT = smem + Smem::T;
-    unsigned char *sRing = smem + Smem::RING;
-    unsigned char *sY = sRing;
-    unsigned char *sXs = smem + Smem::KI;  // X_i staging: K_i and T_ii, 4 slabs of 128 rows
-    static_assert(Smem::T == Smem::KI + 2 * SLAB_BYTES, "the staging slabs must be contiguous");
+    unsigned char *sKR = smem + Smem::KR;
+    unsigned char *sXR = smem + Smem::XR;
+    unsigned char *sYX = sXR;  // Y_i, then the staged X_i
     float *sGC = (float *)(smem + Smem::GC);
     uint64_t *bars = (uint64_t *)(smem + Smem::END);
     uint32_t *tmem_slot = (uint32_t *)(bars + NBAR);
@@ -83,8 +92,10 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) {
-            const bool epi = i == YFULL || i == ACCFREE || i == XSTAGED || (i >= PFULL && i < PFULL + NSB);
-            sm100::mbar_init(&bars[i], epi ? kEpi : 1);
+            uint32_t cnt = 1;
+            if (i == KIEMPTY || i == YFULL || i == XSTAGED || (i >= PFULL && i < PFULL + NSB)) cnt = kEpi;
+            if (i >= KREMPTY && i < KREMPTY + NK) cnt = 1 + kEpi;  // the MMA's commit + the epilogue
+            sm100::mbar_init(&bars[i], cnt);
         }
         sm100::fence_barrier_init();
     }
@@ -96,68 +107,79 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t t_s0 = tbase, t_acc = tbase + 256;
+    const uint32_t t_s0 = tbase, t_acc = tbase + NSB * CT;
     const int nks_d = dk / 16;
     const int nslab_k = (dk + SLAB - 1) / SLAB;
     const int nslab_x = (nc + SLAB - 1) / SLAB;
+    const int nt128 = (L + CT - 1) / CT;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             sm100::tma_prefetch_desc(&tm_k);
-            sm100::tma_prefetch_desc(&tm_x);
+            sm100::tma_prefetch_desc(&tm_x64);
             sm100::tma_prefetch_desc(&tm_t);
-            sm100::tma_prefetch_desc(&tm_g);
-            sm100::tma_prefetch_desc(&tm_cf);
+            sm100::tma_prefetch_desc(&tm_gct);
             sm100::tma_prefetch_desc(&tm_xs);
             bool ok = true;
-            int n = 0;
-            auto load_tile = [&](int jt, int i) -> bool {
-                const int st = n % NSLOT;
-                if (n >= NSLOT && !sm100::mbar_wait(&bars[KXEMPTY + st], ((n / NSLOT) - 1) & 1, err)) return false;
-                if (jt == 2 * (i - 1)) sm100::bulk_wait0();  // the rows of X_{i-1} are in global memory
-                unsigned char *slot = sRing + st * SLOT_BYTES;
-                sm100::mbar_arrive_expect_tx(&bars[KXFULL + st], (uint32_t)((nslab_k + nslab_x) * KJ_SLAB + GC_BYTES));
-                for (int sl = 0; sl < nslab_k; ++sl)
-                    sm100::tma_load_4d(slot + sl * KJ_SLAB, &tm_k, &bars[KXFULL + st], sl * SLAB, h, jt * JT, bf);
-                for (int sl = 0; sl < nslab_x; ++sl)
-                    sm100::tma_load_3d(slot + (2 + sl) * KJ_SLAB, &tm_x, &bars[KXFULL + st], sl * SLAB, jt * JT,
-                                       (int)fh);
-                float *gc = sGC + st * 2 * JT;
-                sm100::tma_load_2d(gc, &tm_g, &bars[KXFULL + st], jt * JT, (int)fh);
-                sm100::tma_load_2d(gc + JT, &tm_cf, &bars[KXFULL + st], jt * JT, (int)fh);
-                ++n;
+            int kn = 0, xn = 0;
+            // K-ring item: the K tile of S tile c with its G and cf, or T_ii (c < 0)
+            auto load_k = [&](int c, int i) -> bool {
+                const int st = kn % NK;
+                if (kn >= NK && !sm100::mbar_wait(&bars[KREMPTY + st], ((kn / NK) - 1) & 1, err)) return false;
+                unsigned char *slot = sKR + st * KSLOT;
+                if (c >= 0) {
+                    sm100::mbar_arrive_expect_tx(&bars[KRFULL + st],
+                                                 (uint32_t)(nslab_k * SLAB_BYTES + GCT_FLOATS * 4));
+                    for (int sl = 0; sl < nslab_k; ++sl)
+                        sm100::tma_load_4d(slot + sl * SLAB_BYTES, &tm_k, &bars[KRFULL + st], sl * SLAB, h, c * CT,
+                                           bf);
+                    sm100::tma_load_2d(sGC + st * GCT_FLOATS, &tm_gct, &bars[KRFULL + st], 0,
+                                       (int)(fh * nt128 + c));
+                } else {
+                    sm100::mbar_arrive_expect_tx(&bars[KRFULL + st], (uint32_t)(2 * SLAB_BYTES));
+                    for (int sl = 0; sl < 2; ++sl)
+                        sm100::tma_load_3d(slot + sl * SLAB_BYTES, &tm_t, &bars[KRFULL + st], sl * SLAB, 0,
+                                           (int)(fh * nblk + i));
+                }
+                ++kn;
                 return true;
             };
-            // store the staged X_{i}: rows past the frame and columns past d_v + d_k are clipped
+            auto load_x = [&](int x, int i) -> bool {
+                const int st = xn % NX;
+                if (xn >= NX && !sm100::mbar_wait(&bars[XREMPTY + st], ((xn / NX) - 1) & 1, err)) return false;
+                if (x >= 2 * (i - 1)) sm100::bulk_wait0();  // the rows of X_{i-1} are in global memory
+                unsigned char *slot = sXR + st * XSLOT;
+                sm100::mbar_arrive_expect_tx(&bars[XRFULL + st], (uint32_t)(nslab_x * XSLAB));
+                for (int sl = 0; sl < nslab_x; ++sl)
+                    sm100::tma_load_3d(slot + sl * XSLAB, &tm_x64, &bars[XRFULL + st], sl * SLAB, x * XT, (int)fh);
+                ++xn;
+                return true;
+            };
+            // store the staged X_i (rows past the frame and columns past d_v + d_k are clipped)
             auto store_x = [&](int i) -> bool {
                 if (!sm100::mbar_wait(&bars[XSTAGED], i & 1, err)) return false;
                 for (int sl = 0; sl < nslab_x; ++sl)
-                    sm100::tma_store_3d(&tm_xs, sXs + sl * SLAB_BYTES, sl * SLAB, i * BM, (int)fh);
+                    sm100::tma_store_3d(&tm_xs, sYX + sl * SLAB_BYTES, sl * SLAB, i * BM, (int)fh);
                 sm100::bulk_commit();
                 sm100::bulk_wait_read0();
                 return true;
             };
             for (int i = 0; i < nblk && ok; ++i) {
-                int jt = 0;
-                if (i >= 1) {
-                    // Y_{i-1} is consumed once X_{i-1} = T Y is in TMEM: the ring may refill
-                    ok = sm100::mbar_wait(&bars[XFULL], (i - 1) & 1, err);
-                    const int pre = min(2 * i - 2, NSLOT);  // tiles that do not read X_{i-1}
-                    for (; jt < pre && ok; ++jt) ok = load_tile(jt, i);
-                    // K_i and T_ii overwrite the staging buffer once the store has read it
-                    if (ok) ok = store_x(i - 1);
-                }
+                // K_i once the previous block's Y build has read K_{i-1}
+                if (i >= 1) ok = sm100::mbar_wait(&bars[KIEMPTY], (i - 1) & 1, err);
                 if (!ok) break;
                 sm100::mbar_arrive_expect_tx(&bars[KIFULL], (uint32_t)(nslab_k * SLAB_BYTES));
                 for (int sl = 0; sl < nslab_k; ++sl)
-                    for (int hf = 0; hf < 2; ++hf)
-                        sm100::tma_load_4d(sKi + sl * SLAB_BYTES + hf * KJ_SLAB, &tm_k, &bars[KIFULL], sl * SLAB, h,
-                                           i * BM + hf * JT, bf);
-                sm100::mbar_arrive_expect_tx(&bars[TFULL], (uint32_t)(2 * SLAB_BYTES));
-                for (int sl = 0; sl < 2; ++sl)
-                    sm100::tma_load_3d(sT + sl * SLAB_BYTES, &tm_t, &bars[TFULL], sl * SLAB, 0, (int)(fh * nblk + i));
-                for (; jt < 2 * i && ok; ++jt) ok = load_tile(jt, i);
+                    sm100::tma_load_4d(sKi + sl * SLAB_BYTES, &tm_k, &bars[KIFULL], sl * SLAB, h, i * BM, bf);
+                for (int c = 0; c < i && ok; ++c) {
+                    ok = load_k(c, i);
+                    // the X ring refills the Y / X_{i-1} buffer only after X_{i-1} has been stored
+                    if (ok && c == 0) ok = store_x(i - 1);
+                    if (ok) ok = load_x(2 * c, i);
+                    if (ok) ok = load_x(2 * c + 1, i);
+                }
+                if (ok) ok = load_k(-1, i);  // T_ii
             }
             if (ok) ok = store_x(nblk - 1);
             sm100::bulk_wait0();  // leave with no store in flight
@@ -165,104 +187,117 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t id_s = sm100::idesc_bf16(BM, JT, 0, 0);
+            const uint32_t id_s = sm100::idesc_bf16(BM, CT, 0, 0);
             const uint32_t id_x = sm100::idesc_bf16(BM, nc, 0, 1);
             bool ok = true;
-            int n = 0;
-            auto issue_px = [&](int m, bool first_of_block, int i) -> bool {
-                const int pb = m % NSB, st = m % NSLOT;
-                if (!sm100::mbar_wait(&bars[PFULL + pb], (m / NSB) & 1, err)) return false;
-                // the first product of a block overwrites acc: X_{i-1} must have been read out
-                if (first_of_block && i >= 1 && !sm100::mbar_wait(&bars[ACCFREE], (i - 1) & 1, err)) return false;
-                sm100::tc_fence_after();
-                const unsigned char *xt = sRing + st * SLOT_BYTES + 2 * KJ_SLAB;
-                // P columns k = 0..31 sit in TMEM columns 0..15, k = 32..63 in columns 32..47
-                for (int ks = 0; ks < JT / 16; ++ks)
-                    sm100::mma_bf16_ts(t_acc, t_s0 + pb * JT + ks * 8 + (ks >> 1) * 16, desc_mnmajor(xt, ks, JT),
-                                       id_x, (first_of_block && ks == 0) ? 0u : 1u);
-                sm100::mma_commit(&bars[SFREE + pb]);
-                sm100::mma_commit(&bars[KXEMPTY + st]);
+            int kn = 0, xn = 0, sn = 0;  // K-ring item, X-ring item, S tile counters
+            // acc += P X for S tile c (its buffer sb): the two 64-token X tiles in turn; P of
+            // tokens 0..63 sits in TMEM columns 0..31 of the buffer, tokens 64..127 in 64..95
+            auto issue_px = [&](int sb, int s_idx, bool first, int i) -> bool {
+                if (!sm100::mbar_wait(&bars[PFULL + sb], (s_idx / NSB) & 1, err)) return false;
+                // the block's first product overwrites acc: X_{i-1} must have been read out
+                if (first && i >= 1 && !sm100::mbar_wait(&bars[XSTAGED], (i - 1) & 1, err)) return false;
+                for (int hx = 0; hx < 2; ++hx) {
+                    const int st = xn % NX;
+                    if (!sm100::mbar_wait(&bars[XRFULL + st], (xn / NX) & 1, err)) return false;
+                    sm100::tc_fence_after();
+                    const unsigned char *xt = sXR + st * XSLOT;
+                    for (int ks = 0; ks < XT / 16; ++ks)
+                        sm100::mma_bf16_ts(t_acc, t_s0 + sb * CT + 64 * hx + ks * 8, desc_mnmajor(xt, ks, XT), id_x,
+                                           (first && hx == 0 && ks == 0) ? 0u : 1u);
+                    sm100::mma_commit(&bars[XREMPTY + st]);
+                    ++xn;
+                }
+                sm100::mma_commit(&bars[SFREE + sb]);
                 return true;
             };
             for (int i = 0; i < nblk && ok; ++i) {
                 ok = sm100::mbar_wait(&bars[KIFULL], i & 1, err);
-                const int first = n;
-                for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
-                    const int st = n % NSLOT, sb = n % NSB;
-                    ok = sm100::mbar_wait(&bars[KXFULL + st], (n / NSLOT) & 1, err);
-                    if (ok && n >= NSB) ok = sm100::mbar_wait(&bars[SFREE + sb], ((n / NSB) - 1) & 1, err);
+                int prev_sb = -1, prev_idx = 0;
+                for (int c = 0; c < i && ok; ++c, ++kn, ++sn) {
+                    const int st = kn % NK, sb = sn % NSB;
+                    ok = sm100::mbar_wait(&bars[KRFULL + st], (kn / NK) & 1, err);
+                    if (ok && sn >= NSB) ok = sm100::mbar_wait(&bars[SFREE + sb], ((sn / NSB) - 1) & 1, err);
                     if (!ok) break;
                     sm100::tc_fence_after();
-                    const unsigned char *kt = sRing + st * SLOT_BYTES;
+                    const unsigned char *kt = sKR + st * KSLOT;
                     for (int ks = 0; ks < nks_d; ++ks)
-                        sm100::mma_bf16_ss(t_s0 + sb * JT, desc_kmajor(sKi, ks, BM), desc_kmajor(kt, ks, JT), id_s,
+                        sm100::mma_bf16_ss(t_s0 + sb * CT, desc_kmajor(sKi, ks, BM), desc_kmajor(kt, ks, CT), id_s,
                                            ks > 0);
                     sm100::mma_commit(&bars[SFULL + sb]);
-                    if (jt >= 1) ok = issue_px(n - 1, n - 1 == first, i);
+                    sm100::mma_commit(&bars[KREMPTY + st]);
+                    // one S tile behind: the tensor cores compute S(c) while the epilogue writes P(c-1)
+                    if (prev_sb >= 0) ok = issue_px(prev_sb, prev_idx, c == 1, i);
+                    prev_sb = sb;
+                    prev_idx = sn;
                 }
-                if (ok && i >= 1) ok = issue_px(n - 1, n - 1 == first, i);
+                if (ok && prev_sb >= 0) ok = issue_px(prev_sb, prev_idx, i == 1, i);
                 if (!ok) break;
                 sm100::mma_commit(&bars[ACCFULL]);
-                ok = sm100::mbar_wait(&bars[YFULL], i & 1, err) && sm100::mbar_wait(&bars[TFULL], i & 1, err);
+                // X_i = T_ii Y_i; T_ii is the block's last K-ring item
+                const int st = kn % NK;
+                ok = sm100::mbar_wait(&bars[KRFULL + st], (kn / NK) & 1, err) &&
+                     sm100::mbar_wait(&bars[YFULL], i & 1, err);
                 if (!ok) break;
                 sm100::tc_fence_after();
+                const unsigned char *tt = sKR + st * KSLOT;
                 for (int ks = 0; ks < BM / 16; ++ks)
-                    sm100::mma_bf16_ss(t_acc, desc_kmajor(sT, ks, BM), desc_mnmajor(sY, ks, BM), id_x, ks > 0);
+                    sm100::mma_bf16_ss(t_acc, desc_kmajor(tt, ks, BM), desc_mnmajor(sYX, ks, BM), id_x, ks > 0);
                 sm100::mma_commit(&bars[XFULL]);
+                sm100::mma_commit(&bars[KREMPTY + st]);
+                ++kn;
             }
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Two warpgroups: each thread owns one block row (TMEM lane quadrant =
-        // warp % 4) and one half of the columns -- 32 of the 64 columns of an
-        // off-diagonal tile, and in the diagonal step the Ub columns (half 0,
-        // which needs v) or the W columns (half 1, which needs k).
         const int q4 = warp & 3;
         const int half = (warp - 2) >> 2;
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
-
         bool ok = true;
-        int n = 0;
+        int kn = 0, sn = 0;
         for (int i = 0; i < nblk && ok; ++i) {
             const int row = i * BM + r;
             const bool valid = row < L;
             const float Gr = valid ? Gf[row] : 0.f;
-            const long long t = f * L + row;
-            const long long tok = ((long long)b * prm.T + t) * prm.H + h;
+            const long long tok = ((long long)b * prm.T + f * L + row) * prm.H + h;
             const float be = valid ? prm.beta[tok] : 0.f;
             // half 0 needs this row's values in the diagonal step: pull them into L2 now
             const __nv_bfloat16 *vp = prm.v + tok * dv;
-            if (half == 0 && valid)
-                for (int by = 0; by < dv * 2; by += 128)
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"((const char *)vp + by));
-            if (half == 0 && valid) asm volatile("prefetch.global.L2 [%0];" ::"l"((const char *)vp + dv * 2 - 1));
-
-            for (int jt = 0; jt < 2 * i && ok; ++jt, ++n) {
-                const int sb = n % NSB, st = n % NSLOT;
-                ok = sm100::mbar_wait(&bars[SFULL + sb], (n / NSB) & 1, err) &&
-                     sm100::mbar_wait(&bars[KXFULL + st], (n / NSLOT) & 1, err);  // G_j, cf_j
+            if (half == 0 && valid) {
+                for (int by = 0; by < dv * 2; by += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"((const char *)vp + by));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"((const char *)vp + dv * 2 - 1));
+            }
+            // ---- S tiles -> P = -beta_r e^{G_r - G_s} S (this half: tile columns 64 half .. 64 half + 63)
+            for (int c = 0; c < i && ok; ++c, ++kn, ++sn) {
+                const int sb = sn % NSB, st = kn % NK;
+                ok = sm100::mbar_wait(&bars[SFULL + sb], (sn / NSB) & 1, err) &&
+                     sm100::mbar_wait(&bars[KRFULL + st], (kn / NK) & 1, err);  // G, cf of the tile
                 if (!ok) break;
                 sm100::tc_fence_after();
-                // the tile is full (it lies before block i): its anchor is G at token 63
-                const float *gj = sGC + st * 2 * JT;
-                const float rf = valid ? -be * __expf(Gr - gj[JT - 1]) : 0.f;
-                const float *cf = gj + JT + 32 * half;
-                float v[32];
-                sm100::tmem_ld32(t_s0 + sb * JT + lane_off + 32 * half, v);
-                sm100::tmem_ld_wait();
-                uint32_t pk[16];
+                const float *gJ = sGC + st * GCT_FLOATS, *cfJ = gJ + CT;
+                // the tile lies before block i, so it is full: the half's anchor is G at its last token
+                const float rf = valid ? -be * __expf(Gr - gJ[64 * half + 63]) : 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) pk[e >> 1] = pack_bf16(rf * cf[e] * v[e], rf * cf[e + 1] * v[e + 1]);
-                // this half's P goes to TMEM columns [32 half, 32 half + 16): S columns it has read
-                sm100::tmem_st16(t_s0 + sb * JT + lane_off + 32 * half, pk);
+                for (int rr = 0; rr < 2; ++rr) {  // two rounds of 32 columns: S read before P overwrites it
+                    const int c0 = 64 * half + 32 * rr;
+                    float v[32];
+                    sm100::tmem_ld32(t_s0 + sb * CT + lane_off + c0, v);
+                    sm100::tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        pk[e >> 1] = pack_bf16(rf * cfJ[c0 + e] * v[e], rf * cfJ[c0 + e + 1] * v[e + 1]);
+                    sm100::tmem_st16(t_s0 + sb * CT + lane_off + 64 * half + 16 * rr, pk);
+                }
                 sm100::tmem_st_wait();
                 sm100::tc_fence_before();
                 sm100::mbar_arrive(&bars[PFULL + sb]);
+                sm100::mbar_arrive(&bars[KREMPTY + st]);  // done with the slot's G and cf
             }
             if (!ok) break;
-            // ---- Y_i = R_i + acc_i  -> sY (MN-major: row = K index of the T_ii Y_i product)
+            // ---- Y_i = R_i + acc_i  -> sYX (MN-major: row = K index of the T_ii Y_i product)
             ok = sm100::mbar_wait(&bars[ACCFULL], i & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
@@ -270,7 +305,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 const uint4 val = valid ? make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]),
                                                      pack_bf16(y[4], y[5]), pack_bf16(y[6], y[7]))
                                         : make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4 *>(sY + (c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4)) = val;
+                *reinterpret_cast<uint4 *>(sYX + yx_offset(c, r)) = val;
             };
             if (half == 0) {  // Ub columns: beta_r v_r + acc
                 uint4 vrow[16];
@@ -320,8 +355,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int kc = kc16 + 8 * u;
-                        const uint4 kv = *reinterpret_cast<const uint4 *>(
-                            sKi + (kc >> 6) * SLAB_BYTES + r * 128 + ((((kc & 63) >> 3) ^ (r & 7)) << 4));
+                        const uint4 kv = *reinterpret_cast<const uint4 *>(sKi + yx_offset(kc, r));
                         const __nv_bfloat162 *kb = reinterpret_cast<const __nv_bfloat162 *>(&kv);
                         float y[8];
 #pragma unroll
@@ -337,7 +371,10 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();
             sm100::mbar_arrive(&bars[YFULL]);
-            // ---- X_i = T_ii Y_i  -> bf16 staging (same layout as Y; half 0 the Ub columns, half 1 the W columns)
+            sm100::mbar_arrive(&bars[KIEMPTY]);
+            sm100::mbar_arrive(&bars[KREMPTY + kn % NK]);  // the T_ii slot: released when T Y completes
+            ++kn;
+            // ---- X_i = T_ii Y_i -> bf16 staging over Y_i (half 0 the Ub columns, half 1 the W columns)
             ok = sm100::mbar_wait(&bars[XFULL], i & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
@@ -347,15 +384,12 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 sm100::tmem_ld16(t_acc + lane_off + c16, x);
                 sm100::tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int c = c16 + 8 * u;
-                    *reinterpret_cast<uint4 *>(sXs + (c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4)) =
+                for (int u = 0; u < 2; ++u)
+                    *reinterpret_cast<uint4 *>(sYX + yx_offset(c16 + 8 * u, r)) =
                         make_uint4(pack_bf16(x[8 * u], x[8 * u + 1]), pack_bf16(x[8 * u + 2], x[8 * u + 3]),
                                    pack_bf16(x[8 * u + 4], x[8 * u + 5]), pack_bf16(x[8 * u + 6], x[8 * u + 7]));
-                }
             }
             sm100::tc_fence_before();
-            sm100::mbar_arrive(&bars[ACCFREE]);
             sm100::fence_proxy_async_smem();
             sm100::mbar_arrive(&bars[XSTAGED]);
         }
@@ -370,13 +404,13 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
 }  // namespace
 
-cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_t,
-                            const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const CUtensorMap &tm_xs,
-                            const IntraParams &prm, long long n_fh, cudaStream_t s) {
+cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x64, const CUtensorMap &tm_t,
+                            const CUtensorMap &tm_gct, const CUtensorMap &tm_xs, const IntraParams &prm,
+                            long long n_fh, cudaStream_t s) {
     const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
     cudaError_t e = cudaFuncSetAttribute(k_intra_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_t, tm_g, tm_cf, tm_xs, prm);
+    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x64, tm_t, tm_gct, tm_xs, prm);
     return cudaGetLastError();
 }
 

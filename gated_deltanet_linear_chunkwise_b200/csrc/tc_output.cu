@@ -10,23 +10,26 @@
 // block) items (ranges balanced by tile count), so a frame's K and U tiles
 // come from HBM once and are re-read from L2 by the same CTA for the frame's
 // other blocks; TMEM and barriers are set up once.  The columns s come in
-// 64-token tiles through a 4-deep ring; the MMA thread issues each tile's
+// 128-token tiles through a 2-deep ring (a tensor-core instruction costs the
+// same for every N up to 128, so S = Q K^T is issued with N = 128); the MMA
+// thread issues each tile's
 // S = Q K^T as soon as its data and an S/P buffer are there and each O += P U
 // as soon as the epilogue has written P (polling both in one loop).
 // Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
 // issues tcgen05.mma from one thread, warps 2-9 are the epilogue: two
 // warpgroups, each thread owning one tile row (TMEM lane quadrant =
-// warp % 4) and one 32-column half of each tile.
-//   TMEM: four S/P buffers (64 columns each) and two O buffers (128 each).
+// warp % 4) and one 64-column half of each tile.
+//   TMEM: two S/P buffers (128 columns each) and two O buffers (128 each).
 //         The epilogue turns S (fp32) into P (bf16) in place -- each half
-//         into the first 16 TMEM columns of its own range -- and O += P U
+//         into the first 32 TMEM columns of its own range -- and O += P U
 //         reads P straight from tensor memory.
-//   SMEM: Q_I double buffer; 4 ring slots of (K_j, U_j) + (G_j, cf_j).
+//   SMEM: Q_I double buffer; 2 ring slots of (K_j, U_j) + (G_j, cf_j).
 // The state term is a pseudo-tile in front of the column tiles: the epilogue
 // writes Q~ = diag(e^G) Q_I into an S/P buffer and a ring slot delivers Sig
 // (bf16, MN-major), so O starts as Q~ Sig.  Off-diagonal decay factors are
 // e^{G_r - a} cf_s with cf_s = e^{a - G_s} (a = G at the tile's last token,
-// both <= 1); the two diagonal tiles take e^{G_r - G_s} per element.  Every
+// both <= 1, a per 64-token half); the diagonal tile takes e^{G_r - G_s} per
+// element.  Every
 // wait is bounded (sm100::mbar_wait).
 #include "tc_common.cuh"
 
@@ -36,17 +39,17 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kEpi = 256;                 // epilogue threads
-constexpr int JT = 64;                    // tokens per column tile
-constexpr int NSLOT = 4;                  // ring depth
-constexpr int NSB = 4;                    // S/P buffers in TMEM
-constexpr int JSLAB = JT * 128;           // one 64-row slab
+constexpr int JT = 128;                   // tokens per column tile (= BM: tile I is block I's diagonal)
+constexpr int NSLOT = 2;                  // ring depth
+constexpr int NSB = 2;                    // S/P buffers in TMEM
+constexpr int JSLAB = JT * 128;           // one 128-row slab
 constexpr int SLOT_BYTES = 4 * JSLAB;     // K (2 slabs) + U (2 slabs); Sig (<= 32 KB) fills a whole slot
 constexpr int GC_BYTES = 2 * JT * 4;      // G and cf of one tile
 
 struct Smem {
     static constexpr uint32_t Q = 0;                          // 2 stages x 2 slabs x 128 rows
-    static constexpr uint32_t RING = Q + 4 * SLAB_BYTES;      // NSLOT x 32 KB
-    static constexpr uint32_t GC = RING + NSLOT * SLOT_BYTES; // NSLOT x (G[64], cf[64])
+    static constexpr uint32_t RING = Q + 4 * SLAB_BYTES;      // NSLOT x 64 KB
+    static constexpr uint32_t GC = RING + NSLOT * SLOT_BYTES; // NSLOT x (G[128], cf[128])
     static constexpr uint32_t END = GC + NSLOT * GC_BYTES;
 };
 
@@ -96,10 +99,10 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
 
     // item w: frame-head w / nblk, block nblk-1 - w % nblk (heaviest block of a frame first);
-    // its column tiles are j = 0 .. min(2I+2, ceil(L/64)) - 1, the last two being diagonal
+    // its column tiles are j = 0 .. I, the last one being the diagonal block
     auto item_blk = [&](long long w) { return nblk - 1 - (int)(w % nblk); };
     auto item_fh = [&](long long w) { return w / nblk; };
-    auto item_ntiles = [&](int I) { return min(2 * I + 2, ntile_frame); };
+    auto item_ntiles = [&](int I) { return min(I + 1, ntile_frame); };
     // CTA c takes items [item_start(c), item_start(c + 1)): equal shares of the
     // total weight, an item weighing its tiles plus two (state term, drain)
     auto item_start = [&](long long c) -> long long {
@@ -225,9 +228,9 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         if (sm100::mbar_test(&bars[PFULL + pb], (cs / NSB) & 1)) {
                             sm100::tc_fence_after();
                             const unsigned char *u = sRing + pst * SLOT_BYTES + 2 * JSLAB;
-                            // P columns k = 0..31 sit in TMEM columns 0..15, k = 32..63 in columns 32..47
+                            // P columns k = 0..63 sit in TMEM columns 0..31, k = 64..127 in columns 64..95
                             for (int ks = 0; ks < JT / 16; ++ks)
-                                sm100::mma_bf16_ts(t_o, t_s0 + pb * JT + ks * 8 + (ks >> 1) * 16,
+                                sm100::mma_bf16_ts(t_o, t_s0 + pb * JT + ks * 8 + (ks >> 2) * 32,
                                                    desc_mnmajor(u, ks, JT), id_o, 1u);
                             sm100::mma_commit(&bars[SFREE + pb]);
                             sm100::mma_commit(&bars[REMPTY + pst]);
@@ -313,32 +316,42 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         auto tiles = [&](const Item &it) -> bool {
             for (int j = 0; j < it.nt; ++j, ++sc, ++n) {
                 const int sb = sc % NSB, st = n % NSLOT;
-                const bool diag = (j >= 2 * it.I);
+                const bool diag = (j == it.I);
                 if (!sm100::mbar_wait(&bars[SFULL + sb], (sc / NSB) & 1, err)) return false;
                 if (!sm100::mbar_wait(&bars[RFULL + st], (n / NSLOT) & 1, err)) return false;  // G, cf
                 sm100::tc_fence_after();
                 const float *gJ = sGC + st * 2 * JT, *cfJ = gJ + JT;
-                float v[32];
-                sm100::tmem_ld32(t_s0 + sb * JT + lane_off + 32 * half, v);
-                sm100::tmem_ld_wait();
-                uint32_t pk[16];
-                if (!diag) {
-                    const float rf = it.valid ? __expf(it.Gr - gJ[JT - 1]) : 0.f;
+                // In the diagonal tile, a row below the half's 64-token group sees all of it
+                // (anchored split as off the diagonal), a row above sees none of it, and only
+                // the group's own rows need the exact per-element factor.
+                const bool none = diag && r < 64 * half;
+                const bool exact = diag && !none && r < 64 * half + 64;
+                // split: the half's anchor is G at the end of its 64-token group
+                const float rf = (it.valid && !none && !exact) ? __expf(it.Gr - gJ[64 * half + 63]) : 0.f;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2)
-                        pk[e >> 1] = pack_bf16(v[e] * rf * cfJ[32 * half + e], v[e + 1] * rf * cfJ[32 * half + e + 1]);
-                } else {
+                for (int rr = 0; rr < 2; ++rr) {  // two rounds of 32 columns: S read before P overwrites it
+                    const int c0 = 64 * half + 32 * rr;
+                    float v[32];
+                    sm100::tmem_ld32(t_s0 + sb * JT + lane_off + c0, v);
+                    sm100::tmem_ld_wait();
+                    uint32_t pk[16];
+                    if (!exact) {  // rf = 0 where the row sees none of the half
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int s = j * JT + 32 * half + e;
-                        const float f0 = (s <= it.row && s < L) ? __expf(it.Gr - gJ[32 * half + e]) : 0.f;
-                        const float f1 =
-                            (s + 1 <= it.row && s + 1 < L) ? __expf(it.Gr - gJ[32 * half + e + 1]) : 0.f;
-                        pk[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
+                        for (int e = 0; e < 32; e += 2)
+                            pk[e >> 1] = pack_bf16(v[e] * rf * cfJ[c0 + e], v[e + 1] * rf * cfJ[c0 + e + 1]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const int s0 = j * JT + c0 + e;
+                            const float f0 = (s0 <= it.row && s0 < L) ? __expf(it.Gr - gJ[c0 + e]) : 0.f;
+                            const float f1 =
+                                (s0 + 1 <= it.row && s0 + 1 < L) ? __expf(it.Gr - gJ[c0 + e + 1]) : 0.f;
+                            pk[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
+                        }
                     }
+                    // P of this half goes to TMEM columns [64 half, 64 half + 32): S columns it has read
+                    sm100::tmem_st16(t_s0 + sb * JT + lane_off + 64 * half + 16 * rr, pk);
                 }
-                // this half's P goes to TMEM columns [32 half, 32 half + 16): S columns it has read
-                sm100::tmem_st16(t_s0 + sb * JT + lane_off + 32 * half, pk);
                 sm100::tmem_st_wait();
                 sm100::tc_fence_before();
                 sm100::mbar_arrive(&bars[PFULL + sb]);
@@ -415,7 +428,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
 }  // namespace
 
-cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k64, const CUtensorMap &tm_u64,
+cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
                              const CUtensorMap &tm_sig, const CUtensorMap &tm_g, const CUtensorMap &tm_cf,
                              const OutParams &prm, int num_sms, cudaStream_t s) {
     const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
@@ -423,7 +436,7 @@ cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k64,
     if (e != cudaSuccess) return e;
     const long long nitems = prm.n_fh * prm.nblk;
     const long long grid = nitems < num_sms ? nitems : num_sms;
-    k_output_tc<<<(unsigned)grid, kThreads, smem, s>>>(tm_q, tm_k64, tm_u64, tm_sig, tm_g, tm_cf, prm);
+    k_output_tc<<<(unsigned)grid, kThreads, smem, s>>>(tm_q, tm_k, tm_u, tm_sig, tm_g, tm_cf, prm);
     return cudaGetLastError();
 }
 
