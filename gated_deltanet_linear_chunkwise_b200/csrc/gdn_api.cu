@@ -4,8 +4,10 @@
 // call returns its status with no launch and no output touched.  No C++
 // exception crosses the ABI (every entry point is noexcept and catches).
 #include <cstdarg>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "gdn_internal.h"
@@ -20,6 +22,39 @@ void set_err(const char *fmt, ...) {
     va_start(ap, fmt);
     vsnprintf(g_err, sizeof(g_err), fmt, ap);
     va_end(ap);
+}
+
+// The library's own scratch (the workspace when the caller passes none, and
+// gdn_fwd_host's device copies) comes from one stream-ordered pool per
+// device whose release threshold is unlimited: memory freed at the end of a
+// call stays reserved for the next one instead of being unmapped, so a
+// repeated call does not pay for mapping gigabytes again.
+cudaError_t scratch_alloc(void **ptr, size_t bytes, cudaStream_t s) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[128] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 128) return cudaMallocAsync(ptr, bytes, s);
+    cudaMemPool_t pool;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!pools[dev]) {
+            cudaMemPoolProps props;
+            memset(&props, 0, sizeof(props));
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            if ((e = cudaMemPoolCreate(&pools[dev], &props)) != cudaSuccess) {
+                pools[dev] = nullptr;
+                return e;
+            }
+            uint64_t keep = UINT64_MAX;
+            cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        pool = pools[dev];
+    }
+    return cudaMallocFromPoolAsync(ptr, bytes, pool, s);
 }
 
 bool misaligned(const void *ptr) { return ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u); }
@@ -180,10 +215,10 @@ int run(const gdn_args &a) noexcept {
                 return GDN_ERR_NO_MEMORY;
             }
         } else {
-            cudaError_t e = cudaMallocAsync(&ws, need, s);
+            cudaError_t e = scratch_alloc(&ws, need, s);
             if (e != cudaSuccess || !ws) {
                 cudaGetLastError();
-                set_err("cudaMallocAsync(%zu bytes) failed: %s", need, cudaGetErrorString(e));
+                set_err("device scratch allocation (%zu bytes) failed: %s", need, cudaGetErrorString(e));
                 return GDN_ERR_NO_MEMORY;
             }
             owned = true;
@@ -341,10 +376,10 @@ int gdn_fwd_host(int dtype, const void *q, const void *k, const void *v, const f
         for (int i = 0; i < 8; ++i) off[i + 1] = off[i] + ((sz[i] + 255) & ~(size_t)255);
         const size_t wsb = gdn_workspace_bytes(B, H, T, frame_len, d_k, d_v, dtype);
         char *dev = nullptr;
-        cudaError_t e = cudaMallocAsync((void **)&dev, off[8] + wsb, s);
+        cudaError_t e = scratch_alloc((void **)&dev, off[8] + wsb, s);
         if (e != cudaSuccess || !dev) {
             cudaGetLastError();
-            set_err("cudaMallocAsync(%zu bytes) failed: %s", off[8] + wsb, cudaGetErrorString(e));
+            set_err("device buffer allocation (%zu bytes) failed: %s", off[8] + wsb, cudaGetErrorString(e));
             return GDN_ERR_NO_MEMORY;
         }
         const void *hin[6] = {q, k, v, alpha, beta, S_in};

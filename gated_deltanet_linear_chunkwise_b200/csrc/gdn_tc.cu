@@ -189,7 +189,7 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 1, s))) return e;
     if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
-                                     nfh, s)))
+                                     nfh, err, s)))
         return e;
     if ((e = mark(ev, 2, s))) return e;
     tc::IntraParams ip;

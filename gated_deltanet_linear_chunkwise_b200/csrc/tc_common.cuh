@@ -91,7 +91,7 @@ cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x64, 
 
 cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
                                 int L, int dk, int H, int nblk, long long F, long long T, long long n_fh,
-                                cudaStream_t s);
+                                int *err, cudaStream_t s);
 
 // tm_q / tm_k / tm_u / tm_g / tm_cf deliver 128-token boxes.
 cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,

@@ -8,16 +8,18 @@
 // over 128-row blocks needs T_ii = (I + A_ii)^{-1} for every diagonal block;
 // they do not depend on each other or on the solve, so this kernel computes
 // all of them in parallel, one CTA per (frame-head, block):
-//   1. S = K_i K_i^T on 16x16 lower blocks (mma.sync bf16 -> fp32) and
-//      A = beta_r e^{G_r - G_s} S (s < r),
+//   1. S = K_i K_i^T on the 5th-generation tensor cores (one 128 x 128 tcgen05
+//      product into TMEM; K_i is copied into shared memory in the 128-byte
+//      swizzled layout by per-thread async copies) and A = beta_r e^{G_r - G_s} S
+//      (s < r) by the epilogue, one row per thread,
 //   2. the eight 16x16 diagonal leaves inverted by forward substitution in
 //      fp32 (one column per lane),
 //   3. three doubling levels 16 -> 32 -> 64 -> 128:
 //      T21 = -T22 (A21 T11)  on the tensor cores (mma.sync, fp32 accumulate).
-// The products are short dependent chains of mma.sync, whose latency is long
-// next to its issue rate, so every warp keeps several independent
-// accumulators in flight (all its Gram blocks at once; two output tiles and
-// two partial sums over K in the doubling steps).
+// The doubling products are short dependent chains of mma.sync, whose
+// latency is long next to its issue rate, so every warp keeps several
+// independent accumulators in flight (two output tiles and two partial sums
+// over K).
 // T_ii is written row-major bf16 [n_fh][nblk][128][128] (unit diagonal,
 // zeros above it), the A operand layout of the solve's T_ii Y_i product.
 #include "tc_common.cuh"
@@ -92,17 +94,23 @@ struct InvParams {
     __nv_bfloat16 *Tinv;     // [n_fh][nblk][128][128]
     int L, dk, H, nblk;
     long long F, T;
+    int *err;                // bounded-wait error word
 };
 
 __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams prm) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __nv_bfloat16 *sK = (__nv_bfloat16 *)smem;          // [128][LDK]
-    __nv_bfloat16 *sA = sK + 128 * LDK;                 // [128][LDT]  A (strictly lower)
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    constexpr uint32_t REG = 128 * LDT * 2;             // one padded 128 x 128 bf16 tile (34 KB)
+    unsigned char *sKs = smem;                          // K_i, SW128 K-major, 2 slabs x 128 rows (32 KB)
+    __nv_bfloat16 *sX = (__nv_bfloat16 *)smem;          // scratch products reuse the K region after the Gram
+    __nv_bfloat16 *sA = (__nv_bfloat16 *)(smem + REG);  // [128][LDT]  A (strictly lower)
     __nv_bfloat16 *sT = sA + 128 * LDT;                 // [128][LDT]  T
-    __nv_bfloat16 *sX = sK;                             // scratch products reuse the K tile (LDK == LDT)
     float *sAd = (float *)(sT + 128 * LDT);             // [8][16][16] fp32 diagonal leaves of A
     float *sG = sAd + 8 * 256;                          // [128]
     float *sB = sG + 128;                               // [128]
+    uint64_t *bar = (uint64_t *)(sB + 128);
+    uint32_t *tslot = (uint32_t *)(bar + 1);
+    int *sok = (int *)(tslot + 1);
 
     const int L = prm.L, dk = prm.dk, nblk = prm.nblk;
     const long long fh = blockIdx.x / nblk;
@@ -112,14 +120,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r_base = blk * 128;
 
-    // ---- load K_i (rows past the frame zero-filled) and the gates with asynchronous
-    //      copies all in flight at once, clear T and A meanwhile
-    for (int e = tid; e < 128 * (dk / 8); e += kThreads) {
-        const int r = e / (dk / 8), c8 = e % (dk / 8);
-        const bool in = r_base + r < L;
-        const long long t = f * L + (in ? r_base + r : 0);
-        sm100::cp_async16(sK + r * LDK + c8 * 8, prm.k + (((long long)b * prm.T + t) * prm.H + h) * dk + c8 * 8,
-                          in ? 16u : 0u);
+    // ---- K_i into the swizzled layout (rows past the frame and columns past d_k zero-filled)
+    //      and the gates, all by asynchronous copies in flight at once; clear T and A meanwhile
+    for (int e = tid; e < 128 * 16; e += kThreads) {
+        const int r = e >> 4, c8 = e & 15;
+        const bool in = r_base + r < L && c8 < dk / 8;
+        const long long t = f * L + (r_base + r < L ? r_base + r : 0);
+        const __nv_bfloat16 *src = prm.k + (((long long)b * prm.T + t) * prm.H + h) * dk + (in ? c8 * 8 : 0);
+        sm100::cp_async16(sKs + (c8 >> 3) * SLAB_BYTES + r * 128 + (((c8 & 7) ^ (r & 7)) << 4), src, in ? 16u : 0u);
     }
     if (tid < 128) {
         const int r = r_base + tid;
@@ -129,64 +137,69 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
         else sB[tid] = 0.f;
     }
     sm100::cp_async_commit();
-    for (int e = tid; e < 128 * ((128 - dk) / 8); e += kThreads) {  // zero the padding columns up to 128
-        const int r = e / ((128 - dk) / 8), c8 = e % ((128 - dk) / 8);
-        *reinterpret_cast<uint4 *>(sK + r * LDK + dk + c8 * 8) = make_uint4(0, 0, 0, 0);
-    }
     for (int e = tid; e < 128 * 16; e += kThreads) {
         const int r = e >> 4, c8 = e & 15;
         *reinterpret_cast<uint4 *>(sT + r * LDT + c8 * 8) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4 *>(sA + r * LDT + c8 * 8) = make_uint4(0, 0, 0, 0);
     }
+    if (tid == 0) {
+        sm100::mbar_init(bar, 1);
+        sm100::fence_barrier_init();
+    }
+    if (warp == 0) {
+        sm100::tmem_alloc(tslot, 128);
+        sm100::tmem_relinquish();
+    }
     sm100::cp_async_wait_all();
+    sm100::fence_proxy_async_smem();  // the copies are visible to the tensor cores
+    sm100::tc_fence_before();
     __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tslot;
 
-    // ---- A = beta_r e^{G_r - G_s} (K K^T)[r][s], s < r, on the 36 lower 16x16 blocks
-    const int g = lane >> 2, q = lane & 3;
-    auto block_of = [](int id, int &ab, int &cb) {  // block row ab, block column cb <= ab
-        ab = 0;
-        while (id > ab) { id -= ab + 1; ++ab; }
-        cb = id;
-    };
-    auto finish = [&](int ab, int cb, const float (&d0)[4], const float (&d1)[4]) {
-        const float *dd[2] = {d0, d1};
+    // ---- S = K K^T in TMEM (one thread issues), then the bounded wait by the same thread
+    if (tid == 0) {
+        const uint32_t id = sm100::idesc_bf16(128, 128, 0, 0);
+        for (int ks = 0; ks < dk / 16; ++ks)
+            sm100::mma_bf16_ss(tmem, desc_kmajor(sKs, ks, 128), desc_kmajor(sKs, ks, 128), id, ks > 0);
+        sm100::mma_commit(bar);
+        *sok = sm100::mbar_wait(bar, 0, prm.err) ? 1 : 0;
+    }
+    __syncthreads();
+    if (*sok) {
+        sm100::tc_fence_after();
+        // ---- A = beta_r e^{G_r - G_s} S[r][s], s < r: thread (warp, lane) owns row r = 32 (warp % 4) + lane
+        //      and columns 64 (warp / 4) .. + 63, read from TMEM 32 at a time (warp-uniform skips)
+        const int q4 = warp & 3, hw = warp >> 2, r = q4 * 32 + lane;
+        const float br = sB[r], gr = sG[r];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+        for (int rr = 0; rr < 2; ++rr) {
+            const int c0 = 64 * hw + 32 * rr;
+            if (c0 >= q4 * 32 + 32) continue;  // no row of this warp has s < r in these columns
+            float v[32];
+            sm100::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + c0, v);
+            sm100::tmem_ld_wait();
+            float a[32];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {  // element (r, s) of this thread's fragments
-                const int r = ab * 16 + g + (e >> 1) * 8;
-                const int s = cb * 16 + nt * 8 + 2 * q + (e & 1);
-                const float val = (s < r) ? sB[r] * __expf(sG[r] - sG[s]) * dd[nt][e] : 0.f;
-                sA[r * LDT + s] = __float2bfloat16_rn(val);
-                if (ab == cb) sAd[ab * 256 + (r - ab * 16) * 16 + (s - cb * 16)] = val;
+            for (int e = 0; e < 32; ++e) {
+                const int s = c0 + e;
+                a[e] = s < r ? br * __expf(gr - sG[s]) * v[e] : 0.f;
             }
-        }
-    };
-    // warp w owns blocks w, w + 8, ..., all accumulated at once: ten independent
-    // accumulation chains hide the latency of the tensor-core instructions
-    constexpr int NB = 5;  // ceil(36 / 8)
-    int ab[NB], cb[NB];
 #pragma unroll
-    for (int u = 0; u < NB; ++u) block_of(min(warp + 8 * u, 35), ab[u], cb[u]);
-    float acc[NB][2][4] = {};
+            for (int u = 0; u < 4; ++u)
+                *reinterpret_cast<uint4 *>(sA + r * LDT + c0 + 8 * u) =
+                    make_uint4(pack_bf16(a[8 * u], a[8 * u + 1]), pack_bf16(a[8 * u + 2], a[8 * u + 3]),
+                               pack_bf16(a[8 * u + 4], a[8 * u + 5]), pack_bf16(a[8 * u + 6], a[8 * u + 7]));
+            // the fp32 diagonal 16 x 16 block of this row, when it lies in these columns
+            const int db = r >> 4;
+            if ((db * 16) >= c0 && (db * 16) < c0 + 32) {
+                const bool lo = db * 16 == c0;
 #pragma unroll
-    for (int kk = 0; kk < 128; kk += 16) {
-        if (kk < dk) {
-#pragma unroll
-            for (int u = 0; u < NB; ++u) {
-                if (warp + 8 * u < 36) {
-                    uint32_t a[4], bb[4];
-                    load_a(a, sK, LDK, ab[u] * 16, kk, lane);
-                    load_b_rows(bb, sK, LDK, cb[u] * 16, kk, lane);
-                    mma16816(acc[u][0], a, bb[0], bb[1]);
-                    mma16816(acc[u][1], a, bb[2], bb[3]);
-                }
+                for (int e = 0; e < 16; ++e) sAd[db * 256 + (r & 15) * 16 + e] = lo ? a[e] : a[16 + e];
             }
         }
     }
-#pragma unroll
-    for (int u = 0; u < NB; ++u)
-        if (warp + 8 * u < 36) finish(ab[u], cb[u], acc[u][0], acc[u][1]);
+    sm100::tc_fence_before();
     __syncthreads();
 
     // ---- leaves: warp w inverts diagonal block w; lane c < 16 owns column c
@@ -268,18 +281,24 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
         const int r = e >> 4, c8 = e & 15;
         *reinterpret_cast<uint4 *>(dst + r * 128 + c8 * 8) = *reinterpret_cast<const uint4 *>(sT + r * LDT + c8 * 8);
     }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, 128);
+    }
 }
 
 }  // namespace
 
 size_t diag_inverse_smem_bytes() {
-    return sizeof(__nv_bfloat16) * (128 * LDK + 2 * 128 * LDT) + sizeof(float) * (8 * 256 + 256);
+    return 1024 + sizeof(__nv_bfloat16) * 3 * 128 * LDT + sizeof(float) * (8 * 256 + 256) + 16;
 }
 
 cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
                                 int L, int dk, int H, int nblk, long long F, long long T, long long n_fh,
-                                cudaStream_t s) {
-    InvParams prm{k, beta, G, Tinv, L, dk, H, nblk, F, T};
+                                int *err, cudaStream_t s) {
+    InvParams prm{k, beta, G, Tinv, L, dk, H, nblk, F, T, err};
     const size_t smem = diag_inverse_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(k_diag_inverse, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -115,7 +115,8 @@ int gdn_step_f32(const float *q, const float *k, const float *v,
  * arguments and layouts as gdn_fwd (dtype = GDN_DTYPE_BF16) or gdn_fwd_f32
  * (GDN_DTYPE_F32), except that q, k, v, alpha, beta, S_in, S_out and o are
  * host pointers (pinned memory gives the fastest copies; pageable works).
- * The call allocates device buffers with cudaMallocAsync on `stream`, copies
+ * The call allocates device buffers (stream-ordered, from the library's
+ * scratch pool; see gdn_fwd_ex's workspace) on `stream`, copies
  * the inputs in, runs the pass, copies o (and S_out) out, frees the buffers
  * and synchronises `stream` before it returns, so the host outputs are
  * ready.  Host pointers need no alignment.  Errors as gdn_fwd, plus
@@ -166,8 +167,11 @@ int gdn_fwd_noalloc(const void *q, const void *k, const void *v,
  *   dtype           GDN_DTYPE_BF16 or GDN_DTYPE_F32 (q/k/v/o element type).
  *   workspace       optional device scratch of workspace_bytes bytes, at
  *                   least gdn_workspace_bytes(...) and 256-byte aligned; NULL
- *                   lets the call take stream-ordered memory (cudaMallocAsync)
- *                   and return it before the call returns.
+ *                   lets the call take stream-ordered scratch and return it
+ *                   before the call returns.  That scratch comes from one
+ *                   pool per device owned by the library, which keeps the
+ *                   freed memory reserved for later calls (up to the largest
+ *                   scratch any call has needed) until the process exits.
  *   reverse         1: reversed-time scan (tokens visited T-1..0, each gate
  *                   applied at its own token; SANA-WM summary, section 3.2,
  *                   paragraph "Bidirectional and Chunk-Causal GDN Variants").
