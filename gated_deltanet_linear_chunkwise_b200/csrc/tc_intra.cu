@@ -113,139 +113,193 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     const int nslab_x = (nc + SLAB - 1) / SLAB;
     const int nt128 = (L + CT - 1) / CT;
 
+    // Item numbering shared by the roles (block b has b S tiles, then T_b in the K ring):
+    //   K-ring item of S tile c of block b: b(b+1)/2 + c, of T_b: b(b+1)/2 + b
+    //   X-ring item of X tile x (64 tokens) of block b: b(b-1) + x
+    //   S tile (and S/P buffer use) of S tile c of block b: b(b-1)/2 + c
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
+        // Polls every kind of load and issues whichever is possible, so the K ring
+        // (S products) never waits behind the X ring (P X products) or the stores.
         if (lane == 0) {
             sm100::tma_prefetch_desc(&tm_k);
             sm100::tma_prefetch_desc(&tm_x64);
             sm100::tma_prefetch_desc(&tm_t);
             sm100::tma_prefetch_desc(&tm_gct);
             sm100::tma_prefetch_desc(&tm_xs);
-            bool ok = true;
+            int ki = 0;              // next K_i block
+            int kb = 0, kc = 0;      // next K-ring item: block kb, item kc (kc == kb: T_kb)
+            int xb = 1, xx = 0;      // next X-ring item: block xb, X tile xx
+            int sxb = 0;             // next X block to store; blocks < sxb have been stored and read out
             int kn = 0, xn = 0;
-            // K-ring item: the K tile of S tile c with its G and cf, or T_ii (c < 0)
-            auto load_k = [&](int c, int i) -> bool {
-                const int st = kn % NK;
-                if (kn >= NK && !sm100::mbar_wait(&bars[KREMPTY + st], ((kn / NK) - 1) & 1, err)) return false;
-                unsigned char *slot = sKR + st * KSLOT;
-                if (c >= 0) {
-                    sm100::mbar_arrive_expect_tx(&bars[KRFULL + st],
-                                                 (uint32_t)(nslab_k * SLAB_BYTES + GCT_FLOATS * 4));
-                    for (int sl = 0; sl < nslab_k; ++sl)
-                        sm100::tma_load_4d(slot + sl * SLAB_BYTES, &tm_k, &bars[KRFULL + st], sl * SLAB, h, c * CT,
-                                           bf);
-                    sm100::tma_load_2d(sGC + st * GCT_FLOATS, &tm_gct, &bars[KRFULL + st], 0,
-                                       (int)(fh * nt128 + c));
-                } else {
-                    sm100::mbar_arrive_expect_tx(&bars[KRFULL + st], (uint32_t)(2 * SLAB_BYTES));
-                    for (int sl = 0; sl < 2; ++sl)
-                        sm100::tma_load_3d(slot + sl * SLAB_BYTES, &tm_t, &bars[KRFULL + st], sl * SLAB, 0,
-                                           (int)(fh * nblk + i));
-                }
-                ++kn;
-                return true;
-            };
-            auto load_x = [&](int x, int i) -> bool {
-                const int st = xn % NX;
-                if (xn >= NX && !sm100::mbar_wait(&bars[XREMPTY + st], ((xn / NX) - 1) & 1, err)) return false;
-                if (x >= 2 * (i - 1)) sm100::bulk_wait0();  // the rows of X_{i-1} are in global memory
-                unsigned char *slot = sXR + st * XSLOT;
-                sm100::mbar_arrive_expect_tx(&bars[XRFULL + st], (uint32_t)(nslab_x * XSLAB));
-                for (int sl = 0; sl < nslab_x; ++sl)
-                    sm100::tma_load_3d(slot + sl * XSLAB, &tm_x64, &bars[XRFULL + st], sl * SLAB, x * XT, (int)fh);
-                ++xn;
-                return true;
-            };
-            // store the staged X_i (rows past the frame and columns past d_v + d_k are clipped)
-            auto store_x = [&](int i) -> bool {
-                if (!sm100::mbar_wait(&bars[XSTAGED], i & 1, err)) return false;
-                for (int sl = 0; sl < nslab_x; ++sl)
-                    sm100::tma_store_3d(&tm_xs, sYX + sl * SLAB_BYTES, sl * SLAB, i * BM, (int)fh);
-                sm100::bulk_commit();
-                sm100::bulk_wait_read0();
-                return true;
-            };
-            for (int i = 0; i < nblk && ok; ++i) {
+            bool ok = true;
+            sm100::Spin spin;
+            while (ok && (ki < nblk || kb < nblk || xb < nblk || sxb < nblk)) {
+                bool prog = false;
                 // K_i once the previous block's Y build has read K_{i-1}
-                if (i >= 1) ok = sm100::mbar_wait(&bars[KIEMPTY], (i - 1) & 1, err);
-                if (!ok) break;
-                sm100::mbar_arrive_expect_tx(&bars[KIFULL], (uint32_t)(nslab_k * SLAB_BYTES));
-                for (int sl = 0; sl < nslab_k; ++sl)
-                    sm100::tma_load_4d(sKi + sl * SLAB_BYTES, &tm_k, &bars[KIFULL], sl * SLAB, h, i * BM, bf);
-                for (int c = 0; c < i && ok; ++c) {
-                    ok = load_k(c, i);
-                    // the X ring refills the Y / X_{i-1} buffer only after X_{i-1} has been stored
-                    if (ok && c == 0) ok = store_x(i - 1);
-                    if (ok) ok = load_x(2 * c, i);
-                    if (ok) ok = load_x(2 * c + 1, i);
+                if (ki < nblk && (ki == 0 || sm100::mbar_test(&bars[KIEMPTY], (ki - 1) & 1))) {
+                    sm100::mbar_arrive_expect_tx(&bars[KIFULL], (uint32_t)(nslab_k * SLAB_BYTES));
+                    for (int sl = 0; sl < nslab_k; ++sl)
+                        sm100::tma_load_4d(sKi + sl * SLAB_BYTES, &tm_k, &bars[KIFULL], sl * SLAB, h, ki * BM, bf);
+                    ++ki;
+                    prog = true;
                 }
-                if (ok) ok = load_k(-1, i);  // T_ii
+                // the next K-ring item: the K tile (+ G, cf) of an S product, or T_kb
+                if (kb < nblk) {
+                    const int st = kn % NK;
+                    if (kn < NK || sm100::mbar_test(&bars[KREMPTY + st], ((kn / NK) - 1) & 1)) {
+                        unsigned char *slot = sKR + st * KSLOT;
+                        if (kc < kb) {
+                            sm100::mbar_arrive_expect_tx(&bars[KRFULL + st],
+                                                         (uint32_t)(nslab_k * SLAB_BYTES + GCT_FLOATS * 4));
+                            for (int sl = 0; sl < nslab_k; ++sl)
+                                sm100::tma_load_4d(slot + sl * SLAB_BYTES, &tm_k, &bars[KRFULL + st], sl * SLAB, h,
+                                                   kc * CT, bf);
+                            sm100::tma_load_2d(sGC + st * GCT_FLOATS, &tm_gct, &bars[KRFULL + st], 0,
+                                               (int)(fh * nt128 + kc));
+                        } else {
+                            sm100::mbar_arrive_expect_tx(&bars[KRFULL + st], (uint32_t)(2 * SLAB_BYTES));
+                            for (int sl = 0; sl < 2; ++sl)
+                                sm100::tma_load_3d(slot + sl * SLAB_BYTES, &tm_t, &bars[KRFULL + st], sl * SLAB, 0,
+                                                   (int)(fh * nblk + kb));
+                        }
+                        ++kn;
+                        if (++kc > kb) {
+                            ++kb;
+                            kc = 0;
+                        }
+                        prog = true;
+                    }
+                }
+                // store the staged X_sxb (rows past the frame, columns past d_v + d_k clipped); the
+                // X ring may refill the first two slots (which hold Y / X) once the store has read them
+                if (sxb < nblk && sm100::mbar_test(&bars[XSTAGED], sxb & 1)) {
+                    for (int sl = 0; sl < nslab_x; ++sl)
+                        sm100::tma_store_3d(&tm_xs, sYX + sl * SLAB_BYTES, sl * SLAB, sxb * BM, (int)fh);
+                    sm100::bulk_commit();
+                    sm100::bulk_wait_read0();
+                    ++sxb;
+                    prog = true;
+                }
+                // the next X-ring item: X tile xx of block xb (the tiles of X_{xb-1} come last)
+                if (xb < nblk && sxb >= xb) {
+                    const int st = xn % NX;
+                    if (xn < NX || sm100::mbar_test(&bars[XREMPTY + st], ((xn / NX) - 1) & 1)) {
+                        if (xx >= 2 * (xb - 1)) sm100::bulk_wait0();  // X_{xb-1} is in global memory
+                        unsigned char *slot = sXR + st * XSLOT;
+                        sm100::mbar_arrive_expect_tx(&bars[XRFULL + st], (uint32_t)(nslab_x * XSLAB));
+                        for (int sl = 0; sl < nslab_x; ++sl)
+                            sm100::tma_load_3d(slot + sl * XSLAB, &tm_x64, &bars[XRFULL + st], sl * SLAB, xx * XT,
+                                               (int)fh);
+                        ++xn;
+                        if (++xx == 2 * xb) {
+                            ++xb;
+                            xx = 0;
+                        }
+                        prog = true;
+                    }
+                }
+                if (prog) spin.reset();
+                else if (!spin.tick(err)) ok = false;
             }
-            if (ok) ok = store_x(nblk - 1);
             sm100::bulk_wait0();  // leave with no store in flight
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Polls: S = K_b K_c^T as soon as K_b, the K tile and an S/P buffer are there;
+        // acc += P X as soon as P and both X halves are there (and acc is free);
+        // X_b = T_b Y_b as soon as Y_b and T_b are there.
         if (lane == 0) {
             const uint32_t id_s = sm100::idesc_bf16(BM, CT, 0, 0);
             const uint32_t id_x = sm100::idesc_bf16(BM, nc, 0, 1);
-            bool ok = true;
-            int kn = 0, xn = 0, sn = 0;  // K-ring item, X-ring item, S tile counters
-            // acc += P X for S tile c (its buffer sb): the two 64-token X tiles in turn; P of
-            // tokens 0..63 sits in TMEM columns 0..31 of the buffer, tokens 64..127 in 64..95
-            auto issue_px = [&](int sb, int s_idx, bool first, int i) -> bool {
-                if (!sm100::mbar_wait(&bars[PFULL + sb], (s_idx / NSB) & 1, err)) return false;
-                // the block's first product overwrites acc: X_{i-1} must have been read out
-                if (first && i >= 1 && !sm100::mbar_wait(&bars[XSTAGED], (i - 1) & 1, err)) return false;
-                for (int hx = 0; hx < 2; ++hx) {
-                    const int st = xn % NX;
-                    if (!sm100::mbar_wait(&bars[XRFULL + st], (xn / NX) & 1, err)) return false;
-                    sm100::tc_fence_after();
-                    const unsigned char *xt = sXR + st * XSLOT;
-                    for (int ks = 0; ks < XT / 16; ++ks)
-                        sm100::mma_bf16_ts(t_acc, t_s0 + sb * CT + 64 * hx + ks * 8, desc_mnmajor(xt, ks, XT), id_x,
-                                           (first && hx == 0 && ks == 0) ? 0u : 1u);
-                    sm100::mma_commit(&bars[XREMPTY + st]);
-                    ++xn;
-                }
-                sm100::mma_commit(&bars[SFREE + sb]);
-                return true;
+            // A parity test is only unambiguous for the phase right after the last one
+            // observed, and the S and T cursors take K-ring items out of order, so the
+            // phases of each K slot (and of K_i) are observed one at a time, in order.
+            int kobs[NK] = {}, kiobs = 0;
+            auto k_ready = [&](int kn) -> bool {
+                const int st = kn % NK, u = kn / NK;
+                while (kobs[st] <= u && sm100::mbar_test(&bars[KRFULL + st], kobs[st] & 1)) ++kobs[st];
+                return kobs[st] > u;
             };
-            for (int i = 0; i < nblk && ok; ++i) {
-                ok = sm100::mbar_wait(&bars[KIFULL], i & 1, err);
-                int prev_sb = -1, prev_idx = 0;
-                for (int c = 0; c < i && ok; ++c, ++kn, ++sn) {
-                    const int st = kn % NK, sb = sn % NSB;
-                    ok = sm100::mbar_wait(&bars[KRFULL + st], (kn / NK) & 1, err);
-                    if (ok && sn >= NSB) ok = sm100::mbar_wait(&bars[SFREE + sb], ((sn / NSB) - 1) & 1, err);
-                    if (!ok) break;
-                    sm100::tc_fence_after();
-                    const unsigned char *kt = sKR + st * KSLOT;
-                    for (int ks = 0; ks < nks_d; ++ks)
-                        sm100::mma_bf16_ss(t_s0 + sb * CT, desc_kmajor(sKi, ks, BM), desc_kmajor(kt, ks, CT), id_s,
-                                           ks > 0);
-                    sm100::mma_commit(&bars[SFULL + sb]);
-                    sm100::mma_commit(&bars[KREMPTY + st]);
-                    // one S tile behind: the tensor cores compute S(c) while the epilogue writes P(c-1)
-                    if (prev_sb >= 0) ok = issue_px(prev_sb, prev_idx, c == 1, i);
-                    prev_sb = sb;
-                    prev_idx = sn;
+            auto ki_ready = [&](int b) -> bool {
+                while (kiobs <= b && sm100::mbar_test(&bars[KIFULL], kiobs & 1)) ++kiobs;
+                return kiobs > b;
+            };
+            // K_1 cannot load before block 0's Y build, which waits for acc_0 = 0 below:
+            // observe K_0 first so that KIFULL never runs two phases ahead
+            bool ok = sm100::mbar_wait(&bars[KIFULL], 0, err);
+            kiobs = 1;
+            sm100::mma_commit(&bars[ACCFULL]);  // block 0 has no S tiles: acc_0 = 0
+            int sb_ = 1, sc_ = 0, sn = 0;       // next S product: block sb_, tile sc_; S tile count
+            int pb_ = 1, pc_ = 0, pn = 0;       // next P X product
+            int ty = 0;                         // next T Y
+            const int ntile = nblk * (nblk - 1) / 2;
+            sm100::Spin spin;
+            while (ok && (pn < ntile || ty < nblk)) {
+                bool prog = false;
+                if (sn < ntile && sn - pn < NSB) {
+                    const int kn = sb_ * (sb_ + 1) / 2 + sc_, st = kn % NK, buf = sn % NSB;
+                    if (ki_ready(sb_) && k_ready(kn) &&
+                        (sn < NSB || sm100::mbar_test(&bars[SFREE + buf], ((sn / NSB) - 1) & 1))) {
+                        sm100::tc_fence_after();
+                        const unsigned char *kt = sKR + st * KSLOT;
+                        for (int ks = 0; ks < nks_d; ++ks)
+                            sm100::mma_bf16_ss(t_s0 + buf * CT, desc_kmajor(sKi, ks, BM), desc_kmajor(kt, ks, CT),
+                                               id_s, ks > 0);
+                        sm100::mma_commit(&bars[SFULL + buf]);
+                        sm100::mma_commit(&bars[KREMPTY + st]);
+                        ++sn;
+                        if (++sc_ == sb_) {
+                            ++sb_;
+                            sc_ = 0;
+                        }
+                        prog = true;
+                    }
                 }
-                if (ok && prev_sb >= 0) ok = issue_px(prev_sb, prev_idx, i == 1, i);
-                if (!ok) break;
-                sm100::mma_commit(&bars[ACCFULL]);
-                // X_i = T_ii Y_i; T_ii is the block's last K-ring item
-                const int st = kn % NK;
-                ok = sm100::mbar_wait(&bars[KRFULL + st], (kn / NK) & 1, err) &&
-                     sm100::mbar_wait(&bars[YFULL], i & 1, err);
-                if (!ok) break;
-                sm100::tc_fence_after();
-                const unsigned char *tt = sKR + st * KSLOT;
-                for (int ks = 0; ks < BM / 16; ++ks)
-                    sm100::mma_bf16_ss(t_acc, desc_kmajor(tt, ks, BM), desc_mnmajor(sYX, ks, BM), id_x, ks > 0);
-                sm100::mma_commit(&bars[XFULL]);
-                sm100::mma_commit(&bars[KREMPTY + st]);
-                ++kn;
+                if (pn < sn) {
+                    const int buf = pn % NSB, xn0 = pb_ * (pb_ - 1) + 2 * pc_;
+                    const int st0 = xn0 % NX, st1 = (xn0 + 1) % NX;
+                    const bool first = pc_ == 0;
+                    // the block's first product overwrites acc: X_{pb_-1} must have been read out
+                    if (sm100::mbar_test(&bars[PFULL + buf], (pn / NSB) & 1) &&
+                        sm100::mbar_test(&bars[XRFULL + st0], (xn0 / NX) & 1) &&
+                        sm100::mbar_test(&bars[XRFULL + st1], ((xn0 + 1) / NX) & 1) &&
+                        (!first || sm100::mbar_test(&bars[XSTAGED], (pb_ - 1) & 1))) {
+                        sm100::tc_fence_after();
+                        // P of tokens 0..63 sits in TMEM columns 0..31 of the buffer, tokens 64..127 in 64..95
+                        for (int hx = 0; hx < 2; ++hx) {
+                            const unsigned char *xt = sXR + (hx ? st1 : st0) * XSLOT;
+                            for (int ks = 0; ks < XT / 16; ++ks)
+                                sm100::mma_bf16_ts(t_acc, t_s0 + buf * CT + 64 * hx + ks * 8, desc_mnmajor(xt, ks, XT),
+                                                   id_x, (first && hx == 0 && ks == 0) ? 0u : 1u);
+                            sm100::mma_commit(&bars[XREMPTY + (hx ? st1 : st0)]);
+                        }
+                        sm100::mma_commit(&bars[SFREE + buf]);
+                        if (pc_ == pb_ - 1) sm100::mma_commit(&bars[ACCFULL]);
+                        ++pn;
+                        if (++pc_ == pb_) {
+                            ++pb_;
+                            pc_ = 0;
+                        }
+                        prog = true;
+                    }
+                }
+                if (ty < nblk && pb_ > ty) {  // every P X product of block ty has been issued
+                    const int kn = ty * (ty + 1) / 2 + ty, st = kn % NK;
+                    if (k_ready(kn) && sm100::mbar_test(&bars[YFULL], ty & 1)) {
+                        sm100::tc_fence_after();
+                        const unsigned char *tt = sKR + st * KSLOT;
+                        for (int ks = 0; ks < BM / 16; ++ks)
+                            sm100::mma_bf16_ss(t_acc, desc_kmajor(tt, ks, BM), desc_mnmajor(sYX, ks, BM), id_x,
+                                               ks > 0);
+                        sm100::mma_commit(&bars[XFULL]);
+                        sm100::mma_commit(&bars[KREMPTY + st]);
+                        ++ty;
+                        prog = true;
+                    }
+                }
+                if (prog) spin.reset();
+                else if (!spin.tick(err)) ok = false;
             }
         }
     } else {
@@ -298,7 +352,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             }
             if (!ok) break;
             // ---- Y_i = R_i + acc_i  -> sYX (MN-major: row = K index of the T_ii Y_i product)
-            ok = sm100::mbar_wait(&bars[ACCFULL], i & 1, err);
+            // (K_i: the W half reads it; block 0 has no S product that waited for it)
+            ok = sm100::mbar_wait(&bars[ACCFULL], i & 1, err) && sm100::mbar_wait(&bars[KIFULL], i & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
             auto store_y = [&](int c, const float (&y)[8]) {
@@ -372,7 +427,11 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::fence_proxy_async_smem();
             sm100::mbar_arrive(&bars[YFULL]);
             sm100::mbar_arrive(&bars[KIEMPTY]);
-            sm100::mbar_arrive(&bars[KREMPTY + kn % NK]);  // the T_ii slot: released when T Y completes
+            // the T_ii slot: observe its load (so this thread sees every phase of the slot in
+            // order), then release it; the slot refills once T Y has completed as well
+            ok = sm100::mbar_wait(&bars[KRFULL + kn % NK], (kn / NK) & 1, err);
+            if (!ok) break;
+            sm100::mbar_arrive(&bars[KREMPTY + kn % NK]);
             ++kn;
             // ---- X_i = T_ii Y_i -> bf16 staging over Y_i (half 0 the Ub columns, half 1 the W columns)
             ok = sm100::mbar_wait(&bars[XFULL], i & 1, err);
