@@ -215,11 +215,13 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             // A parity test is only unambiguous for the phase right after the last one
             // observed, and the S and T cursors take K-ring items out of order, so the
             // phases of each K slot (and of K_i) are observed one at a time, in order.
-            int kobs[NK] = {}, kiobs = 0;
+            static_assert(NK == 2, "one observed-phase counter per K slot");
+            int kobs0 = 0, kobs1 = 0, kiobs = 0;  // scalars: an indexed array would live in local memory
             auto k_ready = [&](int kn) -> bool {
                 const int st = kn % NK, u = kn / NK;
-                while (kobs[st] <= u && sm100::mbar_test(&bars[KRFULL + st], kobs[st] & 1)) ++kobs[st];
-                return kobs[st] > u;
+                int &obs = st ? kobs1 : kobs0;
+                while (obs <= u && sm100::mbar_test(&bars[KRFULL + st], obs & 1)) ++obs;
+                return obs > u;
             };
             auto ki_ready = [&](int b) -> bool {
                 while (kiobs <= b && sm100::mbar_test(&bars[KIFULL], kiobs & 1)) ++kiobs;
