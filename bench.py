@@ -251,6 +251,22 @@ def main():
     ms_total = gdist.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
     ms_step = ms_total / args.steps
 
+    # the bidirectional layer of the minute workload's label (forward + reversed scan, summed),
+    # reported beside the forward metric: device time per pass over the same inputs
+    def bidir():  # scratch from the library's pool (kept between calls)
+        g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, None, S_out=S_out, o=o, stream=stream)
+        g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, None, o=o, reverse=True, accumulate=True,
+                  stream=stream)
+
+    bidir()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for _ in range(3):
+        bidir()
+    b1.record(stream)
+    torch.cuda.synchronize(dev)
+    bidir_ms = gdist.max_over_ranks(b0.elapsed_time(b1) / 3, device=dev)
+
     # per-stage device times (events around each kernel on the same stream)
     stage_sum = [0.0] * NUM_STAGES
     reps = 5
@@ -329,6 +345,8 @@ def main():
                     "d2h_bytes_per_step": d2h},
             # one kernel per stage: gates, diagonal inverses, intra, transition, scan, U, output
             "gpu_launches": NUM_STAGES * args.steps,
+            "bidirectional": {"ms_per_pass": bidir_ms, "tokens_per_s": tokens / (bidir_ms * 1e-3),
+                              "what": "forward + reversed scan summed into o (not the timed metric)"},
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline and world == 1 and args.workload == WORKLOAD:

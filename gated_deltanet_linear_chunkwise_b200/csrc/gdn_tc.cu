@@ -25,7 +25,9 @@ namespace {
 inline int cf_stride(int L) { return (L + 3) & ~3; }
 
 struct TcLayout {
-    size_t G, CF, GCT, Tinv, X, M, N, Sig, SigB, U, err, total;
+    size_t G, CF, GCT, Tinv, X, M, N, Sig, SigB, U, err;
+    size_t Otmp, Qr, Kr, Vr, Ar, Br;  // reversed / accumulating calls only (0 bytes otherwise)
+    size_t total;
 };
 
 TcLayout tc_layout(const Problem &p) {
@@ -44,6 +46,16 @@ TcLayout tc_layout(const Problem &p) {
     lay.SigB = off; off += align256(2 * nfh * p.dk * p.dv);
     lay.U = off;    off += align256(2 * nfh * p.L * p.dv);
     lay.err = off;  off += 256;
+    // A reversed scan runs the forward kernels on token-reversed copies of the inputs; a
+    // reversed or accumulating call writes o to a staging buffer first.
+    const size_t ntok = (size_t)p.B * p.T * p.H;
+    const bool stage_o = p.reverse || p.accumulate, rev = p.reverse;
+    lay.Otmp = off; off += stage_o ? align256(2 * ntok * p.dv) : 0;
+    lay.Qr = off;   off += rev ? align256(2 * ntok * p.dk) : 0;
+    lay.Kr = off;   off += rev ? align256(2 * ntok * p.dk) : 0;
+    lay.Vr = off;   off += rev ? align256(2 * ntok * p.dv) : 0;
+    lay.Ar = off;   off += rev ? align256(4 * ntok) : 0;
+    lay.Br = off;   off += rev ? align256(4 * ntok) : 0;
     lay.total = off;
     return lay;
 }
@@ -146,12 +158,15 @@ bool tc_disabled_by_env() {
 
 bool tc_supports(const Problem &p) {
     static const bool disabled = tc_disabled_by_env();
-    return !disabled && p.dtype == GDN_DTYPE_BF16 && !p.reverse && !p.accumulate;
+    return !disabled && p.dtype == GDN_DTYPE_BF16;
 }
 
 size_t tc_workspace_bytes(const Problem &p) { return tc_layout(p).total; }
 
-cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
+// The forward pass.  `scan_reverse` is the caller's reverse flag: on token-reversed copies the
+// kernels run forward, and only the chunk-reset rule of the scan still follows the original
+// token positions.
+cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cudaStream_t s, cudaEvent_t *ev) {
     const TcLayout lay = tc_layout(p);
     char *base = (char *)ws;
     const long long nfh = (long long)p.B * p.H * p.F;
@@ -203,7 +218,9 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
     if ((e = tc::launch_transition_tc(tm_k64, tm_x, tp, nfh, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
-    if ((e = simt_scan(p, Mb, Nb, Sig, SigB, s))) return e;
+    Problem ps = p;
+    ps.reverse = scan_reverse;
+    if ((e = simt_scan(ps, Mb, Nb, Sig, SigB, s))) return e;
     if ((e = mark(ev, 5, s))) return e;
     tc::UParams up;
     up.X = X; up.U = U;
@@ -223,6 +240,73 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u128, tm_sig, tm_g128, tm_cf128, op, num_sms, s))) return e;
     return mark(ev, 7, s);
+}
+
+namespace {
+
+// dst row (b, T-1-t) = src row (b, t) for rows of `row_words` 32-bit words ([B, T, ...] tensors).
+__global__ void reverse_rows_kernel(const uint32_t *__restrict__ src, uint32_t *__restrict__ dst, int B,
+                                    long long T, int row_words) {
+    const long long total = (long long)B * T * row_words;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long w = e % row_words, row = e / row_words, t = row % T, b = row / T;
+        dst[(b * T + (T - 1 - t)) * row_words + w] = src[e];
+    }
+}
+
+// o (+)= the staged result, rows taken in reverse token order for a reversed scan; the sum
+// of an accumulating call is formed in fp32 and rounded once to bf16.
+__global__ void finish_o_kernel(const __nv_bfloat162 *__restrict__ tmp, __nv_bfloat162 *__restrict__ o, int B,
+                                long long T, int row_pairs, int reverse, int accumulate) {
+    const long long total = (long long)B * T * row_pairs;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long w = e % row_pairs, row = e / row_pairs, t = row % T, b = row / T;
+        const long long src = reverse ? (b * T + (T - 1 - t)) * row_pairs + w : e;
+        float2 v = __bfloat1622float2(tmp[src]);
+        if (accumulate) {
+            const float2 old = __bfloat1622float2(o[e]);
+            v.x += old.x;
+            v.y += old.y;
+        }
+        o[e] = __floats2bfloat162_rn(v.x, v.y);
+    }
+}
+
+cudaError_t reverse_rows(const void *src, void *dst, int B, long long T, size_t row_bytes, cudaStream_t s) {
+    reverse_rows_kernel<<<1184, 256, 0, s>>>((const uint32_t *)src, (uint32_t *)dst, B, T, (int)(row_bytes / 4));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
+    if (!p.reverse && !p.accumulate) return launch_tc_forward(p, ws, 0, s, ev);
+    const TcLayout lay = tc_layout(p);
+    char *base = (char *)ws;
+    Problem q = p;
+    q.reverse = 0;
+    q.accumulate = 0;
+    q.o = base + lay.Otmp;
+    cudaError_t e;
+    if (p.reverse) {  // token-reversed copies: the reversed recurrence is the forward one on them
+        const size_t rq = (size_t)p.H * p.dk * 2, rv = (size_t)p.H * p.dv * 2, rg = (size_t)p.H * 4;
+        if ((e = reverse_rows(p.q, base + lay.Qr, p.B, p.T, rq, s))) return e;
+        if ((e = reverse_rows(p.k, base + lay.Kr, p.B, p.T, rq, s))) return e;
+        if ((e = reverse_rows(p.v, base + lay.Vr, p.B, p.T, rv, s))) return e;
+        if ((e = reverse_rows(p.alpha, base + lay.Ar, p.B, p.T, rg, s))) return e;
+        if ((e = reverse_rows(p.beta, base + lay.Br, p.B, p.T, rg, s))) return e;
+        q.q = base + lay.Qr;
+        q.k = base + lay.Kr;
+        q.v = base + lay.Vr;
+        q.alpha = (const float *)(base + lay.Ar);
+        q.beta = (const float *)(base + lay.Br);
+    }
+    if ((e = launch_tc_forward(q, ws, p.reverse, s, ev))) return e;
+    finish_o_kernel<<<1184, 256, 0, s>>>((const __nv_bfloat162 *)(base + lay.Otmp), (__nv_bfloat162 *)p.o, p.B, p.T,
+                                         p.H * p.dv / 2, p.reverse, p.accumulate);
+    return cudaGetLastError();
 }
 
 int *tc_error_word(const Problem &p, void *ws) { return (int *)((char *)ws + tc_layout(p).err); }

@@ -141,6 +141,21 @@ def test_reverse_and_bidirectional(dtype, chunk):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_reverse_reset_not_dividing_length(dtype):
+    # 5 frames, state restarting every 2 frames counted from token 0: the reversed scan's
+    # restarts do not line up with its own start
+    L = 64
+    inp = W.draw(1, 3, 5 * L, 48, 32, frame_len=L, seed=23, regime="slow", dtype=dtype, state_std=0.2)
+    d = dev(inp)
+    o_acc = (d["v"][..., :32] * 0 + 0.25).contiguous()  # accumulate into a non-zero o
+    o_r, S_r = g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, d["S_in"], return_state=True,
+                         reverse=True, reset_every=2 * L, o=o_acc.clone(), accumulate=True)
+    o_ref, S_ref = ora(inp, inp["S_in"], reverse=True, reset_every=2 * L)
+    assert rel(o_r.double().cpu() - 0.25, o_ref) <= TOL[dtype] + (4e-3 if dtype == "bf16" else 0.0)
+    assert rel(S_r.double().cpu(), S_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_step_chain_equals_single_call(dtype):
     L = 80
     inp = W.draw(2, 3, 7 * L, 64, 64, frame_len=L, seed=31, regime="slow", dtype=dtype, state_std=0.1)
