@@ -27,10 +27,10 @@
 // The state term is a pseudo-tile in front of the column tiles: the epilogue
 // writes Q~ = diag(e^G) Q_I into an S/P buffer and a ring slot delivers Sig
 // (bf16, MN-major), so O starts as Q~ Sig.  Off-diagonal decay factors are
-// e^{G_r - a} cf_s with cf_s = e^{a - G_s} (a = G at the tile's last token,
-// both <= 1, a per 64-token half); the diagonal tile takes e^{G_r - G_s} per
-// element.  Every
-// wait is bounded (sm100::mbar_wait).
+// e^{G_r - a} cf_s with cf_s = e^{a - G_s} (a = G at the end of s's 64-token
+// group, both <= 1); in the diagonal group the row factor is >= 1, bounded by
+// e^60, else the exact e^{G_r - G_s} is taken per element.  Every wait is
+// bounded (sm100::mbar_wait).
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -45,6 +45,7 @@ constexpr int NSB = 2;                    // S/P buffers in TMEM
 constexpr int JSLAB = JT * 128;           // one 128-row slab
 constexpr int SLOT_BYTES = 4 * JSLAB;     // K (2 slabs) + U (2 slabs); Sig (<= 32 KB) fills a whole slot
 constexpr int GC_BYTES = 2 * JT * 4;      // G and cf of one tile
+constexpr float kSplitMax = 60.f;         // largest row exponent the in-group split takes
 
 struct Smem {
     static constexpr uint32_t Q = 0;                          // 2 stages x 2 slabs x 128 rows
@@ -321,13 +322,16 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 if (!sm100::mbar_wait(&bars[RFULL + st], (n / NSLOT) & 1, err)) return false;  // G, cf
                 sm100::tc_fence_after();
                 const float *gJ = sGC + st * 2 * JT, *cfJ = gJ + JT;
-                // In the diagonal tile, a row below the half's 64-token group sees all of it
-                // (anchored split as off the diagonal), a row above sees none of it, and only
-                // the group's own rows need the exact per-element factor.
+                // In the diagonal tile, a row below the half's 64-token group sees all of it,
+                // a row above sees none of it, and a row inside it sees the columns s <= r.
+                // Every row takes the split e^{G_r - a} cf_s with a = G at the group's last
+                // token (the anchor cf was made with); inside the group e^{G_r - a} >= 1, so a
+                // row whose exponent exceeds kSplitMax takes the exact e^{G_r - G_s} instead.
                 const bool none = diag && r < 64 * half;
-                const bool exact = diag && !none && r < 64 * half + 64;
-                // split: the half's anchor is G at the end of its 64-token group
-                const float rf = (it.valid && !none && !exact) ? __expf(it.Gr - gJ[64 * half + 63]) : 0.f;
+                const bool in_group = diag && !none && r < 64 * half + 64;
+                const float dG = it.Gr - gJ[min(64 * half + 63, L - 1 - j * JT)];
+                const bool exact = in_group && !(dG <= kSplitMax);
+                const float rf = (it.valid && !none && !exact) ? __expf(dG) : 0.f;
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr) {  // two rounds of 32 columns: S read before P overwrites it
                     const int c0 = 64 * half + 32 * rr;
@@ -337,8 +341,14 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     uint32_t pk[16];
                     if (!exact) {  // rf = 0 where the row sees none of the half
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2)
-                            pk[e >> 1] = pack_bf16(v[e] * rf * cfJ[c0 + e], v[e + 1] * rf * cfJ[c0 + e + 1]);
+                        for (int e = 0; e < 32; e += 2) {
+                            float f0 = rf * cfJ[c0 + e], f1 = rf * cfJ[c0 + e + 1];
+                            if (in_group) {  // the causal mask inside the group
+                                f0 = c0 + e <= r ? f0 : 0.f;
+                                f1 = c0 + e + 1 <= r ? f1 : 0.f;
+                            }
+                            pk[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
+                        }
                     } else {
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
