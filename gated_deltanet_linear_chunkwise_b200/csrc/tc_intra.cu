@@ -335,12 +335,15 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 const float *gJ = sGC + st * GCT_FLOATS, *cfJ = gJ + CT;
                 // the tile lies before block i, so it is full: the half's anchor is G at its last token
                 const float rf = valid ? -be * __expf(Gr - gJ[64 * half + 63]) : 0.f;
+                // the half's 64 S columns with one wait; P then goes over the first 32 of them
+                float vs[2][32];
+                sm100::tmem_ld32(t_s0 + sb * CT + lane_off + 64 * half, vs[0]);
+                sm100::tmem_ld32(t_s0 + sb * CT + lane_off + 64 * half + 32, vs[1]);
+                sm100::tmem_ld_wait();
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {  // two rounds of 32 columns: S read before P overwrites it
+                for (int rr = 0; rr < 2; ++rr) {
                     const int c0 = 64 * half + 32 * rr;
-                    float v[32];
-                    sm100::tmem_ld32(t_s0 + sb * CT + lane_off + c0, v);
-                    sm100::tmem_ld_wait();
+                    const float (&v)[32] = vs[rr];
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2)
@@ -371,55 +374,58 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     vrow[c8] = (valid && c8 < dv / 8) ? __ldg(reinterpret_cast<const uint4 *>(vp) + c8)
                                                       : make_uint4(0, 0, 0, 0);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int c16 = 16 * j;
-                    if (c16 >= dv) break;
-                    float acc[16];
-                    if (i > 0) {
-                        sm100::tmem_ld16(t_acc + lane_off + c16, acc);
+                for (int j2 = 0; j2 < 4; ++j2) {  // two 16-column loads per wait
+                    if (32 * j2 >= dv) break;
+                    float acc[2][16];
+                    if (i > 0) {  // the second load may read past dv, inside the accumulator
+                        sm100::tmem_ld16(t_acc + lane_off + 32 * j2, acc[0]);
+                        sm100::tmem_ld16(t_acc + lane_off + 32 * j2 + 16, acc[1]);
                         sm100::tmem_ld_wait();
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+                        for (int e = 0; e < 16; ++e) acc[0][e] = acc[1][e] = 0.f;
                     }
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const __nv_bfloat162 *vb = reinterpret_cast<const __nv_bfloat162 *>(&vrow[2 * j + u]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = 32 * j2 + 8 * u;
+                        if (c >= dv) break;
+                        const __nv_bfloat162 *vb = reinterpret_cast<const __nv_bfloat162 *>(&vrow[4 * j2 + u]);
                         float y[8];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 fv = __bfloat1622float2(vb[e]);
-                            y[2 * e] = be * fv.x + acc[u * 8 + 2 * e];
-                            y[2 * e + 1] = be * fv.y + acc[u * 8 + 2 * e + 1];
+                            y[2 * e] = be * fv.x + acc[u >> 1][(u & 1) * 8 + 2 * e];
+                            y[2 * e + 1] = be * fv.y + acc[u >> 1][(u & 1) * 8 + 2 * e + 1];
                         }
-                        store_y(c16 + 8 * u, y);
+                        store_y(c, y);
                     }
                 }
             } else {  // W columns: beta_r e^{G_r} k_r + acc
                 const float rk = be * __expf(Gr);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int kc16 = 16 * j;
-                    if (kc16 >= dk) break;
-                    float acc[16];
-                    if (i > 0) {
-                        sm100::tmem_ld16(t_acc + lane_off + dv + kc16, acc);
+                for (int j2 = 0; j2 < 4; ++j2) {  // two 16-column loads per wait
+                    if (32 * j2 >= dk) break;
+                    float acc[2][16];
+                    if (i > 0) {  // the second load may read past dk, inside the accumulator
+                        sm100::tmem_ld16(t_acc + lane_off + dv + 32 * j2, acc[0]);
+                        sm100::tmem_ld16(t_acc + lane_off + dv + 32 * j2 + 16, acc[1]);
                         sm100::tmem_ld_wait();
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+                        for (int e = 0; e < 16; ++e) acc[0][e] = acc[1][e] = 0.f;
                     }
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int kc = kc16 + 8 * u;
+                    for (int u = 0; u < 4; ++u) {
+                        const int kc = 32 * j2 + 8 * u;
+                        if (kc >= dk) break;
                         const uint4 kv = *reinterpret_cast<const uint4 *>(sKi + yx_offset(kc, r));
                         const __nv_bfloat162 *kb = reinterpret_cast<const __nv_bfloat162 *>(&kv);
                         float y[8];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 fk = __bfloat1622float2(kb[e]);
-                            y[2 * e] = rk * fk.x + acc[u * 8 + 2 * e];
-                            y[2 * e + 1] = rk * fk.y + acc[u * 8 + 2 * e + 1];
+                            y[2 * e] = rk * fk.x + acc[u >> 1][(u & 1) * 8 + 2 * e];
+                            y[2 * e + 1] = rk * fk.y + acc[u >> 1][(u & 1) * 8 + 2 * e + 1];
                         }
                         store_y(dv + kc, y);
                     }
@@ -440,15 +446,22 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             if (!ok) break;
             sm100::tc_fence_after();
             const int c_lo = half ? dv : 0, c_hi = half ? nc : dv;
-            for (int c16 = c_lo; c16 < c_hi; c16 += 16) {
-                float x[16];
-                sm100::tmem_ld16(t_acc + lane_off + c16, x);
+            // two 16-column loads per wait (the second may read past c_hi, inside the
+            // accumulator's 256 columns, and is then not stored)
+            for (int c32 = c_lo; c32 < c_hi; c32 += 32) {
+                float x[2][16];
+                sm100::tmem_ld16(t_acc + lane_off + c32, x[0]);
+                sm100::tmem_ld16(t_acc + lane_off + c32 + 16, x[1]);
                 sm100::tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    *reinterpret_cast<uint4 *>(sYX + yx_offset(c16 + 8 * u, r)) =
-                        make_uint4(pack_bf16(x[8 * u], x[8 * u + 1]), pack_bf16(x[8 * u + 2], x[8 * u + 3]),
-                                   pack_bf16(x[8 * u + 4], x[8 * u + 5]), pack_bf16(x[8 * u + 6], x[8 * u + 7]));
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    if (c32 + 16 * h2 >= c_hi) break;
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+                        *reinterpret_cast<uint4 *>(sYX + yx_offset(c32 + 16 * h2 + 8 * u, r)) = make_uint4(
+                            pack_bf16(x[h2][8 * u], x[h2][8 * u + 1]), pack_bf16(x[h2][8 * u + 2], x[h2][8 * u + 3]),
+                            pack_bf16(x[h2][8 * u + 4], x[h2][8 * u + 5]), pack_bf16(x[h2][8 * u + 6], x[h2][8 * u + 7]));
+                }
             }
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();

@@ -333,11 +333,15 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const bool exact = in_group && !(dG <= kSplitMax);
                 const float rf = (it.valid && !none && !exact) ? __expf(dG) : 0.f;
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {  // two rounds of 32 columns: S read before P overwrites it
+                // the half's 64 S columns with one wait; P then goes over the first 32 of them
+                float vs[2][32];
+                sm100::tmem_ld32(t_s0 + sb * JT + lane_off + 64 * half, vs[0]);
+                sm100::tmem_ld32(t_s0 + sb * JT + lane_off + 64 * half + 32, vs[1]);
+                sm100::tmem_ld_wait();
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
                     const int c0 = 64 * half + 32 * rr;
-                    float v[32];
-                    sm100::tmem_ld32(t_s0 + sb * JT + lane_off + c0, v);
-                    sm100::tmem_ld_wait();
+                    const float (&v)[32] = vs[rr];
                     uint32_t pk[16];
                     if (!exact) {  // rf = 0 where the row sees none of the half
 #pragma unroll
@@ -374,11 +378,21 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             sm100::tc_fence_after();
             const long long tt = it.f * L + it.row;
             __nv_bfloat16 *o = (__nv_bfloat16 *)prm.o + ((((long long)it.b * prm.T + tt) * prm.H + it.h) * dv);
-            for (int c = 16 * half; c < dv; c += 32) {
-                float acc[16];
-                sm100::tmem_ld16(t_o0 + ob * 128 + lane_off + c, acc);
+            // columns c = 16 half + 32 i (dv <= 128), two 16-column loads per wait (the second
+            // may read past dv, inside the O buffer's 128 columns, and is then not stored)
+#pragma unroll
+            for (int i2 = 0; i2 < 2; ++i2) {
+                const int cb = 16 * half + 64 * i2;
+                if (cb >= dv) break;
+                float acc[2][16];
+                sm100::tmem_ld16(t_o0 + ob * 128 + lane_off + cb, acc[0]);
+                sm100::tmem_ld16(t_o0 + ob * 128 + lane_off + cb + 32, acc[1]);
                 sm100::tmem_ld_wait();
-                if (it.valid) {
+                if (!it.valid) continue;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int c = cb + 32 * i;
+                    if (c >= dv) break;
                     if (prm.accumulate) {
                         const uint4 *old = reinterpret_cast<const uint4 *>(o + c);
 #pragma unroll
@@ -388,17 +402,18 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const float2 fl = __bfloat1622float2(xb[e]);
-                                acc[w2 * 8 + 2 * e] += fl.x;
-                                acc[w2 * 8 + 2 * e + 1] += fl.y;
+                                acc[i][w2 * 8 + 2 * e] += fl.x;
+                                acc[i][w2 * 8 + 2 * e + 1] += fl.y;
                             }
                         }
                     }
+                    const float *a16 = acc[i];
                     reinterpret_cast<uint4 *>(o + c)[0] =
-                        make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]), pack_bf16(acc[4], acc[5]),
-                                   pack_bf16(acc[6], acc[7]));
+                        make_uint4(pack_bf16(a16[0], a16[1]), pack_bf16(a16[2], a16[3]), pack_bf16(a16[4], a16[5]),
+                                   pack_bf16(a16[6], a16[7]));
                     reinterpret_cast<uint4 *>(o + c)[1] =
-                        make_uint4(pack_bf16(acc[8], acc[9]), pack_bf16(acc[10], acc[11]),
-                                   pack_bf16(acc[12], acc[13]), pack_bf16(acc[14], acc[15]));
+                        make_uint4(pack_bf16(a16[8], a16[9]), pack_bf16(a16[10], a16[11]),
+                                   pack_bf16(a16[12], a16[13]), pack_bf16(a16[14], a16[15]));
                 }
             }
             sm100::tc_fence_before();

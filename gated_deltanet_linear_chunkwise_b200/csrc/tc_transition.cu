@@ -138,12 +138,18 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
             const float eGL = __expf(GL);
             const int m = r;
-            for (int c0 = 0; c0 < nc; c0 += 16) {
-                float v[16];
-                sm100::tmem_ld16(t_d + lane_off + c0, v);
+            for (int c4 = 0; c4 < nc; c4 += 64) {  // four 16-column loads per wait (the last group may
+                float v4[4][16];                   // read past nc, inside the 256-column buffer, unused)
+#pragma unroll
+                for (int g = 0; g < 4; ++g) sm100::tmem_ld16(t_d + lane_off + c4 + 16 * g, v4[g]);
                 sm100::tmem_ld_wait();
-                if (m < dk) {  // dv is a multiple of 16: a chunk lies wholly in N or in M
-                    float *dst;
+                if (m >= dk) continue;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int c0 = c4 + 16 * g;
+                    if (c0 >= nc) break;
+                    float *v = v4[g];
+                    float *dst;  // dv is a multiple of 16: a chunk lies wholly in N or in M
                     if (c0 < dv) {
                         dst = prm.N + (fh * dk + m) * (long long)dv + c0;
                     } else {
