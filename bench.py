@@ -16,6 +16,7 @@ from __future__ import annotations
 import argparse
 import ctypes
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -72,6 +73,22 @@ def flops_total(L, dk, dv):
 def bytes_alg(B, T, H, dk, dv, elem=2):
     # read q, k, v; write o; alpha and beta fp32; state I/O (fp32 in + out)
     return B * T * H * (2 * dk + 2 * dv) * elem + 8 * B * T * H + 2 * B * H * dk * dv * 4
+
+
+def framewise_line(B, T, H, dk, dv, L, ms, stage, pk, stages):
+    """The frame-wise operator's pass: HBM bound (algorithmic bytes: q, k, v and beta read once,
+    o written once; FLOPs per frame-head 2L d_k (d_k + d_v) + 2 d_k^2 d_v + 2 L d_k d_v)."""
+    nfh = B * H * (T // L)
+    byts = B * T * H * ((2 * dk + 2 * dv) * 2 + 4)
+    flops = nfh * (2 * L * dk * (dk + dv) + 2 * dk * dk * dv + 2 * L * dk * dv)
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"ms_per_pass": ms, "tokens_per_s": B * T / (ms * 1e-3),
+            "what": "frame-wise operator (mode=frame) on the same inputs, keys / sqrt(frame_len); "
+                    "not the timed metric",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "bytes": byts, "flops": flops,
+                         "achieved_tflops": flops / (ms * 1e-3) / 1e12},
+            "stage_ms": {n: stage[i] for i, n in enumerate(stages) if n in ("transition", "scan", "output")}}
 
 
 def peaks():
@@ -267,6 +284,32 @@ def main():
     torch.cuda.synchronize(dev)
     bidir_ms = gdist.max_over_ranks(b0.elapsed_time(b1) / 3, device=dev)
 
+    # the frame-wise operator (NEXT row: one state update per frame) on the same q/k/v/beta,
+    # keys scaled by 1/sqrt(frame_len) so the frame transitions are non-expansive
+    k_fw = (d["k"].float() / math.sqrt(L)).to(d["k"].dtype)
+    gamma = W.draw_frame_decay(B, w.frames, H, seed=W.SEEDS[args.workload] + 7919 * rank + 1,
+                               regime=args.regime).to(dev)
+
+    def framewise(stage_ms=None):
+        g.gdn_fwd(d["q"], k_fw, d["v"], None, d["beta"], L, None, S_out=S_out, o=o, stream=stream,
+                  stage_ms=stage_ms, mode="frame", gamma=gamma)
+
+    for _ in range(3):
+        framewise()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(10):
+        framewise()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    fw_ms = gdist.max_over_ranks(f0.elapsed_time(f1) / 10, device=dev)
+    fw_stage = [0.0] * NUM_STAGES
+    for _ in range(3):
+        arr = (ctypes.c_float * NUM_STAGES)()
+        framewise(stage_ms=arr)
+        for i in range(NUM_STAGES):
+            fw_stage[i] += arr[i] / 3
+
     # per-stage device times (events around each kernel on the same stream)
     stage_sum = [0.0] * NUM_STAGES
     reps = 5
@@ -347,6 +390,7 @@ def main():
             "gpu_launches": NUM_STAGES * args.steps,
             "bidirectional": {"ms_per_pass": bidir_ms, "tokens_per_s": tokens / (bidir_ms * 1e-3),
                               "what": "forward + reversed scan summed into o (not the timed metric)"},
+            "framewise": framewise_line(B * world, T, H, dk, dv, L, fw_ms, fw_stage, pk, STAGES),
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline and world == 1 and args.workload == WORKLOAD:

@@ -46,7 +46,11 @@ class GdnArgs(ctypes.Structure):
         ("reverse", ctypes.c_int), ("accumulate_o", ctypes.c_int),
         ("reset_every", ctypes.c_longlong), ("check_finite", ctypes.c_int),
         ("stream", ctypes.c_void_p), ("stage_ms", ctypes.c_void_p),
+        ("mode", ctypes.c_int), ("gamma", ctypes.c_void_p),
     ]
+
+GDN_MODE_TOKEN = 0
+GDN_MODE_FRAME = 1
 
 NUM_STAGES = 7
 STAGES = ("gates", "diag_inverse", "intra", "transition", "scan", "u", "output")
@@ -113,7 +117,7 @@ def _stream_handle(stream, device):
 
 def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
             return_state=False, reverse=False, accumulate=False, reset_every=0,
-            check_finite=False, workspace=None, stream=None, stage_ms=None):
+            check_finite=False, workspace=None, stream=None, stage_ms=None, mode="token", gamma=None):
     """Chunkwise gated delta rule forward on CUDA tensors.
 
     q,k [B,T,H,d_k], v [B,T,H,d_v] (bf16 or fp32, all the same), alpha/beta
@@ -122,20 +126,31 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     with ``return_state`` and no ``S_out`` a state tensor is allocated.
     ``stage_ms`` (a ``(ctypes.c_float * NUM_STAGES)()``) receives each kernel
     stage's device time; that call synchronises the stream.
+    ``mode="frame"`` runs the frame-wise operator instead (one state update
+    per frame of ``frame_len`` tokens); it reads ``gamma`` [B, T/frame_len, H]
+    fp32, the per-frame decay, and not ``alpha`` (which may be None).
     Returns (o, S_out or None).
     """
     import torch
     B, T, H, d_k = q.shape
     d_v = v.shape[-1]
-    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta)):
+    if mode not in ("token", "frame"):
+        raise GdnError(1, "mode must be 'token' or 'frame'")
+    frame = mode == "frame"
+    gates = (("beta", beta), ("gamma", gamma)) if frame else (("alpha", alpha), ("beta", beta))
+    for name, t in (("q", q), ("k", k), ("v", v)) + gates:
+        if t is None:
+            raise GdnError(1, "%s is required" % name)
         if not t.is_cuda:
             raise GdnError(1, "%s is not a CUDA tensor" % name)
         if not t.is_contiguous():
             raise GdnError(1, "%s is not contiguous" % name)
     if q.dtype != k.dtype or q.dtype != v.dtype or q.dtype not in (torch.bfloat16, torch.float32):
         raise GdnError(1, "q/k/v must share one dtype, bf16 or fp32")
-    if alpha.dtype != torch.float32 or beta.dtype != torch.float32:
-        raise GdnError(1, "alpha and beta must be fp32")
+    if any(t.dtype != torch.float32 for _, t in gates):
+        raise GdnError(1, "%s must be fp32" % " and ".join(n for n, _ in gates))
+    if frame and tuple(gamma.shape) != (B, T // max(int(frame_len), 1), H):
+        raise GdnError(2, "gamma must have shape [B, T / frame_len, H]")
     for name, t in (("S_in", S_in), ("S_out", S_out), ("o", o)):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise GdnError(1, "%s must be a contiguous CUDA tensor" % name)
@@ -147,8 +162,10 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     a.struct_size = ctypes.sizeof(GdnArgs)
     a.dtype = GDN_DTYPE_BF16 if q.dtype == torch.bfloat16 else GDN_DTYPE_F32
     a.q, a.k, a.v = _ptr(q), _ptr(k), _ptr(v)
-    a.alpha, a.beta = _ptr(alpha), _ptr(beta)
+    a.alpha, a.beta = (None if frame else _ptr(alpha)), _ptr(beta)
     a.S_in, a.S_out, a.o = _ptr(S_in), _ptr(S_out), _ptr(o)
+    a.mode = GDN_MODE_FRAME if frame else GDN_MODE_TOKEN
+    a.gamma = _ptr(gamma) if frame else None
     a.B, a.H, a.T = B, H, T
     a.frame_len, a.d_k, a.d_v = int(frame_len), d_k, d_v
     if workspace is not None:

@@ -84,6 +84,10 @@ int validate_sizes(const gdn_args &a) {
     if (a.reverse != 0 && a.reverse != 1) { set_err("reverse must be 0 or 1"); return GDN_ERR_INVALID_ARG; }
     if (a.accumulate_o != 0 && a.accumulate_o != 1) { set_err("accumulate_o must be 0 or 1"); return GDN_ERR_INVALID_ARG; }
     if (a.check_finite != 0 && a.check_finite != 1) { set_err("check_finite must be 0 or 1"); return GDN_ERR_INVALID_ARG; }
+    if (a.mode != GDN_MODE_TOKEN && a.mode != GDN_MODE_FRAME) {
+        set_err("mode must be GDN_MODE_TOKEN or GDN_MODE_FRAME (got %d)", a.mode);
+        return GDN_ERR_INVALID_ARG;
+    }
     if (a.reset_every < 0 || (a.reset_every > 0 && a.reset_every % a.frame_len != 0)) {
         set_err("reset_every (%lld) must be 0 or a positive multiple of frame_len (%d)", a.reset_every, a.frame_len);
         return GDN_ERR_INVALID_ARG;
@@ -120,8 +124,17 @@ int validate(const gdn_args &a, gdn::Problem &p) {
     if (st != GDN_OK) return st;
     const long long F = a.T / a.frame_len;
     const bool empty = (a.B == 0 || a.H == 0 || a.T == 0);
-    if (!empty && (!a.q || !a.k || !a.v || !a.alpha || !a.beta || !a.o)) {
-        set_err("q, k, v, alpha, beta and o are required (one is NULL)");
+    const bool frame = a.mode == GDN_MODE_FRAME;
+    if (!empty && (!a.q || !a.k || !a.v || !a.beta || !a.o)) {
+        set_err("q, k, v, beta and o are required (one is NULL)");
+        return GDN_ERR_INVALID_ARG;
+    }
+    if (!empty && !frame && !a.alpha) {
+        set_err("alpha is required (NULL)");
+        return GDN_ERR_INVALID_ARG;
+    }
+    if (!empty && frame && !a.gamma) {
+        set_err("gamma is required in GDN_MODE_FRAME (NULL)");
         return GDN_ERR_INVALID_ARG;
     }
     const void *ptrs[] = {a.q, a.k, a.v, a.alpha, a.beta, a.S_in, a.S_out, a.o};
@@ -139,15 +152,17 @@ int validate(const gdn_args &a, gdn::Problem &p) {
     const size_t es = a.dtype == GDN_DTYPE_BF16 ? 2 : 4;
     const size_t nqk = (size_t)a.B * a.T * a.H * a.d_k * es, nv = (size_t)a.B * a.T * a.H * a.d_v * es;
     const size_t ng = (size_t)a.B * a.T * a.H * 4, ns = (size_t)a.B * a.H * a.d_v * a.d_k * 4;
-    const void *ins[] = {a.q, a.k, a.v, a.alpha, a.beta, a.S_in};
-    const size_t insz[] = {nqk, nqk, nv, ng, ng, ns};
-    for (int i = 0; i < 6; ++i) {
+    const size_t ngam = frame ? (size_t)a.B * F * a.H * 4 : 0;
+    const void *ins[] = {a.q, a.k, a.v, frame ? nullptr : a.alpha, a.beta, a.S_in, frame ? a.gamma : nullptr};
+    const size_t insz[] = {nqk, nqk, nv, ng, ng, ns, ngam};
+    const char *in_names[] = {"q", "k", "v", "alpha", "beta", "S_in", "gamma"};
+    for (int i = 0; i < 7; ++i) {
         if (overlap(a.o, nv, ins[i], insz[i])) {
-            set_err("o overlaps input %s", names[i]);
+            set_err("o overlaps input %s", in_names[i]);
             return GDN_ERR_INVALID_ARG;
         }
         if (a.S_out && !(i == 5 && a.S_out == a.S_in) && overlap(a.S_out, ns, ins[i], insz[i])) {
-            set_err("S_out overlaps input %s", names[i]);
+            set_err("S_out overlaps input %s", in_names[i]);
             return GDN_ERR_INVALID_ARG;
         }
     }
@@ -160,6 +175,8 @@ int validate(const gdn_args &a, gdn::Problem &p) {
     p.B = a.B; p.H = a.H; p.T = a.T; p.L = a.frame_len;
     p.dk = a.d_k; p.dv = a.d_v; p.F = F;
     p.reverse = a.reverse; p.accumulate = a.accumulate_o; p.reset_every = a.reset_every;
+    p.mode = a.mode; p.gamma = frame ? a.gamma : nullptr;
+    if (frame) p.alpha = nullptr;
     return GDN_OK;
 }
 

@@ -47,7 +47,16 @@ struct Problem {
     int reverse;
     int accumulate;
     long long reset_every;  // tokens; 0 = never
+    int mode;               // GDN_MODE_TOKEN / GDN_MODE_FRAME
+    const float *gamma;     // GDN_MODE_FRAME: [B, F, H] per-frame decay
 };
+
+// Memory index of the frame the scan visits at logical step f.  The
+// token-wise paths store per-frame data in visiting order; the frame-wise
+// operator stores it by time and the scan walks it backwards when reversed.
+__host__ __device__ __forceinline__ long long scan_frame(const Problem &p, long long f) {
+    return (p.mode == GDN_MODE_FRAME && p.reverse) ? p.F - 1 - f : f;
+}
 
 // Physical token index of logical position i of logical frame f.  The
 // reversed-time scan visits frames and the tokens inside them backwards.
@@ -103,5 +112,7 @@ cudaError_t simt_scan(const Problem &p, const float *Mb, const float *Nb, float 
 cudaError_t simt_u_bf16x(const Problem &p, const __nv_bfloat16 *X, const float *Sig, __nv_bfloat16 *U,
                          cudaStream_t s);
 cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
+// The frame-wise operator on the CUDA cores (launch_simt dispatches to it).
+cudaError_t launch_simt_frame(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
 
 }  // namespace gdn

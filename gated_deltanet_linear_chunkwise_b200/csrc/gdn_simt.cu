@@ -232,7 +232,9 @@ __global__ void __launch_bounds__(NT) k2_transition_simt(Problem p, const TX *__
 // ---------------------------------------------------------------- k3 scan over frames
 // grid (B*H, ceil(dv/16)); the block carries 16 columns of Sig = S^T through
 // all frames of its chain (Sig_next = M Sig + N), writing the state entering
-// each frame to SigIn (fp32) and/or SigB (bf16).  The next frame's M is
+// each frame (token-wise operator) or the state after each frame's update
+// (frame-wise operator, whose tokens read the post-update state) to SigIn
+// (fp32) and/or SigB (bf16).  The next frame's M is
 // brought in by cp.async into the other half of a double buffer while the
 // current step computes.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -273,8 +275,9 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
         sS[e] = val;
     }
     constexpr int NVEC = DK * DK / 4;  // 16-byte pieces of one M
+    const bool post = p.mode == GDN_MODE_FRAME;
     if (p.F > 0) {
-        const float4 *src = reinterpret_cast<const float4 *>(Mb + chain * p.F * (long long)DK * DK);
+        const float4 *src = reinterpret_cast<const float4 *>(Mb + (chain * p.F + scan_frame(p, 0)) * (long long)DK * DK);
         for (int e = tid; e < NVEC; e += NT) cp_async16(sM + 4 * e, src + e);
     }
     cp_async_commit();
@@ -285,17 +288,18 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
         const int m = g + 16 * i;
         nxt[i] = make_float2(0.f, 0.f);
         if (kh == 0 && p.F > 0) {
-            const long long idx = (chain * p.F * DK + m) * (long long)dv + c0;
+            const long long idx = ((chain * p.F + scan_frame(p, 0)) * DK + m) * (long long)dv + c0;
             nxt[i].x = ca < ncol ? Nb[idx + ca] : 0.f;
             nxt[i].y = cb < ncol ? Nb[idx + cb] : 0.f;
         }
     }
     __syncthreads();
     for (long long f = 0; f < p.F; ++f) {
-        const long long fh = chain * p.F + f;
+        const long long fh = chain * p.F + scan_frame(p, f);
+        const long long fhn = f + 1 < p.F ? chain * p.F + scan_frame(p, f + 1) : fh;
         const int buf = (int)(f & 1);
         if (f + 1 < p.F) {  // prefetch the next frame's M into the other buffer
-            const float4 *src = reinterpret_cast<const float4 *>(Mb + (fh + 1) * (long long)DK * DK);
+            const float4 *src = reinterpret_cast<const float4 *>(Mb + fhn * (long long)DK * DK);
             float *dst = sM + (buf ^ 1) * DK * DK;
             for (int e = tid; e < NVEC; e += NT) cp_async16(dst + 4 * e, src + e);
         }
@@ -313,9 +317,9 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
             if (kh == 0) {
                 const long long idx = (fh * DK + m) * (long long)dv + c0;
                 const float2 cur = *reinterpret_cast<const float2 *>(&sS[m * SCAN_COLS + ca]);
-                if (SigIn) *reinterpret_cast<float2 *>(SigIn + idx + ca) = cur;
-                if (SigB) *reinterpret_cast<__nv_bfloat162 *>(SigB + idx + ca) = __floats2bfloat162_rn(cur.x, cur.y);
-                if (f + 1 < p.F) nxt[i] = *reinterpret_cast<const float2 *>(Nb + ((fh + 1) * DK + m) * (long long)dv + c0 + ca);
+                if (!post && SigIn) *reinterpret_cast<float2 *>(SigIn + idx + ca) = cur;
+                if (!post && SigB) *reinterpret_cast<__nv_bfloat162 *>(SigB + idx + ca) = __floats2bfloat162_rn(cur.x, cur.y);
+                if (f + 1 < p.F) nxt[i] = *reinterpret_cast<const float2 *>(Nb + (fhn * DK + m) * (long long)dv + c0 + ca);
             }
         }
         cp_async_wait_one();  // this frame's M (committed one step earlier) has landed
@@ -351,7 +355,13 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
             for (int i = 0; i < R; ++i) {
                 const int m = g + 16 * i;
                 const float2 o = sRed[i * 128 + t7];
-                *reinterpret_cast<float2 *>(&sS[m * SCAN_COLS + ca]) = make_float2(acc[i].x + o.x, acc[i].y + o.y);
+                const float2 nw = make_float2(acc[i].x + o.x, acc[i].y + o.y);
+                *reinterpret_cast<float2 *>(&sS[m * SCAN_COLS + ca]) = nw;
+                if (post) {  // the state after this frame's update
+                    const long long idx = (fh * DK + m) * (long long)dv + c0;
+                    if (SigIn) *reinterpret_cast<float2 *>(SigIn + idx + ca) = nw;
+                    if (SigB) *reinterpret_cast<__nv_bfloat162 *>(SigB + idx + ca) = __floats2bfloat162_rn(nw.x, nw.y);
+                }
             }
         }
         __syncthreads();
@@ -653,6 +663,7 @@ SimtLayout simt_layout(const Problem &p) {
 size_t simt_workspace_bytes(const Problem &p) { return simt_layout(p).total; }
 
 cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
+    if (p.mode == GDN_MODE_FRAME) return launch_simt_frame(p, ws, s, ev);
     if (p.dtype == GDN_DTYPE_F32) return launch_typed<float, double>(p, ws, s, ev);
     return launch_typed<__nv_bfloat16, float>(p, ws, s, ev);
 }

@@ -216,7 +216,8 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     tc::TransParams tp;
     tp.G = G; tp.M = Mb; tp.N = Nb;
     tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
-    if ((e = tc::launch_transition_tc(tm_k64, tm_x, tp, nfh, s))) return e;
+    tp.frame = 0; tp.beta = p.beta; tp.gamma = nullptr; tp.T = p.T;
+    if ((e = tc::launch_transition_tc(tm_k64, tm_x, tm_x, tp, nfh, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
     Problem ps = p;
     ps.reverse = scan_reverse;
@@ -225,7 +226,8 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     tc::UParams up;
     up.X = X; up.U = U;
     up.L = p.L; up.dk = p.dk; up.dv = p.dv; up.nblk = nblk; up.err = err;
-    if ((e = tc::launch_u_tc(tm_x128, tm_sig, up, nfh, s))) return e;
+    up.frame = 0; up.o = nullptr; up.T = p.T; up.F = p.F; up.H = p.H; up.accumulate = 0;
+    if ((e = tc::launch_u_tc(tm_x128, tm_q, tm_sig, up, nfh, s))) return e;
     if ((e = mark(ev, 6, s))) return e;
 
     tc::OutParams op;
@@ -281,7 +283,47 @@ cudaError_t reverse_rows(const void *src, void *dst, int B, long long T, size_t 
 
 }  // namespace
 
+// The frame-wise operator (SANA-WM summary, "Memory-Efficient Long-Context Modeling
+// (Section 3.2)", paragraph "Adaptation to video: frame-wise recurrence"): the per-frame
+// maps M = gamma (I - K^T B K), N = K^T B V (transition kernel, frame mode), the scan
+// (states after each frame's update; frames walked backwards when reversed), and
+// o (+)= Q Sig_t (U kernel, frame mode).  Per-frame sums do not depend on token order, so
+// a reversed call needs no reversed copies.
+cudaError_t launch_tc_frame(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
+    const TcLayout lay = tc_layout(p);
+    char *base = (char *)ws;
+    const long long nfh = (long long)p.B * p.H * p.F;
+    const int nblk = (p.L + tc::BM - 1) / tc::BM;
+    float *Mb = (float *)(base + lay.M), *Nb = (float *)(base + lay.N);
+    __nv_bfloat16 *SigB = (__nv_bfloat16 *)(base + lay.SigB);
+    int *err = (int *)(base + lay.err);
+    cudaError_t e;
+    CUtensorMap tm_q, tm_k64, tm_v64, tm_sig;
+    if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k64, p.k, p, p.dk, 64) ||
+        !map_tokens(&tm_v64, p.v, p, p.dv, 64) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk))
+        return cudaErrorInvalidValue;
+    if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
+    // stages 0-2 (gates, inverses, intra solve) and 5 (U) do not exist in this operator
+    for (int i = 0; i <= 3; ++i)
+        if ((e = mark(ev, i, s))) return e;
+    tc::TransParams tp;
+    tp.G = nullptr; tp.M = Mb; tp.N = Nb;
+    tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
+    tp.frame = 1; tp.beta = p.beta; tp.gamma = p.gamma; tp.T = p.T;
+    if ((e = tc::launch_transition_tc(tm_k64, tm_k64, tm_v64, tp, nfh, s))) return e;
+    if ((e = mark(ev, 4, s))) return e;
+    if ((e = simt_scan(p, Mb, Nb, nullptr, SigB, s))) return e;
+    if ((e = mark(ev, 5, s)) || (e = mark(ev, 6, s))) return e;
+    tc::UParams up;
+    up.X = nullptr; up.U = nullptr;
+    up.L = p.L; up.dk = p.dk; up.dv = p.dv; up.nblk = nblk; up.err = err;
+    up.frame = 1; up.o = (__nv_bfloat16 *)p.o; up.T = p.T; up.F = p.F; up.H = p.H; up.accumulate = p.accumulate;
+    if ((e = tc::launch_u_tc(tm_q, tm_q, tm_sig, up, nfh, s))) return e;
+    return mark(ev, 7, s);
+}
+
 cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
+    if (p.mode == GDN_MODE_FRAME) return launch_tc_frame(p, ws, s, ev);
     if (!p.reverse && !p.accumulate) return launch_tc_forward(p, ws, 0, s, ev);
     const TcLayout lay = tc_layout(p);
     char *base = (char *)ws;

@@ -66,6 +66,12 @@ struct TransParams {
     int L, dk, dv, H, nblk;
     long long F;
     int *err;
+    // frame-wise operator: M = gamma (I - K^T diag(beta) K), N = K^T diag(beta) V straight
+    // from the inputs (G and the [Ub | W] rows are not read)
+    int frame;
+    const float *beta;         // [B,T,H]
+    const float *gamma;        // [B,F,H]
+    long long T;
 };
 
 struct UParams {
@@ -73,14 +79,21 @@ struct UParams {
     __nv_bfloat16 *U;          // [n_fh][L][dv]
     int L, dk, dv, nblk;
     int *err;
+    // frame-wise operator: A = the frame's queries (tm_q), o = Q Sig written (or added) to o
+    int frame;
+    __nv_bfloat16 *o;          // [B,T,H,dv]
+    long long T, F;
+    int H, accumulate;
 };
 
-// tm_k / tm_x deliver 64-token boxes.
-cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const TransParams &prm,
-                                 long long n_fh, cudaStream_t s);
-// tm_x delivers 128-row boxes of X, tm_sig the bf16 state of a frame-head.
-cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_sig, const UParams &prm, long long n_fh,
-                        cudaStream_t s);
+// tm_k / tm_x / tm_v deliver 64-token boxes (tm_x the [Ub | W] rows, tm_v the
+// values, read by the frame-wise operator only).
+cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_v,
+                                 const TransParams &prm, long long n_fh, cudaStream_t s);
+// tm_x delivers 128-row boxes of X, tm_q 128-token boxes of q (frame-wise
+// operator), tm_sig the bf16 state of a frame-head.
+cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_q, const CUtensorMap &tm_sig,
+                        const UParams &prm, long long n_fh, cudaStream_t s);
 
 // tm_k delivers 128-token boxes of k, tm_x64 64-row boxes of X, tm_t one
 // 128 x 128 block, tm_gct the G and cf of one 128-token tile; tm_xs stores

@@ -14,6 +14,12 @@
 // in TMEM with one lane per key dimension.  The epilogue warps scale the K
 // rows in shared memory by e^{G_L - G_r} (a per-row factor, so the swizzle
 // does not matter) and finally write M and N in fp32.
+// The same kernel forms the frame-wise operator's map (SANA-WM summary,
+// "Memory-Efficient Long-Context Modeling (Section 3.2)", paragraph
+// "Adaptation to video: frame-wise recurrence"): M = gamma (I - K^T B K),
+// N = K^T B V with B = diag(beta); then the K rows are scaled by beta and the
+// B operand is [V | K] loaded from the inputs (V in the first 64-column slabs,
+// K after them), so D = K^T B [V | K].
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -35,7 +41,7 @@ enum Bar { FULL = 0, SCALED = FULL + NST, EMPTY = SCALED + NST, DONE = EMPTY + N
 
 __global__ void __launch_bounds__(kThreads, 2)
 k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_x,
-                const TransParams prm) {
+                const __grid_constant__ CUtensorMap tm_v, const TransParams prm) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv;
@@ -49,7 +55,12 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint32_t *tmem_slot = (uint32_t *)(bars + NBAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *err = prm.err;
-    const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_x = (nc + SLAB - 1) / SLAB;
+    const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
+    const bool frame = prm.frame != 0;
+    // B operand columns: chunkwise [Ub | W] packed (nc); frame-wise [V | K] slab-aligned
+    const int nslab_x = frame ? nslab_v + nslab_k : (nc + SLAB - 1) / SLAB;
+    const int ncols = frame ? SLAB * nslab_x : nc;
+    const int mcol0 = frame ? SLAB * nslab_v : dv;  // first column of the M part
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) sm100::mbar_init(&bars[i], (i >= SCALED && i < SCALED + NST) ? 128 : 1);
@@ -68,7 +79,7 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (warp == 0) {
         if (lane == 0) {
             sm100::tma_prefetch_desc(&tm_k);
-            sm100::tma_prefetch_desc(&tm_x);
+            sm100::tma_prefetch_desc(frame ? &tm_v : &tm_x);
             bool ok = true;
             for (int c = 0; c < nch && ok; ++c) {
                 const int st = c % NST;
@@ -78,14 +89,23 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 sm100::mbar_arrive_expect_tx(&bars[FULL + st], (uint32_t)((nslab_k + nslab_x) * CSLAB));
                 for (int sl = 0; sl < nslab_k; ++sl)
                     sm100::tma_load_4d(stage + sl * CSLAB, &tm_k, &bars[FULL + st], sl * SLAB, h, c * CH, bf);
-                for (int sl = 0; sl < nslab_x; ++sl)
-                    sm100::tma_load_3d(stage + (2 + sl) * CSLAB, &tm_x, &bars[FULL + st], sl * SLAB, c * CH, (int)fh);
+                if (frame) {
+                    for (int sl = 0; sl < nslab_v; ++sl)
+                        sm100::tma_load_4d(stage + (2 + sl) * CSLAB, &tm_v, &bars[FULL + st], sl * SLAB, h, c * CH, bf);
+                    for (int sl = 0; sl < nslab_k; ++sl)
+                        sm100::tma_load_4d(stage + (2 + nslab_v + sl) * CSLAB, &tm_k, &bars[FULL + st], sl * SLAB, h,
+                                           c * CH, bf);
+                } else {
+                    for (int sl = 0; sl < nslab_x; ++sl)
+                        sm100::tma_load_3d(stage + (2 + sl) * CSLAB, &tm_x, &bars[FULL + st], sl * SLAB, c * CH,
+                                           (int)fh);
+                }
             }
             if (ok) sm100::mbar_wait(&bars[DONE], 0, err);  // no copy left in flight
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id = sm100::idesc_bf16(BM, nc, 1, 1);
+            const uint32_t id = sm100::idesc_bf16(BM, ncols, 1, 1);
             bool ok = true;
             for (int c = 0; c < nch && ok; ++c) {
                 const int st = c % NST;
@@ -105,14 +125,15 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;  // the epilogue's 128 threads; at the end, key dimension m
         const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
-        const float GL = Gf[L - 1];
+        const float GL = frame ? 0.f : Gf[L - 1];
         bool ok = true;
         // thread r scales row r % 64 of the chunk's K, slab r / 64
         const int row_in = r & (CH - 1), sl = r >> 6;
         for (int c = 0; c < nch && ok; ++c) {
             const int st = c % NST;
             const int row = c * CH + row_in;
-            const float sc = row < L ? __expf(GL - Gf[row]) : 0.f;
+            float sc = 0.f;  // the K row's factor: e^{G_L - G_r}, or beta_r for the frame-wise map
+            if (row < L) sc = frame ? prm.beta[((long long)b * prm.T + f * L + row) * prm.H + h] : __expf(GL - Gf[row]);
             ok = sm100::mbar_wait(&bars[FULL + st], (c / NST) & 1, err);
             if (!ok) break;
             if (sl < nslab_k) {
@@ -136,10 +157,12 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (ok) {
             sm100::tc_fence_after();
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-            const float eGL = __expf(GL);
+            // M = c1 I - c2 (K^T-side product): chunkwise c1 = e^{G_L}, c2 = 1; frame-wise c1 = c2 = gamma
+            const float gam = frame ? prm.gamma[((long long)b * F + f) * prm.H + h] : 1.f;
+            const float eGL = frame ? gam : __expf(GL);
             const int m = r;
-            for (int c4 = 0; c4 < nc; c4 += 64) {  // four 16-column loads per wait (the last group may
-                float v4[4][16];                   // read past nc, inside the 256-column buffer, unused)
+            for (int c4 = 0; c4 < ncols; c4 += 64) {  // four 16-column loads per wait (the last group may
+                float v4[4][16];                      // read past ncols, inside the 256-column buffer, unused)
 #pragma unroll
                 for (int g = 0; g < 4; ++g) sm100::tmem_ld16(t_d + lane_off + c4 + 16 * g, v4[g]);
                 sm100::tmem_ld_wait();
@@ -147,16 +170,18 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     const int c0 = c4 + 16 * g;
-                    if (c0 >= nc) break;
+                    if (c0 >= ncols) break;
                     float *v = v4[g];
-                    float *dst;  // dv is a multiple of 16: a chunk lies wholly in N or in M
+                    float *dst;  // dv is a multiple of 16: a chunk lies wholly in N, in M or in padding
                     if (c0 < dv) {
                         dst = prm.N + (fh * dk + m) * (long long)dv + c0;
-                    } else {
-                        const int j0 = c0 - dv;
+                    } else if (c0 >= mcol0 && c0 - mcol0 < dk) {
+                        const int j0 = c0 - mcol0;
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] = (m == j0 + e ? eGL : 0.f) - v[e];
+                        for (int e = 0; e < 16; ++e) v[e] = (m == j0 + e ? eGL : 0.f) - gam * v[e];
                         dst = prm.M + (fh * dk + m) * (long long)dk + j0;
+                    } else {
+                        continue;
                     }
 #pragma unroll
                     for (int e = 0; e < 16; e += 4)
@@ -175,12 +200,12 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 }  // namespace
 
-cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const TransParams &prm,
-                                 long long n_fh, cudaStream_t s) {
+cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_v,
+                                 const TransParams &prm, long long n_fh, cudaStream_t s) {
     const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
     cudaError_t e = cudaFuncSetAttribute(k_transition_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_transition_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, prm);
+    k_transition_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_v, prm);
     return cudaGetLastError();
 }
 

@@ -8,6 +8,10 @@
 // rows), B = Sig in bf16 (MN-major), D = W Sig in a TMEM double buffer;
 // the epilogue subtracts it from Ub (read straight from global) and writes
 // U in bf16, the B operand layout of the output kernel.
+// The same kernel is the frame-wise operator's output (SANA-WM summary,
+// "Memory-Efficient Long-Context Modeling (Section 3.2)", paragraph
+// "Adaptation to video: frame-wise recurrence"): A = the frame's queries,
+// Sig the state after the frame's update, and o = Q Sig written to o.
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -24,8 +28,9 @@ struct Smem {
 
 enum Bar { SIGFULL, WFULL0, WFULL1, WEMPTY0, WEMPTY1, DFULL0, DFULL1, DEMPTY0, DEMPTY1, NBAR };
 
-__global__ void __launch_bounds__(kThreads, 1)
-k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_sig, const UParams prm) {
+__global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
+k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
+       const __grid_constant__ CUtensorMap tm_sig, const UParams prm) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
@@ -37,6 +42,9 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *err = prm.err;
     const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
+    const bool frame = prm.frame != 0;
+    const long long f = frame ? fh % prm.F : 0, chain = frame ? fh / prm.F : 0;
+    const int h = frame ? (int)(chain % prm.H) : 0, b = frame ? (int)(chain / prm.H) : 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) sm100::mbar_init(&bars[i], (i == DEMPTY0 || i == DEMPTY1) ? 128 : 1);
@@ -53,7 +61,7 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
 
     if (warp == 0) {
         if (lane == 0) {
-            sm100::tma_prefetch_desc(&tm_x);
+            sm100::tma_prefetch_desc(frame ? &tm_q : &tm_x);
             sm100::tma_prefetch_desc(&tm_sig);
             sm100::mbar_arrive_expect_tx(&bars[SIGFULL], (uint32_t)(nslab_v * dk * 128));
             for (int sl = 0; sl < nslab_v; ++sl)
@@ -64,9 +72,14 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
                 if (i >= 2) ok = sm100::mbar_wait(&bars[WEMPTY0 + st], ((i - 2) >> 1) & 1, err);
                 if (!ok) break;
                 sm100::mbar_arrive_expect_tx(&bars[WFULL0 + st], (uint32_t)(nslab_k * SLAB_BYTES));
-                for (int sl = 0; sl < nslab_k; ++sl)  // W = columns dv .. dv + dk of the [Ub | W] rows
-                    sm100::tma_load_3d(sW + (st * 2 + sl) * SLAB_BYTES, &tm_x, &bars[WFULL0 + st], dv + sl * SLAB,
-                                       i * BM, (int)fh);
+                for (int sl = 0; sl < nslab_k; ++sl) {
+                    if (frame)  // the frame's queries
+                        sm100::tma_load_4d(sW + (st * 2 + sl) * SLAB_BYTES, &tm_q, &bars[WFULL0 + st], sl * SLAB, h,
+                                           i * BM, (int)(b * prm.F + f));
+                    else  // W = columns dv .. dv + dk of the [Ub | W] rows
+                        sm100::tma_load_3d(sW + (st * 2 + sl) * SLAB_BYTES, &tm_x, &bars[WFULL0 + st],
+                                           dv + sl * SLAB, i * BM, (int)fh);
+                }
             }
             for (int i = (nblk >= 2 ? nblk - 2 : 0); ok && i < nblk; ++i)
                 ok = sm100::mbar_wait(&bars[WEMPTY0 + (i & 1)], (i >> 1) & 1, err);
@@ -98,14 +111,21 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
             const int st = i & 1;
             const int row = i * BM + r;
             const bool valid = row < L;
-            const __nv_bfloat16 *xrow = prm.X + (fh * (long long)L + (valid ? row : 0)) * nc;
-            __nv_bfloat16 *urow = prm.U + (fh * (long long)L + (valid ? row : 0)) * dv;
-            // this row's Ub (bf16) in registers before the wait, so its latency hides behind the MMA
+            // chunkwise: U = Ub - D over the row's [Ub | W]; frame-wise: o (+)= D
+            const __nv_bfloat16 *xrow =
+                frame ? prm.o + (((long long)b * prm.T + f * L + (valid ? row : 0)) * prm.H + h) * dv
+                      : prm.X + (fh * (long long)L + (valid ? row : 0)) * nc;
+            __nv_bfloat16 *urow = frame ? const_cast<__nv_bfloat16 *>(xrow)
+                                        : prm.U + (fh * (long long)L + (valid ? row : 0)) * dv;
+            const bool load_row = !frame || prm.accumulate;
+            const float sgn = frame ? 1.f : -1.f;
+            // this row's Ub (or the o being accumulated into) in registers before the wait, so
+            // its latency hides behind the MMA
             uint4 ub[16];
 #pragma unroll
             for (int c8 = 0; c8 < 16; ++c8)
-                ub[c8] = (valid && c8 < dv / 8) ? __ldg(reinterpret_cast<const uint4 *>(xrow) + c8)
-                                                : make_uint4(0, 0, 0, 0);
+                ub[c8] = (valid && load_row && c8 < dv / 8) ? __ldg(reinterpret_cast<const uint4 *>(xrow) + c8)
+                                                            : make_uint4(0, 0, 0, 0);
             ok = sm100::mbar_wait(&bars[DFULL0 + st], (i >> 1) & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
@@ -125,7 +145,7 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 u = __bfloat1622float2(p2[e]);
-                            p2[e] = __floats2bfloat162_rn(u.x - d[w * 8 + 2 * e], u.y - d[w * 8 + 2 * e + 1]);
+                            p2[e] = __floats2bfloat162_rn(u.x + sgn * d[w * 8 + 2 * e], u.y + sgn * d[w * 8 + 2 * e + 1]);
                         }
                         out[w] = xv;
                     }
@@ -147,12 +167,12 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
 
 }  // namespace
 
-cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_sig, const UParams &prm, long long n_fh,
-                        cudaStream_t s) {
+cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_q, const CUtensorMap &tm_sig,
+                        const UParams &prm, long long n_fh, cudaStream_t s) {
     const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
     cudaError_t e = cudaFuncSetAttribute(k_u_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_u_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_x, tm_sig, prm);
+    k_u_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_x, tm_q, tm_sig, prm);
     return cudaGetLastError();
 }
 

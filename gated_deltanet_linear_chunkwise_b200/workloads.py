@@ -129,6 +129,18 @@ def draw(B, H, T, d_k, d_v, *, frame_len, seed, regime="lit", per_frame_alpha=Fa
     return out
 
 
+def draw_frame_decay(B, F, H, *, seed, regime="slow"):
+    """Per-frame decays gamma [B, F, H] fp32 for the frame-wise operator, drawn
+    with the alpha recipe (exp(-softplus(z + c)), z ~ N(0,1)) once per (batch,
+    frame, head) from their own seeded stream."""
+    import torch
+
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal((B, F, H), dtype=np.float32)
+    gamma = np.exp(-np.logaddexp(0.0, z.astype(np.float64) + GATE_SHIFT[regime])).astype(np.float32)
+    return torch.from_numpy(gamma)
+
+
 def make_inputs(w: Workload | str, regime="lit", *, seed=None, call=None, frames=None):
     """Inputs for a named workload.
 

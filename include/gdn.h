@@ -188,6 +188,21 @@ int gdn_fwd_noalloc(const void *q, const void *k, const void *v,
  *                   CUDA events bracket each kernel stage on `stream` and the
  *                   call synchronises the stream and writes each stage's
  *                   device time in ms (tracing; off in production calls).
+ *   mode            GDN_MODE_TOKEN (0): the token-wise gated delta rule
+ *                   above.  GDN_MODE_FRAME (1): the frame-wise operator
+ *                   (SANA-WM summary, "Memory-Efficient Long-Context Modeling
+ *                   (Section 3.2)", paragraph "Adaptation to video: frame-wise
+ *                   recurrence"): one state update per frame t of frame_len
+ *                   tokens,
+ *                     S_t = S_{t-1} M_t + U_t,  M_t = gamma_t (I - K_t B_t K_t^T),
+ *                     U_t = V_t B_t K_t^T,      o = S_t q for every token of t,
+ *                   with K_t, V_t the frame's keys and values as columns and
+ *                   B_t = diag(beta) over its tokens; alpha is not read (may
+ *                   be NULL).  reverse visits the frames backwards; reset_every
+ *                   and accumulate_o as above.
+ *   gamma           GDN_MODE_FRAME only: device fp32 [B, T / frame_len, H],
+ *                   the per-frame decay gamma_t of each head (required there,
+ *                   ignored otherwise).
  */
 typedef struct gdn_args {
     int struct_size;
@@ -208,7 +223,11 @@ typedef struct gdn_args {
     int check_finite;
     gdn_stream_t stream;
     float *stage_ms;
+    int mode;
+    const float *gamma;
 } gdn_args;
+
+enum { GDN_MODE_TOKEN = 0, GDN_MODE_FRAME = 1 };
 
 /* Kernel stages reported through gdn_args.stage_ms, in launch order:
  * 0 per-frame gate prefix sums, 1 inverses of the 128 x 128 diagonal blocks

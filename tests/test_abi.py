@@ -47,7 +47,29 @@ def test_struct_size_matches_header():
     a.struct_size = ctypes.sizeof(binding.GdnArgs) + 8
     rc = g.load_library().gdn_fwd_ex(ctypes.byref(a))
     assert rc == 1 and "struct_size" in g.last_error()
-    assert ctypes.sizeof(binding.GdnArgs) == 160  # LP64 layout of gdn_args
+    assert ctypes.sizeof(binding.GdnArgs) == 176  # LP64 layout of gdn_args
+
+
+def _ex_args(**kw):
+    a = binding.GdnArgs()
+    a.struct_size = ctypes.sizeof(binding.GdnArgs)
+    a.q, a.k, a.v, a.alpha, a.beta, a.o = FAKE, FAKE + 1024, FAKE + 2048, FAKE + 4096, FAKE + 8192, FAKE + 16384
+    a.B, a.H, a.T, a.frame_len, a.d_k, a.d_v = 1, 2, 128, 64, 64, 64
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+@pytest.mark.parametrize("kw,status,text", [
+    (dict(mode=2), 1, "mode"),                        # neither operator
+    (dict(mode=1), 1, "gamma"),                       # frame-wise operator without its decay
+    (dict(alpha=None), 1, "alpha"),                   # token-wise operator without alpha
+    (dict(mode=1, alpha=None, gamma=FAKE + 16384 + 8), 1, "overlaps"),  # o over gamma
+])
+def test_mode_validation(kw, status, text):
+    # rejected before any device work (no GPU needed)
+    rc = g.load_library().gdn_fwd_ex(ctypes.byref(_ex_args(**kw)))
+    assert rc == status and text in g.last_error()
 
 
 def test_stage_count_matches_header():
