@@ -75,6 +75,15 @@ def bytes_alg(B, T, H, dk, dv, elem=2):
     return B * T * H * (2 * dk + 2 * dv) * elem + 8 * B * T * H + 2 * B * H * dk * dv * 4
 
 
+# DRAM bytes (read + write) per frame-head of the tensor-core kernels, from one ncu capture
+# of the short-clip case (420 frame-heads, L = 880, d_k = d_v = 112; profiles/ holds the
+# summary and the command).  Traffic grows with the frame-heads processed, so a launch's
+# figure is this times its frame-head count; other shapes report null.
+DRAM_BYTES_PER_FH = {"intra": (334.5088e6 + 136.193024e6) / 420,
+                     "output": (467.891712e6 + 72.675328e6) / 420}
+TRAFFIC_SHAPE = (880, 112, 112)
+
+
 def framewise_line(B, T, H, dk, dv, L, ms, stage, pk, stages):
     """The frame-wise operator's pass: HBM bound (algorithmic bytes: q, k, v and beta read once,
     o written once; FLOPs per frame-head 2L d_k (d_k + d_v) + 2 d_k^2 d_v + 2 L d_k d_v)."""
@@ -375,7 +384,9 @@ def main():
                        "l2": "no flush: inputs 1.4 GB per step exceed the 126 MB L2"},
             "roofline": {"bound": "tensor" if tensor_bound else "hbm", "kernel": STAGES[dominant],
                          "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                         "traffic": None,
+                         "traffic": (DRAM_BYTES_PER_FH[STAGES[dominant]] * nfh
+                                     if (L, dk, dv) == TRAFFIC_SHAPE and STAGES[dominant] in DRAM_BYTES_PER_FH
+                                     else None),
                          "peak_source": pk["source"] + (" bf16 burst" if tensor_bound else " copy bandwidth"),
                          "per_launch": {"flops": f_dom, "bytes": b_dom, "ms": dom_ms},
                          "stage_ms": dict(zip(STAGES, stage_sum))},
