@@ -438,6 +438,10 @@ size_t gdn_workspace_bytes(int B, int H, long long T, int frame_len, int d_k, in
     memset(&p, 0, sizeof(p));
     p.dtype = dtype; p.B = B; p.H = H; p.T = T; p.L = frame_len; p.dk = d_k; p.dv = d_v;
     p.F = T / frame_len;
+    // the largest case: a reversed, accumulating call (token-reversed input copies and a
+    // staged o), so a workspace of this size serves every flag combination
+    p.reverse = 1;
+    p.accumulate = 1;
     return workspace_for(p);
 }
 

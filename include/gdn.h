@@ -239,7 +239,9 @@ enum { GDN_NUM_STAGES = 7 };
 
 int gdn_fwd_ex(const gdn_args *a);
 
-/* Device scratch a call with these sizes needs (0 if the sizes are invalid). */
+/* Device scratch a call with these sizes needs with any flags of gdn_fwd_ex
+ * (the size of the largest case, a reversed accumulating call; 0 if the
+ * sizes are invalid). */
 size_t gdn_workspace_bytes(int B, int H, long long T, int frame_len, int d_k, int d_v, int dtype);
 
 /* Static text for a status code; never NULL. */

@@ -156,6 +156,21 @@ def test_reverse_reset_not_dividing_length(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_reverse_accumulate_in_caller_workspace(dtype):
+    # a workspace of gdn_workspace_bytes serves the largest case, a reversed accumulating call
+    B, H, L, F, dk, dv = 1, 2, 64, 3, 32, 48
+    inp = W.draw(B, H, F * L, dk, dv, frame_len=L, seed=25, regime="slow", dtype=dtype)
+    d = dev(inp)
+    ws = torch.empty(g.workspace_bytes(B, H, F * L, L, dk, dv, dtype), dtype=torch.uint8, device="cuda")
+    o0 = torch.full((B, F * L, H, dv), 0.5, dtype=d["q"].dtype, device="cuda")
+    o_r, _ = g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, None, o=o0, reverse=True,
+                       accumulate=True, workspace=ws)
+    torch.cuda.synchronize()
+    o_ref, _ = ora(inp, None, reverse=True)
+    assert rel(o_r.double().cpu() - 0.5, o_ref) <= TOL[dtype] + (4e-3 if dtype == "bf16" else 0.0)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_step_chain_equals_single_call(dtype):
     L = 80
     inp = W.draw(2, 3, 7 * L, 64, 64, frame_len=L, seed=31, regime="slow", dtype=dtype, state_std=0.1)
