@@ -20,6 +20,10 @@ section 3.2 "Memory-Efficient Long-Context Modeling", paragraph
   ``U_t = V_t B_t K_t^T``, ``O_t = S_t Q_t`` with M_t, U_t formed explicitly.
 * ``token_recurrence_numpy`` -- a pure-Python/numpy twin of the token loop,
   for tiny cases only (cross-checks the C build and its layouts).
+* ``key_feature_map`` / ``query_feature_map`` -- the q/k prologue of the same
+  section's paragraph "Algebraic Stabilization for Spatial Token Explosion":
+  ReLU(RMSNorm(x)) over the head dimension, keys further divided by
+  sqrt(D * S).
 
 Inputs are taken in whatever dtype they are stored in and upcast exactly to
 fp64 (bf16 and fp32 both embed in fp64), so a comparison measures only the
@@ -145,6 +149,32 @@ def bidirectional(q, k, v, alpha, beta, *, chunk_len=0, S_in=None, nthreads=0):
     o_r, _ = token_recurrence(q, k, v, alpha, beta, None, reverse=True,
                               reset_every=chunk_len, nthreads=nthreads)
     return o_f + o_r, S_f
+
+
+def key_feature_map(k, *, frame_len, weight=None, eps=1e-6):
+    """Keys of the frame-wise operator (SANA-WM summary, "Memory-Efficient
+    Long-Context Modeling (Section 3.2)", paragraph "Algebraic Stabilization
+    for Spatial Token Explosion"): k_bar = ReLU(RMSNorm(k)) over the head
+    dimension D, then k_hat = k_bar / sqrt(D * S) with S = frame_len tokens.
+    RMSNorm(x) = x / sqrt(mean(x^2) + eps) * weight (weight = ones if None).
+    In fp64; returns a numpy array of k's shape."""
+    y = _rms_relu(k, weight, eps)
+    return y / np.sqrt(y.shape[-1] * float(frame_len))
+
+
+def query_feature_map(q, *, weight=None, eps=1e-6):
+    """Queries: q_hat = ReLU(RMSNorm(q)) (the keys' feature map without the
+    1/sqrt(D*S) scale, which the same paragraph applies to keys only)."""
+    return _rms_relu(q, weight, eps)
+
+
+def _rms_relu(x, weight, eps):
+    x = _f64(x)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    y = x / np.sqrt(ms + eps)
+    if weight is not None:
+        y = y * _f64(weight)
+    return np.maximum(y, 0.0)
 
 
 def token_recurrence_numpy(q, k, v, alpha, beta, S_in=None):

@@ -380,3 +380,47 @@ def test_oracle_rejects_bad_shapes(bad):
     else:
         with pytest.raises(AssertionError):
             oracle.token_recurrence(q, q, q, np.ones((1, 5, 1)), np.ones((1, 6, 1)))
+
+
+# ---------------------------------------------------------------- q/k prologue (feature maps)
+
+def test_key_feature_map_constant_vector():
+    """A constant positive vector has RMS equal to its value: RMSNorm maps it to ones
+    (up to eps), ReLU keeps them, and the key scale makes each entry 1/sqrt(D S)."""
+    D, S = 8, 5
+    k = np.full((1, 1, 1, D), 3.0)
+    kh = oracle.key_feature_map(k, frame_len=S, eps=0.0)
+    np.testing.assert_allclose(kh, np.full_like(k, 1.0 / np.sqrt(D * S)), rtol=1e-15)
+    qh = oracle.query_feature_map(-k, eps=0.0)  # all negative: ReLU zeroes it
+    assert np.count_nonzero(qh) == 0
+
+
+def test_feature_maps_scale_invariant_and_weighted():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((2, 7, 3, 16))
+    np.testing.assert_allclose(oracle.query_feature_map(5.0 * x, eps=0.0), oracle.query_feature_map(x, eps=0.0),
+                               rtol=1e-13)
+    w = rng.uniform(0.5, 2.0, 16)
+    y = oracle.query_feature_map(x, eps=0.0)
+    yw = oracle.query_feature_map(x, weight=w, eps=0.0)
+    np.testing.assert_allclose(yw, y * w, rtol=1e-13)  # the weight multiplies before ReLU; w > 0 commutes
+    # the RMS of the normalised vector (before ReLU) is 1: ReLU keeps sum of squares <= D
+    assert (y * y).sum(-1).max() <= 16 + 1e-9
+    # explicit per-entry formula on one row
+    row = x[0, 0, 0]
+    ref = np.maximum(row / np.sqrt(np.mean(row ** 2) + 1e-6), 0.0)
+    np.testing.assert_allclose(oracle.query_feature_map(x)[0, 0, 0], ref, rtol=1e-15)
+
+
+def test_key_feature_map_bounds_frame_energy():
+    """The pages' bound: with beta in [0, 1], tr(K_hat^T B K_hat) = sum_s beta_s |k_hat_s|^2 <= 1
+    for any frame of S keys, so every eigenvalue of I - K_hat^T B K_hat lies in [0, 1]."""
+    rng = np.random.default_rng(42)
+    for D, S in ((16, 40), (112, 880), (32, 1)):
+        k = rng.standard_normal((1, S, 1, D)) * rng.uniform(0.1, 10.0)
+        kh = oracle.key_feature_map(k, frame_len=S, eps=0.0)[0, :, 0]
+        beta = rng.uniform(0, 1, S)
+        A = (kh * beta[:, None]).T @ kh
+        assert np.trace(A) <= 1.0 + 1e-12
+        ev = np.linalg.eigvalsh(np.eye(D) - A)
+        assert ev.min() >= -1e-12 and ev.max() <= 1.0 + 1e-12
