@@ -319,6 +319,20 @@ def main():
         for i in range(NUM_STAGES):
             fw_stage[i] += arr[i] / 3
 
+    # the same operator on the raw q, k through the library's q/k prologue
+    def framewise_prologue():
+        g.gdn_fwd(d["q"], d["k"], d["v"], None, d["beta"], L, None, S_out=S_out, o=o, stream=stream,
+                  mode="frame", gamma=gamma, norm_keys=True, norm_queries=True)
+
+    for _ in range(3):
+        framewise_prologue()
+    f0.record(stream)
+    for _ in range(10):
+        framewise_prologue()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    fwp_ms = gdist.max_over_ranks(f0.elapsed_time(f1) / 10, device=dev)
+
     # per-stage device times (events around each kernel on the same stream)
     stage_sum = [0.0] * NUM_STAGES
     reps = 5
@@ -401,7 +415,11 @@ def main():
             "gpu_launches": NUM_STAGES * args.steps,
             "bidirectional": {"ms_per_pass": bidir_ms, "tokens_per_s": tokens / (bidir_ms * 1e-3),
                               "what": "forward + reversed scan summed into o (not the timed metric)"},
-            "framewise": framewise_line(B * world, T, H, dk, dv, L, fw_ms, fw_stage, pk, STAGES),
+            "framewise": dict(framewise_line(B * world, T, H, dk, dv, L, fw_ms, fw_stage, pk, STAGES),
+                              with_qk_prologue={"ms_per_pass": fwp_ms,
+                                                "tokens_per_s": tokens / (fwp_ms * 1e-3),
+                                                "what": "raw q, k through norm_keys + norm_queries "
+                                                        "(prologue kernel, not fused)"}),
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline and world == 1 and args.workload == WORKLOAD:

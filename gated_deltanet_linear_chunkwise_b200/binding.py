@@ -47,10 +47,13 @@ class GdnArgs(ctypes.Structure):
         ("reset_every", ctypes.c_longlong), ("check_finite", ctypes.c_int),
         ("stream", ctypes.c_void_p), ("stage_ms", ctypes.c_void_p),
         ("mode", ctypes.c_int), ("gamma", ctypes.c_void_p),
+        ("qk_norm", ctypes.c_int), ("k_norm_weight", ctypes.c_void_p), ("q_norm_weight", ctypes.c_void_p),
     ]
 
 GDN_MODE_TOKEN = 0
 GDN_MODE_FRAME = 1
+GDN_QK_NORM_KEYS = 1
+GDN_QK_NORM_QUERIES = 2
 
 NUM_STAGES = 7
 STAGES = ("gates", "diag_inverse", "intra", "transition", "scan", "u", "output")
@@ -117,7 +120,8 @@ def _stream_handle(stream, device):
 
 def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
             return_state=False, reverse=False, accumulate=False, reset_every=0,
-            check_finite=False, workspace=None, stream=None, stage_ms=None, mode="token", gamma=None):
+            check_finite=False, workspace=None, stream=None, stage_ms=None, mode="token", gamma=None,
+            norm_keys=False, norm_queries=False, k_norm_weight=None, q_norm_weight=None):
     """Chunkwise gated delta rule forward on CUDA tensors.
 
     q,k [B,T,H,d_k], v [B,T,H,d_v] (bf16 or fp32, all the same), alpha/beta
@@ -129,6 +133,9 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     ``mode="frame"`` runs the frame-wise operator instead (one state update
     per frame of ``frame_len`` tokens); it reads ``gamma`` [B, T/frame_len, H]
     fp32, the per-frame decay, and not ``alpha`` (which may be None).
+    ``norm_keys`` / ``norm_queries`` apply the q/k prologue first: keys
+    ReLU(RMSNorm(k)) / sqrt(d_k * frame_len), queries ReLU(RMSNorm(q)), with
+    optional fp32 [d_k] RMSNorm weights.
     Returns (o, S_out or None).
     """
     import torch
@@ -151,6 +158,10 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
         raise GdnError(1, "%s must be fp32" % " and ".join(n for n, _ in gates))
     if frame and tuple(gamma.shape) != (B, T // max(int(frame_len), 1), H):
         raise GdnError(2, "gamma must have shape [B, T / frame_len, H]")
+    for name, wt, on in (("k_norm_weight", k_norm_weight, norm_keys), ("q_norm_weight", q_norm_weight, norm_queries)):
+        if wt is not None and on and (not wt.is_cuda or not wt.is_contiguous() or wt.dtype != torch.float32
+                                      or wt.numel() != d_k):
+            raise GdnError(1, "%s must be a contiguous fp32 CUDA tensor of d_k entries" % name)
     for name, t in (("S_in", S_in), ("S_out", S_out), ("o", o)):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise GdnError(1, "%s must be a contiguous CUDA tensor" % name)
@@ -166,6 +177,9 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     a.S_in, a.S_out, a.o = _ptr(S_in), _ptr(S_out), _ptr(o)
     a.mode = GDN_MODE_FRAME if frame else GDN_MODE_TOKEN
     a.gamma = _ptr(gamma) if frame else None
+    a.qk_norm = (GDN_QK_NORM_KEYS if norm_keys else 0) | (GDN_QK_NORM_QUERIES if norm_queries else 0)
+    a.k_norm_weight = _ptr(k_norm_weight) if norm_keys else None
+    a.q_norm_weight = _ptr(q_norm_weight) if norm_queries else None
     a.B, a.H, a.T = B, H, T
     a.frame_len, a.d_k, a.d_v = int(frame_len), d_k, d_v
     if workspace is not None:

@@ -88,6 +88,10 @@ int validate_sizes(const gdn_args &a) {
         set_err("mode must be GDN_MODE_TOKEN or GDN_MODE_FRAME (got %d)", a.mode);
         return GDN_ERR_INVALID_ARG;
     }
+    if (a.qk_norm < 0 || a.qk_norm > (GDN_QK_NORM_KEYS | GDN_QK_NORM_QUERIES)) {
+        set_err("qk_norm must be a mask of GDN_QK_NORM_KEYS and GDN_QK_NORM_QUERIES (got %d)", a.qk_norm);
+        return GDN_ERR_INVALID_ARG;
+    }
     if (a.reset_every < 0 || (a.reset_every > 0 && a.reset_every % a.frame_len != 0)) {
         set_err("reset_every (%lld) must be 0 or a positive multiple of frame_len (%d)", a.reset_every, a.frame_len);
         return GDN_ERR_INVALID_ARG;
@@ -176,6 +180,9 @@ int validate(const gdn_args &a, gdn::Problem &p) {
     p.dk = a.d_k; p.dv = a.d_v; p.F = F;
     p.reverse = a.reverse; p.accumulate = a.accumulate_o; p.reset_every = a.reset_every;
     p.mode = a.mode; p.gamma = frame ? a.gamma : nullptr;
+    p.qk_norm = a.qk_norm;
+    p.k_norm_weight = (a.qk_norm & GDN_QK_NORM_KEYS) ? a.k_norm_weight : nullptr;
+    p.q_norm_weight = (a.qk_norm & GDN_QK_NORM_QUERIES) ? a.q_norm_weight : nullptr;
     if (frame) p.alpha = nullptr;
     return GDN_OK;
 }
@@ -183,9 +190,12 @@ int validate(const gdn_args &a, gdn::Problem &p) {
 // Which implementation serves this problem, and how much scratch it needs.
 bool use_tc(const gdn::Problem &p) { return gdn::tc_supports(p); }
 
-size_t workspace_for(const gdn::Problem &p) {
+// The operator's scratch (the q/k prologue's copies follow it).
+size_t operator_workspace(const gdn::Problem &p) {
     return use_tc(p) ? gdn::tc_workspace_bytes(p) : gdn::simt_workspace_bytes(p);
 }
+
+size_t workspace_for(const gdn::Problem &p) { return operator_workspace(p) + gdn::qk_prologue_bytes(p); }
 
 __global__ void nonfinite_scan_f32(const float *x, long long n, int *flag) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
@@ -254,7 +264,10 @@ int run(const gdn_args &a) noexcept {
             evp = ev;
         }
         const bool tc = use_tc(p);
-        cudaError_t e = tc ? gdn::launch_tc(p, ws, s, evp) : gdn::launch_simt(p, ws, s, evp);
+        cudaError_t e = cudaSuccess;
+        if (p.qk_norm)  // normalised q / k copies after the operator's scratch; p now points at them
+            e = gdn::launch_qk_prologue(p, (char *)ws + operator_workspace(p), s);
+        if (e == cudaSuccess) e = tc ? gdn::launch_tc(p, ws, s, evp) : gdn::launch_simt(p, ws, s, evp);
         // synchronous modes also report a device-side wait that gave up
         int timed_out = 0;
         if (e == cudaSuccess && tc && (a.stage_ms || a.check_finite)) {
@@ -439,9 +452,11 @@ size_t gdn_workspace_bytes(int B, int H, long long T, int frame_len, int d_k, in
     p.dtype = dtype; p.B = B; p.H = H; p.T = T; p.L = frame_len; p.dk = d_k; p.dv = d_v;
     p.F = T / frame_len;
     // the largest case: a reversed, accumulating call (token-reversed input copies and a
-    // staged o), so a workspace of this size serves every flag combination
+    // staged o) with both prologue copies, so a workspace of this size serves every flag
+    // combination
     p.reverse = 1;
     p.accumulate = 1;
+    p.qk_norm = GDN_QK_NORM_KEYS | GDN_QK_NORM_QUERIES;
     return workspace_for(p);
 }
 

@@ -49,6 +49,8 @@ struct Problem {
     long long reset_every;  // tokens; 0 = never
     int mode;               // GDN_MODE_TOKEN / GDN_MODE_FRAME
     const float *gamma;     // GDN_MODE_FRAME: [B, F, H] per-frame decay
+    int qk_norm;            // GDN_QK_NORM_* bits still to apply (the prologue clears them)
+    const float *k_norm_weight, *q_norm_weight;  // [d_k] or NULL
 };
 
 // Memory index of the frame the scan visits at logical step f.  The
@@ -114,5 +116,10 @@ cudaError_t simt_u_bf16x(const Problem &p, const __nv_bfloat16 *X, const float *
 cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
 // The frame-wise operator on the CUDA cores (launch_simt dispatches to it).
 cudaError_t launch_simt_frame(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);
+
+// The q/k prologue (qk_prologue.cu): scratch bytes it needs, and the launch that writes the
+// normalised copies into `scratch` and points p's q / k at them (clearing p.qk_norm).
+size_t qk_prologue_bytes(const Problem &p);
+cudaError_t launch_qk_prologue(Problem &p, void *scratch, cudaStream_t s);
 
 }  // namespace gdn

@@ -203,6 +203,16 @@ int gdn_fwd_noalloc(const void *q, const void *k, const void *v,
  *   gamma           GDN_MODE_FRAME only: device fp32 [B, T / frame_len, H],
  *                   the per-frame decay gamma_t of each head (required there,
  *                   ignored otherwise).
+ *   qk_norm         bit mask of the q/k prologue (SANA-WM summary, section
+ *                   3.2, paragraph "Algebraic Stabilization for Spatial Token
+ *                   Explosion"), applied to the inputs before the operator:
+ *                   GDN_QK_NORM_KEYS    k <- ReLU(RMSNorm(k)) / sqrt(d_k * frame_len),
+ *                   GDN_QK_NORM_QUERIES q <- ReLU(RMSNorm(q)),
+ *                   RMSNorm(x) = x / sqrt(mean over d_k of x^2 + 1e-6) * weight.
+ *                   The normalised copies live in the workspace; q and k are
+ *                   not modified.  0: the inputs are used as given.
+ *   k_norm_weight,  optional device fp32 [d_k] RMSNorm weights of the keys and
+ *   q_norm_weight   queries (NULL: ones); read only when their bit is set.
  */
 typedef struct gdn_args {
     int struct_size;
@@ -225,9 +235,13 @@ typedef struct gdn_args {
     float *stage_ms;
     int mode;
     const float *gamma;
+    int qk_norm;
+    const float *k_norm_weight;
+    const float *q_norm_weight;
 } gdn_args;
 
 enum { GDN_MODE_TOKEN = 0, GDN_MODE_FRAME = 1 };
+enum { GDN_QK_NORM_KEYS = 1, GDN_QK_NORM_QUERIES = 2 };
 
 /* Kernel stages reported through gdn_args.stage_ms, in launch order:
  * 0 per-frame gate prefix sums, 1 inverses of the 128 x 128 diagonal blocks
