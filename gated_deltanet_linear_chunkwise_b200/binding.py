@@ -148,6 +148,7 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     for name, t in (("q", q), ("k", k), ("v", v)) + gates:
         if t is None:
             raise GdnError(1, "%s is required" % name)
+    for name, t in (("q", q), ("k", k), ("v", v)) + gates:
         if not t.is_cuda:
             raise GdnError(1, "%s is not a CUDA tensor" % name)
         if not t.is_contiguous():

@@ -154,3 +154,27 @@ def test_host_binding_rejects_device_tensors_by_type():
     x = torch.zeros(1, 64, 1, 16, dtype=torch.float16)
     with pytest.raises(g.GdnError):
         g.gdn_fwd_host(x, x, x, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1), 64)
+
+
+def test_python_binding_frame_mode_checks():
+    import torch
+    x = torch.zeros(1, 64, 1, 16)
+    a = torch.zeros(1, 64, 1)
+    with pytest.raises(g.GdnError, match="mode"):
+        g.gdn_fwd(x, x, x, a, a, 64, mode="frames")
+    with pytest.raises(g.GdnError, match="gamma is required"):
+        g.gdn_fwd(x, x, x, None, a, 64, mode="frame")
+    with pytest.raises(g.GdnError, match="alpha is required"):
+        g.gdn_fwd(x, x, x, None, a, 64)
+
+
+def test_workspace_bytes_covers_every_flag():
+    # the public size is the largest case: it grows with neither flag, and a forward-only
+    # problem of the same sizes needs no more
+    from gated_deltanet_linear_chunkwise_b200 import binding as b
+    lib = g.load_library()
+    full = lib.gdn_workspace_bytes(1, 20, 880 * 4, 880, 112, 112, b.GDN_DTYPE_BF16)
+    smaller = lib.gdn_workspace_bytes(1, 20, 880 * 3, 880, 112, 112, b.GDN_DTYPE_BF16)
+    assert full > smaller > 0
+    # bf16 q, k, v, o and the two prologue copies all fit: at least 5 token-major bf16 tensors
+    assert full >= 5 * 2 * 880 * 4 * 20 * 112
