@@ -55,14 +55,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 __device__ __forceinline__ void load_a(uint32_t (&a)[4], const __nv_bfloat16 *t, int ld, int r0, int c0, int lane) {
     ldsm_x4(a, t + (r0 + (lane & 15)) * ld + c0 + (lane >> 4) * 8);
 }
-// B fragments (two n8 tiles) of B[k][n] = M[n][k] for a row-major M: rows n0..n0+15, cols k0..k0+15.
-__device__ __forceinline__ void load_b_rows(uint32_t (&b)[4], const __nv_bfloat16 *t, int ld, int n0, int k0,
-                                            int lane) {
-    // matrices: (n 0-7, k 0-7), (n 0-7, k 8-15), (n 8-15, k 0-7), (n 8-15, k 8-15)
-    const int n = n0 + (lane & 7) + ((lane >> 4) << 3);
-    const int k = k0 + ((lane >> 3) & 1) * 8;
-    ldsm_x4(b, t + n * ld + k);
-}
 // B fragments (two n8 tiles) of B[k][n] = M[k][n] for a row-major M: rows k0..k0+15, cols n0..n0+15.
 __device__ __forceinline__ void load_b_trans(uint32_t (&b)[4], const __nv_bfloat16 *t, int ld, int k0, int n0,
                                              int lane) {
