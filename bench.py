@@ -177,9 +177,17 @@ def cpu_baseline(regime, frames, inp=None, nthreads=0):
     oracle.token_recurrence(x["q"], x["k"], x["v"], x["alpha"], x["beta"], None, nthreads=threads)
     dt = time.perf_counter() - t0
     tokens = w.B * frames * w.frame_len
+    # the same oracle on one thread over the first frame (all 20 heads)
+    y = {k: v[:, :w.frame_len] for k, v in x.items()}
+    t1 = time.perf_counter()
+    oracle.token_recurrence(y["q"], y["k"], y["v"], y["alpha"], y["beta"], None, nthreads=1)
+    dt1 = time.perf_counter() - t1
     return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": "B=1, 20 heads, first %d of 121 frames (%d tokens) of the minute workload, %.1f s"
-                      % (frames, tokens, dt)}
+                      % (frames, tokens, dt),
+            "single_thread": {"value": w.B * w.frame_len / dt1, "unit": "tokens/s",
+                              "sample": "first frame, 20 heads, %.2f s" % dt1},
+            "host_cores": os.cpu_count()}
 
 
 def run_reference(args, rank, world):
@@ -407,6 +415,7 @@ def main():
             "path_roofline": {"flops": f_all, "bytes": bytes_alg(B, T, H, dk, dv),
                               "achieved_tflops": f_all / (ms_step * 1e-3) / 1e12,
                               "frac_tensor": f_all / (ms_step * 1e-3) / 1e12 / pk["bf16_tflops"],
+                              "frac_tensor_datasheet": f_all / (ms_step * 1e-3) / 1e12 / 2250.0,
                               "frac_tensor_sustained": (f_all / (ms_step * 1e-3) / 1e12 / pk["bf16_tflops_sustained"]
                                                         if pk["bf16_tflops_sustained"] else None)},
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
