@@ -478,6 +478,6 @@ const char *gdn_status_string(int s) {
 
 const char *gdn_last_error(void) { return g_err; }
 
-int gdn_version(void) { return 100; }
+int gdn_version(void) { return GDN_VERSION; }
 
 }  // extern "C"

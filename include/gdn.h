@@ -264,7 +264,10 @@ const char *gdn_status_string(int status);
 /* Thread-local detail of the last failure on this thread ("" if none). */
 const char *gdn_last_error(void);
 
-/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH.  The gdn_args layout
+ * belongs to the version: 0.2.0 added mode, gamma, qk_norm and the RMSNorm
+ * weights (struct_size guards a caller built against another layout). */
+#define GDN_VERSION 200
 int gdn_version(void);
 
 #ifdef __cplusplus

@@ -178,3 +178,8 @@ def test_workspace_bytes_covers_every_flag():
     assert full > smaller > 0
     # bf16 q, k, v, o and the two prologue copies all fit: at least 5 token-major bf16 tensors
     assert full >= 5 * 2 * 880 * 4 * 20 * 112
+
+
+def test_version_matches_header():
+    m = re.search(r"#define\s+GDN_VERSION\s+(\d+)", open(HEADER).read())
+    assert m and g.load_library().gdn_version() == int(m.group(1))
