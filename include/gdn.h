@@ -246,9 +246,11 @@ enum { GDN_QK_NORM_KEYS = 1, GDN_QK_NORM_QUERIES = 2 };
 /* Kernel stages reported through gdn_args.stage_ms, in launch order:
  * 0 per-frame gate prefix sums, 1 inverses of the 128 x 128 diagonal blocks
  * of the intra-frame system, 2 intra-frame solve, 3 frame transition,
- * 4 scan over frames, 5 pseudo-values U, 6 output.  A path that folds a
- * stage into the next one (the fp32 and reversed paths fold 0, 1 into 2 and
- * 5 into 6) reports 0 for it. */
+ * 4 scan over frames, 5 pseudo-values U, 6 output.  A path without a stage
+ * reports 0 for it: the fp32 path folds 0, 1 into 2 and 5 into 6; the
+ * frame-wise operator has only 3 (its per-frame maps), 4 and 6.  Work
+ * outside the seven stages is not counted: the q/k prologue, and a reversed
+ * or accumulating bf16 call's input reversal and final write of o. */
 enum { GDN_NUM_STAGES = 7 };
 
 int gdn_fwd_ex(const gdn_args *a);
