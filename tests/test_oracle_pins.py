@@ -319,6 +319,35 @@ def test_framewise_single_token_frames_equal_tokenwise():
     np.testing.assert_allclose(S1, S2, atol=1e-12)
 
 
+def test_framewise_orthogonal_frames_equal_tokenwise_sequence():
+    """With mutually orthogonal keys inside each frame, the rank-S frame update equals
+    the frame's tokens applied one by one with alpha = gamma_t at the frame's first token
+    and 1 after it: the cross terms of prod_s (I - beta_s k_s k_s^T) vanish, and
+    k_s^T (I - beta_s' k_s' k_s'^T) = k_s^T for s' != s.  Every token of frame t reads the
+    state at the frame's end."""
+    rng = np.random.default_rng(23)
+    B, H, D, dv, S, F = 1, 2, 6, 5, 4, 3
+    k = np.zeros((B, F * S, H, D))
+    for f in range(F):
+        for h in range(H):
+            Qm, _ = np.linalg.qr(rng.standard_normal((D, S)))
+            k[0, f * S:(f + 1) * S, h] = Qm.T
+    q = rng.standard_normal((B, F * S, H, D))
+    v = rng.standard_normal((B, F * S, H, dv))
+    beta = rng.uniform(0, 1, (B, F * S, H))
+    gamma = rng.uniform(0.3, 1.0, (B, F, H))
+    S0 = rng.standard_normal((B, H, dv, D))
+    o_fw, S_fw = oracle.framewise(q, k, v, gamma, beta, S0, frame_len=S)
+    alpha = np.ones((B, F * S, H))
+    alpha[:, ::S] = gamma
+    for f in range(F):
+        end = (f + 1) * S
+        _, S_tok = oracle.token_recurrence(q[:, :end], k[:, :end], v[:, :end], alpha[:, :end], beta[:, :end], S0)
+        for s_ in range(f * S, end):
+            np.testing.assert_allclose(o_fw[0, s_], np.einsum("hvd,hd->hv", S_tok[0], q[0, s_]), atol=1e-12)
+    np.testing.assert_allclose(S_fw, S_tok, atol=1e-12)
+
+
 def test_framewise_orthonormal_frame_stores_values():
     """One frame of mutually orthonormal keys, beta = gamma = 1, S_0 = 0:
     every token of the frame reads S_t, and S_t k_j = v_j."""
