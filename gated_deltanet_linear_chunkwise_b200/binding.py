@@ -48,6 +48,7 @@ class GdnArgs(ctypes.Structure):
         ("stream", ctypes.c_void_p), ("stage_ms", ctypes.c_void_p),
         ("mode", ctypes.c_int), ("gamma", ctypes.c_void_p),
         ("qk_norm", ctypes.c_int), ("k_norm_weight", ctypes.c_void_p), ("q_norm_weight", ctypes.c_void_p),
+        ("status_dev", ctypes.c_void_p),
     ]
 
 GDN_MODE_TOKEN = 0
@@ -121,7 +122,7 @@ def _stream_handle(stream, device):
 def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
             return_state=False, reverse=False, accumulate=False, reset_every=0,
             check_finite=False, workspace=None, stream=None, stage_ms=None, mode="token", gamma=None,
-            norm_keys=False, norm_queries=False, k_norm_weight=None, q_norm_weight=None):
+            norm_keys=False, norm_queries=False, k_norm_weight=None, q_norm_weight=None, status=None):
     """Chunkwise gated delta rule forward on CUDA tensors.
 
     q,k [B,T,H,d_k], v [B,T,H,d_v] (bf16 or fp32, all the same), alpha/beta
@@ -136,6 +137,8 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     ``norm_keys`` / ``norm_queries`` apply the q/k prologue first: keys
     ReLU(RMSNorm(k)) / sqrt(d_k * frame_len), queries ReLU(RMSNorm(q)), with
     optional fp32 [d_k] RMSNorm weights.
+    ``status`` (a CUDA int32 tensor of one element) receives, in stream order,
+    0 or a nonzero code when a bounded device-side wait gave up.
     Returns (o, S_out or None).
     """
     import torch
@@ -178,6 +181,9 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     a.S_in, a.S_out, a.o = _ptr(S_in), _ptr(S_out), _ptr(o)
     a.mode = GDN_MODE_FRAME if frame else GDN_MODE_TOKEN
     a.gamma = _ptr(gamma) if frame else None
+    if status is not None and (not status.is_cuda or status.dtype != torch.int32 or status.numel() < 1):
+        raise GdnError(1, "status must be a CUDA int32 tensor")
+    a.status_dev = _ptr(status)
     a.qk_norm = (GDN_QK_NORM_KEYS if norm_keys else 0) | (GDN_QK_NORM_QUERIES if norm_queries else 0)
     a.k_norm_weight = _ptr(k_norm_weight) if norm_keys else None
     a.q_norm_weight = _ptr(q_norm_weight) if norm_queries else None

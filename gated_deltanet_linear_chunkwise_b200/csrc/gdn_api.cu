@@ -148,6 +148,10 @@ int validate(const gdn_args &a, gdn::Problem &p) {
             set_err("%s = %p is not 16-byte aligned", names[i], ptrs[i]);
             return GDN_ERR_ALIGNMENT;
         }
+    if (a.status_dev && (reinterpret_cast<uintptr_t>(a.status_dev) & 3u)) {
+        set_err("status_dev = %p is not 4-byte aligned", (const void *)a.status_dev);
+        return GDN_ERR_ALIGNMENT;
+    }
     if (a.workspace && (reinterpret_cast<uintptr_t>(a.workspace) & 255u)) {
         set_err("workspace = %p is not 256-byte aligned", a.workspace);
         return GDN_ERR_ALIGNMENT;
@@ -224,6 +228,12 @@ int run(const gdn_args &a) noexcept {
         cudaStream_t s = reinterpret_cast<cudaStream_t>(a.stream);
         const size_t sbytes = (size_t)a.B * a.H * a.d_v * a.d_k * sizeof(float);
 
+        if (a.B == 0 || a.H == 0 || a.T == 0) {  // nothing to compute
+            if (a.status_dev) {
+                cudaError_t e = cudaMemsetAsync(a.status_dev, 0, sizeof(int), s);
+                if (e) return cuda_fail(e, "status word");
+            }
+        }
         if (a.B == 0 || a.H == 0) return GDN_OK;
         if (a.T == 0) {  // nothing to scan: the final state is the initial state
             if (a.S_out && a.S_out != a.S_in) {
@@ -268,6 +278,10 @@ int run(const gdn_args &a) noexcept {
         if (p.qk_norm)  // normalised q / k copies after the operator's scratch; p now points at them
             e = gdn::launch_qk_prologue(p, (char *)ws + operator_workspace(p), s);
         if (e == cudaSuccess) e = tc ? gdn::launch_tc(p, ws, s, evp) : gdn::launch_simt(p, ws, s, evp);
+        // the device-side wait status, in stream order, for callers that check it later
+        if (e == cudaSuccess && a.status_dev)
+            e = tc ? cudaMemcpyAsync(a.status_dev, gdn::tc_error_word(p, ws), sizeof(int), cudaMemcpyDeviceToDevice, s)
+                   : cudaMemsetAsync(a.status_dev, 0, sizeof(int), s);
         // synchronous modes also report a device-side wait that gave up
         int timed_out = 0;
         if (e == cudaSuccess && tc && (a.stage_ms || a.check_finite)) {

@@ -213,6 +213,11 @@ int gdn_fwd_noalloc(const void *q, const void *k, const void *v,
  *                   not modified.  0: the inputs are used as given.
  *   k_norm_weight,  optional device fp32 [d_k] RMSNorm weights of the keys and
  *   q_norm_weight   queries (NULL: ones); read only when their bit is set.
+ *   status_dev      optional device int: at the end of the pass (in stream
+ *                   order, without synchronising) the library writes 0 there,
+ *                   or nonzero when a bounded device-side wait gave up and the
+ *                   outputs are not valid (what the synchronous modes report
+ *                   as GDN_ERR_TIMEOUT).  4-byte aligned.
  */
 typedef struct gdn_args {
     int struct_size;
@@ -238,6 +243,7 @@ typedef struct gdn_args {
     int qk_norm;
     const float *k_norm_weight;
     const float *q_norm_weight;
+    int *status_dev;
 } gdn_args;
 
 enum { GDN_MODE_TOKEN = 0, GDN_MODE_FRAME = 1 };
@@ -267,8 +273,9 @@ const char *gdn_status_string(int status);
 const char *gdn_last_error(void);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH.  The gdn_args layout
- * belongs to the version: 0.2.0 added mode, gamma, qk_norm and the RMSNorm
- * weights (struct_size guards a caller built against another layout). */
+ * belongs to the version: 0.2.0 added mode, gamma, qk_norm, the RMSNorm
+ * weights and status_dev (struct_size guards a caller built against another
+ * layout). */
 #define GDN_VERSION 200
 int gdn_version(void);
 

@@ -47,7 +47,7 @@ def test_struct_size_matches_header():
     a.struct_size = ctypes.sizeof(binding.GdnArgs) + 8
     rc = g.load_library().gdn_fwd_ex(ctypes.byref(a))
     assert rc == 1 and "struct_size" in g.last_error()
-    assert ctypes.sizeof(binding.GdnArgs) == 200  # LP64 layout of gdn_args
+    assert ctypes.sizeof(binding.GdnArgs) == 208  # LP64 layout of gdn_args
 
 
 def _ex_args(**kw):
@@ -67,6 +67,7 @@ def _ex_args(**kw):
     (dict(mode=1, alpha=None, gamma=FAKE + 16384 + 8), 1, "overlaps"),  # o over gamma
     (dict(qk_norm=4), 1, "qk_norm"),                  # not a mask of the two prologue bits
     (dict(qk_norm=-1), 1, "qk_norm"),
+    (dict(status_dev=FAKE + 2), 4, "status_dev"),     # not 4-byte aligned
 ])
 def test_mode_validation(kw, status, text):
     # rejected before any device work (no GPU needed)

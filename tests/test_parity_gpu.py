@@ -171,6 +171,24 @@ def test_reverse_accumulate_in_caller_workspace(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_status_word_reports_no_timeout(dtype):
+    # status_dev is written in stream order: 0 after a pass whose device waits all completed
+    inp = W.draw(1, 2, 2 * 64, 32, 32, frame_len=64, seed=27, regime="slow", dtype=dtype)
+    d = dev(inp)
+    st = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    o, _ = g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], 64, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    o_ref, _ = ora(inp)
+    assert rel(o.double().cpu(), o_ref) <= TOL[dtype]
+    st.fill_(7)
+    z = d["q"][:, :0].contiguous()
+    g.gdn_fwd(z, z, z, d["alpha"][:, :0].contiguous(), d["beta"][:, :0].contiguous(), 64, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_step_chain_equals_single_call(dtype):
     L = 80
     inp = W.draw(2, 3, 7 * L, 64, 64, frame_len=L, seed=31, regime="slow", dtype=dtype, state_std=0.1)
