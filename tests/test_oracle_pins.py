@@ -12,6 +12,8 @@ import os
 from fractions import Fraction
 
 import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
 import pytest
 
 import oracle
@@ -138,6 +140,21 @@ def test_numpy_twin_matches_c():
     o2, S2 = oracle.token_recurrence_numpy(q, k, v, alpha, beta, S0)
     np.testing.assert_allclose(o1, o2, atol=1e-12)
     np.testing.assert_allclose(S1, S2, atol=1e-12)
+
+
+@settings(max_examples=40, deadline=None)
+@given(B=st.integers(1, 2), T=st.integers(1, 9), H=st.integers(1, 3), dk=st.integers(1, 5),
+       dv=st.integers(1, 5), seed=st.integers(0, 2 ** 31 - 1), with_state=st.booleans())
+def test_numpy_twin_matches_c_any_shape(B, T, H, dk, dv, seed, with_state):
+    """The C build against the numpy twin over random small shapes (layout and stride
+    mistakes in the C loops show up at odd sizes)."""
+    rng = np.random.default_rng(seed)
+    q, k, v, alpha, beta = _rand(rng, B, T, H, dk, dv, unit_keys=False, alpha_lo=0.0)
+    S0 = rng.standard_normal((B, H, dv, dk)) if with_state else None
+    o1, S1 = oracle.token_recurrence(q, k, v, alpha, beta, S0, nthreads=1)
+    o2, S2 = oracle.token_recurrence_numpy(q, k, v, alpha, beta, S0)
+    np.testing.assert_allclose(o1, o2, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(S1, S2, rtol=1e-10, atol=1e-10)
 
 
 def test_beta0_alpha1_identity():
