@@ -69,6 +69,7 @@ extern "C" int gdn_fwd_noalloc(const void *q, const void *k, const void *v, cons
                                int H, long long T, int frame_len, int d_k, int d_v,
                                gdn_stream_t stream) {
     try {
+        gdn::set_error_text("");  // like every entry point: no stale text after a successful call
         gdn_args a = {};
         a.struct_size = (int)sizeof(gdn_args);
         a.dtype = GDN_DTYPE_BF16;

@@ -32,6 +32,16 @@ def dev(inp):
     return {k: (None if v is None else v.cuda().contiguous()) for k, v in inp.items()}
 
 
+def accumulate_offset(o_ref, dtype, seed):
+    """What o holds before an accumulating call: values exactly representable in the
+    output dtype, a quarter of the result's scale.  o then stores round(o + result) once,
+    so o - offset differs from the result by one rounding at |o + offset| <= 1.25 max|o|,
+    the same order as the rounding of a plain call's output."""
+    gen = torch.Generator().manual_seed(1234 + seed)
+    scale = 0.25 * float(np.abs(o_ref).max())
+    return (torch.randn(o_ref.shape, generator=gen, dtype=torch.float64) * scale).to(dtype)
+
+
 def gpu_fwd(inp, frame_len, S_in=None, **kw):
     d = dev(inp)
     S = None if S_in is None else S_in.cuda().contiguous()
@@ -147,11 +157,11 @@ def test_reverse_reset_not_dividing_length(dtype):
     L = 64
     inp = W.draw(1, 3, 5 * L, 48, 32, frame_len=L, seed=23, regime="slow", dtype=dtype, state_std=0.2)
     d = dev(inp)
-    o_acc = (d["v"][..., :32] * 0 + 0.25).contiguous()  # accumulate into a non-zero o
-    o_r, S_r = g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, d["S_in"], return_state=True,
-                         reverse=True, reset_every=2 * L, o=o_acc.clone(), accumulate=True)
     o_ref, S_ref = ora(inp, inp["S_in"], reverse=True, reset_every=2 * L)
-    assert rel(o_r.double().cpu() - 0.25, o_ref) <= TOL[dtype] + (4e-3 if dtype == "bf16" else 0.0)
+    c = accumulate_offset(o_ref, d["q"].dtype, seed=1)  # accumulate into a non-zero o
+    o_r, S_r = g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, d["S_in"], return_state=True,
+                         reverse=True, reset_every=2 * L, o=c.cuda(), accumulate=True)
+    assert rel(o_r.double().cpu() - c.double(), o_ref) <= TOL[dtype]
     assert rel(S_r.double().cpu(), S_ref) <= TOL[dtype]
 
 
@@ -162,12 +172,12 @@ def test_reverse_accumulate_in_caller_workspace(dtype):
     inp = W.draw(B, H, F * L, dk, dv, frame_len=L, seed=25, regime="slow", dtype=dtype)
     d = dev(inp)
     ws = torch.empty(g.workspace_bytes(B, H, F * L, L, dk, dv, dtype), dtype=torch.uint8, device="cuda")
-    o0 = torch.full((B, F * L, H, dv), 0.5, dtype=d["q"].dtype, device="cuda")
-    o_r, _ = g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, None, o=o0, reverse=True,
+    o_ref, _ = ora(inp, None, reverse=True)
+    c = accumulate_offset(o_ref, d["q"].dtype, seed=2)
+    o_r, _ = g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], L, None, o=c.cuda(), reverse=True,
                        accumulate=True, workspace=ws)
     torch.cuda.synchronize()
-    o_ref, _ = ora(inp, None, reverse=True)
-    assert rel(o_r.double().cpu() - 0.5, o_ref) <= TOL[dtype] + (4e-3 if dtype == "bf16" else 0.0)
+    assert rel(o_r.double().cpu() - c.double(), o_ref) <= TOL[dtype]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

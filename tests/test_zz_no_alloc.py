@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 
 import gated_deltanet_linear_chunkwise_b200 as g
+import oracle
 from gated_deltanet_linear_chunkwise_b200 import workloads as W
 
 TOL = 2e-2  # the bf16-input bar the parity tests use
@@ -51,6 +52,9 @@ def test_noalloc_matches_gdn_fwd_twice():
     lib = _lib()
     L, d, B, H = 880, 112, 2, 4
     stream = torch.cuda.current_stream()
+    # leave an error text behind on this thread; a successful call must clear it
+    assert lib.gdn_fwd_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 1, 2, 100, 64, 64, 64, None) == 2
+    assert g.last_error() != ""
     for call, (seed, with_state) in enumerate([(11, True), (12, False)]):
         inp = W.draw(B, H, 2 * L, d, d, frame_len=L, seed=seed, regime="slow", dtype="bf16", state_std=0.05)
         dv = {k: (None if t is None else t.cuda().contiguous()) for k, t in inp.items()}
@@ -66,7 +70,13 @@ def test_noalloc_matches_gdn_fwd_twice():
                                  None if S_in is None else S_in.data_ptr(), S.data_ptr(), o.data_ptr(),
                                  B, H, 2 * L, L, d, d, stream.cuda_stream)
         assert rc == 0, g.last_error()
+        assert g.last_error() == ""  # no stale text from an earlier failure
         torch.cuda.synchronize()
         assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
         assert _rel(o, o_ref) <= TOL, ("call", call)
         assert _rel(S, S_ref) <= TOL, ("call", call)
+        # and against the fp64 token loop itself, at the same bar
+        S0 = None if S_in is None else inp["S_in"]
+        o_ora, S_ora = oracle.token_recurrence(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], S0)
+        assert _rel(o, torch.from_numpy(o_ora)) <= TOL, ("call", call)
+        assert _rel(S, torch.from_numpy(S_ora)) <= TOL, ("call", call)
