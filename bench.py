@@ -217,6 +217,133 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def other_workloads(g, W, dev, stream, regime, rank):
+    """Device time of the three other timed workloads, each beside its bar (half of the
+    tensor roofline at the measured bf16 peak).  None of them is the headline metric.
+
+    short_clip  one gdn_fwd over 21 frames x 880 tokens, 20 heads (B=1): ms per pass
+    ar_rollout  B=2, 40 chained gdn_step calls (4 + 39 x 3 frames, one alpha per frame and
+                head), the fp32 state carried in place from call to call: total and per call
+    decode      B=8, 100 chained single-frame gdn_step calls from a preloaded N(0, 0.02)
+                state: per-call device time (median) and the whole loop; the calls cycle over
+                4 drawn frames of fresh q/k/v/alpha/beta (each call's inputs, 95 MB, were last
+                touched three calls earlier, so they come from HBM, not L2)
+    """
+    import torch
+    out = {}
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    # ---- short clip: one pass over 18,480 tokens
+    w = W.WORKLOADS["short_clip"]
+    inp = W.make_inputs(w, regime, seed=W.SEEDS["short_clip"] + 7919 * rank)
+    d = {k: (None if t is None else t.to(dev).contiguous()) for k, t in inp.items()}
+    o = torch.empty(w.B, w.T, w.H, w.d_v, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(w.B, w.H, w.d_v, w.d_k, dtype=torch.float32, device=dev)
+    ws = torch.empty(g.workspace_bytes(w.B, w.H, w.T, w.frame_len, w.d_k, w.d_v, "bf16"), dtype=torch.uint8,
+                     device=dev)
+    run = lambda: g.gdn_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], w.frame_len, None,  # noqa: E731
+                            S_out=S, o=o, workspace=ws, stream=stream)
+    for _ in range(3):
+        run()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(20):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / 20
+    f_alg = flops_total(w.frame_len, w.d_k, w.d_v) * w.B * w.H * w.frames
+    out["short_clip"] = {"ms_per_pass": ms, "tokens_per_s": w.B * w.T / (ms * 1e-3),
+                         "frac_tensor": f_alg / (ms * 1e-3) / 1e12 / peaks()["bf16_tflops"],
+                         "bar_ms": 2 * f_alg / (peaks()["bf16_tflops"] * 1e12) * 1e3,
+                         "what": "B=1 H=20 21 frames x 880 tokens, one gdn_fwd"}
+    del d, o, S, ws
+
+    # ---- chunk-causal rollout: 40 gdn_step calls, state carried
+    w = W.WORKLOADS["ar_rollout"]
+    inp = W.make_inputs(w, regime, seed=W.SEEDS["ar_rollout"] + 7919 * rank)
+    L = w.frame_len
+    calls, t0 = [], 0
+    for nf in w.calls:  # contiguous per-call slices, cut before the timed region
+        t1 = t0 + nf * L
+        calls.append({k: inp[k][:, t0:t1].to(dev).contiguous() for k in ("q", "k", "v", "alpha", "beta")})
+        t0 = t1
+    del inp
+    S = torch.zeros(w.B, w.H, w.d_v, w.d_k, dtype=torch.float32, device=dev)
+    o_all = [torch.empty(w.B, c["q"].shape[1], w.H, w.d_v, dtype=torch.bfloat16, device=dev) for c in calls]
+    ws = torch.empty(g.workspace_bytes(w.B, w.H, 4 * L, L, w.d_k, w.d_v, "bf16"), dtype=torch.uint8, device=dev)
+
+    def rollout(events=None):
+        for i, c in enumerate(calls):
+            if events:
+                events[i][0].record(stream)
+            g.gdn_step(c["q"], c["k"], c["v"], c["alpha"], c["beta"], L, S, S_out=S, o=o_all[i], workspace=ws,
+                       stream=stream)
+            if events:
+                events[i][1].record(stream)
+
+    rollout()
+    reps = 3
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(reps):
+        rollout()
+    e1.record(stream)
+    per = [(ev(), ev()) for _ in calls]
+    rollout(per)
+    torch.cuda.synchronize(dev)
+    total = e0.elapsed_time(e1) / reps
+    call_ms = [a.elapsed_time(b) for a, b in per]
+    f_alg = flops_total(L, w.d_k, w.d_v) * w.B * w.H * w.frames
+    out["ar_rollout"] = {"ms_total": total, "ms_per_call_mean": total / len(calls),
+                         "ms_per_call_median": statistics.median(call_ms),
+                         "tokens_per_s": w.B * w.T / (total * 1e-3),
+                         "frac_tensor": f_alg / (total * 1e-3) / 1e12 / peaks()["bf16_tflops"],
+                         "bar_ms_total": 2 * f_alg / (peaks()["bf16_tflops"] * 1e12) * 1e3,
+                         "what": "B=2 H=20, 40 chained gdn_step calls (4 + 39 x 3 frames of 880), "
+                                 "per-frame alpha, state carried in place; host launch gaps included"}
+    del calls, o_all, ws
+
+    # ---- streaming decode: 100 single-frame calls at B=8, state carried
+    w = W.WORKLOADS["decode"]
+    L = w.frame_len
+    seed = W.SEEDS["decode"] + 7919 * rank
+    drawn = [W.make_inputs(w, regime, seed=seed, call=c) for c in range(4)]
+    S = drawn[0]["S_in"].to(dev).contiguous()
+    frames = [{k: x[k].to(dev).contiguous() for k in ("q", "k", "v", "alpha", "beta")} for x in drawn]
+    del drawn
+    o = torch.empty(w.B, L, w.H, w.d_v, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(g.workspace_bytes(w.B, w.H, L, L, w.d_k, w.d_v, "bf16"), dtype=torch.uint8, device=dev)
+
+    def decode(events=None):
+        for i in range(len(w.calls)):
+            c = frames[i % len(frames)]
+            if events:
+                events[i][0].record(stream)
+            g.gdn_step(c["q"], c["k"], c["v"], c["alpha"], c["beta"], L, S, S_out=S, o=o, workspace=ws,
+                       stream=stream)
+            if events:
+                events[i][1].record(stream)
+
+    decode()
+    per = [(ev(), ev()) for _ in w.calls]
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    decode(per)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    call_ms = [a.elapsed_time(b) for a, b in per]
+    f_alg = flops_total(L, w.d_k, w.d_v) * w.B * w.H
+    med = statistics.median(call_ms)
+    out["decode"] = {"ms_per_call_median": med, "ms_loop_per_call": e0.elapsed_time(e1) / len(w.calls),
+                     "tokens_per_s": w.B * L / (med * 1e-3),
+                     "frac_tensor": f_alg / (med * 1e-3) / 1e12 / peaks()["bf16_tflops"],
+                     "bar_ms_per_call": 2 * f_alg / (peaks()["bf16_tflops"] * 1e12) * 1e3,
+                     "what": "B=8 H=20, 100 chained single-frame gdn_step calls, preloaded state; "
+                             "per-call device time between events around each call"}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -375,6 +502,8 @@ def main():
     torch.cuda.synchronize(dev)
     e2e_ms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, device=dev)
 
+    extra = other_workloads(g, W, dev, stream, args.regime, rank) if args.workload == WORKLOAD else {}
+
     pk = peaks()
     nfh = B * H * w.frames
     if rank == 0:
@@ -431,6 +560,7 @@ def main():
                                                         "(prologue kernel, not fused)"}),
             "clocks": clk.summary(),
         }
+        line.update(extra)
         if not args.no_cpu_baseline and world == 1 and args.workload == WORKLOAD:
             line["cpu_baseline"] = cpu_baseline(args.regime, args.cpu_frames, inp)
         print(json.dumps(line), flush=True)
