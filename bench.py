@@ -557,7 +557,7 @@ def main():
                               with_qk_prologue={"ms_per_pass": fwp_ms,
                                                 "tokens_per_s": tokens / (fwp_ms * 1e-3),
                                                 "what": "raw q, k through norm_keys + norm_queries "
-                                                        "(prologue kernel, not fused)"}),
+                                                        "(feature maps applied to the staged tiles)"}),
             "clocks": clk.summary(),
         }
         line.update(extra)

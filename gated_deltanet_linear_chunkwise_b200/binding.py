@@ -23,7 +23,7 @@ STATUS = {
 
 # every symbol include/gdn.h declares
 EXPORTS = ("gdn_fwd", "gdn_fwd_f32", "gdn_step", "gdn_step_f32", "gdn_fwd_ex", "gdn_fwd_host",
-           "gdn_workspace_bytes", "gdn_status_string", "gdn_last_error", "gdn_version")
+           "gdn_apply_maps", "gdn_workspace_bytes", "gdn_status_string", "gdn_last_error", "gdn_version")
 
 
 class GdnError(RuntimeError):
@@ -49,12 +49,14 @@ class GdnArgs(ctypes.Structure):
         ("mode", ctypes.c_int), ("gamma", ctypes.c_void_p),
         ("qk_norm", ctypes.c_int), ("k_norm_weight", ctypes.c_void_p), ("q_norm_weight", ctypes.c_void_p),
         ("status_dev", ctypes.c_void_p),
+        ("phase", ctypes.c_int), ("segment_map", ctypes.c_void_p),
     ]
 
 GDN_MODE_TOKEN = 0
 GDN_MODE_FRAME = 1
 GDN_QK_NORM_KEYS = 1
 GDN_QK_NORM_QUERIES = 2
+PHASES = {"all": 0, "prepare": 1, "finish": 2}
 
 NUM_STAGES = 7
 STAGES = ("gates", "diag_inverse", "intra", "transition", "scan", "u", "output")
@@ -82,6 +84,8 @@ def load_library(path: str = LIB_PATH):
     lib.gdn_fwd_host.restype = I
     lib.gdn_fwd_ex.argtypes = [ctypes.POINTER(GdnArgs)]
     lib.gdn_fwd_ex.restype = I
+    lib.gdn_apply_maps.argtypes = [V, V, I, I, I, I, I, V]
+    lib.gdn_apply_maps.restype = I
     lib.gdn_workspace_bytes.argtypes = [I, I, LL, I, I, I, I]
     lib.gdn_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_status_string.argtypes = [I]
@@ -122,7 +126,8 @@ def _stream_handle(stream, device):
 def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
             return_state=False, reverse=False, accumulate=False, reset_every=0,
             check_finite=False, workspace=None, stream=None, stage_ms=None, mode="token", gamma=None,
-            norm_keys=False, norm_queries=False, k_norm_weight=None, q_norm_weight=None, status=None):
+            norm_keys=False, norm_queries=False, k_norm_weight=None, q_norm_weight=None, status=None,
+            phase="all", segment_map=None):
     """Chunkwise gated delta rule forward on CUDA tensors.
 
     q,k [B,T,H,d_k], v [B,T,H,d_v] (bf16 or fp32, all the same), alpha/beta
@@ -139,7 +144,11 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     optional fp32 [d_k] RMSNorm weights.
     ``status`` (a CUDA int32 tensor of one element) receives, in stream order,
     0 or a nonzero code when a bounded device-side wait gave up.
-    Returns (o, S_out or None).
+    ``phase="prepare"`` runs only the stages that do not depend on the entering
+    state into ``workspace`` (required), and with ``segment_map`` (fp32
+    [B, H, d_k + d_v, d_k]) also writes the call's map S_end = S_begin Phi + Psi;
+    ``phase="finish"`` then runs the rest from ``S_in`` on the same workspace.
+    Returns (o, S_out or None) (o is None for a prepare call).
     """
     import torch
     B, T, H, d_k = q.shape
@@ -169,11 +178,20 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
     for name, t in (("S_in", S_in), ("S_out", S_out), ("o", o)):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise GdnError(1, "%s must be a contiguous CUDA tensor" % name)
-    if o is None:
+    if phase not in PHASES:
+        raise GdnError(1, "phase must be 'all', 'prepare' or 'finish'")
+    prepare = phase == "prepare"
+    if segment_map is not None and (not segment_map.is_cuda or not segment_map.is_contiguous()
+                                    or segment_map.dtype != torch.float32
+                                    or tuple(segment_map.shape) != (B, H, d_k + d_v, d_k)):
+        raise GdnError(1, "segment_map must be a contiguous fp32 CUDA tensor [B, H, d_k + d_v, d_k]")
+    if o is None and not prepare:
         o = (torch.zeros if accumulate else torch.empty)((B, T, H, d_v), dtype=q.dtype, device=q.device)
-    if S_out is None and return_state:
+    if S_out is None and return_state and not prepare:
         S_out = torch.empty((B, H, d_v, d_k), dtype=torch.float32, device=q.device)
     a = GdnArgs()
+    a.phase = PHASES[phase]
+    a.segment_map = _ptr(segment_map)
     a.struct_size = ctypes.sizeof(GdnArgs)
     a.dtype = GDN_DTYPE_BF16 if q.dtype == torch.bfloat16 else GDN_DTYPE_F32
     a.q, a.k, a.v = _ptr(q), _ptr(k), _ptr(v)
@@ -199,6 +217,22 @@ def gdn_fwd(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,
         a.stage_ms = ctypes.cast(stage_ms, ctypes.c_void_p)
     check(load_library().gdn_fwd_ex(ctypes.byref(a)))
     return o, S_out
+
+
+def apply_maps(S, maps, *, stream=None):
+    """S <- S Phi_j + Psi_j for each segment map in order, in place (``gdn_apply_maps``):
+    S fp32 [B, H, d_v, d_k], maps fp32 [n, B, H, d_k + d_v, d_k] (CUDA, contiguous).
+    Returns S."""
+    import torch
+    B, H, d_v, d_k = S.shape
+    for name, t in (("S", S), ("maps", maps)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float32:
+            raise GdnError(1, "%s must be a contiguous fp32 CUDA tensor" % name)
+    if maps.dim() != 5 or tuple(maps.shape[1:]) != (B, H, d_k + d_v, d_k):
+        raise GdnError(2, "maps must have shape [n, B, H, d_k + d_v, d_k]")
+    check(load_library().gdn_apply_maps(_ptr(S), _ptr(maps), maps.shape[0], B, H, d_k, d_v,
+                                        _stream_handle(stream, S.device)))
+    return S
 
 
 def gdn_fwd_host(q, k, v, alpha, beta, frame_len, S_in=None, *, S_out=None, o=None,

@@ -4,6 +4,7 @@
 // call returns its status with no launch and no output touched.  No C++
 // exception crosses the ABI (every entry point is noexcept and catches).
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -129,7 +130,30 @@ int validate(const gdn_args &a, gdn::Problem &p) {
     const long long F = a.T / a.frame_len;
     const bool empty = (a.B == 0 || a.H == 0 || a.T == 0);
     const bool frame = a.mode == GDN_MODE_FRAME;
-    if (!empty && (!a.q || !a.k || !a.v || !a.beta || !a.o)) {
+    if (a.phase != GDN_PHASE_ALL && a.phase != GDN_PHASE_PREPARE && a.phase != GDN_PHASE_FINISH) {
+        set_err("phase must be GDN_PHASE_ALL, GDN_PHASE_PREPARE or GDN_PHASE_FINISH (got %d)", a.phase);
+        return GDN_ERR_INVALID_ARG;
+    }
+    if (a.phase != GDN_PHASE_ALL) {
+        if (!a.workspace) {
+            set_err("a PREPARE / FINISH call keeps its state in a caller workspace (workspace is NULL)");
+            return GDN_ERR_INVALID_ARG;
+        }
+        if (frame || a.reverse || a.accumulate_o || a.qk_norm) {
+            set_err("PREPARE / FINISH calls take the token-wise forward scan without reverse, accumulate_o or qk_norm");
+            return GDN_ERR_NOT_IMPLEMENTED;
+        }
+    }
+    if (a.segment_map && a.phase != GDN_PHASE_PREPARE) {
+        set_err("segment_map is written by GDN_PHASE_PREPARE calls only");
+        return GDN_ERR_INVALID_ARG;
+    }
+    if (misaligned(a.segment_map)) {
+        set_err("segment_map = %p is not 16-byte aligned", (const void *)a.segment_map);
+        return GDN_ERR_ALIGNMENT;
+    }
+    const bool need_o = a.phase != GDN_PHASE_PREPARE;
+    if (!empty && (!a.q || !a.k || !a.v || !a.beta || (need_o && !a.o))) {
         set_err("q, k, v, beta and o are required (one is NULL)");
         return GDN_ERR_INVALID_ARG;
     }
@@ -175,6 +199,14 @@ int validate(const gdn_args &a, gdn::Problem &p) {
         }
     }
     if (overlap(a.o, nv, a.S_out, ns)) { set_err("o overlaps S_out"); return GDN_ERR_INVALID_ARG; }
+    if (a.segment_map) {
+        const size_t nm = (size_t)a.B * a.H * (a.d_k + a.d_v) * a.d_k * 4;
+        for (int i = 0; i < 7; ++i)
+            if (overlap(a.segment_map, nm, ins[i], insz[i])) {
+                set_err("segment_map overlaps input %s", in_names[i]);
+                return GDN_ERR_INVALID_ARG;
+            }
+    }
 
     p.dtype = a.dtype;
     p.q = a.q; p.k = a.k; p.v = a.v;
@@ -188,6 +220,13 @@ int validate(const gdn_args &a, gdn::Problem &p) {
     p.k_norm_weight = (a.qk_norm & GDN_QK_NORM_KEYS) ? a.k_norm_weight : nullptr;
     p.q_norm_weight = (a.qk_norm & GDN_QK_NORM_QUERIES) ? a.q_norm_weight : nullptr;
     if (frame) p.alpha = nullptr;
+    p.phase = a.phase;
+    p.map_out = a.segment_map;
+    if (p.phase == GDN_PHASE_PREPARE) {  // nothing of the state or the output is touched
+        p.S_in = nullptr;
+        p.S_out = nullptr;
+        p.o = nullptr;
+    }
     return GDN_OK;
 }
 
@@ -199,7 +238,13 @@ size_t operator_workspace(const gdn::Problem &p) {
     return use_tc(p) ? gdn::tc_workspace_bytes(p) : gdn::simt_workspace_bytes(p);
 }
 
-size_t workspace_for(const gdn::Problem &p) { return operator_workspace(p) + gdn::qk_prologue_bytes(p); }
+// The q/k prologue runs as its own pass (normalised copies after the operator's scratch)
+// except where the kernels apply it to their staged tiles.
+bool separate_prologue(const gdn::Problem &p) { return p.qk_norm && !gdn::tc_fuses_qk_prologue(p); }
+
+size_t workspace_for(const gdn::Problem &p) {
+    return operator_workspace(p) + (separate_prologue(p) ? gdn::qk_prologue_bytes(p) : 0);
+}
 
 __global__ void nonfinite_scan_f32(const float *x, long long n, int *flag) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
@@ -235,6 +280,13 @@ int run(const gdn_args &a) noexcept {
             }
         }
         if (a.B == 0 || a.H == 0) return GDN_OK;
+        if (a.T == 0 && a.phase == GDN_PHASE_PREPARE) {  // an empty segment maps every state to itself
+            if (a.segment_map) {
+                cudaError_t e = gdn::launch_identity_map(a.segment_map, a.B, a.H, a.d_k, a.d_v, s);
+                if (e) return cuda_fail(e, "segment map");
+            }
+            return GDN_OK;
+        }
         if (a.T == 0) {  // nothing to scan: the final state is the initial state
             if (a.S_out && a.S_out != a.S_in) {
                 cudaError_t e = a.S_in ? cudaMemcpyAsync(a.S_out, a.S_in, sbytes, cudaMemcpyDeviceToDevice, s)
@@ -275,7 +327,7 @@ int run(const gdn_args &a) noexcept {
         }
         const bool tc = use_tc(p);
         cudaError_t e = cudaSuccess;
-        if (p.qk_norm)  // normalised q / k copies after the operator's scratch; p now points at them
+        if (separate_prologue(p))  // normalised q / k copies after the operator's scratch; p now points at them
             e = gdn::launch_qk_prologue(p, (char *)ws + operator_workspace(p), s);
         if (e == cudaSuccess) e = tc ? gdn::launch_tc(p, ws, s, evp) : gdn::launch_simt(p, ws, s, evp);
         // the device-side wait status, in stream order, for callers that check it later
@@ -351,6 +403,20 @@ namespace gdn {
 // Validation and error text shared with the other entry-point files.
 int validate_args(const gdn_args &a, Problem &p) { return validate(a, p); }
 void set_error_text(const char *msg) { set_err("%s", msg); }
+
+int debug_drop_signal() {
+    const char *e = getenv("GDN_DEBUG_DROP_SIGNAL");
+    return (e && e[0] == '1') ? 1 : 0;
+}
+
+uint64_t wait_limit_ns() {
+    const char *e = getenv("GDN_DEBUG_WAIT_LIMIT_US");
+    if (!e || !*e) return 2000000000ull;
+    char *end = nullptr;
+    const unsigned long long us = strtoull(e, &end, 10);
+    if (end == e || us >= 2000000ull) return 2000000000ull;
+    return (uint64_t)us * 1000ull;
+}
 }  // namespace gdn
 
 extern "C" {
@@ -385,6 +451,44 @@ int gdn_step_f32(const float *q, const float *k, const float *v, const float *al
         return GDN_ERR_INVALID_ARG;
     }
     return gdn_fwd_f32(q, k, v, alpha, beta, S_in, S_out, o, B, H, T, frame_len, d_k, d_v, stream);
+}
+
+int gdn_apply_maps(float *S, const float *maps, int n_maps, int B, int H, int d_k, int d_v, gdn_stream_t stream) {
+    try {
+        g_err[0] = '\0';
+        if (B < 0 || H < 0 || n_maps < 0) {
+            set_err("negative size: B=%d H=%d n_maps=%d", B, H, n_maps);
+            return GDN_ERR_INVALID_ARG;
+        }
+        if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) {
+            set_err("head dims d_k=%d d_v=%d: each must be a multiple of 16 in [16, 128]", d_k, d_v);
+            return GDN_ERR_UNSUPPORTED;
+        }
+        if ((long long)B * H >= 2147483648ll) {
+            set_err("B*H exceeds 2^31");
+            return GDN_ERR_SHAPE;
+        }
+        if ((long long)B * H == 0 || n_maps == 0) return GDN_OK;
+        if (!S || !maps) {
+            set_err("S and maps are required (one is NULL)");
+            return GDN_ERR_INVALID_ARG;
+        }
+        if (misaligned(S) || misaligned(maps)) {
+            set_err("S = %p or maps = %p is not 16-byte aligned", (void *)S, (const void *)maps);
+            return GDN_ERR_ALIGNMENT;
+        }
+        const size_t ns = (size_t)B * H * d_v * d_k * 4, nm = (size_t)n_maps * B * H * (d_k + d_v) * d_k * 4;
+        if (overlap(S, ns, maps, nm)) {
+            set_err("S overlaps maps");
+            return GDN_ERR_INVALID_ARG;
+        }
+        cudaError_t e = gdn::launch_apply_maps(S, maps, n_maps, B, H, d_k, d_v, reinterpret_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "apply maps");
+        return GDN_OK;
+    } catch (...) {
+        set_err("internal error (exception caught at the ABI boundary)");
+        return GDN_ERR_CUDA;
+    }
 }
 
 int gdn_fwd_ex(const gdn_args *a) {

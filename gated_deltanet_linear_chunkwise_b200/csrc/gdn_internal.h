@@ -51,6 +51,8 @@ struct Problem {
     const float *gamma;     // GDN_MODE_FRAME: [B, F, H] per-frame decay
     int qk_norm;            // GDN_QK_NORM_* bits still to apply (the prologue clears them)
     const float *k_norm_weight, *q_norm_weight;  // [d_k] or NULL
+    int phase;              // GDN_PHASE_ALL / _PREPARE (state-independent stages) / _FINISH (scan on)
+    float *map_out;         // PREPARE: the segment's map [B, H, d_k + d_v, d_k] (Phi rows, then Psi), or NULL
 };
 
 // Memory index of the frame the scan visits at logical step f.  The
@@ -91,6 +93,15 @@ inline cudaError_t mark(cudaEvent_t *ev, int i, cudaStream_t s) {
     return ev ? cudaEventRecord(ev[i], s) : cudaSuccess;
 }
 
+// Limit of the kernels' bounded device-side waits for this call, in ns: 2 s, unless the
+// debug variable GDN_DEBUG_WAIT_LIMIT_US (read at every call) sets a shorter one so a
+// test can make the waits give up (gdn_api.cu).
+uint64_t wait_limit_ns();
+// Debug: GDN_DEBUG_DROP_SIGNAL=1 (read at every call) makes the diagonal-inverse kernel
+// withhold its first load, so the wait on it gives up at the limit above and the pass
+// reports GDN_ERR_TIMEOUT without any fault (the bounded-wait test).  0 otherwise.
+int debug_drop_signal();
+
 // Argument validation of the C ABI (gdn_api.cu): fills p or returns a gdn_status.
 int validate_args(const gdn_args &a, Problem &p);
 // Sets the thread-local text gdn_last_error() returns.
@@ -111,6 +122,14 @@ cudaError_t simt_intra_bf16x(const Problem &p, __nv_bfloat16 *X, cudaStream_t s)
 cudaError_t simt_transition_bf16x(const Problem &p, const __nv_bfloat16 *X, float *Mb, float *Nb, cudaStream_t s);
 cudaError_t simt_scan(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
                       cudaStream_t s);
+// The segment's composed map (p.map_out): the same scan over the augmented state
+// [Sig | P] from [0 | I], N added to the Sig part only, written as Phi = P^T, Psi = Sig^T so
+// that S_end = S_begin Phi + Psi over the call's frames.
+cudaError_t simt_segment_map(const Problem &p, const float *Mb, const float *Nb, cudaStream_t s);
+// S <- S Phi_j + Psi_j for the n maps in order (maps [n][B, H, d_k + d_v, d_k]).
+cudaError_t launch_apply_maps(float *S, const float *maps, int n, int B, int H, int dk, int dv, cudaStream_t s);
+// Phi = I, Psi = 0: the map of an empty segment.
+cudaError_t launch_identity_map(float *map, int B, int H, int dk, int dv, cudaStream_t s);
 cudaError_t simt_u_bf16x(const Problem &p, const __nv_bfloat16 *X, const float *Sig, __nv_bfloat16 *U,
                          cudaStream_t s);
 cudaError_t launch_simt(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev);

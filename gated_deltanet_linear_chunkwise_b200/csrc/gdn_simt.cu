@@ -259,7 +259,12 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
     constexpr int HALF = DK / 2;                     // contraction length per thread half
     const int dv = p.dv;
     const long long chain = blockIdx.x;
-    const int c0 = blockIdx.y * SCAN_COLS, ncol = min(SCAN_COLS, dv - c0);
+    // segment-map mode: the state is [Sig | P] (d_v + d_k columns) starting from [0 | I]; N is
+    // added to the Sig columns only (d_v is a multiple of 16, so a group lies in one part)
+    const bool map = p.map_out != nullptr;
+    const int ncols_all = map ? dv + DK : dv;
+    const int c0 = blockIdx.y * SCAN_COLS, ncol = min(SCAN_COLS, ncols_all - c0);
+    const bool add_n = c0 < dv;
     float *sM = (float *)smem;                       // 2 x [DK][DK]
     float *sS = sM + 2 * DK * DK;                    // [DK][16]
     float2 *sRed = reinterpret_cast<float2 *>(sS + DK * SCAN_COLS);  // [R][128] partial sums of the upper half
@@ -271,7 +276,8 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
     for (int e = tid; e < DK * SCAN_COLS; e += NT) {
         const int m = e >> 4, cc = e & 15;
         float val = 0.f;
-        if (p.S_in && cc < ncol) val = p.S_in[(chain * dv + c0 + cc) * (long long)DK + m];
+        if (map) val = (cc < ncol && c0 + cc >= dv && m == c0 + cc - dv) ? 1.f : 0.f;
+        else if (p.S_in && cc < ncol) val = p.S_in[(chain * dv + c0 + cc) * (long long)DK + m];
         sS[e] = val;
     }
     constexpr int NVEC = DK * DK / 4;  // 16-byte pieces of one M
@@ -287,7 +293,7 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
     for (int i = 0; i < R; ++i) {
         const int m = g + 16 * i;
         nxt[i] = make_float2(0.f, 0.f);
-        if (kh == 0 && p.F > 0) {
+        if (kh == 0 && p.F > 0 && add_n) {
             const long long idx = ((chain * p.F + scan_frame(p, 0)) * DK + m) * (long long)dv + c0;
             nxt[i].x = ca < ncol ? Nb[idx + ca] : 0.f;
             nxt[i].y = cb < ncol ? Nb[idx + cb] : 0.f;
@@ -319,7 +325,8 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
                 const float2 cur = *reinterpret_cast<const float2 *>(&sS[m * SCAN_COLS + ca]);
                 if (!post && SigIn) *reinterpret_cast<float2 *>(SigIn + idx + ca) = cur;
                 if (!post && SigB) *reinterpret_cast<__nv_bfloat162 *>(SigB + idx + ca) = __floats2bfloat162_rn(cur.x, cur.y);
-                if (f + 1 < p.F) nxt[i] = *reinterpret_cast<const float2 *>(Nb + (fhn * DK + m) * (long long)dv + c0 + ca);
+                if (f + 1 < p.F && add_n)
+                    nxt[i] = *reinterpret_cast<const float2 *>(Nb + (fhn * DK + m) * (long long)dv + c0 + ca);
             }
         }
         cp_async_wait_one();  // this frame's M (committed one step earlier) has landed
@@ -366,7 +373,14 @@ __global__ void __launch_bounds__(NT) k3_scan_simt(Problem p, const float *__res
         }
         __syncthreads();
     }
-    if (p.S_out) {
+    if (map) {  // Phi[l][m] = P[m][l] (rows 0 .. d_k - 1), Psi[c][m] = Sig[m][c] (rows d_k ..)
+        for (int e = tid; e < DK * SCAN_COLS; e += NT) {
+            const int m = e >> 4, cc = e & 15;
+            if (cc >= ncol) continue;
+            const int col = c0 + cc, row = col >= dv ? col - dv : DK + col;
+            p.map_out[(chain * (DK + dv) + row) * (long long)DK + m] = sS[e];
+        }
+    } else if (p.S_out) {
         for (int e = tid; e < DK * SCAN_COLS; e += NT) {
             const int m = e >> 4, cc = e & 15;
             if (cc < ncol) p.S_out[(chain * dv + c0 + cc) * (long long)DK + m] = sS[e];
@@ -381,8 +395,9 @@ cudaError_t launch_scan_dk(const Problem &p, const float *Mb, const float *Nb, f
     const size_t sm = sizeof(float) * (2 * DK * DK + DK * SCAN_COLS) + sizeof(float2) * (DK / 16) * 128;
     cudaError_t e = cudaFuncSetAttribute(k3_scan_simt<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e) return e;
-    k3_scan_simt<DK><<<dim3((unsigned)(p.B * p.H), (p.dv + SCAN_COLS - 1) / SCAN_COLS), NT, sm, s>>>(p, Mb, Nb, Sig,
-                                                                                                      SigB);
+    const int ncols_all = p.map_out ? p.dv + DK : p.dv;
+    k3_scan_simt<DK><<<dim3((unsigned)(p.B * p.H), (ncols_all + SCAN_COLS - 1) / SCAN_COLS), NT, sm, s>>>(p, Mb, Nb,
+                                                                                                          Sig, SigB);
     return cudaGetLastError();
 }
 
@@ -631,11 +646,21 @@ cudaError_t launch_typed(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t
     // stages 0, 1 (gates, diagonal inverses) are folded into the intra kernel, 5 (U) into the output
     for (int i = 0; i <= 2; ++i)
         if ((e = mark(ev, i, s))) return e;
-    k1_intra_simt<TIn, TG, float><<<(unsigned)nfh, NT, sm1, s>>>(p, X);
-    if ((e = cudaGetLastError())) return e;
-    if ((e = mark(ev, 3, s))) return e;
-    k2_transition_simt<TIn, TG, float><<<dim3((unsigned)nfh, (dk + 31) / 32), NT, sm2, s>>>(p, X, Mb, Nb);
-    if ((e = cudaGetLastError())) return e;
+    if (p.phase != GDN_PHASE_FINISH) {  // the state-independent stages
+        k1_intra_simt<TIn, TG, float><<<(unsigned)nfh, NT, sm1, s>>>(p, X);
+        if ((e = cudaGetLastError())) return e;
+        if ((e = mark(ev, 3, s))) return e;
+        k2_transition_simt<TIn, TG, float><<<dim3((unsigned)nfh, (dk + 31) / 32), NT, sm2, s>>>(p, X, Mb, Nb);
+        if ((e = cudaGetLastError())) return e;
+        if (p.map_out && (e = simt_segment_map(p, Mb, Nb, s))) return e;
+        if (p.phase == GDN_PHASE_PREPARE) {
+            for (int i = 4; i <= GDN_NUM_STAGES; ++i)
+                if ((e = mark(ev, i, s))) return e;
+            return cudaSuccess;
+        }
+    } else if ((e = mark(ev, 3, s))) {
+        return e;
+    }
     if ((e = mark(ev, 4, s))) return e;
     if ((e = launch_scan(p, Mb, Nb, Sig, nullptr, s))) return e;
     if ((e = cudaGetLastError())) return e;
@@ -691,6 +716,68 @@ cudaError_t simt_transition_bf16x(const Problem &p, const __nv_bfloat16 *X, floa
 cudaError_t simt_scan(const Problem &p, const float *Mb, const float *Nb, float *Sig, __nv_bfloat16 *SigB,
                       cudaStream_t s) {
     return launch_scan(p, Mb, Nb, Sig, SigB, s);
+}
+
+cudaError_t simt_segment_map(const Problem &p, const float *Mb, const float *Nb, cudaStream_t s) {
+    Problem q = p;
+    q.S_in = nullptr;
+    q.S_out = nullptr;
+    return launch_scan(q, Mb, Nb, nullptr, nullptr, s);
+}
+
+namespace {
+
+// S <- S Phi + Psi per (b, h) chain, for each map in turn: S [d_v][d_k] and Phi [d_k][d_k] in
+// shared memory, each thread owning output columns m of a few rows c.
+__global__ void __launch_bounds__(NT) apply_maps_kernel(float *S, const float *maps, int n, int dk, int dv) {
+    extern __shared__ __align__(16) float sm[];
+    float *sS = sm, *sP = sm + dv * dk, *sNew = sP + dk * dk;
+    const long long chain = blockIdx.x;
+    float *Sc = S + chain * (long long)dv * dk;
+    for (int e = threadIdx.x; e < dv * dk; e += NT) sS[e] = Sc[e];
+    for (int j = 0; j < n; ++j) {
+        const float *mp = maps + ((long long)j * gridDim.x + chain) * (long long)(dk + dv) * dk;
+        __syncthreads();
+        for (int e = threadIdx.x; e < dk * dk; e += NT) sP[e] = mp[e];
+        __syncthreads();
+        for (int e = threadIdx.x; e < dv * dk; e += NT) {
+            const int c = e / dk, m = e - c * dk;
+            float acc = mp[(long long)(dk + c) * dk + m];  // Psi[c][m]
+            for (int l = 0; l < dk; ++l) acc = fmaf(sS[c * dk + l], sP[l * dk + m], acc);
+            sNew[e] = acc;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < dv * dk; e += NT) sS[e] = sNew[e];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < dv * dk; e += NT) Sc[e] = sS[e];
+}
+
+}  // namespace
+
+namespace {
+__global__ void identity_map_kernel(float *map, long long n, int dk, int rows) {
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+        const int m = (int)(e % dk), r = (int)((e / dk) % rows);
+        map[e] = (r == m) ? 1.f : 0.f;  // rows r < dk: Phi = I; rows dk ..: Psi = 0
+    }
+}
+}  // namespace
+
+cudaError_t launch_identity_map(float *map, int B, int H, int dk, int dv, cudaStream_t s) {
+    const long long n = (long long)B * H * (dk + dv) * dk;
+    if (n == 0) return cudaSuccess;
+    identity_map_kernel<<<148, 256, 0, s>>>(map, n, dk, dk + dv);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_apply_maps(float *S, const float *maps, int n, int B, int H, int dk, int dv, cudaStream_t s) {
+    const size_t sm = sizeof(float) * (2 * (size_t)dv * dk + (size_t)dk * dk);
+    cudaError_t e = cudaFuncSetAttribute(apply_maps_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e) return e;
+    if ((long long)B * H == 0 || n == 0) return cudaSuccess;
+    apply_maps_kernel<<<(unsigned)((long long)B * H), NT, sm, s>>>(S, maps, n, dk, dv);
+    return cudaGetLastError();
 }
 
 cudaError_t simt_u_bf16x(const Problem &p, const __nv_bfloat16 *X, const float *Sig, __nv_bfloat16 *U,

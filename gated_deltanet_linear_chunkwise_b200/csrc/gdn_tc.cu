@@ -6,7 +6,8 @@
 //   inverse     T_ii = (I + A_ii)^{-1} per 128-row diagonal block (mma.sync)
 //   intra       [Ub | W] per frame-head, bf16, blocked forward substitution (tcgen05)
 //   transition  M, N per frame-head, fp32                 (tcgen05)
-//   scan        entering state per frame, fp32 + bf16     (CUDA cores)
+//   scan        entering state per frame, bf16             (tcgen05; CUDA cores where its
+//                                                          shared memory does not fit)
 //   output      U = Ub - W Sig (bf16, tcgen05), then the tcgen05 output kernel
 #include <cstdlib>
 #include <mutex>
@@ -25,7 +26,7 @@ namespace {
 inline int cf_stride(int L) { return (L + 3) & ~3; }
 
 struct TcLayout {
-    size_t G, CF, GCT, Tinv, X, M, N, Sig, SigB, U, err;
+    size_t G, CF, GCT, Tinv, X, M, Mimg, N, Sig, SigB, U, err;
     size_t Otmp, Qr, Kr, Vr, Ar, Br;  // reversed / accumulating calls only (0 bytes otherwise)
     size_t total;
 };
@@ -40,9 +41,12 @@ TcLayout tc_layout(const Problem &p) {
     lay.GCT = off;  off += align256(sizeof(float) * nfh * (size_t)((p.L + 127) / 128) * 256);
     lay.Tinv = off; off += align256(2 * nfh * (size_t)((p.L + 127) / 128) * 128 * 128);
     lay.X = off;    off += align256(2 * nfh * p.L * nc);
-    lay.M = off;    off += align256(sizeof(float) * nfh * p.dk * p.dk);
+    // the scan takes M as the tensor-core scan's operand images (or fp32 for the CUDA-core one)
+    const bool scan_tc = tc::scan_tc_supported(p.dk, p.dv);
+    lay.M = off;    off += align256(sizeof(float) * nfh * p.dk * p.dk);  // CUDA-core scan, segment maps
+    lay.Mimg = off; off += scan_tc ? align256(nfh * tc::scan_mimg_bytes(p.dk)) : 0;
     lay.N = off;    off += align256(sizeof(float) * nfh * p.dk * p.dv);
-    lay.Sig = off;  off += align256(sizeof(float) * nfh * p.dk * p.dv);
+    lay.Sig = off;  off += scan_tc ? 0 : align256(sizeof(float) * nfh * p.dk * p.dv);
     lay.SigB = off; off += align256(2 * nfh * p.dk * p.dv);
     lay.U = off;    off += align256(2 * nfh * p.L * p.dv);
     lay.err = off;  off += 256;
@@ -156,6 +160,8 @@ bool tc_disabled_by_env() {
 
 }  // namespace
 
+bool tc_fuses_qk_prologue(const Problem &p) { return tc_supports(p) && p.mode == GDN_MODE_FRAME; }
+
 bool tc_supports(const Problem &p) {
     static const bool disabled = tc_disabled_by_env();
     return !disabled && p.dtype == GDN_DTYPE_BF16;
@@ -194,6 +200,17 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
         !map_f32_rows(&tm_cf128, CF, nfh, p.L, cf_stride(p.L), 128))
         return cudaErrorInvalidValue;
 
+    int dev = 0, num_sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    const uint64_t wait_ns = wait_limit_ns();
+    const bool scan_tc = tc::scan_tc_supported(p.dk, p.dv);
+    __nv_bfloat16 *Mimg = (__nv_bfloat16 *)(base + lay.Mimg);
+    if (p.phase == GDN_PHASE_FINISH) {  // the state-independent stages ran in a PREPARE call
+        for (int i = 0; i <= 4; ++i)
+            if ((e = mark(ev, i, s))) return e;
+        goto finish;
+    }
+    {
     if ((e = cudaMemsetAsync(err, 0, sizeof(int), s))) return e;
     const size_t gsm = sizeof(float) * (2 * p.L + 32);
     if (gsm > 48 * 1024 &&
@@ -203,8 +220,8 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF, GCT);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 1, s))) return e;
-    if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
-                                     nfh, err, s)))
+    if ((e = tc::launch_diag_inverse(tm_k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T, nfh, err, wait_ns,
+                                     debug_drop_signal(), num_sms, s)))
         return e;
     if ((e = mark(ev, 2, s))) return e;
     tc::IntraParams ip;
@@ -214,19 +231,34 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     if ((e = tc::launch_intra_tc(tm_k, tm_x, tm_t, tm_gct, tm_x128, ip, nfh, s))) return e;
     if ((e = mark(ev, 3, s))) return e;
     tc::TransParams tp;
-    tp.G = G; tp.M = Mb; tp.N = Nb;
+    // fp32 M for the CUDA-core scan (also the segment-map scan); the operand images for the tensor-core one
+    tp.G = G; tp.M = (!scan_tc || p.map_out) ? Mb : nullptr; tp.Mimg = scan_tc ? Mimg : nullptr; tp.N = Nb;
     tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
     tp.frame = 0; tp.beta = p.beta; tp.gamma = nullptr; tp.T = p.T;
+    tp.norm_k = 0; tp.k_w = nullptr; tp.k_post = 1.f;
     if ((e = tc::launch_transition_tc(tm_k64, tm_x, tm_x, tp, nfh, s))) return e;
+    if (p.map_out && (e = simt_segment_map(p, Mb, Nb, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
+    if (p.phase == GDN_PHASE_PREPARE) {
+        for (int i = 5; i <= GDN_NUM_STAGES; ++i)
+            if ((e = mark(ev, i, s))) return e;
+        return cudaSuccess;
+    }
+    }
+finish:
     Problem ps = p;
     ps.reverse = scan_reverse;
-    if ((e = simt_scan(ps, Mb, Nb, Sig, SigB, s))) return e;
+    if (scan_tc) {
+        if ((e = tc::launch_scan_tc(ps, Mimg, Nb, SigB, nullptr, err, wait_limit_ns(), s))) return e;
+    } else if ((e = simt_scan(ps, Mb, Nb, Sig, SigB, s))) {
+        return e;
+    }
     if ((e = mark(ev, 5, s))) return e;
     tc::UParams up;
     up.X = X; up.U = U;
     up.L = p.L; up.dk = p.dk; up.dv = p.dv; up.nblk = nblk; up.err = err;
     up.frame = 0; up.o = nullptr; up.T = p.T; up.F = p.F; up.H = p.H; up.accumulate = 0;
+    up.norm_q = 0; up.q_w = nullptr;
     if ((e = tc::launch_u_tc(tm_x128, tm_q, tm_sig, up, nfh, s))) return e;
     if ((e = mark(ev, 6, s))) return e;
 
@@ -238,46 +270,55 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     op.F = p.F; op.T = p.T; op.n_fh = nfh;
     op.accumulate = p.accumulate;
     op.err = err;
-    int dev = 0, num_sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u128, tm_sig, tm_g128, tm_cf128, op, num_sms, s))) return e;
     return mark(ev, 7, s);
 }
 
 namespace {
 
-// dst row (b, T-1-t) = src row (b, t) for rows of `row_words` 32-bit words ([B, T, ...] tensors).
-__global__ void reverse_rows_kernel(const uint32_t *__restrict__ src, uint32_t *__restrict__ dst, int B,
-                                    long long T, int row_words) {
-    const long long total = (long long)B * T * row_words;
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-         e += (long long)gridDim.x * blockDim.x) {
-        const long long w = e % row_words, row = e / row_words, t = row % T, b = row / T;
-        dst[(b * T + (T - 1 - t)) * row_words + w] = src[e];
-    }
+// dst row (b, T-1-t) = src row (b, t) of a [B, T, ...] tensor, one warp per row, 16-byte
+// pieces when the row length allows (else 4-byte words); bandwidth bound.
+template <typename V>
+__global__ void __launch_bounds__(256) reverse_rows_kernel(const V *__restrict__ src, V *__restrict__ dst,
+                                                           long long rows, long long T, int row_vecs) {
+    const long long row = blockIdx.x * 8ll + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const long long t = row % T, b = row / T;
+    const V *s = src + row * row_vecs;
+    V *d = dst + (b * T + (T - 1 - t)) * row_vecs;
+    for (int i = threadIdx.x & 31; i < row_vecs; i += 32) d[i] = s[i];
 }
 
-// o (+)= the staged result, rows taken in reverse token order for a reversed scan; the sum
-// of an accumulating call is formed in fp32 and rounded once to bf16.
-__global__ void finish_o_kernel(const __nv_bfloat162 *__restrict__ tmp, __nv_bfloat162 *__restrict__ o, int B,
-                                long long T, int row_pairs, int reverse, int accumulate) {
-    const long long total = (long long)B * T * row_pairs;
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-         e += (long long)gridDim.x * blockDim.x) {
-        const long long w = e % row_pairs, row = e / row_pairs, t = row % T, b = row / T;
-        const long long src = reverse ? (b * T + (T - 1 - t)) * row_pairs + w : e;
-        float2 v = __bfloat1622float2(tmp[src]);
+// o (+)= the staged result, rows taken in reverse token order for a reversed scan, one warp
+// per row; the sum of an accumulating call is formed in fp32 and rounded once to bf16.
+__global__ void __launch_bounds__(256) finish_o_kernel(const __nv_bfloat162 *__restrict__ tmp,
+                                                       __nv_bfloat162 *__restrict__ o, long long rows, long long T,
+                                                       int row_pairs, int reverse, int accumulate) {
+    const long long row = blockIdx.x * 8ll + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const long long t = row % T, b = row / T;
+    const __nv_bfloat162 *s = tmp + (reverse ? (b * T + (T - 1 - t)) : row) * row_pairs;
+    __nv_bfloat162 *d = o + row * row_pairs;
+    for (int i = threadIdx.x & 31; i < row_pairs; i += 32) {
+        float2 v = __bfloat1622float2(s[i]);
         if (accumulate) {
-            const float2 old = __bfloat1622float2(o[e]);
+            const float2 old = __bfloat1622float2(d[i]);
             v.x += old.x;
             v.y += old.y;
         }
-        o[e] = __floats2bfloat162_rn(v.x, v.y);
+        d[i] = __floats2bfloat162_rn(v.x, v.y);
     }
 }
 
 cudaError_t reverse_rows(const void *src, void *dst, int B, long long T, size_t row_bytes, cudaStream_t s) {
-    reverse_rows_kernel<<<1184, 256, 0, s>>>((const uint32_t *)src, (uint32_t *)dst, B, T, (int)(row_bytes / 4));
+    const long long rows = (long long)B * T;
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+    if (rows == 0) return cudaSuccess;
+    if (row_bytes % 16 == 0 && ((uintptr_t)src | (uintptr_t)dst) % 16 == 0)
+        reverse_rows_kernel<uint4><<<grid, 256, 0, s>>>((const uint4 *)src, (uint4 *)dst, rows, T, (int)(row_bytes / 16));
+    else
+        reverse_rows_kernel<uint32_t><<<grid, 256, 0, s>>>((const uint32_t *)src, (uint32_t *)dst, rows, T,
+                                                           (int)(row_bytes / 4));
     return cudaGetLastError();
 }
 
@@ -295,6 +336,8 @@ cudaError_t launch_tc_frame(const Problem &p, void *ws, cudaStream_t s, cudaEven
     const long long nfh = (long long)p.B * p.H * p.F;
     const int nblk = (p.L + tc::BM - 1) / tc::BM;
     float *Mb = (float *)(base + lay.M), *Nb = (float *)(base + lay.N);
+    __nv_bfloat16 *Mimg = (__nv_bfloat16 *)(base + lay.Mimg);
+    const bool scan_tc = tc::scan_tc_supported(p.dk, p.dv);
     __nv_bfloat16 *SigB = (__nv_bfloat16 *)(base + lay.SigB);
     int *err = (int *)(base + lay.err);
     cudaError_t e;
@@ -307,17 +350,27 @@ cudaError_t launch_tc_frame(const Problem &p, void *ws, cudaStream_t s, cudaEven
     for (int i = 0; i <= 3; ++i)
         if ((e = mark(ev, i, s))) return e;
     tc::TransParams tp;
-    tp.G = nullptr; tp.M = Mb; tp.N = Nb;
+    tp.G = nullptr; tp.M = scan_tc ? nullptr : Mb; tp.Mimg = scan_tc ? Mimg : nullptr; tp.N = Nb;
     tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
     tp.frame = 1; tp.beta = p.beta; tp.gamma = p.gamma; tp.T = p.T;
+    // the q/k feature maps, when requested, are applied to the staged tiles (no copy pass)
+    tp.norm_k = (p.qk_norm & GDN_QK_NORM_KEYS) ? 1 : 0;
+    tp.k_w = p.k_norm_weight;
+    tp.k_post = 1.f / sqrtf((float)p.dk * (float)p.L);
     if ((e = tc::launch_transition_tc(tm_k64, tm_k64, tm_v64, tp, nfh, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
-    if ((e = simt_scan(p, Mb, Nb, nullptr, SigB, s))) return e;
+    if (scan_tc) {
+        if ((e = tc::launch_scan_tc(p, Mimg, Nb, SigB, nullptr, err, wait_limit_ns(), s))) return e;
+    } else if ((e = simt_scan(p, Mb, Nb, nullptr, SigB, s))) {
+        return e;
+    }
     if ((e = mark(ev, 5, s)) || (e = mark(ev, 6, s))) return e;
     tc::UParams up;
     up.X = nullptr; up.U = nullptr;
     up.L = p.L; up.dk = p.dk; up.dv = p.dv; up.nblk = nblk; up.err = err;
     up.frame = 1; up.o = (__nv_bfloat16 *)p.o; up.T = p.T; up.F = p.F; up.H = p.H; up.accumulate = p.accumulate;
+    up.norm_q = (p.qk_norm & GDN_QK_NORM_QUERIES) ? 1 : 0;
+    up.q_w = p.q_norm_weight;
     if ((e = tc::launch_u_tc(tm_q, tm_q, tm_sig, up, nfh, s))) return e;
     return mark(ev, 7, s);
 }
@@ -346,8 +399,11 @@ cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *e
         q.beta = (const float *)(base + lay.Br);
     }
     if ((e = launch_tc_forward(q, ws, p.reverse, s, ev))) return e;
-    finish_o_kernel<<<1184, 256, 0, s>>>((const __nv_bfloat162 *)(base + lay.Otmp), (__nv_bfloat162 *)p.o, p.B, p.T,
-                                         p.H * p.dv / 2, p.reverse, p.accumulate);
+    const long long rows = (long long)p.B * p.T;
+    if (rows > 0)
+        finish_o_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const __nv_bfloat162 *)(base + lay.Otmp),
+                                                                  (__nv_bfloat162 *)p.o, rows, p.T, p.H * p.dv / 2,
+                                                                  p.reverse, p.accumulate);
     return cudaGetLastError();
 }
 

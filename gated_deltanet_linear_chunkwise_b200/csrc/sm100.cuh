@@ -71,16 +71,21 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, records kErrTimeout in *err and returns false; every caller
-// then leaves its loop so the kernel can release TMEM and exit.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err) {
+// limit_ns (kWaitLimitNs unless a launch passes a shorter, test-only limit),
+// records kErrTimeout in *err and returns false; every caller then leaves its
+// loop so the kernel can release TMEM and exit.  A `drain` wait is the one a
+// thread makes on its own copies or products in flight before it leaves: it
+// ignores the error word (which is already set then) and gives up only at
+// limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err,
+                                          uint64_t limit_ns = kWaitLimitNs, bool drain = false) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 255u) {
-            if (*(volatile int *)err != kErrNone) return false;  // someone else gave up
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (!drain && *(volatile int *)err != kErrNone) return false;  // someone else gave up
+            if (globaltimer_ns() - t0 > limit_ns) {
                 atomicCAS(err, kErrNone, kErrTimeout);
                 return false;
             }
@@ -94,12 +99,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
 struct Spin {
     uint32_t it = 0;
     uint64_t t0 = 0;
+    uint64_t limit_ns = kWaitLimitNs;
+    __device__ __forceinline__ Spin() {}
+    __device__ __forceinline__ explicit Spin(uint64_t limit) : limit_ns(limit) {}
     __device__ __forceinline__ void reset() { it = 0; }
     __device__ __forceinline__ bool tick(int *err) {
         if (it == 0) t0 = globaltimer_ns();
         if ((++it & 255u) == 0) {
             if (*(volatile int *)err != kErrNone) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 atomicCAS(err, kErrNone, kErrTimeout);
                 return false;
             }
@@ -136,6 +144,54 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const void *tmap, ui
         "[%2];" ::"r"(smem_u32(smem_dst)),
         "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
+}
+
+// L2 eviction policies for the copies' cache hints: data read once goes first,
+// tiles that later blocks of the same frame read again stay longest.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void tma_load_3d_hint(void *smem_dst, const void *tmap, uint64_t *bar, int c0, int c1,
+                                                 int c2, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+        "%4, %5}], [%2], %6;" ::"r"(smem_u32(smem_dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d_hint(void *smem_dst, const void *tmap, uint64_t *bar, int c0, int c1,
+                                                 int c2, int c3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+        "%4, %5, %6}], [%2], %7;" ::"r"(smem_u32(smem_dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d_hint(const void *tmap, const void *smem_src, int c0, int c1, int c2,
+                                                  uint64_t policy) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;" ::"l"(
+                     tmap),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+                 : "memory");
+}
+
+// 16-byte read-only load with an L2 eviction policy (data a kernel reads once).
+__device__ __forceinline__ uint4 ld_nc_hint(const void *p, uint64_t policy) {
+    uint4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(policy));
+    return v;
 }
 
 // Shared -> global tiled store (out-of-range rows and columns are not written).

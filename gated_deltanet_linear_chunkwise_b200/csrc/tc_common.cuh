@@ -24,6 +24,32 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// The same barrier, returning the AND of every participant's `ok`: threads that each
+// made a bounded wait take one common decision to go on or to leave, so no thread is
+// left waiting at a later barrier for one that left.
+__device__ __forceinline__ bool named_sync_and(int id, int nthreads, bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+// A kernel of a pass whose earlier stage recorded a failure in the error word does
+// nothing: every thread learns it before any barrier is armed or TMEM allocated, so a
+// pass that gave up leaves no copy or product in flight behind it.
+__device__ __forceinline__ bool pass_failed(const int *err) {
+    __shared__ int s_failed;
+    if (threadIdx.x == 0) s_failed = *(volatile const int *)err;
+    __syncthreads();
+    return s_failed != 0;
+}
+
 // K-major SW128 operand: tile of `rows` rows, 64-column slabs; K step ks (16 columns).
 __device__ __forceinline__ uint64_t desc_kmajor(const void *tile, int ks, int rows) {
     const uint32_t a = sm100::smem_u32(tile) + (uint32_t)((ks >> 2) * rows * 128 + (ks & 3) * 32);
@@ -61,7 +87,9 @@ struct IntraParams {
 
 struct TransParams {
     const float *G;            // [n_fh][(L+3)&~3]
-    float *M;                  // [n_fh][dk][dk]
+    float *M;                  // [n_fh][dk][dk] fp32, or null
+    __nv_bfloat16 *Mimg;       // or null: M split into bf16 hi + lo, each in the 128-byte-swizzled
+                               // K-major image of 64-column slabs of dk rows (the scan's A operand)
     float *N;                  // [n_fh][dk][dv]
     int L, dk, dv, H, nblk;
     long long F;
@@ -72,6 +100,11 @@ struct TransParams {
     const float *beta;         // [B,T,H]
     const float *gamma;        // [B,F,H]
     long long T;
+    // frame-wise operator: the key feature map applied to the staged K rows (both copies)
+    // before the products, K <- max(RMSNorm(K) * w, 0) * k_post; 0: keys used as given
+    int norm_k;
+    const float *k_w;          // [dk] RMSNorm weight or null (ones)
+    float k_post;              // 1 / sqrt(dk * L)
 };
 
 struct UParams {
@@ -84,7 +117,14 @@ struct UParams {
     __nv_bfloat16 *o;          // [B,T,H,dv]
     long long T, F;
     int H, accumulate;
+    // frame-wise operator: the query feature map applied to the staged Q rows before the
+    // product, Q <- max(RMSNorm(Q) * w, 0); 0: queries used as given
+    int norm_q;
+    const float *q_w;          // [dk] RMSNorm weight or null (ones)
 };
+
+// RMSNorm epsilon of the q/k feature maps (the pages give none; 1e-6).
+constexpr float kRmsEps = 1e-6f;
 
 // tm_k / tm_x / tm_v deliver 64-token boxes (tm_x the [Ub | W] rows, tm_v the
 // values, read by the frame-wise operator only).
@@ -102,11 +142,20 @@ cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x64, 
                             const CUtensorMap &tm_gct, const CUtensorMap &tm_xs, const IntraParams &prm,
                             long long n_fh, cudaStream_t s);
 
-cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
+// tm_k delivers 128-token boxes of k (the Gram's operand).  Persistent: at most num_sms CTAs.
+cudaError_t launch_diag_inverse(const CUtensorMap &tm_k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
                                 int L, int dk, int H, int nblk, long long F, long long T, long long n_fh,
-                                int *err, cudaStream_t s);
+                                int *err, uint64_t wait_ns, int drop_first_load, int num_sms, cudaStream_t s);
 
 // tm_q / tm_k / tm_u / tm_g / tm_cf deliver 128-token boxes.
+// The scan over frames on the tensor cores (tc_scan.cu): M from the transition
+// kernel's images, N fp32; writes the bf16 (and optionally fp32) state of every
+// frame and S_out.  scan_tc_supported: whether its shared memory fits these dims.
+bool scan_tc_supported(int dk, int dv);
+size_t scan_mimg_bytes(int dk);
+cudaError_t launch_scan_tc(const Problem &p, const __nv_bfloat16 *Mimg, const float *Nb, __nv_bfloat16 *SigB,
+                           float *SigF, int *err, uint64_t wait_ns, cudaStream_t s);
+
 cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
                              const CUtensorMap &tm_sig, const CUtensorMap &tm_g, const CUtensorMap &tm_cf,
                              const OutParams &prm, int num_sms, cudaStream_t s);

@@ -90,6 +90,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *err = prm.err;
 
+    if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) {
             uint32_t cnt = 1;
@@ -127,6 +128,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::tma_prefetch_desc(&tm_t);
             sm100::tma_prefetch_desc(&tm_gct);
             sm100::tma_prefetch_desc(&tm_xs);
+            // L2 policies: K and X tiles are read again by the frame's later blocks, T_ii once
+            const uint64_t keep = sm100::policy_evict_last(), once = sm100::policy_evict_first();
             int ki = 0;              // next K_i block
             int kb = 0, kc = 0;      // next K-ring item: block kb, item kc (kc == kb: T_kb)
             int xb = 1, xx = 0;      // next X-ring item: block xb, X tile xx
@@ -140,7 +143,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 if (ki < nblk && (ki == 0 || sm100::mbar_test(&bars[KIEMPTY], (ki - 1) & 1))) {
                     sm100::mbar_arrive_expect_tx(&bars[KIFULL], (uint32_t)(nslab_k * SLAB_BYTES));
                     for (int sl = 0; sl < nslab_k; ++sl)
-                        sm100::tma_load_4d(sKi + sl * SLAB_BYTES, &tm_k, &bars[KIFULL], sl * SLAB, h, ki * BM, bf);
+                        sm100::tma_load_4d_hint(sKi + sl * SLAB_BYTES, &tm_k, &bars[KIFULL], sl * SLAB, h, ki * BM, bf,
+                                                keep);
                     ++ki;
                     prog = true;
                 }
@@ -153,15 +157,15 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                             sm100::mbar_arrive_expect_tx(&bars[KRFULL + st],
                                                          (uint32_t)(nslab_k * SLAB_BYTES + GCT_FLOATS * 4));
                             for (int sl = 0; sl < nslab_k; ++sl)
-                                sm100::tma_load_4d(slot + sl * SLAB_BYTES, &tm_k, &bars[KRFULL + st], sl * SLAB, h,
-                                                   kc * CT, bf);
+                                sm100::tma_load_4d_hint(slot + sl * SLAB_BYTES, &tm_k, &bars[KRFULL + st], sl * SLAB, h,
+                                                        kc * CT, bf, keep);
                             sm100::tma_load_2d(sGC + st * GCT_FLOATS, &tm_gct, &bars[KRFULL + st], 0,
                                                (int)(fh * nt128 + kc));
                         } else {
                             sm100::mbar_arrive_expect_tx(&bars[KRFULL + st], (uint32_t)(2 * SLAB_BYTES));
                             for (int sl = 0; sl < 2; ++sl)
-                                sm100::tma_load_3d(slot + sl * SLAB_BYTES, &tm_t, &bars[KRFULL + st], sl * SLAB, 0,
-                                                   (int)(fh * nblk + kb));
+                                sm100::tma_load_3d_hint(slot + sl * SLAB_BYTES, &tm_t, &bars[KRFULL + st], sl * SLAB, 0,
+                                                        (int)(fh * nblk + kb), once);
                         }
                         ++kn;
                         if (++kc > kb) {
@@ -175,7 +179,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 // X ring may refill the first two slots (which hold Y / X) once the store has read them
                 if (sxb < nblk && sm100::mbar_test(&bars[XSTAGED], sxb & 1)) {
                     for (int sl = 0; sl < nslab_x; ++sl)
-                        sm100::tma_store_3d(&tm_xs, sYX + sl * SLAB_BYTES, sl * SLAB, sxb * BM, (int)fh);
+                        sm100::tma_store_3d_hint(&tm_xs, sYX + sl * SLAB_BYTES, sl * SLAB, sxb * BM, (int)fh, keep);
                     sm100::bulk_commit();
                     sm100::bulk_wait_read0();
                     ++sxb;
@@ -189,8 +193,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                         unsigned char *slot = sXR + st * XSLOT;
                         sm100::mbar_arrive_expect_tx(&bars[XRFULL + st], (uint32_t)(nslab_x * XSLAB));
                         for (int sl = 0; sl < nslab_x; ++sl)
-                            sm100::tma_load_3d(slot + sl * XSLAB, &tm_x64, &bars[XRFULL + st], sl * SLAB, xx * XT,
-                                               (int)fh);
+                            sm100::tma_load_3d_hint(slot + sl * XSLAB, &tm_x64, &bars[XRFULL + st], sl * SLAB, xx * XT,
+                                                    (int)fh, keep);
                         ++xn;
                         if (++xx == 2 * xb) {
                             ++xb;
@@ -368,10 +372,11 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 *reinterpret_cast<uint4 *>(sYX + yx_offset(c, r)) = val;
             };
             if (half == 0) {  // Ub columns: beta_r v_r + acc
+                const uint64_t once = sm100::policy_evict_first();  // v is read once: keep K and X in L2
                 uint4 vrow[16];
 #pragma unroll
                 for (int c8 = 0; c8 < 16; ++c8)
-                    vrow[c8] = (valid && c8 < dv / 8) ? __ldg(reinterpret_cast<const uint4 *>(vp) + c8)
+                    vrow[c8] = (valid && c8 < dv / 8) ? sm100::ld_nc_hint(reinterpret_cast<const uint4 *>(vp) + c8, once)
                                                       : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int j2 = 0; j2 < 4; ++j2) {  // two 16-column loads per wait

@@ -79,6 +79,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *err = prm.err;
 
+    if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) {
             const bool epi = (i >= PFULL && i < PFULL + NSB) || (i >= OEMPTY && i < OEMPTY + 2);
@@ -127,6 +128,8 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             sm100::tma_prefetch_desc(&tm_sig);
             sm100::tma_prefetch_desc(&tm_g);
             sm100::tma_prefetch_desc(&tm_cf);
+            // L2 policies: a frame's K and U tiles are read again by its other blocks, Q once
+            const uint64_t keep = sm100::policy_evict_last(), once = sm100::policy_evict_first();
             bool ok = true;
             int n = 0, t = 0;
             for (long long w = w_begin; w < w_end && ok; ++w, ++t) {
@@ -140,8 +143,8 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 if (!ok) break;
                 sm100::mbar_arrive_expect_tx(&bars[QFULL + qb], (uint32_t)(nslab_k * SLAB_BYTES));
                 for (int sl = 0; sl < nslab_k; ++sl)
-                    sm100::tma_load_4d(sQ + (qb * 2 + sl) * SLAB_BYTES, &tm_q, &bars[QFULL + qb], sl * SLAB, h,
-                                       I * BM, bf);
+                    sm100::tma_load_4d_hint(sQ + (qb * 2 + sl) * SLAB_BYTES, &tm_q, &bars[QFULL + qb], sl * SLAB, h,
+                                            I * BM, bf, once);
                 const int nt = item_ntiles(I);
                 for (int j = -1; j < nt && ok; ++j, ++n) {
                     const int st = n % NSLOT;
@@ -156,10 +159,11 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         sm100::mbar_arrive_expect_tx(&bars[RFULL + st],
                                                      (uint32_t)((nslab_k + nslab_v) * JSLAB + GC_BYTES));
                         for (int sl = 0; sl < nslab_k; ++sl)
-                            sm100::tma_load_4d(slot + sl * JSLAB, &tm_k, &bars[RFULL + st], sl * SLAB, h, j * JT, bf);
+                            sm100::tma_load_4d_hint(slot + sl * JSLAB, &tm_k, &bars[RFULL + st], sl * SLAB, h, j * JT, bf,
+                                                    keep);
                         for (int sl = 0; sl < nslab_v; ++sl)
-                            sm100::tma_load_3d(slot + (2 + sl) * JSLAB, &tm_u, &bars[RFULL + st], sl * SLAB, j * JT,
-                                               (int)fh);
+                            sm100::tma_load_3d_hint(slot + (2 + sl) * JSLAB, &tm_u, &bars[RFULL + st], sl * SLAB, j * JT,
+                                                    (int)fh, keep);
                         float *gc = sGC + st * 2 * JT;
                         sm100::tma_load_2d(gc, &tm_g, &bars[RFULL + st], j * JT, (int)fh);
                         sm100::tma_load_2d(gc + JT, &tm_cf, &bars[RFULL + st], j * JT, (int)fh);

@@ -62,6 +62,7 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int ncols = frame ? SLAB * nslab_x : nc;
     const int mcol0 = frame ? SLAB * nslab_v : dv;  // first column of the M part
 
+    if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) sm100::mbar_init(&bars[i], (i >= SCALED && i < SCALED + NST) ? 128 : 1);
         sm100::fence_barrier_init();
@@ -129,14 +130,63 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         bool ok = true;
         // thread r scales row r % 64 of the chunk's K, slab r / 64
         const int row_in = r & (CH - 1), sl = r >> 6;
+        float *sSS = reinterpret_cast<float *>(bars + NBAR + 1);  // [2][64] partial sums of squares
+        const bool normk = frame && prm.norm_k;
         for (int c = 0; c < nch && ok; ++c) {
             const int st = c % NST;
             const int row = c * CH + row_in;
             float sc = 0.f;  // the K row's factor: e^{G_L - G_r}, or beta_r for the frame-wise map
             if (row < L) sc = frame ? prm.beta[((long long)b * prm.T + f * L + row) * prm.H + h] : __expf(GL - Gf[row]);
             ok = sm100::mbar_wait(&bars[FULL + st], (c / NST) & 1, err);
+            if (normk) ok = named_sync_and(1, 128, ok);  // the row's two halves meet below
             if (!ok) break;
-            if (sl < nslab_k) {
+            if (normk) {
+                // key feature map of the frame-wise operator (SANA-WM summary, section 3.2,
+                // "Algebraic Stabilization for Spatial Token Explosion"): y = max(RMSNorm(k) w, 0)
+                // / sqrt(d_k S); the row's mean square is summed over both 64-column halves
+                uint4 *rowp = reinterpret_cast<uint4 *>(sRing + st * STAGE + sl * CSLAB + row_in * 128);
+                float ss = 0.f;
+                if (sl < nslab_k) {
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        const uint4 v = rowp[cc];
+                        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 x = __bfloat1622float2(p2[e]);
+                            ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
+                        }
+                    }
+                }
+                sSS[sl * CH + row_in] = ss;
+                named_sync(1, 128);
+                const float inv = 1.f / sqrtf((sSS[row_in] + sSS[CH + row_in]) / (float)dk + kRmsEps);
+                named_sync(1, 128);  // both halves read before the next chunk writes sSS
+                if (sl < nslab_k) {
+                    uint4 *rowb = reinterpret_cast<uint4 *>(sRing + st * STAGE + (2 + nslab_v + sl) * CSLAB +
+                                                            row_in * 128);
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint4 v = rowp[cc], vb;
+                        __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&v);
+                        __nv_bfloat162 *b2 = reinterpret_cast<__nv_bfloat162 *>(&vb);
+                        const int c0 = sl * 64 + ((cc ^ (row_in & 7)) << 3);  // logical column of the chunk
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 x = __bfloat1622float2(p2[e]);
+                            const int ca = c0 + 2 * e;
+                            const float wa = (prm.k_w && ca < dk) ? prm.k_w[ca] : 1.f;
+                            const float wb = (prm.k_w && ca + 1 < dk) ? prm.k_w[ca + 1] : 1.f;
+                            const float ya = fmaxf(x.x * inv * wa, 0.f) * prm.k_post;
+                            const float yb = fmaxf(x.y * inv * wb, 0.f) * prm.k_post;
+                            b2[e] = __floats2bfloat162_rn(ya, yb);            // K (the B operand's copy)
+                            p2[e] = __floats2bfloat162_rn(sc * ya, sc * yb);  // beta K (the A operand)
+                        }
+                        rowp[cc] = v;
+                        rowb[cc] = vb;
+                    }
+                }
+            } else if (sl < nslab_k) {
                 uint4 *rowp = reinterpret_cast<uint4 *>(sRing + st * STAGE + sl * CSLAB + row_in * 128);
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
@@ -179,6 +229,28 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         const int j0 = c0 - mcol0;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = (m == j0 + e ? eGL : 0.f) - gam * v[e];
+                        if (prm.Mimg) {  // hi + lo bf16 images of the scan's A operand
+                            const int nslab = (dk + SLAB - 1) / SLAB;
+                            unsigned char *img = reinterpret_cast<unsigned char *>(prm.Mimg) +
+                                                 fh * (long long)(2 * nslab * dk * 128);
+#pragma unroll
+                            for (int h8 = 0; h8 < 2; ++h8) {
+                                uint32_t hi[4], lo[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float a = v[8 * h8 + 2 * e], bb = v[8 * h8 + 2 * e + 1];
+                                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
+                                    const float2 hf = __bfloat1622float2(h2);
+                                    hi[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                                    lo[e] = pack_bf16(a - hf.x, bb - hf.y);
+                                }
+                                const uint32_t off = sm100::sw128_kmajor_offset(m, j0 + 8 * h8, dk);
+                                *reinterpret_cast<uint4 *>(img + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                                *reinterpret_cast<uint4 *>(img + nslab * dk * 128 + off) =
+                                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                            }
+                        }
+                        if (!prm.M) continue;
                         dst = prm.M + (fh * dk + m) * (long long)dk + j0;
                     } else {
                         continue;
@@ -202,7 +274,7 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_v,
                                  const TransParams &prm, long long n_fh, cudaStream_t s) {
-    const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
+    const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16 + 2 * CH * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(k_transition_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k_transition_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_v, prm);

@@ -26,7 +26,7 @@ struct Smem {
     static constexpr uint32_t END = W + 4 * SLAB_BYTES;
 };
 
-enum Bar { SIGFULL, WFULL0, WFULL1, WEMPTY0, WEMPTY1, DFULL0, DFULL1, DEMPTY0, DEMPTY1, NBAR };
+enum Bar { SIGFULL, WFULL0, WFULL1, WEMPTY0, WEMPTY1, DFULL0, DFULL1, DEMPTY0, DEMPTY1, QREADY0, QREADY1, NBAR };
 
 __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
 k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
@@ -43,11 +43,14 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
     int *err = prm.err;
     const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
     const bool frame = prm.frame != 0;
+    const bool normq = frame && prm.norm_q;
     const long long f = frame ? fh % prm.F : 0, chain = frame ? fh / prm.F : 0;
     const int h = frame ? (int)(chain % prm.H) : 0, b = frame ? (int)(chain / prm.H) : 0;
 
+    if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NBAR; ++i) sm100::mbar_init(&bars[i], (i == DEMPTY0 || i == DEMPTY1) ? 128 : 1);
+        for (int i = 0; i < NBAR; ++i)
+            sm100::mbar_init(&bars[i], (i == DEMPTY0 || i == DEMPTY1 || i == QREADY0 || i == QREADY1) ? 128 : 1);
         sm100::fence_barrier_init();
     }
     if (warp == 1) {
@@ -90,7 +93,9 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
             bool ok = sm100::mbar_wait(&bars[SIGFULL], 0, err);
             for (int i = 0; i < nblk && ok; ++i) {
                 const int st = i & 1;
-                ok = sm100::mbar_wait(&bars[WFULL0 + st], (i >> 1) & 1, err);
+                // the operand is ready when it has landed, or (query feature map) once the
+                // epilogue has normalised it in place
+                ok = sm100::mbar_wait(&bars[(normq ? QREADY0 : WFULL0) + st], (i >> 1) & 1, err);
                 if (ok && i >= 2) ok = sm100::mbar_wait(&bars[DEMPTY0 + st], ((i - 2) >> 1) & 1, err);
                 if (!ok) break;
                 sm100::tc_fence_after();
@@ -107,7 +112,52 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
         const int r = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         bool ok = true;
+        // query feature map of the frame-wise operator (SANA-WM summary, section 3.2, "Algebraic
+        // Stabilization for Spatial Token Explosion"): row r of block i's staged Q becomes
+        // max(RMSNorm(q) w, 0) in place before the product reads it
+        auto normalize = [&](int i) -> bool {
+            const int st = i & 1;
+            if (!sm100::mbar_wait(&bars[WFULL0 + st], (i >> 1) & 1, err)) return false;
+            float ss = 0.f;
+            for (int sl = 0; sl < nslab_k; ++sl) {
+                const uint4 *rowp = reinterpret_cast<const uint4 *>(sW + (st * 2 + sl) * SLAB_BYTES + r * 128);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint4 v = rowp[cc];
+                    const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = __bfloat1622float2(p2[e]);
+                        ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
+                    }
+                }
+            }
+            const float inv = 1.f / sqrtf(ss / (float)dk + kRmsEps);
+            for (int sl = 0; sl < nslab_k; ++sl) {
+                uint4 *rowp = reinterpret_cast<uint4 *>(sW + (st * 2 + sl) * SLAB_BYTES + r * 128);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint4 v = rowp[cc];
+                    __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&v);
+                    const int c0 = sl * 64 + ((cc ^ (r & 7)) << 3);  // logical column of the chunk
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = __bfloat1622float2(p2[e]);
+                        const int ca = c0 + 2 * e;
+                        const float wa = (prm.q_w && ca < dk) ? prm.q_w[ca] : 1.f;
+                        const float wb = (prm.q_w && ca + 1 < dk) ? prm.q_w[ca + 1] : 1.f;
+                        p2[e] = __floats2bfloat162_rn(fmaxf(x.x * inv * wa, 0.f), fmaxf(x.y * inv * wb, 0.f));
+                    }
+                    rowp[cc] = v;
+                }
+            }
+            sm100::fence_proxy_async_smem();
+            sm100::mbar_arrive(&bars[QREADY0 + st]);
+            return true;
+        };
+        if (normq && nblk > 0) ok = normalize(0);
         for (int i = 0; i < nblk && ok; ++i) {
+            if (normq && i + 1 < nblk && !(ok = normalize(i + 1))) break;
             const int st = i & 1;
             const int row = i * BM + r;
             const bool valid = row < L;

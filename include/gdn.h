@@ -218,6 +218,25 @@ int gdn_fwd_noalloc(const void *q, const void *k, const void *v,
  *                   or nonzero when a bounded device-side wait gave up and the
  *                   outputs are not valid (what the synchronous modes report
  *                   as GDN_ERR_TIMEOUT).  4-byte aligned.
+ *   phase           GDN_PHASE_ALL (0): the whole pass.  The two halves of a
+ *                   pass, for context parallelism over time (SANA-WM summary,
+ *                   section 3.1, Stage 3: the sequence split over GPUs; the
+ *                   cliffmar.tech article, "NVIDIA SANA-WM", training section:
+ *                   "prefix-sum composition of GDN transition matrices"):
+ *                   GDN_PHASE_PREPARE (1) runs only the stages that do not
+ *                   depend on the entering state (gates, diagonal inverses,
+ *                   intra-frame solve, per-frame maps) into `workspace`;
+ *                   o, S_in and S_out are not touched.  GDN_PHASE_FINISH (2)
+ *                   runs the rest (scan from S_in, pseudo-values, output) from
+ *                   the workspace a PREPARE call with the same inputs and
+ *                   sizes filled on the same stream.  Both require a caller
+ *                   workspace, mode = GDN_MODE_TOKEN and no reverse,
+ *                   accumulate_o or qk_norm (else GDN_ERR_NOT_IMPLEMENTED).
+ *   segment_map     PREPARE only, optional: device fp32 [B, H, d_k + d_v, d_k]
+ *                   (16-byte aligned) that receives the affine map of this
+ *                   call's tokens on the state, S_end = S_begin Phi + Psi:
+ *                   rows 0 .. d_k-1 hold Phi (d_k x d_k), rows d_k .. hold Psi
+ *                   (d_v x d_k), per (b, h).  gdn_apply_maps composes maps.
  */
 typedef struct gdn_args {
     int struct_size;
@@ -244,9 +263,12 @@ typedef struct gdn_args {
     const float *k_norm_weight;
     const float *q_norm_weight;
     int *status_dev;
+    int phase;
+    float *segment_map;
 } gdn_args;
 
 enum { GDN_MODE_TOKEN = 0, GDN_MODE_FRAME = 1 };
+enum { GDN_PHASE_ALL = 0, GDN_PHASE_PREPARE = 1, GDN_PHASE_FINISH = 2 };
 enum { GDN_QK_NORM_KEYS = 1, GDN_QK_NORM_QUERIES = 2 };
 
 /* Kernel stages reported through gdn_args.stage_ms, in launch order:
@@ -261,6 +283,20 @@ enum { GDN_NUM_STAGES = 7 };
 
 int gdn_fwd_ex(const gdn_args *a);
 
+/*
+ * gdn_apply_maps -- S <- S Phi_j + Psi_j for j = 0 .. n_maps-1 in order, in
+ * place: the state entering a segment of a sequence split over ranks, from
+ * the state entering the sequence and the segment maps of the segments before
+ * it (the exclusive prefix of the maps; same passages as gdn_args.phase).
+ *   S     device fp32 [B, H, d_v, d_k], read and written (16-byte aligned)
+ *   maps  device fp32 [n_maps][B, H, d_k + d_v, d_k], each as gdn_fwd_ex's
+ *         segment_map writes it (16-byte aligned; may not overlap S)
+ * Sizes as gdn_fwd (d_k, d_v in {16, ..., 128}); n_maps >= 0.  Asynchronous
+ * on `stream`; argument errors return before anything is enqueued.
+ */
+int gdn_apply_maps(float *S, const float *maps, int n_maps, int B, int H, int d_k, int d_v,
+                   gdn_stream_t stream);
+
 /* Device scratch a call with these sizes needs with any flags of gdn_fwd_ex
  * (the size of the largest case, a reversed accumulating call; 0 if the
  * sizes are invalid). */
@@ -274,9 +310,9 @@ const char *gdn_last_error(void);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH.  The gdn_args layout
  * belongs to the version: 0.2.0 added mode, gamma, qk_norm, the RMSNorm
- * weights and status_dev (struct_size guards a caller built against another
- * layout). */
-#define GDN_VERSION 200
+ * weights and status_dev; 0.3.0 added phase and segment_map (struct_size
+ * guards a caller built against another layout). */
+#define GDN_VERSION 300
 int gdn_version(void);
 
 #ifdef __cplusplus

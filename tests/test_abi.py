@@ -47,7 +47,7 @@ def test_struct_size_matches_header():
     a.struct_size = ctypes.sizeof(binding.GdnArgs) + 8
     rc = g.load_library().gdn_fwd_ex(ctypes.byref(a))
     assert rc == 1 and "struct_size" in g.last_error()
-    assert ctypes.sizeof(binding.GdnArgs) == 208  # LP64 layout of gdn_args
+    assert ctypes.sizeof(binding.GdnArgs) == 224  # LP64 layout of gdn_args
 
 
 def _ex_args(**kw):
@@ -68,6 +68,15 @@ def _ex_args(**kw):
     (dict(qk_norm=4), 1, "qk_norm"),                  # not a mask of the two prologue bits
     (dict(qk_norm=-1), 1, "qk_norm"),
     (dict(status_dev=FAKE + 2), 4, "status_dev"),     # not 4-byte aligned
+    (dict(phase=3), 1, "phase"),                      # no such phase
+    (dict(phase=1), 1, "workspace"),                  # the phases keep their state in a caller workspace
+    (dict(phase=2, workspace=FAKE + (1 << 30), workspace_bytes=1 << 30, reverse=1), 9, "reverse"),
+    (dict(phase=1, workspace=FAKE + (1 << 30), workspace_bytes=1 << 30, mode=1, alpha=None,
+          gamma=FAKE + (1 << 29)), 9, "token-wise"),
+    (dict(segment_map=FAKE + (1 << 29)), 1, "segment_map"),                  # only a PREPARE call writes it
+    (dict(phase=1, workspace=FAKE + (1 << 30), workspace_bytes=1 << 30,
+          segment_map=FAKE + (1 << 29) + 4), 4, "segment_map"),              # misaligned
+    (dict(phase=1, workspace=FAKE + (1 << 30), workspace_bytes=1 << 30, segment_map=FAKE), 1, "overlaps"),
 ])
 def test_mode_validation(kw, status, text):
     # rejected before any device work (no GPU needed)
@@ -100,6 +109,18 @@ def _call(fn="gdn_fwd", q=FAKE, k=FAKE + 1024, v=FAKE + 2048, alpha=FAKE + 4096,
 def test_validation_errors(kw, status):
     assert _call(**kw) == status
     assert g.last_error() != ""
+
+
+def test_apply_maps_validation():
+    lib = g.load_library()
+    assert lib.gdn_apply_maps(FAKE, FAKE + (1 << 30), 1, 1, 2, 120, 64, None) == 3   # head dim
+    assert lib.gdn_apply_maps(FAKE + 4, FAKE + (1 << 30), 1, 1, 2, 64, 64, None) == 4  # alignment
+    assert lib.gdn_apply_maps(None, FAKE, 1, 1, 2, 64, 64, None) == 1                 # NULL state
+    assert lib.gdn_apply_maps(FAKE, FAKE + 1024, 1, 1, 2, 64, 64, None) == 1          # overlap
+    assert "overlaps" in g.last_error()
+    assert lib.gdn_apply_maps(FAKE, FAKE + (1 << 30), -1, 1, 2, 64, 64, None) == 1    # negative count
+    assert lib.gdn_apply_maps(None, None, 0, 1, 2, 64, 64, None) == 0                 # nothing to apply
+    assert g.last_error() == ""
 
 
 def test_overlap_rejected():

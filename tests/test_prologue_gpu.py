@@ -65,8 +65,10 @@ def features(inp, L, wk=None, wq=None):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("weighted", [False, True])
-def test_prologue_framewise(dtype, weighted):
-    B, H, F, L, dk, dv = 1, 2, 4, 200, 64, 48
+@pytest.mark.parametrize("dk", [48, 64, 112])  # one 64-column slab, one full slab, a slab and a part
+def test_prologue_framewise(dtype, weighted, dk):
+    # bf16: the feature maps are applied to the kernels' staged tiles; fp32: a prologue pass
+    B, H, F, L, dv = 1, 2, 4, 200, 48
     inp = raw_inputs(B, H, F, L, dk, dv, dtype, seed=51, state_std=0.1)
     wk, wq = weights(dk, 52) if weighted else (None, None)
     o, S = run(inp, L, "frame", wk, wq)
@@ -75,6 +77,24 @@ def test_prologue_framewise(dtype, weighted):
                                     nthreads=NTHREADS)
     assert rel(o, o_ref) <= TOL[dtype]
     assert rel(S, S_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_prologue_framewise_reverse_accumulate(dtype):
+    B, H, F, L, dk, dv = 1, 2, 5, 64, 64, 64
+    inp = raw_inputs(B, H, F, L, dk, dv, dtype, seed=57)
+    wk, wq = weights(dk, 58)
+    qh, kh = features(inp, L, wk, wq)
+    flip = lambda x: None if x is None else torch.flip(torch.as_tensor(x), dims=[1])  # noqa: E731
+    # the reversed frame-wise operator visits the frames backwards, each with its own gamma
+    o_r, S_r = oracle.framewise(flip(qh), flip(kh), flip(inp["v"]), flip(inp["gamma"]), flip(inp["beta"]), None,
+                                frame_len=L, nthreads=NTHREADS)
+    o_ref = np.flip(o_r, axis=1)
+    o0 = (torch.randn(B, F * L, H, dv, generator=torch.Generator().manual_seed(59), dtype=torch.float64)
+          * 0.25 * float(np.abs(o_ref).max())).to(inp["q"].dtype)
+    o, S = run(inp, L, "frame", wk, wq, o=o0.cuda(), reverse=True, accumulate=True)
+    assert rel(o - o0.double().numpy(), o_ref) <= TOL[dtype]
+    assert rel(S, S_r) <= TOL[dtype]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
