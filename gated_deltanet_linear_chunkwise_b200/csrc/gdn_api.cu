@@ -262,6 +262,9 @@ int cuda_fail(cudaError_t e, const char *what) {
 
 int run(const gdn_args &a) noexcept {
     try {
+        gdn::NvtxRange range(a.phase == GDN_PHASE_PREPARE  ? "gdn_fwd_ex (prepare)"
+                             : a.phase == GDN_PHASE_FINISH ? "gdn_fwd_ex (finish)"
+                                                           : "gdn_fwd_ex");
         g_err[0] = '\0';
         if (a.struct_size != (int)sizeof(gdn_args)) {
             set_err("gdn_args.struct_size = %d, this library expects %d", a.struct_size, (int)sizeof(gdn_args));

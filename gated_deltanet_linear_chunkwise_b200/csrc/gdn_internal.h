@@ -25,6 +25,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/gdn.h"
 
@@ -89,17 +90,30 @@ struct Workspace {
 
 // Optional stage timing: when `ev` is non-null it holds GDN_NUM_STAGES + 1
 // events; ev[i] is recorded before stage i and ev[GDN_NUM_STAGES] after the last.
+// Every call also leaves an NVTX marker at each stage boundary (host side; free when no
+// profiler is attached), inside the NVTX range the entry point opens for the call.
 inline cudaError_t mark(cudaEvent_t *ev, int i, cudaStream_t s) {
+    static const char *const names[GDN_NUM_STAGES + 1] = {"gdn: gates",      "gdn: diagonal inverses",
+                                                          "gdn: intra-frame solve", "gdn: frame transition",
+                                                          "gdn: scan",       "gdn: pseudo-values",
+                                                          "gdn: output",     "gdn: end"};
+    nvtxMarkA(names[i]);
     return ev ? cudaEventRecord(ev[i], s) : cudaSuccess;
 }
+
+// NVTX range around one call of the library (RAII).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 // Limit of the kernels' bounded device-side waits for this call, in ns: 2 s, unless the
 // debug variable GDN_DEBUG_WAIT_LIMIT_US (read at every call) sets a shorter one so a
 // test can make the waits give up (gdn_api.cu).
 uint64_t wait_limit_ns();
 // Debug: GDN_DEBUG_DROP_SIGNAL=1 (read at every call) makes the diagonal-inverse kernel
-// withhold its first load, so the wait on it gives up at the limit above and the pass
-// reports GDN_ERR_TIMEOUT without any fault (the bounded-wait test).  0 otherwise.
+// withhold its first block's product, so the wait on it gives up at the limit above and the
+// pass reports GDN_ERR_TIMEOUT without any fault (the bounded-wait test).  0 otherwise.
 int debug_drop_signal();
 
 // Argument validation of the C ABI (gdn_api.cu): fills p or returns a gdn_status.

@@ -27,7 +27,7 @@ inline int cf_stride(int L) { return (L + 3) & ~3; }
 
 struct TcLayout {
     size_t G, CF, GCT, Tinv, X, M, Mimg, N, Sig, SigB, U, err;
-    size_t Otmp, Qr, Kr, Vr, Ar, Br;  // reversed / accumulating calls only (0 bytes otherwise)
+    size_t Qr, Kr, Vr, Ar, Br;  // token-reversed input copies: reversed calls only (0 bytes otherwise)
     size_t total;
 };
 
@@ -50,11 +50,9 @@ TcLayout tc_layout(const Problem &p) {
     lay.SigB = off; off += align256(2 * nfh * p.dk * p.dv);
     lay.U = off;    off += align256(2 * nfh * p.L * p.dv);
     lay.err = off;  off += 256;
-    // A reversed scan runs the forward kernels on token-reversed copies of the inputs; a
-    // reversed or accumulating call writes o to a staging buffer first.
+    // A reversed scan runs the forward kernels on token-reversed copies of the inputs.
     const size_t ntok = (size_t)p.B * p.T * p.H;
-    const bool stage_o = p.reverse || p.accumulate, rev = p.reverse;
-    lay.Otmp = off; off += stage_o ? align256(2 * ntok * p.dv) : 0;
+    const bool rev = p.reverse;
     lay.Qr = off;   off += rev ? align256(2 * ntok * p.dk) : 0;
     lay.Kr = off;   off += rev ? align256(2 * ntok * p.dk) : 0;
     lay.Vr = off;   off += rev ? align256(2 * ntok * p.dv) : 0;
@@ -220,8 +218,8 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF, GCT);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 1, s))) return e;
-    if ((e = tc::launch_diag_inverse(tm_k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T, nfh, err, wait_ns,
-                                     debug_drop_signal(), num_sms, s)))
+    if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
+                                     nfh, err, wait_ns, debug_drop_signal(), s)))
         return e;
     if ((e = mark(ev, 2, s))) return e;
     tc::IntraParams ip;
@@ -235,8 +233,8 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     tp.G = G; tp.M = (!scan_tc || p.map_out) ? Mb : nullptr; tp.Mimg = scan_tc ? Mimg : nullptr; tp.N = Nb;
     tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
     tp.frame = 0; tp.beta = p.beta; tp.gamma = nullptr; tp.T = p.T;
-    tp.norm_k = 0; tp.k_w = nullptr; tp.k_post = 1.f;
-    if ((e = tc::launch_transition_tc(tm_k64, tm_x, tm_x, tp, nfh, s))) return e;
+    tp.norm_k = 0; tp.k_w = nullptr; tp.k_post = 1.f; tp.wait_ns = wait_ns;
+    if ((e = tc::launch_transition_tc(tm_k64, tm_x, tm_x, tp, nfh, num_sms, s))) return e;
     if (p.map_out && (e = simt_segment_map(p, Mb, Nb, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
     if (p.phase == GDN_PHASE_PREPARE) {
@@ -258,8 +256,8 @@ finish:
     up.X = X; up.U = U;
     up.L = p.L; up.dk = p.dk; up.dv = p.dv; up.nblk = nblk; up.err = err;
     up.frame = 0; up.o = nullptr; up.T = p.T; up.F = p.F; up.H = p.H; up.accumulate = 0;
-    up.norm_q = 0; up.q_w = nullptr;
-    if ((e = tc::launch_u_tc(tm_x128, tm_q, tm_sig, up, nfh, s))) return e;
+    up.norm_q = 0; up.q_w = nullptr; up.wait_ns = wait_ns;
+    if ((e = tc::launch_u_tc(tm_x128, tm_q, tm_sig, up, nfh, num_sms, s))) return e;
     if ((e = mark(ev, 6, s))) return e;
 
     tc::OutParams op;
@@ -269,6 +267,7 @@ finish:
     op.L = p.L; op.dk = p.dk; op.dv = p.dv; op.H = p.H; op.nblk = nblk;
     op.F = p.F; op.T = p.T; op.n_fh = nfh;
     op.accumulate = p.accumulate;
+    op.reverse_out = scan_reverse;
     op.err = err;
     if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u128, tm_sig, tm_g128, tm_cf128, op, num_sms, s))) return e;
     return mark(ev, 7, s);
@@ -287,27 +286,6 @@ __global__ void __launch_bounds__(256) reverse_rows_kernel(const V *__restrict__
     const V *s = src + row * row_vecs;
     V *d = dst + (b * T + (T - 1 - t)) * row_vecs;
     for (int i = threadIdx.x & 31; i < row_vecs; i += 32) d[i] = s[i];
-}
-
-// o (+)= the staged result, rows taken in reverse token order for a reversed scan, one warp
-// per row; the sum of an accumulating call is formed in fp32 and rounded once to bf16.
-__global__ void __launch_bounds__(256) finish_o_kernel(const __nv_bfloat162 *__restrict__ tmp,
-                                                       __nv_bfloat162 *__restrict__ o, long long rows, long long T,
-                                                       int row_pairs, int reverse, int accumulate) {
-    const long long row = blockIdx.x * 8ll + (threadIdx.x >> 5);
-    if (row >= rows) return;
-    const long long t = row % T, b = row / T;
-    const __nv_bfloat162 *s = tmp + (reverse ? (b * T + (T - 1 - t)) : row) * row_pairs;
-    __nv_bfloat162 *d = o + row * row_pairs;
-    for (int i = threadIdx.x & 31; i < row_pairs; i += 32) {
-        float2 v = __bfloat1622float2(s[i]);
-        if (accumulate) {
-            const float2 old = __bfloat1622float2(d[i]);
-            v.x += old.x;
-            v.y += old.y;
-        }
-        d[i] = __floats2bfloat162_rn(v.x, v.y);
-    }
 }
 
 cudaError_t reverse_rows(const void *src, void *dst, int B, long long T, size_t row_bytes, cudaStream_t s) {
@@ -357,7 +335,10 @@ cudaError_t launch_tc_frame(const Problem &p, void *ws, cudaStream_t s, cudaEven
     tp.norm_k = (p.qk_norm & GDN_QK_NORM_KEYS) ? 1 : 0;
     tp.k_w = p.k_norm_weight;
     tp.k_post = 1.f / sqrtf((float)p.dk * (float)p.L);
-    if ((e = tc::launch_transition_tc(tm_k64, tm_k64, tm_v64, tp, nfh, s))) return e;
+    tp.wait_ns = wait_limit_ns();
+    int dev = 0, num_sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if ((e = tc::launch_transition_tc(tm_k64, tm_k64, tm_v64, tp, nfh, num_sms, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
     if (scan_tc) {
         if ((e = tc::launch_scan_tc(p, Mimg, Nb, SigB, nullptr, err, wait_limit_ns(), s))) return e;
@@ -371,40 +352,35 @@ cudaError_t launch_tc_frame(const Problem &p, void *ws, cudaStream_t s, cudaEven
     up.frame = 1; up.o = (__nv_bfloat16 *)p.o; up.T = p.T; up.F = p.F; up.H = p.H; up.accumulate = p.accumulate;
     up.norm_q = (p.qk_norm & GDN_QK_NORM_QUERIES) ? 1 : 0;
     up.q_w = p.q_norm_weight;
-    if ((e = tc::launch_u_tc(tm_q, tm_q, tm_sig, up, nfh, s))) return e;
+    up.wait_ns = tp.wait_ns;
+    if ((e = tc::launch_u_tc(tm_q, tm_q, tm_sig, up, nfh, num_sms, s))) return e;
     return mark(ev, 7, s);
 }
 
 cudaError_t launch_tc(const Problem &p, void *ws, cudaStream_t s, cudaEvent_t *ev) {
     if (p.mode == GDN_MODE_FRAME) return launch_tc_frame(p, ws, s, ev);
-    if (!p.reverse && !p.accumulate) return launch_tc_forward(p, ws, 0, s, ev);
+    if (!p.reverse) return launch_tc_forward(p, ws, 0, s, ev);  // accumulate_o is the output kernel's
+    // A reversed scan runs the forward kernels on token-reversed copies of the inputs (the
+    // reversed recurrence is the forward one on them); the output kernel writes each row back
+    // to its own token (adding to o when accumulating), and the chunk-reset rule of the scan
+    // follows the original token positions.
     const TcLayout lay = tc_layout(p);
     char *base = (char *)ws;
     Problem q = p;
     q.reverse = 0;
-    q.accumulate = 0;
-    q.o = base + lay.Otmp;
     cudaError_t e;
-    if (p.reverse) {  // token-reversed copies: the reversed recurrence is the forward one on them
-        const size_t rq = (size_t)p.H * p.dk * 2, rv = (size_t)p.H * p.dv * 2, rg = (size_t)p.H * 4;
-        if ((e = reverse_rows(p.q, base + lay.Qr, p.B, p.T, rq, s))) return e;
-        if ((e = reverse_rows(p.k, base + lay.Kr, p.B, p.T, rq, s))) return e;
-        if ((e = reverse_rows(p.v, base + lay.Vr, p.B, p.T, rv, s))) return e;
-        if ((e = reverse_rows(p.alpha, base + lay.Ar, p.B, p.T, rg, s))) return e;
-        if ((e = reverse_rows(p.beta, base + lay.Br, p.B, p.T, rg, s))) return e;
-        q.q = base + lay.Qr;
-        q.k = base + lay.Kr;
-        q.v = base + lay.Vr;
-        q.alpha = (const float *)(base + lay.Ar);
-        q.beta = (const float *)(base + lay.Br);
-    }
-    if ((e = launch_tc_forward(q, ws, p.reverse, s, ev))) return e;
-    const long long rows = (long long)p.B * p.T;
-    if (rows > 0)
-        finish_o_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const __nv_bfloat162 *)(base + lay.Otmp),
-                                                                  (__nv_bfloat162 *)p.o, rows, p.T, p.H * p.dv / 2,
-                                                                  p.reverse, p.accumulate);
-    return cudaGetLastError();
+    const size_t rq = (size_t)p.H * p.dk * 2, rv = (size_t)p.H * p.dv * 2, rg = (size_t)p.H * 4;
+    if ((e = reverse_rows(p.q, base + lay.Qr, p.B, p.T, rq, s))) return e;
+    if ((e = reverse_rows(p.k, base + lay.Kr, p.B, p.T, rq, s))) return e;
+    if ((e = reverse_rows(p.v, base + lay.Vr, p.B, p.T, rv, s))) return e;
+    if ((e = reverse_rows(p.alpha, base + lay.Ar, p.B, p.T, rg, s))) return e;
+    if ((e = reverse_rows(p.beta, base + lay.Br, p.B, p.T, rg, s))) return e;
+    q.q = base + lay.Qr;
+    q.k = base + lay.Kr;
+    q.v = base + lay.Vr;
+    q.alpha = (const float *)(base + lay.Ar);
+    q.beta = (const float *)(base + lay.Br);
+    return launch_tc_forward(q, ws, p.reverse, s, ev);
 }
 
 int *tc_error_word(const Problem &p, void *ws) { return (int *)((char *)ws + tc_layout(p).err); }

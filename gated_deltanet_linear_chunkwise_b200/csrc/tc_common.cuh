@@ -41,14 +41,11 @@ __device__ __forceinline__ bool named_sync_and(int id, int nthreads, bool ok) {
 }
 
 // A kernel of a pass whose earlier stage recorded a failure in the error word does
-// nothing: every thread learns it before any barrier is armed or TMEM allocated, so a
-// pass that gave up leaves no copy or product in flight behind it.
-__device__ __forceinline__ bool pass_failed(const int *err) {
-    __shared__ int s_failed;
-    if (threadIdx.x == 0) s_failed = *(volatile const int *)err;
-    __syncthreads();
-    return s_failed != 0;
-}
+// nothing: every thread reads the word before any barrier is armed or TMEM allocated, so a
+// pass that gave up leaves no copy or product in flight behind it.  Only earlier kernels of
+// the same stream write the word, so every thread of this kernel reads the same value (and
+// no shared memory is spent on it: occupancy stays as the kernel's own budget sets it).
+__device__ __forceinline__ bool pass_failed(const int *err) { return *(volatile const int *)err != 0; }
 
 // K-major SW128 operand: tile of `rows` rows, 64-column slabs; K step ks (16 columns).
 __device__ __forceinline__ uint64_t desc_kmajor(const void *tile, int ks, int rows) {
@@ -70,7 +67,8 @@ struct OutParams {
     void *o;                 // [B,T,H,dv] bf16
     int L, dk, dv, H, nblk;
     long long F, T, n_fh;
-    int accumulate;
+    int accumulate;          // o += result (formed in fp32, rounded once)
+    int reverse_out;         // the pass ran on token-reversed inputs: row t goes to token T - 1 - t
     int *err;
 };
 
@@ -100,6 +98,7 @@ struct TransParams {
     const float *beta;         // [B,T,H]
     const float *gamma;        // [B,F,H]
     long long T;
+    uint64_t wait_ns;          // limit of the bounded waits
     // frame-wise operator: the key feature map applied to the staged K rows (both copies)
     // before the products, K <- max(RMSNorm(K) * w, 0) * k_post; 0: keys used as given
     int norm_k;
@@ -117,6 +116,7 @@ struct UParams {
     __nv_bfloat16 *o;          // [B,T,H,dv]
     long long T, F;
     int H, accumulate;
+    uint64_t wait_ns;          // limit of the bounded waits
     // frame-wise operator: the query feature map applied to the staged Q rows before the
     // product, Q <- max(RMSNorm(Q) * w, 0); 0: queries used as given
     int norm_q;
@@ -129,11 +129,11 @@ constexpr float kRmsEps = 1e-6f;
 // tm_k / tm_x / tm_v deliver 64-token boxes (tm_x the [Ub | W] rows, tm_v the
 // values, read by the frame-wise operator only).
 cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_v,
-                                 const TransParams &prm, long long n_fh, cudaStream_t s);
+                                 const TransParams &prm, long long n_fh, int num_sms, cudaStream_t s);
 // tm_x delivers 128-row boxes of X, tm_q 128-token boxes of q (frame-wise
 // operator), tm_sig the bf16 state of a frame-head.
 cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_q, const CUtensorMap &tm_sig,
-                        const UParams &prm, long long n_fh, cudaStream_t s);
+                        const UParams &prm, long long n_fh, int num_sms, cudaStream_t s);
 
 // tm_k delivers 128-token boxes of k, tm_x64 64-row boxes of X, tm_t one
 // 128 x 128 block, tm_gct the G and cf of one 128-token tile; tm_xs stores
@@ -142,10 +142,11 @@ cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x64, 
                             const CUtensorMap &tm_gct, const CUtensorMap &tm_xs, const IntraParams &prm,
                             long long n_fh, cudaStream_t s);
 
-// tm_k delivers 128-token boxes of k (the Gram's operand).  Persistent: at most num_sms CTAs.
-cudaError_t launch_diag_inverse(const CUtensorMap &tm_k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
+// One CTA per (frame-head, 128-row block).  drop_first (debug): the first block's Gram is not
+// issued, so its bounded wait gives up and the pass reports a timeout without any fault.
+cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
                                 int L, int dk, int H, int nblk, long long F, long long T, long long n_fh,
-                                int *err, uint64_t wait_ns, int drop_first_load, int num_sms, cudaStream_t s);
+                                int *err, uint64_t wait_ns, int drop_first, cudaStream_t s);
 
 // tm_q / tm_k / tm_u / tm_g / tm_cf deliver 128-token boxes.
 // The scan over frames on the tensor cores (tc_scan.cu): M from the transition

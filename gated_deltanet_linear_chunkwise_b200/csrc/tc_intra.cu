@@ -317,12 +317,21 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
         bool ok = true;
         int kn = 0, sn = 0;
+        // this row's G and beta, read one block ahead so their latency stays off the S -> P steps
+        auto row_gates = [&](int i, float &g, float &bb) {
+            const int rw = i * BM + r;
+            const bool ok_row = i < nblk && rw < L;
+            g = ok_row ? Gf[rw] : 0.f;
+            bb = ok_row ? prm.beta[((long long)b * prm.T + f * L + rw) * prm.H + h] : 0.f;
+        };
+        float G_next, be_next;
+        row_gates(0, G_next, be_next);
         for (int i = 0; i < nblk && ok; ++i) {
             const int row = i * BM + r;
             const bool valid = row < L;
-            const float Gr = valid ? Gf[row] : 0.f;
+            const float Gr = G_next, be = be_next;
+            row_gates(i + 1, G_next, be_next);
             const long long tok = ((long long)b * prm.T + f * L + row) * prm.H + h;
-            const float be = valid ? prm.beta[tok] : 0.f;
             // half 0 needs this row's values in the diagonal step: pull them into L2 now
             const __nv_bfloat16 *vp = prm.v + tok * dv;
             if (half == 0 && valid) {
@@ -362,6 +371,16 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             if (!ok) break;
             // ---- Y_i = R_i + acc_i  -> sYX (MN-major: row = K index of the T_ii Y_i product)
             // (K_i: the W half reads it; block 0 has no S product that waited for it)
+            // half 0: this row's values, read before the accumulator wait so their latency hides
+            // behind the block's last products (v is read once: evict first, keep K and X in L2)
+            uint4 vrow[16];
+            if (half == 0) {
+                const uint64_t once = sm100::policy_evict_first();
+#pragma unroll
+                for (int c8 = 0; c8 < 16; ++c8)
+                    vrow[c8] = (valid && c8 < dv / 8) ? sm100::ld_nc_hint(reinterpret_cast<const uint4 *>(vp) + c8, once)
+                                                      : make_uint4(0, 0, 0, 0);
+            }
             ok = sm100::mbar_wait(&bars[ACCFULL], i & 1, err) && sm100::mbar_wait(&bars[KIFULL], i & 1, err);
             if (!ok) break;
             sm100::tc_fence_after();
@@ -372,12 +391,6 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 *reinterpret_cast<uint4 *>(sYX + yx_offset(c, r)) = val;
             };
             if (half == 0) {  // Ub columns: beta_r v_r + acc
-                const uint64_t once = sm100::policy_evict_first();  // v is read once: keep K and X in L2
-                uint4 vrow[16];
-#pragma unroll
-                for (int c8 = 0; c8 < 16; ++c8)
-                    vrow[c8] = (valid && c8 < dv / 8) ? sm100::ld_nc_hint(reinterpret_cast<const uint4 *>(vp) + c8, once)
-                                                      : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int j2 = 0; j2 < 4; ++j2) {  // two 16-column loads per wait
                     if (32 * j2 >= dv) break;

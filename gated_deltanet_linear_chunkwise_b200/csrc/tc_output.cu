@@ -40,23 +40,22 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kEpi = 256;                 // epilogue threads
 constexpr int JT = 128;                   // tokens per column tile (= BM: tile I is block I's diagonal)
-constexpr int NSLOT = 2;                  // ring depth
+constexpr int NSLOT = 3;                  // ring depth
 constexpr int NSB = 2;                    // S/P buffers in TMEM
 constexpr int JSLAB = JT * 128;           // one 128-row slab
-constexpr int SLOT_BYTES = 4 * JSLAB;     // K (2 slabs) + U (2 slabs); Sig (<= 32 KB) fills a whole slot
+constexpr int SLOT_BYTES = 4 * JSLAB;     // K (2 slabs) + U (2 slabs); or an item's Q (2 slabs) + Sig (<= 32 KB)
 constexpr int GC_BYTES = 2 * JT * 4;      // G and cf of one tile
 constexpr float kSplitMax = 60.f;         // largest row exponent the in-group split takes
 
 struct Smem {
-    static constexpr uint32_t Q = 0;                          // 2 stages x 2 slabs x 128 rows
-    static constexpr uint32_t RING = Q + 4 * SLAB_BYTES;      // NSLOT x 64 KB
+    static constexpr uint32_t RING = 0;                       // NSLOT x 64 KB
     static constexpr uint32_t GC = RING + NSLOT * SLOT_BYTES; // NSLOT x (G[128], cf[128])
     static constexpr uint32_t END = GC + NSLOT * GC_BYTES;
 };
 
 enum Bar {
-    QFULL = 0, QEMPTY = 2, RFULL = 4, REMPTY = RFULL + NSLOT, SFULL = REMPTY + NSLOT, SFREE = SFULL + NSB,
-    PFULL = SFREE + NSB, OFULL = PFULL + NSB, OEMPTY = OFULL + 2, NBAR = OEMPTY + 2
+    RFULL = 0, REMPTY = RFULL + NSLOT, SFULL = REMPTY + NSLOT, SFREE = SFULL + NSB, PFULL = SFREE + NSB,
+    OFULL = PFULL + NSB, OEMPTY = OFULL + 1, QFREE = OEMPTY + 1, DRAIN = QFREE + 2, NBAR = DRAIN + 1
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -71,7 +70,6 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int gs = (L + 3) & ~3;           // row stride of G and cf
     const int ntile_frame = (L + JT - 1) / JT;
 
-    unsigned char *sQ = smem + Smem::Q;
     unsigned char *sRing = smem + Smem::RING;
     float *sGC = (float *)(smem + Smem::GC);
     uint64_t *bars = (uint64_t *)(smem + Smem::END);
@@ -82,7 +80,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i) {
-            const bool epi = (i >= PFULL && i < PFULL + NSB) || (i >= OEMPTY && i < OEMPTY + 2);
+            const bool epi = (i >= PFULL && i < PFULL + NSB) || i == OEMPTY;
             sm100::mbar_init(&bars[i], epi ? kEpi : 1);
         }
         sm100::fence_barrier_init();
@@ -95,7 +93,9 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t t_s0 = tbase, t_o0 = tbase + 256;
+    // TMEM: two S/P buffers (128 columns each), the O accumulator (128), and the item's Q in two
+    // buffers of 64 columns (two bf16 per column: the A operand of S = Q K^T, read from TMEM)
+    const uint32_t t_s0 = tbase, t_o = tbase + 256, t_q0 = tbase + 384;
 
     const int nks_d = dk / 16;
     const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
@@ -138,23 +138,21 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const long long f = fh % F, chain = fh / F;
                 const int h = (int)(chain % prm.H), b = (int)(chain / prm.H);
                 const int bf = (int)(b * F + f);
-                const int qb = t & 1;
-                if (t >= 2) ok = sm100::mbar_wait(&bars[QEMPTY + qb], ((t - 2) >> 1) & 1, err);
-                if (!ok) break;
-                sm100::mbar_arrive_expect_tx(&bars[QFULL + qb], (uint32_t)(nslab_k * SLAB_BYTES));
-                for (int sl = 0; sl < nslab_k; ++sl)
-                    sm100::tma_load_4d_hint(sQ + (qb * 2 + sl) * SLAB_BYTES, &tm_q, &bars[QFULL + qb], sl * SLAB, h,
-                                            I * BM, bf, once);
                 const int nt = item_ntiles(I);
                 for (int j = -1; j < nt && ok; ++j, ++n) {
                     const int st = n % NSLOT;
                     if (n >= NSLOT) ok = sm100::mbar_wait(&bars[REMPTY + st], ((n / NSLOT) - 1) & 1, err);
                     if (!ok) break;
                     unsigned char *slot = sRing + st * SLOT_BYTES;
-                    if (j < 0) {  // the state term: Sig fills the slot
-                        sm100::mbar_arrive_expect_tx(&bars[RFULL + st], (uint32_t)(nslab_v * dk * 128));
+                    if (j < 0) {  // the item's Q (2 slabs) and the state term's Sig (after them)
+                        sm100::mbar_arrive_expect_tx(&bars[RFULL + st],
+                                                     (uint32_t)(nslab_k * JSLAB + nslab_v * dk * 128));
+                        for (int sl = 0; sl < nslab_k; ++sl)
+                            sm100::tma_load_4d_hint(slot + sl * JSLAB, &tm_q, &bars[RFULL + st], sl * SLAB, h, I * BM,
+                                                    bf, once);
                         for (int sl = 0; sl < nslab_v; ++sl)
-                            sm100::tma_load_3d(slot + sl * dk * 128, &tm_sig, &bars[RFULL + st], sl * SLAB, 0, (int)fh);
+                            sm100::tma_load_3d(slot + 2 * JSLAB + sl * dk * 128, &tm_sig, &bars[RFULL + st], sl * SLAB,
+                                               0, (int)fh);
                     } else {
                         sm100::mbar_arrive_expect_tx(&bars[RFULL + st],
                                                      (uint32_t)((nslab_k + nslab_v) * JSLAB + GC_BYTES));
@@ -170,8 +168,10 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     }
                 }
             }
-            // leave with no copy in flight: the last item's MMAs consumed everything
-            if (ok && t >= 1) sm100::mbar_wait(&bars[QEMPTY + ((t - 1) & 1)], ((t - 1) >> 1) & 1, err);
+            // leave with no copy in flight: the last NSLOT uses of the ring have landed (full limit)
+            for (int u = n > NSLOT ? n - NSLOT : 0; u < n; ++u)
+                sm100::mbar_wait(&bars[RFULL + (u % NSLOT)], (uint32_t)((u / NSLOT) & 1), err, sm100::kWaitLimitNs,
+                                 true);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -183,51 +183,55 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             for (long long w = w_begin; w < w_end && ok; ++w, ++t) {
                 const int I = item_blk(w);
                 const int nt = item_ntiles(I);
-                const int ob = t & 1, qb = t & 1;
-                const uint32_t t_o = t_o0 + ob * 128;
-                const unsigned char *qt = sQ + qb * 2 * SLAB_BYTES;
-                // ---- state pseudo-tile: hand an S/P buffer to the epilogue, then O = Q~ Sig
-                int sb = sc % NSB, st = n % NSLOT;
-                if (sc >= NSB) ok = sm100::mbar_wait(&bars[SFREE + sb], ((sc / NSB) - 1) & 1, err);
+                const int qb = t & 1;
+                // ---- state pseudo-tile: hand an S/P buffer to the epilogue, which writes
+                //      Q~ = diag(e^G) Q there and Q into TMEM buffer qb
+                const int sb0 = sc % NSB, st0 = n % NSLOT, sc0 = sc;
+                if (sc >= NSB) ok = sm100::mbar_wait(&bars[SFREE + sb0], ((sc / NSB) - 1) & 1, err);
                 if (!ok) break;
-                sm100::mma_commit(&bars[SFULL + sb]);
-                ok = sm100::mbar_wait(&bars[RFULL + st], (n / NSLOT) & 1, err) &&
-                     sm100::mbar_wait(&bars[PFULL + sb], (sc / NSB) & 1, err);
-                if (ok && t >= 2) ok = sm100::mbar_wait(&bars[OEMPTY + ob], ((t - 2) >> 1) & 1, err);
-                if (!ok) break;
-                sm100::tc_fence_after();
-                for (int ks = 0; ks < nks_d; ++ks)
-                    sm100::mma_bf16_ts(t_o, t_s0 + sb * JT + ks * 8, desc_mnmajor(sRing + st * SLOT_BYTES, ks, dk),
-                                       id_o, ks > 0);
-                sm100::mma_commit(&bars[SFREE + sb]);
-                sm100::mma_commit(&bars[REMPTY + st]);
+                sm100::mma_commit(&bars[SFULL + sb0]);
                 ++n;
                 ++sc;
-                // ---- column tiles: S = Q K^T as soon as a tile and an S/P buffer are ready,
-                //      O += P U as soon as the epilogue has written P
-                if (ok) ok = sm100::mbar_wait(&bars[QFULL + qb], (t >> 1) & 1, err);
+                // ---- then, polling: O = Q~ Sig once Q~ is written and the previous item's O has
+                //      drained; S = Q K^T (Q from TMEM) as soon as Q, a tile and an S/P buffer are
+                //      ready; O += P U (after O = Q~ Sig) as soon as the epilogue has written P
                 const int n0 = n, s0 = sc;
                 int js = 0, jp = 0;
+                bool q_ready = false, o_started = false;
                 sm100::Spin spin;
                 while (ok && jp < nt) {
                     bool prog = false;
-                    if (js < nt && js - jp < NSB) {  // the buffer's previous product has been issued
+                    if (!q_ready && sm100::mbar_test(&bars[PFULL + sb0], (uint32_t)((sc0 / NSB) & 1))) {
+                        q_ready = true;
+                        prog = true;
+                    }
+                    if (q_ready && !o_started && (t == 0 || sm100::mbar_test(&bars[OEMPTY], (uint32_t)((t - 1) & 1)))) {
+                        sm100::tc_fence_after();
+                        const unsigned char *sig = sRing + st0 * SLOT_BYTES + 2 * JSLAB;
+                        for (int ks = 0; ks < nks_d; ++ks)
+                            sm100::mma_bf16_ts(t_o, t_s0 + sb0 * JT + ks * 8, desc_mnmajor(sig, ks, dk), id_o, ks > 0);
+                        sm100::mma_commit(&bars[SFREE + sb0]);
+                        sm100::mma_commit(&bars[REMPTY + st0]);
+                        o_started = true;
+                        prog = true;
+                    }
+                    if (q_ready && js < nt && js - jp < NSB) {  // the buffer's previous product has been issued
                         const int cs = s0 + js, nn = n0 + js;
-                        sb = cs % NSB;
-                        st = nn % NSLOT;
+                        const int sb = cs % NSB, st = nn % NSLOT;
                         if (sm100::mbar_test(&bars[RFULL + st], (nn / NSLOT) & 1) &&
                             (cs < NSB || sm100::mbar_test(&bars[SFREE + sb], ((cs / NSB) - 1) & 1))) {
                             sm100::tc_fence_after();
                             const unsigned char *kt = sRing + st * SLOT_BYTES;
                             for (int ks = 0; ks < nks_d; ++ks)
-                                sm100::mma_bf16_ss(t_s0 + sb * JT, desc_kmajor(qt, ks, BM), desc_kmajor(kt, ks, JT),
+                                sm100::mma_bf16_ts(t_s0 + sb * JT, t_q0 + qb * 64 + ks * 8, desc_kmajor(kt, ks, JT),
                                                    id_s, ks > 0);
                             sm100::mma_commit(&bars[SFULL + sb]);
                             ++js;
+                            if (js == nt) sm100::mma_commit(&bars[QFREE + qb]);  // Q buffer qb may be rewritten
                             prog = true;
                         }
                     }
-                    if (jp < js) {
+                    if (o_started && jp < js) {
                         const int cs = s0 + jp, nn = n0 + jp;
                         const int pb = cs % NSB, pst = nn % NSLOT;
                         if (sm100::mbar_test(&bars[PFULL + pb], (cs / NSB) & 1)) {
@@ -249,9 +253,10 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 n = n0 + nt;
                 sc = s0 + nt;
                 if (!ok) break;
-                sm100::mma_commit(&bars[OFULL + ob]);
-                sm100::mma_commit(&bars[QEMPTY + qb]);
+                sm100::mma_commit(&bars[OFULL]);
             }
+            sm100::mma_commit(&bars[DRAIN]);  // every product issued completes before TMEM is released
+            sm100::mbar_wait(&bars[DRAIN], 0u, err, sm100::kWaitLimitNs, true);
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -284,32 +289,37 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         };
         // state pseudo-tile: P <- diag(e^G) Q_I, written into the S/P buffer as bf16
         auto pseudo = [&](const Item &it, int t) -> bool {
-            const int qb = t & 1, sb = sc % NSB;
+            const int qb = t & 1, sb = sc % NSB, st = n % NSLOT;
             if (!sm100::mbar_wait(&bars[SFULL + sb], (sc / NSB) & 1, err)) return false;
-            if (!sm100::mbar_wait(&bars[QFULL + qb], (t >> 1) & 1, err)) return false;
+            if (!sm100::mbar_wait(&bars[RFULL + st], (n / NSLOT) & 1, err)) return false;  // Q and Sig
+            // Q buffer qb: the S products of item t - 2 that read it have completed
+            if (t >= 2 && !sm100::mbar_wait(&bars[QFREE + qb], (uint32_t)(((t - 2) >> 1) & 1), err)) return false;
             sm100::tc_fence_after();
+            const unsigned char *sq = sRing + st * SLOT_BYTES;
             const float eg = it.valid ? __expf(it.Gr) : 0.f;
             for (int c16 = half; c16 * 32 < dk; c16 += 2) {  // 32 bf16 -> 16 TMEM columns per group
-                uint32_t pk[16];
+                uint32_t pk[16], qk[16];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int lc = c16 * 4 + u;  // logical 8-column chunk
                     if (lc * 8 < dk) {
                         const int sl = lc >> 3, cc = lc & 7;
-                        uint4 v = *reinterpret_cast<const uint4 *>(sQ + (qb * 2 + sl) * SLAB_BYTES + r * 128 +
-                                                                   ((cc ^ (r & 7)) << 4));
+                        uint4 v = *reinterpret_cast<const uint4 *>(sq + sl * JSLAB + r * 128 + ((cc ^ (r & 7)) << 4));
                         const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+                        const uint32_t *q2 = reinterpret_cast<const uint32_t *>(&v);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 x = __bfloat1622float2(p2[e]);
                             pk[u * 4 + e] = pack_bf16(eg * x.x, eg * x.y);
+                            qk[u * 4 + e] = q2[e];
                         }
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) pk[u * 4 + e] = 0u;
+                        for (int e = 0; e < 4; ++e) pk[u * 4 + e] = qk[u * 4 + e] = 0u;
                     }
                 }
                 sm100::tmem_st16(t_s0 + sb * JT + lane_off + c16 * 16, pk);
+                sm100::tmem_st16(t_q0 + qb * 64 + lane_off + c16 * 16, qk);
             }
             sm100::tmem_st_wait();
             sm100::tc_fence_before();
@@ -377,10 +387,10 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             return true;
         };
         auto drain = [&](const Item &it, int t) -> bool {
-            const int ob = t & 1;
-            if (!sm100::mbar_wait(&bars[OFULL + ob], (t >> 1) & 1, err)) return false;
+            if (!sm100::mbar_wait(&bars[OFULL], (uint32_t)(t & 1), err)) return false;
             sm100::tc_fence_after();
-            const long long tt = it.f * L + it.row;
+            const long long tt0 = it.f * L + it.row;
+            const long long tt = prm.reverse_out ? prm.T - 1 - tt0 : tt0;  // a reversed scan's row, back in place
             __nv_bfloat16 *o = (__nv_bfloat16 *)prm.o + ((((long long)it.b * prm.T + tt) * prm.H + it.h) * dv);
             // columns c = 16 half + 32 i (dv <= 128), two 16-column loads per wait (the second
             // may read past dv, inside the O buffer's 128 columns, and is then not stored)
@@ -389,8 +399,8 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int cb = 16 * half + 64 * i2;
                 if (cb >= dv) break;
                 float acc[2][16];
-                sm100::tmem_ld16(t_o0 + ob * 128 + lane_off + cb, acc[0]);
-                sm100::tmem_ld16(t_o0 + ob * 128 + lane_off + cb + 32, acc[1]);
+                sm100::tmem_ld16(t_o + lane_off + cb, acc[0]);
+                sm100::tmem_ld16(t_o + lane_off + cb + 32, acc[1]);
                 sm100::tmem_ld_wait();
                 if (!it.valid) continue;
 #pragma unroll
@@ -421,7 +431,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
             sm100::tc_fence_before();
-            sm100::mbar_arrive(&bars[OEMPTY + ob]);
+            sm100::mbar_arrive(&bars[OEMPTY]);
             return true;
         };
         long long w = w_begin;
@@ -432,12 +442,13 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             ok = pseudo(cur, 0);
         }
         for (int t = 0; ok; ++t) {
-            ok = tiles(cur);
-            if (!ok) break;
+            // the next item's row (and its G, a global load) is read before this item's tiles
             const long long wn = w + 1;
             Item nxt;
+            if (wn < w_end) nxt = item_of(wn);
+            ok = tiles(cur);
+            if (!ok) break;
             if (wn < w_end) {
-                nxt = item_of(wn);
                 ok = pseudo(nxt, t + 1);
                 if (!ok) break;
             }

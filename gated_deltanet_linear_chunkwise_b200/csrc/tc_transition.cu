@@ -132,12 +132,21 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int row_in = r & (CH - 1), sl = r >> 6;
         float *sSS = reinterpret_cast<float *>(bars + NBAR + 1);  // [2][64] partial sums of squares
         const bool normk = frame && prm.norm_k;
+        // the K row's factor: e^{G_L - G_r}, or beta_r for the frame-wise map; read one chunk
+        // ahead so the load's latency stays off the scaling step
+        auto row_gate = [&](int c) -> float {
+            const int row = c * CH + row_in;
+            if (c >= nch || row >= L) return 0.f;
+            return frame ? prm.beta[((long long)b * prm.T + f * L + row) * prm.H + h] : Gf[row];
+        };
+        float g_next = row_gate(0);
         for (int c = 0; c < nch && ok; ++c) {
             const int st = c % NST;
             const int row = c * CH + row_in;
-            float sc = 0.f;  // the K row's factor: e^{G_L - G_r}, or beta_r for the frame-wise map
-            if (row < L) sc = frame ? prm.beta[((long long)b * prm.T + f * L + row) * prm.H + h] : __expf(GL - Gf[row]);
-            ok = sm100::mbar_wait(&bars[FULL + st], (c / NST) & 1, err);
+            const float g_row = g_next;
+            g_next = row_gate(c + 1);
+            const float sc = row >= L ? 0.f : (frame ? g_row : __expf(GL - g_row));
+            ok = sm100::mbar_wait(&bars[FULL + st], (c / NST) & 1, err, prm.wait_ns);
             if (normk) ok = named_sync_and(1, 128, ok);  // the row's two halves meet below
             if (!ok) break;
             if (normk) {
@@ -273,7 +282,8 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 }  // namespace
 
 cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_v,
-                                 const TransParams &prm, long long n_fh, cudaStream_t s) {
+                                 const TransParams &prm, long long n_fh, int /*num_sms: one CTA per frame-head*/,
+                                 cudaStream_t s) {
     const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16 + 2 * CH * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(k_transition_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -3,9 +3,11 @@
 // With the state Sig entering a frame known, the frame's pseudo-values are
 // U = Ub - W Sig (U = T (beta V - decayed K S) in the UT form of the delta
 // rule; SANA-WM summary, "Memory-Efficient Long-Context Modeling
-// (Section 3.2)", frame-wise GDN).  One CTA per frame-head walks its
-// 128-row blocks: A = W (K-major, the last d_k columns of the [Ub | W]
-// rows), B = Sig in bf16 (MN-major), D = W Sig in a TMEM double buffer;
+// (Section 3.2)", frame-wise GDN).  Persistent: one CTA per SM walks the
+// 128-row blocks of its frame-heads: A = W (K-major, the last d_k columns of
+// the [Ub | W] rows, through a 4-deep ring), B = Sig in bf16 (MN-major, the
+// next frame-head's state loading into a second buffer), D = W Sig in a TMEM
+// double buffer;
 // the epilogue subtracts it from Ub (read straight from global) and writes
 // U in bf16, the B operand layout of the output kernel.
 // The same kernel is the frame-wise operator's output (SANA-WM summary,
@@ -19,38 +21,48 @@ namespace tc {
 namespace {
 
 constexpr int kThreads = 192;
+constexpr int NW = 4;  // ring depth of the W (or Q) tiles
 
 struct Smem {
-    static constexpr uint32_t SIG = 0;                     // 2 slabs x d_k rows (<= 32 KB)
-    static constexpr uint32_t W = SIG + 2 * SLAB_BYTES;    // 2 stages x 2 slabs x 128 rows
-    static constexpr uint32_t END = W + 4 * SLAB_BYTES;
+    static constexpr uint32_t SIG = 0;                     // 2 buffers x 2 slabs x d_k rows (<= 32 KB each)
+    static constexpr uint32_t W = SIG + 4 * SLAB_BYTES;    // NW stages x 2 slabs x 128 rows
+    static constexpr uint32_t END = W + NW * 2 * SLAB_BYTES;
 };
 
-enum Bar { SIGFULL, WFULL0, WFULL1, WEMPTY0, WEMPTY1, DFULL0, DFULL1, DEMPTY0, DEMPTY1, QREADY0, QREADY1, NBAR };
+enum Bar {
+    SIGFULL = 0, SIGEMPTY = 2, WFULL = 4, WEMPTY = WFULL + NW, QREADY = WEMPTY + NW, DFULL = QREADY + NW,
+    DEMPTY = DFULL + 2, DRAIN = DEMPTY + 2, NBAR
+};
 
-__global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
+// Persistent: one CTA per SM walks the 128-row blocks of its frame-heads (blockIdx.x +
+// t gridDim.x); block i of the CTA's t-th frame-head is ring use g = t nblk + i, so the W
+// tiles stream without a pause between frame-heads while the next state loads.
+__global__ void __launch_bounds__(kThreads, 1)
 k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_q,
-       const __grid_constant__ CUtensorMap tm_sig, const UParams prm) {
+       const __grid_constant__ CUtensorMap tm_sig, const UParams prm, long long n_fh) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
-    const long long fh = blockIdx.x;
-    unsigned char *sSig = smem + Smem::SIG;
     unsigned char *sW = smem + Smem::W;
     uint64_t *bars = (uint64_t *)(smem + Smem::END);
     uint32_t *tmem_slot = (uint32_t *)(bars + NBAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *err = prm.err;
+    const uint64_t wait_ns = prm.wait_ns;
     const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
     const bool frame = prm.frame != 0;
     const bool normq = frame && prm.norm_q;
-    const long long f = frame ? fh % prm.F : 0, chain = frame ? fh / prm.F : 0;
-    const int h = frame ? (int)(chain % prm.H) : 0, b = frame ? (int)(chain / prm.H) : 0;
+    const long long nmine = n_fh > blockIdx.x ? (n_fh - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const long long total = nmine * nblk;
+    auto fh_of = [&](long long t) { return blockIdx.x + t * gridDim.x; };
+    auto sig_buf = [&](long long t) { return smem + Smem::SIG + (t & 1) * 2 * SLAB_BYTES; };
 
     if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NBAR; ++i)
-            sm100::mbar_init(&bars[i], (i == DEMPTY0 || i == DEMPTY1 || i == QREADY0 || i == QREADY1) ? 128 : 1);
+        for (int i = 0; i < NBAR; ++i) {
+            const bool many = (i >= QREADY && i < QREADY + NW) || i == DEMPTY || i == DEMPTY + 1;
+            sm100::mbar_init(&bars[i], many ? 128 : 1);
+        }
         sm100::fence_barrier_init();
     }
     if (warp == 1) {
@@ -66,46 +78,72 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
         if (lane == 0) {
             sm100::tma_prefetch_desc(frame ? &tm_q : &tm_x);
             sm100::tma_prefetch_desc(&tm_sig);
-            sm100::mbar_arrive_expect_tx(&bars[SIGFULL], (uint32_t)(nslab_v * dk * 128));
-            for (int sl = 0; sl < nslab_v; ++sl)
-                sm100::tma_load_3d(sSig + sl * dk * 128, &tm_sig, &bars[SIGFULL], sl * SLAB, 0, (int)fh);
+            long long g = 0, tsig = 0;  // next ring use; next frame-head whose state to load
             bool ok = true;
-            for (int i = 0; i < nblk && ok; ++i) {
-                const int st = i & 1;
-                if (i >= 2) ok = sm100::mbar_wait(&bars[WEMPTY0 + st], ((i - 2) >> 1) & 1, err);
+            for (; g < total && ok; ++g) {
+                const long long t = g / nblk;
+                const int i = (int)(g % nblk), st = (int)(g % NW);
+                // the frame-head's state (ahead of its first block; its buffer's previous frame-head
+                // (t - 2) has finished its products)
+                while (ok && tsig <= t && tsig < nmine) {
+                    if (tsig >= 2)
+                        ok = sm100::mbar_wait(&bars[SIGEMPTY + (tsig & 1)], (uint32_t)(((tsig >> 1) - 1) & 1), err, wait_ns);
+                    if (!ok) break;
+                    sm100::mbar_arrive_expect_tx(&bars[SIGFULL + (tsig & 1)], (uint32_t)(nslab_v * dk * 128));
+                    for (int sl = 0; sl < nslab_v; ++sl)
+                        sm100::tma_load_3d(sig_buf(tsig) + sl * dk * 128, &tm_sig, &bars[SIGFULL + (tsig & 1)],
+                                           sl * SLAB, 0, (int)fh_of(tsig));
+                    ++tsig;
+                }
+                if (ok && g >= NW) ok = sm100::mbar_wait(&bars[WEMPTY + st], (uint32_t)(((g / NW) - 1) & 1), err, wait_ns);
                 if (!ok) break;
-                sm100::mbar_arrive_expect_tx(&bars[WFULL0 + st], (uint32_t)(nslab_k * SLAB_BYTES));
+                const long long fh = fh_of(t);
+                unsigned char *wst = sW + st * 2 * SLAB_BYTES;
+                sm100::mbar_arrive_expect_tx(&bars[WFULL + st], (uint32_t)(nslab_k * SLAB_BYTES));
                 for (int sl = 0; sl < nslab_k; ++sl) {
-                    if (frame)  // the frame's queries
-                        sm100::tma_load_4d(sW + (st * 2 + sl) * SLAB_BYTES, &tm_q, &bars[WFULL0 + st], sl * SLAB, h,
-                                           i * BM, (int)(b * prm.F + f));
-                    else  // W = columns dv .. dv + dk of the [Ub | W] rows
-                        sm100::tma_load_3d(sW + (st * 2 + sl) * SLAB_BYTES, &tm_x, &bars[WFULL0 + st],
-                                           dv + sl * SLAB, i * BM, (int)fh);
+                    if (frame) {  // the frame's queries
+                        const long long f = fh % prm.F, chain = fh / prm.F;
+                        const int h = (int)(chain % prm.H), b = (int)(chain / prm.H);
+                        sm100::tma_load_4d(wst + sl * SLAB_BYTES, &tm_q, &bars[WFULL + st], sl * SLAB, h, i * BM,
+                                           (int)(b * prm.F + f));
+                    } else {  // W = columns dv .. dv + dk of the [Ub | W] rows
+                        sm100::tma_load_3d(wst + sl * SLAB_BYTES, &tm_x, &bars[WFULL + st], dv + sl * SLAB, i * BM,
+                                           (int)fh);
+                    }
                 }
             }
-            for (int i = (nblk >= 2 ? nblk - 2 : 0); ok && i < nblk; ++i)
-                ok = sm100::mbar_wait(&bars[WEMPTY0 + (i & 1)], (i >> 1) & 1, err);
+            // leave with no copy in flight (full-limit drain waits): the last NW tiles and the
+            // states loaded for the last two frame-heads
+            for (long long u = g > NW ? g - NW : 0; u < g; ++u)
+                sm100::mbar_wait(&bars[WFULL + (u % NW)], (uint32_t)((u / NW) & 1), err, sm100::kWaitLimitNs, true);
+            for (long long u = tsig > 2 ? tsig - 2 : 0; u < tsig; ++u)
+                sm100::mbar_wait(&bars[SIGFULL + (u & 1)], (uint32_t)((u >> 1) & 1), err, sm100::kWaitLimitNs, true);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t id = sm100::idesc_bf16(BM, dv, 0, 1);
-            bool ok = sm100::mbar_wait(&bars[SIGFULL], 0, err);
-            for (int i = 0; i < nblk && ok; ++i) {
-                const int st = i & 1;
+            bool ok = true;
+            for (long long g = 0; g < total && ok; ++g) {
+                const long long t = g / nblk;
+                const int i = (int)(g % nblk), st = (int)(g % NW), db = (int)(g & 1);
+                if (i == 0) ok = sm100::mbar_wait(&bars[SIGFULL + (t & 1)], (uint32_t)((t >> 1) & 1), err, wait_ns);
                 // the operand is ready when it has landed, or (query feature map) once the
                 // epilogue has normalised it in place
-                ok = sm100::mbar_wait(&bars[(normq ? QREADY0 : WFULL0) + st], (i >> 1) & 1, err);
-                if (ok && i >= 2) ok = sm100::mbar_wait(&bars[DEMPTY0 + st], ((i - 2) >> 1) & 1, err);
+                if (ok) ok = sm100::mbar_wait(&bars[(normq ? QREADY : WFULL) + st], (uint32_t)((g / NW) & 1), err, wait_ns);
+                if (ok && g >= 2) ok = sm100::mbar_wait(&bars[DEMPTY + db], (uint32_t)(((g >> 1) - 1) & 1), err, wait_ns);
                 if (!ok) break;
                 sm100::tc_fence_after();
                 const unsigned char *wt = sW + st * 2 * SLAB_BYTES;
+                const unsigned char *sg = sig_buf(t);
                 for (int ks = 0; ks < dk / 16; ++ks)
-                    sm100::mma_bf16_ss(t_d + st * 128, desc_kmajor(wt, ks, BM), desc_mnmajor(sSig, ks, dk), id,
+                    sm100::mma_bf16_ss(t_d + db * 128, desc_kmajor(wt, ks, BM), desc_mnmajor(sg, ks, dk), id,
                                        ks > 0);
-                sm100::mma_commit(&bars[DFULL0 + st]);
-                sm100::mma_commit(&bars[WEMPTY0 + st]);
+                sm100::mma_commit(&bars[DFULL + db]);
+                sm100::mma_commit(&bars[WEMPTY + st]);
+                if (i == nblk - 1) sm100::mma_commit(&bars[SIGEMPTY + (t & 1)]);
             }
+            sm100::mma_commit(&bars[DRAIN]);  // every product issued completes before TMEM is released
+            sm100::mbar_wait(&bars[DRAIN], 0u, err, sm100::kWaitLimitNs, true);
         }
     } else {
         const int q4 = warp & 3;
@@ -113,14 +151,15 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         bool ok = true;
         // query feature map of the frame-wise operator (SANA-WM summary, section 3.2, "Algebraic
-        // Stabilization for Spatial Token Explosion"): row r of block i's staged Q becomes
+        // Stabilization for Spatial Token Explosion"): row r of use g's staged Q becomes
         // max(RMSNorm(q) w, 0) in place before the product reads it
-        auto normalize = [&](int i) -> bool {
-            const int st = i & 1;
-            if (!sm100::mbar_wait(&bars[WFULL0 + st], (i >> 1) & 1, err)) return false;
+        auto normalize = [&](long long g) -> bool {
+            const int st = (int)(g % NW);
+            if (!sm100::mbar_wait(&bars[WFULL + st], (uint32_t)((g / NW) & 1), err, wait_ns)) return false;
+            unsigned char *wst = sW + st * 2 * SLAB_BYTES;
             float ss = 0.f;
             for (int sl = 0; sl < nslab_k; ++sl) {
-                const uint4 *rowp = reinterpret_cast<const uint4 *>(sW + (st * 2 + sl) * SLAB_BYTES + r * 128);
+                const uint4 *rowp = reinterpret_cast<const uint4 *>(wst + sl * SLAB_BYTES + r * 128);
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
                     const uint4 v = rowp[cc];
@@ -134,7 +173,7 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
             }
             const float inv = 1.f / sqrtf(ss / (float)dk + kRmsEps);
             for (int sl = 0; sl < nslab_k; ++sl) {
-                uint4 *rowp = reinterpret_cast<uint4 *>(sW + (st * 2 + sl) * SLAB_BYTES + r * 128);
+                uint4 *rowp = reinterpret_cast<uint4 *>(wst + sl * SLAB_BYTES + r * 128);
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
                     uint4 v = rowp[cc];
@@ -152,13 +191,17 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
                 }
             }
             sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(&bars[QREADY0 + st]);
+            sm100::mbar_arrive(&bars[QREADY + st]);
             return true;
         };
-        if (normq && nblk > 0) ok = normalize(0);
-        for (int i = 0; i < nblk && ok; ++i) {
-            if (normq && i + 1 < nblk && !(ok = normalize(i + 1))) break;
-            const int st = i & 1;
+        if (normq && total > 0) ok = normalize(0);
+        for (long long g = 0; g < total && ok; ++g) {
+            if (normq && g + 1 < total && !(ok = normalize(g + 1))) break;
+            const long long t = g / nblk;
+            const int i = (int)(g % nblk), db = (int)(g & 1);
+            const long long fh = fh_of(t);
+            const long long f = frame ? fh % prm.F : 0, chain = frame ? fh / prm.F : 0;
+            const int h = frame ? (int)(chain % prm.H) : 0, b = frame ? (int)(chain / prm.H) : 0;
             const int row = i * BM + r;
             const bool valid = row < L;
             // chunkwise: U = Ub - D over the row's [Ub | W]; frame-wise: o (+)= D
@@ -176,7 +219,7 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
             for (int c8 = 0; c8 < 16; ++c8)
                 ub[c8] = (valid && load_row && c8 < dv / 8) ? __ldg(reinterpret_cast<const uint4 *>(xrow) + c8)
                                                             : make_uint4(0, 0, 0, 0);
-            ok = sm100::mbar_wait(&bars[DFULL0 + st], (i >> 1) & 1, err);
+            ok = sm100::mbar_wait(&bars[DFULL + db], (uint32_t)((g >> 1) & 1), err, wait_ns);
             if (!ok) break;
             sm100::tc_fence_after();
 #pragma unroll
@@ -184,7 +227,7 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
                 const int c0 = 16 * j;
                 if (c0 >= dv) break;
                 float d[16];
-                sm100::tmem_ld16(t_d + st * 128 + lane_off + c0, d);
+                sm100::tmem_ld16(t_d + db * 128 + lane_off + c0, d);
                 sm100::tmem_ld_wait();
                 if (valid) {
                     uint4 out[2];
@@ -204,7 +247,7 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
                 }
             }
             sm100::tc_fence_before();
-            sm100::mbar_arrive(&bars[DEMPTY0 + st]);
+            sm100::mbar_arrive(&bars[DEMPTY + db]);
         }
     }
     sm100::tc_fence_before();
@@ -218,11 +261,13 @@ k_u_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtenso
 }  // namespace
 
 cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_q, const CUtensorMap &tm_sig,
-                        const UParams &prm, long long n_fh, cudaStream_t s) {
+                        const UParams &prm, long long n_fh, int num_sms, cudaStream_t s) {
     const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
     cudaError_t e = cudaFuncSetAttribute(k_u_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_u_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_x, tm_q, tm_sig, prm);
+    const long long grid = n_fh < num_sms ? n_fh : num_sms;
+    if (grid <= 0) return cudaSuccess;
+    k_u_tc<<<(unsigned)grid, kThreads, smem, s>>>(tm_x, tm_q, tm_sig, prm, n_fh);
     return cudaGetLastError();
 }
 

@@ -277,8 +277,9 @@ enum { GDN_QK_NORM_KEYS = 1, GDN_QK_NORM_QUERIES = 2 };
  * 4 scan over frames, 5 pseudo-values U, 6 output.  A path without a stage
  * reports 0 for it: the fp32 path folds 0, 1 into 2 and 5 into 6; the
  * frame-wise operator has only 3 (its per-frame maps), 4 and 6.  Work
- * outside the seven stages is not counted: the q/k prologue, and a reversed
- * or accumulating bf16 call's input reversal and final write of o. */
+ * outside the seven stages is not counted: the q/k prologue pass (where the
+ * kernels do not apply it themselves) and a reversed bf16 call's copies of
+ * its inputs in reversed token order. */
 enum { GDN_NUM_STAGES = 7 };
 
 int gdn_fwd_ex(const gdn_args *a);

@@ -1,11 +1,11 @@
 """A bounded device-side wait that gives up (no GPU fault, trap or hang).
 
 The debug switch GDN_DEBUG_DROP_SIGNAL=1 makes the diagonal-inverse kernel
-withhold its first load, so the Gram issuer's wait on it can never complete;
+withhold its first block's Gram product, so the wait on it can never complete;
 GDN_DEBUG_WAIT_LIMIT_US shortens the waits' limit from 2 s to 1 ms.  The
-waiting thread records a timeout in the pass's error word, every other role
-of the kernel sees it and leaves after draining what it has in flight, TMEM is
-released, and the later kernels of the pass skip their work.  The host then
+waiting thread records a timeout in the pass's error word, the block's other
+threads skip their work, TMEM is released, and the later kernels of the pass
+skip theirs.  The host then
 learns it through the status word (asynchronous calls) or GDN_ERR_TIMEOUT
 (synchronous calls), and the next call on the same context is correct.
 """
