@@ -357,6 +357,10 @@ int run(const gdn_args &a) noexcept {
             for (int i = 0; i <= GDN_NUM_STAGES; ++i) cudaEventDestroy(ev[i]);
         }
         if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+        if (timed_out == 2) {  // sm100::kErrSmemAlign
+            set_err("a kernel's dynamic shared memory did not start on a 1024-byte boundary; it did no work");
+            return GDN_ERR_CUDA;
+        }
         if (timed_out) {
             set_err("a bounded device-side wait gave up (error word %d)", timed_out);
             return GDN_ERR_TIMEOUT;

@@ -26,7 +26,7 @@ namespace {
 inline int cf_stride(int L) { return (L + 3) & ~3; }
 
 struct TcLayout {
-    size_t G, CF, GCT, Tinv, X, M, Mimg, N, Sig, SigB, U, err;
+    size_t G, CF, Tinv, X, M, Mimg, N, Sig, SigB, U, err;
     size_t Qr, Kr, Vr, Ar, Br;  // token-reversed input copies: reversed calls only (0 bytes otherwise)
     size_t total;
 };
@@ -38,7 +38,6 @@ TcLayout tc_layout(const Problem &p) {
     size_t off = 0;
     lay.G = off;    off += align256(sizeof(float) * nfh * (size_t)cf_stride(p.L));
     lay.CF = off;   off += align256(sizeof(float) * nfh * (size_t)cf_stride(p.L));
-    lay.GCT = off;  off += align256(sizeof(float) * nfh * (size_t)((p.L + 127) / 128) * 256);
     lay.Tinv = off; off += align256(2 * nfh * (size_t)((p.L + 127) / 128) * 128 * 128);
     lay.X = off;    off += align256(2 * nfh * p.L * nc);
     // the scan takes M as the tensor-core scan's operand images (or fp32 for the CUDA-core one)
@@ -122,10 +121,8 @@ bool map_rows(CUtensorMap *m, const void *x, long long nfh, int rows, int cols, 
 // G = per-frame inclusive prefix of log alpha; CF = e^{a(s) - G_s} with a(s)
 // = G at the last token of s's 64-token tile (<= 1): the column half of the
 // split decay factor e^{G_r - G_s} = e^{G_r - a} e^{a - G_s}.
-// GCT = the same G and CF regrouped per 128-token tile, [n_fh][tile][G[128], CF[128]]
-// (zeros past the frame), so one TMA box delivers both for a tile.
 __global__ void __launch_bounds__(256)
-gate_prefix_kernel(Problem p, float *__restrict__ G, float *__restrict__ CF, float *__restrict__ GCT) {
+gate_prefix_kernel(Problem p, float *__restrict__ G, float *__restrict__ CF) {
     extern __shared__ __align__(16) unsigned char smem[];
     const long long fh = blockIdx.x;
     const long long f = fh % p.F, chain = fh / p.F;
@@ -135,19 +132,10 @@ gate_prefix_kernel(Problem p, float *__restrict__ G, float *__restrict__ CF, flo
     float *sScr = sB + p.L;
     frame_gates<float>(p, b, h, f, sG, sB, sScr);
     const int cfs = (p.L + 3) & ~3;  // cf_stride(L): G and CF rows start on 16-byte boundaries
-    const int nt = (p.L + 127) / 128;
-    float *gct = GCT + fh * (long long)nt * 256;
-    for (int i = threadIdx.x; i < nt * 128; i += blockDim.x) {
-        float g = 0.f, cf = 0.f;
-        if (i < p.L) {
-            const int end = min((i / 64) * 64 + 63, p.L - 1);
-            g = sG[i];
-            cf = __expf(sG[end] - sG[i]);
-            G[fh * cfs + i] = g;
-            CF[fh * cfs + i] = cf;
-        }
-        gct[(i / 128) * 256 + (i & 127)] = g;
-        gct[(i / 128) * 256 + 128 + (i & 127)] = cf;
+    for (int i = threadIdx.x; i < p.L; i += blockDim.x) {
+        const int end = min((i / 64) * 64 + 63, p.L - 1);
+        G[fh * cfs + i] = sG[i];
+        CF[fh * cfs + i] = __expf(sG[end] - sG[i]);
     }
 }
 
@@ -177,7 +165,6 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     const int nblk = (p.L + tc::BM - 1) / tc::BM;
     float *G = (float *)(base + lay.G);
     float *CF = (float *)(base + lay.CF);
-    float *GCT = (float *)(base + lay.GCT);
     __nv_bfloat16 *X = (__nv_bfloat16 *)(base + lay.X);
     float *Mb = (float *)(base + lay.M), *Nb = (float *)(base + lay.N), *Sig = (float *)(base + lay.Sig);
     __nv_bfloat16 *SigB = (__nv_bfloat16 *)(base + lay.SigB);
@@ -187,13 +174,10 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
 
     __nv_bfloat16 *Tinv = (__nv_bfloat16 *)(base + lay.Tinv);
     const int nc = p.dk + p.dv;
-    CUtensorMap tm_q, tm_k, tm_u128, tm_sig, tm_k64, tm_x, tm_t, tm_x128, tm_g128, tm_cf128, tm_gct;
-    const int nt128 = (p.L + 127) / 128;
+    CUtensorMap tm_q, tm_k, tm_u128, tm_sig, tm_t, tm_x128, tm_g128, tm_cf128;
     if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
         !map_rows(&tm_u128, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
-        !map_tokens(&tm_k64, p.k, p, p.dk, 64) || !map_rows(&tm_x, X, nfh, p.L, nc, 64) ||
         !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128) || !map_rows(&tm_x128, X, nfh, p.L, nc, 128) ||
-        !map_f32_rows(&tm_gct, GCT, nfh * nt128, 256, 256, 256) ||
         !map_f32_rows(&tm_g128, G, nfh, p.L, cf_stride(p.L), 128) ||
         !map_f32_rows(&tm_cf128, CF, nfh, p.L, cf_stride(p.L), 128))
         return cudaErrorInvalidValue;
@@ -215,26 +199,22 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
         (e = cudaFuncSetAttribute(gate_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm)))
         return e;
     if ((e = mark(ev, 0, s))) return e;
-    gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF, GCT);
+    gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 1, s))) return e;
     if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
                                      nfh, err, wait_ns, debug_drop_signal(), s)))
         return e;
     if ((e = mark(ev, 2, s))) return e;
+    // the intra-frame solve also forms the frame's transition: fp32 M for the CUDA-core scan (and the
+    // segment-map scan), the operand images for the tensor-core one
     tc::IntraParams ip;
-    ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.k = (const __nv_bfloat16 *)p.k; ip.X = X;
+    ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.X = X;
+    ip.M = (!scan_tc || p.map_out) ? Mb : nullptr; ip.Mimg = scan_tc ? Mimg : nullptr; ip.N = Nb;
     ip.L = p.L; ip.dk = p.dk; ip.dv = p.dv; ip.H = p.H; ip.nblk = nblk;
-    ip.F = p.F; ip.T = p.T; ip.err = err;
-    if ((e = tc::launch_intra_tc(tm_k, tm_x, tm_t, tm_gct, tm_x128, ip, nfh, s))) return e;
+    ip.F = p.F; ip.T = p.T; ip.err = err; ip.wait_ns = wait_ns;
+    if ((e = tc::launch_intra_tc(tm_k, tm_t, tm_x128, ip, nfh, s))) return e;
     if ((e = mark(ev, 3, s))) return e;
-    tc::TransParams tp;
-    // fp32 M for the CUDA-core scan (also the segment-map scan); the operand images for the tensor-core one
-    tp.G = G; tp.M = (!scan_tc || p.map_out) ? Mb : nullptr; tp.Mimg = scan_tc ? Mimg : nullptr; tp.N = Nb;
-    tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
-    tp.frame = 0; tp.beta = p.beta; tp.gamma = nullptr; tp.T = p.T;
-    tp.norm_k = 0; tp.k_w = nullptr; tp.k_post = 1.f; tp.wait_ns = wait_ns;
-    if ((e = tc::launch_transition_tc(tm_k64, tm_x, tm_x, tp, nfh, num_sms, s))) return e;
     if (p.map_out && (e = simt_segment_map(p, Mb, Nb, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
     if (p.phase == GDN_PHASE_PREPARE) {

@@ -23,8 +23,10 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
-// Error word written when a bounded wait gives up (first writer wins).
-enum : int { kErrNone = 0, kErrTimeout = 1 };
+// Error word (first writer wins): a bounded wait that gave up, or a kernel whose dynamic
+// shared memory did not start on the 1024-byte boundary its swizzled tiles need (it then
+// does no work).
+enum : int { kErrNone = 0, kErrTimeout = 1, kErrSmemAlign = 2 };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 // ------------------------------------------------------------------ mbarrier
