@@ -174,8 +174,8 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
 
     __nv_bfloat16 *Tinv = (__nv_bfloat16 *)(base + lay.Tinv);
     const int nc = p.dk + p.dv;
-    CUtensorMap tm_q, tm_k, tm_u128, tm_sig, tm_t, tm_x128, tm_g128, tm_cf128;
-    if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) ||
+    CUtensorMap tm_q, tm_k, tm_v, tm_u128, tm_sig, tm_t, tm_x128, tm_g128, tm_cf128;
+    if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) || !map_tokens(&tm_v, p.v, p, p.dv) ||
         !map_rows(&tm_u128, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
         !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128) || !map_rows(&tm_x128, X, nfh, p.L, nc, 128) ||
         !map_f32_rows(&tm_g128, G, nfh, p.L, cf_stride(p.L), 128) ||
@@ -209,11 +209,11 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     // the intra-frame solve also forms the frame's transition: fp32 M for the CUDA-core scan (and the
     // segment-map scan), the operand images for the tensor-core one
     tc::IntraParams ip;
-    ip.G = G; ip.beta = p.beta; ip.v = (const __nv_bfloat16 *)p.v; ip.X = X;
+    ip.G = G; ip.beta = p.beta; ip.X = X;
     ip.M = (!scan_tc || p.map_out) ? Mb : nullptr; ip.Mimg = scan_tc ? Mimg : nullptr; ip.N = Nb;
     ip.L = p.L; ip.dk = p.dk; ip.dv = p.dv; ip.H = p.H; ip.nblk = nblk;
     ip.F = p.F; ip.T = p.T; ip.err = err; ip.wait_ns = wait_ns;
-    if ((e = tc::launch_intra_tc(tm_k, tm_t, tm_x128, ip, nfh, s))) return e;
+    if ((e = tc::launch_intra_tc(tm_k, tm_v, tm_t, tm_x128, ip, nfh, s))) return e;
     if ((e = mark(ev, 3, s))) return e;
     if (p.map_out && (e = simt_segment_map(p, Mb, Nb, s))) return e;
     if ((e = mark(ev, 4, s))) return e;

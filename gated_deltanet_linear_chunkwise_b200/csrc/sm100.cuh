@@ -179,6 +179,13 @@ __device__ __forceinline__ void tma_load_4d_hint(void *smem_dst, const void *tma
         : "memory");
 }
 
+// Bring a 4-D tile into L2 ahead of its load (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const void *tmap, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(tmap), "r"(c0),
+                 "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_store_3d_hint(const void *tmap, const void *smem_src, int c0, int c1, int c2,
                                                   uint64_t policy) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;" ::"l"(

@@ -47,7 +47,7 @@ constexpr int TILE = 2 * SLAB_BYTES;         // 128 rows x 2 slabs (K_i or T_ii)
 constexpr int WIDE = 4 * SLAB_BYTES;         // 128 rows x 4 slabs (Y_i / X_i, H)
 
 enum Bar {
-    ACCFULL = 0, YFULL, XFULL, XSTAGED, UFULL, HREADY, TFULL, TFREE, STFREE, DRAIN,
+    ACCFULL = 0, YFULL, XFULL, XSTAGED, UFULL, HREADY, TFULL, TFREE, VFULL, DRAIN,
     KFULL, KEMPTY = KFULL + 2, NBAR = KEMPTY + 2
 };
 
@@ -71,9 +71,30 @@ __device__ __forceinline__ uint32_t sw_offset(int c, int r) {
     return (uint32_t)((c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
 }
 
+// Walks n16 16-column chunks of this warp's TMEM lanes from taddr, loading each chunk while
+// fn(j, chunk) works on the one before it (tcgen05.wait::ld waits for every load in flight,
+// so one load is ahead at a time).  Warp-uniform: every lane takes part in the loads.
+template <typename F>
+__device__ __forceinline__ void tmem_walk16(uint32_t taddr, int n16, F &&fn) {
+    float buf[2][16];
+    sm100::tmem_ld16(taddr, buf[0]);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        if (j >= n16) break;
+        sm100::tmem_ld_wait();
+        if (j + 1 < n16) sm100::tmem_ld16(taddr + 16 * (j + 1), buf[(j + 1) & 1]);
+        fn(j, buf[j & 1]);
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float *x) {
+    return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_t,
-           const __grid_constant__ CUtensorMap tm_xs, const IntraParams prm) {
+k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+           const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_xs,
+           const IntraParams prm) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
     const long long fh = blockIdx.x;
@@ -93,6 +114,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     int *err = prm.err;
     const uint64_t wait_ns = prm.wait_ns;
     const int nslab_k = (dk + SLAB - 1) / SLAB;
+    const int nslab_v = (dv + SLAB - 1) / SLAB;
     const int nslab_x = (nc + SLAB - 1) / SLAB;
 
     if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
@@ -125,17 +147,20 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         // K_j (double-buffered: once block j-2's Kh^T X has read its buffer), T_j (once T_{j-1}
-        // Y_{j-1} has read the tile), and the store of each staged X_j.
+        // Y_{j-1} has read the tile), V_j into the staging tile's first slabs (once X_{j-1} has
+        // been read there by its store and by Kh^T X_{j-1}), and the store of each staged X_j.
         if (lane == 0) {
             sm100::tma_prefetch_desc(&tm_k);
+            sm100::tma_prefetch_desc(&tm_v);
             sm100::tma_prefetch_desc(&tm_t);
             sm100::tma_prefetch_desc(&tm_xs);
             // L2 policies: K and T are read once here; X is read again by the next stages
             const uint64_t once = sm100::policy_evict_first(), keep = sm100::policy_evict_last();
-            int kj = 0, tj = 0, sx = 0;
+            int kj = 0, tj = 0, vj = 0, sx = 0;
+            for (int sl = 0; sl < nslab_v; ++sl) sm100::tma_prefetch_l2_4d(&tm_v, sl * SLAB, h, 0, bf);
             bool ok = true;
             sm100::Spin spin(wait_ns);
-            while (ok && (kj < nblk || tj < nblk || sx < nblk)) {
+            while (ok && (kj < nblk || tj < nblk || vj < nblk || sx < nblk)) {
                 bool prog = false;
                 if (kj < nblk && (kj < 2 || sm100::mbar_test(&bars[KEMPTY + (kj & 1)], ((kj >> 1) - 1) & 1))) {
                     uint64_t *bar = &bars[KFULL + (kj & 1)];
@@ -154,6 +179,17 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     ++tj;
                     prog = true;
                 }
+                if (vj < nblk && (vj == 0 || (sx >= vj && sm100::mbar_test(&bars[UFULL], (vj - 1) & 1)))) {
+                    sm100::mbar_arrive_expect_tx(&bars[VFULL], (uint32_t)(nslab_v * SLAB_BYTES));
+                    for (int sl = 0; sl < nslab_v; ++sl)
+                        sm100::tma_load_4d_hint(sST + sl * SLAB_BYTES, &tm_v, &bars[VFULL], sl * SLAB, h, vj * BM, bf,
+                                                once);
+                    if (vj + 1 < nblk)  // the next block's values into L2 meanwhile
+                        for (int sl = 0; sl < nslab_v; ++sl)
+                            sm100::tma_prefetch_l2_4d(&tm_v, sl * SLAB, h, (vj + 1) * BM, bf);
+                    ++vj;
+                    prog = true;
+                }
                 // store the staged X_sx (rows past the frame, columns past d_v + d_k clipped); the
                 // staging tile takes Y_{sx+1} once the store has read it (and Kh^T X_sx has, too)
                 if (sx < nblk && sm100::mbar_test(&bars[XSTAGED], sx & 1)) {
@@ -161,18 +197,23 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                         sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, sx * BM, (int)fh, keep);
                     sm100::bulk_commit();
                     sm100::bulk_wait_read0();
-                    sm100::mbar_arrive(&bars[STFREE]);
                     ++sx;
                     prog = true;
                 }
-                if (prog) spin.reset();
-                else if (!spin.tick(err)) ok = false;
+                if (prog) {
+                    spin.reset();
+                } else if (!spin.tick(err)) {
+                    ok = false;
+                } else {
+                    __nanosleep(64);  // leave the issue slots to the epilogue warps of this sub-partition
+                }
             }
             sm100::bulk_wait0();  // leave with no store in flight
             if (!ok) {  // and no load in flight (full-limit drain waits)
                 for (int j = kj > 2 ? kj - 2 : 0; j < kj; ++j)
                     sm100::mbar_wait(&bars[KFULL + (j & 1)], (uint32_t)((j >> 1) & 1), err, sm100::kWaitLimitNs, true);
                 if (tj > 0) sm100::mbar_wait(&bars[TFULL], (uint32_t)((tj - 1) & 1), err, sm100::kWaitLimitNs, true);
+                if (vj > 0) sm100::mbar_wait(&bars[VFULL], (uint32_t)((vj - 1) & 1), err, sm100::kWaitLimitNs, true);
             }
         }
     } else if (warp == 1) {
@@ -223,7 +264,6 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         const int r = q4 * 32 + lane;  // block row (token); for H, the key dimension
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
-        const uint64_t once = sm100::policy_evict_first();
         // G at the anchor of block j >= 1 (the last token before it; the frame's last token for j = nblk)
         auto anchor = [&](int j) -> float { return Gf[min(j * BM, L) - 1]; };
         // this row's G and beta, read one block ahead
@@ -233,20 +273,9 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             g = ok_row ? Gf[rw] : 0.f;
             bb = ok_row ? prm.beta[((long long)b * prm.T + f * L + rw) * prm.H + h] : 0.f;
         };
-        // half 0: this row's values for block i (read once: evict first)
-        auto load_v = [&](int i, uint4 (&x)[16]) {
-            const int rw = i * BM + r;
-            const bool ok_row = half == 0 && i < nblk && rw < L;
-            const uint4 *vp = reinterpret_cast<const uint4 *>(prm.v + (((long long)b * prm.T + f * L + rw) * prm.H + h) * dv);
-#pragma unroll
-            for (int c8 = 0; c8 < 16; ++c8)
-                x[c8] = (ok_row && c8 < dv / 8) ? sm100::ld_nc_hint(vp + c8, once) : make_uint4(0, 0, 0, 0);
-        };
         bool ok = true;
         float G_next, be_next;
         row_gates(0, G_next, be_next);
-        uint4 vrow[16];
-        load_v(0, vrow);
         float an0 = 0.f, an1 = anchor(1), an2 = nblk >= 2 ? anchor(2) : 0.f;
         for (int i = 0; i < nblk && ok; ++i) {
             const int row = i * BM + r;
@@ -260,82 +289,66 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             unsigned char *kt = sK + (i & 1) * TILE;
 
             // ---- Y_i = R_i - diag(beta e^{G_r - G_{a_i}}) K_i H_i -> staging (MN-major: row = K index
-            //      of T_ii Y_i); half 1 also turns its K_i row into Kh_i in place
-            if (i > 0) ok = sm100::mbar_wait(&bars[ACCFULL], (uint32_t)((i - 1) & 1), err, wait_ns) &&
-                            sm100::mbar_wait(&bars[STFREE], (uint32_t)((i - 1) & 1), err, wait_ns);
-            if (ok) ok = sm100::mbar_wait(&bars[KFULL + (i & 1)], (uint32_t)((i >> 1) & 1), err, wait_ns);
+            //      of T_ii Y_i)
+            if (i > 0) ok = sm100::mbar_wait(&bars[ACCFULL], (uint32_t)((i - 1) & 1), err, wait_ns);
+            if (ok) ok = sm100::mbar_wait(&bars[VFULL], (uint32_t)(i & 1), err, wait_ns) &&
+                         sm100::mbar_wait(&bars[KFULL + (i & 1)], (uint32_t)((i >> 1) & 1), err, wait_ns);
             if (!ok) break;
             sm100::tc_fence_after();
             const float rf = (valid && i > 0) ? be * __expf(Gr - aI) : 0.f;
             const int rlen = half ? dk : dv, c_base = half ? dv : 0;
+            const int n16 = rlen >> 4;  // the half's 16-column chunks (d_v and d_k are multiples of 16)
             const float rs = half ? be * __expf(Gr) : be;
-            const float ksc = valid ? __expf(aI1 - Gr) : 0.f;  // Kh_i row factor
+            // y = rs x - rf acc over 8 columns from c, x this row's v (landed in the staging tile,
+            // overwritten in place) or k
+            auto build = [&](int c, const float *acc) {
+                const uint4 xin = *reinterpret_cast<const uint4 *>((half ? kt : sST) + sw_offset(c, r));
+                const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&xin);
+                float y[8];
 #pragma unroll
-            for (int j2 = 0; j2 < 4; ++j2) {  // two 16-column loads per wait
-                if (32 * j2 >= rlen) break;
-                float acc[2][16];
-                if (i > 0) {  // the second load may read past the half's columns, inside the product
-                    sm100::tmem_ld16(t_p + lane_off + c_base + 32 * j2, acc[0]);
-                    sm100::tmem_ld16(t_p + lane_off + c_base + 32 * j2 + 16, acc[1]);
-                    sm100::tmem_ld_wait();
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) acc[0][e] = acc[1][e] = 0.f;
+                for (int e = 0; e < 4; ++e) {
+                    const float2 fx = __bfloat1622float2(x2[e]);
+                    y[2 * e] = fmaf(rs, fx.x, -rf * acc[2 * e]);
+                    y[2 * e + 1] = fmaf(rs, fx.y, -rf * acc[2 * e + 1]);
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = 32 * j2 + 8 * u;
-                    if (c >= rlen) break;
-                    uint4 xin;
-                    if (half == 0) {
-                        xin = vrow[4 * j2 + u];
-                    } else {
-                        xin = *reinterpret_cast<const uint4 *>(kt + sw_offset(c, r));
-                    }
-                    const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&xin);
-                    float y[8];
-                    uint32_t kh[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 fx = __bfloat1622float2(x2[e]);
-                        y[2 * e] = rs * fx.x - rf * acc[u >> 1][(u & 1) * 8 + 2 * e];
-                        y[2 * e + 1] = rs * fx.y - rf * acc[u >> 1][(u & 1) * 8 + 2 * e + 1];
-                        kh[e] = pack_bf16(ksc * fx.x, ksc * fx.y);
-                    }
-                    const uint4 val = valid ? make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]),
-                                                         pack_bf16(y[4], y[5]), pack_bf16(y[6], y[7]))
-                                            : make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(sST + sw_offset(c_base + c, r)) = val;
-                    if (half == 1) *reinterpret_cast<uint4 *>(kt + sw_offset(c, r)) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-                }
+                *reinterpret_cast<uint4 *>(sST + sw_offset(c_base + c, r)) = valid ? pack8(y) : make_uint4(0, 0, 0, 0);
+            };
+            if (i > 0) {
+                tmem_walk16(t_p + lane_off + c_base, n16, [&](int j, const float (&acc)[16]) {
+                    build(16 * j, acc);
+                    build(16 * j + 8, acc + 8);
+                });
+            } else {
+                const float zero[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                for (int c = 0; c < rlen; c += 8) build(c, zero);
             }
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();
             sm100::mbar_arrive(&bars[YFULL]);
-            load_v(i + 1, vrow);  // the next block's values, a whole block ahead of their use
+            if (half == 1) {  // off the chain: K_i becomes Kh_i in place (read by Kh_i^T X_i after X_i is staged)
+                const float ksc = valid ? __expf(aI1 - Gr) : 0.f;
+                for (int c = 0; c < dk; c += 8) {
+                    uint4 *kp = reinterpret_cast<uint4 *>(kt + sw_offset(c, r));
+                    uint4 kv = *kp;
+                    __nv_bfloat162 *k2 = reinterpret_cast<__nv_bfloat162 *>(&kv);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 fk = __bfloat1622float2(k2[e]);
+                        k2[e] = __floats2bfloat162_rn(ksc * fk.x, ksc * fk.y);
+                    }
+                    *kp = kv;
+                }
+            }
 
             // ---- X_i = T_ii Y_i -> bf16 staging over Y_i (half 0 the Ub columns, half 1 the W columns)
             ok = sm100::mbar_wait(&bars[XFULL], (uint32_t)(i & 1), err, wait_ns);
             if (!ok) break;
             sm100::tc_fence_after();
-            const int c_lo = half ? dv : 0, c_hi = half ? nc : dv;
-            // two 16-column loads per wait (the second may read past c_hi, inside the
-            // product's 256 columns, and is then not stored)
-            for (int c32 = c_lo; c32 < c_hi; c32 += 32) {
-                float x[2][16];
-                sm100::tmem_ld16(t_p + lane_off + c32, x[0]);
-                sm100::tmem_ld16(t_p + lane_off + c32 + 16, x[1]);
-                sm100::tmem_ld_wait();
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    if (c32 + 16 * h2 >= c_hi) break;
-#pragma unroll
-                    for (int u = 0; u < 2; ++u)
-                        *reinterpret_cast<uint4 *>(sST + sw_offset(c32 + 16 * h2 + 8 * u, r)) = make_uint4(
-                            pack_bf16(x[h2][8 * u], x[h2][8 * u + 1]), pack_bf16(x[h2][8 * u + 2], x[h2][8 * u + 3]),
-                            pack_bf16(x[h2][8 * u + 4], x[h2][8 * u + 5]), pack_bf16(x[h2][8 * u + 6], x[h2][8 * u + 7]));
-                }
-            }
+            const int c_lo = half ? dv : 0;
+            tmem_walk16(t_p + lane_off + c_lo, n16, [&](int j, const float (&x)[16]) {
+                *reinterpret_cast<uint4 *>(sST + sw_offset(c_lo + 16 * j, r)) = pack8(x);
+                *reinterpret_cast<uint4 *>(sST + sw_offset(c_lo + 16 * j + 8, r)) = pack8(x + 8);
+            });
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();
             sm100::mbar_arrive(&bars[XSTAGED]);
@@ -347,26 +360,14 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::tc_fence_after();
             if (i + 1 < nblk) {
                 const float gam = __expf(aI2 - aI1);
-                for (int c32 = c_lo; c32 < c_hi; c32 += 32) {
-                    float x[2][16];
-                    sm100::tmem_ld16(t_h + lane_off + c32, x[0]);
-                    sm100::tmem_ld16(t_h + lane_off + c32 + 16, x[1]);
-                    sm100::tmem_ld_wait();
+                tmem_walk16(t_h + lane_off + c_lo, n16, [&](int j, const float (&x)[16]) {
+                    *reinterpret_cast<uint4 *>(sH + sw_offset(c_lo + 16 * j, r)) = pack8(x);
+                    *reinterpret_cast<uint4 *>(sH + sw_offset(c_lo + 16 * j + 8, r)) = pack8(x + 8);
+                    uint32_t sc[16];
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        if (c32 + 16 * h2 >= c_hi) break;
-#pragma unroll
-                        for (int u = 0; u < 2; ++u)
-                            *reinterpret_cast<uint4 *>(sH + sw_offset(c32 + 16 * h2 + 8 * u, r)) = make_uint4(
-                                pack_bf16(x[h2][8 * u], x[h2][8 * u + 1]), pack_bf16(x[h2][8 * u + 2], x[h2][8 * u + 3]),
-                                pack_bf16(x[h2][8 * u + 4], x[h2][8 * u + 5]),
-                                pack_bf16(x[h2][8 * u + 6], x[h2][8 * u + 7]));
-                        uint32_t sc[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) sc[e] = __float_as_uint(gam * x[h2][e]);
-                        sm100::tmem_st16(t_h + lane_off + c32 + 16 * h2, sc);
-                    }
-                }
+                    for (int e = 0; e < 16; ++e) sc[e] = __float_as_uint(gam * x[e]);
+                    sm100::tmem_st16(t_h + lane_off + c_lo + 16 * j, sc);
+                });
                 sm100::tmem_st_wait();
                 sm100::tc_fence_before();
                 sm100::fence_proxy_async_smem();
@@ -380,6 +381,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 unsigned char *img = prm.Mimg ? reinterpret_cast<unsigned char *>(prm.Mimg) +
                                                     fh * (long long)(2 * nslab * dk * 128)
                                               : nullptr;
+                const int c_hi = c_lo + rlen;
                 for (int c16 = c_lo; c16 < c_hi; c16 += 16) {  // dv is a multiple of 16
                     float v[16];
                     sm100::tmem_ld16(t_h + lane_off + c16, v);
@@ -430,12 +432,12 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
 }  // namespace
 
-cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_t, const CUtensorMap &tm_xs,
-                            const IntraParams &prm, long long n_fh, cudaStream_t s) {
+cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const CUtensorMap &tm_t,
+                            const CUtensorMap &tm_xs, const IntraParams &prm, long long n_fh, cudaStream_t s) {
     const size_t smem = Smem::END;
     cudaError_t e = cudaFuncSetAttribute(k_intra_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_t, tm_xs, prm);
+    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_v, tm_t, tm_xs, prm);
     return cudaGetLastError();
 }
 
