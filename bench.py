@@ -41,10 +41,11 @@ def kernel_work(L, dk, dv, BM=128):
       gates        G and cf of every token: read alpha, write G, cf (fp32)
       diag_inverse Gram of each 128-row diagonal block (lower half) and its
                    unit triangular inverse (n^3 / 3)
-      intra        off-diagonal S = K_i K_j^T and P X_j over the 128-column
-                   blocks before each row's block, plus the lower-triangular
-                   T_ii Y_i
-      transition   Kt^T [Ub | W]
+      intra        the triangular solve's off-diagonal part (S = K_i K_j^T and
+                   P X_j over the 128-column blocks before each row's block)
+                   and the lower-triangular T_ii Y_i, plus the frame's
+                   transition Kt^T [Ub | W]: the intra kernel forms both
+      transition   (no separate kernel in the chunked pass)
       scan         Sig M + N per frame (fp32 M, N in; fp32 + bf16 Sig out)
       u            W Sig
       output       masked Q K^T (lower triangle incl. diagonal), its product
@@ -58,8 +59,9 @@ def kernel_work(L, dk, dv, BM=128):
     return {
         "gates": (0, 12 * L),
         "diag_inverse": (sum(n * n * dk + n ** 3 // 3 for n in blk), 2 * L * dk + 2 * L * BM),
-        "intra": (2 * off * (dk + nc) + 2 * tri * nc, 2 * L * (dk + dv) + 2 * L * nc),
-        "transition": (2 * L * dk * nc, 2 * L * dk + 2 * L * nc + 4 * dk * nc),
+        "intra": (2 * off * (dk + nc) + 2 * tri * nc + 2 * L * dk * nc,
+                  2 * L * (dk + dv) + 2 * L * nc + 4 * dk * nc),
+        "transition": (0, 0),
         "scan": (2 * dk * dk * dv, 4 * dk * dk + 4 * dk * dv + 6 * dk * dv),
         "u": (2 * L * dk * dv, 2 * L * dk + 2 * dk * dv + 4 * L * dv),
         "output": (tri * 2 * (dk + dv) + 2 * L * dk * dv, 2 * L * (dk + dk + dv + dv) + 2 * dk * dv),
@@ -79,8 +81,7 @@ def bytes_alg(B, T, H, dk, dv, elem=2):
 # of the short-clip case (420 frame-heads, L = 880, d_k = d_v = 112; profiles/ holds the
 # summary and the command).  Traffic grows with the frame-heads processed, so a launch's
 # figure is this times its frame-head count; other shapes report null.
-DRAM_BYTES_PER_FH = {"intra": (334.5088e6 + 136.193024e6) / 420,
-                     "output": (467.891712e6 + 72.675328e6) / 420}
+DRAM_BYTES_PER_FH = {}
 TRAFFIC_SHAPE = (880, 112, 112)
 
 
@@ -549,8 +550,9 @@ def main():
                                                         if pk["bf16_tflops_sustained"] else None)},
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            # one kernel per stage: gates, diagonal inverses, intra, transition, scan, U, output
-            "gpu_launches": NUM_STAGES * args.steps,
+            # one kernel per stage that runs: gates, diagonal inverses, intra (with the
+            # transition), scan, U, output
+            "gpu_launches": 6 * args.steps,
             "bidirectional": {"ms_per_pass": bidir_ms, "tokens_per_s": tokens / (bidir_ms * 1e-3),
                               "what": "forward + reversed scan summed into o (not the timed metric)"},
             "framewise": dict(framewise_line(B * world, T, H, dk, dv, L, fw_ms, fw_stage, pk, STAGES),

@@ -47,7 +47,7 @@ constexpr int TILE = 2 * SLAB_BYTES;         // 128 rows x 2 slabs (K_i or T_ii)
 constexpr int WIDE = 4 * SLAB_BYTES;         // 128 rows x 4 slabs (Y_i / X_i, H)
 
 enum Bar {
-    ACCFULL = 0, YFULL, XFULL, XSTAGED, UFULL, HREADY, TFULL, TFREE, VFULL, DRAIN,
+    ACCFULL = 0, YFULL, XFULL, XSTG0, XSTG1, UFULL, HREADY, TFULL, TFREE, VFULL, DRAIN,
     KFULL, KEMPTY = KFULL + 2, NBAR = KEMPTY + 2
 };
 
@@ -87,6 +87,21 @@ __device__ __forceinline__ void tmem_walk16(uint32_t taddr, int n16, F &&fn) {
     }
 }
 
+// Packed fp32 pairs (lane 0 in the low word).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ __forceinline__ uint4 pack8(const float *x) {
     return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
 }
@@ -124,7 +139,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i)
-            sm100::mbar_init(&bars[i], (i == YFULL || i == XSTAGED || i == HREADY) ? kEpi : 1);
+            sm100::mbar_init(&bars[i], (i == YFULL || i == HREADY) ? kEpi : (i == XSTG0 || i == XSTG1) ? kEpi / 2 : 1);
         sm100::fence_barrier_init();
     }
     if (warp == 1) {
@@ -156,11 +171,14 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::tma_prefetch_desc(&tm_xs);
             // L2 policies: K and T are read once here; X is read again by the next stages
             const uint64_t once = sm100::policy_evict_first(), keep = sm100::policy_evict_last();
-            int kj = 0, tj = 0, vj = 0, sx = 0;
+            int kj = 0, tj = 0, vj = 0;
+            const int nsA = dv / SLAB;
+            const bool v_shares = (dv % SLAB) != 0;
+            int sa = 0, sb = 0;
             for (int sl = 0; sl < nslab_v; ++sl) sm100::tma_prefetch_l2_4d(&tm_v, sl * SLAB, h, 0, bf);
             bool ok = true;
             sm100::Spin spin(wait_ns);
-            while (ok && (kj < nblk || tj < nblk || vj < nblk || sx < nblk)) {
+            while (ok && (kj < nblk || tj < nblk || vj < nblk || sb < nblk)) {
                 bool prog = false;
                 if (kj < nblk && (kj < 2 || sm100::mbar_test(&bars[KEMPTY + (kj & 1)], ((kj >> 1) - 1) & 1))) {
                     uint64_t *bar = &bars[KFULL + (kj & 1)];
@@ -179,7 +197,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     ++tj;
                     prog = true;
                 }
-                if (vj < nblk && (vj == 0 || (sx >= vj && sm100::mbar_test(&bars[UFULL], (vj - 1) & 1)))) {
+                if (vj < nblk && (vj == 0 || (sa >= vj && sb >= vj - 1 && (!v_shares || sb >= vj) &&
+                                              sm100::mbar_test(&bars[UFULL], (vj - 1) & 1)))) {
                     sm100::mbar_arrive_expect_tx(&bars[VFULL], (uint32_t)(nslab_v * SLAB_BYTES));
                     for (int sl = 0; sl < nslab_v; ++sl)
                         sm100::tma_load_4d_hint(sST + sl * SLAB_BYTES, &tm_v, &bars[VFULL], sl * SLAB, h, vj * BM, bf,
@@ -192,12 +211,20 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 }
                 // store the staged X_sx (rows past the frame, columns past d_v + d_k clipped); the
                 // staging tile takes Y_{sx+1} once the store has read it (and Kh^T X_sx has, too)
-                if (sx < nblk && sm100::mbar_test(&bars[XSTAGED], sx & 1)) {
-                    for (int sl = 0; sl < nslab_x; ++sl)
-                        sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, sx * BM, (int)fh, keep);
+                if (sa < nblk && sm100::mbar_test(&bars[XSTG0], sa & 1)) {
+                    for (int sl = 0; sl < nsA; ++sl)
+                        sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, sa * BM, (int)fh, keep);
                     sm100::bulk_commit();
                     sm100::bulk_wait_read0();
-                    ++sx;
+                    ++sa;
+                    prog = true;
+                }
+                if (sb < sa && sm100::mbar_test(&bars[XSTG1], sb & 1)) {
+                    for (int sl = nsA; sl < nslab_x; ++sl)
+                        sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, sb * BM, (int)fh, keep);
+                    sm100::bulk_commit();
+                    sm100::bulk_wait_read0();
+                    ++sb;
                     prog = true;
                 }
                 if (prog) {
@@ -245,7 +272,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 sm100::mma_commit(&bars[XFULL]);
                 sm100::mma_commit(&bars[TFREE]);
                 // H (already rescaled to this block's end by the epilogue) += Kh_i^T X_i
-                ok = sm100::mbar_wait(&bars[XSTAGED], (uint32_t)(i & 1), err, wait_ns);
+                ok = sm100::mbar_wait(&bars[XSTG0], (uint32_t)(i & 1), err, wait_ns) &&
+                     sm100::mbar_wait(&bars[XSTG1], (uint32_t)(i & 1), err, wait_ns);
                 if (!ok) break;
                 sm100::tc_fence_after();
                 for (int ks = 0; ks < BM / 16; ++ks)
@@ -300,16 +328,19 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             const int n16 = rlen >> 4;  // the half's 16-column chunks (d_v and d_k are multiples of 16)
             const float rs = half ? be * __expf(Gr) : be;
             // y = rs x - rf acc over 8 columns from c, x this row's v (landed in the staging tile,
-            // overwritten in place) or k
+            // overwritten in place) or k; pairs of columns in packed fp32 x2 arithmetic
+            const uint64_t rs2 = f32x2(rs, rs), nrf2 = f32x2(-rf, -rf);
             auto build = [&](int c, const float *acc) {
                 const uint4 xin = *reinterpret_cast<const uint4 *>((half ? kt : sST) + sw_offset(c, r));
-                const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&xin);
+                const uint32_t xw[4] = {xin.x, xin.y, xin.z, xin.w};
                 float y[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 fx = __bfloat1622float2(x2[e]);
-                    y[2 * e] = fmaf(rs, fx.x, -rf * acc[2 * e]);
-                    y[2 * e + 1] = fmaf(rs, fx.y, -rf * acc[2 * e + 1]);
+                    // bf16 pair -> fp32 pair: the low half shifted up, the high half masked
+                    const uint64_t xp = f32x2(__uint_as_float(xw[e] << 16), __uint_as_float(xw[e] & 0xffff0000u));
+                    const uint64_t yp = fma_f32x2(nrf2, f32x2(acc[2 * e], acc[2 * e + 1]), mul_f32x2(rs2, xp));
+                    y[2 * e] = __uint_as_float((uint32_t)yp);
+                    y[2 * e + 1] = __uint_as_float((uint32_t)(yp >> 32));
                 }
                 *reinterpret_cast<uint4 *>(sST + sw_offset(c_base + c, r)) = valid ? pack8(y) : make_uint4(0, 0, 0, 0);
             };
@@ -351,7 +382,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             });
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(&bars[XSTAGED]);
+            sm100::mbar_arrive(&bars[half ? XSTG1 : XSTG0]);
 
             // ---- H_{i+1} (TMEM lane = key dimension m = r): bf16 copy for K_{i+1} H_{i+1}, and the
             //      fp32 accumulator rescaled to the next anchor; after the last block, M and N
