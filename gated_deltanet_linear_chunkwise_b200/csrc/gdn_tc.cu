@@ -248,8 +248,10 @@ finish:
     op.F = p.F; op.T = p.T; op.n_fh = nfh;
     op.accumulate = p.accumulate;
     op.reverse_out = scan_reverse;
+    op.SigB = SigB;
     op.err = err;
-    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u128, tm_sig, tm_g128, tm_cf128, op, num_sms, s))) return e;
+    op.wait_ns = wait_ns;
+    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u128, tm_g128, tm_cf128, op, s))) return e;
     return mark(ev, 7, s);
 }
 

@@ -60,6 +60,31 @@ __device__ __forceinline__ uint64_t desc_mnmajor(const void *tile, int ks, int k
     return sm100::smem_desc(a, (uint32_t)krows * 128, 1024, sm100::kSwizzle128B);
 }
 
+// bf16 column c, row r of a 128-row tile of 64-column SW128 slabs (K-major rows)
+__device__ __forceinline__ uint32_t sw_offset(int c, int r) {
+    return (uint32_t)((c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
+}
+
+// Walks n16 16-column chunks of this warp's TMEM lanes from taddr, loading each chunk while
+// fn(j, chunk) works on the one before it (tcgen05.wait::ld waits for every load in flight,
+// so one load is ahead at a time).  Warp-uniform: every lane takes part in the loads.
+template <typename F>
+__device__ __forceinline__ void tmem_walk16(uint32_t taddr, int n16, F &&fn) {
+    float buf[2][16];
+    sm100::tmem_ld16(taddr, buf[0]);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        if (j >= n16) break;
+        sm100::tmem_ld_wait();
+        if (j + 1 < n16) sm100::tmem_ld16(taddr + 16 * (j + 1), buf[(j + 1) & 1]);
+        fn(j, buf[j & 1]);
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float *x) {
+    return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+}
+
 struct OutParams {
     const float *G;          // [n_fh][(L+3)&~3] inclusive prefix of clamped log alpha per frame
     const float *CF;         // [n_fh][(L+3)&~3] column decay factors e^{a(s) - G_s}, a = G at the end of s's
@@ -69,7 +94,9 @@ struct OutParams {
     long long F, T, n_fh;
     int accumulate;          // o += result (formed in fp32, rounded once)
     int reverse_out;         // the pass ran on token-reversed inputs: row t goes to token T - 1 - t
+    const __nv_bfloat16 *SigB;  // [n_fh][dk][dv] bf16 state entering each frame (from the scan)
     int *err;
+    uint64_t wait_ns;
 };
 
 struct IntraParams {
@@ -158,8 +185,8 @@ cudaError_t launch_scan_tc(const Problem &p, const __nv_bfloat16 *Mimg, const fl
                            float *SigF, int *err, uint64_t wait_ns, cudaStream_t s);
 
 cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
-                             const CUtensorMap &tm_sig, const CUtensorMap &tm_g, const CUtensorMap &tm_cf,
-                             const OutParams &prm, int num_sms, cudaStream_t s);
+                             const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const OutParams &prm,
+                             cudaStream_t s);
 
 }  // namespace tc
 }  // namespace gdn

@@ -66,27 +66,6 @@ struct Smem {
 static_assert(Smem::TSLOT + 4 <= Smem::KB, "barriers overlap the tiles");
 static_assert(Smem::END <= 232448, "over the 227 KB a CTA may use");
 
-// bf16 column c, row r of a 128-row tile of 64-column SW128 slabs (K-major rows)
-__device__ __forceinline__ uint32_t sw_offset(int c, int r) {
-    return (uint32_t)((c >> 6) * SLAB_BYTES + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
-}
-
-// Walks n16 16-column chunks of this warp's TMEM lanes from taddr, loading each chunk while
-// fn(j, chunk) works on the one before it (tcgen05.wait::ld waits for every load in flight,
-// so one load is ahead at a time).  Warp-uniform: every lane takes part in the loads.
-template <typename F>
-__device__ __forceinline__ void tmem_walk16(uint32_t taddr, int n16, F &&fn) {
-    float buf[2][16];
-    sm100::tmem_ld16(taddr, buf[0]);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        if (j >= n16) break;
-        sm100::tmem_ld_wait();
-        if (j + 1 < n16) sm100::tmem_ld16(taddr + 16 * (j + 1), buf[(j + 1) & 1]);
-        fn(j, buf[j & 1]);
-    }
-}
-
 // Packed fp32 pairs (lane 0 in the low word).
 __device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
     return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
@@ -102,9 +81,6 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
     return d;
 }
 
-__device__ __forceinline__ uint4 pack8(const float *x) {
-    return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,

@@ -1,36 +1,33 @@
 // tc_output.cu -- output stage on the 5th-generation tensor cores.
 //
-// For one 128-row block I of one frame-head (rows r, columns s of the frame):
-//   O_I = diag(e^G) Q_I Sig + sum_{s <= r} (q_r . k_s) e^{G_r - G_s} u_s
-// (the intra-frame term of the chunkwise gated delta rule; o_r reads S_r, so
-// the causal mask includes the diagonal; SANA-WM summary, "Memory-Efficient
-// Long-Context Modeling (Section 3.2)", frame-wise GDN).
+// For one frame-head, block by block (128 rows; rows r, columns s of the frame):
+//   o_r = q_r . S_r,  S_r = e^{G_r} Sig + sum_{s <= r} e^{G_r - G_s} k_s^T u_s
+// (the output of the chunkwise gated delta rule: the state entering the frame
+// plus the frame's own pseudo-values; o_r reads S_r, so the causal mask
+// includes the diagonal; SANA-WM summary, "Memory-Efficient Long-Context
+// Modeling (Section 3.2)", frame-wise GDN).  The columns before block i enter
+// it through the state at the block's anchor a_i (the last token before it),
+// carried from block to block:
+//   Z_0     = Sig,   Z_{i+1} = e^{G_{a_{i+1}} - G_{a_i}} Z_i + Kh_i^T U_i,
+//   Kh_i    = diag(e^{G_{a_{i+1}} - G_s}) K_i                 (every factor <= 1)
+//   O_i     = Qt_i Z_i + P_i U_i,   Qt_i = diag(e^{G_r - G_{a_i}}) Q_i,
+//   P_i     = causal(Q_i K_i^T o e^{G_r - G_s})               (the diagonal block only)
+// so each block costs four 128 x 128 x 128 products (Q_i K_i^T, Qt_i Z_i,
+// P_i U_i, Kh_i^T U_i) however many blocks come before it.
 //
-// Persistent kernel: one CTA per SM walks a contiguous range of (frame-head,
-// block) items (ranges balanced by tile count), so a frame's K and U tiles
-// come from HBM once and are re-read from L2 by the same CTA for the frame's
-// other blocks; TMEM and barriers are set up once.  The columns s come in
-// 128-token tiles through a 2-deep ring (a tensor-core instruction costs the
-// same for every N up to 128, so S = Q K^T is issued with N = 128); the MMA
-// thread issues each tile's
-// S = Q K^T as soon as its data and an S/P buffer are there and each O += P U
-// as soon as the epilogue has written P (polling both in one loop).
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues tcgen05.mma from one thread, warps 2-9 are the epilogue: two
-// warpgroups, each thread owning one tile row (TMEM lane quadrant =
-// warp % 4) and one 64-column half of each tile.
-//   TMEM: two S/P buffers (128 columns each) and two O buffers (128 each).
-//         The epilogue turns S (fp32) into P (bf16) in place -- each half
-//         into the first 32 TMEM columns of its own range -- and O += P U
-//         reads P straight from tensor memory.
-//   SMEM: Q_I double buffer; 2 ring slots of (K_j, U_j) + (G_j, cf_j).
-// The state term is a pseudo-tile in front of the column tiles: the epilogue
-// writes Q~ = diag(e^G) Q_I into an S/P buffer and a ring slot delivers Sig
-// (bf16, MN-major), so O starts as Q~ Sig.  Off-diagonal decay factors are
-// e^{G_r - a} cf_s with cf_s = e^{a - G_s} (a = G at the end of s's 64-token
-// group, both <= 1); in the diagonal group the row factor is >= 1, bounded by
+// One CTA per frame-head.  Warp roles (320 threads): warp 0 issues TMA loads,
+// warp 1 owns TMEM and issues tcgen05.mma from one thread, warps 2-5 (group A)
+// carry the state -- Z_i to bf16 for Qt_i Z_i, the fp32 Z rescaled to the next
+// anchor -- and write O out; warps 6-9 (group B) turn each S = Q_i K_i^T into
+// bf16 P in tensor memory and scale Q_i, K_i into Qt_i, Kh_i in place.  Each
+// epilogue thread owns one row (TMEM lane quadrant = warp % 4).
+//   TMEM: Z (fp32, lane = key dimension), two S/P buffers, O.
+//   SMEM: Q_i, K_i, U_i (+ G, cf rows) double-buffered; bf16 Z_i.
+// Decay in P: e^{G_r - a} cf_s with cf_s = e^{a - G_s} (a = G at the end of
+// s's 64-token group); inside the group the row factor is >= 1, bounded by
 // e^60, else the exact e^{G_r - G_s} is taken per element.  Every wait is
-// bounded (sm100::mbar_wait).
+// bounded (sm100::mbar_wait); the MMA thread drains its products before TMEM
+// is released and the producer its copies.
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -38,86 +35,97 @@ namespace tc {
 namespace {
 
 constexpr int kThreads = 320;
-constexpr int kEpi = 256;                 // epilogue threads
-constexpr int JT = 128;                   // tokens per column tile (= BM: tile I is block I's diagonal)
-constexpr int NSLOT = 3;                  // ring depth
-constexpr int NSB = 2;                    // S/P buffers in TMEM
-constexpr int JSLAB = JT * 128;           // one 128-row slab
-constexpr int SLOT_BYTES = 4 * JSLAB;     // K (2 slabs) + U (2 slabs); or an item's Q (2 slabs) + Sig (<= 32 KB)
-constexpr int GC_BYTES = 2 * JT * 4;      // G and cf of one tile
+constexpr int kGrp = 128;                 // threads per epilogue group
+constexpr int TILE = 2 * SLAB_BYTES;      // 128 rows x 2 slabs
+constexpr int BUF = 3 * TILE;             // Q, K, U of one block
 constexpr float kSplitMax = 60.f;         // largest row exponent the in-group split takes
 
-struct Smem {
-    static constexpr uint32_t RING = 0;                       // NSLOT x 64 KB
-    static constexpr uint32_t GC = RING + NSLOT * SLOT_BYTES; // NSLOT x (G[128], cf[128])
-    static constexpr uint32_t END = GC + NSLOT * GC_BYTES;
+enum Bar {
+    FULL = 0, BFREE = FULL + 2, SFULL = BFREE + 2, SPFREE = SFULL + 2, PREADY = SPFREE + 2, SREADY, ZFULL,
+    OFULL, OFREE, DRAIN, NBAR
 };
 
-enum Bar {
-    RFULL = 0, REMPTY = RFULL + NSLOT, SFULL = REMPTY + NSLOT, SFREE = SFULL + NSB, PFULL = SFREE + NSB,
-    OFULL = PFULL + NSB, OEMPTY = OFULL + 1, QFREE = OEMPTY + 1, DRAIN = QFREE + 2, NBAR = DRAIN + 1
+// Small objects first, then the swizzled tiles from a 1024-byte boundary (the dynamic shared
+// memory base is itself 1024-aligned; the kernel checks it).
+struct Smem {
+    static constexpr uint32_t BARS = 0;
+    static constexpr uint32_t TSLOT = BARS + NBAR * 8;
+    static constexpr uint32_t GC = 1024;                  // 2 x (G[128], cf[128])
+    static constexpr uint32_t BUFS = 3072;                // 2 x (Q, K, U)
+    static constexpr uint32_t ZB = BUFS + 2 * BUF;        // bf16 Z_i (key dimension x value columns)
+    static constexpr uint32_t END = ZB + TILE;
 };
+static_assert(Smem::TSLOT + 4 <= Smem::GC, "barriers overlap the gate rows");
+static_assert(Smem::GC + 2 * 2 * BM * 4 <= Smem::BUFS, "gate rows overlap the tiles");
+static_assert(Smem::END <= 232448, "over the 227 KB a CTA may use");
+
+// A row of 16-byte bf16 chunks of a swizzled tile scaled in place by f (0 clears it).
+__device__ __forceinline__ void scale_row(unsigned char *tile, int r, int ncols, float f) {
+    for (int c = 0; c < ncols; c += 8) {
+        uint4 *p = reinterpret_cast<uint4 *>(tile + sw_offset(c, r));
+        uint4 v = *p;
+        __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 x = __bfloat1622float2(h2[e]);
+            h2[e] = __floats2bfloat162_rn(f * x.x, f * x.y);
+        }
+        *p = v;
+    }
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-            const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_sig,
-            const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_cf,
-            const OutParams prm) {
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+            const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_g,
+            const __grid_constant__ CUtensorMap tm_cf, const OutParams prm) {
+    extern __shared__ __align__(1024) unsigned char smem[];
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nblk = prm.nblk;
-    const long long F = prm.F, nfh = prm.n_fh, nitems = nfh * nblk;
-    const int gs = (L + 3) & ~3;           // row stride of G and cf
-    const int ntile_frame = (L + JT - 1) / JT;
+    const long long fh = blockIdx.x;
+    const long long F = prm.F;
+    const long long f = fh % F, chain = fh / F;
+    const int h = (int)(chain % prm.H), b = (int)(chain / prm.H);
+    const int bf = (int)(b * F + f);
+    const int gs = (L + 3) & ~3;  // G and cf row stride
 
-    unsigned char *sRing = smem + Smem::RING;
+    uint64_t *bars = (uint64_t *)(smem + Smem::BARS);
+    uint32_t *tmem_slot = (uint32_t *)(smem + Smem::TSLOT);
     float *sGC = (float *)(smem + Smem::GC);
-    uint64_t *bars = (uint64_t *)(smem + Smem::END);
-    uint32_t *tmem_slot = (uint32_t *)(bars + NBAR);
+    unsigned char *sZ = smem + Smem::ZB;
+    auto sQ = [&](int buf) { return smem + Smem::BUFS + buf * BUF; };
+    auto sK = [&](int buf) { return smem + Smem::BUFS + buf * BUF + TILE; };
+    auto sU = [&](int buf) { return smem + Smem::BUFS + buf * BUF + 2 * TILE; };
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *err = prm.err;
+    const uint64_t wait_ns = prm.wait_ns;
+    const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
 
     if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
+    if (sm100::smem_u32(smem) & 1023u) {  // every thread sees the same base: all leave together
+        if (threadIdx.x == 0) atomicCAS(err, sm100::kErrNone, sm100::kErrSmemAlign);
+        return;
+    }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NBAR; ++i) {
-            const bool epi = (i >= PFULL && i < PFULL + NSB) || i == OEMPTY;
-            sm100::mbar_init(&bars[i], epi ? kEpi : 1);
-        }
+        for (int i = 0; i < NBAR; ++i)
+            sm100::mbar_init(&bars[i], (i == PREADY || i == SREADY || i == OFREE) ? kGrp : 1);
         sm100::fence_barrier_init();
     }
     if (warp == 1) {
         sm100::tmem_alloc(tmem_slot, 512);
         sm100::tmem_relinquish();
     }
+    if (nslab_k == 1) {  // K_i^T as a 128-row operand: key dimensions past the one loaded slab are zero
+        for (int o = threadIdx.x * 16; o < SLAB_BYTES; o += kThreads * 16) {
+            *reinterpret_cast<uint4 *>(sK(0) + SLAB_BYTES + o) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sK(1) + SLAB_BYTES + o) = make_uint4(0, 0, 0, 0);
+        }
+        sm100::fence_proxy_async_smem();
+    }
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    // TMEM: two S/P buffers (128 columns each), the O accumulator (128), and the item's Q in two
-    // buffers of 64 columns (two bf16 per column: the A operand of S = Q K^T, read from TMEM)
-    const uint32_t t_s0 = tbase, t_o = tbase + 256, t_q0 = tbase + 384;
-
-    const int nks_d = dk / 16;
-    const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
-
-    // item w: frame-head w / nblk, block nblk-1 - w % nblk (heaviest block of a frame first);
-    // its column tiles are j = 0 .. I, the last one being the diagonal block
-    auto item_blk = [&](long long w) { return nblk - 1 - (int)(w % nblk); };
-    auto item_fh = [&](long long w) { return w / nblk; };
-    auto item_ntiles = [&](int I) { return min(I + 1, ntile_frame); };
-    // CTA c takes items [item_start(c), item_start(c + 1)): equal shares of the
-    // total weight, an item weighing its tiles plus two (state term, drain)
-    auto item_start = [&](long long c) -> long long {
-        long long wfh = 0;
-        for (int I = 0; I < nblk; ++I) wfh += item_ntiles(I) + 2;
-        const long long target = (c * wfh * nfh + gridDim.x - 1) / gridDim.x;
-        const long long fh = target / wfh;
-        long long rem = target - fh * wfh;
-        int k = 0;
-        while (k < nblk && rem > 0) rem -= item_ntiles(nblk - 1 - k++) + 2;
-        return min(fh * nblk + k, nitems);
-    };
-    const long long w_begin = item_start(blockIdx.x), w_end = item_start(blockIdx.x + 1);
+    const uint32_t t_z = tbase, t_sp = tbase + 128, t_o = tbase + 384;  // Z; S/P x 2; O
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -125,243 +133,237 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             sm100::tma_prefetch_desc(&tm_q);
             sm100::tma_prefetch_desc(&tm_k);
             sm100::tma_prefetch_desc(&tm_u);
-            sm100::tma_prefetch_desc(&tm_sig);
             sm100::tma_prefetch_desc(&tm_g);
             sm100::tma_prefetch_desc(&tm_cf);
-            // L2 policies: a frame's K and U tiles are read again by its other blocks, Q once
-            const uint64_t keep = sm100::policy_evict_last(), once = sm100::policy_evict_first();
+            const uint64_t once = sm100::policy_evict_first();
+            const uint32_t bytes = (uint32_t)((2 * nslab_k + nslab_v) * SLAB_BYTES + 2 * BM * 4);
+            int j = 0;
             bool ok = true;
-            int n = 0, t = 0;
-            for (long long w = w_begin; w < w_end && ok; ++w, ++t) {
-                const int I = item_blk(w);
-                const long long fh = item_fh(w);
-                const long long f = fh % F, chain = fh / F;
-                const int h = (int)(chain % prm.H), b = (int)(chain / prm.H);
-                const int bf = (int)(b * F + f);
-                const int nt = item_ntiles(I);
-                for (int j = -1; j < nt && ok; ++j, ++n) {
-                    const int st = n % NSLOT;
-                    if (n >= NSLOT) ok = sm100::mbar_wait(&bars[REMPTY + st], ((n / NSLOT) - 1) & 1, err);
-                    if (!ok) break;
-                    unsigned char *slot = sRing + st * SLOT_BYTES;
-                    if (j < 0) {  // the item's Q (2 slabs) and the state term's Sig (after them)
-                        sm100::mbar_arrive_expect_tx(&bars[RFULL + st],
-                                                     (uint32_t)(nslab_k * JSLAB + nslab_v * dk * 128));
-                        for (int sl = 0; sl < nslab_k; ++sl)
-                            sm100::tma_load_4d_hint(slot + sl * JSLAB, &tm_q, &bars[RFULL + st], sl * SLAB, h, I * BM,
-                                                    bf, once);
-                        for (int sl = 0; sl < nslab_v; ++sl)
-                            sm100::tma_load_3d(slot + 2 * JSLAB + sl * dk * 128, &tm_sig, &bars[RFULL + st], sl * SLAB,
-                                               0, (int)fh);
-                    } else {
-                        sm100::mbar_arrive_expect_tx(&bars[RFULL + st],
-                                                     (uint32_t)((nslab_k + nslab_v) * JSLAB + GC_BYTES));
-                        for (int sl = 0; sl < nslab_k; ++sl)
-                            sm100::tma_load_4d_hint(slot + sl * JSLAB, &tm_k, &bars[RFULL + st], sl * SLAB, h, j * JT, bf,
-                                                    keep);
-                        for (int sl = 0; sl < nslab_v; ++sl)
-                            sm100::tma_load_3d_hint(slot + (2 + sl) * JSLAB, &tm_u, &bars[RFULL + st], sl * SLAB, j * JT,
-                                                    (int)fh, keep);
-                        float *gc = sGC + st * 2 * JT;
-                        sm100::tma_load_2d(gc, &tm_g, &bars[RFULL + st], j * JT, (int)fh);
-                        sm100::tma_load_2d(gc + JT, &tm_cf, &bars[RFULL + st], j * JT, (int)fh);
-                    }
+            for (; j < nblk && ok; ++j) {  // block j into buffer j & 1 once block j - 2 is done with it
+                const int buf = j & 1;
+                if (j >= 2) ok = sm100::mbar_wait(&bars[BFREE + buf], (uint32_t)(((j >> 1) - 1) & 1), err, wait_ns);
+                if (!ok) break;
+                uint64_t *bar = &bars[FULL + buf];
+                sm100::mbar_arrive_expect_tx(bar, bytes);
+                for (int sl = 0; sl < nslab_k; ++sl) {
+                    sm100::tma_load_4d_hint(sQ(buf) + sl * SLAB_BYTES, &tm_q, bar, sl * SLAB, h, j * BM, bf, once);
+                    sm100::tma_load_4d_hint(sK(buf) + sl * SLAB_BYTES, &tm_k, bar, sl * SLAB, h, j * BM, bf, once);
                 }
+                for (int sl = 0; sl < nslab_v; ++sl)
+                    sm100::tma_load_3d_hint(sU(buf) + sl * SLAB_BYTES, &tm_u, bar, sl * SLAB, j * BM, (int)fh, once);
+                sm100::tma_load_2d(sGC + buf * 2 * BM, &tm_g, bar, j * BM, (int)fh);
+                sm100::tma_load_2d(sGC + buf * 2 * BM + BM, &tm_cf, bar, j * BM, (int)fh);
             }
-            // leave with no copy in flight: the last NSLOT uses of the ring have landed (full limit)
-            for (int u = n > NSLOT ? n - NSLOT : 0; u < n; ++u)
-                sm100::mbar_wait(&bars[RFULL + (u % NSLOT)], (uint32_t)((u / NSLOT) & 1), err, sm100::kWaitLimitNs,
-                                 true);
+            if (!ok)  // leave with no copy in flight (full-limit drain waits)
+                for (int u = j > 2 ? j - 2 : 0; u < j; ++u)
+                    sm100::mbar_wait(&bars[FULL + (u & 1)], (uint32_t)((u >> 1) & 1), err, sm100::kWaitLimitNs, true);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Polls: S_j = Q_j K_j^T as soon as block j has landed and its S/P buffer is free; then,
+        // per block i in order, O_i = Qt_i Z_i + P_i U_i and Z += Kh_i^T U_i once P_i (with Qt_i,
+        // Kh_i) and bf16 Z_i (with the rescaled fp32 Z) are ready and O has been drained.
         if (lane == 0) {
-            const uint32_t id_s = sm100::idesc_bf16(BM, JT, 0, 0);
-            const uint32_t id_o = sm100::idesc_bf16(BM, dv, 0, 1);
+            const uint32_t id_s = sm100::idesc_bf16(BM, BM, 0, 0);  // Q (K-major) x K^T (K-major)
+            const uint32_t id_o = sm100::idesc_bf16(BM, dv, 0, 1);  // Qt or P (K-major) x Z or U (MN-major)
+            const uint32_t id_z = sm100::idesc_bf16(BM, dv, 1, 1);  // Kh^T (MN-major) x U (MN-major)
+            const int nks_d = dk / 16;
+            // A parity test is unambiguous only for the phase right after the last one observed:
+            // the group barriers are observed one phase at a time, in order, and no block's S is
+            // issued before the previous block's P has been observed (so P can run one ahead at
+            // most); Z_{i+1} needs Z += Kh_i^T U_i and O needs the drain, both issued from here.
+            int pobs = 0, sobs = 0, oobs = 0;
+            int cs = 0, ie = 0;  // next S product; next block's O / Z products
             bool ok = true;
-            int n = 0, sc = 0, t = 0;
-            for (long long w = w_begin; w < w_end && ok; ++w, ++t) {
-                const int I = item_blk(w);
-                const int nt = item_ntiles(I);
-                const int qb = t & 1;
-                // ---- state pseudo-tile: hand an S/P buffer to the epilogue, which writes
-                //      Q~ = diag(e^G) Q there and Q into TMEM buffer qb
-                const int sb0 = sc % NSB, st0 = n % NSLOT, sc0 = sc;
-                if (sc >= NSB) ok = sm100::mbar_wait(&bars[SFREE + sb0], ((sc / NSB) - 1) & 1, err);
-                if (!ok) break;
-                sm100::mma_commit(&bars[SFULL + sb0]);
-                ++n;
-                ++sc;
-                // ---- then, polling: O = Q~ Sig once Q~ is written and the previous item's O has
-                //      drained; S = Q K^T (Q from TMEM) as soon as Q, a tile and an S/P buffer are
-                //      ready; O += P U (after O = Q~ Sig) as soon as the epilogue has written P
-                const int n0 = n, s0 = sc;
-                int js = 0, jp = 0;
-                bool q_ready = false, o_started = false;
-                sm100::Spin spin;
-                while (ok && jp < nt) {
-                    bool prog = false;
-                    if (!q_ready && sm100::mbar_test(&bars[PFULL + sb0], (uint32_t)((sc0 / NSB) & 1))) {
-                        q_ready = true;
-                        prog = true;
-                    }
-                    if (q_ready && !o_started && (t == 0 || sm100::mbar_test(&bars[OEMPTY], (uint32_t)((t - 1) & 1)))) {
+            sm100::Spin spin(wait_ns);
+            while (ok && ie < nblk) {
+                bool prog = false;
+                while (pobs < cs && sm100::mbar_test(&bars[PREADY], pobs & 1)) ++pobs;
+                while (sobs <= ie && sobs < nblk && sm100::mbar_test(&bars[SREADY], sobs & 1)) ++sobs;
+                while (oobs < ie && sm100::mbar_test(&bars[OFREE], oobs & 1)) ++oobs;
+                if (cs < nblk && cs <= pobs) {
+                    const int buf = cs & 1;
+                    if (sm100::mbar_test(&bars[FULL + buf], (cs >> 1) & 1) &&
+                        (cs < 2 || sm100::mbar_test(&bars[SPFREE + buf], ((cs >> 1) - 1) & 1))) {
                         sm100::tc_fence_after();
-                        const unsigned char *sig = sRing + st0 * SLOT_BYTES + 2 * JSLAB;
                         for (int ks = 0; ks < nks_d; ++ks)
-                            sm100::mma_bf16_ts(t_o, t_s0 + sb0 * JT + ks * 8, desc_mnmajor(sig, ks, dk), id_o, ks > 0);
-                        sm100::mma_commit(&bars[SFREE + sb0]);
-                        sm100::mma_commit(&bars[REMPTY + st0]);
-                        o_started = true;
+                            sm100::mma_bf16_ss(t_sp + buf * 128, desc_kmajor(sQ(buf), ks, BM),
+                                               desc_kmajor(sK(buf), ks, BM), id_s, ks > 0);
+                        sm100::mma_commit(&bars[SFULL + buf]);
+                        ++cs;
                         prog = true;
                     }
-                    if (q_ready && js < nt && js - jp < NSB) {  // the buffer's previous product has been issued
-                        const int cs = s0 + js, nn = n0 + js;
-                        const int sb = cs % NSB, st = nn % NSLOT;
-                        if (sm100::mbar_test(&bars[RFULL + st], (nn / NSLOT) & 1) &&
-                            (cs < NSB || sm100::mbar_test(&bars[SFREE + sb], ((cs / NSB) - 1) & 1))) {
-                            sm100::tc_fence_after();
-                            const unsigned char *kt = sRing + st * SLOT_BYTES;
-                            for (int ks = 0; ks < nks_d; ++ks)
-                                sm100::mma_bf16_ts(t_s0 + sb * JT, t_q0 + qb * 64 + ks * 8, desc_kmajor(kt, ks, JT),
-                                                   id_s, ks > 0);
-                            sm100::mma_commit(&bars[SFULL + sb]);
-                            ++js;
-                            if (js == nt) sm100::mma_commit(&bars[QFREE + qb]);  // Q buffer qb may be rewritten
-                            prog = true;
-                        }
-                    }
-                    if (o_started && jp < js) {
-                        const int cs = s0 + jp, nn = n0 + jp;
-                        const int pb = cs % NSB, pst = nn % NSLOT;
-                        if (sm100::mbar_test(&bars[PFULL + pb], (cs / NSB) & 1)) {
-                            sm100::tc_fence_after();
-                            const unsigned char *u = sRing + pst * SLOT_BYTES + 2 * JSLAB;
-                            // P columns k = 0..63 sit in TMEM columns 0..31, k = 64..127 in columns 64..95
-                            for (int ks = 0; ks < JT / 16; ++ks)
-                                sm100::mma_bf16_ts(t_o, t_s0 + pb * JT + ks * 8 + (ks >> 2) * 32,
-                                                   desc_mnmajor(u, ks, JT), id_o, 1u);
-                            sm100::mma_commit(&bars[SFREE + pb]);
-                            sm100::mma_commit(&bars[REMPTY + pst]);
-                            ++jp;
-                            prog = true;
-                        }
-                    }
-                    if (prog) spin.reset();
-                    else if (!spin.tick(err)) ok = false;
                 }
-                n = n0 + nt;
-                sc = s0 + nt;
-                if (!ok) break;
-                sm100::mma_commit(&bars[OFULL]);
+                if (ie < cs && ie < pobs && ie < sobs && (ie == 0 || oobs >= ie)) {
+                    const int buf = ie & 1;
+                    sm100::tc_fence_after();
+                    // O_i = Qt_i Z_i + P_i U_i (P of tokens 0..63 in TMEM columns 0..31 of the
+                    // buffer, tokens 64..127 in 64..95)
+                    for (int ks = 0; ks < nks_d; ++ks)
+                        sm100::mma_bf16_ss(t_o, desc_kmajor(sQ(buf), ks, BM), desc_mnmajor(sZ, ks, BM), id_o, ks > 0);
+                    for (int ks = 0; ks < BM / 16; ++ks)
+                        sm100::mma_bf16_ts(t_o, t_sp + buf * 128 + (ks >> 2) * 64 + (ks & 3) * 8,
+                                           desc_mnmajor(sU(buf), ks, BM), id_o, 1u);
+                    sm100::mma_commit(&bars[OFULL]);
+                    sm100::mma_commit(&bars[SPFREE + buf]);
+                    if (ie + 1 < nblk) {  // Z_{i+1}: the fp32 Z was rescaled to a_{i+1} with Z_i's bf16 copy
+                        for (int ks = 0; ks < BM / 16; ++ks)
+                            sm100::mma_bf16_ss(t_z, desc_mnmajor(sK(buf), ks, BM), desc_mnmajor(sU(buf), ks, BM),
+                                               id_z, 1u);
+                        sm100::mma_commit(&bars[ZFULL]);
+                    }
+                    sm100::mma_commit(&bars[BFREE + buf]);
+                    ++ie;
+                    prog = true;
+                }
+                if (prog) spin.reset();
+                else if (!spin.tick(err)) ok = false;
             }
             sm100::mma_commit(&bars[DRAIN]);  // every product issued completes before TMEM is released
             sm100::mbar_wait(&bars[DRAIN], 0u, err, sm100::kWaitLimitNs, true);
         }
-    } else {
-        // ------------------------------------------------------------ epilogue
-        // Order: pseudo(0), tiles(0), pseudo(1), drain(0), tiles(1), pseudo(2), drain(1), ...
-        // so one item's O drains while the tensor cores work on the next.
-        const int q4 = warp & 3;                  // TMEM lane quadrant
-        const int r = q4 * 32 + lane;             // tile row owned by this thread
-        const int half = (warp - 2) >> 2;         // which 32-column half of each tile
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ group A: the state and O
+        const int q4 = warp & 3;
+        const int m = q4 * 32 + lane;  // TMEM lane: key dimension of Z, token row of O
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        int sc = 0, n = 0;
-        struct Item {
-            int I, h, b, row, nt;
-            long long fh, f;
-            bool valid;
-            float Gr;
-        };
-        auto item_of = [&](long long w) {
-            Item it;
-            it.I = item_blk(w);
-            it.nt = item_ntiles(it.I);
-            it.fh = item_fh(w);
-            it.f = it.fh % F;
-            const long long chain = it.fh / F;
-            it.h = (int)(chain % prm.H);
-            it.b = (int)(chain / prm.H);
-            it.row = it.I * BM + r;
-            it.valid = it.row < L;
-            it.Gr = prm.G[it.fh * (long long)gs + (it.valid ? it.row : L - 1)];
-            return it;
-        };
-        // state pseudo-tile: P <- diag(e^G) Q_I, written into the S/P buffer as bf16
-        auto pseudo = [&](const Item &it, int t) -> bool {
-            const int qb = t & 1, sb = sc % NSB, st = n % NSLOT;
-            if (!sm100::mbar_wait(&bars[SFULL + sb], (sc / NSB) & 1, err)) return false;
-            if (!sm100::mbar_wait(&bars[RFULL + st], (n / NSLOT) & 1, err)) return false;  // Q and Sig
-            // Q buffer qb: the S products of item t - 2 that read it have completed
-            if (t >= 2 && !sm100::mbar_wait(&bars[QFREE + qb], (uint32_t)(((t - 2) >> 1) & 1), err)) return false;
+        const float *Gf = prm.G + fh * (long long)gs;
+        const int n16 = dv >> 4;  // d_v is a multiple of 16
+        auto gend = [&](int j) { return Gf[min((j + 1) * BM, L) - 1]; };  // G at the last token of block j
+        // O_j out: rows past the frame are not stored; a reversed scan's rows go back in place
+        auto drain = [&](int j) -> bool {
+            if (!sm100::mbar_wait(&bars[OFULL], (uint32_t)(j & 1), err, wait_ns)) return false;
             sm100::tc_fence_after();
-            const unsigned char *sq = sRing + st * SLOT_BYTES;
-            const float eg = it.valid ? __expf(it.Gr) : 0.f;
-            for (int c16 = half; c16 * 32 < dk; c16 += 2) {  // 32 bf16 -> 16 TMEM columns per group
-                uint32_t pk[16], qk[16];
+            const int row = j * BM + m;
+            const bool valid = row < L;
+            const long long tt0 = f * L + row;
+            const long long tt = prm.reverse_out ? prm.T - 1 - tt0 : tt0;
+            __nv_bfloat16 *o = (__nv_bfloat16 *)prm.o + ((((long long)b * prm.T + tt) * prm.H + h) * dv);
+            tmem_walk16(t_o + lane_off, n16, [&](int c16, const float (&x)[16]) {
+                if (!valid) return;
+                float y[16];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int lc = c16 * 4 + u;  // logical 8-column chunk
-                    if (lc * 8 < dk) {
-                        const int sl = lc >> 3, cc = lc & 7;
-                        uint4 v = *reinterpret_cast<const uint4 *>(sq + sl * JSLAB + r * 128 + ((cc ^ (r & 7)) << 4));
-                        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
-                        const uint32_t *q2 = reinterpret_cast<const uint32_t *>(&v);
+                for (int e = 0; e < 16; ++e) y[e] = x[e];
+                uint4 *dst = reinterpret_cast<uint4 *>(o + 16 * c16);
+                if (prm.accumulate) {
+#pragma unroll
+                    for (int w2 = 0; w2 < 2; ++w2) {
+                        uint4 old = dst[w2];
+                        const __nv_bfloat162 *ob = reinterpret_cast<const __nv_bfloat162 *>(&old);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const float2 x = __bfloat1622float2(p2[e]);
-                            pk[u * 4 + e] = pack_bf16(eg * x.x, eg * x.y);
-                            qk[u * 4 + e] = q2[e];
+                            const float2 fl = __bfloat1622float2(ob[e]);
+                            y[8 * w2 + 2 * e] += fl.x;
+                            y[8 * w2 + 2 * e + 1] += fl.y;
                         }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) pk[u * 4 + e] = qk[u * 4 + e] = 0u;
                     }
                 }
-                sm100::tmem_st16(t_s0 + sb * JT + lane_off + c16 * 16, pk);
-                sm100::tmem_st16(t_q0 + qb * 64 + lane_off + c16 * 16, qk);
+                dst[0] = pack8(y);
+                dst[1] = pack8(y + 8);
+            });
+            sm100::tc_fence_before();
+            sm100::mbar_arrive(&bars[OFREE]);
+            return true;
+        };
+        bool ok = true;
+        float gA = 0.f;  // G at the anchor of block i (block 0: the frame's start, G = 0)
+        float gE = gend(0);
+        for (int i = 0; i < nblk && ok; ++i) {
+            const float gE_next = i + 1 < nblk ? gend(i + 1) : 0.f;  // read a block ahead
+            const bool carry = i + 1 < nblk;
+            const float gam = __expf(gE - gA);  // Z_i -> anchor a_{i+1}
+            if (i == 0) {
+                // Z_0 = Sig: the bf16 copy is the scan's own; fp32 (rescaled) into TMEM
+                const __nv_bfloat16 *sig = prm.SigB + (fh * dk + (m < dk ? m : 0)) * (long long)dv;
+                for (int c16 = 0; c16 < n16; ++c16) {
+                    uint4 w[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+                    if (m < dk) {
+                        w[0] = reinterpret_cast<const uint4 *>(sig + 16 * c16)[0];
+                        w[1] = reinterpret_cast<const uint4 *>(sig + 16 * c16)[1];
+                    }
+                    *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16, m)) = w[0];
+                    *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16 + 8, m)) = w[1];
+                    if (carry) {
+                        uint32_t zs[16];
+                        const __nv_bfloat162 *z2 = reinterpret_cast<const __nv_bfloat162 *>(w);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float2 zf = __bfloat1622float2(z2[e]);
+                            zs[2 * e] = __float_as_uint(gam * zf.x);
+                            zs[2 * e + 1] = __float_as_uint(gam * zf.y);
+                        }
+                        sm100::tmem_st16(t_z + lane_off + 16 * c16, zs);
+                    }
+                }
+            } else {
+                ok = sm100::mbar_wait(&bars[ZFULL], (uint32_t)((i - 1) & 1), err, wait_ns);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                tmem_walk16(t_z + lane_off, n16, [&](int c16, const float (&x)[16]) {
+                    *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16, m)) = pack8(x);
+                    *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16 + 8, m)) = pack8(x + 8);
+                    if (carry) {
+                        uint32_t zs[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) zs[e] = __float_as_uint(gam * x[e]);
+                        sm100::tmem_st16(t_z + lane_off + 16 * c16, zs);
+                    }
+                });
             }
             sm100::tmem_st_wait();
             sm100::tc_fence_before();
-            sm100::mbar_arrive(&bars[PFULL + sb]);
-            ++sc;
-            ++n;  // the pseudo-tile's ring slot
-            return true;
-        };
-        auto tiles = [&](const Item &it) -> bool {
-            for (int j = 0; j < it.nt; ++j, ++sc, ++n) {
-                const int sb = sc % NSB, st = n % NSLOT;
-                const bool diag = (j == it.I);
-                if (!sm100::mbar_wait(&bars[SFULL + sb], (sc / NSB) & 1, err)) return false;
-                if (!sm100::mbar_wait(&bars[RFULL + st], (n / NSLOT) & 1, err)) return false;  // G, cf
-                sm100::tc_fence_after();
-                const float *gJ = sGC + st * 2 * JT, *cfJ = gJ + JT;
-                // In the diagonal tile, a row below the half's 64-token group sees all of it,
-                // a row above sees none of it, and a row inside it sees the columns s <= r.
-                // Every row takes the split e^{G_r - a} cf_s with a = G at the group's last
-                // token (the anchor cf was made with); inside the group e^{G_r - a} >= 1, so a
-                // row whose exponent exceeds kSplitMax takes the exact e^{G_r - G_s} instead.
-                const bool none = diag && r < 64 * half;
-                const bool in_group = diag && !none && r < 64 * half + 64;
-                const float dG = it.Gr - gJ[min(64 * half + 63, L - 1 - j * JT)];
-                const bool exact = in_group && !(dG <= kSplitMax);
-                const float rf = (it.valid && !none && !exact) ? __expf(dG) : 0.f;
+            sm100::fence_proxy_async_smem();
+            sm100::mbar_arrive(&bars[SREADY]);
+            if (i > 0) ok = drain(i - 1);
+            gA = gE;
+            gE = gE_next;
+        }
+        if (ok) drain(nblk - 1);
+    } else {
+        // ------------------------------------------------------------ group B: P, Qt, Kh
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;  // block row
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        bool ok = true;
+        float gA = 0.f;  // G at the anchor of block i
+        for (int i = 0; i < nblk && ok; ++i) {
+            const int buf = i & 1;
+            ok = sm100::mbar_wait(&bars[FULL + buf], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
+                 sm100::mbar_wait(&bars[SFULL + buf], (uint32_t)((i >> 1) & 1), err, wait_ns);
+            if (!ok) break;
+            sm100::tc_fence_after();
+            const float *gJ = sGC + buf * 2 * BM, *cfJ = gJ + BM;
+            const int nrow = min(BM, L - i * BM);
+            const bool valid = r < nrow;
+            const float Gr = valid ? gJ[r] : 0.f;
+            const float gEnd = gJ[nrow - 1];
+            const uint32_t t_s = t_sp + buf * 128 + lane_off;
+            // P = causal(S o e^{G_r - G_s}) over the two 64-token groups of the block: a row before
+            // a group sees none of it, a row after it all of it, a row inside it the columns
+            // s <= r.  Decay e^{G_r - a} cf_s (a = G at the group's last token, which cf was made
+            // with); inside the group e^{G_r - a} >= 1, so a row whose exponent exceeds kSplitMax
+            // takes the exact e^{G_r - G_s} instead.
 #pragma unroll
-                // the half's 64 S columns with one wait; P then goes over the first 32 of them
-                float vs[2][32];
-                sm100::tmem_ld32(t_s0 + sb * JT + lane_off + 64 * half, vs[0]);
-                sm100::tmem_ld32(t_s0 + sb * JT + lane_off + 64 * half + 32, vs[1]);
+            for (int hh = 0; hh < 2; ++hh) {
+                const bool none = r < 64 * hh;
+                const bool in_group = !none && r < 64 * hh + 64;
+                const float dG = Gr - gJ[min(64 * hh + 63, nrow - 1)];
+                const bool exact = in_group && !(dG <= kSplitMax);
+                const float rf = (valid && !none && !exact) ? __expf(dG) : 0.f;
+                float vs[2][32];  // the group's 64 S columns with one wait; P then goes over the first 32
+                sm100::tmem_ld32(t_s + 64 * hh, vs[0]);
+                sm100::tmem_ld32(t_s + 64 * hh + 32, vs[1]);
                 sm100::tmem_ld_wait();
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr) {
-                    const int c0 = 64 * half + 32 * rr;
+                    const int c0 = 64 * hh + 32 * rr;
                     const float (&v)[32] = vs[rr];
                     uint32_t pk[16];
-                    if (!exact) {  // rf = 0 where the row sees none of the half
+                    if (!exact) {  // rf = 0 where the row sees none of the group
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
                             float f0 = rf * cfJ[c0 + e], f1 = rf * cfJ[c0 + e + 1];
-                            if (in_group) {  // the causal mask inside the group
+                            if (in_group) {
                                 f0 = c0 + e <= r ? f0 : 0.f;
                                 f1 = c0 + e + 1 <= r ? f1 : 0.f;
                             }
@@ -370,92 +372,24 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     } else {
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
-                            const int s0 = j * JT + c0 + e;
-                            const float f0 = (s0 <= it.row && s0 < L) ? __expf(it.Gr - gJ[c0 + e]) : 0.f;
-                            const float f1 =
-                                (s0 + 1 <= it.row && s0 + 1 < L) ? __expf(it.Gr - gJ[c0 + e + 1]) : 0.f;
+                            const int s0 = c0 + e;
+                            const float f0 = (s0 <= r && s0 < nrow) ? __expf(Gr - gJ[s0]) : 0.f;
+                            const float f1 = (s0 + 1 <= r && s0 + 1 < nrow) ? __expf(Gr - gJ[s0 + 1]) : 0.f;
                             pk[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
                         }
                     }
-                    // P of this half goes to TMEM columns [64 half, 64 half + 32): S columns it has read
-                    sm100::tmem_st16(t_s0 + sb * JT + lane_off + 64 * half + 16 * rr, pk);
-                }
-                sm100::tmem_st_wait();
-                sm100::tc_fence_before();
-                sm100::mbar_arrive(&bars[PFULL + sb]);
-            }
-            return true;
-        };
-        auto drain = [&](const Item &it, int t) -> bool {
-            if (!sm100::mbar_wait(&bars[OFULL], (uint32_t)(t & 1), err)) return false;
-            sm100::tc_fence_after();
-            const long long tt0 = it.f * L + it.row;
-            const long long tt = prm.reverse_out ? prm.T - 1 - tt0 : tt0;  // a reversed scan's row, back in place
-            __nv_bfloat16 *o = (__nv_bfloat16 *)prm.o + ((((long long)it.b * prm.T + tt) * prm.H + it.h) * dv);
-            // columns c = 16 half + 32 i (dv <= 128), two 16-column loads per wait (the second
-            // may read past dv, inside the O buffer's 128 columns, and is then not stored)
-#pragma unroll
-            for (int i2 = 0; i2 < 2; ++i2) {
-                const int cb = 16 * half + 64 * i2;
-                if (cb >= dv) break;
-                float acc[2][16];
-                sm100::tmem_ld16(t_o + lane_off + cb, acc[0]);
-                sm100::tmem_ld16(t_o + lane_off + cb + 32, acc[1]);
-                sm100::tmem_ld_wait();
-                if (!it.valid) continue;
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int c = cb + 32 * i;
-                    if (c >= dv) break;
-                    if (prm.accumulate) {
-                        const uint4 *old = reinterpret_cast<const uint4 *>(o + c);
-#pragma unroll
-                        for (int w2 = 0; w2 < 2; ++w2) {
-                            uint4 x = old[w2];
-                            const __nv_bfloat162 *xb = reinterpret_cast<const __nv_bfloat162 *>(&x);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 fl = __bfloat1622float2(xb[e]);
-                                acc[i][w2 * 8 + 2 * e] += fl.x;
-                                acc[i][w2 * 8 + 2 * e + 1] += fl.y;
-                            }
-                        }
-                    }
-                    const float *a16 = acc[i];
-                    reinterpret_cast<uint4 *>(o + c)[0] =
-                        make_uint4(pack_bf16(a16[0], a16[1]), pack_bf16(a16[2], a16[3]), pack_bf16(a16[4], a16[5]),
-                                   pack_bf16(a16[6], a16[7]));
-                    reinterpret_cast<uint4 *>(o + c)[1] =
-                        make_uint4(pack_bf16(a16[8], a16[9]), pack_bf16(a16[10], a16[11]),
-                                   pack_bf16(a16[12], a16[13]), pack_bf16(a16[14], a16[15]));
+                    sm100::tmem_st16(t_s + 64 * hh + 16 * rr, pk);  // S columns this row has read
                 }
             }
+            sm100::tmem_st_wait();
+            // Qt_i = diag(e^{G_r - G_{a_i}}) Q_i and (for Z_{i+1}) Kh_i = diag(e^{G_{a_{i+1}} - G_r}) K_i,
+            // in place now that S_i has read them; rows past the frame become zero
+            scale_row(sQ(buf), r, dk, valid ? __expf(Gr - gA) : 0.f);
+            if (i + 1 < nblk) scale_row(sK(buf), r, dk, valid ? __expf(gEnd - Gr) : 0.f);
             sm100::tc_fence_before();
-            sm100::mbar_arrive(&bars[OEMPTY]);
-            return true;
-        };
-        long long w = w_begin;
-        bool ok = w < w_end;
-        Item cur;
-        if (ok) {
-            cur = item_of(w);
-            ok = pseudo(cur, 0);
-        }
-        for (int t = 0; ok; ++t) {
-            // the next item's row (and its G, a global load) is read before this item's tiles
-            const long long wn = w + 1;
-            Item nxt;
-            if (wn < w_end) nxt = item_of(wn);
-            ok = tiles(cur);
-            if (!ok) break;
-            if (wn < w_end) {
-                ok = pseudo(nxt, t + 1);
-                if (!ok) break;
-            }
-            ok = drain(cur, t);
-            if (!ok || wn >= w_end) break;
-            w = wn;
-            cur = nxt;
+            sm100::fence_proxy_async_smem();
+            sm100::mbar_arrive(&bars[PREADY]);
+            gA = gEnd;
         }
     }
     sm100::tc_fence_before();
@@ -469,14 +403,12 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 }  // namespace
 
 cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
-                             const CUtensorMap &tm_sig, const CUtensorMap &tm_g, const CUtensorMap &tm_cf,
-                             const OutParams &prm, int num_sms, cudaStream_t s) {
-    const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16;
+                             const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const OutParams &prm,
+                             cudaStream_t s) {
+    const size_t smem = Smem::END;
     cudaError_t e = cudaFuncSetAttribute(k_output_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const long long nitems = prm.n_fh * prm.nblk;
-    const long long grid = nitems < num_sms ? nitems : num_sms;
-    k_output_tc<<<(unsigned)grid, kThreads, smem, s>>>(tm_q, tm_k, tm_u, tm_sig, tm_g, tm_cf, prm);
+    k_output_tc<<<(unsigned)prm.n_fh, kThreads, smem, s>>>(tm_q, tm_k, tm_u, tm_g, tm_cf, prm);
     return cudaGetLastError();
 }
 
