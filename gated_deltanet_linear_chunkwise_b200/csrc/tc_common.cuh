@@ -67,17 +67,21 @@ __device__ __forceinline__ uint32_t sw_offset(int c, int r) {
 
 // Walks n16 16-column chunks of this warp's TMEM lanes from taddr, loading each chunk while
 // fn(j, chunk) works on the one before it (tcgen05.wait::ld waits for every load in flight,
-// so one load is ahead at a time).  Warp-uniform: every lane takes part in the loads.
+// so one load is ahead at a time).  Two chunks per loop turn: a small body, because a
+// kernel's warp roles share the instruction cache.  Warp-uniform: every lane takes part.
 template <typename F>
 __device__ __forceinline__ void tmem_walk16(uint32_t taddr, int n16, F &&fn) {
-    float buf[2][16];
-    sm100::tmem_ld16(taddr, buf[0]);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        if (j >= n16) break;
+    float b0[16], b1[16];
+    sm100::tmem_ld16(taddr, b0);
+#pragma unroll 1
+    for (int j = 0; j < n16; j += 2) {
         sm100::tmem_ld_wait();
-        if (j + 1 < n16) sm100::tmem_ld16(taddr + 16 * (j + 1), buf[(j + 1) & 1]);
-        fn(j, buf[j & 1]);
+        if (j + 1 < n16) sm100::tmem_ld16(taddr + 16 * (j + 1), b1);
+        fn(j, b0);
+        if (j + 1 >= n16) break;
+        sm100::tmem_ld_wait();
+        if (j + 2 < n16) sm100::tmem_ld16(taddr + 16 * (j + 2), b0);
+        fn(j + 1, b1);
     }
 }
 

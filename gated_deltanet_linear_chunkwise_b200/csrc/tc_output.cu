@@ -15,12 +15,16 @@
 // so each block costs four 128 x 128 x 128 products (Q_i K_i^T, Qt_i Z_i,
 // P_i U_i, Kh_i^T U_i) however many blocks come before it.
 //
-// One CTA per frame-head.  Warp roles (320 threads): warp 0 issues TMA loads,
-// warp 1 owns TMEM and issues tcgen05.mma from one thread, warps 2-5 (group A)
-// carry the state -- Z_i to bf16 for Qt_i Z_i, the fp32 Z rescaled to the next
-// anchor -- and write O out; warps 6-9 (group B) turn each S = Q_i K_i^T into
-// bf16 P in tensor memory and scale Q_i, K_i into Qt_i, Kh_i in place.  Each
-// epilogue thread owns one row (TMEM lane quadrant = warp % 4).
+// One CTA per frame-head.  Warp roles (576 threads): warp 0 issues TMA loads,
+// warp 1 owns TMEM and issues tcgen05.mma from one thread, and four epilogue
+// groups of four warps (each thread one row, TMEM lane quadrant = warp % 4):
+//   A (warps 2-5)   carries the state: Z_i to bf16 for Qt_i Z_i, the fp32 Z
+//                   rescaled to the next anchor (the only epilogue step on the
+//                   block-to-block chain);
+//   B (warps 6-9)   turns S = Q_i K_i^T into bf16 P in tensor memory;
+//   C (warps 10-13) scales Q_i, K_i into Qt_i, Kh_i in place;
+//   D (warps 14-17) writes O out.
+// S of block i+1 is issued while block i is still in the epilogue.
 //   TMEM: Z (fp32, lane = key dimension), two S/P buffers, O.
 //   SMEM: Q_i, K_i, U_i (+ G, cf rows) double-buffered; bf16 Z_i.
 // Decay in P: e^{G_r - a} cf_s with cf_s = e^{a - G_s} (a = G at the end of
@@ -34,15 +38,15 @@ namespace gdn {
 namespace tc {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
 constexpr int kGrp = 128;                 // threads per epilogue group
 constexpr int TILE = 2 * SLAB_BYTES;      // 128 rows x 2 slabs
 constexpr int BUF = 3 * TILE;             // Q, K, U of one block
 constexpr float kSplitMax = 60.f;         // largest row exponent the in-group split takes
 
 enum Bar {
-    FULL = 0, BFREE = FULL + 2, SFULL = BFREE + 2, SPFREE = SFULL + 2, PREADY = SPFREE + 2, SREADY, ZFULL,
-    OFULL, OFREE, DRAIN, NBAR
+    FULL = 0, BFREE = FULL + 2, SFULL = BFREE + 2, SPFREE = SFULL + 2, PREADY = SPFREE + 2, QKREADY = PREADY + 2,
+    SREADY = QKREADY + 2, ZFULL, OFULL, OFREE, DRAIN, NBAR
 };
 
 // Small objects first, then the swizzled tiles from a 1024-byte boundary (the dynamic shared
@@ -59,18 +63,27 @@ static_assert(Smem::TSLOT + 4 <= Smem::GC, "barriers overlap the gate rows");
 static_assert(Smem::GC + 2 * 2 * BM * 4 <= Smem::BUFS, "gate rows overlap the tiles");
 static_assert(Smem::END <= 232448, "over the 227 KB a CTA may use");
 
-// A row of 16-byte bf16 chunks of a swizzled tile scaled in place by f (0 clears it).
+// A row of 16-byte bf16 chunks of a swizzled tile scaled in place by f (0 clears it); the
+// row's chunks are read before any is written back, so the loads overlap.
 __device__ __forceinline__ void scale_row(unsigned char *tile, int r, int ncols, float f) {
-    for (int c = 0; c < ncols; c += 8) {
-        uint4 *p = reinterpret_cast<uint4 *>(tile + sw_offset(c, r));
-        uint4 v = *p;
-        __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&v);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 x = __bfloat1622float2(h2[e]);
-            h2[e] = __floats2bfloat162_rn(f * x.x, f * x.y);
+    for (int c0 = 0; c0 < 128; c0 += 64) {
+        if (c0 >= ncols) break;
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (c0 + 8 * u < ncols) v[u] = *reinterpret_cast<const uint4 *>(tile + sw_offset(c0 + 8 * u, r));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (c0 + 8 * u >= ncols) break;
+            __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&v[u]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = __bfloat1622float2(h2[e]);
+                h2[e] = __floats2bfloat162_rn(f * x.x, f * x.y);
+            }
+            *reinterpret_cast<uint4 *>(tile + sw_offset(c0 + 8 * u, r)) = v[u];
         }
-        *p = v;
     }
 }
 
@@ -107,7 +120,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i)
-            sm100::mbar_init(&bars[i], (i == PREADY || i == SREADY || i == OFREE) ? kGrp : 1);
+            sm100::mbar_init(&bars[i], (i >= PREADY && i < SREADY + 1) || i == OFREE ? kGrp : 1);
         sm100::fence_barrier_init();
     }
     if (warp == 1) {
@@ -160,236 +173,244 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // Polls: S_j = Q_j K_j^T as soon as block j has landed and its S/P buffer is free; then,
-        // per block i in order, O_i = Qt_i Z_i + P_i U_i and Z += Kh_i^T U_i once P_i (with Qt_i,
-        // Kh_i) and bf16 Z_i (with the rescaled fp32 Z) are ready and O has been drained.
+        // Per block i in order: S_{i+1} = Q_{i+1} K_{i+1}^T ahead (its buffer's previous S/P has
+        // been consumed), then, once P_i, Qt_i / Kh_i and bf16 Z_i (with the rescaled fp32 Z) are
+        // ready and O has been drained, O_i = Qt_i Z_i + P_i U_i and Z += Kh_i^T U_i.  Each wait
+        // is on a phase whose successor needs a product issued after it, so no parity is ambiguous.
         if (lane == 0) {
             const uint32_t id_s = sm100::idesc_bf16(BM, BM, 0, 0);  // Q (K-major) x K^T (K-major)
             const uint32_t id_o = sm100::idesc_bf16(BM, dv, 0, 1);  // Qt or P (K-major) x Z or U (MN-major)
             const uint32_t id_z = sm100::idesc_bf16(BM, dv, 1, 1);  // Kh^T (MN-major) x U (MN-major)
             const int nks_d = dk / 16;
-            // A parity test is unambiguous only for the phase right after the last one observed:
-            // the group barriers are observed one phase at a time, in order, and no block's S is
-            // issued before the previous block's P has been observed (so P can run one ahead at
-            // most); Z_{i+1} needs Z += Kh_i^T U_i and O needs the drain, both issued from here.
-            int pobs = 0, sobs = 0, oobs = 0;
-            int cs = 0, ie = 0;  // next S product; next block's O / Z products
-            bool ok = true;
-            sm100::Spin spin(wait_ns);
-            while (ok && ie < nblk) {
-                bool prog = false;
-                while (pobs < cs && sm100::mbar_test(&bars[PREADY], pobs & 1)) ++pobs;
-                while (sobs <= ie && sobs < nblk && sm100::mbar_test(&bars[SREADY], sobs & 1)) ++sobs;
-                while (oobs < ie && sm100::mbar_test(&bars[OFREE], oobs & 1)) ++oobs;
-                if (cs < nblk && cs <= pobs) {
-                    const int buf = cs & 1;
-                    if (sm100::mbar_test(&bars[FULL + buf], (cs >> 1) & 1) &&
-                        (cs < 2 || sm100::mbar_test(&bars[SPFREE + buf], ((cs >> 1) - 1) & 1))) {
-                        sm100::tc_fence_after();
-                        for (int ks = 0; ks < nks_d; ++ks)
-                            sm100::mma_bf16_ss(t_sp + buf * 128, desc_kmajor(sQ(buf), ks, BM),
-                                               desc_kmajor(sK(buf), ks, BM), id_s, ks > 0);
-                        sm100::mma_commit(&bars[SFULL + buf]);
-                        ++cs;
-                        prog = true;
-                    }
-                }
-                if (ie < cs && ie < pobs && ie < sobs && (ie == 0 || oobs >= ie)) {
-                    const int buf = ie & 1;
-                    sm100::tc_fence_after();
-                    // O_i = Qt_i Z_i + P_i U_i (P of tokens 0..63 in TMEM columns 0..31 of the
-                    // buffer, tokens 64..127 in 64..95)
-                    for (int ks = 0; ks < nks_d; ++ks)
-                        sm100::mma_bf16_ss(t_o, desc_kmajor(sQ(buf), ks, BM), desc_mnmajor(sZ, ks, BM), id_o, ks > 0);
+            auto issue_s = [&](int j) -> bool {
+                const int buf = j & 1;
+                if (!sm100::mbar_wait(&bars[FULL + buf], (uint32_t)((j >> 1) & 1), err, wait_ns)) return false;
+                if (j >= 2 && !sm100::mbar_wait(&bars[SPFREE + buf], (uint32_t)(((j >> 1) - 1) & 1), err, wait_ns))
+                    return false;
+                sm100::tc_fence_after();
+                for (int ks = 0; ks < nks_d; ++ks)
+                    sm100::mma_bf16_ss(t_sp + buf * 128, desc_kmajor(sQ(buf), ks, BM), desc_kmajor(sK(buf), ks, BM),
+                                       id_s, ks > 0);
+                sm100::mma_commit(&bars[SFULL + buf]);
+                return true;
+            };
+            bool ok = issue_s(0);
+            for (int i = 0; i < nblk && ok; ++i) {
+                const int buf = i & 1;
+                if (i + 1 < nblk) ok = issue_s(i + 1);
+                ok = ok && sm100::mbar_wait(&bars[PREADY + buf], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
+                     sm100::mbar_wait(&bars[QKREADY + buf], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
+                     sm100::mbar_wait(&bars[SREADY], (uint32_t)(i & 1), err, wait_ns) &&
+                     (i == 0 || sm100::mbar_wait(&bars[OFREE], (uint32_t)((i - 1) & 1), err, wait_ns));
+                if (!ok) break;
+                sm100::tc_fence_after();
+                // O_i = Qt_i Z_i + P_i U_i (P of tokens 0..63 in TMEM columns 0..31 of the buffer,
+                // tokens 64..127 in 64..95)
+                for (int ks = 0; ks < nks_d; ++ks)
+                    sm100::mma_bf16_ss(t_o, desc_kmajor(sQ(buf), ks, BM), desc_mnmajor(sZ, ks, BM), id_o, ks > 0);
+                for (int ks = 0; ks < BM / 16; ++ks)
+                    sm100::mma_bf16_ts(t_o, t_sp + buf * 128 + (ks >> 2) * 64 + (ks & 3) * 8,
+                                       desc_mnmajor(sU(buf), ks, BM), id_o, 1u);
+                sm100::mma_commit(&bars[OFULL]);
+                sm100::mma_commit(&bars[SPFREE + buf]);
+                if (i + 1 < nblk) {  // Z_{i+1}: the fp32 Z was rescaled to a_{i+1} with Z_i's bf16 copy
                     for (int ks = 0; ks < BM / 16; ++ks)
-                        sm100::mma_bf16_ts(t_o, t_sp + buf * 128 + (ks >> 2) * 64 + (ks & 3) * 8,
-                                           desc_mnmajor(sU(buf), ks, BM), id_o, 1u);
-                    sm100::mma_commit(&bars[OFULL]);
-                    sm100::mma_commit(&bars[SPFREE + buf]);
-                    if (ie + 1 < nblk) {  // Z_{i+1}: the fp32 Z was rescaled to a_{i+1} with Z_i's bf16 copy
-                        for (int ks = 0; ks < BM / 16; ++ks)
-                            sm100::mma_bf16_ss(t_z, desc_mnmajor(sK(buf), ks, BM), desc_mnmajor(sU(buf), ks, BM),
-                                               id_z, 1u);
-                        sm100::mma_commit(&bars[ZFULL]);
-                    }
-                    sm100::mma_commit(&bars[BFREE + buf]);
-                    ++ie;
-                    prog = true;
+                        sm100::mma_bf16_ss(t_z, desc_mnmajor(sK(buf), ks, BM), desc_mnmajor(sU(buf), ks, BM), id_z,
+                                           1u);
+                    sm100::mma_commit(&bars[ZFULL]);
                 }
-                if (prog) spin.reset();
-                else if (!spin.tick(err)) ok = false;
+                sm100::mma_commit(&bars[BFREE + buf]);
             }
             sm100::mma_commit(&bars[DRAIN]);  // every product issued completes before TMEM is released
             sm100::mbar_wait(&bars[DRAIN], 0u, err, sm100::kWaitLimitNs, true);
         }
-    } else if (warp < 6) {
-        // ------------------------------------------------------------ group A: the state and O
+    } else {
+        const int grp = (warp - 2) >> 2;  // 0 A, 1 B, 2 C, 3 D
         const int q4 = warp & 3;
-        const int m = q4 * 32 + lane;  // TMEM lane: key dimension of Z, token row of O
+        const int r = q4 * 32 + lane;  // TMEM lane: block row (token), or key dimension of Z
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        const float *Gf = prm.G + fh * (long long)gs;
-        const int n16 = dv >> 4;  // d_v is a multiple of 16
-        auto gend = [&](int j) { return Gf[min((j + 1) * BM, L) - 1]; };  // G at the last token of block j
-        // O_j out: rows past the frame are not stored; a reversed scan's rows go back in place
-        auto drain = [&](int j) -> bool {
-            if (!sm100::mbar_wait(&bars[OFULL], (uint32_t)(j & 1), err, wait_ns)) return false;
-            sm100::tc_fence_after();
-            const int row = j * BM + m;
-            const bool valid = row < L;
-            const long long tt0 = f * L + row;
-            const long long tt = prm.reverse_out ? prm.T - 1 - tt0 : tt0;
-            __nv_bfloat16 *o = (__nv_bfloat16 *)prm.o + ((((long long)b * prm.T + tt) * prm.H + h) * dv);
-            tmem_walk16(t_o + lane_off, n16, [&](int c16, const float (&x)[16]) {
-                if (!valid) return;
-                float y[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) y[e] = x[e];
-                uint4 *dst = reinterpret_cast<uint4 *>(o + 16 * c16);
-                if (prm.accumulate) {
-#pragma unroll
-                    for (int w2 = 0; w2 < 2; ++w2) {
-                        uint4 old = dst[w2];
-                        const __nv_bfloat162 *ob = reinterpret_cast<const __nv_bfloat162 *>(&old);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 fl = __bfloat1622float2(ob[e]);
-                            y[8 * w2 + 2 * e] += fl.x;
-                            y[8 * w2 + 2 * e + 1] += fl.y;
-                        }
-                    }
-                }
-                dst[0] = pack8(y);
-                dst[1] = pack8(y + 8);
-            });
-            sm100::tc_fence_before();
-            sm100::mbar_arrive(&bars[OFREE]);
-            return true;
-        };
+        const int n16 = dv >> 4;       // d_v is a multiple of 16
         bool ok = true;
-        float gA = 0.f;  // G at the anchor of block i (block 0: the frame's start, G = 0)
-        float gE = gend(0);
-        for (int i = 0; i < nblk && ok; ++i) {
-            const float gE_next = i + 1 < nblk ? gend(i + 1) : 0.f;  // read a block ahead
-            const bool carry = i + 1 < nblk;
-            const float gam = __expf(gE - gA);  // Z_i -> anchor a_{i+1}
-            if (i == 0) {
-                // Z_0 = Sig: the bf16 copy is the scan's own; fp32 (rescaled) into TMEM
-                const __nv_bfloat16 *sig = prm.SigB + (fh * dk + (m < dk ? m : 0)) * (long long)dv;
-                for (int c16 = 0; c16 < n16; ++c16) {
-                    uint4 w[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-                    if (m < dk) {
-                        w[0] = reinterpret_cast<const uint4 *>(sig + 16 * c16)[0];
-                        w[1] = reinterpret_cast<const uint4 *>(sig + 16 * c16)[1];
-                    }
-                    *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16, m)) = w[0];
-                    *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16 + 8, m)) = w[1];
-                    if (carry) {
-                        uint32_t zs[16];
-                        const __nv_bfloat162 *z2 = reinterpret_cast<const __nv_bfloat162 *>(w);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float2 zf = __bfloat1622float2(z2[e]);
-                            zs[2 * e] = __float_as_uint(gam * zf.x);
-                            zs[2 * e + 1] = __float_as_uint(gam * zf.y);
+        if (grp == 0) {
+            // -------------------------------------------------------- A: the state
+            const float *Gf = prm.G + fh * (long long)gs;
+            auto gend = [&](int j) { return Gf[min((j + 1) * BM, L) - 1]; };  // G at the last token of block j
+            float gA = 0.f;  // G at the anchor of block i (block 0: the frame's start, G = 0)
+            float gE = gend(0);
+            for (int i = 0; i < nblk && ok; ++i) {
+                const float gE_next = i + 1 < nblk ? gend(i + 1) : 0.f;  // read a block ahead
+                const bool carry = i + 1 < nblk;
+                const float gam = __expf(gE - gA);  // Z_i -> anchor a_{i+1}
+                if (i == 0) {
+                    // Z_0 = Sig: the bf16 copy is the scan's own; fp32 (rescaled) into TMEM
+                    const __nv_bfloat16 *sig = prm.SigB + (fh * dk + (r < dk ? r : 0)) * (long long)dv;
+                    for (int c16 = 0; c16 < n16; ++c16) {
+                        uint4 w[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+                        if (r < dk) {
+                            w[0] = reinterpret_cast<const uint4 *>(sig + 16 * c16)[0];
+                            w[1] = reinterpret_cast<const uint4 *>(sig + 16 * c16)[1];
                         }
-                        sm100::tmem_st16(t_z + lane_off + 16 * c16, zs);
+                        *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16, r)) = w[0];
+                        *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16 + 8, r)) = w[1];
+                        if (carry) {
+                            uint32_t zs[16];
+                            const __nv_bfloat162 *z2 = reinterpret_cast<const __nv_bfloat162 *>(w);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float2 zf = __bfloat1622float2(z2[e]);
+                                zs[2 * e] = __float_as_uint(gam * zf.x);
+                                zs[2 * e + 1] = __float_as_uint(gam * zf.y);
+                            }
+                            sm100::tmem_st16(t_z + lane_off + 16 * c16, zs);
+                        }
                     }
+                } else {
+                    ok = sm100::mbar_wait(&bars[ZFULL], (uint32_t)((i - 1) & 1), err, wait_ns);
+                    if (!ok) break;
+                    sm100::tc_fence_after();
+                    tmem_walk16(t_z + lane_off, n16, [&](int c16, const float (&x)[16]) {
+                        *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16, r)) = pack8(x);
+                        *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16 + 8, r)) = pack8(x + 8);
+                        if (carry) {
+                            uint32_t zs[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) zs[e] = __float_as_uint(gam * x[e]);
+                            sm100::tmem_st16(t_z + lane_off + 16 * c16, zs);
+                        }
+                    });
                 }
-            } else {
-                ok = sm100::mbar_wait(&bars[ZFULL], (uint32_t)((i - 1) & 1), err, wait_ns);
+                sm100::tmem_st_wait();
+                sm100::tc_fence_before();
+                sm100::fence_proxy_async_smem();
+                sm100::mbar_arrive(&bars[SREADY]);
+                gA = gE;
+                gE = gE_next;
+            }
+        } else if (grp == 1) {
+            // -------------------------------------------------------- B: P
+            for (int i = 0; i < nblk && ok; ++i) {
+                const int buf = i & 1;
+                ok = sm100::mbar_wait(&bars[FULL + buf], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
+                     sm100::mbar_wait(&bars[SFULL + buf], (uint32_t)((i >> 1) & 1), err, wait_ns);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                tmem_walk16(t_z + lane_off, n16, [&](int c16, const float (&x)[16]) {
-                    *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16, m)) = pack8(x);
-                    *reinterpret_cast<uint4 *>(sZ + sw_offset(16 * c16 + 8, m)) = pack8(x + 8);
-                    if (carry) {
-                        uint32_t zs[16];
+                const float *gJ = sGC + buf * 2 * BM, *cfJ = gJ + BM;
+                const int nrow = min(BM, L - i * BM);
+                const bool valid = r < nrow;
+                const float Gr = valid ? gJ[r] : 0.f;
+                // P = causal(S o e^{G_r - G_s}) over the two 64-token groups of the block: a row before
+                // a group sees none of it, a row after it all of it, a row inside it the columns
+                // s <= r.  Decay e^{G_r - a} cf_s (a = G at the group's last token, which cf was
+                // made with); inside the group e^{G_r - a} >= 1, so a row whose exponent exceeds
+                // kSplitMax takes the exact e^{G_r - G_s} instead.
+                float rfh[2];
+                bool inh[2], exh[2];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) zs[e] = __float_as_uint(gam * x[e]);
-                        sm100::tmem_st16(t_z + lane_off + 16 * c16, zs);
-                    }
-                });
-            }
-            sm100::tmem_st_wait();
-            sm100::tc_fence_before();
-            sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(&bars[SREADY]);
-            if (i > 0) ok = drain(i - 1);
-            gA = gE;
-            gE = gE_next;
-        }
-        if (ok) drain(nblk - 1);
-    } else {
-        // ------------------------------------------------------------ group B: P, Qt, Kh
-        const int q4 = warp & 3;
-        const int r = q4 * 32 + lane;  // block row
-        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        bool ok = true;
-        float gA = 0.f;  // G at the anchor of block i
-        for (int i = 0; i < nblk && ok; ++i) {
-            const int buf = i & 1;
-            ok = sm100::mbar_wait(&bars[FULL + buf], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
-                 sm100::mbar_wait(&bars[SFULL + buf], (uint32_t)((i >> 1) & 1), err, wait_ns);
-            if (!ok) break;
-            sm100::tc_fence_after();
-            const float *gJ = sGC + buf * 2 * BM, *cfJ = gJ + BM;
-            const int nrow = min(BM, L - i * BM);
-            const bool valid = r < nrow;
-            const float Gr = valid ? gJ[r] : 0.f;
-            const float gEnd = gJ[nrow - 1];
-            const uint32_t t_s = t_sp + buf * 128 + lane_off;
-            // P = causal(S o e^{G_r - G_s}) over the two 64-token groups of the block: a row before
-            // a group sees none of it, a row after it all of it, a row inside it the columns
-            // s <= r.  Decay e^{G_r - a} cf_s (a = G at the group's last token, which cf was made
-            // with); inside the group e^{G_r - a} >= 1, so a row whose exponent exceeds kSplitMax
-            // takes the exact e^{G_r - G_s} instead.
+                for (int hh = 0; hh < 2; ++hh) {
+                    const bool none = r < 64 * hh;
+                    inh[hh] = !none && r < 64 * hh + 64;
+                    const float dG = Gr - gJ[min(64 * hh + 63, nrow - 1)];
+                    exh[hh] = inh[hh] && !(dG <= kSplitMax);
+                    rfh[hh] = (valid && !none && !exh[hh]) ? __expf(dG) : 0.f;
+                }
+                const uint32_t t_s = t_sp + buf * 128 + lane_off;
+                uint32_t pk[16];
+                // P of each 32 S columns goes, packed, over the first 16 of them (already read)
+                tmem_walk16(t_s, 8, [&](int c16, const float (&v)[16]) {
+                    const bool g1 = c16 >= 4;
+                    const int c0 = 16 * c16;
+                    const bool in_g = g1 ? inh[1] : inh[0], ex = g1 ? exh[1] : exh[0];
+                    const float rf = g1 ? rfh[1] : rfh[0];
+                    uint32_t q[8];
+                    if (!ex) {  // rf = 0 where the row sees none of the group
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const bool none = r < 64 * hh;
-                const bool in_group = !none && r < 64 * hh + 64;
-                const float dG = Gr - gJ[min(64 * hh + 63, nrow - 1)];
-                const bool exact = in_group && !(dG <= kSplitMax);
-                const float rf = (valid && !none && !exact) ? __expf(dG) : 0.f;
-                float vs[2][32];  // the group's 64 S columns with one wait; P then goes over the first 32
-                sm100::tmem_ld32(t_s + 64 * hh, vs[0]);
-                sm100::tmem_ld32(t_s + 64 * hh + 32, vs[1]);
-                sm100::tmem_ld_wait();
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int c0 = 64 * hh + 32 * rr;
-                    const float (&v)[32] = vs[rr];
-                    uint32_t pk[16];
-                    if (!exact) {  // rf = 0 where the row sees none of the group
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
+                        for (int e = 0; e < 16; e += 2) {
                             float f0 = rf * cfJ[c0 + e], f1 = rf * cfJ[c0 + e + 1];
-                            if (in_group) {
+                            if (in_g) {
                                 f0 = c0 + e <= r ? f0 : 0.f;
                                 f1 = c0 + e + 1 <= r ? f1 : 0.f;
                             }
-                            pk[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
+                            q[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
                         }
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
+                        for (int e = 0; e < 16; e += 2) {
                             const int s0 = c0 + e;
                             const float f0 = (s0 <= r && s0 < nrow) ? __expf(Gr - gJ[s0]) : 0.f;
                             const float f1 = (s0 + 1 <= r && s0 + 1 < nrow) ? __expf(Gr - gJ[s0 + 1]) : 0.f;
-                            pk[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
+                            q[e >> 1] = pack_bf16(v[e] * f0, v[e + 1] * f1);
                         }
                     }
-                    sm100::tmem_st16(t_s + 64 * hh + 16 * rr, pk);  // S columns this row has read
-                }
+                    if (c16 & 1) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) pk[8 + e] = q[e];
+                        sm100::tmem_st16(t_s + 64 * (c16 >> 2) + 16 * ((c16 & 3) >> 1), pk);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) pk[e] = q[e];
+                    }
+                });
+                sm100::tmem_st_wait();
+                sm100::tc_fence_before();
+                sm100::mbar_arrive(&bars[PREADY + buf]);
             }
-            sm100::tmem_st_wait();
-            // Qt_i = diag(e^{G_r - G_{a_i}}) Q_i and (for Z_{i+1}) Kh_i = diag(e^{G_{a_{i+1}} - G_r}) K_i,
-            // in place now that S_i has read them; rows past the frame become zero
-            scale_row(sQ(buf), r, dk, valid ? __expf(Gr - gA) : 0.f);
-            if (i + 1 < nblk) scale_row(sK(buf), r, dk, valid ? __expf(gEnd - Gr) : 0.f);
-            sm100::tc_fence_before();
-            sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(&bars[PREADY]);
-            gA = gEnd;
+        } else if (grp == 2) {
+            // -------------------------------------------------------- C: Qt, Kh
+            float gA = 0.f;  // G at the anchor of block i
+            for (int i = 0; i < nblk && ok; ++i) {
+                const int buf = i & 1;
+                ok = sm100::mbar_wait(&bars[FULL + buf], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
+                     sm100::mbar_wait(&bars[SFULL + buf], (uint32_t)((i >> 1) & 1), err, wait_ns);
+                if (!ok) break;
+                const float *gJ = sGC + buf * 2 * BM;
+                const int nrow = min(BM, L - i * BM);
+                const bool valid = r < nrow;
+                const float Gr = valid ? gJ[r] : 0.f, gEnd = gJ[nrow - 1];
+                // Qt_i = diag(e^{G_r - G_{a_i}}) Q_i and (for Z_{i+1}) Kh_i = diag(e^{G_{a_{i+1}} - G_r}) K_i,
+                // in place now that S_i has read them; rows past the frame become zero
+                scale_row(sQ(buf), r, dk, valid ? __expf(Gr - gA) : 0.f);
+                if (i + 1 < nblk) scale_row(sK(buf), r, dk, valid ? __expf(gEnd - Gr) : 0.f);
+                sm100::fence_proxy_async_smem();
+                sm100::mbar_arrive(&bars[QKREADY + buf]);
+                gA = gEnd;
+            }
+        } else {
+            // -------------------------------------------------------- D: O out
+            // rows past the frame are not stored; a reversed scan's rows go back in place
+            for (int j = 0; j < nblk && ok; ++j) {
+                ok = sm100::mbar_wait(&bars[OFULL], (uint32_t)(j & 1), err, wait_ns);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                const int row = j * BM + r;
+                const bool valid = row < L;
+                const long long tt0 = f * L + row;
+                const long long tt = prm.reverse_out ? prm.T - 1 - tt0 : tt0;
+                __nv_bfloat16 *o = (__nv_bfloat16 *)prm.o + ((((long long)b * prm.T + tt) * prm.H + h) * dv);
+                tmem_walk16(t_o + lane_off, n16, [&](int c16, const float (&x)[16]) {
+                    if (!valid) return;
+                    float y[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) y[e] = x[e];
+                    uint4 *dst = reinterpret_cast<uint4 *>(o + 16 * c16);
+                    if (prm.accumulate) {
+#pragma unroll
+                        for (int w2 = 0; w2 < 2; ++w2) {
+                            uint4 old = dst[w2];
+                            const __nv_bfloat162 *ob = reinterpret_cast<const __nv_bfloat162 *>(&old);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 fl = __bfloat1622float2(ob[e]);
+                                y[8 * w2 + 2 * e] += fl.x;
+                                y[8 * w2 + 2 * e + 1] += fl.y;
+                            }
+                        }
+                    }
+                    dst[0] = pack8(y);
+                    dst[1] = pack8(y + 8);
+                });
+                sm100::tc_fence_before();
+                sm100::mbar_arrive(&bars[OFREE]);
+            }
         }
     }
     sm100::tc_fence_before();
