@@ -71,6 +71,7 @@ __device__ __forceinline__ uint32_t sw_offset(int c, int r) {
 // kernel's warp roles share the instruction cache.  Warp-uniform: every lane takes part.
 template <typename F>
 __device__ __forceinline__ void tmem_walk16(uint32_t taddr, int n16, F &&fn) {
+    if (n16 <= 0) return;
     float b0[16], b1[16];
     sm100::tmem_ld16(taddr, b0);
 #pragma unroll 1

@@ -6,7 +6,7 @@
 // matrices": cliffmar.tech article, "NVIDIA SANA-WM", training section on
 // context parallelism).  The frames of one (b, h) chain are visited in order and
 // the columns of the state evolve independently, so a few CTAs per chain, each
-// owning up to 32 columns, keep the state on chip for the whole scan:
+// owning up to 16 columns, keep the state on chip for the whole scan:
 //   * the state lives in shared memory as the B operand of the next product,
 //     split into bf16 hi + lo parts (hi = bf16(x), lo = bf16(x - hi));
 //   * M_f arrives already split the same way (the transition kernel writes it in
@@ -42,9 +42,10 @@ struct ScanGeom {
 
 // Columns of the state one CTA carries: the columns of Sig evolve independently
 // (Sig_{f+1}[:, c] = M_f Sig_f[:, c] + N_f[:, c]), so each chain's state is split over
-// CTAs of at most 32 columns; each CTA streams the full M_f, and the chain's other CTAs
+// CTAs of at most 16 columns; each CTA streams the full M_f, and the chain's other CTAs
 // find it in L2.
-constexpr int kScanCols = 32;
+constexpr int kScanCols = 16;  // state columns per CTA (one 16-column TMEM chunk)
+constexpr int kTmemCols = 32;  // the smallest TMEM allocation
 
 __host__ __device__ inline ScanGeom scan_geom(int dk, int dv) {  // dv: the columns of one CTA
     ScanGeom g;
@@ -103,7 +104,7 @@ k_scan_tc(const Problem p, const __nv_bfloat16 *__restrict__ Mimg, const float *
         sm100::fence_barrier_init();
     }
     if (warp == 4) {
-        sm100::tmem_alloc(tmem_slot, kScanCols);
+        sm100::tmem_alloc(tmem_slot, kTmemCols);
         sm100::tmem_relinquish();
     }
     sm100::tc_fence_before();
@@ -175,11 +176,11 @@ k_scan_tc(const Problem p, const __nv_bfloat16 *__restrict__ Mimg, const float *
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         float *sNrow = sN + m * geo.nstride;  // this thread's row of N_f (only this thread touches it)
         auto out_row = [&](long long f) -> long long { return (fh_of(f) * dk + m) * (long long)ldv + c_base; };
-        // 32 columns [c0, c0 + 32) of a state row: the next product's operand (hi, lo) and
+        // 16 columns [c0, c0 + 16) of a state row: the next product's operand (hi, lo) and
         // the bf16 / fp32 output rows
-        auto put_operand = [&](const float (&x)[32], int c0) {
+        auto put_operand = [&](const float (&x)[kScanCols], int c0) {
 #pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
+            for (int c8 = 0; c8 < kScanCols / 8; ++c8) {
                 if (c0 + c8 * 8 >= dv) break;
                 uint32_t hi[4], lo[4];
 #pragma unroll
@@ -195,11 +196,11 @@ k_scan_tc(const Problem p, const __nv_bfloat16 *__restrict__ Mimg, const float *
                 *reinterpret_cast<uint4 *>(sSl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
         };
-        auto put_out = [&](const float (&x)[32], int c0, long long f) {
+        auto put_out = [&](const float (&x)[kScanCols], int c0, long long f) {
             if (SigB) {
                 __nv_bfloat16 *bd = SigB + out_row(f) + c0;
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
+                for (int c8 = 0; c8 < kScanCols / 8; ++c8) {
                     if (c0 + c8 * 8 >= dv) break;
                     *reinterpret_cast<uint4 *>(bd + c8 * 8) = make_uint4(
                         pack_bf16(x[c8 * 8], x[c8 * 8 + 1]), pack_bf16(x[c8 * 8 + 2], x[c8 * 8 + 3]),
@@ -209,7 +210,7 @@ k_scan_tc(const Problem p, const __nv_bfloat16 *__restrict__ Mimg, const float *
             if (SigF) {
                 float *fd = SigF + out_row(f) + c0;
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
+                for (int c4 = 0; c4 < kScanCols / 4; ++c4) {
                     if (c0 + c4 * 4 >= dv) break;
                     *reinterpret_cast<float4 *>(fd + c4 * 4) =
                         make_float4(x[c4 * 4], x[c4 * 4 + 1], x[c4 * 4 + 2], x[c4 * 4 + 3]);
@@ -218,10 +219,10 @@ k_scan_tc(const Problem p, const __nv_bfloat16 *__restrict__ Mimg, const float *
         };
         // ---- the initial state Sig_0 = S_in^T (or zero), the operand of frame 0's products
         if (row && F > 0) {
-            for (int c0 = 0; c0 < dv; c0 += 32) {
-                float x[32];
+            for (int c0 = 0; c0 < dv; c0 += kScanCols) {
+                float x[kScanCols];
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
+                for (int e = 0; e < kScanCols; ++e)
                     x[e] = (p.S_in && c0 + e < dv) ? p.S_in[(chain * ldv + c_base + c0 + e) * (long long)dk + m] : 0.f;
                 put_operand(x, c0);
                 if (!post) put_out(x, c0, 0);  // token-wise: the state entering frame 0
@@ -243,13 +244,13 @@ k_scan_tc(const Problem p, const __nv_bfloat16 *__restrict__ Mimg, const float *
             sm100::tc_fence_after();
             const bool last = f + 1 == F;
             const bool reset_next = !last && frame_resets(p, f + 1);
-            for (int c0 = 0; c0 < dv; c0 += 32) {
-                float x[32];
-                sm100::tmem_ld32(t_d + lane_off + c0, x);
+            for (int c0 = 0; c0 < dv; c0 += kScanCols) {
+                float x[kScanCols];
+                sm100::tmem_ld16(t_d + lane_off + c0, x);
                 sm100::tmem_ld_wait();
                 if (!row) continue;
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
+                for (int e = 0; e < kScanCols; e += 4) {
                     const float4 nn = *reinterpret_cast<const float4 *>(sNrow + c0 + e);
                     x[e] += nn.x;
                     x[e + 1] += nn.y;
@@ -260,13 +261,13 @@ k_scan_tc(const Problem p, const __nv_bfloat16 *__restrict__ Mimg, const float *
                 if (!last) {
                     if (reset_next) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                        for (int e = 0; e < kScanCols; ++e) x[e] = 0.f;
                     }
                     put_operand(x, c0);
                     if (!post) put_out(x, c0, f + 1);  // token-wise: the state entering frame f + 1
                 } else if (p.S_out) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
+                    for (int e = 0; e < kScanCols; ++e)
                         if (c0 + e < dv) p.S_out[(chain * ldv + c_base + c0 + e) * (long long)dk + m] = x[e];
                 }
             }
@@ -281,7 +282,7 @@ k_scan_tc(const Problem p, const __nv_bfloat16 *__restrict__ Mimg, const float *
     __syncthreads();
     if (warp == 4) {
         sm100::tc_fence_after();
-        sm100::tmem_dealloc(t_d, kScanCols);
+        sm100::tmem_dealloc(t_d, kTmemCols);
     }
 }
 
