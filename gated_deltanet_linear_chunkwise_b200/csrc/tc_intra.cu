@@ -29,10 +29,12 @@
 // source of X_i's TMA store) and bf16 H_i (the B operand of K_i H_i).
 // TMEM: the block's product (K_i H_i, then X_i; 256 columns) and H (fp32,
 // 256 columns; lanes = key dimension).
-// Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner + MMA issuer (one
-// thread), warps 2-9 epilogue: two warpgroups, each thread owning one row
+// Warp roles (352 threads): warp 0 TMA loads, warp 1 TMEM owner + MMA issuer
+// (one thread), warps 2-9 epilogue: two warpgroups, each thread owning one row
 // (TMEM lane quadrant = warp % 4) and one half of the columns (half 0 the Ub
-// columns, half 1 the W columns; for H, rows are key dimensions).
+// columns, half 1 the W columns; for H, rows are key dimensions); warp 10
+// stores X (a thread of its own, so that waiting for a store's reads holds up
+// no load).
 // Every wait is bounded (sm100::mbar_wait); a role that gives up waits for its
 // own copies and products in flight before the CTA leaves.
 #include "tc_common.cuh"
@@ -41,13 +43,13 @@ namespace gdn {
 namespace tc {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kEpi = 256;                    // epilogue threads
 constexpr int TILE = 2 * SLAB_BYTES;         // 128 rows x 2 slabs (K_i or T_ii)
 constexpr int WIDE = 4 * SLAB_BYTES;         // 128 rows x 4 slabs (Y_i / X_i, H)
 
 enum Bar {
-    ACCFULL = 0, YFULL, XFULL, XSTG0, XSTG1, UFULL, HREADY, TFULL, TFREE, VFULL, DRAIN,
+    ACCFULL = 0, YFULL, XFULL, XSTG0, XSTG1, UFULL, HREADY, TFULL, TFREE, VFULL, STAFREE, STBFREE, DRAIN,
     KFULL, KEMPTY = KFULL + 2, NBAR = KEMPTY + 2
 };
 
@@ -139,22 +141,20 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         // ------------------------------------------------------------ TMA producer
         // K_j (double-buffered: once block j-2's Kh^T X has read its buffer), T_j (once T_{j-1}
         // Y_{j-1} has read the tile), V_j into the staging tile's first slabs (once X_{j-1} has
-        // been read there by its store and by Kh^T X_{j-1}), and the store of each staged X_j.
+        // been read there by its store and by Kh^T X_{j-1}).
         if (lane == 0) {
             sm100::tma_prefetch_desc(&tm_k);
             sm100::tma_prefetch_desc(&tm_v);
             sm100::tma_prefetch_desc(&tm_t);
             sm100::tma_prefetch_desc(&tm_xs);
             // L2 policies: K and T are read once here; X is read again by the next stages
-            const uint64_t once = sm100::policy_evict_first(), keep = sm100::policy_evict_last();
+            const uint64_t once = sm100::policy_evict_first();
             int kj = 0, tj = 0, vj = 0;
-            const int nsA = dv / SLAB;
-            const bool v_shares = (dv % SLAB) != 0;
-            int sa = 0, sb = 0;
+            const bool v_shares = (dv % SLAB) != 0;  // V's last slab also holds W columns
             for (int sl = 0; sl < nslab_v; ++sl) sm100::tma_prefetch_l2_4d(&tm_v, sl * SLAB, h, 0, bf);
             bool ok = true;
             sm100::Spin spin(wait_ns);
-            while (ok && (kj < nblk || tj < nblk || vj < nblk || sb < nblk)) {
+            while (ok && (kj < nblk || tj < nblk || vj < nblk)) {
                 bool prog = false;
                 if (kj < nblk && (kj < 2 || sm100::mbar_test(&bars[KEMPTY + (kj & 1)], ((kj >> 1) - 1) & 1))) {
                     uint64_t *bar = &bars[KFULL + (kj & 1)];
@@ -173,7 +173,10 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     ++tj;
                     prog = true;
                 }
-                if (vj < nblk && (vj == 0 || (sa >= vj && sb >= vj - 1 && (!v_shares || sb >= vj) &&
+                // V_vj once X_{vj-1}'s Ub-only slabs have been read by their store (all of X_{vj-1}
+                // when V's last slab also holds W columns) and by Kh^T X_{vj-1}
+                if (vj < nblk && (vj == 0 || (sm100::mbar_test(&bars[STAFREE], (vj - 1) & 1) &&
+                                              (!v_shares || sm100::mbar_test(&bars[STBFREE], (vj - 1) & 1)) &&
                                               sm100::mbar_test(&bars[UFULL], (vj - 1) & 1)))) {
                     sm100::mbar_arrive_expect_tx(&bars[VFULL], (uint32_t)(nslab_v * SLAB_BYTES));
                     for (int sl = 0; sl < nslab_v; ++sl)
@@ -185,24 +188,6 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     ++vj;
                     prog = true;
                 }
-                // store the staged X_sx (rows past the frame, columns past d_v + d_k clipped); the
-                // staging tile takes Y_{sx+1} once the store has read it (and Kh^T X_sx has, too)
-                if (sa < nblk && sm100::mbar_test(&bars[XSTG0], sa & 1)) {
-                    for (int sl = 0; sl < nsA; ++sl)
-                        sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, sa * BM, (int)fh, keep);
-                    sm100::bulk_commit();
-                    sm100::bulk_wait_read0();
-                    ++sa;
-                    prog = true;
-                }
-                if (sb < sa && sm100::mbar_test(&bars[XSTG1], sb & 1)) {
-                    for (int sl = nsA; sl < nslab_x; ++sl)
-                        sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, sb * BM, (int)fh, keep);
-                    sm100::bulk_commit();
-                    sm100::bulk_wait_read0();
-                    ++sb;
-                    prog = true;
-                }
                 if (prog) {
                     spin.reset();
                 } else if (!spin.tick(err)) {
@@ -211,13 +196,39 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     __nanosleep(64);  // leave the issue slots to the epilogue warps of this sub-partition
                 }
             }
-            sm100::bulk_wait0();  // leave with no store in flight
-            if (!ok) {  // and no load in flight (full-limit drain waits)
+            if (!ok) {  // leave with no load in flight (full-limit drain waits)
                 for (int j = kj > 2 ? kj - 2 : 0; j < kj; ++j)
                     sm100::mbar_wait(&bars[KFULL + (j & 1)], (uint32_t)((j >> 1) & 1), err, sm100::kWaitLimitNs, true);
                 if (tj > 0) sm100::mbar_wait(&bars[TFULL], (uint32_t)((tj - 1) & 1), err, sm100::kWaitLimitNs, true);
                 if (vj > 0) sm100::mbar_wait(&bars[VFULL], (uint32_t)((vj - 1) & 1), err, sm100::kWaitLimitNs, true);
             }
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ X stores
+        // X_j in two parts: the slabs that hold only Ub columns once the Ub half has
+        // staged them (the next block's v may then land there), the rest once both halves have;
+        // a thread of its own, so that waiting for a store's reads holds up no load.
+        if (lane == 0) {
+            const int nsA = dv / SLAB;
+            const uint64_t keep = sm100::policy_evict_last();  // X is read again by the next stages
+            bool ok = true;
+            for (int j = 0; j < nblk && ok; ++j) {
+                ok = sm100::mbar_wait(&bars[XSTG0], (uint32_t)(j & 1), err, wait_ns);
+                if (!ok) break;
+                for (int sl = 0; sl < nsA; ++sl)
+                    sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, j * BM, (int)fh, keep);
+                sm100::bulk_commit();
+                sm100::bulk_wait_read0();
+                sm100::mbar_arrive(&bars[STAFREE]);
+                ok = sm100::mbar_wait(&bars[XSTG1], (uint32_t)(j & 1), err, wait_ns);
+                if (!ok) break;
+                for (int sl = nsA; sl < nslab_x; ++sl)
+                    sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, j * BM, (int)fh, keep);
+                sm100::bulk_commit();
+                sm100::bulk_wait_read0();
+                sm100::mbar_arrive(&bars[STBFREE]);
+            }
+            sm100::bulk_wait0();  // leave with no store in flight
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -295,6 +306,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             // ---- Y_i = R_i - diag(beta e^{G_r - G_{a_i}}) K_i H_i -> staging (MN-major: row = K index
             //      of T_ii Y_i)
             if (i > 0) ok = sm100::mbar_wait(&bars[ACCFULL], (uint32_t)((i - 1) & 1), err, wait_ns);
+            // the W half writes over X_{i-1}'s last slabs: their store must have read them
+            if (ok && half == 1 && i > 0) ok = sm100::mbar_wait(&bars[STBFREE], (uint32_t)((i - 1) & 1), err, wait_ns);
             if (ok) ok = sm100::mbar_wait(&bars[VFULL], (uint32_t)(i & 1), err, wait_ns) &&
                          sm100::mbar_wait(&bars[KFULL + (i & 1)], (uint32_t)((i >> 1) & 1), err, wait_ns);
             if (!ok) break;
