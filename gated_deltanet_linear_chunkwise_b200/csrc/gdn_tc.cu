@@ -2,13 +2,17 @@
 // tensor maps, the gate prologue and the stage sequence.
 //
 // Stage sequence (forward scans, bf16 q/k/v/o):
-//   gates       G = per-frame prefix of log alpha (fp32)
-//   inverse     T_ii = (I + A_ii)^{-1} per 128-row diagonal block (mma.sync)
-//   intra       [Ub | W] per frame-head, bf16, blocked forward substitution (tcgen05)
-//   transition  M, N per frame-head, fp32                 (tcgen05)
+//   gates       G = per-frame prefix of log alpha and the column factors (fp32)
+//   inverse     T_ii = (I + A_ii)^{-1} per 128-row diagonal block (Gram on tcgen05,
+//               doubling on mma.sync)
+//   intra       [Ub | W] per frame-head (bf16) by the block recurrence, and the frame's
+//               map M, N from its carried matrix (tcgen05)
 //   scan        entering state per frame, bf16             (tcgen05; CUDA cores where its
 //                                                          shared memory does not fit)
-//   output      U = Ub - W Sig (bf16, tcgen05), then the tcgen05 output kernel
+//   U, output   U = Ub - W Sig (tcgen05), then the output by the block recurrence over
+//               the frame's state (tcgen05)
+// The frame-wise operator: its per-frame maps (the transition kernel), the scan, and the
+// U kernel in its output mode.
 #include <cstdlib>
 #include <mutex>
 
@@ -310,9 +314,9 @@ cudaError_t launch_tc_frame(const Problem &p, void *ws, cudaStream_t s, cudaEven
     for (int i = 0; i <= 3; ++i)
         if ((e = mark(ev, i, s))) return e;
     tc::TransParams tp;
-    tp.G = nullptr; tp.M = scan_tc ? nullptr : Mb; tp.Mimg = scan_tc ? Mimg : nullptr; tp.N = Nb;
-    tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.nblk = nblk; tp.F = p.F; tp.err = err;
-    tp.frame = 1; tp.beta = p.beta; tp.gamma = p.gamma; tp.T = p.T;
+    tp.M = scan_tc ? nullptr : Mb; tp.Mimg = scan_tc ? Mimg : nullptr; tp.N = Nb;
+    tp.L = p.L; tp.dk = p.dk; tp.dv = p.dv; tp.H = p.H; tp.F = p.F; tp.err = err;
+    tp.beta = p.beta; tp.gamma = p.gamma; tp.T = p.T;
     // the q/k feature maps, when requested, are applied to the staged tiles (no copy pass)
     tp.norm_k = (p.qk_norm & GDN_QK_NORM_KEYS) ? 1 : 0;
     tp.k_w = p.k_norm_weight;
@@ -320,7 +324,7 @@ cudaError_t launch_tc_frame(const Problem &p, void *ws, cudaStream_t s, cudaEven
     tp.wait_ns = wait_limit_ns();
     int dev = 0, num_sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if ((e = tc::launch_transition_tc(tm_k64, tm_k64, tm_v64, tp, nfh, num_sms, s))) return e;
+    if ((e = tc::launch_transition_tc(tm_k64, tm_v64, tp, nfh, s))) return e;
     if ((e = mark(ev, 4, s))) return e;
     if (scan_tc) {
         if ((e = tc::launch_scan_tc(p, Mimg, Nb, SigB, nullptr, err, wait_limit_ns(), s))) return e;

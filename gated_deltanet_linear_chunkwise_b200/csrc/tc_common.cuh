@@ -118,23 +118,20 @@ struct IntraParams {
 };
 
 struct TransParams {
-    const float *G;            // [n_fh][(L+3)&~3]
     float *M;                  // [n_fh][dk][dk] fp32, or null
     __nv_bfloat16 *Mimg;       // or null: M split into bf16 hi + lo, each in the 128-byte-swizzled
                                // K-major image of 64-column slabs of dk rows (the scan's A operand)
     float *N;                  // [n_fh][dk][dv]
-    int L, dk, dv, H, nblk;
+    int L, dk, dv, H;
     long long F;
     int *err;
-    // frame-wise operator: M = gamma (I - K^T diag(beta) K), N = K^T diag(beta) V straight
-    // from the inputs (G and the [Ub | W] rows are not read)
-    int frame;
+    // the frame-wise operator's map: M = gamma (I - K^T diag(beta) K), N = K^T diag(beta) V
     const float *beta;         // [B,T,H]
     const float *gamma;        // [B,F,H]
     long long T;
     uint64_t wait_ns;          // limit of the bounded waits
-    // frame-wise operator: the key feature map applied to the staged K rows (both copies)
-    // before the products, K <- max(RMSNorm(K) * w, 0) * k_post; 0: keys used as given
+    // the key feature map applied to the staged K rows (both copies) before the products,
+    // K <- max(RMSNorm(K) * w, 0) * k_post; 0: keys used as given
     int norm_k;
     const float *k_w;          // [dk] RMSNorm weight or null (ones)
     float k_post;              // 1 / sqrt(dk * L)
@@ -160,10 +157,9 @@ struct UParams {
 // RMSNorm epsilon of the q/k feature maps (the pages give none; 1e-6).
 constexpr float kRmsEps = 1e-6f;
 
-// tm_k / tm_x / tm_v deliver 64-token boxes (tm_x the [Ub | W] rows, tm_v the
-// values, read by the frame-wise operator only).
-cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_v,
-                                 const TransParams &prm, long long n_fh, int num_sms, cudaStream_t s);
+// tm_k / tm_v deliver 64-token boxes of k / v.  The frame-wise operator's per-frame map.
+cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const TransParams &prm,
+                                 long long n_fh, cudaStream_t s);
 // tm_x delivers 128-row boxes of X, tm_q 128-token boxes of q (frame-wise
 // operator), tm_sig the bf16 state of a frame-head.
 cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_q, const CUtensorMap &tm_sig,

@@ -1,25 +1,23 @@
-// tc_transition.cu -- per-frame affine map of the state on the tensor cores.
+// tc_transition.cu -- the frame-wise operator's per-frame map on the tensor cores.
 //
-// Carrying the state across a frame is the affine map
-//   Sig_next = M Sig + N,   M = e^{G_L} I - Kt^T W,   N = Kt^T Ub,
-//   Kt = diag(e^{G_L - G}) K
-// (the per-frame transition of the chunk = frame decomposition; the pages
-// compose these maps with a prefix sum over frames: cliffmar.tech article,
-// "NVIDIA SANA-WM", the training section on context parallelism).
-// One CTA per frame-head accumulates Kt^T [Ub | W] over 64-token chunks that
+// The frame-wise operator (SANA-WM summary, "Memory-Efficient Long-Context
+// Modeling (Section 3.2)", paragraph "Adaptation to video: frame-wise
+// recurrence") carries the state across frame f by the affine map
+//   Sig_next = M Sig + N,   M = gamma (I - K^T B K),   N = K^T B V,   B = diag(beta)
+// (the pages compose such maps with a prefix sum over frames: cliffmar.tech
+// article, "NVIDIA SANA-WM", the training section on context parallelism).
+// The chunked (token-wise) pass does not use this kernel: its maps come out of
+// the intra-frame kernel.
+// One CTA per frame-head accumulates K^T B [V | K] over 64-token chunks that
 // stream through a 2-deep ring, two CTAs per SM so that one CTA's loads
 // overlap the other's start-up and final stores (the kernel is bound by the
-// rate at which the chunks arrive from HBM): A = Kt as an MN-major operand (the K chunk's rows are
-// tokens, i.e. the contraction index), B = the [Ub | W] chunk (MN-major), D
-// in TMEM with one lane per key dimension.  The epilogue warps scale the K
-// rows in shared memory by e^{G_L - G_r} (a per-row factor, so the swizzle
-// does not matter) and finally write M and N in fp32.
-// The same kernel forms the frame-wise operator's map (SANA-WM summary,
-// "Memory-Efficient Long-Context Modeling (Section 3.2)", paragraph
-// "Adaptation to video: frame-wise recurrence"): M = gamma (I - K^T B K),
-// N = K^T B V with B = diag(beta); then the K rows are scaled by beta and the
-// B operand is [V | K] loaded from the inputs (V in the first 64-column slabs,
-// K after them), so D = K^T B [V | K].
+// rate at which the chunks arrive from HBM): A = B K as an MN-major operand
+// (the K chunk's rows are tokens, i.e. the contraction index), B = the [V | K]
+// chunk (V in the first 64-column slabs, K after them; MN-major), D in TMEM
+// with one lane per key dimension.  The epilogue warps scale the K rows in
+// shared memory by beta (a per-row factor, so the swizzle does not matter),
+// apply the key feature map when asked, and finally write M and N in fp32
+// (and/or the scan's bf16 operand images of M).
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -40,11 +38,11 @@ struct Smem {
 enum Bar { FULL = 0, SCALED = FULL + NST, EMPTY = SCALED + NST, DONE = EMPTY + NST, NBAR };
 
 __global__ void __launch_bounds__(kThreads, 2)
-k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_x,
-                const __grid_constant__ CUtensorMap tm_v, const TransParams prm) {
+k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const TransParams prm) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv;
+    const int L = prm.L, dk = prm.dk, dv = prm.dv;
     const long long fh = blockIdx.x;
     const long long F = prm.F;
     const long long f = fh % F, chain = fh / F;
@@ -56,11 +54,10 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int *err = prm.err;
     const int nslab_k = (dk + SLAB - 1) / SLAB, nslab_v = (dv + SLAB - 1) / SLAB;
-    const bool frame = prm.frame != 0;
-    // B operand columns: chunkwise [Ub | W] packed (nc); frame-wise [V | K] slab-aligned
-    const int nslab_x = frame ? nslab_v + nslab_k : (nc + SLAB - 1) / SLAB;
-    const int ncols = frame ? SLAB * nslab_x : nc;
-    const int mcol0 = frame ? SLAB * nslab_v : dv;  // first column of the M part
+    // B operand columns: [V | K], slab-aligned
+    const int nslab_x = nslab_v + nslab_k;
+    const int ncols = SLAB * nslab_x;
+    const int mcol0 = SLAB * nslab_v;  // first column of the M part
 
     if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
     if (threadIdx.x == 0) {
@@ -80,7 +77,7 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (warp == 0) {
         if (lane == 0) {
             sm100::tma_prefetch_desc(&tm_k);
-            sm100::tma_prefetch_desc(frame ? &tm_v : &tm_x);
+            sm100::tma_prefetch_desc(&tm_v);
             bool ok = true;
             for (int c = 0; c < nch && ok; ++c) {
                 const int st = c % NST;
@@ -90,17 +87,11 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 sm100::mbar_arrive_expect_tx(&bars[FULL + st], (uint32_t)((nslab_k + nslab_x) * CSLAB));
                 for (int sl = 0; sl < nslab_k; ++sl)
                     sm100::tma_load_4d(stage + sl * CSLAB, &tm_k, &bars[FULL + st], sl * SLAB, h, c * CH, bf);
-                if (frame) {
-                    for (int sl = 0; sl < nslab_v; ++sl)
-                        sm100::tma_load_4d(stage + (2 + sl) * CSLAB, &tm_v, &bars[FULL + st], sl * SLAB, h, c * CH, bf);
-                    for (int sl = 0; sl < nslab_k; ++sl)
-                        sm100::tma_load_4d(stage + (2 + nslab_v + sl) * CSLAB, &tm_k, &bars[FULL + st], sl * SLAB, h,
-                                           c * CH, bf);
-                } else {
-                    for (int sl = 0; sl < nslab_x; ++sl)
-                        sm100::tma_load_3d(stage + (2 + sl) * CSLAB, &tm_x, &bars[FULL + st], sl * SLAB, c * CH,
-                                           (int)fh);
-                }
+                for (int sl = 0; sl < nslab_v; ++sl)
+                    sm100::tma_load_4d(stage + (2 + sl) * CSLAB, &tm_v, &bars[FULL + st], sl * SLAB, h, c * CH, bf);
+                for (int sl = 0; sl < nslab_k; ++sl)
+                    sm100::tma_load_4d(stage + (2 + nslab_v + sl) * CSLAB, &tm_k, &bars[FULL + st], sl * SLAB, h,
+                                       c * CH, bf);
             }
             if (ok) sm100::mbar_wait(&bars[DONE], 0, err);  // no copy left in flight
         }
@@ -125,19 +116,17 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     } else {
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;  // the epilogue's 128 threads; at the end, key dimension m
-        const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
-        const float GL = frame ? 0.f : Gf[L - 1];
         bool ok = true;
         // thread r scales row r % 64 of the chunk's K, slab r / 64
         const int row_in = r & (CH - 1), sl = r >> 6;
         float *sSS = reinterpret_cast<float *>(bars + NBAR + 1);  // [2][64] partial sums of squares
-        const bool normk = frame && prm.norm_k;
-        // the K row's factor: e^{G_L - G_r}, or beta_r for the frame-wise map; read one chunk
-        // ahead so the load's latency stays off the scaling step
+        const bool normk = prm.norm_k != 0;
+        // the K row's factor beta_r, read one chunk ahead so the load's latency stays off the
+        // scaling step
         auto row_gate = [&](int c) -> float {
             const int row = c * CH + row_in;
             if (c >= nch || row >= L) return 0.f;
-            return frame ? prm.beta[((long long)b * prm.T + f * L + row) * prm.H + h] : Gf[row];
+            return prm.beta[((long long)b * prm.T + f * L + row) * prm.H + h];
         };
         float g_next = row_gate(0);
         for (int c = 0; c < nch && ok; ++c) {
@@ -145,7 +134,7 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const int row = c * CH + row_in;
             const float g_row = g_next;
             g_next = row_gate(c + 1);
-            const float sc = row >= L ? 0.f : (frame ? g_row : __expf(GL - g_row));
+            const float sc = row >= L ? 0.f : g_row;
             ok = sm100::mbar_wait(&bars[FULL + st], (c / NST) & 1, err, prm.wait_ns);
             if (normk) ok = named_sync_and(1, 128, ok);  // the row's two halves meet below
             if (!ok) break;
@@ -216,9 +205,9 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (ok) {
             sm100::tc_fence_after();
             const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-            // M = c1 I - c2 (K^T-side product): chunkwise c1 = e^{G_L}, c2 = 1; frame-wise c1 = c2 = gamma
-            const float gam = frame ? prm.gamma[((long long)b * F + f) * prm.H + h] : 1.f;
-            const float eGL = frame ? gam : __expf(GL);
+            // M = gamma I - gamma (K^T B K)
+            const float gam = prm.gamma[((long long)b * F + f) * prm.H + h];
+            const float eGL = gam;
             const int m = r;
             for (int c4 = 0; c4 < ncols; c4 += 64) {  // four 16-column loads per wait (the last group may
                 float v4[4][16];                      // read past ncols, inside the 256-column buffer, unused)
@@ -281,13 +270,12 @@ k_transition_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 }  // namespace
 
-cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_x, const CUtensorMap &tm_v,
-                                 const TransParams &prm, long long n_fh, int /*num_sms: one CTA per frame-head*/,
-                                 cudaStream_t s) {
+cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const TransParams &prm,
+                                 long long n_fh, cudaStream_t s) {
     const size_t smem = 1024 + Smem::END + sizeof(uint64_t) * NBAR + 16 + 2 * CH * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(k_transition_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_transition_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_x, tm_v, prm);
+    k_transition_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_v, prm);
     return cudaGetLastError();
 }
 
