@@ -206,7 +206,7 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 1, s))) return e;
-    if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
+    if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, CF, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
                                      nfh, err, wait_ns, debug_drop_signal(), s)))
         return e;
     if ((e = mark(ev, 2, s))) return e;

@@ -31,6 +31,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int LDK = 128 + 8;   // bf16 row stride of the K tile (conflict-free ldmatrix)
 constexpr int LDT = 128 + 8;   // bf16 row stride of the A / T / scratch tiles
+constexpr int AD = 17;         // fp32 row stride of a diagonal leaf (odd: rows hit distinct banks)
+constexpr float kSplitMax = 60.f;  // largest row exponent the split decay takes (else the exact one)
 static_assert(LDK == LDT, "the scratch tile reuses the K tile");
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
@@ -82,7 +84,8 @@ __device__ __forceinline__ void store16(__nv_bfloat16 *t, int r0, int c0, const 
 struct InvParams {
     const __nv_bfloat16 *k;  // [B,T,H,dk]
     const float *beta;       // [B,T,H]
-    const float *G;          // [n_fh][L]
+    const float *G;          // [n_fh][(L+3)&~3]
+    const float *CF;         // [n_fh][(L+3)&~3] column factors e^{a - G_s} (a = G at the end of s's 64-token group)
     __nv_bfloat16 *Tinv;     // [n_fh][nblk][128][128]
     int L, dk, H, nblk;
     long long F, T;
@@ -92,21 +95,27 @@ struct InvParams {
 };
 
 __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams prm) {
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    // the K tile's 128-byte swizzle needs a 1024-aligned base: the dynamic shared memory base is
+    // (the kernel declares no static shared memory), and it is checked below
+    extern __shared__ __align__(1024) unsigned char smem[];
     constexpr uint32_t REG = 128 * LDT * 2;             // one padded 128 x 128 bf16 tile (34 KB)
     unsigned char *sKs = smem;                          // K_i, SW128 K-major, 2 slabs x 128 rows (32 KB)
     __nv_bfloat16 *sX = (__nv_bfloat16 *)smem;          // scratch products reuse the K region after the Gram
     __nv_bfloat16 *sA = (__nv_bfloat16 *)(smem + REG);  // [128][LDT]  A (strictly lower)
     __nv_bfloat16 *sT = sA + 128 * LDT;                 // [128][LDT]  T
-    float *sAd = (float *)(sT + 128 * LDT);             // [8][16][16] fp32 diagonal leaves of A
-    float *sG = sAd + 8 * 256;                          // [128]
-    float *sB = sG + 128;                               // [128]
+    float *sAd = (float *)(sT + 128 * LDT);             // [8][16][AD] fp32 diagonal leaves of A
+    float *sG = sAd + 8 * 16 * AD;                      // [128]
+    float *sCF = sG + 128;                              // [128]
+    float *sB = sCF + 128;                              // [128]
     uint64_t *bar = (uint64_t *)(sB + 128);
     uint32_t *tslot = (uint32_t *)(bar + 1);
     int *sok = (int *)(tslot + 1);
 
     if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
+    if (sm100::smem_u32(smem) & 1023u) {  // every thread sees the same base: all leave together
+        if (threadIdx.x == 0) atomicCAS(prm.err, sm100::kErrNone, sm100::kErrSmemAlign);
+        return;
+    }
     const int L = prm.L, dk = prm.dk, nblk = prm.nblk;
     const long long fh = blockIdx.x / nblk;
     const int blk = (int)(blockIdx.x % nblk);
@@ -128,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
         const int r = r_base + tid;
         const float *Gf = prm.G + fh * (long long)((L + 3) & ~3);  // G rows are padded to 16 bytes
         sm100::cp_async4(sG + tid, Gf + (r < L ? r : L - 1));
+        sm100::cp_async4(sCF + tid, prm.CF + fh * (long long)((L + 3) & ~3) + (r < L ? r : L - 1));
         if (r < L) sm100::cp_async4(sB + tid, prm.beta + ((long long)b * prm.T + f * L + r) * prm.H + h);
         else sB[tid] = 0.f;
     }
@@ -173,6 +183,15 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
         //      and columns 64 (warp / 4) .. + 63, read from TMEM 32 at a time (warp-uniform skips)
         const int q4 = warp & 3, hw = warp >> 2, r = q4 * 32 + lane;
         const float br = sB[r], gr = sG[r];
+        // Decay e^{G_r - G_s} = e^{G_r - a} cf_s, a = G at the end of the 64-token group of
+        // columns 64 hw .. 64 hw + 63 (the anchor cf was made with; the block starts on a group
+        // boundary).  A row after the group: e^{G_r - a} <= 1.  A row inside it: >= 1, bounded by
+        // e^{kSplitMax}, else the exact per-element exponential.  A row before it sees none of it.
+        const int nrow = min(128, L - r_base);
+        const float dG = gr - sG[min(64 * hw + 63, nrow - 1)];
+        const bool before = r < 64 * hw, inside = !before && r < 64 * hw + 64;
+        const bool exact = inside && !(dG <= kSplitMax);
+        const float rf = (before || exact) ? 0.f : br * __expf(dG);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
             const int c0 = 64 * hw + 32 * rr;
@@ -181,10 +200,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
             sm100::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + c0, v);
             sm100::tmem_ld_wait();
             float a[32];
+            if (!exact) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int s = c0 + e;
-                a[e] = s < r ? br * __expf(gr - sG[s]) * v[e] : 0.f;
+                for (int e = 0; e < 32; ++e) a[e] = c0 + e < r ? rf * sCF[c0 + e] * v[e] : 0.f;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) a[e] = c0 + e < r ? br * __expf(gr - sG[c0 + e]) * v[e] : 0.f;
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u)
@@ -196,27 +217,29 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
             if ((db * 16) >= c0 && (db * 16) < c0 + 32) {
                 const bool lo = db * 16 == c0;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) sAd[db * 256 + (r & 15) * 16 + e] = lo ? a[e] : a[16 + e];
+                for (int e = 0; e < 16; ++e) sAd[(db * 16 + (r & 15)) * AD + e] = lo ? a[e] : a[16 + e];
             }
         }
     }
     sm100::tc_fence_before();
     __syncthreads();
 
-    // ---- leaves: warp w inverts diagonal block w; lane c < 16 owns column c
+    // ---- leaves: warp w inverts diagonal block w; lane c < 16 owns column c.  Right-looking:
+    //      once t_s is final it is taken out of every later row at once, so each step's
+    //      updates are independent (the chain is 16 steps deep, not 120)
     if (lane < 16) {
-        const float *ad = sAd + warp * 256;
+        const float *ad = sAd + warp * 16 * AD;
         const int c = lane;
-        float t[16];
+        float x[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float x = (r == c) ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) x -= ad[r * 16 + s] * t[s];
-            t[r] = x;
+        for (int s = 0; s < 15; ++s) {
+#pragma unroll
+            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-ad[r * AD + s], x[s], x[r]);
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(warp * 16 + r) * LDT + warp * 16 + c] = __float2bfloat16_rn(t[r]);
+        for (int r = 0; r < 16; ++r) sT[(warp * 16 + r) * LDT + warp * 16 + c] = __float2bfloat16_rn(x[r]);
     }
     __syncthreads();
 
@@ -293,13 +316,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
 }  // namespace
 
 size_t diag_inverse_smem_bytes() {
-    return 1024 + sizeof(__nv_bfloat16) * 3 * 128 * LDT + sizeof(float) * (8 * 256 + 256) + 16;
+    return sizeof(__nv_bfloat16) * 3 * 128 * LDT + sizeof(float) * (8 * 16 * AD + 3 * 128) + 16;
 }
 
-cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, __nv_bfloat16 *Tinv,
-                                int L, int dk, int H, int nblk, long long F, long long T, long long n_fh,
-                                int *err, uint64_t wait_ns, int drop_first, cudaStream_t s) {
-    InvParams prm{k, beta, G, Tinv, L, dk, H, nblk, F, T, err, wait_ns, drop_first};
+cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, const float *CF,
+                                __nv_bfloat16 *Tinv, int L, int dk, int H, int nblk, long long F, long long T,
+                                long long n_fh, int *err, uint64_t wait_ns, int drop_first, cudaStream_t s) {
+    InvParams prm{k, beta, G, CF, Tinv, L, dk, H, nblk, F, T, err, wait_ns, drop_first};
     const size_t smem = diag_inverse_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(k_diag_inverse, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
