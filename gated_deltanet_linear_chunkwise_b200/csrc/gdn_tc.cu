@@ -115,6 +115,17 @@ bool map_f32_rows(CUtensorMap *m, const float *x, long long nfh, int len, int st
 }
 
 // Workspace [n_fh][rows][cols] bf16 seen as 3-D (cols, rows, n_fh).
+// Columns [col0, col0 + ncols) of rows of `cols` bf16 ([n_fh][rows][cols]) seen as 3-D
+// (ncols, rows, n_fh): stores clip at the part's last column.  col0 * 2 bytes must be a
+// multiple of 16 (the map's base).
+bool map_row_part(CUtensorMap *m, const void *x, long long nfh, int rows, int cols, int col0, int ncols,
+                  int box_rows) {
+    const cuuint64_t dims[3] = {(cuuint64_t)ncols, (cuuint64_t)rows, (cuuint64_t)nfh};
+    const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)rows * cols * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    return make_map(m, (const __nv_bfloat16 *)x + col0, 3, dims, strides, box);
+}
+
 bool map_rows(CUtensorMap *m, const void *x, long long nfh, int rows, int cols, int box_rows) {
     const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)nfh};
     const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)rows * cols * 2};
@@ -178,10 +189,11 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
 
     __nv_bfloat16 *Tinv = (__nv_bfloat16 *)(base + lay.Tinv);
     const int nc = p.dk + p.dv;
-    CUtensorMap tm_q, tm_k, tm_v, tm_u128, tm_sig, tm_t, tm_x128, tm_g128, tm_cf128;
+    CUtensorMap tm_q, tm_k, tm_v, tm_u128, tm_sig, tm_t, tm_x128, tm_xu, tm_xw, tm_g128, tm_cf128;
     if (!map_tokens(&tm_q, p.q, p, p.dk) || !map_tokens(&tm_k, p.k, p, p.dk) || !map_tokens(&tm_v, p.v, p, p.dv) ||
         !map_rows(&tm_u128, U, nfh, p.L, p.dv, 128) || !map_rows(&tm_sig, SigB, nfh, p.dk, p.dv, p.dk) ||
         !map_rows(&tm_t, Tinv, nfh * nblk, 128, 128, 128) || !map_rows(&tm_x128, X, nfh, p.L, nc, 128) ||
+        !map_row_part(&tm_xu, X, nfh, p.L, nc, 0, p.dv, 128) || !map_row_part(&tm_xw, X, nfh, p.L, nc, p.dv, p.dk, 128) ||
         !map_f32_rows(&tm_g128, G, nfh, p.L, cf_stride(p.L), 128) ||
         !map_f32_rows(&tm_cf128, CF, nfh, p.L, cf_stride(p.L), 128))
         return cudaErrorInvalidValue;
@@ -217,7 +229,7 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     ip.M = (!scan_tc || p.map_out) ? Mb : nullptr; ip.Mimg = scan_tc ? Mimg : nullptr; ip.N = Nb;
     ip.L = p.L; ip.dk = p.dk; ip.dv = p.dv; ip.H = p.H; ip.nblk = nblk;
     ip.F = p.F; ip.T = p.T; ip.err = err; ip.wait_ns = wait_ns;
-    if ((e = tc::launch_intra_tc(tm_k, tm_v, tm_t, tm_x128, ip, nfh, s))) return e;
+    if ((e = tc::launch_intra_tc(tm_k, tm_v, tm_t, tm_xu, tm_xw, ip, nfh, s))) return e;
     if ((e = mark(ev, 3, s))) return e;
     if (p.map_out && (e = simt_segment_map(p, Mb, Nb, s))) return e;
     if ((e = mark(ev, 4, s))) return e;

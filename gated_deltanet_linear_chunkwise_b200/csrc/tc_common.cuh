@@ -165,10 +165,12 @@ cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_
 cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_q, const CUtensorMap &tm_sig,
                         const UParams &prm, long long n_fh, int num_sms, cudaStream_t s);
 
-// tm_k / tm_v deliver 128-token boxes of k / v, tm_t one 128 x 128 block of T, tm_xs
-// stores 128-row boxes of X.  Also writes the frame's transition (N, and M and/or its images).
+// tm_k / tm_v deliver 128-token boxes of k / v, tm_t one 128 x 128 block of T; tm_xu / tm_xw
+// store 128-row boxes of X's Ub columns / W columns (maps over those columns of the
+// [Ub | W] rows).  Also writes the frame's transition (N, and M and/or its images).
 cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const CUtensorMap &tm_t,
-                            const CUtensorMap &tm_xs, const IntraParams &prm, long long n_fh, cudaStream_t s);
+                            const CUtensorMap &tm_xu, const CUtensorMap &tm_xw, const IntraParams &prm,
+                            long long n_fh, cudaStream_t s);
 
 // One CTA per (frame-head, 128-row block).  drop_first (debug): the first block's Gram is not
 // issued, so its bounded wait gives up and the pass reports a timeout without any fault.

@@ -29,12 +29,17 @@
 // source of X_i's TMA store) and bf16 H_i (the B operand of K_i H_i).
 // TMEM: the block's product (K_i H_i, then X_i; 256 columns) and H (fp32,
 // 256 columns; lanes = key dimension).
+// The Ub columns and the W columns never mix (each column of Y, X and H
+// depends on the same column alone), so the two halves run as two chains that
+// share K_i, T_ii and Kh_i: each half has its own products (N = d_v or d_k)
+// and barriers, and one half's epilogue overlaps the other's products.  In
+// shared and tensor memory the W columns start on a 64-column slab (column
+// dvp = d_v rounded up to 64), so each half is a whole number of swizzle slabs.
 // Warp roles (352 threads): warp 0 TMA loads, warp 1 TMEM owner + MMA issuer
 // (one thread), warps 2-9 epilogue: two warpgroups, each thread owning one row
-// (TMEM lane quadrant = warp % 4) and one half of the columns (half 0 the Ub
-// columns, half 1 the W columns; for H, rows are key dimensions); warp 10
-// stores X (a thread of its own, so that waiting for a store's reads holds up
-// no load).
+// (TMEM lane quadrant = warp % 4) of one half (warps 2-5 the Ub columns, warps
+// 6-9 the W columns; for H, rows are key dimensions); warp 10 stores X (a
+// thread of its own, so that waiting for a store's reads holds up no load).
 // Every wait is bounded (sm100::mbar_wait); a role that gives up waits for its
 // own copies and products in flight before the CTA leaves.
 #include "tc_common.cuh"
@@ -48,8 +53,10 @@ constexpr int kEpi = 256;                    // epilogue threads
 constexpr int TILE = 2 * SLAB_BYTES;         // 128 rows x 2 slabs (K_i or T_ii)
 constexpr int WIDE = 4 * SLAB_BYTES;         // 128 rows x 4 slabs (Y_i / X_i, H)
 
+// ACCFULL .. HREADY come per half (index + half); XSTG0 / XSTG1 are the halves' X staged.
 enum Bar {
-    ACCFULL = 0, YFULL, XFULL, XSTG0, XSTG1, UFULL, HREADY, TFULL, TFREE, VFULL, STAFREE, STBFREE, DRAIN,
+    ACCFULL = 0, YFULL = ACCFULL + 2, XFULL = YFULL + 2, UFULL = XFULL + 2, HREADY = UFULL + 2,
+    XSTG0 = HREADY + 2, XSTG1, KHREADY, TFULL, TFREE, VFULL, STAFREE, STBFREE, DRAIN,
     KFULL, KEMPTY = KFULL + 2, NBAR = KEMPTY + 2
 };
 
@@ -86,10 +93,11 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-           const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_xs,
-           const IntraParams prm) {
+           const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_xu,
+           const __grid_constant__ CUtensorMap tm_xw, const IntraParams prm) {
     extern __shared__ __align__(1024) unsigned char smem[];
-    const int L = prm.L, dk = prm.dk, dv = prm.dv, nc = dk + dv, nblk = prm.nblk;
+    const int L = prm.L, dk = prm.dk, dv = prm.dv, nblk = prm.nblk;
+    const int dvp = (dv + SLAB - 1) / SLAB * SLAB;  // first column of the W half in SMEM and TMEM
     const long long fh = blockIdx.x;
     const long long F = prm.F;
     const long long f = fh % F, chain = fh / F;
@@ -107,8 +115,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     int *err = prm.err;
     const uint64_t wait_ns = prm.wait_ns;
     const int nslab_k = (dk + SLAB - 1) / SLAB;
-    const int nslab_v = (dv + SLAB - 1) / SLAB;
-    const int nslab_x = (nc + SLAB - 1) / SLAB;
+    const int nslab_v = dvp / SLAB;
 
     if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
     if (sm100::smem_u32(smem) & 1023u) {  // every thread sees the same base: all leave together
@@ -117,7 +124,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i)
-            sm100::mbar_init(&bars[i], (i == YFULL || i == HREADY) ? kEpi : (i == XSTG0 || i == XSTG1) ? kEpi / 2 : 1);
+            sm100::mbar_init(&bars[i], ((i >= YFULL && i < YFULL + 2) || (i >= HREADY && i < HREADY + 2) ||
+                                        i == XSTG0 || i == XSTG1 || i == KHREADY) ? kEpi / 2 : 1);
         sm100::fence_barrier_init();
     }
     if (warp == 1) {
@@ -146,11 +154,11 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             sm100::tma_prefetch_desc(&tm_k);
             sm100::tma_prefetch_desc(&tm_v);
             sm100::tma_prefetch_desc(&tm_t);
-            sm100::tma_prefetch_desc(&tm_xs);
+            sm100::tma_prefetch_desc(&tm_xu);
+            sm100::tma_prefetch_desc(&tm_xw);
             // L2 policies: K and T are read once here; X is read again by the next stages
             const uint64_t once = sm100::policy_evict_first();
             int kj = 0, tj = 0, vj = 0;
-            const bool v_shares = (dv % SLAB) != 0;  // V's last slab also holds W columns
             for (int sl = 0; sl < nslab_v; ++sl) sm100::tma_prefetch_l2_4d(&tm_v, sl * SLAB, h, 0, bf);
             bool ok = true;
             sm100::Spin spin(wait_ns);
@@ -173,11 +181,10 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     ++tj;
                     prog = true;
                 }
-                // V_vj once X_{vj-1}'s Ub-only slabs have been read by their store (all of X_{vj-1}
-                // when V's last slab also holds W columns) and by Kh^T X_{vj-1}
+                // V_vj into the Ub slabs once X_{vj-1}'s Ub half has been read there by its store and
+                // by Kh^T X_{vj-1}
                 if (vj < nblk && (vj == 0 || (sm100::mbar_test(&bars[STAFREE], (vj - 1) & 1) &&
-                                              (!v_shares || sm100::mbar_test(&bars[STBFREE], (vj - 1) & 1)) &&
-                                              sm100::mbar_test(&bars[UFULL], (vj - 1) & 1)))) {
+                                              sm100::mbar_test(&bars[UFULL + 0], (vj - 1) & 1)))) {
                     sm100::mbar_arrive_expect_tx(&bars[VFULL], (uint32_t)(nslab_v * SLAB_BYTES));
                     for (int sl = 0; sl < nslab_v; ++sl)
                         sm100::tma_load_4d_hint(sST + sl * SLAB_BYTES, &tm_v, &bars[VFULL], sl * SLAB, h, vj * BM, bf,
@@ -205,25 +212,26 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         }
     } else if (warp == 10) {
         // ------------------------------------------------------------ X stores
-        // X_j in two parts: the slabs that hold only Ub columns once the Ub half has
-        // staged them (the next block's v may then land there), the rest once both halves have;
-        // a thread of its own, so that waiting for a store's reads holds up no load.
+        // X_j's Ub slabs once the Ub half has staged them (the next block's v may then land
+        // there), its W slabs once the W half has; each through a map of its own columns of
+        // the [Ub | W] rows.  A thread of its own, so that waiting for a store's reads holds up
+        // no load.
         if (lane == 0) {
-            const int nsA = dv / SLAB;
             const uint64_t keep = sm100::policy_evict_last();  // X is read again by the next stages
+            unsigned char *sW = sST + nslab_v * SLAB_BYTES;
             bool ok = true;
             for (int j = 0; j < nblk && ok; ++j) {
                 ok = sm100::mbar_wait(&bars[XSTG0], (uint32_t)(j & 1), err, wait_ns);
                 if (!ok) break;
-                for (int sl = 0; sl < nsA; ++sl)
-                    sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, j * BM, (int)fh, keep);
+                for (int sl = 0; sl < nslab_v; ++sl)
+                    sm100::tma_store_3d_hint(&tm_xu, sST + sl * SLAB_BYTES, sl * SLAB, j * BM, (int)fh, keep);
                 sm100::bulk_commit();
                 sm100::bulk_wait_read0();
                 sm100::mbar_arrive(&bars[STAFREE]);
                 ok = sm100::mbar_wait(&bars[XSTG1], (uint32_t)(j & 1), err, wait_ns);
                 if (!ok) break;
-                for (int sl = nsA; sl < nslab_x; ++sl)
-                    sm100::tma_store_3d_hint(&tm_xs, sST + sl * SLAB_BYTES, sl * SLAB, j * BM, (int)fh, keep);
+                for (int sl = 0; sl < nslab_k; ++sl)
+                    sm100::tma_store_3d_hint(&tm_xw, sW + sl * SLAB_BYTES, sl * SLAB, j * BM, (int)fh, keep);
                 sm100::bulk_commit();
                 sm100::bulk_wait_read0();
                 sm100::mbar_arrive(&bars[STBFREE]);
@@ -232,42 +240,78 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // One chain: per block, K_i H_i (from block 1), T_ii Y_i, then H += Kh_i^T X_i.
+        // Two chains, one per half (hf), polled: per block, K_i H_i (from block 1), T_ii Y_i,
+        // then H += Kh_i^T X_i, each on the half's columns only.  TFREE / KEMPTY are committed
+        // once both halves have issued their T_ii Y_i / Kh_i^T X_i.  T_ii and Kh_i, which both
+        // chains read, are observed one phase at a time, in order, through counters.
         if (lane == 0) {
-            const uint32_t id_kb = sm100::idesc_bf16(BM, nc, 0, 1);  // K-major A, MN-major B
-            const uint32_t id_tb = sm100::idesc_bf16(BM, nc, 1, 1);  // MN-major A (Kh^T), MN-major B
             const int nks_d = dk / 16;
+            int op0 = 1, op1 = 1, blk0 = 0, blk1 = 0;  // next product per half: 0 K_i H_i, 1 T_ii Y_i, 2 Kh^T X
+            int tobs = 0, khobs = 0;
+            int ty_done = 0, u_done = 0;          // blocks whose T Y / Kh^T X both halves have issued
+            // K_i is KFULL[i & 1]'s phase i >> 1; the phase after it needs K_{i+2}, which loads
+            // only once both halves' Kh_i^T X_i are done, so a direct parity test is unambiguous
+            // (a counter would have to observe K_0, which no product here waits for)
+            auto k_ready = [&](int i) -> bool {
+                return sm100::mbar_test(&bars[KFULL + (i & 1)], (uint32_t)((i >> 1) & 1));
+            };
+            auto seen = [&](int bar, int &obs, int i) -> bool {
+                while (obs <= i && sm100::mbar_test(&bars[bar], obs & 1)) ++obs;
+                return obs > i;
+            };
             bool ok = true;
-            for (int i = 0; i < nblk && ok; ++i) {
-                unsigned char *kt = sK + (i & 1) * TILE;
-                if (i > 0) {  // acc = K_i H_i, once K_i has landed and H_i is staged in bf16
-                    ok = sm100::mbar_wait(&bars[KFULL + (i & 1)], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
-                         sm100::mbar_wait(&bars[HREADY], (uint32_t)((i - 1) & 1), err, wait_ns);
-                    if (!ok) break;
-                    sm100::tc_fence_after();
-                    for (int ks = 0; ks < nks_d; ++ks)
-                        sm100::mma_bf16_ss(t_p, desc_kmajor(kt, ks, BM), desc_mnmajor(sH, ks, BM), id_kb, ks > 0);
-                    sm100::mma_commit(&bars[ACCFULL]);
+            sm100::Spin spin(wait_ns);
+            while (ok && (blk0 < nblk || blk1 < nblk)) {
+                bool prog = false;
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    int &opr = hf ? op1 : op0, &blkr = hf ? blk1 : blk0;
+                    const int i = blkr;
+                    if (i >= nblk) continue;
+                    const int n = hf ? dk : dv;                              // the half's columns
+                    const uint32_t coff = hf ? (uint32_t)dvp : 0u;           // ... in TMEM
+                    const uint32_t soff = hf ? (uint32_t)(nslab_v * SLAB_BYTES) : 0u;  // ... in SMEM
+                    unsigned char *kt = sK + (i & 1) * TILE;
+                    if (opr == 0) {  // acc = K_i H_i, once K_i has landed and H_i is staged in bf16
+                        if (k_ready(i) && sm100::mbar_test(&bars[HREADY + hf], (i - 1) & 1)) {
+                            sm100::tc_fence_after();
+                            const uint32_t id = sm100::idesc_bf16(BM, n, 0, 1);  // K-major A, MN-major B
+                            for (int ks = 0; ks < nks_d; ++ks)
+                                sm100::mma_bf16_ss(t_p + coff, desc_kmajor(kt, ks, BM), desc_mnmajor(sH + soff, ks, BM),
+                                                   id, ks > 0);
+                            sm100::mma_commit(&bars[ACCFULL + hf]);
+                            opr = 1;
+                            prog = true;
+                        }
+                    } else if (opr == 1) {  // X_i = T_ii Y_i
+                        if (seen(TFULL, tobs, i) && sm100::mbar_test(&bars[YFULL + hf], i & 1)) {
+                            sm100::tc_fence_after();
+                            const uint32_t id = sm100::idesc_bf16(BM, n, 0, 1);
+                            for (int ks = 0; ks < BM / 16; ++ks)
+                                sm100::mma_bf16_ss(t_p + coff, desc_kmajor(sT, ks, BM), desc_mnmajor(sST + soff, ks, BM),
+                                                   id, ks > 0);
+                            sm100::mma_commit(&bars[XFULL + hf]);
+                            if (++ty_done == 2 * (i + 1)) sm100::mma_commit(&bars[TFREE]);
+                            opr = 2;
+                            prog = true;
+                        }
+                    } else {  // H (rescaled to this block's end by the epilogue) += Kh_i^T X_i
+                        if (sm100::mbar_test(&bars[hf ? XSTG1 : XSTG0], i & 1) && seen(KHREADY, khobs, i)) {
+                            sm100::tc_fence_after();
+                            const uint32_t id = sm100::idesc_bf16(BM, n, 1, 1);  // MN-major A (Kh^T), MN-major B
+                            for (int ks = 0; ks < BM / 16; ++ks)
+                                sm100::mma_bf16_ss(t_h + coff, desc_mnmajor(kt, ks, BM), desc_mnmajor(sST + soff, ks, BM),
+                                                   id, (i > 0 || ks > 0) ? 1u : 0u);
+                            sm100::mma_commit(&bars[UFULL + hf]);
+                            if (++u_done == 2 * (i + 1)) sm100::mma_commit(&bars[KEMPTY + (i & 1)]);
+                            blkr = i + 1;
+                            opr = 0;
+                            prog = true;
+                        }
+                    }
                 }
-                // X_i = T_ii Y_i
-                ok = sm100::mbar_wait(&bars[TFULL], (uint32_t)(i & 1), err, wait_ns) &&
-                     sm100::mbar_wait(&bars[YFULL], (uint32_t)(i & 1), err, wait_ns);
-                if (!ok) break;
-                sm100::tc_fence_after();
-                for (int ks = 0; ks < BM / 16; ++ks)
-                    sm100::mma_bf16_ss(t_p, desc_kmajor(sT, ks, BM), desc_mnmajor(sST, ks, BM), id_kb, ks > 0);
-                sm100::mma_commit(&bars[XFULL]);
-                sm100::mma_commit(&bars[TFREE]);
-                // H (already rescaled to this block's end by the epilogue) += Kh_i^T X_i
-                ok = sm100::mbar_wait(&bars[XSTG0], (uint32_t)(i & 1), err, wait_ns) &&
-                     sm100::mbar_wait(&bars[XSTG1], (uint32_t)(i & 1), err, wait_ns);
-                if (!ok) break;
-                sm100::tc_fence_after();
-                for (int ks = 0; ks < BM / 16; ++ks)
-                    sm100::mma_bf16_ss(t_h, desc_mnmajor(kt, ks, BM), desc_mnmajor(sST, ks, BM), id_tb,
-                                       (i > 0 || ks > 0) ? 1u : 0u);
-                sm100::mma_commit(&bars[UFULL]);
-                sm100::mma_commit(&bars[KEMPTY + (i & 1)]);
+                if (prog) spin.reset();
+                else if (!spin.tick(err)) ok = false;
             }
             sm100::mma_commit(&bars[DRAIN]);  // every product issued completes before TMEM is released
             sm100::mbar_wait(&bars[DRAIN], 0u, err, sm100::kWaitLimitNs, true);
@@ -305,15 +349,17 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
             // ---- Y_i = R_i - diag(beta e^{G_r - G_{a_i}}) K_i H_i -> staging (MN-major: row = K index
             //      of T_ii Y_i)
-            if (i > 0) ok = sm100::mbar_wait(&bars[ACCFULL], (uint32_t)((i - 1) & 1), err, wait_ns);
-            // the W half writes over X_{i-1}'s last slabs: their store must have read them
-            if (ok && half == 1 && i > 0) ok = sm100::mbar_wait(&bars[STBFREE], (uint32_t)((i - 1) & 1), err, wait_ns);
-            if (ok) ok = sm100::mbar_wait(&bars[VFULL], (uint32_t)(i & 1), err, wait_ns) &&
-                         sm100::mbar_wait(&bars[KFULL + (i & 1)], (uint32_t)((i >> 1) & 1), err, wait_ns);
+            if (i > 0) ok = sm100::mbar_wait(&bars[ACCFULL + half], (uint32_t)((i - 1) & 1), err, wait_ns);
+            // the Ub half reads its v from (and writes Y over) the staging tile's Ub slabs; the W
+            // half reads k from K_i and writes over X_{i-1}'s W slabs, once their store has read them
+            if (ok && half == 0) ok = sm100::mbar_wait(&bars[VFULL], (uint32_t)(i & 1), err, wait_ns);
+            if (ok && half == 1)
+                ok = (i == 0 || sm100::mbar_wait(&bars[STBFREE], (uint32_t)((i - 1) & 1), err, wait_ns)) &&
+                     sm100::mbar_wait(&bars[KFULL + (i & 1)], (uint32_t)((i >> 1) & 1), err, wait_ns);
             if (!ok) break;
             sm100::tc_fence_after();
             const float rf = (valid && i > 0) ? be * __expf(Gr - aI) : 0.f;
-            const int rlen = half ? dk : dv, c_base = half ? dv : 0;
+            const int rlen = half ? dk : dv, c_base = half ? dvp : 0;
             const int n16 = rlen >> 4;  // the half's 16-column chunks (d_v and d_k are multiples of 16)
             const float rs = half ? be * __expf(Gr) : be;
             // y = rs x - rf acc over 8 columns from c, x this row's v (landed in the staging tile,
@@ -344,8 +390,10 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             }
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();
-            sm100::mbar_arrive(&bars[YFULL]);
-            if (half == 1) {  // off the chain: K_i becomes Kh_i in place (read by Kh_i^T X_i after X_i is staged)
+            sm100::mbar_arrive(&bars[YFULL + half]);
+            if (half == 1) {  // off the chain: K_i becomes Kh_i in place once the Ub half's K_i H_i has read it
+                if (i > 0) ok = sm100::mbar_wait(&bars[ACCFULL + 0], (uint32_t)((i - 1) & 1), err, wait_ns);
+                if (!ok) break;
                 const float ksc = valid ? __expf(aI1 - Gr) : 0.f;
                 for (int c = 0; c < dk; c += 8) {
                     uint4 *kp = reinterpret_cast<uint4 *>(kt + sw_offset(c, r));
@@ -358,13 +406,15 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     }
                     *kp = kv;
                 }
+                sm100::fence_proxy_async_smem();
+                sm100::mbar_arrive(&bars[KHREADY]);
             }
 
             // ---- X_i = T_ii Y_i -> bf16 staging over Y_i (half 0 the Ub columns, half 1 the W columns)
-            ok = sm100::mbar_wait(&bars[XFULL], (uint32_t)(i & 1), err, wait_ns);
+            ok = sm100::mbar_wait(&bars[XFULL + half], (uint32_t)(i & 1), err, wait_ns);
             if (!ok) break;
             sm100::tc_fence_after();
-            const int c_lo = half ? dv : 0;
+            const int c_lo = half ? dvp : 0;
             tmem_walk16(t_p + lane_off + c_lo, n16, [&](int j, const float (&x)[16]) {
                 *reinterpret_cast<uint4 *>(sST + sw_offset(c_lo + 16 * j, r)) = pack8(x);
                 *reinterpret_cast<uint4 *>(sST + sw_offset(c_lo + 16 * j + 8, r)) = pack8(x + 8);
@@ -375,7 +425,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 
             // ---- H_{i+1} (TMEM lane = key dimension m = r): bf16 copy for K_{i+1} H_{i+1}, and the
             //      fp32 accumulator rescaled to the next anchor; after the last block, M and N
-            ok = sm100::mbar_wait(&bars[UFULL], (uint32_t)(i & 1), err, wait_ns);
+            ok = sm100::mbar_wait(&bars[UFULL + half], (uint32_t)(i & 1), err, wait_ns);
             if (!ok) break;
             sm100::tc_fence_after();
             if (i + 1 < nblk) {
@@ -391,7 +441,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 sm100::tmem_st_wait();
                 sm100::tc_fence_before();
                 sm100::fence_proxy_async_smem();
-                sm100::mbar_arrive(&bars[HREADY]);
+                sm100::mbar_arrive(&bars[HREADY + half]);
             } else {
                 // H = Kt^T [Ub | W]: N = Kt^T Ub (half 0), M = e^{G_L} I - Kt^T W (half 1); every
                 // lane takes part in the (warp-wide) TMEM loads, rows m >= d_k store nothing
@@ -411,7 +461,7 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     if (half == 0) {
                         dst = prm.N + (fh * dk + m) * (long long)dv + c16;
                     } else {
-                        const int j0 = c16 - dv;
+                        const int j0 = c16 - dvp;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = (m == j0 + e ? eGL : 0.f) - v[e];
                         if (img) {  // hi + lo bf16 images of the scan's A operand
@@ -453,11 +503,12 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 }  // namespace
 
 cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const CUtensorMap &tm_t,
-                            const CUtensorMap &tm_xs, const IntraParams &prm, long long n_fh, cudaStream_t s) {
+                            const CUtensorMap &tm_xu, const CUtensorMap &tm_xw, const IntraParams &prm,
+                            long long n_fh, cudaStream_t s) {
     const size_t smem = Smem::END;
     cudaError_t e = cudaFuncSetAttribute(k_intra_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_v, tm_t, tm_xs, prm);
+    k_intra_tc<<<(unsigned)n_fh, kThreads, smem, s>>>(tm_k, tm_v, tm_t, tm_xu, tm_xw, prm);
     return cudaGetLastError();
 }
 
