@@ -365,8 +365,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
             // y = rs x - rf acc over 8 columns from c, x this row's v (landed in the staging tile,
             // overwritten in place) or k; pairs of columns in packed fp32 x2 arithmetic
             const uint64_t rs2 = f32x2(rs, rs), nrf2 = f32x2(-rf, -rf);
-            auto build = [&](int c, const float *acc) {
-                const uint4 xin = *reinterpret_cast<const uint4 *>((half ? kt : sST) + sw_offset(c, r));
+            const unsigned char *xsrc = half ? kt : sST;
+            auto build = [&](int c, const float *acc, const uint4 xin) {
                 const uint32_t xw[4] = {xin.x, xin.y, xin.z, xin.w};
                 float y[8];
 #pragma unroll
@@ -379,14 +379,23 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 }
                 *reinterpret_cast<uint4 *>(sST + sw_offset(c_base + c, r)) = valid ? pack8(y) : make_uint4(0, 0, 0, 0);
             };
+            // the row's next 16 columns are read from shared memory while these are worked on
+            uint4 xn0 = *reinterpret_cast<const uint4 *>(xsrc + sw_offset(0, r));
+            uint4 xn1 = *reinterpret_cast<const uint4 *>(xsrc + sw_offset(8, r));
+            auto chunk = [&](int j, const float *acc) {
+                const uint4 x0 = xn0, x1 = xn1;
+                if (j + 1 < n16) {
+                    xn0 = *reinterpret_cast<const uint4 *>(xsrc + sw_offset(16 * j + 16, r));
+                    xn1 = *reinterpret_cast<const uint4 *>(xsrc + sw_offset(16 * j + 24, r));
+                }
+                build(16 * j, acc, x0);
+                build(16 * j + 8, acc + 8, x1);
+            };
             if (i > 0) {
-                tmem_walk16(t_p + lane_off + c_base, n16, [&](int j, const float (&acc)[16]) {
-                    build(16 * j, acc);
-                    build(16 * j + 8, acc + 8);
-                });
+                tmem_walk16(t_p + lane_off + c_base, n16, [&](int j, const float (&acc)[16]) { chunk(j, acc); });
             } else {
-                const float zero[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                for (int c = 0; c < rlen; c += 8) build(c, zero);
+                const float zero[16] = {};
+                for (int j = 0; j < n16; ++j) chunk(j, zero);
             }
             sm100::tc_fence_before();
             sm100::fence_proxy_async_smem();
