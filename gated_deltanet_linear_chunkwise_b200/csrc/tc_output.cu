@@ -323,9 +323,15 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const float rf = g1 ? rfh[1] : rfh[0];
                     uint32_t q[8];
                     if (!ex) {  // rf = 0 where the row sees none of the group
+                        float cf[16];  // the chunk's column factors, four 16-byte reads
+#pragma unroll
+                        for (int q4c = 0; q4c < 4; ++q4c) {
+                            const float4 t4 = reinterpret_cast<const float4 *>(cfJ + c0)[q4c];
+                            cf[4 * q4c] = t4.x, cf[4 * q4c + 1] = t4.y, cf[4 * q4c + 2] = t4.z, cf[4 * q4c + 3] = t4.w;
+                        }
 #pragma unroll
                         for (int e = 0; e < 16; e += 2) {
-                            float f0 = rf * cfJ[c0 + e], f1 = rf * cfJ[c0 + e + 1];
+                            float f0 = rf * cf[e], f1 = rf * cf[e + 1];
                             if (in_g) {
                                 f0 = c0 + e <= r ? f0 : 0.f;
                                 f1 = c0 + e + 1 <= r ? f1 : 0.f;
