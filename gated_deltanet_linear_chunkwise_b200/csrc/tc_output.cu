@@ -173,53 +173,60 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // Per block i in order: S_{i+1} = Q_{i+1} K_{i+1}^T ahead (its buffer's previous S/P has
-        // been consumed), then, once P_i, Qt_i / Kh_i and bf16 Z_i (with the rescaled fp32 Z) are
-        // ready and O has been drained, O_i = Qt_i Z_i + P_i U_i and Z += Kh_i^T U_i.  Each wait
-        // is on a phase whose successor needs a product issued after it, so no parity is ambiguous.
+        // Two streams of products, polled so that neither waits on the other's inputs: S_j =
+        // Q_j K_j^T as soon as block j has landed and its S/P buffer is free (at most one block
+        // ahead of the O product), and, per block i in order, once P_i, Qt_i / Kh_i and bf16 Z_i
+        // (with the rescaled fp32 Z) are ready and O has been drained, O_i = Qt_i Z_i + P_i U_i
+        // and Z += Kh_i^T U_i.  Each barrier tested is either at the phase tested for or one
+        // before it: its next phase needs a product that has not been issued yet.
         if (lane == 0) {
             const uint32_t id_s = sm100::idesc_bf16(BM, BM, 0, 0);  // Q (K-major) x K^T (K-major)
             const uint32_t id_o = sm100::idesc_bf16(BM, dv, 0, 1);  // Qt or P (K-major) x Z or U (MN-major)
             const uint32_t id_z = sm100::idesc_bf16(BM, dv, 1, 1);  // Kh^T (MN-major) x U (MN-major)
             const int nks_d = dk / 16;
-            auto issue_s = [&](int j) -> bool {
-                const int buf = j & 1;
-                if (!sm100::mbar_wait(&bars[FULL + buf], (uint32_t)((j >> 1) & 1), err, wait_ns)) return false;
-                if (j >= 2 && !sm100::mbar_wait(&bars[SPFREE + buf], (uint32_t)(((j >> 1) - 1) & 1), err, wait_ns))
-                    return false;
-                sm100::tc_fence_after();
-                for (int ks = 0; ks < nks_d; ++ks)
-                    sm100::mma_bf16_ss(t_sp + buf * 128, desc_kmajor(sQ(buf), ks, BM), desc_kmajor(sK(buf), ks, BM),
-                                       id_s, ks > 0);
-                sm100::mma_commit(&bars[SFULL + buf]);
-                return true;
-            };
-            bool ok = issue_s(0);
-            for (int i = 0; i < nblk && ok; ++i) {
-                const int buf = i & 1;
-                if (i + 1 < nblk) ok = issue_s(i + 1);
-                ok = ok && sm100::mbar_wait(&bars[PREADY + buf], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
-                     sm100::mbar_wait(&bars[QKREADY + buf], (uint32_t)((i >> 1) & 1), err, wait_ns) &&
-                     sm100::mbar_wait(&bars[SREADY], (uint32_t)(i & 1), err, wait_ns) &&
-                     (i == 0 || sm100::mbar_wait(&bars[OFREE], (uint32_t)((i - 1) & 1), err, wait_ns));
-                if (!ok) break;
-                sm100::tc_fence_after();
-                // O_i = Qt_i Z_i + P_i U_i (P of tokens 0..63 in TMEM columns 0..31 of the buffer,
-                // tokens 64..127 in 64..95)
-                for (int ks = 0; ks < nks_d; ++ks)
-                    sm100::mma_bf16_ss(t_o, desc_kmajor(sQ(buf), ks, BM), desc_mnmajor(sZ, ks, BM), id_o, ks > 0);
-                for (int ks = 0; ks < BM / 16; ++ks)
-                    sm100::mma_bf16_ts(t_o, t_sp + buf * 128 + (ks >> 2) * 64 + (ks & 3) * 8,
-                                       desc_mnmajor(sU(buf), ks, BM), id_o, 1u);
-                sm100::mma_commit(&bars[OFULL]);
-                sm100::mma_commit(&bars[SPFREE + buf]);
-                if (i + 1 < nblk) {  // Z_{i+1}: the fp32 Z was rescaled to a_{i+1} with Z_i's bf16 copy
-                    for (int ks = 0; ks < BM / 16; ++ks)
-                        sm100::mma_bf16_ss(t_z, desc_mnmajor(sK(buf), ks, BM), desc_mnmajor(sU(buf), ks, BM), id_z,
-                                           1u);
-                    sm100::mma_commit(&bars[ZFULL]);
+            int js = 0, i = 0;  // next S, next O
+            bool ok = true;
+            sm100::Spin spin(wait_ns);
+            while (ok && i < nblk) {
+                bool prog = false;
+                if (js < nblk && js <= i + 1 && sm100::mbar_test(&bars[FULL + (js & 1)], (uint32_t)((js >> 1) & 1)) &&
+                    (js < 2 || sm100::mbar_test(&bars[SPFREE + (js & 1)], (uint32_t)(((js >> 1) - 1) & 1)))) {
+                    const int buf = js & 1;
+                    sm100::tc_fence_after();
+                    for (int ks = 0; ks < nks_d; ++ks)
+                        sm100::mma_bf16_ss(t_sp + buf * 128, desc_kmajor(sQ(buf), ks, BM), desc_kmajor(sK(buf), ks, BM),
+                                           id_s, ks > 0);
+                    sm100::mma_commit(&bars[SFULL + buf]);
+                    ++js;
+                    prog = true;
                 }
-                sm100::mma_commit(&bars[BFREE + buf]);
+                const int buf = i & 1;
+                if (js > i && sm100::mbar_test(&bars[PREADY + buf], (uint32_t)((i >> 1) & 1)) &&
+                    sm100::mbar_test(&bars[QKREADY + buf], (uint32_t)((i >> 1) & 1)) &&
+                    sm100::mbar_test(&bars[SREADY], (uint32_t)(i & 1)) &&
+                    (i == 0 || sm100::mbar_test(&bars[OFREE], (uint32_t)((i - 1) & 1)))) {
+                    sm100::tc_fence_after();
+                    // O_i = Qt_i Z_i + P_i U_i (P of tokens 0..63 in TMEM columns 0..31 of the buffer,
+                    // tokens 64..127 in 64..95)
+                    for (int ks = 0; ks < nks_d; ++ks)
+                        sm100::mma_bf16_ss(t_o, desc_kmajor(sQ(buf), ks, BM), desc_mnmajor(sZ, ks, BM), id_o, ks > 0);
+                    for (int ks = 0; ks < BM / 16; ++ks)
+                        sm100::mma_bf16_ts(t_o, t_sp + buf * 128 + (ks >> 2) * 64 + (ks & 3) * 8,
+                                           desc_mnmajor(sU(buf), ks, BM), id_o, 1u);
+                    sm100::mma_commit(&bars[OFULL]);
+                    sm100::mma_commit(&bars[SPFREE + buf]);
+                    if (i + 1 < nblk) {  // Z_{i+1}: the fp32 Z was rescaled to a_{i+1} with Z_i's bf16 copy
+                        for (int ks = 0; ks < BM / 16; ++ks)
+                            sm100::mma_bf16_ss(t_z, desc_mnmajor(sK(buf), ks, BM), desc_mnmajor(sU(buf), ks, BM), id_z,
+                                               1u);
+                        sm100::mma_commit(&bars[ZFULL]);
+                    }
+                    sm100::mma_commit(&bars[BFREE + buf]);
+                    ++i;
+                    prog = true;
+                }
+                if (prog) spin.reset();
+                else if (!spin.tick(err)) ok = false;
             }
             sm100::mma_commit(&bars[DRAIN]);  // every product issued completes before TMEM is released
             sm100::mbar_wait(&bars[DRAIN], 0u, err, sm100::kWaitLimitNs, true);
