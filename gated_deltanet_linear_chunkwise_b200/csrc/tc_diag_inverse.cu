@@ -15,11 +15,12 @@
 //   2. the eight 16x16 diagonal leaves inverted by forward substitution in
 //      fp32 (one column per lane),
 //   3. three doubling levels 16 -> 32 -> 64 -> 128:
-//      T21 = -T22 (A21 T11)  on the tensor cores (mma.sync, fp32 accumulate).
-// The doubling products are short dependent chains of mma.sync, whose
-// latency is long next to its issue rate, so every warp keeps several
-// independent accumulators in flight (two output tiles and two partial sums
-// over K).
+//      T21 = -(T22 A21) T11  on the tensor cores (mma.sync, fp32 accumulate),
+//      one pass per level: each of four warps owns a 16-row panel of T21 and
+//      keeps the intermediate T22 A21 in registers, where the accumulator
+//      layout is already the A operand layout of the second product, so a
+//      level needs no scratch tile and one block barrier; the zero triangles
+//      of T11 and T22 are skipped.
 // T_ii is written row-major bf16 [n_fh][nblk][128][128] (unit diagonal,
 // zeros above it), the A operand layout of the solve's T_ii Y_i product.
 #include "tc_common.cuh"
@@ -29,11 +30,9 @@ namespace tc {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int LDK = 128 + 8;   // bf16 row stride of the K tile (conflict-free ldmatrix)
-constexpr int LDT = 128 + 8;   // bf16 row stride of the A / T / scratch tiles
+constexpr int LDT = 128 + 8;   // bf16 row stride of the A and T tiles (conflict-free ldmatrix)
 constexpr int AD = 17;         // fp32 row stride of a diagonal leaf (odd: rows hit distinct banks)
 constexpr float kSplitMax = 60.f;  // largest row exponent the split decay takes (else the exact one)
-static_assert(LDK == LDT, "the scratch tile reuses the K tile");
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -81,6 +80,62 @@ __device__ __forceinline__ void store16(__nv_bfloat16 *t, int r0, int c0, const 
     *p = __floats2bfloat162_rn(scale * d1[2], scale * d1[3]);
 }
 
+// One doubling level: for each pair of SZ x SZ diagonal blocks of T (inverses T11, T22 of the
+// diagonal blocks of I + A, already in place), the block below the diagonal
+//   T21 = -(T22 A21) T11,
+// the off-diagonal block of the inverse of [[I + A11, 0], [A21, I + A22]].  There are always four
+// 16-row panels of T21 per level; warp p < 4 takes one: W = T22[panel, :] A21 (16 x SZ, k-steps up
+// to the panel's diagonal only, T22 being lower triangular) stays in registers as fp32
+// accumulators, is rounded to bf16 A fragments (the accumulator layout of m16n8k16 is the A
+// fragment layout), and T21[panel, c] = -W T11[:, c] takes only the k-steps at or below c's
+// (T11 is lower triangular).
+template <int SZ>
+__device__ __forceinline__ void merge_level(__nv_bfloat16 *sT, const __nv_bfloat16 *sA, int warp, int lane) {
+    constexpr int NP = SZ / 16;  // 16-row panels per merge; 128 / (2 SZ) merges x NP panels = 4
+    if (warp >= 4) return;
+    const int m = warp / NP, p = warp % NP;
+    const int base = m * 2 * SZ;
+    const int r0 = base + SZ + 16 * p;  // the panel's rows (of T22, A21 and T21)
+    float w[2 * NP][4];
+#pragma unroll
+    for (int t = 0; t < 2 * NP; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[t][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < NP; ++ks) {
+        if (ks > p) break;  // T22[panel][k] = 0 past the panel's diagonal block
+        uint32_t af[4];
+        load_a(af, sT, LDT, r0, base + SZ + 16 * ks, lane);
+#pragma unroll
+        for (int n2 = 0; n2 < NP; ++n2) {
+            uint32_t bf[4];
+            load_b_trans(bf, sA, LDT, base + SZ + 16 * ks, base + 16 * n2, lane);
+            mma16816(w[2 * n2], af, bf[0], bf[1]);
+            mma16816(w[2 * n2 + 1], af, bf[2], bf[3]);
+        }
+    }
+    uint32_t wa[NP][4];
+#pragma unroll
+    for (int js = 0; js < NP; ++js) {
+        wa[js][0] = pack_bf16(w[2 * js][0], w[2 * js][1]);
+        wa[js][1] = pack_bf16(w[2 * js][2], w[2 * js][3]);
+        wa[js][2] = pack_bf16(w[2 * js + 1][0], w[2 * js + 1][1]);
+        wa[js][3] = pack_bf16(w[2 * js + 1][2], w[2 * js + 1][3]);
+    }
+#pragma unroll
+    for (int cp = 0; cp < NP; ++cp) {
+        float d[2][4] = {};
+#pragma unroll
+        for (int js = cp; js < NP; ++js) {  // T11[j][c] = 0 for j above c's block
+            uint32_t bf[4];
+            load_b_trans(bf, sT, LDT, base + 16 * js, base + 16 * cp, lane);
+            mma16816(d[0], wa[js], bf[0], bf[1]);
+            mma16816(d[1], wa[js], bf[2], bf[3]);
+        }
+        store16(sT, r0, base + 16 * cp, d[0], d[1], -1.f, lane);
+    }
+}
+
 struct InvParams {
     const __nv_bfloat16 *k;  // [B,T,H,dk]
     const float *beta;       // [B,T,H]
@@ -100,7 +155,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
     extern __shared__ __align__(1024) unsigned char smem[];
     constexpr uint32_t REG = 128 * LDT * 2;             // one padded 128 x 128 bf16 tile (34 KB)
     unsigned char *sKs = smem;                          // K_i, SW128 K-major, 2 slabs x 128 rows (32 KB)
-    __nv_bfloat16 *sX = (__nv_bfloat16 *)smem;          // scratch products reuse the K region after the Gram
     __nv_bfloat16 *sA = (__nv_bfloat16 *)(smem + REG);  // [128][LDT]  A (strictly lower)
     __nv_bfloat16 *sT = sA + 128 * LDT;                 // [128][LDT]  T
     float *sAd = (float *)(sT + 128 * LDT);             // [8][16][AD] fp32 diagonal leaves of A
@@ -243,61 +297,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
     }
     __syncthreads();
 
-    // ---- doubling: T21 = -T22 (A21 T11) for block sizes 16, 32, 64; each warp runs two
-    //      16x16 output tiles at a time
-    for (int sz = 16; sz <= 64; sz <<= 1) {
-        const int per = (sz / 16) * (sz / 16);  // 16x16 output tiles per merge
-        const int total = (128 / (2 * sz)) * per;
-        for (int pass = 0; pass < 2; ++pass) {
-            // pass 0: X = A21 T11 -> sX;  pass 1: T21 = -T22 X -> sT
-            const __nv_bfloat16 *Am = pass ? sT : sA;
-            const __nv_bfloat16 *Bm = pass ? sX : sT;
-            __nv_bfloat16 *Dm = pass ? sT : sX;
-            for (int w0 = warp; w0 < total; w0 += 16) {
-                const int w1 = w0 + 8;
-                const bool two = w1 < total;
-                int ra[2], ca[2], kb[2], nb[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int w = (u && two) ? w1 : w0;
-                    const int m = w / per, tt = w % per;
-                    const int base = m * 2 * sz;
-                    const int tr = (tt / (sz / 16)) * 16, tc = (tt % (sz / 16)) * 16;
-                    ra[u] = base + sz + tr;                 // output / A rows (lower half)
-                    ca[u] = pass ? base + sz : base;        // A columns: T22 or A21
-                    kb[u] = pass ? base + sz : base;        // B rows: X (lower half) or T11
-                    nb[u] = base + tc;                      // output columns (upper half)
-                }
-                // two tiles, each as two partial sums over alternate 16-wide K slices
-                float d[2][2][2][4] = {};
-                for (int k = 0; k < sz; k += 32) {
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        if (k + 16 * h2 < sz) {
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                uint32_t af[4], bf[4];
-                                load_a(af, Am, LDT, ra[u], ca[u] + k + 16 * h2, lane);
-                                load_b_trans(bf, Bm, LDT, kb[u] + k + 16 * h2, nb[u], lane);
-                                mma16816(d[u][h2][0], af, bf[0], bf[1]);
-                                mma16816(d[u][h2][1], af, bf[2], bf[3]);
-                            }
-                        }
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        d[u][0][0][e] += d[u][1][0][e];
-                        d[u][0][1][e] += d[u][1][1][e];
-                    }
-                store16(Dm, ra[0], nb[0], d[0][0][0], d[0][0][1], pass ? -1.f : 1.f, lane);
-                if (two) store16(Dm, ra[1], nb[1], d[1][0][0], d[1][0][1], pass ? -1.f : 1.f, lane);
-            }
-            __syncthreads();
-        }
-    }
+    // ---- doubling: T21 = -(T22 A21) T11 for block sizes 16, 32, 64 (one merge level per pass)
+    merge_level<16>(sT, sA, warp, lane);
+    __syncthreads();
+    merge_level<32>(sT, sA, warp, lane);
+    __syncthreads();
+    merge_level<64>(sT, sA, warp, lane);
+    __syncthreads();
 
     // ---- write T_ii row-major
     __nv_bfloat16 *dst = prm.Tinv + (fh * nblk + blk) * (long long)(128 * 128);
