@@ -23,6 +23,9 @@
 //      of T11 and T22 are skipped.
 // T_ii is written row-major bf16 [n_fh][nblk][128][128] (unit diagonal,
 // zeros above it), the A operand layout of the solve's T_ii Y_i product.
+// Shared memory per CTA: A written over K once the Gram has read it, T, and
+// the fp32 leaves (74 KB), so three CTAs share an SM and one's loads overlap
+// the others' arithmetic.
 #include "tc_common.cuh"
 
 namespace gdn {
@@ -30,7 +33,7 @@ namespace tc {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int LDT = 128 + 8;   // bf16 row stride of the A and T tiles (conflict-free ldmatrix)
+constexpr uint32_t TILE = 128 * 256;  // one 128 x 128 bf16 tile (32 KB)
 constexpr int AD = 17;         // fp32 row stride of a diagonal leaf (odd: rows hit distinct banks)
 constexpr float kSplitMax = 60.f;  // largest row exponent the split decay takes (else the exact one)
 
@@ -52,32 +55,33 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// A fragment of the 16x16 row-major bf16 block at (r0, c0) of a tile with row stride ld.
-__device__ __forceinline__ void load_a(uint32_t (&a)[4], const __nv_bfloat16 *t, int ld, int r0, int c0, int lane) {
-    ldsm_x4(a, t + (r0 + (lane & 15)) * ld + c0 + (lane >> 4) * 8);
+// Byte offset of element (row, col) of a 128 x 128 bf16 tile: 256-byte rows whose 16-byte
+// chunks are permuted within each half-row by the row's low three bits, so the eight rows one
+// ldmatrix matrix reads, or one chunk of 32 consecutive rows, fall in distinct banks.
+__device__ __forceinline__ uint32_t swz(int row, int col) {
+    return (uint32_t)(row * 256 + (((col >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
 }
-// B fragments (two n8 tiles) of B[k][n] = M[k][n] for a row-major M: rows k0..k0+15, cols n0..n0+15.
-__device__ __forceinline__ void load_b_trans(uint32_t (&b)[4], const __nv_bfloat16 *t, int ld, int k0, int n0,
-                                             int lane) {
+
+// A fragment of the 16x16 block at (r0, c0) of a tile.
+__device__ __forceinline__ void load_a(uint32_t (&a)[4], const unsigned char *t, int r0, int c0, int lane) {
+    ldsm_x4(a, t + swz(r0 + (lane & 15), c0 + (lane >> 4) * 8));
+}
+// B fragments (two n8 tiles) of B[k][n] = M[k][n] for the tile M: rows k0..k0+15, cols n0..n0+15.
+__device__ __forceinline__ void load_b_trans(uint32_t (&b)[4], const unsigned char *t, int k0, int n0, int lane) {
     // matrices: (k 0-7, n 0-7), (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15)
     const int k = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
     const int n = n0 + (lane >> 4) * 8;
-    ldsm_x4_t(b, t + k * ld + n);
+    ldsm_x4_t(b, t + swz(k, n));
 }
 
 // Store a 16x16 fp32 accumulator pair as bf16 at (r0, c0), times `scale`.
-__device__ __forceinline__ void store16(__nv_bfloat16 *t, int r0, int c0, const float (&d0)[4],
-                                        const float (&d1)[4], float scale, int lane) {
+__device__ __forceinline__ void store16(unsigned char *t, int r0, int c0, const float (&d0)[4], const float (&d1)[4],
+                                        float scale, int lane) {
     const int g = lane >> 2, q = lane & 3;
-    __nv_bfloat162 *p;
-    p = reinterpret_cast<__nv_bfloat162 *>(t + (r0 + g) * LDT + c0 + 2 * q);
-    *p = __floats2bfloat162_rn(scale * d0[0], scale * d0[1]);
-    p = reinterpret_cast<__nv_bfloat162 *>(t + (r0 + g + 8) * LDT + c0 + 2 * q);
-    *p = __floats2bfloat162_rn(scale * d0[2], scale * d0[3]);
-    p = reinterpret_cast<__nv_bfloat162 *>(t + (r0 + g) * LDT + c0 + 8 + 2 * q);
-    *p = __floats2bfloat162_rn(scale * d1[0], scale * d1[1]);
-    p = reinterpret_cast<__nv_bfloat162 *>(t + (r0 + g + 8) * LDT + c0 + 8 + 2 * q);
-    *p = __floats2bfloat162_rn(scale * d1[2], scale * d1[3]);
+    *reinterpret_cast<uint32_t *>(t + swz(r0 + g, c0 + 2 * q)) = pack_bf16(scale * d0[0], scale * d0[1]);
+    *reinterpret_cast<uint32_t *>(t + swz(r0 + g + 8, c0 + 2 * q)) = pack_bf16(scale * d0[2], scale * d0[3]);
+    *reinterpret_cast<uint32_t *>(t + swz(r0 + g, c0 + 8 + 2 * q)) = pack_bf16(scale * d1[0], scale * d1[1]);
+    *reinterpret_cast<uint32_t *>(t + swz(r0 + g + 8, c0 + 8 + 2 * q)) = pack_bf16(scale * d1[2], scale * d1[3]);
 }
 
 // One doubling level: for each pair of SZ x SZ diagonal blocks of T (inverses T11, T22 of the
@@ -90,7 +94,7 @@ __device__ __forceinline__ void store16(__nv_bfloat16 *t, int r0, int c0, const 
 // fragment layout), and T21[panel, c] = -W T11[:, c] takes only the k-steps at or below c's
 // (T11 is lower triangular).
 template <int SZ>
-__device__ __forceinline__ void merge_level(__nv_bfloat16 *sT, const __nv_bfloat16 *sA, int warp, int lane) {
+__device__ __forceinline__ void merge_level(unsigned char *sT, const unsigned char *sA, int warp, int lane) {
     constexpr int NP = SZ / 16;  // 16-row panels per merge; 128 / (2 SZ) merges x NP panels = 4
     if (warp >= 4) return;
     const int m = warp / NP, p = warp % NP;
@@ -105,11 +109,11 @@ __device__ __forceinline__ void merge_level(__nv_bfloat16 *sT, const __nv_bfloat
     for (int ks = 0; ks < NP; ++ks) {
         if (ks > p) break;  // T22[panel][k] = 0 past the panel's diagonal block
         uint32_t af[4];
-        load_a(af, sT, LDT, r0, base + SZ + 16 * ks, lane);
+        load_a(af, sT, r0, base + SZ + 16 * ks, lane);
 #pragma unroll
         for (int n2 = 0; n2 < NP; ++n2) {
             uint32_t bf[4];
-            load_b_trans(bf, sA, LDT, base + SZ + 16 * ks, base + 16 * n2, lane);
+            load_b_trans(bf, sA, base + SZ + 16 * ks, base + 16 * n2, lane);
             mma16816(w[2 * n2], af, bf[0], bf[1]);
             mma16816(w[2 * n2 + 1], af, bf[2], bf[3]);
         }
@@ -128,7 +132,7 @@ __device__ __forceinline__ void merge_level(__nv_bfloat16 *sT, const __nv_bfloat
 #pragma unroll
         for (int js = cp; js < NP; ++js) {  // T11[j][c] = 0 for j above c's block
             uint32_t bf[4];
-            load_b_trans(bf, sT, LDT, base + 16 * js, base + 16 * cp, lane);
+            load_b_trans(bf, sT, base + 16 * js, base + 16 * cp, lane);
             mma16816(d[0], wa[js], bf[0], bf[1]);
             mma16816(d[1], wa[js], bf[2], bf[3]);
         }
@@ -149,15 +153,14 @@ struct InvParams {
     int drop_first;          // debug: the first block's Gram is not issued, so its wait gives up
 };
 
-__global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams prm) {
+__global__ void __launch_bounds__(kThreads, 3) k_diag_inverse(const InvParams prm) {
     // the K tile's 128-byte swizzle needs a 1024-aligned base: the dynamic shared memory base is
     // (the kernel declares no static shared memory), and it is checked below
     extern __shared__ __align__(1024) unsigned char smem[];
-    constexpr uint32_t REG = 128 * LDT * 2;             // one padded 128 x 128 bf16 tile (34 KB)
-    unsigned char *sKs = smem;                          // K_i, SW128 K-major, 2 slabs x 128 rows (32 KB)
-    __nv_bfloat16 *sA = (__nv_bfloat16 *)(smem + REG);  // [128][LDT]  A (strictly lower)
-    __nv_bfloat16 *sT = sA + 128 * LDT;                 // [128][LDT]  T
-    float *sAd = (float *)(sT + 128 * LDT);             // [8][16][AD] fp32 diagonal leaves of A
+    unsigned char *sKs = smem;             // K_i, SW128 K-major, 2 slabs x 128 rows (32 KB), read by the Gram
+    unsigned char *sA = smem;              // A (strictly lower), written over K once the Gram has completed
+    unsigned char *sT = smem + TILE;       // T
+    float *sAd = (float *)(smem + 2 * TILE);  // [8][16][AD] fp32 diagonal leaves of A
     float *sG = sAd + 8 * 16 * AD;                      // [128]
     float *sCF = sG + 128;                              // [128]
     float *sB = sCF + 128;                              // [128]
@@ -179,7 +182,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
     const int r_base = blk * 128;
 
     // ---- K_i into the swizzled layout (rows past the frame and columns past d_k zero-filled)
-    //      and the gates, all by asynchronous copies in flight at once; clear T and A meanwhile
+    //      and the gates, all by asynchronous copies in flight at once.  Neither A nor T is cleared:
+    //      every element a later step reads is written first, and T's upper triangle is written
+    //      out as zeros directly
     for (int e = tid; e < 128 * 16; e += kThreads) {
         const int r = e >> 4, c8 = e & 15;
         const bool in = r_base + r < L && c8 < dk / 8;
@@ -196,11 +201,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
         else sB[tid] = 0.f;
     }
     sm100::cp_async_commit();
-    for (int e = tid; e < 128 * 16; e += kThreads) {
-        const int r = e >> 4, c8 = e & 15;
-        *reinterpret_cast<uint4 *>(sT + r * LDT + c8 * 8) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4 *>(sA + r * LDT + c8 * 8) = make_uint4(0, 0, 0, 0);
-    }
     if (tid == 0) {
         sm100::mbar_init(bar, 1);
         sm100::fence_barrier_init();
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                *reinterpret_cast<uint4 *>(sA + r * LDT + c0 + 8 * u) =
+                *reinterpret_cast<uint4 *>(sA + swz(r, c0 + 8 * u)) =
                     make_uint4(pack_bf16(a[8 * u], a[8 * u + 1]), pack_bf16(a[8 * u + 2], a[8 * u + 3]),
                                pack_bf16(a[8 * u + 4], a[8 * u + 5]), pack_bf16(a[8 * u + 6], a[8 * u + 7]));
             // the fp32 diagonal 16 x 16 block of this row, when it lies in these columns
@@ -293,7 +293,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
             for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-ad[r * AD + s], x[s], x[r]);
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(warp * 16 + r) * LDT + warp * 16 + c] = __float2bfloat16_rn(x[r]);
+        for (int r = 0; r < 16; ++r)
+            *reinterpret_cast<__nv_bfloat16 *>(sT + swz(warp * 16 + r, warp * 16 + c)) = __float2bfloat16_rn(x[r]);
     }
     __syncthreads();
 
@@ -309,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
     __nv_bfloat16 *dst = prm.Tinv + (fh * nblk + blk) * (long long)(128 * 128);
     for (int e = tid; e < 128 * 16; e += kThreads) {
         const int r = e >> 4, c8 = e & 15;
-        *reinterpret_cast<uint4 *>(dst + r * 128 + c8 * 8) = *reinterpret_cast<const uint4 *>(sT + r * LDT + c8 * 8);
+        *reinterpret_cast<uint4 *>(dst + r * 128 + c8 * 8) =
+            8 * c8 > r ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4 *>(sT + swz(r, 8 * c8));
     }
     sm100::tc_fence_before();
     __syncthreads();
@@ -322,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_diag_inverse(const InvParams pr
 }  // namespace
 
 size_t diag_inverse_smem_bytes() {
-    return sizeof(__nv_bfloat16) * 3 * 128 * LDT + sizeof(float) * (8 * 16 * AD + 3 * 128) + 16;
+    return 2 * TILE + sizeof(float) * (8 * 16 * AD + 3 * 128) + 16;
 }
 
 cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, const float *CF,
@@ -331,6 +333,9 @@ cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const
     InvParams prm{k, beta, G, CF, Tinv, L, dk, H, nblk, F, T, err, wait_ns, drop_first};
     const size_t smem = diag_inverse_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(k_diag_inverse, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // three CTAs per SM (their shared memory, registers and TMEM columns all fit three times)
+    e = cudaFuncSetAttribute(k_diag_inverse, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     k_diag_inverse<<<(unsigned)(n_fh * nblk), kThreads, smem, s>>>(prm);
     return cudaGetLastError();
