@@ -14,6 +14,7 @@
 // The frame-wise operator: its per-frame maps (the transition kernel), the scan, and the
 // U kernel in its output mode.
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -267,7 +268,11 @@ finish:
     op.SigB = SigB;
     op.err = err;
     op.wait_ns = wait_ns;
-    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u128, tm_g128, tm_cf128, op, s))) return e;
+    // o by tiled stores when it is written plainly and its map can be made (16-byte aligned base)
+    CUtensorMap tm_o;
+    memset(&tm_o, 0, sizeof(tm_o));
+    op.o_tma = !p.accumulate && !scan_reverse && map_tokens(&tm_o, p.o, p, p.dv);
+    if ((e = tc::launch_output_tc(tm_q, tm_k, tm_u128, tm_g128, tm_cf128, tm_o, op, s))) return e;
     return mark(ev, 7, s);
 }
 

@@ -102,6 +102,7 @@ struct OutParams {
     const __nv_bfloat16 *SigB;  // [n_fh][dk][dv] bf16 state entering each frame (from the scan)
     int *err;
     uint64_t wait_ns;
+    int o_tma;               // o is written by tiled stores through tm_o (neither accumulate nor reverse_out)
 };
 
 struct IntraParams {
@@ -187,9 +188,10 @@ size_t scan_mimg_bytes(int dk);
 cudaError_t launch_scan_tc(const Problem &p, const __nv_bfloat16 *Mimg, const float *Nb, __nv_bfloat16 *SigB,
                            float *SigF, int *err, uint64_t wait_ns, cudaStream_t s);
 
+// tm_o: o [B,T,H,dv] seen like q (used when prm.o_tma is set).
 cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
-                             const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const OutParams &prm,
-                             cudaStream_t s);
+                             const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const CUtensorMap &tm_o,
+                             const OutParams &prm, cudaStream_t s);
 
 }  // namespace tc
 }  // namespace gdn

@@ -23,10 +23,13 @@
 //                   block-to-block chain);
 //   B (warps 6-9)   turns S = Q_i K_i^T into bf16 P in tensor memory;
 //   C (warps 10-13) scales Q_i, K_i into Qt_i, Kh_i in place;
-//   D (warps 14-17) writes O out.
+//   D (warps 14-17) writes O out: as a bf16 tile over Q_i's (Qt_i has been read
+//                   by then) that the producer stores with the tensor map of o,
+//                   or, when o accumulates or goes out token-reversed, row by
+//                   row from registers.
 // S of block i+1 is issued while block i is still in the epilogue.
 //   TMEM: Z (fp32, lane = key dimension), two S/P buffers, O.
-//   SMEM: Q_i, K_i, U_i (+ G, cf rows) double-buffered; bf16 Z_i.
+//   SMEM: Q_i (then O_i), K_i, U_i (+ G, cf rows) double-buffered; bf16 Z_i.
 // Decay in P: e^{G_r - a} cf_s with cf_s = e^{a - G_s} (a = G at the end of
 // s's 64-token group); inside the group the row factor is >= 1, bounded by
 // e^60, else the exact e^{G_r - G_s} is taken per element.  Every wait is
@@ -46,7 +49,7 @@ constexpr float kSplitMax = 60.f;         // largest row exponent the in-group s
 
 enum Bar {
     FULL = 0, BFREE = FULL + 2, SFULL = BFREE + 2, SPFREE = SFULL + 2, PREADY = SPFREE + 2, QKREADY = PREADY + 2,
-    SREADY = QKREADY + 2, ZFULL, OFULL, OFREE, DRAIN, NBAR
+    SREADY = QKREADY + 2, OSTAGED = SREADY + 1, ZFULL = OSTAGED + 2, OFULL, OFREE, DRAIN, NBAR
 };
 
 // Small objects first, then the swizzled tiles from a 1024-byte boundary (the dynamic shared
@@ -90,7 +93,8 @@ __device__ __forceinline__ void scale_row(unsigned char *tile, int r, int ncols,
 __global__ void __launch_bounds__(kThreads, 1)
 k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_g,
-            const __grid_constant__ CUtensorMap tm_cf, const OutParams prm) {
+            const __grid_constant__ CUtensorMap tm_cf, const __grid_constant__ CUtensorMap tm_o,
+            const OutParams prm) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int L = prm.L, dk = prm.dk, dv = prm.dv, nblk = prm.nblk;
     const long long fh = blockIdx.x;
@@ -120,7 +124,7 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < NBAR; ++i)
-            sm100::mbar_init(&bars[i], (i >= PREADY && i < SREADY + 1) || i == OFREE ? kGrp : 1);
+            sm100::mbar_init(&bars[i], (i >= PREADY && i < OSTAGED + 2) || i == OFREE ? kGrp : 1);
         sm100::fence_barrier_init();
     }
     if (warp == 1) {
@@ -148,13 +152,29 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             sm100::tma_prefetch_desc(&tm_u);
             sm100::tma_prefetch_desc(&tm_g);
             sm100::tma_prefetch_desc(&tm_cf);
+            if (prm.o_tma) sm100::tma_prefetch_desc(&tm_o);
+            // O_u, staged over Q_u's tile by group D, stored with the tensor map of o
+            auto store_o = [&](int u) {
+                for (int sl = 0; sl < nslab_v; ++sl)
+                    sm100::tma_store_4d(&tm_o, sQ(u & 1) + sl * SLAB_BYTES, sl * SLAB, h, u * BM, bf);
+                sm100::bulk_commit();
+            };
             const uint64_t once = sm100::policy_evict_first();
             const uint32_t bytes = (uint32_t)((2 * nslab_k + nslab_v) * SLAB_BYTES + 2 * BM * 4);
             int j = 0;
             bool ok = true;
             for (; j < nblk && ok; ++j) {  // block j into buffer j & 1 once block j - 2 is done with it
                 const int buf = j & 1;
-                if (j >= 2) ok = sm100::mbar_wait(&bars[BFREE + buf], (uint32_t)(((j >> 1) - 1) & 1), err, wait_ns);
+                if (j >= 2) {
+                    ok = sm100::mbar_wait(&bars[BFREE + buf], (uint32_t)(((j >> 1) - 1) & 1), err, wait_ns);
+                    if (ok && prm.o_tma) {  // block j - 2's O out of Q's tile before Q_j lands there
+                        ok = sm100::mbar_wait(&bars[OSTAGED + buf], (uint32_t)(((j >> 1) - 1) & 1), err, wait_ns);
+                        if (ok) {
+                            store_o(j - 2);
+                            sm100::bulk_wait_read0();
+                        }
+                    }
+                }
                 if (!ok) break;
                 uint64_t *bar = &bars[FULL + buf];
                 sm100::mbar_arrive_expect_tx(bar, bytes);
@@ -167,9 +187,15 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 sm100::tma_load_2d(sGC + buf * 2 * BM, &tm_g, bar, j * BM, (int)fh);
                 sm100::tma_load_2d(sGC + buf * 2 * BM + BM, &tm_cf, bar, j * BM, (int)fh);
             }
+            // the last two blocks' O (no later load waited for them)
+            for (int u = nblk > 2 ? nblk - 2 : 0; ok && prm.o_tma && u < nblk; ++u) {
+                ok = sm100::mbar_wait(&bars[OSTAGED + (u & 1)], (uint32_t)((u >> 1) & 1), err, wait_ns);
+                if (ok) store_o(u);
+            }
             if (!ok)  // leave with no copy in flight (full-limit drain waits)
                 for (int u = j > 2 ? j - 2 : 0; u < j; ++u)
                     sm100::mbar_wait(&bars[FULL + (u & 1)], (uint32_t)((u >> 1) & 1), err, sm100::kWaitLimitNs, true);
+            sm100::bulk_wait0();  // and with no store in flight
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -389,11 +415,24 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         } else {
             // -------------------------------------------------------- D: O out
-            // rows past the frame are not stored; a reversed scan's rows go back in place
+            // through Q_j's tile and the producer's tiled store; else row by row (rows past the frame
+            // are not stored; a reversed scan's rows go back in place)
             for (int j = 0; j < nblk && ok; ++j) {
                 ok = sm100::mbar_wait(&bars[OFULL], (uint32_t)(j & 1), err, wait_ns);
                 if (!ok) break;
                 sm100::tc_fence_after();
+                if (prm.o_tma) {  // O_j's product has read Qt_j: its tile takes O_j
+                    unsigned char *so = sQ(j & 1);
+                    tmem_walk16(t_o + lane_off, n16, [&](int c16, const float (&x)[16]) {
+                        *reinterpret_cast<uint4 *>(so + sw_offset(16 * c16, r)) = pack8(x);
+                        *reinterpret_cast<uint4 *>(so + sw_offset(16 * c16 + 8, r)) = pack8(x + 8);
+                    });
+                    sm100::tc_fence_before();
+                    sm100::mbar_arrive(&bars[OFREE]);
+                    sm100::fence_proxy_async_smem();
+                    sm100::mbar_arrive(&bars[OSTAGED + (j & 1)]);
+                    continue;
+                }
                 const int row = j * BM + r;
                 const bool valid = row < L;
                 const long long tt0 = f * L + row;
@@ -437,12 +476,12 @@ k_output_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 }  // namespace
 
 cudaError_t launch_output_tc(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_u,
-                             const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const OutParams &prm,
-                             cudaStream_t s) {
+                             const CUtensorMap &tm_g, const CUtensorMap &tm_cf, const CUtensorMap &tm_o,
+                             const OutParams &prm, cudaStream_t s) {
     const size_t smem = Smem::END;
     cudaError_t e = cudaFuncSetAttribute(k_output_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_output_tc<<<(unsigned)prm.n_fh, kThreads, smem, s>>>(tm_q, tm_k, tm_u, tm_g, tm_cf, prm);
+    k_output_tc<<<(unsigned)prm.n_fh, kThreads, smem, s>>>(tm_q, tm_k, tm_u, tm_g, tm_cf, tm_o, prm);
     return cudaGetLastError();
 }
 
