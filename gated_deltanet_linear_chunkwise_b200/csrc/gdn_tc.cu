@@ -219,8 +219,8 @@ cudaError_t launch_tc_forward(const Problem &p, void *ws, int scan_reverse, cuda
     gate_prefix_kernel<<<(unsigned)nfh, 256, gsm, s>>>(p, G, CF);
     if ((e = cudaGetLastError())) return e;
     if ((e = mark(ev, 1, s))) return e;
-    if ((e = tc::launch_diag_inverse((const __nv_bfloat16 *)p.k, p.beta, G, CF, Tinv, p.L, p.dk, p.H, nblk, p.F, p.T,
-                                     nfh, err, wait_ns, debug_drop_signal(), s)))
+    if ((e = tc::launch_diag_inverse(tm_k, tm_t, p.beta, G, CF, p.L, p.dk, p.H, nblk, p.F, p.T, nfh, err, wait_ns,
+                                     debug_drop_signal(), s)))
         return e;
     if ((e = mark(ev, 2, s))) return e;
     // the intra-frame solve also forms the frame's transition: fp32 M for the CUDA-core scan (and the

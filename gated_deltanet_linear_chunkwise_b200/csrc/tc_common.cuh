@@ -175,8 +175,10 @@ cudaError_t launch_intra_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_v, co
 
 // One CTA per (frame-head, 128-row block).  drop_first (debug): the first block's Gram is not
 // issued, so its bounded wait gives up and the pass reports a timeout without any fault.
-cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, const float *CF,
-                                __nv_bfloat16 *Tinv, int L, int dk, int H, int nblk, long long F, long long T,
+// tm_k delivers 128-token boxes of k (as for intra); tm_t is T's map (the one intra loads with),
+// through which the kernel stores each T_ii.
+cudaError_t launch_diag_inverse(const CUtensorMap &tm_k, const CUtensorMap &tm_t, const float *beta, const float *G,
+                                const float *CF, int L, int dk, int H, int nblk, long long F, long long T,
                                 long long n_fh, int *err, uint64_t wait_ns, int drop_first, cudaStream_t s);
 
 // tm_q / tm_k / tm_u / tm_g / tm_cf deliver 128-token boxes.

@@ -9,8 +9,8 @@
 // they do not depend on each other or on the solve, so this kernel computes
 // all of them in parallel, one CTA per (frame-head, block):
 //   1. S = K_i K_i^T on the 5th-generation tensor cores (one 128 x 128 tcgen05
-//      product into TMEM; K_i is copied into shared memory in the 128-byte
-//      swizzled layout by per-thread async copies) and A = beta_r e^{G_r - G_s} S
+//      product into TMEM; K_i arrives in the 128-byte swizzled layout by two
+//      tiled loads through k's tensor map) and A = beta_r e^{G_r - G_s} S
 //      (s < r) by the epilogue, one row per thread,
 //   2. the eight 16x16 diagonal leaves inverted by forward substitution in
 //      fp32 (one column per lane),
@@ -22,7 +22,9 @@
 //      level needs no scratch tile and one block barrier; the zero triangles
 //      of T11 and T22 are skipped.
 // T_ii is written row-major bf16 [n_fh][nblk][128][128] (unit diagonal,
-// zeros above it), the A operand layout of the solve's T_ii Y_i product.
+// zeros above it), the A operand layout of the solve's T_ii Y_i product, by
+// two tiled stores of the shared-memory tile (held in the tensor map's
+// swizzle throughout).
 // Shared memory per CTA: A written over K once the Gram has read it, T, and
 // the fp32 leaves (74 KB), so three CTAs share an SM and one's loads overlap
 // the others' arithmetic.
@@ -55,11 +57,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Byte offset of element (row, col) of a 128 x 128 bf16 tile: 256-byte rows whose 16-byte
-// chunks are permuted within each half-row by the row's low three bits, so the eight rows one
-// ldmatrix matrix reads, or one chunk of 32 consecutive rows, fall in distinct banks.
+// Byte offset of element (row, col) of a 128 x 128 bf16 tile in the tensor maps' 128-byte
+// swizzle: two 64-column slabs of 128-byte rows whose 16-byte chunks are permuted by the row's
+// low three bits, so the eight rows one ldmatrix matrix reads, or one chunk of 32 consecutive
+// rows, fall in distinct banks, and T leaves by two tiled stores as it is.
 __device__ __forceinline__ uint32_t swz(int row, int col) {
-    return (uint32_t)(row * 256 + (((col >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
+    return (uint32_t)((col >> 6) * SLAB_BYTES + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
+                      ((col & 7) << 1));
 }
 
 // A fragment of the 16x16 block at (r0, c0) of a tile.
@@ -140,12 +144,10 @@ __device__ __forceinline__ void merge_level(unsigned char *sT, const unsigned ch
     }
 }
 
-struct InvParams {
-    const __nv_bfloat16 *k;  // [B,T,H,dk]
+struct InvParams {        // k and T_ii move through tensor maps (tm_k, tm_t)
     const float *beta;       // [B,T,H]
     const float *G;          // [n_fh][(L+3)&~3]
     const float *CF;         // [n_fh][(L+3)&~3] column factors e^{a - G_s} (a = G at the end of s's 64-token group)
-    __nv_bfloat16 *Tinv;     // [n_fh][nblk][128][128]
     int L, dk, H, nblk;
     long long F, T;
     int *err;                // bounded-wait error word
@@ -153,7 +155,9 @@ struct InvParams {
     int drop_first;          // debug: the first block's Gram is not issued, so its wait gives up
 };
 
-__global__ void __launch_bounds__(kThreads, 3) k_diag_inverse(const InvParams prm) {
+__global__ void __launch_bounds__(kThreads, 3)
+k_diag_inverse(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_t,
+               const InvParams prm) {
     // the K tile's 128-byte swizzle needs a 1024-aligned base: the dynamic shared memory base is
     // (the kernel declares no static shared memory), and it is checked below
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -164,8 +168,9 @@ __global__ void __launch_bounds__(kThreads, 3) k_diag_inverse(const InvParams pr
     float *sG = sAd + 8 * 16 * AD;                      // [128]
     float *sCF = sG + 128;                              // [128]
     float *sB = sCF + 128;                              // [128]
-    uint64_t *bar = (uint64_t *)(sB + 128);
-    uint32_t *tslot = (uint32_t *)(bar + 1);
+    uint64_t *bar = (uint64_t *)(sB + 128);  // the Gram's completion
+    uint64_t *lbar = bar + 1;                 // K_i landed
+    uint32_t *tslot = (uint32_t *)(bar + 2);
     int *sok = (int *)(tslot + 1);
 
     if (pass_failed(prm.err)) return;  // an earlier stage of this pass gave up
@@ -181,16 +186,21 @@ __global__ void __launch_bounds__(kThreads, 3) k_diag_inverse(const InvParams pr
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r_base = blk * 128;
 
-    // ---- K_i into the swizzled layout (rows past the frame and columns past d_k zero-filled)
-    //      and the gates, all by asynchronous copies in flight at once.  Neither A nor T is cleared:
-    //      every element a later step reads is written first, and T's upper triangle is written
-    //      out as zeros directly
+    // ---- K_i by two tiled loads (rows past the frame and columns past d_k read as zeros), the
+    //      gates by asynchronous copies; meanwhile the 16x16 tiles of T above its diagonal are
+    //      cleared (T leaves by tiled stores; nothing else writes them)
+    if (tid == 0) {
+        sm100::mbar_init(bar, 1);
+        sm100::mbar_init(lbar, 1);
+        sm100::fence_barrier_init();
+        const int nslab = (dk + 63) / 64;
+        sm100::mbar_arrive_expect_tx(lbar, (uint32_t)(nslab * SLAB_BYTES));
+        for (int sl = 0; sl < nslab; ++sl)
+            sm100::tma_load_4d(sKs + sl * SLAB_BYTES, &tm_k, lbar, sl * 64, h, r_base, (int)(b * prm.F + f));
+    }
     for (int e = tid; e < 128 * 16; e += kThreads) {
         const int r = e >> 4, c8 = e & 15;
-        const bool in = r_base + r < L && c8 < dk / 8;
-        const long long t = f * L + (r_base + r < L ? r_base + r : 0);
-        const __nv_bfloat16 *src = prm.k + (((long long)b * prm.T + t) * prm.H + h) * dk + (in ? c8 * 8 : 0);
-        sm100::cp_async16(sKs + (c8 >> 3) * SLAB_BYTES + r * 128 + (((c8 & 7) ^ (r & 7)) << 4), src, in ? 16u : 0u);
+        if ((c8 >> 1) > (r >> 4)) *reinterpret_cast<uint4 *>(sT + swz(r, 8 * c8)) = make_uint4(0, 0, 0, 0);
     }
     if (tid < 128) {
         const int r = r_base + tid;
@@ -201,25 +211,23 @@ __global__ void __launch_bounds__(kThreads, 3) k_diag_inverse(const InvParams pr
         else sB[tid] = 0.f;
     }
     sm100::cp_async_commit();
-    if (tid == 0) {
-        sm100::mbar_init(bar, 1);
-        sm100::fence_barrier_init();
-    }
     if (warp == 0) {
         sm100::tmem_alloc(tslot, 128);
         sm100::tmem_relinquish();
     }
     sm100::cp_async_wait_all();
-    sm100::fence_proxy_async_smem();  // the copies are visible to the tensor cores
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    // ---- S = K K^T in TMEM (one thread issues), then the bounded wait by the same thread
+    // ---- S = K K^T in TMEM (one thread issues once K_i has landed), then the bounded wait by the
+    //      same thread
     if (tid == 0) {
+        const bool landed = sm100::mbar_wait(lbar, 0, prm.err, prm.wait_ns);
+        if (!landed) sm100::mbar_wait(lbar, 0, prm.err, sm100::kWaitLimitNs, true);  // no copy left in flight
         // debug switch: the first block's product is never issued, so this wait gives up (no fault)
-        const bool issue = !(prm.drop_first && blockIdx.x == 0);
+        const bool issue = landed && !(prm.drop_first && blockIdx.x == 0);
         if (issue) {
             const uint32_t id = sm100::idesc_bf16(128, 128, 0, 0);
             for (int ks = 0; ks < dk / 16; ++ks)
@@ -304,14 +312,15 @@ __global__ void __launch_bounds__(kThreads, 3) k_diag_inverse(const InvParams pr
     merge_level<32>(sT, sA, warp, lane);
     __syncthreads();
     merge_level<64>(sT, sA, warp, lane);
+    sm100::fence_proxy_async_smem();  // T's writes are visible to the tiled stores
     __syncthreads();
 
-    // ---- write T_ii row-major
-    __nv_bfloat16 *dst = prm.Tinv + (fh * nblk + blk) * (long long)(128 * 128);
-    for (int e = tid; e < 128 * 16; e += kThreads) {
-        const int r = e >> 4, c8 = e & 15;
-        *reinterpret_cast<uint4 *>(dst + r * 128 + c8 * 8) =
-            8 * c8 > r ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4 *>(sT + swz(r, 8 * c8));
+    // ---- T_ii out: two tiled stores (its layout is the tensor map's), complete before the CTA leaves
+    if (tid == 0) {
+        for (int sl = 0; sl < 2; ++sl)
+            sm100::tma_store_3d(&tm_t, sT + sl * SLAB_BYTES, sl * 64, 0, (int)(fh * nblk + blk));
+        sm100::bulk_commit();
+        sm100::bulk_wait0();
     }
     sm100::tc_fence_before();
     __syncthreads();
@@ -324,20 +333,20 @@ __global__ void __launch_bounds__(kThreads, 3) k_diag_inverse(const InvParams pr
 }  // namespace
 
 size_t diag_inverse_smem_bytes() {
-    return 2 * TILE + sizeof(float) * (8 * 16 * AD + 3 * 128) + 16;
+    return 2 * TILE + sizeof(float) * (8 * 16 * AD + 3 * 128) + 24;
 }
 
-cudaError_t launch_diag_inverse(const __nv_bfloat16 *k, const float *beta, const float *G, const float *CF,
-                                __nv_bfloat16 *Tinv, int L, int dk, int H, int nblk, long long F, long long T,
+cudaError_t launch_diag_inverse(const CUtensorMap &tm_k, const CUtensorMap &tm_t, const float *beta, const float *G,
+                                const float *CF, int L, int dk, int H, int nblk, long long F, long long T,
                                 long long n_fh, int *err, uint64_t wait_ns, int drop_first, cudaStream_t s) {
-    InvParams prm{k, beta, G, CF, Tinv, L, dk, H, nblk, F, T, err, wait_ns, drop_first};
+    InvParams prm{beta, G, CF, L, dk, H, nblk, F, T, err, wait_ns, drop_first};
     const size_t smem = diag_inverse_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(k_diag_inverse, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // three CTAs per SM (their shared memory, registers and TMEM columns all fit three times)
     e = cudaFuncSetAttribute(k_diag_inverse, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    k_diag_inverse<<<(unsigned)(n_fh * nblk), kThreads, smem, s>>>(prm);
+    k_diag_inverse<<<(unsigned)(n_fh * nblk), kThreads, smem, s>>>(tm_k, tm_t, prm);
     return cudaGetLastError();
 }
 
