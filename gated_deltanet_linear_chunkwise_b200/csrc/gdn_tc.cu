@@ -254,7 +254,7 @@ finish:
     up.L = p.L; up.dk = p.dk; up.dv = p.dv; up.nblk = nblk; up.err = err;
     up.frame = 0; up.o = nullptr; up.T = p.T; up.F = p.F; up.H = p.H; up.accumulate = 0;
     up.norm_q = 0; up.q_w = nullptr; up.wait_ns = wait_ns;
-    if ((e = tc::launch_u_tc(tm_x128, tm_q, tm_sig, up, nfh, num_sms, s))) return e;
+    if ((e = tc::launch_u_tc(tm_x128, tm_q, tm_sig, tm_u128, up, nfh, num_sms, s))) return e;
     if ((e = mark(ev, 6, s))) return e;
 
     tc::OutParams op;
@@ -356,7 +356,7 @@ cudaError_t launch_tc_frame(const Problem &p, void *ws, cudaStream_t s, cudaEven
     up.norm_q = (p.qk_norm & GDN_QK_NORM_QUERIES) ? 1 : 0;
     up.q_w = p.q_norm_weight;
     up.wait_ns = tp.wait_ns;
-    if ((e = tc::launch_u_tc(tm_q, tm_q, tm_sig, up, nfh, num_sms, s))) return e;
+    if ((e = tc::launch_u_tc(tm_q, tm_q, tm_sig, tm_q, up, nfh, num_sms, s))) return e;
     return mark(ev, 7, s);
 }
 

@@ -163,8 +163,9 @@ cudaError_t launch_transition_tc(const CUtensorMap &tm_k, const CUtensorMap &tm_
                                  long long n_fh, cudaStream_t s);
 // tm_x delivers 128-row boxes of X, tm_q 128-token boxes of q (frame-wise
 // operator), tm_sig the bf16 state of a frame-head.
+// tm_u stores 128-row boxes of U (chunkwise; unused by the frame-wise operator).
 cudaError_t launch_u_tc(const CUtensorMap &tm_x, const CUtensorMap &tm_q, const CUtensorMap &tm_sig,
-                        const UParams &prm, long long n_fh, int num_sms, cudaStream_t s);
+                        const CUtensorMap &tm_u, const UParams &prm, long long n_fh, int num_sms, cudaStream_t s);
 
 // tm_k / tm_v deliver 128-token boxes of k / v, tm_t one 128 x 128 block of T; tm_xu / tm_xw
 // store 128-row boxes of X's Ub columns / W columns (maps over those columns of the
