@@ -91,6 +91,30 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
 }
 
 
+// Where a column half stages the frame's transition after its last block: its own slabs of the
+// staging tile (stA) and of bf16 H (stB).  N (half 0) as fp32 rows at a pitch of an odd number of
+// 16-byte units (one warp's row pieces fall in distinct banks), rows_per rows in each region;
+// M's hi / lo images (half 1) in the scan's operand layout, hi over stB, lo over stA.
+struct FinalStage {
+    unsigned char *stA, *stB, *img;
+    int nslab, pitch, rows_per;
+    bool stage_n;
+    __device__ __forceinline__ FinalStage(unsigned char *sST, unsigned char *sH, int half, int dk, int dv, int dvp,
+                                          int nslab_v, __nv_bfloat16 *Mimg, long long fh) {
+        const int sl0 = half ? dvp / SLAB : 0;
+        stA = sST + sl0 * SLAB_BYTES;
+        stB = sH + sl0 * SLAB_BYTES;
+        nslab = (dk + SLAB - 1) / SLAB;
+        img = Mimg ? reinterpret_cast<unsigned char *>(Mimg) + fh * (long long)(2 * nslab * dk * 128) : nullptr;
+        pitch = dv * 4 + 16;
+        rows_per = nslab_v * SLAB_BYTES / pitch;
+        stage_n = 2 * rows_per >= dk;
+    }
+    __device__ __forceinline__ unsigned char *nrow(int row) const {
+        return (row < rows_per ? stA : stB) + (row % rows_per) * pitch;
+    }
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
 k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
            const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_xu,
@@ -453,13 +477,19 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                 sm100::mbar_arrive(&bars[HREADY + half]);
             } else {
                 // H = Kt^T [Ub | W]: N = Kt^T Ub (half 0), M = e^{G_L} I - Kt^T W (half 1); every
-                // lane takes part in the (warp-wide) TMEM loads, rows m >= d_k store nothing
+                // lane takes part in the (warp-wide) TMEM loads, rows m >= d_k store nothing.
+                // N and the scan's images of M are staged in shared memory that nothing reads any
+                // more (the half's own slabs of the staging tile, once X's last store has read
+                // them, and of bf16 H) and leave as whole lines once every role is done (below);
+                // fp32 M, when asked for, goes out row by row.
                 const float eGL = __expf(aI1);
                 const int m = r;
-                const int nslab = (dk + SLAB - 1) / SLAB;
-                unsigned char *img = prm.Mimg ? reinterpret_cast<unsigned char *>(prm.Mimg) +
-                                                    fh * (long long)(2 * nslab * dk * 128)
-                                              : nullptr;
+                const FinalStage fs(sST, sH, half, dk, dv, dvp, nslab_v, prm.Mimg, fh);
+                ok = sm100::mbar_wait(&bars[half ? STBFREE : STAFREE], (uint32_t)((nblk - 1) & 1), err, wait_ns);
+                if (!ok) break;
+                unsigned char *stA = fs.stA, *stB = fs.stB;
+                const bool stage_n = fs.stage_n;
+                unsigned char *img = fs.img;
                 const int c_hi = c_lo + rlen;
                 for (int c16 = c_lo; c16 < c_hi; c16 += 16) {  // dv is a multiple of 16
                     float v[16];
@@ -468,12 +498,18 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     if (m >= dk) continue;
                     float *dst;
                     if (half == 0) {
+                        if (stage_n) {
+                            float4 *sp = reinterpret_cast<float4 *>(fs.nrow(m) + c16 * 4);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) sp[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+                            continue;
+                        }
                         dst = prm.N + (fh * dk + m) * (long long)dv + c16;
                     } else {
                         const int j0 = c16 - dvp;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = (m == j0 + e ? eGL : 0.f) - v[e];
-                        if (img) {  // hi + lo bf16 images of the scan's A operand
+                        if (img) {  // hi + lo bf16 images of the scan's A operand: hi over bf16 H's W slabs, lo over the staging tile's
 #pragma unroll
                             for (int h8 = 0; h8 < 2; ++h8) {
                                 uint32_t hi[4], lo[4];
@@ -486,9 +522,8 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                                     lo[e] = pack_bf16(a - hf.x, bb - hf.y);
                                 }
                                 const uint32_t off = sm100::sw128_kmajor_offset(m, j0 + 8 * h8, dk);
-                                *reinterpret_cast<uint4 *>(img + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                                *reinterpret_cast<uint4 *>(img + nslab * dk * 128 + off) =
-                                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                                *reinterpret_cast<uint4 *>(stB + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                                *reinterpret_cast<uint4 *>(stA + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                             }
                         }
                         if (!prm.M) continue;
@@ -498,11 +533,30 @@ k_intra_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
                     for (int e = 0; e < 16; e += 4)
                         *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                 }
+                sm100::fence_proxy_async_smem();  // the images are visible to the bulk copies
             }
         }
     }
     sm100::tc_fence_before();
     __syncthreads();
+    if (warp >= 2 && warp < 10) {  // N and M's images out of shared memory (after a failed wait: whatever is there)
+        const int half = (warp - 2) >> 2, r = (warp & 3) * 32 + lane;
+        const FinalStage fs(sST, sH, half, dk, dv, dvp, nslab_v, prm.Mimg, fh);
+        if (half == 0 && fs.stage_n) {  // N of this frame-head is contiguous: 16-byte pieces in order
+            const int n4 = dv / 4;
+            float4 *dn = reinterpret_cast<float4 *>(prm.N + fh * (long long)dk * dv);
+            for (int c = r; c < dk * n4; c += kEpi / 2) {
+                const int row = c / n4;
+                dn[c] = *reinterpret_cast<const float4 *>(fs.nrow(row) + (c - row * n4) * 16);
+            }
+        } else if (half == 1 && fs.img && r == 0) {
+            const uint32_t part = (uint32_t)(fs.nslab * dk * 128);
+            sm100::bulk_copy_s2g(fs.img, fs.stB, part);
+            sm100::bulk_copy_s2g(fs.img + part, fs.stA, part);
+            sm100::bulk_commit();
+            sm100::bulk_wait0();
+        }
+    }
     if (warp == 1) {
         sm100::tc_fence_after();
         sm100::tmem_dealloc(tbase, 512);
