@@ -81,11 +81,11 @@ def bytes_alg(B, T, H, dk, dv, elem=2):
 # of the short-clip case (420 frame-heads, L = 880, d_k = d_v = 112; profiles/ holds the
 # summary and the command).  Traffic grows with the frame-heads processed, so a launch's
 # figure is this times its frame-head count; other shapes report null.
-DRAM_BYTES_PER_FH = {"intra": (306.549760e6 + 133.350912e6) / 420,
+DRAM_BYTES_PER_FH = {"intra": (307.306496e6 + 134.093312e6) / 420,
                      "output": (283.816704e6 + 29.959936e6) / 420,
-                     "diag_inverse": (87.335168e6 + 51.471872e6) / 420,
+                     "diag_inverse": (88.742656e6 + 50.603264e6) / 420,
                      "scan": (45.200896e6 + 0.630528e6) / 420,
-                     "u": (180.985344e6 + 47.667712e6) / 420}
+                     "u": (176.373504e6 + 51.713024e6) / 420}
 TRAFFIC_SHAPE = (880, 112, 112)
 
 
